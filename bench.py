@@ -1,0 +1,363 @@
+"""Benchmark of the NVFP4 W4A4 routed-MoE feed-forward layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode] [--impl ours|reference]
+
+One step = one full pass of the layer (route, permute, quantise x, gate/up + SwiGLU +
+requantise, down, combine) over one batch of synthetic tokens, inputs resident in HBM.
+L2 is flushed (a 256 MiB write) before every timed step, outside the timed events.
+Prints one JSON line on rank 0.  With N > 1 (torchrun) every rank runs an independent
+replica on its own GPU (the layer has no cross-GPU exchange on one device's batch), the
+timed region is bracketed by barriers and the reported time is the max over ranks.
+
+--impl reference times the CPU oracle (the plain C++ implementation the tests check
+against) on the machine's host cores on the same workload: a deliberately slow baseline.
+"""
+from __future__ import annotations
+
+import argparse
+import concurrent.futures as cf
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from nvfp4_mixture_experts_w4a4_b200 import _lib as C  # noqa: E402
+from nvfp4_mixture_experts_w4a4_b200 import ops, workloads as W  # noqa: E402
+
+METRIC = "NVFP4 MoE-layer tokens/s; % of HBM BW (decode) / % FP4 TC peak (prefill)"
+FP4_BYTES_PER_ELT = 0.5625  # 4-bit code + one E4M3 scale per 16 elements
+L2_FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def setup_layer(wl: W.Workload, dev, seed: int = 0):
+    """Draws the workload on the device, quantises the weights with the library, and
+    calibrates the per-expert requantisation scales with one forward (h_amax / 2688)."""
+    act = W.make_activations(wl, seed, dev)
+    wts = W.make_weights(wl, seed, dev)
+    experts = ops.NVFP4Experts.from_float(wts["w_gate"], wts["w_up"], wts["w_down"])
+    ones = torch.ones(wl.E, dtype=torch.float32, device=dev)
+    layer = ops.MoeFFN(experts, wl.k, ones)
+    h_amax = torch.empty(wl.E, dtype=torch.float32, device=dev)
+    layer(act["x"], act["logits"], h_amax=h_amax)
+    torch.cuda.synchronize()
+    s_h = torch.where(h_amax > 0, h_amax / 2688.0, ones)
+    layer = ops.MoeFFN(experts, wl.k, s_h)
+    return act, wts, experts, layer
+
+
+def algorithmic(wl: W.Workload, n_active: int):
+    """Algorithmic bytes and FLOPs of one layer pass and of its gate/up stage."""
+    e = FP4_BYTES_PER_ELT
+    P = wl.T * wl.k
+    w13 = n_active * 2 * wl.I * wl.H * e
+    w2 = n_active * wl.H * wl.I * e
+    x_q = wl.T * wl.H * e
+    h_q = P * wl.I * e
+    gate_up_bytes = w13 + x_q + h_q
+    layer_bytes = w13 + w2 + wl.T * wl.H * 2 * 2 + x_q + 2 * h_q + wl.T * wl.E * 4
+    flops = 2.0 * P * 3 * wl.H * wl.I
+    return {"gate_up_bytes": gate_up_bytes, "layer_bytes": layer_bytes, "flops": flops,
+            "gate_up_flops": 2.0 * P * 2 * wl.H * wl.I}
+
+
+def time_steps(layer, act, steps: int, warmup: int, flush: torch.Tensor, dist_on: bool):
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(C.STAGES)] for _ in range(steps)]
+    out = torch.empty(act["x"].shape[0], layer.w.H, dtype=torch.bfloat16, device=act["x"].device)
+    for _ in range(warmup):
+        flush.zero_()
+        layer(act["x"], act["logits"], out=out)
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.zero_()
+        layer(act["x"], act["logits"], out=out, stage_events=ev[i])
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    step_ms = [e[0].elapsed_time(e[C.STAGES - 1]) for e in ev]
+    stage_ms = {name: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in ev)
+                for j, name in enumerate(C.STAGE_NAMES)}
+    return step_ms, stage_ms
+
+
+def time_e2e(layer, act, steps: int, warmup: int, flush: torch.Tensor):
+    """The same pass through the public API with host buffers: pinned host -> device copy of
+    x and logits, the layer, device -> host copy of the output, all inside the events."""
+    x_h = act["x"].cpu().pin_memory()
+    l_h = act["logits"].cpu().pin_memory()
+    o_h = torch.empty(x_h.shape[0], layer.w.H, dtype=torch.bfloat16).pin_memory()
+    x_d = torch.empty_like(act["x"])
+    l_d = torch.empty_like(act["logits"])
+    ms = []
+    for i in range(warmup + steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        x_d.copy_(x_h, non_blocking=True)
+        l_d.copy_(l_h, non_blocking=True)
+        out = layer(x_d, l_d)
+        o_h.copy_(out, non_blocking=True)
+        b.record()
+        b.synchronize()
+        if i >= warmup:
+            ms.append(a.elapsed_time(b))
+    h2d = x_h.numel() * x_h.element_size() + l_h.numel() * l_h.element_size()
+    d2h = o_h.numel() * o_h.element_size()
+    return statistics.mean(ms), h2d, d2h
+
+
+# ----------------------------------------------------------- oracle (CPU) ----
+def oracle_inputs(wl: W.Workload, act, wts, tokens: np.ndarray):
+    """Host copies of the inputs for the oracle: x and logits of the sampled tokens and the
+    oracle's own quantisation of the fp32 weights of every expert those tokens select."""
+    import oracle as O
+    x = act["x"].cpu().view(torch.int16).numpy().view(np.uint16)
+    logits = act["logits"].cpu().numpy()
+    ids, _ = O.route(logits[tokens], wl.k)
+    need = np.unique(ids)
+    shp = {"g": (wl.E, wl.I, wl.H), "d": (wl.E, wl.H, wl.I)}
+    arrays = {}
+    for key, name in (("g", "w_gate"), ("u", "w_up"), ("d", "w_down")):
+        s = shp["d" if key == "d" else "g"]
+        codes = np.zeros((s[0], s[1], s[2] // 2), np.uint8)
+        sf = np.zeros((s[0], s[1], s[2] // 16), np.uint8)
+        sc = np.ones(s[0], np.float32)
+        host = {int(e): wts[name][int(e)].cpu().numpy() for e in need}
+
+        def one(e):
+            c, f, t = O.quantize(host[e])
+            codes[e], sf[e], sc[e] = c, f, t
+
+        # ctypes releases the GIL while the oracle runs, so threads quantise in parallel
+        with cf.ThreadPoolExecutor(O.default_threads()) as ex:
+            list(ex.map(one, host))
+        arrays[key] = (codes, sf, sc)
+    s_x = np.float32(np.abs((x.astype(np.uint32) << 16).view(np.float32)).max()) / np.float32(2688)
+    return x[tokens], logits[tokens], arrays, float(s_x)
+
+
+def oracle_rate(wl: W.Workload, act, wts, layer, budget_s: float, max_tokens: int):
+    """Tokens/s of the oracle on a bounded token sample of the workload (host cores)."""
+    import oracle as O
+    n = min(wl.T, max_tokens)
+    tokens = np.arange(n)
+    x, logits, arr, s_x = oracle_inputs(wl, act, wts, tokens)
+    s_h = layer.h_scale.cpu().numpy()
+    nth = O.default_threads()
+    done, t0 = 0, time.perf_counter()
+    while True:
+        O.moe_ffn(x, logits, wl.k, arr["g"], arr["u"], arr["d"], x_scale=s_x, h_scale=s_h, nthreads=nth)
+        done += n
+        el = time.perf_counter() - t0
+        if el >= budget_s or done >= 64 * n:
+            break
+    return done / el, nth, f"{n} of {wl.T} tokens per pass, {done // n} passes, {el:.1f} s"
+
+
+def gpu_launches_per_step(layer) -> int:
+    # route, permute, amax pre-pass (dynamic x scale), quantise, gate/up, down, combine
+    return 6 + (1 if layer.x_scale is None else 0)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="decode", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist_on = world > 1
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if dist_on:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=dev)
+    wl = W.WORKLOADS[args.workload]
+    cfg = {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "top_k": wl.k,
+           "zipf_s": wl.zipf_s, "outlier_frac": wl.outlier_frac, "l2": "flushed before every step (256 MiB write)",
+           "seed": 0, "parallelism": f"replicas x{world}"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            if dist_on:
+                torch.distributed.destroy_process_group()
+            return
+        act, wts, _, layer = setup_layer(wl, dev)
+        import oracle as O
+        n = wl.T
+        tokens = np.arange(n)
+        x, logits, arr, s_x = oracle_inputs(wl, act, wts, tokens)
+        s_h = layer.h_scale.cpu().numpy()
+        nth = O.default_threads()
+        # a step is a bounded sample of the workload's tokens, sized to keep the run short
+        per = time.perf_counter()
+        O.moe_ffn(x[:1], logits[:1], wl.k, arr["g"], arr["u"], arr["d"], x_scale=s_x, h_scale=s_h, nthreads=nth)
+        one = time.perf_counter() - per
+        budget_tok = max(1, int(4.0 / max(one, 1e-6)))
+        sample = min(n, budget_tok)
+        for _ in range(args.warmup):
+            O.moe_ffn(x[:sample], logits[:sample], wl.k, arr["g"], arr["u"], arr["d"], x_scale=s_x,
+                      h_scale=s_h, nthreads=nth)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            O.moe_ffn(x[:sample], logits[:sample], wl.k, arr["g"], arr["u"], arr["d"], x_scale=s_x,
+                      h_scale=s_h, nthreads=nth)
+        el = time.perf_counter() - t0
+        value = sample * args.steps / el
+        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": cfg,
+                "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nth, "kind": "oracle",
+                                 "sample": f"{sample} of {n} tokens per step"},
+                "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        if dist_on:
+            torch.distributed.destroy_process_group()
+        return
+
+    act, wts, experts, layer = setup_layer(wl, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    with ClockSampler(local) as clk:
+        step_ms, stage_ms = time_steps(layer, act, args.steps, args.warmup, flush, dist_on)
+    total_ms = sum(step_ms)
+    if dist_on:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * wl.T / (ms_per_step * 1e-3)
+
+    e2e_ms, h2d, d2h = time_e2e(layer, act, args.steps, args.warmup, flush)
+    if dist_on:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    im = layer.intermediates(wl.T)
+    n_active = int(im["active"][0].item())
+    alg = algorithmic(wl, n_active)
+    pk = peaks()
+    dom_ms = stage_ms["gate_up"]
+    achieved = alg["gate_up_bytes"] / (dom_ms * 1e-3) / 1e9
+    roof = {"kernel": "gate_up (GEMV + SwiGLU + requant)", "bound": "hbm", "achieved": achieved,
+            "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
+            "peak_source": pk["source"], "algorithmic_bytes_per_launch": alg["gate_up_bytes"],
+            "touched_experts": n_active}
+    layer_bw = alg["layer_bytes"] / (ms_per_step * 1e-3) / 1e9
+    if dist_on:
+        torch.distributed.barrier()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, sample = oracle_rate(wl, act, wts, layer, args.cpu_budget, max_tokens=16)
+        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3, fp32 accumulate)", "data": "synthetic",
+            "config": cfg, "roofline": roof, "cpu_baseline": cpu,
+            "e2e": {"value": world * wl.T / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": gpu_launches_per_step(layer) * args.steps,
+            "clocks": clk.summary(),
+            "stages_ms": stage_ms,
+            "layer": {"bytes": alg["layer_bytes"], "flops": alg["flops"], "hbm_gbs": layer_bw,
+                      "hbm_frac": layer_bw / pk["hbm_gbs"], "hbm_frac_of_8tbs": layer_bw / 8000.0},
+            "path": {C.PATH_GEMV: "gemv", C.PATH_GEMM: "tcgen05"}.get(im["path"], "?"),
+        }
+        print(json.dumps(line), flush=True)
+    if dist_on:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,243 @@
+/*
+ * nvfp4moe.h - C ABI of the NVFP4 W4A4 routed mixture-of-experts feed-forward layer
+ * for NVIDIA B200 (sm_100a).  Library: libnvfp4moe.so.
+ *
+ * What the layer computes.  The pages describe routed experts stored and run as
+ * "NVFP4 W4A4" (Qwen3.8-Flash-Next-NVFP4-SSD-Stream model card, "What this model is"),
+ * two NVFP4 values per packed byte (same card, "Why Hugging Face shows 68B parameters and
+ * 8-bit precision"), 512 routed experts and prefill batches of up to 512 tokens that reuse
+ * the routed expert weights (Eider, "Qwen3.8 Flash Next", "Performance"), and grouped
+ * routed kernels for many decode rows (DwarfStar CUDA multi-GPU doc).  The pages do not
+ * define the arithmetic; this library implements the standard NVFP4 format:
+ *
+ *   value = e2m1(code) * e4m3(block scale) * fp32 tensor scale,
+ *   one E4M3 block scale per 16 consecutive elements along K,
+ *   dynamic tensor scale = amax / (6 * 448),
+ *
+ * and the routed feed-forward layer
+ *
+ *   ids, w   = top-k of the router logits (ties -> lower expert index),
+ *              w = softmax over the k selected logits
+ *   xq       = NVFP4(x)                      (one tensor scale for the layer input)
+ *   g, u     = xq . Wg[e]^T, xq . Wu[e]^T     (per selected expert e)
+ *   h        = NVFP4(silu(g) * u)            (per-expert tensor scale s_h[e], given)
+ *   y        = h . Wd[e]^T
+ *   out[t]   = bf16( sum_j w[t][j] * y[t][j] )
+ *
+ * Conventions (all entry points):
+ *  - Every pointer argument is a DEVICE pointer owned by the caller unless stated.
+ *    The library never allocates device memory: scratch comes from a caller-provided
+ *    workspace whose size is given by the matching *_workspace_size() query.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default).
+ *  - Argument checks are synchronous and return an error status before any launch.
+ *    Problems only the device can see (an expert id out of range, a duplicate id in a
+ *    token) set a sticky device status word; nvfp4moe_device_status() reads it.
+ *    Kernels never trap and never spin.
+ *  - nvfp4moe_last_error() returns a message for the last failing call of this thread.
+ *
+ * Layouts:
+ *  - codes: row-major [rows][K/2] bytes; element 2i in the low nibble of byte i,
+ *    element 2i+1 in the high nibble.  Rows start every K/2 bytes.
+ *  - block scales (SF), one E4M3 byte per 16 elements, in one of two layouts:
+ *      NVFP4MOE_SF_ROWMAJOR: [rows][K/16];
+ *      NVFP4MOE_SF_MMA: the tcgen05 block-scaled MMA layout.  Rows are grouped in
+ *        blocks of 128, K in atoms of 64 elements (4 scales).  The scale of row r,
+ *        16-element block b sits at byte
+ *          ((r/128) * (K/64) + b/4) * 512 + (r%32) * 16 + ((r%128)/32) * 4 + b%4.
+ *        The buffer spans ceil(rows/128)*128 rows; K must be a multiple of 64.
+ *  - gate/up weights of one expert are stored as ONE matrix W13 [2I][H]: its row 32c+j
+ *    is gate row 16c+j for j < 16 and up row 16c+j-16 for j >= 16 (groups of 16 rows).
+ *    Requires I % 64 == 0.
+ */
+#ifndef NVFP4MOE_H
+#define NVFP4MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Every declaration below is exported from the shared library, whatever the default
+ * symbol visibility of the translation unit that includes this header. */
+#if defined(__GNUC__)
+#pragma GCC visibility push(default)
+#endif
+
+typedef struct CUstream_st* nvfp4moe_stream_t; /* == cudaStream_t */
+
+typedef enum {
+  NVFP4MOE_OK = 0,
+  NVFP4MOE_INVALID_ARG = 1,       /* null pointer, negative size, bad enum, misalignment */
+  NVFP4MOE_UNSUPPORTED_SHAPE = 2, /* a size the kernels do not implement */
+  NVFP4MOE_WORKSPACE_TOO_SMALL = 3,
+  NVFP4MOE_CUDA_ERROR = 4,        /* a CUDA runtime call or launch failed */
+  NVFP4MOE_DEVICE_FAULT = 5       /* the device status word is non-zero */
+} nvfp4moe_status;
+
+enum { NVFP4MOE_SF_ROWMAJOR = 0, NVFP4MOE_SF_MMA = 1 };
+enum { NVFP4MOE_SCALE_GIVEN = 0, NVFP4MOE_SCALE_DYNAMIC = 1 };
+enum { NVFP4MOE_DTYPE_BF16 = 0, NVFP4MOE_DTYPE_F32 = 1 };
+
+/* Device status bits (nvfp4moe_device_status). */
+enum {
+  NVFP4MOE_DEV_BAD_EXPERT_ID = 1u << 0,  /* a routing id outside [0, E) was skipped */
+  NVFP4MOE_DEV_DUPLICATE_ID = 1u << 1,   /* a token listed the same expert twice */
+  NVFP4MOE_DEV_ROW_OVERFLOW = 1u << 2    /* permuted rows exceeded the stated capacity */
+};
+
+/* Message for the last failing call on this host thread ("" if none). */
+const char* nvfp4moe_last_error(void);
+
+/* Library version, e.g. 0x000100 = 0.1.0. */
+int32_t nvfp4moe_version(void);
+
+/* Waits for `stream`, then returns the sticky device status word of the current device
+ * in *status (0 = no fault).  If `clear` is non-zero the word is reset to 0 afterwards.
+ * Returns NVFP4MOE_OK or NVFP4MOE_CUDA_ERROR. */
+nvfp4moe_status nvfp4moe_device_status(nvfp4moe_stream_t stream, int32_t clear,
+                                       uint32_t* status);
+
+/* ------------------------------------------------------------------------------
+ * nvfp4_codec_convert - the element encoders every kernel uses, exposed for checking.
+ * in: fp32 [n].  e2m1: one code per byte in the low nibble (round to nearest, ties to
+ * the even code, saturate to +-6, sign kept).  e4m3: one E4M3 byte (round to nearest
+ * even, saturate to +-448).  Either output may be NULL.
+ * ---------------------------------------------------------------------------- */
+nvfp4moe_status nvfp4_codec_convert(const float* in, int64_t n, uint8_t* e2m1,
+                                    uint8_t* e4m3, nvfp4moe_stream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * nvfp4_quantize - bf16/fp32 -> NVFP4 block quantiser (the "A4" of W4A4 and the weight
+ * preparation step).
+ *
+ * x: [batch][rows][K] of dtype x_dtype, row stride ldx elements, batch stride
+ *    x_batch_stride elements.  x must be 16-byte aligned and ldx*elt, x_batch_stride*elt
+ *    multiples of 16 bytes.
+ * row_gather (nullable): [out_rows]; output row r of every batch item reads input row
+ *    row_gather[r] of the same item; a negative entry leaves output row r unwritten.
+ *    NULL means out_rows == rows and row r reads row r.
+ * scale_mode: GIVEN reads tensor_scale[b] for batch item b; DYNAMIC computes
+ *    tensor_scale[b] = amax(|x[b]|) / 2688 over the item's `rows` input rows and writes it.
+ * codes: [batch][out_rows][K/2] with batch stride codes_batch_stride bytes.
+ * sf: block scales in sf_layout with batch stride sf_batch_stride bytes (ROWMAJOR:
+ *    out_rows*K/16 at least; MMA: ceil(out_rows/128)*128*K/16 at least).
+ * Per 16-element block (every step one IEEE fp32 operation, round to nearest):
+ *    sf = e4m3(amax_b / (6*s_t)); if e4m3 value is 0 all codes are 0; otherwise
+ *    inv = 1 / (e4m3val(sf) * s_t) and code_i = e2m1(x_i * inv).  s_t == 0 gives
+ *    all-zero codes and scales.  Requires K % 16 == 0 (K % 64 == 0 for the MMA layout).
+ * workspace: DYNAMIC mode needs nvfp4_quantize_workspace_size() bytes; GIVEN needs none.
+ * ---------------------------------------------------------------------------- */
+size_t nvfp4_quantize_workspace_size(int64_t batch, int64_t rows, int64_t K);
+nvfp4moe_status nvfp4_quantize(const void* x, int32_t x_dtype, int64_t batch, int64_t rows,
+                               int64_t K, int64_t ldx, int64_t x_batch_stride,
+                               const int32_t* row_gather, int64_t out_rows, int32_t scale_mode,
+                               float* tensor_scale, uint8_t* codes, int64_t codes_batch_stride,
+                               uint8_t* sf, int64_t sf_batch_stride, int32_t sf_layout,
+                               void* workspace, size_t workspace_bytes,
+                               nvfp4moe_stream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * moe_route - router top-k (DwarfStar CUDA multi-GPU doc: routers run replicated next to
+ * the routed experts).
+ * logits: fp32 [T][E] (finite).  ids: int32 [T][k], experts in descending logit order,
+ * equal logits (including +0 / -0) in ascending expert index.  w: fp32 [T][k], the
+ * softmax of the k selected logits.  1 <= k <= min(E, 32), 1 <= E <= 1024.
+ * ---------------------------------------------------------------------------- */
+nvfp4moe_status moe_route(const float* logits, int32_t T, int32_t E, int32_t k, int32_t* ids,
+                          float* w, nvfp4moe_stream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * moe_permute - expert histogram and prefix-scan permutation into per-expert row groups
+ * (the grouped routed kernels of the DwarfStar doc and Eider's grouped MoE prefill).
+ *
+ * ids: int32 [T][k].  m_tile: row padding of each expert group (1 = none; 128 for the
+ * tensor-core path).  Rows of expert e occupy [padded_offsets[e], padded_offsets[e] +
+ * counts[e]) in ascending token order; experts in ascending index.  Outputs:
+ *   counts [E], offsets [E+1] (exclusive scan of counts), padded_offsets [E+1]
+ *   (exclusive scan of counts rounded up to m_tile), pair_to_row [T*k] (pair t*k+j ->
+ *   padded row), row_token [rows_cap] and row_pair [rows_cap] (padded row -> token /
+ *   pair; -1 on padding rows), tile_expert [rows_cap/m_tile] (expert of each m_tile-row
+ *   tile), active [E+1] (active[0] = number of experts with rows, then their indices in
+ *   ascending order), and zero_f32 (nullable, [E] floats set to 0; used for the optional
+ *   per-expert amax output of moe_ffn_forward).
+ * rows_cap must be >= moe_permute_rows_capacity(T, E, k, m_tile).  Out-of-range or
+ * duplicate ids are skipped (pair_to_row = -1) and flag the device status word.
+ * T*k <= 2^24, E <= 1024, k <= 32, m_tile in {1, 128}.
+ * ---------------------------------------------------------------------------- */
+int64_t moe_permute_rows_capacity(int32_t T, int32_t E, int32_t k, int32_t m_tile);
+nvfp4moe_status moe_permute(const int32_t* ids, int32_t T, int32_t E, int32_t k,
+                            int32_t m_tile, int64_t rows_cap, int32_t* counts,
+                            int32_t* offsets, int32_t* padded_offsets, int32_t* pair_to_row,
+                            int32_t* row_token, int32_t* row_pair, int32_t* tile_expert,
+                            int32_t* active, float* zero_f32, nvfp4moe_stream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * nvfp4_gemm - one NVFP4 x NVFP4 GEMM, D[M][N] = (A . B^T) * a_scale[0] * b_scale[0].
+ * A: codes [M][K/2] + SF (MMA layout over M rows); B: codes [N][K/2] + SF (MMA layout
+ * over N rows); both K-major.  D: [M][N] row-major, d_dtype BF16 or F32.
+ * M <= 16 runs the split-K GEMV kernel, larger M the tcgen05 block-scaled MMA kernel.
+ * Requires K % 256 == 0, N % 128 == 0, 16-byte aligned pointers.
+ * ---------------------------------------------------------------------------- */
+size_t nvfp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
+nvfp4moe_status nvfp4_gemm(const uint8_t* A, const uint8_t* A_sf, const float* a_scale,
+                           const uint8_t* B, const uint8_t* B_sf, const float* b_scale,
+                           int64_t M, int64_t N, int64_t K, void* D, int32_t d_dtype,
+                           void* workspace, size_t workspace_bytes, nvfp4moe_stream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * moe_ffn_forward - the whole routed feed-forward layer.
+ * ---------------------------------------------------------------------------- */
+enum { NVFP4MOE_PATH_AUTO = 0, NVFP4MOE_PATH_GEMV = 1, NVFP4MOE_PATH_GEMM = 2 };
+
+typedef struct {
+  int32_t T, H, I, E, top_k;
+  int32_t path;               /* NVFP4MOE_PATH_*; AUTO picks GEMV for T <= 16 */
+  int32_t x_scale_mode;       /* NVFP4MOE_SCALE_GIVEN or _DYNAMIC */
+  const float* x_scale;       /* [1], read when GIVEN */
+  const uint8_t* w13_codes;   /* [E][2I][H/2], gate/up rows interleaved (see above) */
+  const uint8_t* w13_sf;      /* [E][2I*H/16], MMA layout per expert */
+  const float* w13_scale;     /* [E][2]: tensor scales of gate and up */
+  const uint8_t* w2_codes;    /* [E][H][I/2] */
+  const uint8_t* w2_sf;       /* [E][H*I/16], MMA layout per expert */
+  const float* w2_scale;      /* [E] */
+  const float* h_scale;       /* [E]: requantisation tensor scale of h per expert */
+  float* h_amax;              /* nullable [E]: receives amax|h| per expert (calibration) */
+  /* nullable: NVFP4MOE_STAGES cudaEvent_t handles (created by the caller) that the call
+   * records on `stream` at its stage boundaries, for per-stage timing: [0] start,
+   * [1] after routing, [2] after the permutation, [3] after quantising x, [4] after the
+   * gate/up GEMM, [5] after the down GEMM, [6] after the combine. */
+  void* const* stage_events;
+} moe_ffn_desc;
+
+enum { NVFP4MOE_STAGES = 7 };
+
+/* Byte offsets of the intermediates inside the workspace (for inspection and tests). */
+typedef struct {
+  int64_t topk_ids, topk_w, counts, offsets, padded_offsets, pair_to_row, row_token,
+      row_pair, tile_expert, active, x_scale, x_codes, x_sf, h_codes, h_sf, slots,
+      amax_partials, total;
+  int64_t x_rows;   /* rows of x_codes / x_sf (T on the GEMV path, rows_cap otherwise) */
+  int64_t h_rows;   /* rows of h_codes / h_sf */
+  int32_t m_tile;   /* 1 on the GEMV path, 128 on the GEMM path */
+  int32_t path;     /* resolved path */
+} moe_ffn_ws_layout;
+
+nvfp4moe_status moe_ffn_workspace_layout(const moe_ffn_desc* d, moe_ffn_ws_layout* layout);
+size_t moe_ffn_workspace_size(const moe_ffn_desc* d);
+
+/* x: bf16 [T][H]; logits: fp32 [T][E]; out: bf16 [T][H]; desc is a HOST pointer.
+ * Requires H % 256 == 0, I % 64 == 0, E <= 1024, 1 <= top_k <= min(E, 32). */
+nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* desc, const void* x, const float* logits,
+                                void* out, void* workspace, size_t workspace_bytes,
+                                nvfp4moe_stream_t stream);
+
+#if defined(__GNUC__)
+#pragma GCC visibility pop
+#endif
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4MOE_H */

@@ -1,0 +1,205 @@
+// moe_ffn_forward: the routed NVFP4 W4A4 feed-forward layer, end to end on one stream.
+//
+//   route -> permute -> quantise x -> gate/up (+SwiGLU+requant) -> down -> combine
+//
+// All intermediates live in the caller's workspace at the offsets moe_ffn_workspace_layout
+// reports; group sizes stay on the device (no host synchronisation anywhere).
+#include "ffn_gemv.cuh"
+#include "ffn_gemm.cuh"
+
+namespace nvfp4moe {
+namespace {
+
+constexpr int64_t kAlign = 256;
+
+int64_t align_up(int64_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+nvfp4moe_status check_desc(const moe_ffn_desc* d, const char* fn) {
+  NVFP4_REQUIRE(d != nullptr, NVFP4MOE_INVALID_ARG, "%s: desc is NULL", fn);
+  NVFP4_REQUIRE(d->T >= 0, NVFP4MOE_INVALID_ARG, "%s: T < 0", fn);
+  NVFP4_REQUIRE(d->H > 0 && d->H % 256 == 0, NVFP4MOE_UNSUPPORTED_SHAPE, "%s: H=%d must be a positive multiple of 256", fn, d->H);
+  NVFP4_REQUIRE(d->I > 0 && d->I % 64 == 0, NVFP4MOE_UNSUPPORTED_SHAPE, "%s: I=%d must be a positive multiple of 64", fn, d->I);
+  NVFP4_REQUIRE(d->E >= 1 && d->E <= 1024, NVFP4MOE_UNSUPPORTED_SHAPE, "%s: E=%d outside [1, 1024]", fn, d->E);
+  NVFP4_REQUIRE(d->top_k >= 1 && d->top_k <= 32 && d->top_k <= d->E, NVFP4MOE_UNSUPPORTED_SHAPE,
+                "%s: top_k=%d outside [1, min(E, 32)]", fn, d->top_k);
+  NVFP4_REQUIRE(int64_t(d->T) * d->top_k <= (int64_t(1) << 24), NVFP4MOE_UNSUPPORTED_SHAPE, "%s: T*top_k > 2^24", fn);
+  NVFP4_REQUIRE(d->path >= NVFP4MOE_PATH_AUTO && d->path <= NVFP4MOE_PATH_GEMM, NVFP4MOE_INVALID_ARG,
+                "%s: bad path %d", fn, d->path);
+  NVFP4_REQUIRE(d->x_scale_mode == NVFP4MOE_SCALE_GIVEN || d->x_scale_mode == NVFP4MOE_SCALE_DYNAMIC,
+                NVFP4MOE_INVALID_ARG, "%s: bad x_scale_mode", fn);
+  return NVFP4MOE_OK;
+}
+
+int resolve_path(const moe_ffn_desc* d) {
+  if (d->path != NVFP4MOE_PATH_AUTO) return d->path;
+  return (d->T <= 16 || !gemm_path_available()) ? NVFP4MOE_PATH_GEMV : NVFP4MOE_PATH_GEMM;
+}
+
+int64_t max_active_experts(const moe_ffn_desc* d) {
+  const int64_t P = int64_t(d->T) * d->top_k;
+  return P < d->E ? P : d->E;
+}
+
+void make_layout(const moe_ffn_desc* d, moe_ffn_ws_layout* L) {
+  const int path = resolve_path(d);
+  const int64_t T = d->T, H = d->H, I = d->I, E = d->E, k = d->top_k, P = T * k;
+  const int m_tile = path == NVFP4MOE_PATH_GEMM ? 128 : 1;
+  const int64_t rows_cap = moe_permute_rows_capacity(d->T, d->E, d->top_k, m_tile);
+  int64_t o = 0;
+  auto take = [&](int64_t bytes) {
+    const int64_t at = o;
+    o = align_up(o + (bytes > 0 ? bytes : 0));
+    return at;
+  };
+  L->path = path;
+  L->m_tile = m_tile;
+  L->topk_ids = take(P * 4);
+  L->topk_w = take(P * 4);
+  L->counts = take(E * 4);
+  L->offsets = take((E + 1) * 4);
+  L->padded_offsets = take((E + 1) * 4);
+  L->pair_to_row = take(P * 4);
+  L->row_token = take(rows_cap * 4);
+  L->row_pair = take(rows_cap * 4);
+  L->tile_expert = take((rows_cap / m_tile + 1) * 4);
+  L->active = take((E + 1) * 4);
+  L->x_scale = take(4);
+  L->amax_partials = take(static_cast<int64_t>(nvfp4_quantize_workspace_size(1, T > 0 ? T : 1, H)));
+  L->x_rows = path == NVFP4MOE_PATH_GEMM ? rows_cap : T;
+  L->x_codes = take(L->x_rows * H / 2);
+  L->x_sf = take(sf_mma_bytes(L->x_rows, H));
+  L->h_rows = path == NVFP4MOE_PATH_GEMM ? rows_cap : P;
+  L->h_codes = take(L->h_rows * I / 2);
+  L->h_sf = take(sf_mma_bytes(L->h_rows, I));
+  const int ksplit = path == NVFP4MOE_PATH_GEMM ? 1 : gemv_down_ksplit(max_active_experts(d), H, I);
+  L->slots = take(int64_t(ksplit) * P * H * 4);
+  L->total = o;
+}
+
+}  // namespace
+}  // namespace nvfp4moe
+
+using namespace nvfp4moe;
+
+extern "C" {
+
+nvfp4moe_status moe_ffn_workspace_layout(const moe_ffn_desc* d, moe_ffn_ws_layout* layout) {
+  nvfp4moe_status st = check_desc(d, "moe_ffn_workspace_layout");
+  if (st != NVFP4MOE_OK) return st;
+  NVFP4_REQUIRE(layout != nullptr, NVFP4MOE_INVALID_ARG, "moe_ffn_workspace_layout: layout is NULL");
+  make_layout(d, layout);
+  return NVFP4MOE_OK;
+}
+
+size_t moe_ffn_workspace_size(const moe_ffn_desc* d) {
+  if (check_desc(d, "moe_ffn_workspace_size") != NVFP4MOE_OK) return 0;
+  moe_ffn_ws_layout L;
+  make_layout(d, &L);
+  return static_cast<size_t>(L.total);
+}
+
+nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const float* logits, void* out,
+                                void* workspace, size_t workspace_bytes, nvfp4moe_stream_t stream) {
+  const char* fn = "moe_ffn_forward";
+  nvfp4moe_status st = check_desc(d, fn);
+  if (st != NVFP4MOE_OK) return st;
+  if (d->T == 0) return NVFP4MOE_OK;
+  NVFP4_REQUIRE(x && logits && out && workspace, NVFP4MOE_INVALID_ARG, "%s: NULL pointer", fn);
+  NVFP4_REQUIRE(d->w13_codes && d->w13_sf && d->w13_scale && d->w2_codes && d->w2_sf && d->w2_scale &&
+                    d->h_scale,
+                NVFP4MOE_INVALID_ARG, "%s: NULL weight pointer in desc", fn);
+  NVFP4_REQUIRE(d->x_scale_mode == NVFP4MOE_SCALE_DYNAMIC || d->x_scale != nullptr, NVFP4MOE_INVALID_ARG,
+                "%s: GIVEN x scale needs desc->x_scale", fn);
+  NVFP4_REQUIRE(aligned16(x) && aligned16(out) && aligned16(workspace) && aligned16(d->w13_codes) &&
+                    aligned16(d->w13_sf) && aligned16(d->w2_codes) && aligned16(d->w2_sf),
+                NVFP4MOE_INVALID_ARG, "%s: x, out, workspace and weights must be 16-byte aligned", fn);
+  moe_ffn_ws_layout L;
+  make_layout(d, &L);
+  NVFP4_REQUIRE(workspace_bytes >= static_cast<size_t>(L.total), NVFP4MOE_WORKSPACE_TOO_SMALL,
+                "%s: workspace %zu < %lld bytes", fn, workspace_bytes, (long long)L.total);
+  if (L.path == NVFP4MOE_PATH_GEMM && !gemm_path_available())
+    return fail(NVFP4MOE_UNSUPPORTED_SHAPE, "%s: the tensor-core path is not built", fn);
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  auto I32 = [&](int64_t off) { return reinterpret_cast<int32_t*>(ws + off); };
+  auto F32 = [&](int64_t off) { return reinterpret_cast<float*>(ws + off); };
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int T = d->T, H = d->H, I = d->I, E = d->E, k = d->top_k;
+  const int64_t rows_cap = moe_permute_rows_capacity(T, E, k, L.m_tile);
+  auto mark = [&](int i) {
+    if (d->stage_events) cudaEventRecord(reinterpret_cast<cudaEvent_t>(d->stage_events[i]), s);
+  };
+
+  mark(0);
+  st = moe_route(logits, T, E, k, I32(L.topk_ids), F32(L.topk_w), stream);
+  if (st != NVFP4MOE_OK) return st;
+  mark(1);
+  st = moe_permute(I32(L.topk_ids), T, E, k, L.m_tile, rows_cap, I32(L.counts), I32(L.offsets),
+                   I32(L.padded_offsets), I32(L.pair_to_row), I32(L.row_token), I32(L.row_pair),
+                   I32(L.tile_expert), I32(L.active), d->h_amax, stream);
+  if (st != NVFP4MOE_OK) return st;
+  mark(2);
+
+  const bool dyn = d->x_scale_mode == NVFP4MOE_SCALE_DYNAMIC;
+  float* xs = dyn ? F32(L.x_scale) : const_cast<float*>(d->x_scale);
+  const size_t qws = nvfp4_quantize_workspace_size(1, T, H);
+  if (L.path == NVFP4MOE_PATH_GEMV) {
+    // x quantised once per token, token-major
+    st = nvfp4_quantize(x, NVFP4MOE_DTYPE_BF16, 1, T, H, H, 0, nullptr, T, d->x_scale_mode, xs,
+                        ws + L.x_codes, 0, ws + L.x_sf, 0, NVFP4MOE_SF_MMA, ws + L.amax_partials, qws, stream);
+    if (st != NVFP4MOE_OK) return st;
+    mark(3);
+    GemvGateUpArgs g;
+    g.H = H; g.I = I;
+    g.x_codes = ws + L.x_codes; g.x_sf = ws + L.x_sf; g.x_scale = xs;
+    g.offsets = I32(L.offsets); g.row_token = I32(L.row_token); g.active = I32(L.active);
+    g.w13_codes = d->w13_codes; g.w13_sf = d->w13_sf; g.w13_scale = d->w13_scale;
+    g.h_scale = d->h_scale; g.h_amax = d->h_amax;
+    g.h_codes = ws + L.h_codes; g.h_sf = ws + L.h_sf;
+    st = launch_gemv_gateup(g, max_active_experts(d), s);
+    if (st != NVFP4MOE_OK) return st;
+    mark(4);
+    GemvDownArgs dn;
+    dn.H = H; dn.I = I;
+    dn.ksplit = gemv_down_ksplit(max_active_experts(d), H, I);
+    dn.h_codes = ws + L.h_codes; dn.h_sf = ws + L.h_sf;
+    dn.offsets = I32(L.offsets); dn.row_pair = I32(L.row_pair); dn.active = I32(L.active);
+    dn.w2_codes = d->w2_codes; dn.w2_sf = d->w2_sf; dn.w2_scale = d->w2_scale;
+    dn.h_scale = d->h_scale; dn.topk_w = F32(L.topk_w);
+    dn.slots = F32(L.slots); dn.slot_stride = int64_t(T) * k * H;
+    st = launch_gemv_down(dn, max_active_experts(d), s);
+    if (st != NVFP4MOE_OK) return st;
+    mark(5);
+    st = launch_combine(F32(L.slots), dn.slot_stride, dn.ksplit, I32(L.pair_to_row), T, H, k, out, s);
+    if (st != NVFP4MOE_OK) return st;
+    mark(6);
+    return NVFP4MOE_OK;
+  }
+
+  // tensor-core path: x quantised straight into the padded permuted rows
+  st = nvfp4_quantize(x, NVFP4MOE_DTYPE_BF16, 1, T, H, H, 0, I32(L.row_token), rows_cap, d->x_scale_mode,
+                      xs, ws + L.x_codes, 0, ws + L.x_sf, 0, NVFP4MOE_SF_MMA, ws + L.amax_partials, qws, stream);
+  if (st != NVFP4MOE_OK) return st;
+  mark(3);
+  GemmFfnArgs a;
+  a.T = T; a.H = H; a.I = I; a.E = E; a.k = k;
+  a.rows_cap = rows_cap;
+  a.x_codes = ws + L.x_codes; a.x_sf = ws + L.x_sf; a.x_scale = xs;
+  a.padded_offsets = I32(L.padded_offsets); a.counts = I32(L.counts);
+  a.tile_expert = I32(L.tile_expert); a.row_pair = I32(L.row_pair);
+  a.w13_codes = d->w13_codes; a.w13_sf = d->w13_sf; a.w13_scale = d->w13_scale;
+  a.w2_codes = d->w2_codes; a.w2_sf = d->w2_sf; a.w2_scale = d->w2_scale;
+  a.h_scale = d->h_scale; a.h_amax = d->h_amax;
+  a.h_codes = ws + L.h_codes; a.h_sf = ws + L.h_sf;
+  a.topk_w = F32(L.topk_w); a.slots = F32(L.slots);
+  a.stage_events = d->stage_events;
+  st = launch_gemm_ffn(a, s);
+  if (st != NVFP4MOE_OK) return st;
+  mark(5);
+  st = launch_combine(F32(L.slots), int64_t(T) * k * H, 1, I32(L.pair_to_row), T, H, k, out, s);
+  if (st != NVFP4MOE_OK) return st;
+  mark(6);
+  return NVFP4MOE_OK;
+}
+
+}  // extern "C"

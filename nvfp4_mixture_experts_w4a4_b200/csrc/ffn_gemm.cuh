@@ -1,0 +1,36 @@
+// Launch interface of the tensor-core (tcgen05 block-scaled MMA) grouped GEMM path.
+#pragma once
+
+#include "common.cuh"
+
+namespace nvfp4moe {
+
+struct GemmFfnArgs {
+  int T, H, I, E, k;
+  int64_t rows_cap;               // padded permuted rows (m_tile = 128)
+  const uint8_t* x_codes;         // [rows_cap][H/2], padded permuted rows
+  const uint8_t* x_sf;            // MMA layout over rows_cap rows
+  const float* x_scale;           // [1]
+  const int32_t* padded_offsets;  // [E+1]
+  const int32_t* counts;          // [E]
+  const int32_t* tile_expert;     // [rows_cap/128]
+  const int32_t* row_pair;        // [rows_cap], -1 on padding rows
+  const uint8_t* w13_codes;
+  const uint8_t* w13_sf;
+  const float* w13_scale;         // [E][2]
+  const uint8_t* w2_codes;
+  const uint8_t* w2_sf;
+  const float* w2_scale;          // [E]
+  const float* h_scale;           // [E]
+  float* h_amax;                  // nullable
+  uint8_t* h_codes;               // [rows_cap][I/2]
+  uint8_t* h_sf;                  // MMA layout over rows_cap rows
+  const float* topk_w;            // [T*k] by pair
+  float* slots;                   // [T*k][H] by pair
+  void* const* stage_events;      // nullable; [4] is recorded between gate/up and down
+};
+
+bool gemm_path_available();
+nvfp4moe_status launch_gemm_ffn(const GemmFfnArgs& a, cudaStream_t s);
+
+}  // namespace nvfp4moe

@@ -1,0 +1,50 @@
+// Launch interface of the decode (GEMV) kernels.
+#pragma once
+
+#include "common.cuh"
+
+namespace nvfp4moe {
+
+struct GemvGateUpArgs {
+  int H, I;
+  const uint8_t* x_codes;   // [T][H/2], token-major
+  const uint8_t* x_sf;      // MMA layout over T rows
+  const float* x_scale;     // [1]
+  const int32_t* offsets;   // [E+1] rows of each expert (unpadded permutation)
+  const int32_t* row_token; // [P]
+  const int32_t* active;    // [E+1]
+  const uint8_t* w13_codes;
+  const uint8_t* w13_sf;
+  const float* w13_scale;   // [E][2]
+  const float* h_scale;     // [E]
+  float* h_amax;            // nullable [E]
+  uint8_t* h_codes;         // [P][I/2]
+  uint8_t* h_sf;            // MMA layout over P rows
+};
+
+struct GemvDownArgs {
+  int H, I;
+  int ksplit;
+  const uint8_t* h_codes;
+  const uint8_t* h_sf;
+  const int32_t* offsets;
+  const int32_t* row_pair;  // [P] permuted row -> pair
+  const int32_t* active;
+  const uint8_t* w2_codes;
+  const uint8_t* w2_sf;
+  const float* w2_scale;    // [E]
+  const float* h_scale;     // [E]
+  const float* topk_w;      // [P] by pair; nullable (weight 1)
+  float* slots;             // [ksplit][P][H]
+  int64_t slot_stride;      // P*H
+};
+
+int gemv_lanes_per_row(int64_t K);
+int gemv_down_ksplit(int64_t max_active, int64_t H, int64_t I);
+nvfp4moe_status launch_gemv_gateup(const GemvGateUpArgs& a, int64_t max_active, cudaStream_t s);
+nvfp4moe_status launch_gemv_down(const GemvDownArgs& a, int64_t max_active, cudaStream_t s);
+nvfp4moe_status launch_combine(const float* slots, int64_t slot_stride, int ksplit,
+                               const int32_t* pair_to_row, int T, int H, int k, void* out,
+                               cudaStream_t s);
+
+}  // namespace nvfp4moe

@@ -1,0 +1,283 @@
+"""PyTorch-facing binding of libnvfp4moe: the C ABI's entry points under the same names.
+
+Every function here only marshals arguments: it allocates outputs and workspaces with torch
+(device memory is torch's job), passes raw device pointers and the current CUDA stream to
+the library, and raises on a non-OK status.  All arithmetic runs in the library's kernels.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib as C
+from ._lib import check, lib
+
+__all__ = [
+    "nvfp4_quantize", "moe_route", "moe_permute", "nvfp4_gemm", "moe_ffn_forward", "codec_convert",
+    "device_status", "sf_mma_bytes", "NVFP4Experts", "MoeFFN",
+]
+
+
+def _p(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _s(stream=None):
+    st = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(st.cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libnvfp4moe takes CUDA tensors only")
+
+
+def sf_mma_bytes(rows: int, K: int) -> int:
+    return ((rows + 127) // 128) * 128 * (K // 16)
+
+
+def _sf_bytes(rows: int, K: int, layout: int) -> int:
+    return sf_mma_bytes(rows, K) if layout == C.SF_MMA else rows * (K // 16)
+
+
+def codec_convert(x: torch.Tensor):
+    """fp32 -> (E2M1 code per byte, E4M3 byte) with the kernels' element encoders."""
+    _need_cuda(x)
+    x = x.contiguous().view(-1)
+    e2m1 = torch.empty(x.numel(), dtype=torch.uint8, device=x.device)
+    e4m3 = torch.empty_like(e2m1)
+    check(lib().nvfp4_codec_convert(_p(x), x.numel(), _p(e2m1), _p(e4m3), _s()), "nvfp4_codec_convert")
+    return e2m1, e4m3
+
+
+def device_status(clear: bool = True) -> int:
+    v = ctypes.c_uint32(0)
+    check(lib().nvfp4moe_device_status(_s(), int(clear), ctypes.byref(v)), "nvfp4moe_device_status")
+    return int(v.value)
+
+
+def nvfp4_quantize(x: torch.Tensor, tensor_scale: torch.Tensor | None = None, *, sf_layout: int = C.SF_MMA,
+                   row_gather: torch.Tensor | None = None, out_rows: int | None = None,
+                   codes: torch.Tensor | None = None, sf: torch.Tensor | None = None,
+                   scale_out: torch.Tensor | None = None):
+    """Quantises x ([rows, K] or [batch, rows, K], bf16 or fp32) to NVFP4.
+
+    tensor_scale: None -> dynamic (amax / 2688 per batch item, returned); otherwise a CUDA
+    fp32 tensor with one scale per batch item.  Returns (codes, sf, scale) where codes is
+    uint8 [batch?, out_rows, K/2] and sf uint8 [batch?, sf bytes] in `sf_layout`.
+    """
+    _need_cuda(x, tensor_scale, row_gather)
+    squeeze = x.dim() == 2
+    x3 = x.unsqueeze(0) if squeeze else x
+    if x3.stride(-1) != 1:
+        raise ValueError("x must have unit stride along K")
+    B, rows, K = x3.shape
+    if x3.dtype == torch.bfloat16:
+        dt = C.DTYPE_BF16
+    elif x3.dtype == torch.float32:
+        dt = C.DTYPE_F32
+    else:
+        raise ValueError("x must be bf16 or fp32")
+    orow = rows if row_gather is None else int(out_rows if out_rows is not None else row_gather.numel())
+    dev = x.device
+    if codes is None:
+        codes = torch.empty(B, orow, K // 2, dtype=torch.uint8, device=dev)
+    sfb = _sf_bytes(orow, K, sf_layout)
+    if sf is None:
+        sf = torch.empty(B, sfb, dtype=torch.uint8, device=dev)
+    dynamic = tensor_scale is None
+    if dynamic:
+        scale = scale_out if scale_out is not None else torch.empty(B, dtype=torch.float32, device=dev)
+    else:
+        scale = tensor_scale.to(torch.float32).contiguous().view(-1)
+    wsb = lib().nvfp4_quantize_workspace_size(B, rows, K) if dynamic else 0
+    ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+    rg = None if row_gather is None else row_gather.to(torch.int32).contiguous()
+    st = lib().nvfp4_quantize(
+        _p(x3), dt, B, rows, K, x3.stride(1), x3.stride(0) if B > 1 else rows * x3.stride(1), _p(rg), orow,
+        C.SCALE_DYNAMIC if dynamic else C.SCALE_GIVEN, _p(scale), _p(codes),
+        codes.stride(0) if codes.dim() == 3 else 0, _p(sf), sf.stride(0) if sf.dim() == 2 else 0,
+        sf_layout, _p(ws), wsb, _s())
+    check(st, "nvfp4_quantize")
+    if squeeze:
+        return codes[0], sf[0], scale
+    return codes, sf, scale
+
+
+def moe_route(logits: torch.Tensor, k: int):
+    """Top-k expert ids (int32 [T, k]) and softmax-over-k weights (fp32 [T, k])."""
+    _need_cuda(logits)
+    logits = logits.to(torch.float32).contiguous()
+    T, E = logits.shape
+    ids = torch.empty(T, k, dtype=torch.int32, device=logits.device)
+    w = torch.empty(T, k, dtype=torch.float32, device=logits.device)
+    check(lib().moe_route(_p(logits), T, E, k, _p(ids), _p(w), _s()), "moe_route")
+    return ids, w
+
+
+def moe_permute(ids: torch.Tensor, E: int, m_tile: int = 1, zero_f32: torch.Tensor | None = None) -> dict:
+    _need_cuda(ids)
+    ids = ids.to(torch.int32).contiguous()
+    T, k = ids.shape
+    cap = int(lib().moe_permute_rows_capacity(T, E, k, m_tile))
+    dev = ids.device
+    i32 = dict(dtype=torch.int32, device=dev)
+    r = dict(
+        counts=torch.empty(E, **i32), offsets=torch.empty(E + 1, **i32),
+        padded_offsets=torch.empty(E + 1, **i32), pair_to_row=torch.empty(max(T * k, 1), **i32),
+        row_token=torch.empty(max(cap, 1), **i32), row_pair=torch.empty(max(cap, 1), **i32),
+        tile_expert=torch.empty(max(cap // m_tile, 1), **i32), active=torch.empty(E + 1, **i32),
+    )
+    st = lib().moe_permute(_p(ids), T, E, k, m_tile, cap, _p(r["counts"]), _p(r["offsets"]),
+                           _p(r["padded_offsets"]), _p(r["pair_to_row"]), _p(r["row_token"]),
+                           _p(r["row_pair"]), _p(r["tile_expert"]), _p(r["active"]), _p(zero_f32), _s())
+    check(st, "moe_permute")
+    r["rows_cap"] = cap
+    return r
+
+
+def nvfp4_gemm(A: torch.Tensor, A_sf: torch.Tensor, a_scale: torch.Tensor, B: torch.Tensor, B_sf: torch.Tensor,
+               b_scale: torch.Tensor, out_dtype=torch.bfloat16) -> torch.Tensor:
+    """D = (A . B^T) * a_scale * b_scale for NVFP4 A [M, K/2] and B [N, K/2] (MMA-layout scales)."""
+    _need_cuda(A, A_sf, a_scale, B, B_sf, b_scale)
+    M, N, K = A.shape[0], B.shape[0], A.shape[1] * 2
+    D = torch.empty(M, N, dtype=out_dtype, device=A.device)
+    wsb = lib().nvfp4_gemm_workspace_size(M, N, K)
+    ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=A.device)
+    dt = C.DTYPE_F32 if out_dtype == torch.float32 else C.DTYPE_BF16
+    st = lib().nvfp4_gemm(_p(A), _p(A_sf), _p(a_scale), _p(B), _p(B_sf), _p(b_scale), M, N, K, _p(D), dt,
+                          _p(ws), wsb, _s())
+    check(st, "nvfp4_gemm")
+    return D
+
+
+class NVFP4Experts:
+    """Per-expert NVFP4 weights in the library's layout (W13 interleaved, MMA scales)."""
+
+    def __init__(self, w13_codes, w13_sf, w13_scale, w2_codes, w2_sf, w2_scale):
+        self.w13_codes, self.w13_sf, self.w13_scale = w13_codes, w13_sf, w13_scale
+        self.w2_codes, self.w2_sf, self.w2_scale = w2_codes, w2_sf, w2_scale
+        self.E, twoI, h2 = w13_codes.shape
+        self.I, self.H = twoI // 2, h2 * 2
+
+    @staticmethod
+    def interleave_maps(I: int, device) -> tuple[torch.Tensor, torch.Tensor]:
+        """Row gathers that place gate rows at W13 rows 32c+j (j<16) and up rows at 32c+16+j."""
+        r = torch.arange(2 * I, device=device, dtype=torch.int32)
+        c, j = r // 32, r % 32
+        gate = torch.where(j < 16, 16 * c + j, torch.full_like(r, -1))
+        up = torch.where(j >= 16, 16 * c + j - 16, torch.full_like(r, -1))
+        return gate, up
+
+    @classmethod
+    def from_float(cls, w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor) -> "NVFP4Experts":
+        """Quantises fp32 weights [E, I, H] / [E, H, I] with one dynamic scale per expert and matrix."""
+        E, I, H = w_gate.shape
+        dev = w_gate.device
+        g_map, u_map = cls.interleave_maps(I, dev)
+        w13_codes = torch.empty(E, 2 * I, H // 2, dtype=torch.uint8, device=dev)
+        w13_sf = torch.empty(E, sf_mma_bytes(2 * I, H), dtype=torch.uint8, device=dev)
+        _, _, sg = nvfp4_quantize(w_gate, None, row_gather=g_map, out_rows=2 * I, codes=w13_codes, sf=w13_sf)
+        _, _, su = nvfp4_quantize(w_up, None, row_gather=u_map, out_rows=2 * I, codes=w13_codes, sf=w13_sf)
+        w2_codes, w2_sf, sd = nvfp4_quantize(w_down, None)
+        return cls(w13_codes, w13_sf, torch.stack([sg, su], 1).contiguous(), w2_codes, w2_sf, sd.contiguous())
+
+
+class MoeFFN:
+    """The routed NVFP4 W4A4 feed-forward layer (moe_ffn_forward) with a cached workspace."""
+
+    def __init__(self, experts: NVFP4Experts, top_k: int, h_scale: torch.Tensor, x_scale: torch.Tensor | None = None,
+                 path: int = C.PATH_AUTO):
+        self.w = experts
+        self.top_k = top_k
+        self.h_scale = h_scale.to(torch.float32).contiguous()
+        self.x_scale = None if x_scale is None else x_scale.to(torch.float32).contiguous().view(1)
+        self.path = path
+        self._ws = {}
+
+    def desc(self, T: int, h_amax: torch.Tensor | None = None, events=None) -> C.MoeFfnDesc:
+        w = self.w
+        d = C.MoeFfnDesc()
+        d.T, d.H, d.I, d.E, d.top_k = T, w.H, w.I, w.E, self.top_k
+        d.path = self.path
+        d.x_scale_mode = C.SCALE_DYNAMIC if self.x_scale is None else C.SCALE_GIVEN
+        d.x_scale = None if self.x_scale is None else self.x_scale.data_ptr()
+        d.w13_codes, d.w13_sf, d.w13_scale = w.w13_codes.data_ptr(), w.w13_sf.data_ptr(), w.w13_scale.data_ptr()
+        d.w2_codes, d.w2_sf, d.w2_scale = w.w2_codes.data_ptr(), w.w2_sf.data_ptr(), w.w2_scale.data_ptr()
+        d.h_scale = self.h_scale.data_ptr()
+        d.h_amax = None if h_amax is None else h_amax.data_ptr()
+        d.stage_events = None if events is None else ctypes.cast(events, ctypes.c_void_p).value
+        return d
+
+    def layout(self, T: int) -> C.MoeFfnWsLayout:
+        L = C.MoeFfnWsLayout()
+        d = self.desc(T)
+        check(lib().moe_ffn_workspace_layout(ctypes.byref(d), ctypes.byref(L)), "moe_ffn_workspace_layout")
+        return L
+
+    def workspace(self, T: int) -> torch.Tensor:
+        if T not in self._ws:
+            L = self.layout(T)
+            self._ws[T] = torch.empty(max(L.total, 16), dtype=torch.uint8, device=self.w.w13_codes.device)
+        return self._ws[T]
+
+    def forward(self, x: torch.Tensor, logits: torch.Tensor, out: torch.Tensor | None = None,
+                h_amax: torch.Tensor | None = None, stage_events=None) -> torch.Tensor:
+        """stage_events: optional list of 7 torch.cuda.Event (enable_timing) recorded at the
+        layer's stage boundaries (see NVFP4MOE_STAGES)."""
+        _need_cuda(x, logits, out, h_amax)
+        T = x.shape[0]
+        x = x.contiguous()
+        logits = logits.to(torch.float32).contiguous()
+        if out is None:
+            out = torch.empty(T, self.w.H, dtype=torch.bfloat16, device=x.device)
+        ws = self.workspace(T)
+        ev = None
+        if stage_events is not None:
+            if len(stage_events) != C.STAGES:
+                raise ValueError(f"stage_events needs {C.STAGES} events")
+            for e in stage_events:
+                if not e.cuda_event:  # torch creates the event lazily: materialise it
+                    e.record()
+            ev = (ctypes.c_void_p * C.STAGES)(*[e.cuda_event for e in stage_events])
+        d = self.desc(T, h_amax, ev)
+        st = lib().moe_ffn_forward(ctypes.byref(d), _p(x), _p(logits), _p(out), _p(ws), ws.numel(), _s())
+        check(st, "moe_ffn_forward")
+        return out
+
+    __call__ = forward
+
+    def intermediates(self, T: int) -> dict:
+        """Views of the intermediates of the last forward with T tokens (for inspection)."""
+        L = self.layout(T)
+        ws = self.workspace(T)
+        w, k = self.w, self.top_k
+        P = T * k
+
+        def view(off, n, dtype):
+            nbytes = n * torch.tensor([], dtype=dtype).element_size()
+            return ws[off:off + nbytes].view(dtype)
+
+        return dict(
+            path=L.path, m_tile=L.m_tile,
+            topk_ids=view(L.topk_ids, P, torch.int32).view(T, k),
+            topk_w=view(L.topk_w, P, torch.float32).view(T, k),
+            counts=view(L.counts, w.E, torch.int32), offsets=view(L.offsets, w.E + 1, torch.int32),
+            padded_offsets=view(L.padded_offsets, w.E + 1, torch.int32),
+            pair_to_row=view(L.pair_to_row, P, torch.int32),
+            row_token=view(L.row_token, L.h_rows if L.path == C.PATH_GEMM else P, torch.int32),
+            row_pair=view(L.row_pair, L.h_rows if L.path == C.PATH_GEMM else P, torch.int32),
+            active=view(L.active, w.E + 1, torch.int32),
+            x_scale=view(L.x_scale, 1, torch.float32),
+            x_codes=view(L.x_codes, L.x_rows * w.H // 2, torch.uint8).view(L.x_rows, w.H // 2),
+            x_sf=view(L.x_sf, sf_mma_bytes(L.x_rows, w.H), torch.uint8),
+            h_codes=view(L.h_codes, L.h_rows * w.I // 2, torch.uint8).view(L.h_rows, w.I // 2),
+            h_sf=view(L.h_sf, sf_mma_bytes(L.h_rows, w.I), torch.uint8),
+            x_rows=L.x_rows, h_rows=L.h_rows,
+        )
+
+
+def moe_ffn_forward(layer: MoeFFN, x: torch.Tensor, logits: torch.Tensor, **kw) -> torch.Tensor:
+    return layer.forward(x, logits, **kw)

@@ -1,0 +1,173 @@
+"""Shared helpers of the GPU parity tests: running the oracle and the library on the same
+seeded inputs and applying the stated tolerances."""
+from __future__ import annotations
+
+import concurrent.futures as cf
+import os
+
+import numpy as np
+import torch
+
+import oracle as O
+from nvfp4_mixture_experts_w4a4_b200 import _lib as C
+from nvfp4_mixture_experts_w4a4_b200 import ops, workloads as W
+from tests.helpers import layouts as LY
+from tests.helpers import refquant as R
+
+# Output tolerance of the layer: |gpu - oracle| <= 1e-2 * max(|oracle|, RMS of the oracle row).
+OUT_RTOL = 1e-2
+# At most this fraction of requantised h codes may differ, each by one grid step.
+H_CODE_FRAC = 1e-3
+
+
+def need_gpu():
+    if not torch.cuda.is_available():
+        raise RuntimeError("this test needs a CUDA device")
+    return torch.device("cuda:0")
+
+
+def bf16_bits(x: torch.Tensor) -> np.ndarray:
+    return x.detach().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (b.astype(np.uint32) << 16).view(np.float32)
+
+
+def quantize_experts_parallel(w: np.ndarray, nthreads: int | None = None):
+    """Oracle quantisation of stacked weights [E, N, K] on several threads (ctypes releases
+    the GIL while the oracle runs)."""
+    E, N, K = w.shape
+    codes = np.zeros((E, N, K // 2), np.uint8)
+    sf = np.zeros((E, N, K // 16), np.uint8)
+    sc = np.zeros(E, np.float32)
+
+    def one(e):
+        c, s, t = O.quantize(w[e])
+        codes[e], sf[e], sc[e] = c, s, t
+
+    with cf.ThreadPoolExecutor(nthreads or O.default_threads()) as ex:
+        list(ex.map(one, range(E)))
+    return codes, sf, sc
+
+
+def check_out(gpu_bf16: np.ndarray, ref_f64: np.ndarray, rtol: float = OUT_RTOL):
+    g = bits_to_f32(gpu_bf16).astype(np.float64)
+    rms = np.sqrt((ref_f64 ** 2).mean(axis=1, keepdims=True))
+    bound = rtol * np.maximum(np.abs(ref_f64), rms)
+    err = np.abs(g - ref_f64)
+    bad = err > bound
+    assert not bad.any(), (f"{bad.sum()} of {bad.size} outputs outside tolerance; worst "
+                           f"err/bound={float((err / np.maximum(bound, 1e-30)).max()):.3g}")
+    return float((err / np.maximum(bound, 1e-30)).max())
+
+
+def _signed_index(codes: np.ndarray) -> np.ndarray:
+    mag = (codes & 7).astype(np.int32)
+    return np.where(codes & 8, -mag, mag)
+
+
+def unpack(codes: np.ndarray) -> np.ndarray:
+    out = np.empty(codes.shape[:-1] + (codes.shape[-1] * 2,), np.uint8)
+    out[..., 0::2] = codes & 0xF
+    out[..., 1::2] = codes >> 4
+    return out
+
+
+def check_h_codes(gpu_codes, gpu_sf, ref_codes, ref_sf, frac: float = H_CODE_FRAC):
+    """Requantised h: at most `frac` of the codes differ; where the block scale agrees, a
+    differing code is one grid step away (signed grid index within 1)."""
+    gc, rc = unpack(gpu_codes), unpack(ref_codes)
+    rows, K = gc.shape
+    gs = np.repeat(gpu_sf, 16, axis=1)
+    rs = np.repeat(ref_sf, 16, axis=1)
+    same_sf = gs == rs
+    differ = (gc != rc) | ~same_sf
+    n = int(differ.sum())
+    assert n <= frac * differ.size, f"{n} of {differ.size} h codes differ"
+    step = np.abs(_signed_index(gc) - _signed_index(rc))
+    # -0 and +0 are the same value
+    zero_pair = ((gc & 7) == 0) & ((rc & 7) == 0)
+    step = np.where(zero_pair, 0, step)
+    assert (step[same_sf] <= 1).all(), "an h code differs by more than one grid step"
+    return n
+
+
+def layer_inputs(wl: W.Workload, seed: int = 0):
+    """CPU-drawn inputs and oracle-quantised weights of a workload small enough to draw on the CPU."""
+    act = W.make_activations(wl, seed, "cpu")
+    wts = W.make_weights(wl, seed, "cpu")
+    wg = quantize_experts_parallel(wts["w_gate"].numpy())
+    wu = quantize_experts_parallel(wts["w_up"].numpy())
+    wd = quantize_experts_parallel(wts["w_down"].numpy())
+    return act, wts, wg, wu, wd
+
+
+def experts_from_oracle(wg, wu, wd, dev) -> ops.NVFP4Experts:
+    arrs = LY.experts_to_device_layout(wg, wu, wd)
+    t = [torch.from_numpy(np.ascontiguousarray(a)).to(dev) for a in arrs]
+    return ops.NVFP4Experts(*t)
+
+
+def run_layer_pair(wl: W.Workload, path: int, seed: int = 0, dev=None, given_x_scale: bool = False):
+    """Runs oracle and library on the same inputs; returns (oracle result, gpu out, layer)."""
+    dev = dev or need_gpu()
+    act, wts, wg, wu, wd = layer_inputs(wl, seed)
+    x_bits = bf16_bits(act["x"])
+    logits = act["logits"].numpy()
+    xs = None
+    if given_x_scale:
+        xs = float(np.float32(np.abs(bits_to_f32(x_bits)).max()) / np.float32(2688) * np.float32(1.5))
+    ref = O.moe_ffn(x_bits, logits, wl.k, wg, wu, wd, x_scale=xs)
+    experts = experts_from_oracle(wg, wu, wd, dev)
+    layer = ops.MoeFFN(experts, wl.k, torch.from_numpy(ref["h_scale"]).to(dev),
+                       x_scale=None if xs is None else torch.tensor([xs], device=dev), path=path)
+    h_amax = torch.empty(wl.E, dtype=torch.float32, device=dev)
+    out = layer(act["x"].to(dev), act["logits"].to(dev), h_amax=h_amax)
+    torch.cuda.synchronize()
+    return ref, out, layer, h_amax
+
+
+def check_layer(wl: W.Workload, ref: dict, out: torch.Tensor, layer: ops.MoeFFN, h_amax: torch.Tensor):
+    T, k, H, I, E = wl.T, wl.k, wl.H, wl.I, wl.E
+    im = layer.intermediates(T)
+    # routing and permutation: bit-exact
+    assert np.array_equal(im["topk_ids"].cpu().numpy(), ref["ids"])
+    np.testing.assert_allclose(im["topk_w"].cpu().numpy(), ref["w"], rtol=2e-6, atol=1e-7)
+    assert np.array_equal(im["counts"].cpu().numpy(), ref["counts"])
+    assert np.array_equal(im["offsets"].cpu().numpy(), ref["offsets"])
+    # x scale and codes: bit-exact
+    assert im["x_scale"].item() == np.float32(ref["x_scale"]) or layer.x_scale is not None
+    p2r = im["pair_to_row"].cpu().numpy()
+    if im["path"] == C.PATH_GEMV:
+        assert np.array_equal(p2r, ref["pair_to_row"])
+        assert np.array_equal(im["row_token"].cpu().numpy()[:T * k], ref["row_token"])
+        xc = im["x_codes"].cpu().numpy()
+        xsf = LY.from_mma(im["x_sf"].cpu().numpy(), T, H)
+        assert np.array_equal(xc, ref["x_codes"])
+        assert np.array_equal(xsf, ref["x_sf"])
+        hrows = np.arange(T * k)
+    else:
+        po = im["padded_offsets"].cpu().numpy()
+        off = ref["offsets"]
+        counts = ref["counts"]
+        assert np.array_equal(po, np.concatenate([[0], np.cumsum((counts + 127) // 128 * 128)]))
+        # padded row -> unpadded row: same expert, same rank
+        e_of_pair = ref["ids"].reshape(-1)
+        assert np.array_equal(p2r - po[e_of_pair] + off[e_of_pair], ref["pair_to_row"])
+        hrows = p2r[np.argsort(ref["pair_to_row"])]  # padded row of each oracle row
+        rt = im["row_token"].cpu().numpy()
+        assert np.array_equal(rt[hrows], ref["row_token"])
+        xc = im["x_codes"].cpu().numpy()[hrows]
+        xsf = LY.from_mma(im["x_sf"].cpu().numpy(), im["x_rows"], H)[hrows]
+        assert np.array_equal(xc, ref["x_codes"][ref["row_token"]])
+        assert np.array_equal(xsf, ref["x_sf"][ref["row_token"]])
+    # h: within the requantisation tolerance
+    hc = im["h_codes"].cpu().numpy()[hrows]
+    hsf = LY.from_mma(im["h_sf"].cpu().numpy(), im["h_rows"], I)[hrows]
+    check_h_codes(hc, hsf, ref["h_codes"], ref["h_sf"])
+    # calibration output: amax of h per expert, within fp32 accumulation differences
+    ha = h_amax.cpu().numpy()
+    np.testing.assert_allclose(ha[ref["counts"] > 0], ref["h_amax"][ref["counts"] > 0], rtol=1e-4)
+    # layer output
+    return check_out(bf16_bits(out), ref["out_f64"])

@@ -1,0 +1,87 @@
+"""Host-side checks of the C ABI (no GPU needed): the library builds, loads, exports every
+function that include/*.h declares, the binding declares each of them, and argument
+errors come back as status codes with a message before anything is launched."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s+\*?([A-Za-z_][A-Za-z0-9_]*)\s*\(",
+                             src, flags=re.M):
+            names.add(m.group(1))
+    return names
+
+
+@pytest.fixture(scope="module")
+def so():
+    from nvfp4_mixture_experts_w4a4_b200 import build, _lib
+    path = build.build()
+    assert os.path.samefile(path, _lib.LIB_PATH)
+    return _lib.lib()
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for fn in ("nvfp4_quantize", "moe_route", "moe_permute", "moe_ffn_forward", "nvfp4_gemm"):
+        assert fn in names
+
+
+def test_library_exports_every_declared_symbol(so):
+    for fn in sorted(_declared_functions()):
+        assert hasattr(so, fn), f"{fn} declared in include/ but not exported"
+
+
+def test_binding_declares_every_symbol():
+    from nvfp4_mixture_experts_w4a4_b200 import _lib
+    assert _declared_functions() == set(_lib.SIGNATURES)
+
+
+def test_argument_errors_are_statuses(so):
+    from nvfp4_mixture_experts_w4a4_b200 import _lib as C
+    assert so.nvfp4moe_version() == 0x000100
+    # bad E, bad k: rejected before any device work
+    assert so.moe_route(None, 4, 2000, 2, None, None, None) == C.UNSUPPORTED_SHAPE
+    assert b"E=2000" in so.nvfp4moe_last_error()
+    assert so.moe_route(None, 4, 8, 9, None, None, None) == C.UNSUPPORTED_SHAPE
+    assert so.moe_route(None, 4, 8, 2, None, None, None) == C.INVALID_ARG
+    # quantiser: K not a multiple of 16, MMA layout with K % 64 != 0
+    assert so.nvfp4_quantize(None, 0, 1, 4, 24, 24, 0, None, 4, 0, None, None, 0, None, 0, 0, None, 0,
+                             None) == C.UNSUPPORTED_SHAPE
+    assert so.nvfp4_quantize(None, 0, 1, 4, 32, 32, 0, None, 4, 0, None, None, 0, None, 0, 1, None, 0,
+                             None) == C.UNSUPPORTED_SHAPE
+    assert so.nvfp4_quantize(None, 7, 1, 4, 32, 32, 0, None, 4, 0, None, None, 0, None, 0, 0, None, 0,
+                             None) == C.INVALID_ARG
+    # empty work is a no-op success
+    assert so.moe_route(None, 0, 8, 2, None, None, None) == C.OK
+    assert so.nvfp4_gemm(None, None, None, None, None, None, 0, 128, 256, None, 0, None, 0, None) == C.OK
+    assert so.nvfp4_gemm(None, None, None, None, None, None, 4, 100, 256, None, 0, None, 0, None) == \
+        C.UNSUPPORTED_SHAPE
+
+
+def test_workspace_queries(so):
+    from nvfp4_mixture_experts_w4a4_b200 import _lib as C
+    d = C.MoeFfnDesc()
+    d.T, d.H, d.I, d.E, d.top_k = 16, 2048, 512, 512, 10
+    d.x_scale_mode = C.SCALE_DYNAMIC
+    L = C.MoeFfnWsLayout()
+    assert so.moe_ffn_workspace_layout(ctypes.byref(d), ctypes.byref(L)) == C.OK
+    assert L.path == C.PATH_GEMV and L.m_tile == 1
+    assert so.moe_ffn_workspace_size(ctypes.byref(d)) == L.total > 0
+    offs = sorted([L.topk_ids, L.topk_w, L.counts, L.offsets, L.padded_offsets, L.pair_to_row, L.row_token,
+                   L.row_pair, L.tile_expert, L.active, L.x_scale, L.x_codes, L.x_sf, L.h_codes, L.h_sf,
+                   L.slots])
+    assert all(o % 256 == 0 for o in offs) and len(set(offs)) == len(offs) and offs[-1] < L.total
+    d.H = 100
+    assert so.moe_ffn_workspace_layout(ctypes.byref(d), ctypes.byref(L)) == C.UNSUPPORTED_SHAPE
+    assert so.moe_permute_rows_capacity(16, 512, 10, 128) == 160 + 160 * 127
+    assert so.moe_permute_rows_capacity(4096, 256, 8, 128) == 32768 + 256 * 127

@@ -1,0 +1,190 @@
+"""GPU parity of the individual kernels against the CPU oracle (through the C ABI)."""
+import concurrent.futures as cf
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from nvfp4_mixture_experts_w4a4_b200 import _lib as C
+from nvfp4_mixture_experts_w4a4_b200 import ops
+from tests import gpu_util as G
+from tests.helpers import layouts as LY
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dev():
+    return G.need_gpu()
+
+
+# ------------------------------------------------------------------ codec ----
+def test_codec_every_fp32_bit_pattern(dev):
+    """The kernels' E2M1 and E4M3 encoders against the oracle on all 2^32 fp32 patterns
+    (NaN inputs excluded: their codes are unspecified)."""
+    chunk = 1 << 27
+    pool = cf.ThreadPoolExecutor(O.default_threads())
+    for start in range(0, 1 << 32, chunk):
+        bits = torch.arange(start, start + chunk, dtype=torch.int64, device=dev).to(torch.int32)
+        vals = bits.view(torch.float32)
+        e2, e4 = ops.codec_convert(vals)
+        v = vals.cpu().numpy()
+        g2, g4 = e2.cpu().numpy(), e4.cpu().numpy()
+        parts = np.array_split(np.arange(v.size), 64)
+
+        def ref(ix):
+            return O.e2m1_encode_array(v[ix]), O.e4m3_encode_array(v[ix])
+
+        r = list(pool.map(ref, parts))
+        r2 = np.concatenate([a for a, _ in r])
+        r4 = np.concatenate([b for _, b in r])
+        ok = ~np.isnan(v)
+        bad2 = np.nonzero((g2 != r2) & ok)[0]
+        bad4 = np.nonzero((g4 != r4) & ok)[0]
+        assert bad2.size == 0, (hex(start + int(bad2[0])), v[bad2[0]], g2[bad2[0]], r2[bad2[0]])
+        assert bad4.size == 0, (hex(start + int(bad4[0])), v[bad4[0]], g4[bad4[0]], r4[bad4[0]])
+
+
+# -------------------------------------------------------------- quantiser ----
+@pytest.mark.parametrize("rows,K,dtype,given", [
+    (1, 64, torch.bfloat16, None), (37, 256, torch.bfloat16, None), (130, 2048, torch.bfloat16, None),
+    (129, 320, torch.float32, None), (5, 64, torch.float32, 0.01), (300, 512, torch.bfloat16, 0.5),
+])
+def test_quantize_parity(dev, rows, K, dtype, given):
+    g = torch.Generator().manual_seed(rows * 7 + K)
+    x = torch.randn(rows, K, generator=g, dtype=torch.float32)
+    x[:, :: max(1, K // 10)] *= 25.0            # outlier channels
+    x[min(3, rows - 1), :16] = 0.0              # a zero block
+    x[0, 16:32] *= 1e-7                          # an underflowing block
+    x = x.to(dtype)
+    xf = x.float().numpy()
+    rc, rs, rt = O.quantize(xf, tensor_scale=given)
+    for layout in (C.SF_MMA, C.SF_ROWMAJOR):
+        ts = None if given is None else torch.tensor([given], dtype=torch.float32, device=dev)
+        codes, sf, scale = ops.nvfp4_quantize(x.to(dev), ts, sf_layout=layout)
+        torch.cuda.synchronize()
+        assert scale.item() == np.float32(rt)
+        assert np.array_equal(codes.cpu().numpy(), rc)
+        sfn = sf.cpu().numpy()
+        sfr = LY.from_mma(sfn, rows, K) if layout == C.SF_MMA else sfn.reshape(rows, K // 16)
+        assert np.array_equal(sfr, rs)
+
+
+def test_quantize_batched_gather(dev):
+    """Batch of matrices, one dynamic scale each, rows gathered into an interleaved layout
+    with skipped rows left untouched (the weight-preparation use)."""
+    E, I, H = 3, 64, 256
+    g = torch.Generator().manual_seed(11)
+    w = torch.randn(E, I, H, generator=g) / 16
+    w[1] *= 3.0
+    gmap, umap = ops.NVFP4Experts.interleave_maps(I, dev)
+    codes = torch.full((E, 2 * I, H // 2), 0xAB, dtype=torch.uint8, device=dev)
+    sf = torch.zeros(E, LY.sf_mma_bytes(2 * I, H), dtype=torch.uint8, device=dev)
+    _, _, sc = ops.nvfp4_quantize(w.to(dev), None, row_gather=gmap, out_rows=2 * I, codes=codes, sf=sf)
+    torch.cuda.synchronize()
+    cn, sfn = codes.cpu().numpy(), sf.cpu().numpy()
+    for e in range(E):
+        rc, rs, rt = O.quantize(w[e].numpy())
+        assert sc[e].item() == np.float32(rt)
+        gate_rows = np.nonzero(gmap.cpu().numpy() >= 0)[0]
+        assert np.array_equal(cn[e][gate_rows], rc)
+        assert np.array_equal(LY.from_mma(sfn[e], 2 * I, H)[gate_rows], rs)
+        up_rows = np.nonzero(umap.cpu().numpy() >= 0)[0]
+        assert (cn[e][up_rows] == 0xAB).all()
+
+
+def test_quantize_empty_and_errors(dev):
+    x = torch.zeros(0, 64, dtype=torch.bfloat16, device=dev)
+    codes, sf, _ = ops.nvfp4_quantize(x, torch.ones(1, device=dev))
+    assert codes.numel() == 0
+    with pytest.raises(C.Nvfp4MoeError):
+        ops.nvfp4_quantize(torch.zeros(4, 48, device=dev), None)  # MMA layout needs K % 64
+
+
+# ---------------------------------------------------------------- routing ----
+@pytest.mark.parametrize("T,E,k", [(8, 8, 2), (16, 512, 10), (37, 256, 8), (5, 1024, 32), (3, 1, 1), (64, 33, 33)])
+def test_route_parity(dev, T, E, k):
+    g = torch.Generator().manual_seed(T * E + k)
+    logits = torch.randn(T, E, generator=g)
+    logits[0, :] = 0.25                      # all tied
+    if T > 1:
+        logits[1, ::2] = 0.0
+        logits[1, 1::2] = -0.0               # +0 / -0 ties
+    if T > 2 and E > 5:
+        logits[2, [1, 3, 5]] = 7.0           # tied winners
+    ids, w = ops.moe_route(logits.to(dev), k)
+    rid, rw = O.route(logits.numpy(), k)
+    assert np.array_equal(ids.cpu().numpy(), rid)
+    np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=2e-6, atol=1e-7)
+
+
+# ------------------------------------------------------------ permutation ----
+@pytest.mark.parametrize("T,E,k", [(8, 8, 2), (16, 512, 10), (512, 512, 10), (4096, 256, 8), (1, 4, 4), (100, 1, 1)])
+@pytest.mark.parametrize("m_tile", [1, 128])
+def test_permute_parity(dev, T, E, k, m_tile):
+    g = torch.Generator().manual_seed(T + E)
+    logits = torch.randn(T, E, generator=g)
+    if E > 4:
+        logits[:, 3] += 3.0                      # one popular expert
+        logits[:, 4] -= 50.0                     # one expert no token picks
+    ids, _ = O.route(logits.numpy(), k)
+    ref = O.permute(ids, E)
+    zero = torch.full((E,), 5.0, device=dev)
+    r = ops.moe_permute(torch.from_numpy(ids).to(dev), E, m_tile, zero_f32=zero)
+    torch.cuda.synchronize()
+    assert (zero == 0).all()
+    counts = r["counts"].cpu().numpy()
+    assert np.array_equal(counts, ref["counts"])
+    assert np.array_equal(r["offsets"].cpu().numpy(), ref["offsets"])
+    po = r["padded_offsets"].cpu().numpy()
+    assert np.array_equal(po, np.concatenate([[0], np.cumsum((counts + m_tile - 1) // m_tile * m_tile)]))
+    p2r = r["pair_to_row"].cpu().numpy()[: T * k]
+    e_of_pair = ids.reshape(-1)
+    assert np.array_equal(p2r - po[e_of_pair] + ref["offsets"][e_of_pair], ref["pair_to_row"])
+    rt, rp = r["row_token"].cpu().numpy(), r["row_pair"].cpu().numpy()
+    assert np.array_equal(rt[p2r], np.arange(T * k) // k)
+    assert np.array_equal(rp[p2r], np.arange(T * k))
+    pad = np.ones(po[-1], bool)
+    pad[p2r] = False
+    assert (rt[: po[-1]][pad] == -1).all() and (rp[: po[-1]][pad] == -1).all()
+    te = r["tile_expert"].cpu().numpy()
+    for e in range(E):
+        assert (te[po[e] // m_tile: po[e + 1] // m_tile] == e).all()
+    act = r["active"].cpu().numpy()
+    nz = np.nonzero(ref["counts"])[0]
+    assert act[0] == nz.size and np.array_equal(act[1:1 + nz.size], nz)
+    assert ops.device_status() == 0
+
+
+def test_permute_flags_bad_ids_without_hanging(dev):
+    ids = torch.tensor([[0, 1], [2, 9], [3, 3], [1, 0]], dtype=torch.int32, device=dev)
+    assert ops.device_status(clear=True) == 0
+    r = ops.moe_permute(ids, 4, 1)
+    st = ops.device_status(clear=True)
+    assert st & C.DEV_BAD_EXPERT_ID and st & C.DEV_DUPLICATE_ID
+    p2r = r["pair_to_row"].cpu().numpy()
+    assert p2r[3] == -1 and p2r[5] == -1 and (p2r[[0, 1, 2, 4, 6, 7]] >= 0).all()
+    assert ops.device_status() == 0
+
+
+# ------------------------------------------------------------------- GEMM ----
+@pytest.mark.parametrize("M,N,K", [(1, 128, 256), (3, 256, 512), (16, 384, 2048), (7, 128, 5120)])
+def test_gemm_parity(dev, M, N, K):
+    g = torch.Generator().manual_seed(M * N + K)
+    a = torch.randn(M, K, generator=g)
+    b = torch.randn(N, K, generator=g) / K ** 0.5
+    ac, asf, sa = O.quantize(a.numpy())
+    bc, bsf, sb = O.quantize(b.numpy())
+    ref = O.gemm(ac, asf, sa, bc, bsf, sb)
+    t = lambda v: torch.from_numpy(np.ascontiguousarray(v)).to(dev)
+    D = ops.nvfp4_gemm(t(ac), t(LY.to_mma(asf, K)), torch.tensor([sa], device=dev), t(bc),
+                       t(LY.to_mma(bsf, K)), torch.tensor([sb], device=dev), out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    d = D.cpu().numpy().astype(np.float64)
+    # fp32 accumulation of exact block sums: relative to the sum of |terms|
+    scale = np.abs(O.dequantize(ac, asf, sa)) @ np.abs(O.dequantize(bc, bsf, sb)).T
+    assert (np.abs(d - ref) <= 1e-5 * scale + 1e-30).all()
+    Db = ops.nvfp4_gemm(t(ac), t(LY.to_mma(asf, K)), torch.tensor([sa], device=dev), t(bc),
+                        t(LY.to_mma(bsf, K)), torch.tensor([sb], device=dev), out_dtype=torch.bfloat16)
+    G.check_out(G.bf16_bits(Db), ref)

@@ -1,0 +1,85 @@
+"""GPU parity of the whole routed layer (moe_ffn_forward through the C ABI) against the
+CPU oracle: routing, permutation and activation codes bit-exact, requantised h within the
+one-grid-step rule, outputs within 1e-2 * max(|oracle|, row RMS)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from nvfp4_mixture_experts_w4a4_b200 import _lib as C
+from nvfp4_mixture_experts_w4a4_b200 import ops, workloads as W
+from tests import gpu_util as G
+
+pytestmark = pytest.mark.gpu
+
+TINY = W.WORKLOADS["tiny"]
+# reduced versions of the larger workloads that the oracle finishes in seconds, spanning
+# several tiles and a ragged tail
+CASES = {
+    "tiny": TINY,
+    "decode_small_E": W.scaled(W.WORKLOADS["decode"], E=64, H=1024, I=256),
+    "decode_T1": W.scaled(W.WORKLOADS["decode"], T=1, E=64, H=1024, I=256),
+    "prefill_chunk_small": W.scaled(W.WORKLOADS["prefill_chunk"], T=40, E=32, H=512, I=192),
+    "long_prefill_small": W.scaled(W.WORKLOADS["long_prefill"], T=67, E=16, H=768, I=320, k=4),
+    "dense_small": W.scaled(W.WORKLOADS["dense"], T=9, H=512, I=576),
+    "top1_E2": W.scaled(TINY, T=13, E=2, k=1),
+}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_layer_gemv_path(name):
+    wl = CASES[name]
+    ref, out, layer, h_amax = G.run_layer_pair(wl, C.PATH_GEMV)
+    G.check_layer(wl, ref, out, layer, h_amax)
+    assert ops.device_status() == 0
+
+
+def test_layer_given_x_scale():
+    wl = CASES["decode_small_E"]
+    ref, out, layer, h_amax = G.run_layer_pair(wl, C.PATH_GEMV, given_x_scale=True)
+    G.check_layer(wl, ref, out, layer, h_amax)
+
+
+def test_layer_all_tokens_one_expert_and_idle_experts():
+    wl = W.scaled(TINY, T=21, E=6, k=2)
+    dev = G.need_gpu()
+    act, wts, wg, wu, wd = G.layer_inputs(wl, 3)
+    logits = np.full((wl.T, wl.E), -4.0, np.float32)
+    logits[:, 1] = 2.0           # every token's first choice
+    logits[::3, 4] = 1.0         # a third of the tokens also pick expert 4
+    x_bits = G.bf16_bits(act["x"])
+    ref = O.moe_ffn(x_bits, logits, wl.k, wg, wu, wd)
+    assert ref["counts"][1] == wl.T and ref["counts"][0] == 0
+    layer = ops.MoeFFN(G.experts_from_oracle(wg, wu, wd, dev), wl.k, torch.from_numpy(ref["h_scale"]).to(dev),
+                       path=C.PATH_GEMV)
+    h_amax = torch.empty(wl.E, device=dev)
+    out = layer(act["x"].to(dev), torch.from_numpy(logits).to(dev), h_amax=h_amax)
+    torch.cuda.synchronize()
+    G.check_layer(wl, ref, out, layer, h_amax)
+
+
+def test_layer_repeatable():
+    wl = CASES["decode_small_E"]
+    ref, out, layer, h_amax = G.run_layer_pair(wl, C.PATH_GEMV)
+    act = W.make_activations(wl, 0, "cpu")
+    again = layer(act["x"].cuda(), act["logits"].cuda())
+    torch.cuda.synchronize()
+    assert torch.equal(out, again)
+
+
+def test_weights_quantised_on_gpu_match_oracle():
+    """NVFP4Experts.from_float (the library quantiser, batched, gate/up interleaved) produces the
+    oracle's codes, scales and tensor scales bit for bit."""
+    wl = W.scaled(TINY, E=5, H=512, I=192)
+    dev = G.need_gpu()
+    wts = W.make_weights(wl, 0, "cpu")
+    ex = ops.NVFP4Experts.from_float(wts["w_gate"].to(dev), wts["w_up"].to(dev), wts["w_down"].to(dev))
+    torch.cuda.synchronize()
+    wg = G.quantize_experts_parallel(wts["w_gate"].numpy())
+    wu = G.quantize_experts_parallel(wts["w_up"].numpy())
+    wd = G.quantize_experts_parallel(wts["w_down"].numpy())
+    from tests.helpers import layouts as LY
+    ref = LY.experts_to_device_layout(wg, wu, wd)
+    got = [ex.w13_codes, ex.w13_sf, ex.w13_scale, ex.w2_codes, ex.w2_sf, ex.w2_scale]
+    for r, g in zip(ref, got):
+        assert np.array_equal(g.cpu().numpy(), r)
