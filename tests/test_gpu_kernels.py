@@ -103,7 +103,7 @@ def test_quantize_empty_and_errors(dev):
 
 
 # ---------------------------------------------------------------- routing ----
-@pytest.mark.parametrize("T,E,k", [(8, 8, 2), (16, 512, 10), (37, 256, 8), (5, 1024, 32), (3, 1, 1), (64, 33, 33)])
+@pytest.mark.parametrize("T,E,k", [(8, 8, 2), (16, 512, 10), (37, 256, 8), (5, 1024, 32), (3, 1, 1), (64, 33, 32)])
 def test_route_parity(dev, T, E, k):
     g = torch.Generator().manual_seed(T * E + k)
     logits = torch.randn(T, E, generator=g)
@@ -117,6 +117,11 @@ def test_route_parity(dev, T, E, k):
     rid, rw = O.route(logits.numpy(), k)
     assert np.array_equal(ids.cpu().numpy(), rid)
     np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=2e-6, atol=1e-7)
+
+
+def test_route_rejects_k_above_32(dev):
+    with pytest.raises(C.Nvfp4MoeError, match="k=33"):
+        ops.moe_route(torch.zeros(4, 64, device=dev), 33)
 
 
 # ------------------------------------------------------------ permutation ----

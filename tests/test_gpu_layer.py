@@ -46,10 +46,11 @@ def test_layer_all_tokens_one_expert_and_idle_experts():
     act, wts, wg, wu, wd = G.layer_inputs(wl, 3)
     logits = np.full((wl.T, wl.E), -4.0, np.float32)
     logits[:, 1] = 2.0           # every token's first choice
-    logits[::3, 4] = 1.0         # a third of the tokens also pick expert 4
+    logits[:, 5] = 0.5           # second choice of most tokens
+    logits[::3, 4] = 1.0         # a third of the tokens take expert 4 second instead
     x_bits = G.bf16_bits(act["x"])
     ref = O.moe_ffn(x_bits, logits, wl.k, wg, wu, wd)
-    assert ref["counts"][1] == wl.T and ref["counts"][0] == 0
+    assert ref["counts"][1] == wl.T and list(ref["counts"][[0, 2, 3]]) == [0, 0, 0]
     layer = ops.MoeFFN(G.experts_from_oracle(wg, wu, wd, dev), wl.k, torch.from_numpy(ref["h_scale"]).to(dev),
                        path=C.PATH_GEMV)
     h_amax = torch.empty(wl.E, device=dev)
