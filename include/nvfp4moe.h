@@ -139,6 +139,35 @@ nvfp4moe_status nvfp4_quantize(const void* x, int32_t x_dtype, int64_t batch, in
                                nvfp4moe_stream_t stream);
 
 /* ------------------------------------------------------------------------------
+ * nvfp4_quantize_dynamic_noalloc - nvfp4_quantize in DYNAMIC scale mode for callers that
+ * cannot allocate device memory.  (The pages have no counterpart: this is a packaging
+ * variant of the quantiser above, not a step of the method.)
+ *
+ * Some callers cannot hand the library a workspace or call cudaMalloc: plug-ins running
+ * inside a host framework that owns the device allocator and forbids side allocations, and
+ * deployments that fix their whole device-memory footprint up front.  This entry point
+ * takes no workspace.  Its scratch (the per-CTA amax partials of the dynamic scale) is a
+ * 64 KiB array compiled into the library, which every GPU that loads the library keeps
+ * until the process exits.  Arguments, layouts and results are those of nvfp4_quantize with
+ * scale_mode = NVFP4MOE_SCALE_DYNAMIC (tensor_scale is written).
+ *  - Sizes whose scratch need (nvfp4_quantize_workspace_size(batch, rows, K)) exceeds
+ *    65536 bytes are rejected with NVFP4MOE_UNSUPPORTED_SHAPE before any work.
+ *  - The first call on a device looks up the device address of the array (once per
+ *    device, with that device current); make that first call before any stream capture.
+ *  - Every call on a device shares the array and it keeps the last call's contents; each
+ *    call overwrites every partial it reads, so nothing has to be cleared.  Calls whose
+ *    kernels overlap on the GPU (unordered streams) race on the array: order them.
+ *  - The call itself allocates nothing.
+ * ---------------------------------------------------------------------------- */
+nvfp4moe_status nvfp4_quantize_dynamic_noalloc(const void* x, int32_t x_dtype, int64_t batch,
+                                               int64_t rows, int64_t K, int64_t ldx,
+                                               int64_t x_batch_stride, const int32_t* row_gather,
+                                               int64_t out_rows, float* tensor_scale,
+                                               uint8_t* codes, int64_t codes_batch_stride,
+                                               uint8_t* sf, int64_t sf_batch_stride,
+                                               int32_t sf_layout, nvfp4moe_stream_t stream);
+
+/* ------------------------------------------------------------------------------
  * moe_route - router top-k (DwarfStar CUDA multi-GPU doc: routers run replicated next to
  * the routed experts).
  * logits: fp32 [T][E] (finite).  ids: int32 [T][k], experts in descending logit order,
