@@ -84,7 +84,8 @@ enum { NVFP4MOE_DTYPE_BF16 = 0, NVFP4MOE_DTYPE_F32 = 1 };
 enum {
   NVFP4MOE_DEV_BAD_EXPERT_ID = 1u << 0,  /* a routing id outside [0, E) was skipped */
   NVFP4MOE_DEV_DUPLICATE_ID = 1u << 1,   /* a token listed the same expert twice */
-  NVFP4MOE_DEV_ROW_OVERFLOW = 1u << 2    /* permuted rows exceeded the stated capacity */
+  NVFP4MOE_DEV_ROW_OVERFLOW = 1u << 2,   /* permuted rows exceeded the stated capacity */
+  NVFP4MOE_DEV_TIMEOUT = 1u << 3         /* a bounded wait inside a kernel gave up */
 };
 
 /* Message for the last failing call on this host thread ("" if none). */
@@ -207,7 +208,7 @@ nvfp4moe_status moe_permute(const int32_t* ids, int32_t T, int32_t E, int32_t k,
  * A: codes [M][K/2] + SF (MMA layout over M rows); B: codes [N][K/2] + SF (MMA layout
  * over N rows); both K-major.  D: [M][N] row-major, d_dtype BF16 or F32.
  * M <= 16 runs the split-K GEMV kernel, larger M the tcgen05 block-scaled MMA kernel.
- * Requires K % 256 == 0, N % 128 == 0, 16-byte aligned pointers.
+ * Requires K % 128 == 0, N % 128 == 0, 16-byte aligned pointers.
  * ---------------------------------------------------------------------------- */
 size_t nvfp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
 nvfp4moe_status nvfp4_gemm(const uint8_t* A, const uint8_t* A_sf, const float* a_scale,

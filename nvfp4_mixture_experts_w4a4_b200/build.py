@@ -64,7 +64,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
             and os.path.getmtime(LIB) >= max(os.path.getmtime(o) for o in objs)):
         return LIB
     tmp = f"{LIB}.{os.getpid()}.tmp"
-    cmd = [NVCC, *ARCH, "-shared", "-o", tmp, *objs, "-lcuda"]
+    cmd = [NVCC, *ARCH, "-shared", "-o", tmp, *objs]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")

@@ -32,7 +32,8 @@ nvfp4moe_status check_desc(const moe_ffn_desc* d, const char* fn) {
 
 int resolve_path(const moe_ffn_desc* d) {
   if (d->path != NVFP4MOE_PATH_AUTO) return d->path;
-  return (d->T <= 16 || !gemm_path_available()) ? NVFP4MOE_PATH_GEMV : NVFP4MOE_PATH_GEMM;
+  if (d->T <= 16 || d->I % 128 != 0) return NVFP4MOE_PATH_GEMV;
+  return gemm_path_available() ? NVFP4MOE_PATH_GEMM : NVFP4MOE_PATH_GEMV;
 }
 
 int64_t max_active_experts(const moe_ffn_desc* d) {
@@ -117,8 +118,11 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   make_layout(d, &L);
   NVFP4_REQUIRE(workspace_bytes >= static_cast<size_t>(L.total), NVFP4MOE_WORKSPACE_TOO_SMALL,
                 "%s: workspace %zu < %lld bytes", fn, workspace_bytes, (long long)L.total);
-  if (L.path == NVFP4MOE_PATH_GEMM && !gemm_path_available())
-    return fail(NVFP4MOE_UNSUPPORTED_SHAPE, "%s: the tensor-core path is not built", fn);
+  if (L.path == NVFP4MOE_PATH_GEMM) {
+    NVFP4_REQUIRE(d->I % 128 == 0, NVFP4MOE_UNSUPPORTED_SHAPE, "%s: the tensor-core path needs I %% 128 == 0 (I=%d)",
+                  fn, d->I);
+    NVFP4_REQUIRE(gemm_path_available(), NVFP4MOE_CUDA_ERROR, "%s: the tensor-core path is unavailable", fn);
+  }
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   auto I32 = [&](int64_t off) { return reinterpret_cast<int32_t*>(ws + off); };
@@ -186,7 +190,7 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   a.rows_cap = rows_cap;
   a.x_codes = ws + L.x_codes; a.x_sf = ws + L.x_sf; a.x_scale = xs;
   a.padded_offsets = I32(L.padded_offsets); a.counts = I32(L.counts);
-  a.tile_expert = I32(L.tile_expert); a.row_pair = I32(L.row_pair);
+  a.tile_expert = I32(L.tile_expert); a.row_token = I32(L.row_token); a.row_pair = I32(L.row_pair);
   a.w13_codes = d->w13_codes; a.w13_sf = d->w13_sf; a.w13_scale = d->w13_scale;
   a.w2_codes = d->w2_codes; a.w2_sf = d->w2_sf; a.w2_scale = d->w2_scale;
   a.h_scale = d->h_scale; a.h_amax = d->h_amax;

@@ -14,6 +14,7 @@ struct GemmFfnArgs {
   const int32_t* padded_offsets;  // [E+1]
   const int32_t* counts;          // [E]
   const int32_t* tile_expert;     // [rows_cap/128]
+  const int32_t* row_token;       // [rows_cap], -1 on padding rows
   const int32_t* row_pair;        // [rows_cap], -1 on padding rows
   const uint8_t* w13_codes;
   const uint8_t* w13_sf;
@@ -32,5 +33,9 @@ struct GemmFfnArgs {
 
 bool gemm_path_available();
 nvfp4moe_status launch_gemm_ffn(const GemmFfnArgs& a, cudaStream_t s);
+// D[M][N] = A . B^T * a_scale[0] * b_scale[0]; N % 128 == 0, K % 128 == 0.
+nvfp4moe_status launch_gemm_plain(const uint8_t* A, const uint8_t* A_sf, const float* a_scale, const uint8_t* B,
+                                  const uint8_t* B_sf, const float* b_scale, int64_t M, int64_t N, int64_t K, void* D,
+                                  int d_f32, cudaStream_t s);
 
 }  // namespace nvfp4moe

@@ -1,6 +1,8 @@
 // nvfp4_gemm: one NVFP4 x NVFP4 GEMM, D = A . B^T * a_scale * b_scale.
-// Small M runs the split-K warp GEMV kernels of the decode path with one "expert" whose
-// rows are the rows of A; partial sums are reduced in a fixed order by a second kernel.
+// M <= 16 runs the split-K warp GEMV kernels of the decode path with one "expert" whose
+// rows are the rows of A (partial sums reduced in a fixed order by a second kernel); larger
+// M runs the tcgen05 block-scaled MMA kernel.
+#include "ffn_gemm.cuh"
 #include "ffn_gemv.cuh"
 
 namespace nvfp4moe {
@@ -66,14 +68,19 @@ nvfp4moe_status nvfp4_gemm(const uint8_t* A, const uint8_t* A_sf, const float* a
   NVFP4_REQUIRE(M >= 0 && N >= 0 && K >= 0, NVFP4MOE_INVALID_ARG, "%s: negative size", fn);
   NVFP4_REQUIRE(d_dtype == NVFP4MOE_DTYPE_BF16 || d_dtype == NVFP4MOE_DTYPE_F32, NVFP4MOE_INVALID_ARG,
                 "%s: bad d_dtype", fn);
-  NVFP4_REQUIRE(K % 256 == 0, NVFP4MOE_UNSUPPORTED_SHAPE, "%s: K=%lld must be a multiple of 256", fn, (long long)K);
+  NVFP4_REQUIRE(K % 128 == 0, NVFP4MOE_UNSUPPORTED_SHAPE, "%s: K=%lld must be a multiple of 128", fn, (long long)K);
   NVFP4_REQUIRE(N % 128 == 0, NVFP4MOE_UNSUPPORTED_SHAPE, "%s: N=%lld must be a multiple of 128", fn, (long long)N);
   NVFP4_REQUIRE(M <= (int64_t(1) << 24), NVFP4MOE_UNSUPPORTED_SHAPE, "%s: M too large", fn);
   if (M == 0 || N == 0) return NVFP4MOE_OK;
-  NVFP4_REQUIRE(A && A_sf && a_scale && B && B_sf && b_scale && D && workspace, NVFP4MOE_INVALID_ARG,
+  NVFP4_REQUIRE(A && A_sf && a_scale && B && B_sf && b_scale && D && (workspace || M > 16), NVFP4MOE_INVALID_ARG,
                 "%s: NULL pointer", fn);
-  NVFP4_REQUIRE(aligned16(A) && aligned16(B) && aligned16(workspace), NVFP4MOE_INVALID_ARG,
+  NVFP4_REQUIRE(aligned16(A) && aligned16(B) && aligned16(workspace) && aligned16(D), NVFP4MOE_INVALID_ARG,
                 "%s: A, B and workspace must be 16-byte aligned", fn);
+  if (M > 16) {
+    NVFP4_REQUIRE(gemm_path_available(), NVFP4MOE_CUDA_ERROR, "%s: the tensor-core path is unavailable", fn);
+    return launch_gemm_plain(A, A_sf, a_scale, B, B_sf, b_scale, M, N, K, D, d_dtype == NVFP4MOE_DTYPE_F32,
+                             reinterpret_cast<cudaStream_t>(stream));
+  }
   const GemvGemmLayout L = gemv_gemm_layout(M, N, K);
   NVFP4_REQUIRE(workspace_bytes >= size_t(L.total), NVFP4MOE_WORKSPACE_TOO_SMALL, "%s: workspace %zu < %lld",
                 fn, workspace_bytes, (long long)L.total);

@@ -51,15 +51,24 @@ def quantize_experts_parallel(w: np.ndarray, nthreads: int | None = None):
     return codes, sf, sc
 
 
-def check_out(gpu_bf16: np.ndarray, ref_f64: np.ndarray, rtol: float = OUT_RTOL):
+def check_out(gpu_bf16: np.ndarray, ref_f64: np.ndarray, rtol: float = OUT_RTOL, extra=None):
+    """|gpu - oracle| <= rtol * max(|oracle|, row RMS) (+ `extra`, the propagated effect of
+    the allowed one-grid-step differences of intermediate codes, when given)."""
     g = bits_to_f32(gpu_bf16).astype(np.float64)
     rms = np.sqrt((ref_f64 ** 2).mean(axis=1, keepdims=True))
     bound = rtol * np.maximum(np.abs(ref_f64), rms)
+    if extra is not None:
+        bound = bound + extra
     err = np.abs(g - ref_f64)
+    ratio = err / np.maximum(bound, 1e-30)
     bad = err > bound
-    assert not bad.any(), (f"{bad.sum()} of {bad.size} outputs outside tolerance; worst "
-                           f"err/bound={float((err / np.maximum(bound, 1e-30)).max()):.3g}")
-    return float((err / np.maximum(bound, 1e-30)).max())
+    if bad.any():
+        t, n = np.unravel_index(int(np.argmax(ratio)), ratio.shape)
+        raise AssertionError(
+            f"{bad.sum()} of {bad.size} outputs outside tolerance; worst at [{t},{n}]: gpu={g[t, n]:.6g} "
+            f"oracle={ref_f64[t, n]:.6g} err={err[t, n]:.3g} bound={bound[t, n]:.3g} row_rms={rms[t, 0]:.3g} "
+            f"extra={0.0 if extra is None else extra[t, n]:.3g}")
+    return float(ratio.max())
 
 
 def _signed_index(codes: np.ndarray) -> np.ndarray:
@@ -125,10 +134,16 @@ def run_layer_pair(wl: W.Workload, path: int, seed: int = 0, dev=None, given_x_s
     h_amax = torch.empty(wl.E, dtype=torch.float32, device=dev)
     out = layer(act["x"].to(dev), act["logits"].to(dev), h_amax=h_amax)
     torch.cuda.synchronize()
+    layer.oracle_wd = wd
     return ref, out, layer, h_amax
 
 
-def check_layer(wl: W.Workload, ref: dict, out: torch.Tensor, layer: ops.MoeFFN, h_amax: torch.Tensor):
+def check_layer(wl: W.Workload, ref: dict, out: torch.Tensor, layer: ops.MoeFFN, h_amax: torch.Tensor,
+                wd=None):
+    """wd: the oracle's (codes, sf, scale) of the down weights, used to bound the effect of
+    differing h codes; when omitted, differing h codes get no output allowance."""
+    wd = wd if wd is not None else getattr(layer, "oracle_wd", None)
+    wd_dequant = None if wd is None else (lambda e: R.dequantize(wd[0][e], wd[1][e], wd[2][e]))
     T, k, H, I, E = wl.T, wl.k, wl.H, wl.I, wl.E
     im = layer.intermediates(T)
     # routing and permutation: bit-exact
@@ -165,9 +180,32 @@ def check_layer(wl: W.Workload, ref: dict, out: torch.Tensor, layer: ops.MoeFFN,
     # h: within the requantisation tolerance
     hc = im["h_codes"].cpu().numpy()[hrows]
     hsf = LY.from_mma(im["h_sf"].cpu().numpy(), im["h_rows"], I)[hrows]
-    check_h_codes(hc, hsf, ref["h_codes"], ref["h_sf"])
+    n_h_diff = check_h_codes(hc, hsf, ref["h_codes"], ref["h_sf"])
     # calibration output: amax of h per expert, within fp32 accumulation differences
     ha = h_amax.cpu().numpy()
     np.testing.assert_allclose(ha[ref["counts"] > 0], ref["h_amax"][ref["counts"] > 0], rtol=1e-4)
-    # layer output
-    return check_out(bf16_bits(out), ref["out_f64"])
+    # layer output: the oracle's output, with the bound widened by the first-order effect of
+    # the (allowed, one-grid-step) h code differences on the rows where they occurred
+    extra = None
+    if n_h_diff and wd_dequant is not None:
+        extra = h_diff_effect(hc, hsf, ref, wl, wd_dequant)
+    print(f"[parity] {wl.name} T={T}: {n_h_diff} of {hc.size * 2} h codes differ")
+    return check_out(bf16_bits(out), ref["out_f64"], extra=extra)
+
+
+def h_diff_effect(hc, hsf, ref, wl, wd_dequant):
+    """Per output element, sum over the differing h elements of w[t][j] * |dh| * |Wd[e][n][i]|,
+    with dh the difference of the two dequantised values (both at the oracle's s_h)."""
+    from tests.helpers import refquant as RQ
+    T, H, k = wl.T, wl.H, wl.k
+    s_h = ref["h_scale"]
+    extra = np.zeros((T, H))
+    gv = RQ.dequantize(hc, hsf, 1.0)
+    rv = RQ.dequantize(ref["h_codes"], ref["h_sf"], 1.0)
+    rows = np.nonzero((gv != rv).any(axis=1))[0]
+    for r in rows:
+        t, j = int(ref["row_token"][r]), int(ref["row_slot"][r])
+        e = int(ref["ids"][t, j])
+        dh = np.abs(gv[r] - rv[r]) * s_h[e]
+        extra[t] += ref["w"][t, j] * (np.abs(wd_dequant(e)) @ dh)
+    return extra

@@ -64,6 +64,8 @@ def test_argument_errors_are_statuses(so):
     # empty work is a no-op success
     assert so.moe_route(None, 0, 8, 2, None, None, None) == C.OK
     assert so.nvfp4_gemm(None, None, None, None, None, None, 0, 128, 256, None, 0, None, 0, None) == C.OK
+    assert so.nvfp4_gemm(None, None, None, None, None, None, 4, 128, 192, None, 0, None, 0, None) == \
+        C.UNSUPPORTED_SHAPE
     assert so.nvfp4_gemm(None, None, None, None, None, None, 4, 100, 256, None, 0, None, 0, None) == \
         C.UNSUPPORTED_SHAPE
 

@@ -174,8 +174,12 @@ def test_permute_flags_bad_ids_without_hanging(dev):
 
 
 # ------------------------------------------------------------------- GEMM ----
-@pytest.mark.parametrize("M,N,K", [(1, 128, 256), (3, 256, 512), (16, 384, 2048), (7, 128, 5120)])
+@pytest.mark.parametrize("M,N,K", [(1, 128, 256), (3, 256, 512), (16, 384, 2048), (7, 128, 5120),
+                                   (17, 128, 256), (128, 256, 512), (300, 512, 1024), (200, 384, 640),
+                                   (513, 256, 2048)])
 def test_gemm_parity(dev, M, N, K):
+    """M <= 16: split-K GEMV; M > 16: tcgen05 block-scaled MMA (ragged M, N tiles of 128 and
+    256, a K that ends in half a stage)."""
     g = torch.Generator().manual_seed(M * N + K)
     a = torch.randn(M, K, generator=g)
     b = torch.randn(N, K, generator=g) / K ** 0.5

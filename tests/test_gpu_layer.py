@@ -26,6 +26,25 @@ CASES = {
 }
 
 
+# the tensor-core path needs I % 128 == 0 (and H % 256 == 0)
+GEMM_CASES = {
+    "tiny": TINY,
+    "prefill_chunk_small": W.scaled(W.WORKLOADS["prefill_chunk"], T=40, E=32, H=512, I=256),
+    "long_prefill_small": W.scaled(W.WORKLOADS["long_prefill"], T=67, E=16, H=768, I=384, k=4),
+    "dense_small": W.scaled(W.WORKLOADS["dense"], T=150, H=512, I=640),
+    "one_expert_many_tiles": W.scaled(TINY, T=300, E=3, k=1, H=256, I=128),
+}
+
+
+@pytest.mark.parametrize("name", list(GEMM_CASES))
+def test_layer_gemm_path(name):
+    wl = GEMM_CASES[name]
+    ref, out, layer, h_amax = G.run_layer_pair(wl, C.PATH_GEMM)
+    assert layer.intermediates(wl.T)["path"] == C.PATH_GEMM
+    G.check_layer(wl, ref, out, layer, h_amax)
+    assert ops.device_status() == 0
+
+
 @pytest.mark.parametrize("name", list(CASES))
 def test_layer_gemv_path(name):
     wl = CASES[name]
