@@ -19,7 +19,6 @@ import concurrent.futures as cf
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -43,95 +42,138 @@ def peaks():
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
-                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
-    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+        pk = {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+              "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    else:
+        pk = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+    # dense FP4 tensor peak: the measured bf16 burst figure times the nominal FP4/BF16 ratio (9 / 2.25)
+    pk["fp4_tflops"] = pk["bf16_tflops"] * 4.0
+    return pk
+
+
+# tokens of the workload the oracle runs per CPU-baseline pass / reference step
+ORACLE_SAMPLE = {"tiny": 8, "decode": 16, "prefill_chunk": 16, "long_prefill": 4, "dense": 2, "dense_t1": 1}
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    """SM clocks and clock-event (throttle) reasons of this rank's GPU, sampled through NVML
+    every millisecond while the timed region runs (nvidia-smi's fastest period is too coarse
+    for a region of a few milliseconds)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap"}
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
+    def __init__(self, cuda_index: int, period_s: float = 0.001):
+        self.cuda_index = cuda_index
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self.ok = False
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-        except OSError:
-            self.proc = None
+            import pynvml as N
+            N.nvmlInit()
+            props = torch.cuda.get_device_properties(self.cuda_index)
+            busid = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            try:
+                self.h = N.nvmlDeviceGetHandleByPciBusId_v2(busid)
+            except Exception:
+                self.h = N.nvmlDeviceGetHandleByIndex(self.cuda_index)
+            self.N = N
+            self.max_mhz = N.nvmlDeviceGetMaxClockInfo(self.h, N.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            return self
+        self.stop = threading.Event()
+        self.t = threading.Thread(target=self._run, daemon=True)
+        self.t.start()
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _reasons(self):
+        N = self.N
+        try:
+            return N.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            return N.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+
+    def _run(self):
+        N = self.N
+        while not self.stop.is_set():
+            try:
+                self.samples.append((N.nvmlDeviceGetClockInfo(self.h, N.NVML_CLOCK_SM), self._reasons()))
+            except Exception:
+                pass
+            time.sleep(self.period)
 
     def __exit__(self, *a):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        if self.ok:
+            self.stop.set()
             self.t.join(timeout=2)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        sm = [c for c, _ in self.samples]
+        reasons = set()
+        for _, r in self.samples:
+            for bit, name in self.REASONS.items():
+                if r & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvml" if self.ok else "unavailable"}
 
 
-def setup_layer(wl: W.Workload, dev, seed: int = 0):
+def setup_layer(wl: W.Workload, dev, seed: int = 0, keep_tokens: int = 0, path: int = C.PATH_AUTO):
     """Draws the workload on the device, quantises the weights with the library, and
-    calibrates the per-expert requantisation scales with one forward (h_amax / 2688)."""
+    calibrates the per-expert requantisation scales with one forward (h_amax / 2688).
+
+    The fp32 weights are freed afterwards; host copies are kept only for the experts that
+    the first `keep_tokens` tokens select (what the CPU baseline needs)."""
     act = W.make_activations(wl, seed, dev)
     wts = W.make_weights(wl, seed, dev)
     experts = ops.NVFP4Experts.from_float(wts["w_gate"], wts["w_up"], wts["w_down"])
     ones = torch.ones(wl.E, dtype=torch.float32, device=dev)
-    layer = ops.MoeFFN(experts, wl.k, ones)
+    layer = ops.MoeFFN(experts, wl.k, ones, path=path)
     h_amax = torch.empty(wl.E, dtype=torch.float32, device=dev)
     layer(act["x"], act["logits"], h_amax=h_amax)
     torch.cuda.synchronize()
+    host = {}
+    if keep_tokens:
+        ids = layer.intermediates(wl.T)["topk_ids"][:keep_tokens].cpu().numpy()
+        for e in np.unique(ids):
+            host[int(e)] = {n: wts[n][int(e)].cpu().numpy() for n in ("w_gate", "w_up", "w_down")}
+    del wts
+    torch.cuda.empty_cache()
     s_h = torch.where(h_amax > 0, h_amax / 2688.0, ones)
-    layer = ops.MoeFFN(experts, wl.k, s_h)
-    return act, wts, experts, layer
+    layer = ops.MoeFFN(experts, wl.k, s_h, path=path)
+    return act, host, experts, layer
 
 
-def algorithmic(wl: W.Workload, n_active: int):
-    """Algorithmic bytes and FLOPs of one layer pass and of its gate/up stage."""
+def algorithmic(wl: W.Workload, n_active: int, gemm_path: bool):
+    """Algorithmic (compulsory) bytes and FLOPs of one layer pass and of its gate/up stage:
+    each touched expert's weights once, the quantised activations once (per permuted row on
+    the tensor-core path, which gathers x into expert order), h written and read once."""
     e = FP4_BYTES_PER_ELT
     P = wl.T * wl.k
     w13 = n_active * 2 * wl.I * wl.H * e
     w2 = n_active * wl.H * wl.I * e
-    x_q = wl.T * wl.H * e
+    x_q = (P if gemm_path else wl.T) * wl.H * e
     h_q = P * wl.I * e
     gate_up_bytes = w13 + x_q + h_q
     layer_bytes = w13 + w2 + wl.T * wl.H * 2 * 2 + x_q + 2 * h_q + wl.T * wl.E * 4
     flops = 2.0 * P * 3 * wl.H * wl.I
     return {"gate_up_bytes": gate_up_bytes, "layer_bytes": layer_bytes, "flops": flops,
             "gate_up_flops": 2.0 * P * 2 * wl.H * wl.I}
+
+
+def roofline(bytes_, flops, ms, pk):
+    """Binding roofline of a kernel that moves `bytes_` and does `flops` in `ms`."""
+    t_hbm = bytes_ / (pk["hbm_gbs"] * 1e9)
+    t_tc = flops / (pk["fp4_tflops"] * 1e12)
+    if t_hbm >= t_tc:
+        ach = bytes_ / (ms * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": ach / pk["hbm_gbs"]}
+    ach = flops / (ms * 1e-3) / 1e12
+    return {"bound": "tensor", "achieved": ach, "peak": pk["fp4_tflops"], "unit": "TFLOP/s",
+            "frac": ach / pk["fp4_tflops"]}
 
 
 def time_steps(layer, act, steps: int, warmup: int, flush: torch.Tensor, dist_on: bool):
@@ -184,7 +226,7 @@ def time_e2e(layer, act, steps: int, warmup: int, flush: torch.Tensor):
 
 
 # ----------------------------------------------------------- oracle (CPU) ----
-def oracle_inputs(wl: W.Workload, act, wts, tokens: np.ndarray):
+def oracle_inputs(wl: W.Workload, act, host, tokens: np.ndarray):
     """Host copies of the inputs for the oracle: x and logits of the sampled tokens and the
     oracle's own quantisation of the fp32 weights of every expert those tokens select."""
     import oracle as O
@@ -192,6 +234,9 @@ def oracle_inputs(wl: W.Workload, act, wts, tokens: np.ndarray):
     logits = act["logits"].cpu().numpy()
     ids, _ = O.route(logits[tokens], wl.k)
     need = np.unique(ids)
+    missing = [int(e) for e in need if int(e) not in host]
+    if missing:
+        raise RuntimeError(f"host weights missing for experts {missing[:8]}")
     shp = {"g": (wl.E, wl.I, wl.H), "d": (wl.E, wl.H, wl.I)}
     arrays = {}
     for key, name in (("g", "w_gate"), ("u", "w_up"), ("d", "w_down")):
@@ -199,26 +244,26 @@ def oracle_inputs(wl: W.Workload, act, wts, tokens: np.ndarray):
         codes = np.zeros((s[0], s[1], s[2] // 2), np.uint8)
         sf = np.zeros((s[0], s[1], s[2] // 16), np.uint8)
         sc = np.ones(s[0], np.float32)
-        host = {int(e): wts[name][int(e)].cpu().numpy() for e in need}
+        src = {int(e): host[int(e)][name] for e in need}
 
         def one(e):
-            c, f, t = O.quantize(host[e])
+            c, f, t = O.quantize(src[e])
             codes[e], sf[e], sc[e] = c, f, t
 
         # ctypes releases the GIL while the oracle runs, so threads quantise in parallel
         with cf.ThreadPoolExecutor(O.default_threads()) as ex:
-            list(ex.map(one, host))
+            list(ex.map(one, src))
         arrays[key] = (codes, sf, sc)
     s_x = np.float32(np.abs((x.astype(np.uint32) << 16).view(np.float32)).max()) / np.float32(2688)
     return x[tokens], logits[tokens], arrays, float(s_x)
 
 
-def oracle_rate(wl: W.Workload, act, wts, layer, budget_s: float, max_tokens: int):
+def oracle_rate(wl: W.Workload, act, host, layer, budget_s: float, max_tokens: int):
     """Tokens/s of the oracle on a bounded token sample of the workload (host cores)."""
     import oracle as O
     n = min(wl.T, max_tokens)
     tokens = np.arange(n)
-    x, logits, arr, s_x = oracle_inputs(wl, act, wts, tokens)
+    x, logits, arr, s_x = oracle_inputs(wl, act, host, tokens)
     s_h = layer.h_scale.cpu().numpy()
     nth = O.default_threads()
     done, t0 = 0, time.perf_counter()
@@ -245,6 +290,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", default="auto", choices=["auto", "gemv", "tcgen05"],
+                    help="layer path: auto (GEMV for T <= 16), the GEMV path or the tcgen05 grouped GEMM")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -268,19 +315,15 @@ def main():
             if dist_on:
                 torch.distributed.destroy_process_group()
             return
-        act, wts, _, layer = setup_layer(wl, dev)
+        n = min(wl.T, ORACLE_SAMPLE.get(wl.name, 4))
+        act, host, _, layer = setup_layer(wl, dev, keep_tokens=n)
         import oracle as O
-        n = wl.T
         tokens = np.arange(n)
-        x, logits, arr, s_x = oracle_inputs(wl, act, wts, tokens)
+        x, logits, arr, s_x = oracle_inputs(wl, act, host, tokens)
         s_h = layer.h_scale.cpu().numpy()
         nth = O.default_threads()
         # a step is a bounded sample of the workload's tokens, sized to keep the run short
-        per = time.perf_counter()
-        O.moe_ffn(x[:1], logits[:1], wl.k, arr["g"], arr["u"], arr["d"], x_scale=s_x, h_scale=s_h, nthreads=nth)
-        one = time.perf_counter() - per
-        budget_tok = max(1, int(4.0 / max(one, 1e-6)))
-        sample = min(n, budget_tok)
+        sample = n
         for _ in range(args.warmup):
             O.moe_ffn(x[:sample], logits[:sample], wl.k, arr["g"], arr["u"], arr["d"], x_scale=s_x,
                       h_scale=s_h, nthreads=nth)
@@ -295,14 +338,17 @@ def main():
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic", "config": cfg,
                 "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nth, "kind": "oracle",
-                                 "sample": f"{sample} of {n} tokens per step"},
+                                 "sample": f"{sample} of {wl.T} tokens per step"},
                 "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         if dist_on:
             torch.distributed.destroy_process_group()
         return
 
-    act, wts, experts, layer = setup_layer(wl, dev)
+    n_cpu = min(wl.T, ORACLE_SAMPLE.get(wl.name, 4))
+    path = {"auto": C.PATH_AUTO, "gemv": C.PATH_GEMV, "tcgen05": C.PATH_GEMM}[args.path]
+    act, host, experts, layer = setup_layer(wl, dev, keep_tokens=n_cpu if (rank == 0 and world == 1) else 0,
+                                            path=path)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     with ClockSampler(local) as clk:
         step_ms, stage_ms = time_steps(layer, act, args.steps, args.warmup, flush, dist_on)
@@ -322,21 +368,26 @@ def main():
 
     im = layer.intermediates(wl.T)
     n_active = int(im["active"][0].item())
-    alg = algorithmic(wl, n_active)
+    gemm_path = im["path"] == C.PATH_GEMM
+    alg = algorithmic(wl, n_active, gemm_path)
     pk = peaks()
     dom_ms = stage_ms["gate_up"]
-    achieved = alg["gate_up_bytes"] / (dom_ms * 1e-3) / 1e9
-    roof = {"kernel": "gate_up (GEMV + SwiGLU + requant)", "bound": "hbm", "achieved": achieved,
-            "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
-            "peak_source": pk["source"], "algorithmic_bytes_per_launch": alg["gate_up_bytes"],
-            "touched_experts": n_active}
+    roof = roofline(alg["gate_up_bytes"], alg["gate_up_flops"], dom_ms, pk)
+    roof.update({"kernel": ("gate_up tcgen05 grouped GEMM + SwiGLU + requant" if gemm_path
+                            else "gate_up GEMV + SwiGLU + requant"),
+                 "traffic": None, "peak_source": pk["source"] + (" (fp4 = bf16 burst x 4)" if roof["bound"] == "tensor"
+                                                                else ""),
+                 "algorithmic_bytes_per_launch": alg["gate_up_bytes"],
+                 "algorithmic_flops_per_launch": alg["gate_up_flops"], "touched_experts": n_active,
+                 "launch_ms": dom_ms})
+    layer_roof = roofline(alg["layer_bytes"], alg["flops"], ms_per_step, pk)
     layer_bw = alg["layer_bytes"] / (ms_per_step * 1e-3) / 1e9
     if dist_on:
         torch.distributed.barrier()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, sample = oracle_rate(wl, act, wts, layer, args.cpu_budget, max_tokens=16)
+        v, cores, sample = oracle_rate(wl, act, host, layer, args.cpu_budget, max_tokens=n_cpu)
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
 
     if rank == 0:
@@ -351,7 +402,10 @@ def main():
             "clocks": clk.summary(),
             "stages_ms": stage_ms,
             "layer": {"bytes": alg["layer_bytes"], "flops": alg["flops"], "hbm_gbs": layer_bw,
-                      "hbm_frac": layer_bw / pk["hbm_gbs"], "hbm_frac_of_8tbs": layer_bw / 8000.0},
+                      "hbm_frac": layer_bw / pk["hbm_gbs"], "hbm_frac_of_8tbs": layer_bw / 8000.0,
+                      "tflops": alg["flops"] / (ms_per_step * 1e-3) / 1e12,
+                      "fp4_frac": alg["flops"] / (ms_per_step * 1e-3) / 1e12 / pk["fp4_tflops"],
+                      "binding": layer_roof},
             "path": {C.PATH_GEMV: "gemv", C.PATH_GEMM: "tcgen05"}.get(im["path"], "?"),
         }
         print(json.dumps(line), flush=True)

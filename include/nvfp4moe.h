@@ -182,8 +182,8 @@ nvfp4moe_status moe_route(const float* logits, int32_t T, int32_t E, int32_t k, 
  * moe_permute - expert histogram and prefix-scan permutation into per-expert row groups
  * (the grouped routed kernels of the DwarfStar doc and Eider's grouped MoE prefill).
  *
- * ids: int32 [T][k].  m_tile: row padding of each expert group (1 = none; 128 for the
- * tensor-core path).  Rows of expert e occupy [padded_offsets[e], padded_offsets[e] +
+ * ids: int32 [T][k].  m_tile: row padding of each expert group (1 = none; 64 for the
+ * tensor-core layer path; 32 and 128 are also accepted).  Rows of expert e occupy [padded_offsets[e], padded_offsets[e] +
  * counts[e]) in ascending token order; experts in ascending index.  Outputs:
  *   counts [E], offsets [E+1] (exclusive scan of counts), padded_offsets [E+1]
  *   (exclusive scan of counts rounded up to m_tile), pair_to_row [T*k] (pair t*k+j ->
@@ -194,7 +194,7 @@ nvfp4moe_status moe_route(const float* logits, int32_t T, int32_t E, int32_t k, 
  *   per-expert amax output of moe_ffn_forward).
  * rows_cap must be >= moe_permute_rows_capacity(T, E, k, m_tile).  Out-of-range or
  * duplicate ids are skipped (pair_to_row = -1) and flag the device status word.
- * T*k <= 2^24, E <= 1024, k <= 32, m_tile in {1, 128}.
+ * T*k <= 2^24, E <= 1024, k <= 32, m_tile in {1, 32, 64, 128}.
  * ---------------------------------------------------------------------------- */
 int64_t moe_permute_rows_capacity(int32_t T, int32_t E, int32_t k, int32_t m_tile);
 nvfp4moe_status moe_permute(const int32_t* ids, int32_t T, int32_t E, int32_t k,
@@ -223,7 +223,7 @@ enum { NVFP4MOE_PATH_AUTO = 0, NVFP4MOE_PATH_GEMV = 1, NVFP4MOE_PATH_GEMM = 2 };
 
 typedef struct {
   int32_t T, H, I, E, top_k;
-  int32_t path;               /* NVFP4MOE_PATH_*; AUTO picks GEMV for T <= 16 */
+  int32_t path;               /* NVFP4MOE_PATH_*; AUTO: tensor cores when I % 128 == 0, else GEMV */
   int32_t x_scale_mode;       /* NVFP4MOE_SCALE_GIVEN or _DYNAMIC */
   const float* x_scale;       /* [1], read when GIVEN */
   const uint8_t* w13_codes;   /* [E][2I][H/2], gate/up rows interleaved (see above) */
@@ -250,7 +250,7 @@ typedef struct {
       amax_partials, total;
   int64_t x_rows;   /* rows of x_codes / x_sf (T on the GEMV path, rows_cap otherwise) */
   int64_t h_rows;   /* rows of h_codes / h_sf */
-  int32_t m_tile;   /* 1 on the GEMV path, 128 on the GEMM path */
+  int32_t m_tile;   /* 1 on the GEMV path, 64 on the GEMM path */
   int32_t path;     /* resolved path */
 } moe_ffn_ws_layout;
 

@@ -4,6 +4,8 @@
 //
 // All intermediates live in the caller's workspace at the offsets moe_ffn_workspace_layout
 // reports; group sizes stay on the device (no host synchronisation anywhere).
+#include <algorithm>
+
 #include "ffn_gemv.cuh"
 #include "ffn_gemm.cuh"
 
@@ -32,7 +34,9 @@ nvfp4moe_status check_desc(const moe_ffn_desc* d, const char* fn) {
 
 int resolve_path(const moe_ffn_desc* d) {
   if (d->path != NVFP4MOE_PATH_AUTO) return d->path;
-  if (d->T <= 16 || d->I % 128 != 0) return NVFP4MOE_PATH_GEMV;
+  // the weight-stationary tensor-core kernel is faster than the GEMV at every measured size
+  // (decode included); the GEMV serves the shapes it does not (I % 128 != 0)
+  if (d->I % 128 != 0) return NVFP4MOE_PATH_GEMV;
   return gemm_path_available() ? NVFP4MOE_PATH_GEMM : NVFP4MOE_PATH_GEMV;
 }
 
@@ -44,7 +48,7 @@ int64_t max_active_experts(const moe_ffn_desc* d) {
 void make_layout(const moe_ffn_desc* d, moe_ffn_ws_layout* L) {
   const int path = resolve_path(d);
   const int64_t T = d->T, H = d->H, I = d->I, E = d->E, k = d->top_k, P = T * k;
-  const int m_tile = path == NVFP4MOE_PATH_GEMM ? 128 : 1;
+  const int m_tile = path == NVFP4MOE_PATH_GEMM ? grouped_token_align() : 1;
   const int64_t rows_cap = moe_permute_rows_capacity(d->T, d->E, d->top_k, m_tile);
   int64_t o = 0;
   auto take = [&](int64_t bytes) {
@@ -72,8 +76,12 @@ void make_layout(const moe_ffn_desc* d, moe_ffn_ws_layout* L) {
   L->h_rows = path == NVFP4MOE_PATH_GEMM ? rows_cap : P;
   L->h_codes = take(L->h_rows * I / 2);
   L->h_sf = take(sf_mma_bytes(L->h_rows, I));
-  const int ksplit = path == NVFP4MOE_PATH_GEMM ? 1 : gemv_down_ksplit(max_active_experts(d), H, I);
-  L->slots = take(int64_t(ksplit) * P * H * 4);
+  // per-slot rows of the down projection: fp32 split-K partials on the GEMV path, bf16 on
+  // the tensor-core path (halves the slot round trip of large prefills)
+  if (path == NVFP4MOE_PATH_GEMM)  // also holds x quantised per token until the down GEMM
+    L->slots = take(std::max<int64_t>(P * H * 2, ((T * H / 2 + 255) / 256) * 256 + sf_mma_bytes(T, H)));
+  else
+    L->slots = take(int64_t(gemv_down_ksplit(max_active_experts(d), H, I)) * P * H * 4);
   L->total = o;
 }
 
@@ -121,6 +129,7 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   if (L.path == NVFP4MOE_PATH_GEMM) {
     NVFP4_REQUIRE(d->I % 128 == 0, NVFP4MOE_UNSUPPORTED_SHAPE, "%s: the tensor-core path needs I %% 128 == 0 (I=%d)",
                   fn, d->I);
+    NVFP4_REQUIRE(d->E <= 1024, NVFP4MOE_UNSUPPORTED_SHAPE, "%s: E > 1024", fn);
     NVFP4_REQUIRE(gemm_path_available(), NVFP4MOE_CUDA_ERROR, "%s: the tensor-core path is unavailable", fn);
   }
 
@@ -180,27 +189,33 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
     return NVFP4MOE_OK;
   }
 
-  // tensor-core path: x quantised straight into the padded permuted rows
-  st = nvfp4_quantize(x, NVFP4MOE_DTYPE_BF16, 1, T, H, H, 0, I32(L.row_token), rows_cap, d->x_scale_mode,
-                      xs, ws + L.x_codes, 0, ws + L.x_sf, 0, NVFP4MOE_SF_MMA, ws + L.amax_partials, qws, stream);
+  // tensor-core path: x quantised once per token (into the slot region, which is free until
+  // the down GEMM), then copied into the padded expert-order rows
+  uint8_t* xt_codes = ws + L.slots;
+  uint8_t* xt_sf = xt_codes + ((int64_t(T) * H / 2 + 255) / 256) * 256;
+  st = nvfp4_quantize(x, NVFP4MOE_DTYPE_BF16, 1, T, H, H, 0, nullptr, T, d->x_scale_mode, xs, xt_codes, 0, xt_sf, 0,
+                      NVFP4MOE_SF_MMA, ws + L.amax_partials, qws, stream);
+  if (st != NVFP4MOE_OK) return st;
+  st = launch_replicate_rows(xt_codes, xt_sf, I32(L.row_token), I32(L.padded_offsets) + E, rows_cap, T, H,
+                             ws + L.x_codes, ws + L.x_sf, s);
   if (st != NVFP4MOE_OK) return st;
   mark(3);
   GemmFfnArgs a;
   a.T = T; a.H = H; a.I = I; a.E = E; a.k = k;
   a.rows_cap = rows_cap;
   a.x_codes = ws + L.x_codes; a.x_sf = ws + L.x_sf; a.x_scale = xs;
-  a.padded_offsets = I32(L.padded_offsets); a.counts = I32(L.counts);
-  a.tile_expert = I32(L.tile_expert); a.row_token = I32(L.row_token); a.row_pair = I32(L.row_pair);
+  a.padded_offsets = I32(L.padded_offsets); a.counts = I32(L.counts); a.active = I32(L.active);
+  a.row_token = I32(L.row_token); a.row_pair = I32(L.row_pair);
   a.w13_codes = d->w13_codes; a.w13_sf = d->w13_sf; a.w13_scale = d->w13_scale;
   a.w2_codes = d->w2_codes; a.w2_sf = d->w2_sf; a.w2_scale = d->w2_scale;
   a.h_scale = d->h_scale; a.h_amax = d->h_amax;
   a.h_codes = ws + L.h_codes; a.h_sf = ws + L.h_sf;
-  a.topk_w = F32(L.topk_w); a.slots = F32(L.slots);
+  a.topk_w = F32(L.topk_w); a.slots_bf16 = ws + L.slots;
   a.stage_events = d->stage_events;
-  st = launch_gemm_ffn(a, s);
+  st = launch_grouped_ffn(a, s);
   if (st != NVFP4MOE_OK) return st;
   mark(5);
-  st = launch_combine(F32(L.slots), int64_t(T) * k * H, 1, I32(L.pair_to_row), T, H, k, out, s);
+  st = launch_combine_bf16(ws + L.slots, I32(L.pair_to_row), T, H, k, out, s);
   if (st != NVFP4MOE_OK) return st;
   mark(6);
   return NVFP4MOE_OK;

@@ -1,10 +1,8 @@
-// Tensor-core path: NVFP4 x NVFP4 grouped GEMM on tcgen05 block-scaled MMA
-// (.kind::mxf4nvf4, E2M1 operands, UE4M3 scales per 16 elements, fp32 accumulation in TMEM).
+// nvfp4_gemm on tcgen05 block-scaled MMA (.kind::mxf4nvf4, E2M1 operands, UE4M3 scales
+// per 16 elements, fp32 accumulation in TMEM): D[M][N] = A . B^T * a_scale * b_scale.
 //
 // One persistent CTA per SM walks the output tiles (128 rows of A x BN rows of B) with a
-// static stride.  Tiles are ordered row-tile-major, so the CTAs of one wave share the A
-// tile of a row-tile and the weight tiles of an expert whose tokens span two row-tiles,
-// and those re-reads hit L2.  Warp roles:
+// static stride, row-tile-major, so the CTAs of one wave share an A tile.  Warp roles:
 //   warp 0      one elected thread issues TMA loads of the A and B code tiles (128-byte
 //               swizzle, 256 K-elements = 128 bytes per row per stage) and bulk copies of
 //               their 512-byte scale atoms into a 4-stage shared-memory ring;
@@ -12,14 +10,12 @@
 //               scales to TMEM (tcgen05.cp) and issues four K=64 MMAs per stage into the
 //               fp32 accumulator (TMEM columns [0, BN)), then commits;
 //   warps 2..5  the epilogue: each warp reads its 32 TMEM lanes (= 32 rows) in
-//               32-column slices and finishes the tile (SwiGLU + requantise for gate/up,
-//               weighted per-slot rows for down, plain D otherwise).
+//               32-column slices, scales them and stores bf16 or fp32 D.
 // Every wait is bounded: on a timeout the CTA raises a status bit, drains what it issued
 // and returns instead of spinning.
 #include "ffn_gemm.cuh"
 #include "tcgen05.cuh"
-
-#include <cudaTypedefs.h>
+#include "tma.cuh"
 
 namespace nvfp4moe {
 namespace {
@@ -34,26 +30,14 @@ constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kDevTimeout = 1u << 3;
 
-enum { EPI_GATEUP = 0, EPI_DOWN = 1, EPI_PLAIN = 2 };
 
 struct GemmParams {
-  int K, N, E, M;
-  int num_m_static;                 // >= 0: number of row tiles; < 0: padded_offsets[E] / 128
-  const int32_t* padded_offsets;
-  const int32_t* tile_expert;       // nullable: expert 0 for every tile
-  const int32_t* row_token;         // gate/up: < 0 marks a padding row
-  const int32_t* row_pair;          // down: < 0 marks a padding row
+  int K, N, M;
+  int num_m;
   const uint8_t* a_sf;
-  const uint8_t* b_sf;              // per expert N*K/16 bytes
-  const float* a_scale;             // gate/up, plain: [1]
-  const float* b_scale;             // gate/up: [E][2]; down: [E]; plain: [1]
-  const float* h_scale;             // gate/up: requantisation scale [E]; down: A's tensor scale [E]
-  float* h_amax;
-  uint8_t* h_codes;
-  uint8_t* h_sf;
-  int I;
-  const float* topk_w;
-  float* slots;
+  const uint8_t* b_sf;
+  const float* a_scale;
+  const float* b_scale;
   void* D;
   int d_f32;
   uint32_t* status;
@@ -70,9 +54,7 @@ struct Smem {
   static constexpr int BYTES = 1024 + STAGES * STAGE + BARS * 8 + 16;
 };
 
-__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
-
-template <int BN, int EPI>
+template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p) {
   using S = Smem<BN>;
@@ -116,7 +98,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  const int num_m = p.num_m_static >= 0 ? p.num_m_static : p.padded_offsets[p.E] / BM;
+  const int num_m = p.num_m;
   const int n_tiles = p.N / BN;
   const int total = num_m * n_tiles;
   const int k_tiles = (p.K + BK - 1) / BK;
@@ -132,8 +114,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       uint32_t it = 0;
       for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
         const int mt = t / n_tiles, nt = t % n_tiles;
-        const int e = p.tile_expert ? p.tile_expert[mt] : 0;
-        const uint8_t* bsf = p.b_sf + int64_t(e) * p.N * (p.K / 16);
+        const uint8_t* bsf = p.b_sf;
         for (int kt = 0; kt < k_tiles; ++kt, ++it) {
           const int s = it % STAGES;
           if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1)) {
@@ -144,7 +125,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
           const uint32_t sf_bytes = nkb * 512;
           mbar_arrive_expect_tx(&full[s], S::A + S::B + sf_bytes * (1 + BN / 128));
           tma_load_2d(sA + s * S::A, &tmA, kt * KB, mt * BM, &full[s]);
-          tma_load_2d(sB + s * S::B, &tmB, kt * KB, e * p.N + nt * BN, &full[s]);
+          tma_load_2d(sB + s * S::B, &tmB, kt * KB, nt * BN, &full[s]);
           bulk_load(sSFA + s * S::SFA, p.a_sf + (int64_t(mt) * katoms + kt * 4) * 512, sf_bytes, &full[s]);
 #pragma unroll
           for (int h = 0; h < BN / 128; ++h)
@@ -217,57 +198,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       }
       tc_fence_after();
       const int mt = t / n_tiles, nt = t % n_tiles;
-      const int e = p.tile_expert ? p.tile_expert[mt] : 0;
       const int64_t row = int64_t(mt) * BM + rt;
-      if constexpr (EPI == EPI_GATEUP) {
-        const bool valid = p.row_token[row] >= 0;
-        const float sx = p.a_scale[0];
-        const float sg = sx * p.b_scale[2 * e], su = sx * p.b_scale[2 * e + 1], sh = p.h_scale[e];
-        float amax_all = 0.0f;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(trow + c * 32, r);
-          tmem_ld_wait();
-          if (valid) {
-            float h[16];
-            float amax = 0.0f;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              h[j] = silu_mul(__uint_as_float(r[j]) * sg, __uint_as_float(r[16 + j]) * su);
-              amax = fmaxf(amax, fabsf(h[j]));
-            }
-            float inv;
-            const uint32_t sf = block_scale(amax, sh, &inv);
-            const int64_t iblk = int64_t(nt) * (BN / 32) + c;
-            *reinterpret_cast<uint2*>(p.h_codes + row * (p.I / 2) + iblk * 8) = encode_block16(h, inv);
-            p.h_sf[sf_mma_offset(row, iblk, p.I)] = static_cast<uint8_t>(sf);
-            amax_all = fmaxf(amax_all, amax);
-          }
-        }
-        if (p.h_amax) {
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) amax_all = fmaxf(amax_all, __shfl_xor_sync(0xffffffffu, amax_all, o));
-          if (lane == 0 && amax_all > 0.0f) atomicMax(reinterpret_cast<int*>(p.h_amax + e), __float_as_int(amax_all));
-        }
-      } else if constexpr (EPI == EPI_DOWN) {
-        const int32_t pair = p.row_pair[row];
-        const float sc = pair >= 0 ? p.h_scale[e] * p.b_scale[e] * p.topk_w[pair] : 0.0f;
-        float* dst = p.slots + int64_t(pair) * p.N + int64_t(nt) * BN;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(trow + c * 32, r);
-          tmem_ld_wait();
-          if (pair >= 0) {
-#pragma unroll
-            for (int j = 0; j < 32; j += 4)
-              *reinterpret_cast<float4*>(dst + c * 32 + j) =
-                  make_float4(__uint_as_float(r[j]) * sc, __uint_as_float(r[j + 1]) * sc,
-                              __uint_as_float(r[j + 2]) * sc, __uint_as_float(r[j + 3]) * sc);
-          }
-        }
-      } else {
+      {
         const bool valid = row < p.M;
         const float sc = p.a_scale[0] * p.b_scale[0];
 #pragma unroll 1
@@ -314,37 +246,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 }
 
 // ------------------------------------------------------------------ host side ----
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-// K-major code matrix [rows][K/2] bytes; box = 128 bytes x box_rows rows, 128-byte swizzle.
-nvfp4moe_status make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int box_rows) {
-  auto fn = encode_fn();
-  if (!fn) return fail(NVFP4MOE_CUDA_ERROR, "cuTensorMapEncodeTiled is unavailable");
-  const cuuint64_t dims[2] = {cuuint64_t(K / 2), cuuint64_t(rows)};
-  const cuuint64_t strides[1] = {cuuint64_t(K / 2)};
-  const cuuint32_t box[2] = {cuuint32_t(KB), cuuint32_t(box_rows)};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(NVFP4MOE_CUDA_ERROR, "cuTensorMapEncodeTiled failed (%d)", int(r));
-  return NVFP4MOE_OK;
-}
-
-template <int BN, int EPI>
+template <int BN>
 nvfp4moe_status launch(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p, int64_t max_tiles,
                        cudaStream_t s) {
-  auto kern = gemm_kernel<BN, EPI>;
+  auto kern = gemm_kernel<BN>;
   static int configured[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -361,58 +266,7 @@ nvfp4moe_status launch(const CUtensorMap& a, const CUtensorMap& b, const GemmPar
 
 }  // namespace
 
-bool gemm_path_available() { return encode_fn() != nullptr; }
-
-nvfp4moe_status launch_gemm_ffn(const GemmFfnArgs& a, cudaStream_t s) {
-  uint32_t* status = device_status_ptr();
-  if (!status) return fail(NVFP4MOE_CUDA_ERROR, "device status word unavailable");
-  const int64_t max_m = a.rows_cap / BM + 1;
-  CUtensorMap ta, tb;
-  GemmParams p{};
-  p.E = a.E;
-  p.num_m_static = -1;
-  p.padded_offsets = a.padded_offsets;
-  p.tile_expert = a.tile_expert;
-  p.status = status;
-  // gate/up: A = x rows [rows_cap][H], B = W13 [E*2I][H]
-  nvfp4moe_status st = make_map(&ta, a.x_codes, a.rows_cap, a.H, BM);
-  if (st != NVFP4MOE_OK) return st;
-  st = make_map(&tb, a.w13_codes, int64_t(a.E) * 2 * a.I, a.H, 256);
-  if (st != NVFP4MOE_OK) return st;
-  p.K = a.H;
-  p.N = 2 * a.I;
-  p.row_token = a.row_token;
-  p.a_sf = a.x_sf;
-  p.b_sf = a.w13_sf;
-  p.a_scale = a.x_scale;
-  p.b_scale = a.w13_scale;
-  p.h_scale = a.h_scale;
-  p.h_amax = a.h_amax;
-  p.h_codes = a.h_codes;
-  p.h_sf = a.h_sf;
-  p.I = a.I;
-  st = launch<256, EPI_GATEUP>(ta, tb, p, max_m * (p.N / 256), s);
-  if (st != NVFP4MOE_OK) return st;
-  if (a.stage_events) cudaEventRecord(reinterpret_cast<cudaEvent_t>(a.stage_events[4]), s);
-  // down: A = h rows [rows_cap][I], B = W2 [E*H][I]
-  st = make_map(&ta, a.h_codes, a.rows_cap, a.I, BM);
-  if (st != NVFP4MOE_OK) return st;
-  st = make_map(&tb, a.w2_codes, int64_t(a.E) * a.H, a.I, 256);
-  if (st != NVFP4MOE_OK) return st;
-  p.K = a.I;
-  p.N = a.H;
-  p.row_token = nullptr;
-  p.row_pair = a.row_pair;
-  p.a_sf = a.h_sf;
-  p.b_sf = a.w2_sf;
-  p.a_scale = nullptr;
-  p.b_scale = a.w2_scale;
-  p.h_scale = a.h_scale;
-  p.h_amax = nullptr;
-  p.topk_w = a.topk_w;
-  p.slots = a.slots;
-  return launch<256, EPI_DOWN>(ta, tb, p, max_m * (p.N / 256), s);
-}
+bool gemm_path_available() { return tensor_map_encoder() != nullptr; }
 
 nvfp4moe_status launch_gemm_plain(const uint8_t* A, const uint8_t* A_sf, const float* a_scale, const uint8_t* B,
                                   const uint8_t* B_sf, const float* b_scale, int64_t M, int64_t N, int64_t K, void* D,
@@ -421,16 +275,15 @@ nvfp4moe_status launch_gemm_plain(const uint8_t* A, const uint8_t* A_sf, const f
   if (!status) return fail(NVFP4MOE_CUDA_ERROR, "device status word unavailable");
   const int BN = (N % 256 == 0) ? 256 : 128;
   CUtensorMap ta, tb;
-  nvfp4moe_status st = make_map(&ta, A, M, K, BM);
+  nvfp4moe_status st = make_code_map(&ta, A, M, K, BM);
   if (st != NVFP4MOE_OK) return st;
-  st = make_map(&tb, B, N, K, BN);
+  st = make_code_map(&tb, B, N, K, BN);
   if (st != NVFP4MOE_OK) return st;
   GemmParams p{};
   p.K = static_cast<int>(K);
   p.N = static_cast<int>(N);
-  p.E = 1;
   p.M = static_cast<int>(M);
-  p.num_m_static = static_cast<int>((M + BM - 1) / BM);
+  p.num_m = static_cast<int>((M + BM - 1) / BM);
   p.a_sf = A_sf;
   p.b_sf = B_sf;
   p.a_scale = a_scale;
@@ -438,9 +291,9 @@ nvfp4moe_status launch_gemm_plain(const uint8_t* A, const uint8_t* A_sf, const f
   p.D = D;
   p.d_f32 = d_f32;
   p.status = status;
-  const int64_t tiles = int64_t(p.num_m_static) * (N / BN);
-  if (BN == 256) return launch<256, EPI_PLAIN>(ta, tb, p, tiles, s);
-  return launch<128, EPI_PLAIN>(ta, tb, p, tiles, s);
+  const int64_t tiles = int64_t(p.num_m) * (N / BN);
+  if (BN == 256) return launch<256>(ta, tb, p, tiles, s);
+  return launch<128>(ta, tb, p, tiles, s);
 }
 
 }  // namespace nvfp4moe

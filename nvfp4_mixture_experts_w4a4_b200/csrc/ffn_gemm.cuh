@@ -7,13 +7,13 @@ namespace nvfp4moe {
 
 struct GemmFfnArgs {
   int T, H, I, E, k;
-  int64_t rows_cap;               // padded permuted rows (m_tile = 128)
+  int64_t rows_cap;               // padded permuted rows (m_tile = grouped_token_align())
   const uint8_t* x_codes;         // [rows_cap][H/2], padded permuted rows
   const uint8_t* x_sf;            // MMA layout over rows_cap rows
   const float* x_scale;           // [1]
   const int32_t* padded_offsets;  // [E+1]
   const int32_t* counts;          // [E]
-  const int32_t* tile_expert;     // [rows_cap/128]
+  const int32_t* active;          // [E+1]
   const int32_t* row_token;       // [rows_cap], -1 on padding rows
   const int32_t* row_pair;        // [rows_cap], -1 on padding rows
   const uint8_t* w13_codes;
@@ -27,12 +27,14 @@ struct GemmFfnArgs {
   uint8_t* h_codes;               // [rows_cap][I/2]
   uint8_t* h_sf;                  // MMA layout over rows_cap rows
   const float* topk_w;            // [T*k] by pair
-  float* slots;                   // [T*k][H] by pair
+  void* slots_bf16;               // [T*k][H] bf16, by pair
   void* const* stage_events;      // nullable; [4] is recorded between gate/up and down
 };
 
 bool gemm_path_available();
-nvfp4moe_status launch_gemm_ffn(const GemmFfnArgs& a, cudaStream_t s);
+int grouped_token_align();
+// gate/up (SwiGLU + requant) then down (weighted bf16 slots), weight-stationary grouped GEMM
+nvfp4moe_status launch_grouped_ffn(const GemmFfnArgs& a, cudaStream_t s);
 // D[M][N] = A . B^T * a_scale[0] * b_scale[0]; N % 128 == 0, K % 128 == 0.
 nvfp4moe_status launch_gemm_plain(const uint8_t* A, const uint8_t* A_sf, const float* a_scale, const uint8_t* B,
                                   const uint8_t* B_sf, const float* b_scale, int64_t M, int64_t N, int64_t K, void* D,

@@ -173,14 +173,26 @@ __global__ void combine_kernel(const float* __restrict__ slots, int64_t slot_str
        i += int64_t(gridDim.x) * blockDim.x) {
     const int64_t t = i / per_row, n = (i - t * per_row) * 8;
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int j = 0; j < k; ++j) {
-      const int64_t p = t * k + j;
-      if (pair_to_row[p] < 0) continue;
+    for (int j0 = 0; j0 < k; j0 += 4) {
+      // up to four slots' rows in flight at once; summed in slot order
+      bool ok[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) ok[u] = j0 + u < k && pair_to_row[t * k + j0 + u] >= 0;
       for (int s = 0; s < ksplit; ++s) {
-        const float4* src = reinterpret_cast<const float4*>(slots + s * slot_stride + p * H + n);
-        const float4 u = src[0], v = src[1];
-        acc[0] += u.x; acc[1] += u.y; acc[2] += u.z; acc[3] += u.w;
-        acc[4] += v.x; acc[5] += v.y; acc[6] += v.z; acc[7] += v.w;
+        float4 a[4], b[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (ok[u]) {
+            const float4* src = reinterpret_cast<const float4*>(slots + s * slot_stride + (t * k + j0 + u) * H + n);
+            a[u] = src[0];
+            b[u] = src[1];
+          }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (ok[u]) {
+            acc[0] += a[u].x; acc[1] += a[u].y; acc[2] += a[u].z; acc[3] += a[u].w;
+            acc[4] += b[u].x; acc[5] += b[u].y; acc[6] += b[u].z; acc[7] += b[u].w;
+          }
       }
     }
     uint4 o;
@@ -191,6 +203,70 @@ __global__ void combine_kernel(const float* __restrict__ slots, int64_t slot_str
       ow[q] = *reinterpret_cast<const uint32_t*>(&b);
     }
     *reinterpret_cast<uint4*>(out + t * H + n) = o;
+  }
+}
+
+// Same as combine_kernel over bf16 slot rows: 8 outputs per thread, eight slots in flight.
+__global__ void combine_bf16_kernel(const __nv_bfloat16* __restrict__ slots, const int32_t* __restrict__ pair_to_row,
+                                    int T, int H, int k, __nv_bfloat16* __restrict__ out) {
+  const int64_t per_row = H / 8;
+  const int64_t total = int64_t(T) * per_row;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t t = i / per_row, n = (i - t * per_row) * 8;
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int j0 = 0; j0 < k; j0 += 8) {
+      uint4 v[8];
+      bool ok[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) ok[u] = j0 + u < k && pair_to_row[t * k + j0 + u] >= 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (ok[u]) v[u] = *reinterpret_cast<const uint4*>(slots + (t * k + j0 + u) * H + n);
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (ok[u]) {
+          const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            acc[2 * q] += __uint_as_float(w[q] << 16);
+            acc[2 * q + 1] += __uint_as_float(w[q] & 0xFFFF0000u);
+          }
+        }
+    }
+    uint4 o;
+    uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
+      ow[q] = *reinterpret_cast<const uint32_t*>(&b);
+    }
+    *reinterpret_cast<uint4*>(out + t * H + n) = o;
+  }
+}
+
+// Copies quantised token rows into the padded expert-order rows: codes (32 bytes) and the
+// 4-byte scale word of one 64-element group per thread; padding rows are left untouched.
+// Only rows below *rows_used (the permutation's padded total) carry a row -> token entry;
+// the token index is checked against T as well.
+__global__ void replicate_rows_kernel(const uint8_t* __restrict__ codes_tok, const uint8_t* __restrict__ sf_tok,
+                                      const int32_t* __restrict__ row_token, const int32_t* __restrict__ rows_used,
+                                      int64_t rows_cap, int64_t T, int64_t K, uint8_t* __restrict__ codes_out,
+                                      uint8_t* __restrict__ sf_out) {
+  const int64_t groups = K / 64;
+  const int64_t rows = min(rows_cap, int64_t(*rows_used));
+  const int64_t total = rows * groups;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = i / groups, g = i - r * groups;
+    const int32_t t = row_token[r];
+    if (t < 0 || t >= T) continue;
+    const uint4* src = reinterpret_cast<const uint4*>(codes_tok + int64_t(t) * (K / 2) + g * 32);
+    uint4* dst = reinterpret_cast<uint4*>(codes_out + r * (K / 2) + g * 32);
+    dst[0] = src[0];
+    dst[1] = src[1];
+    *reinterpret_cast<uint32_t*>(sf_out + sf_mma_offset(r, 4 * g, K)) =
+        *reinterpret_cast<const uint32_t*>(sf_tok + sf_mma_offset(t, 4 * g, K));
   }
 }
 
@@ -262,6 +338,29 @@ nvfp4moe_status launch_combine(const float* slots, int64_t slot_stride, int kspl
   if (blocks > int64_t(num_sms()) * 8) blocks = int64_t(num_sms()) * 8;
   combine_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(slots, slot_stride, ksplit, pair_to_row, T,
                                                          H, k, static_cast<__nv_bfloat16*>(out));
+  return check_launch("combine");
+}
+
+nvfp4moe_status launch_replicate_rows(const uint8_t* codes_tok, const uint8_t* sf_tok, const int32_t* row_token,
+                                      const int32_t* rows_used, int64_t rows_cap, int64_t T, int64_t K,
+                                      uint8_t* codes_out, uint8_t* sf_out, cudaStream_t s) {
+  const int64_t total = rows_cap * (K / 64);
+  if (total == 0) return NVFP4MOE_OK;
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > int64_t(num_sms()) * 16) blocks = int64_t(num_sms()) * 16;
+  replicate_rows_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(codes_tok, sf_tok, row_token, rows_used, rows_cap, T,
+                                                                 K, codes_out, sf_out);
+  return check_launch("replicate rows");
+}
+
+nvfp4moe_status launch_combine_bf16(const void* slots, const int32_t* pair_to_row, int T, int H, int k, void* out,
+                                    cudaStream_t s) {
+  const int64_t total = int64_t(T) * (H / 8);
+  if (total == 0) return NVFP4MOE_OK;
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > int64_t(num_sms()) * 16) blocks = int64_t(num_sms()) * 16;
+  combine_bf16_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(slots), pair_to_row,
+                                                              T, H, k, static_cast<__nv_bfloat16*>(out));
   return check_launch("combine");
 }
 

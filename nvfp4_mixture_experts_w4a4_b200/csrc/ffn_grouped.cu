@@ -1,0 +1,479 @@
+// Weight-stationary grouped GEMM of the routed layer on tcgen05 block-scaled MMA.
+//
+// The expert weights are the MMA's M operand (128 weight rows per tile) and an expert's
+// tokens are its N operand: N = the expert's token count rounded up to 64 (tokens are
+// grouped in 64-row blocks by the permutation), at most 192 per tile.  So a weight tile is
+// streamed once per 192 tokens of its expert whatever the skew, and no MMA work or load is
+// spent on 128-row padding of experts that received a handful of tokens.  This one kernel
+// serves decode (N = 64 for 1..64 tokens) and prefill.
+//
+// Persistent CTA per SM; work items ordered (expert, weight tile, token chunk) with the
+// chunk fastest, so CTAs of one wave that share a weight tile run together (L2 hits).
+//   warp 0      TMA producer: weights (128 rows x 128 B, 128-byte swizzle), tokens (64-row
+//               boxes), and bulk copies of the 512-byte scale atoms, 4-stage ring;
+//   warp 1      TMEM owner and MMA issuer: tcgen05.cp of the scales, four K=64 MMAs per
+//               stage into one of two fp32 accumulators (double buffered, 192 columns);
+//   warps 2..5  epilogue, one 32-row slice of weight rows each: SwiGLU + requantise (gate/up,
+//               gate row i and up row i are lanes i and 16+i of the same warp by the W13
+//               interleave) or the weighted bf16 slot rows (down).
+// Scale atoms of the tokens start at a 64-row boundary inside a 128-row atom, so the MMA
+// reads them at a TMEM column offset of 0 or 2.  Waits are bounded (status bit on timeout).
+#include "ffn_gemm.cuh"
+#include "tcgen05.cuh"
+#include "tma.cuh"
+
+namespace nvfp4moe {
+namespace {
+
+using namespace sm100;
+
+constexpr int WM = 128;         // weight rows per tile
+constexpr int BNMAX = 192;      // tokens per tile (max MMA N)
+constexpr int TOK_ALIGN = 64;   // token rows per permutation block (scale atoms start at 0 or 64)
+constexpr int NQ = 16;          // MMA N granularity and the small token box height
+constexpr int BK = 256;
+constexpr int KB = BK / 2;
+constexpr int STAGES = 4;
+constexpr int EPI_WARPS = 8;    // two per TMEM lane quarter
+constexpr int kThreads = 64 + 32 * EPI_WARPS;
+constexpr uint32_t kTmemCols = 512;
+constexpr int ACC_COLS = BNMAX;          // two accumulators: [0, 192), [192, 384)
+constexpr int SFA_COL = 2 * ACC_COLS;    // 16 columns
+constexpr int SFB_COL = SFA_COL + 16;    // 8 columns per k-block, 32 in all
+constexpr int SFB_PER_KB = 8;
+constexpr int MAX_E = 1024;
+constexpr uint32_t kDevTimeout = 1u << 3;
+
+constexpr int A_BYTES = WM * KB;         // 16 KB
+constexpr int B_BYTES = BNMAX * KB;      // 24 KB
+constexpr int SFA_BYTES = WM * BK / 16;  // 2 KB
+constexpr int SFB_BYTES = 2 * 2048;      // up to two 128-row atom rows
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+constexpr int TR_STRIDE = 17;                      // h transpose tile: 32 tokens x 16 (+1) floats
+constexpr int TR_FLOATS = 32 * TR_STRIDE;
+constexpr int SMEM_BYTES =
+    1024 + STAGES * STAGE_BYTES + (2 * STAGES + 5) * 8 + 16 + (5 * MAX_E + 1) * 4 + EPI_WARPS * TR_FLOATS * 4;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+constexpr int MAX_CHUNKS = BNMAX / 32;
+
+enum { EPI_GATEUP = 0, EPI_DOWN = 1 };
+
+struct GroupedParams {
+  int K;             // reduction size
+  int NW;            // weight rows per expert
+  const int32_t* counts;
+  const int32_t* padded_offsets;
+  const int32_t* active;
+  const int32_t* row_pair;
+  const uint8_t* x_sf;   // token scales, MMA layout over the padded permuted rows
+  const uint8_t* w_sf;   // per expert NW*K/16 bytes
+  // gate/up
+  const float* x_scale;
+  const float* w13_scale;
+  const float* h_scale;
+  float* h_amax;
+  uint8_t* h_codes;
+  uint8_t* h_sf;
+  int I;
+  // down
+  const float* w2_scale;
+  const float* topk_w;
+  __nv_bfloat16* slots;
+  int H;
+  uint32_t* status;
+};
+
+struct Item {
+  int e, mt, r0, n_rows, N;
+};
+
+// Work item idx -> (expert, weight tile, token chunk); every input comes from shared memory.
+__device__ __forceinline__ Item get_item(int idx, int na, const int* prefix, const int* s_e, const int* s_ch,
+                                         const int* s_off, const int* s_cnt) {
+  int lo = 0, hi = na;  // find a with prefix[a] <= idx < prefix[a+1]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (prefix[mid] <= idx) lo = mid; else hi = mid;
+  }
+  Item it;
+  it.e = s_e[lo];
+  const int ch = s_ch[lo];
+  const int rem = idx - prefix[lo];
+  it.mt = rem / ch;
+  const int c = rem - it.mt * ch;
+  it.r0 = s_off[lo] + c * BNMAX;
+  it.n_rows = min(BNMAX, s_cnt[lo] - c * BNMAX);
+  it.N = (it.n_rows + NQ - 1) / NQ * NQ;
+  return it;
+}
+
+// silu(g) * u with the fast exponential and division (h is requantised to E2M1 right after;
+// a few ulp here only move values that sit on a rounding boundary of the 4-bit grid).
+__device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
+
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+               const __grid_constant__ CUtensorMap tmXs, GroupedParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + STAGES * A_BYTES;
+  uint8_t* sSFA = sB + STAGES * B_BYTES;
+  uint8_t* sSFB = sSFA + STAGES * SFA_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sSFB + STAGES * SFB_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* acc_full = bars + 2 * STAGES;   // [2]
+  uint64_t* acc_empty = acc_full + 2;       // [2]
+  uint64_t* drain = acc_full + 4;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int* prefix = reinterpret_cast<int*>(tmem_holder + 4);  // [MAX_E + 1]
+  int* s_e = prefix + MAX_E + 1;                           // [MAX_E]
+  int* s_ch = s_e + MAX_E;                                 // [MAX_E]
+  int* s_off = s_ch + MAX_E;                               // [MAX_E] first padded row
+  int* s_cnt = s_off + MAX_E;                              // [MAX_E] rows
+  float* s_tr = reinterpret_cast<float*>(s_cnt + MAX_E);   // [EPI_WARPS][TR_FLOATS]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int na = p.active[0];
+  const int wtiles = p.NW / WM;
+  // per active expert: chunks of <= BNMAX tokens, and the number of work items before it
+  for (int a = threadIdx.x; a < na; a += kThreads) {
+    const int e = p.active[1 + a];
+    const int c = p.counts[e];
+    s_e[a] = e;
+    s_cnt[a] = c;
+    s_off[a] = p.padded_offsets[e];
+    s_ch[a] = (c + BNMAX - 1) / BNMAX;
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], EPI_WARPS * 32);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmW);
+    prefetch_tensormap(&tmX);
+    prefetch_tensormap(&tmXs);
+  }
+  __syncthreads();
+  if (warp == 2) {  // exclusive scan of items per active expert
+    int carry = 0;
+    for (int base = 0; base < na; base += 32) {
+      const int a = base + lane;
+      const int v = a < na ? s_ch[a] * wtiles : 0;
+      int sum = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, sum, o);
+        if (lane >= o) sum += y;
+      }
+      if (a < na) prefix[a] = carry + sum - v;
+      carry += __shfl_sync(0xffffffffu, sum, 31);
+    }
+    if (lane == 0) prefix[na] = carry;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int total = prefix[na];
+  const int k_tiles = (p.K + BK - 1) / BK;
+  const int64_t katoms = p.K / 64;
+  auto abort_now = [&]() {
+    *abort_flag = 1;
+    atomicOr(p.status, kDevTimeout);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer ----
+    if (elect_one()) {
+      uint32_t it = 0;
+      for (int idx = blockIdx.x; idx < total && !*abort_flag; idx += gridDim.x) {
+        const Item w = get_item(idx, na, prefix, s_e, s_ch, s_off, s_cnt);
+        const uint8_t* wsf = p.w_sf + int64_t(w.e) * p.NW * (p.K / 16);
+        const int a0 = w.r0 / 128;
+        const int natoms = (w.r0 + w.N - 1) / 128 - a0 + 1;
+        for (int kt = 0; kt < k_tiles; ++kt, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1)) {
+            abort_now();
+            break;
+          }
+          const int nkb = min(4, (p.K - kt * BK) / 64);
+          const uint32_t sfb = nkb * 512;
+          mbar_arrive_expect_tx(&full[s], A_BYTES + w.N * KB + sfb * (1 + natoms));
+          tma_load_2d(sA + s * A_BYTES, &tmW, kt * KB, w.e * p.NW + w.mt * WM, &full[s]);
+          int b = 0;
+          for (; b + TOK_ALIGN <= w.N; b += TOK_ALIGN)
+            tma_load_2d(sB + s * B_BYTES + b * KB, &tmX, kt * KB, w.r0 + b, &full[s]);
+          for (; b < w.N; b += NQ) tma_load_2d(sB + s * B_BYTES + b * KB, &tmXs, kt * KB, w.r0 + b, &full[s]);
+          bulk_load(sSFA + s * SFA_BYTES, wsf + (int64_t(w.mt) * katoms + kt * 4) * 512, sfb, &full[s]);
+          for (int ar = 0; ar < natoms; ++ar)
+            bulk_load(sSFB + s * SFB_BYTES + ar * 2048, p.x_sf + (int64_t(a0 + ar) * katoms + kt * 4) * 512, sfb,
+                      &full[s]);
+        }
+      }
+      if (*abort_flag) {
+        for (uint32_t back = 0; back < STAGES && back < it; ++back) {
+          const uint32_t j = it - 1 - back;
+          mbar_wait(&full[j % STAGES], (j / STAGES) & 1, 1u << 16);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA ----
+    if (elect_one()) {
+      uint32_t it = 0, li = 0;
+      for (int idx = blockIdx.x; idx < total && !*abort_flag; idx += gridDim.x, ++li) {
+        const Item w = get_item(idx, na, prefix, s_e, s_ch, s_off, s_cnt);
+        const uint32_t ab = li & 1;
+        if (!mbar_wait(&acc_empty[ab], ((li >> 1) & 1) ^ 1)) {
+          abort_now();
+          break;
+        }
+        tc_fence_after();
+        const uint32_t idesc = idesc_mxf4nvf4(WM, w.N);
+        const int natoms = (w.r0 + w.N - 1) / 128 - w.r0 / 128 + 1;
+        const uint32_t g0 = (w.r0 % 128) / 32;  // 0 or 2
+        const uint32_t d_acc = tmem + ab * ACC_COLS;
+        bool ok = true;
+        for (int kt = 0; kt < k_tiles; ++kt, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&full[s], (it / STAGES) & 1)) {
+            abort_now();
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nkb = min(4, (p.K - kt * BK) / 64);
+          // descriptor start addresses advance in 16-byte units: 512-byte atoms (32), 32 bytes of K (2)
+          const uint64_t sfa_d = desc_sf_atom(sSFA + s * SFA_BYTES);
+          const uint64_t sfb_d = desc_sf_atom(sSFB + s * SFB_BYTES);
+          const uint64_t a_d = desc_kmajor_sw128(sA + s * A_BYTES);
+          const uint64_t b_d = desc_kmajor_sw128(sB + s * B_BYTES);
+          if (nkb == 4) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              tc_cp_sf(tmem + SFA_COL + 4 * j, sfa_d + 32 * j);
+              tc_cp_sf(tmem + SFB_COL + SFB_PER_KB * j, sfb_d + 32 * j);
+              if (natoms > 1) tc_cp_sf(tmem + SFB_COL + SFB_PER_KB * j + 4, sfb_d + 128 + 32 * j);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              tc_mma_mxf4nvf4(d_acc, a_d + 2 * j, b_d + 2 * j, idesc, tmem + SFA_COL + 4 * j,
+                              tmem + SFB_COL + SFB_PER_KB * j + g0, (kt | j) != 0 ? 1u : 0u);
+          } else {
+            for (int j = 0; j < nkb; ++j) {
+              tc_cp_sf(tmem + SFA_COL + 4 * j, sfa_d + 32 * j);
+              for (int ar = 0; ar < natoms; ++ar)
+                tc_cp_sf(tmem + SFB_COL + SFB_PER_KB * j + 4 * ar, sfb_d + 128 * ar + 32 * j);
+            }
+            for (int j = 0; j < nkb; ++j)
+              tc_mma_mxf4nvf4(d_acc, a_d + 2 * j, b_d + 2 * j, idesc, tmem + SFA_COL + 4 * j,
+                              tmem + SFB_COL + SFB_PER_KB * j + g0, (kt | j) != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[s]);
+        }
+        if (!ok) break;
+        tc_commit(&acc_full[ab]);
+      }
+      tc_commit(drain);
+      mbar_wait(drain, 0, 1u << 20);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue ----
+    const int q = warp & 3;                 // TMEM lane quarter this warp may read
+    const int half = (warp - 2) >> 2;       // the two warps of a quarter split the token chunks
+    const uint32_t trow = tmem + (uint32_t(q * 32) << 16);
+    float* tr = s_tr + (warp - 2) * TR_FLOATS;
+    uint32_t li = 0;
+    for (int idx = blockIdx.x; idx < total && !*abort_flag; idx += gridDim.x, ++li) {
+      const Item w = get_item(idx, na, prefix, s_e, s_ch, s_off, s_cnt);
+      const uint32_t ab = li & 1;
+      const int wrow = w.mt * WM + q * 32 + lane;  // this lane's weight row inside the expert
+      // per-item data, fetched before the accumulator is ready so its latency is hidden
+      float sg = 0.f, su = 0.f, sh = 0.f, sc = 0.f;
+      int32_t pr[MAX_CHUNKS / 2];
+      float wt[MAX_CHUNKS / 2];
+      if constexpr (EPI == EPI_GATEUP) {
+        const float sx = p.x_scale[0];
+        sg = sx * p.w13_scale[2 * w.e];
+        su = sx * p.w13_scale[2 * w.e + 1];
+        sh = p.h_scale[w.e];
+      } else {
+        sc = p.h_scale[w.e] * p.w2_scale[w.e];
+#pragma unroll
+        for (int c2 = 0; c2 < MAX_CHUNKS / 2; ++c2) {
+          const int tok = (2 * c2 + half) * 32 + lane;
+          pr[c2] = tok < w.n_rows ? p.row_pair[w.r0 + tok] : -1;
+        }
+#pragma unroll
+        for (int c2 = 0; c2 < MAX_CHUNKS / 2; ++c2) wt[c2] = pr[c2] >= 0 ? p.topk_w[pr[c2]] * sc : 0.0f;
+      }
+      if (!mbar_wait(&acc_full[ab], (li >> 1) & 1)) {
+        abort_now();
+        break;
+      }
+      tc_fence_after();
+      if constexpr (EPI == EPI_GATEUP) {
+        // lanes 0..15 hold gate rows i, lanes 16..31 the up rows i of one 16-wide block of h
+        const int64_t iblk = wrow >> 5;
+        float amax_all = 0.0f;
+#pragma unroll 1
+        for (int cc = half; cc * 32 < w.N; cc += 2) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(trow + ab * ACC_COLS + cc * 32, r);
+          tmem_ld_wait();
+          // lane l < 16 finishes tokens 0..15 of gate/up row pair l, lane l + 16 tokens 16..31
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float mine_lo = __uint_as_float(r[j]), mine_hi = __uint_as_float(r[16 + j]);
+            const float other = __shfl_xor_sync(0xffffffffu, lane < 16 ? mine_hi : mine_lo, 16);
+            const float g = lane < 16 ? mine_lo : other;
+            const float u = lane < 16 ? other : mine_hi;
+            tr[(j + 16 * (lane >> 4)) * TR_STRIDE + (lane & 15)] = silu_mul(g * sg, u * su);
+          }
+          __syncwarp();
+          // lane t quantises token t's 16 values (one block) in-thread
+          float hb[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) hb[i] = tr[lane * TR_STRIDE + i];
+          __syncwarp();
+          const int tok = cc * 32 + lane;
+          if (tok < w.n_rows) {
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(hb[i]));
+            float inv;
+            const uint32_t sf = block_scale(amax, sh, &inv);
+            const int64_t row = int64_t(w.r0) + tok;
+            *reinterpret_cast<uint2*>(p.h_codes + row * (p.I / 2) + iblk * 8) = encode_block16(hb, inv);
+            p.h_sf[sf_mma_offset(row, iblk, p.I)] = static_cast<uint8_t>(sf);
+            amax_all = fmaxf(amax_all, amax);
+          }
+        }
+        if (p.h_amax) {
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) amax_all = fmaxf(amax_all, __shfl_xor_sync(0xffffffffu, amax_all, o));
+          if (lane == 0 && amax_all > 0.0f) atomicMax(reinterpret_cast<int*>(p.h_amax + w.e), __float_as_int(amax_all));
+        }
+      } else {
+#pragma unroll
+        for (int c2 = 0; c2 < MAX_CHUNKS / 2; ++c2) {
+          const int cc = 2 * c2 + half;
+          if (cc * 32 >= w.N) break;
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(trow + ab * ACC_COLS + cc * 32, r);
+          tmem_ld_wait();
+          const int nj = min(32, w.n_rows - cc * 32);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            if (j >= nj) break;
+            const int32_t pair = __shfl_sync(0xffffffffu, pr[c2], j);
+            const float wj = __shfl_sync(0xffffffffu, wt[c2], j);
+            if (pair >= 0) p.slots[int64_t(pair) * p.H + wrow] = __float2bfloat16_rn(__uint_as_float(r[j]) * wj);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[ab]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+template <int EPI>
+nvfp4moe_status launch(const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& xs, const GroupedParams& p,
+                       int64_t max_items, cudaStream_t s) {
+  auto kern = grouped_kernel<EPI>;
+  static int configured[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return fail(NVFP4MOE_CUDA_ERROR, "grouped GEMM smem attribute: %s", cudaGetErrorString(e));
+    configured[dev] = 1;
+  }
+  int64_t grid = num_sms();
+  if (max_items < grid) grid = max_items > 0 ? max_items : 1;
+  kern<<<static_cast<int>(grid), kThreads, SMEM_BYTES, s>>>(w, x, xs, p);
+  return check_launch("grouped tcgen05 GEMM");
+}
+
+}  // namespace
+
+int grouped_token_align() { return TOK_ALIGN; }
+
+nvfp4moe_status launch_grouped_ffn(const GemmFfnArgs& a, cudaStream_t s) {
+  uint32_t* status = device_status_ptr();
+  if (!status) return fail(NVFP4MOE_CUDA_ERROR, "device status word unavailable");
+  if (a.E > MAX_E) return fail(NVFP4MOE_UNSUPPORTED_SHAPE, "grouped GEMM: E > %d", MAX_E);
+  // upper bound of work items: every pair its own chunk
+  const int64_t P = int64_t(a.T) * a.k;
+  const int64_t max_chunks = (P < a.E ? P : a.E) + P / BNMAX + 1;
+  CUtensorMap tw, tx, txs;
+  GroupedParams p{};
+  p.counts = a.counts;
+  p.padded_offsets = a.padded_offsets;
+  p.active = a.active;
+  p.row_pair = a.row_pair;
+  p.status = status;
+  // gate/up: weights W13 [E*2I][H], tokens x [rows_cap][H]
+  nvfp4moe_status st = make_code_map(&tw, a.w13_codes, int64_t(a.E) * 2 * a.I, a.H, WM);
+  if (st != NVFP4MOE_OK) return st;
+  st = make_code_map(&tx, a.x_codes, a.rows_cap, a.H, TOK_ALIGN);
+  if (st != NVFP4MOE_OK) return st;
+  st = make_code_map(&txs, a.x_codes, a.rows_cap, a.H, NQ);
+  if (st != NVFP4MOE_OK) return st;
+  p.K = a.H;
+  p.NW = 2 * a.I;
+  p.x_sf = a.x_sf;
+  p.w_sf = a.w13_sf;
+  p.x_scale = a.x_scale;
+  p.w13_scale = a.w13_scale;
+  p.h_scale = a.h_scale;
+  p.h_amax = a.h_amax;
+  p.h_codes = a.h_codes;
+  p.h_sf = a.h_sf;
+  p.I = a.I;
+  st = launch<EPI_GATEUP>(tw, tx, txs, p, max_chunks * (p.NW / WM), s);
+  if (st != NVFP4MOE_OK) return st;
+  if (a.stage_events) cudaEventRecord(reinterpret_cast<cudaEvent_t>(a.stage_events[4]), s);
+  // down: weights W2 [E*H][I], tokens h [rows_cap][I]
+  st = make_code_map(&tw, a.w2_codes, int64_t(a.E) * a.H, a.I, WM);
+  if (st != NVFP4MOE_OK) return st;
+  st = make_code_map(&tx, a.h_codes, a.rows_cap, a.I, TOK_ALIGN);
+  if (st != NVFP4MOE_OK) return st;
+  st = make_code_map(&txs, a.h_codes, a.rows_cap, a.I, NQ);
+  if (st != NVFP4MOE_OK) return st;
+  p.K = a.I;
+  p.NW = a.H;
+  p.x_sf = a.h_sf;
+  p.w_sf = a.w2_sf;
+  p.w2_scale = a.w2_scale;
+  p.topk_w = a.topk_w;
+  p.slots = static_cast<__nv_bfloat16*>(a.slots_bf16);
+  p.H = a.H;
+  return launch<EPI_DOWN>(tw, tx, txs, p, max_chunks * (p.NW / WM), s);
+}
+
+}  // namespace nvfp4moe

@@ -166,7 +166,8 @@ def check_layer(wl: W.Workload, ref: dict, out: torch.Tensor, layer: ops.MoeFFN,
         po = im["padded_offsets"].cpu().numpy()
         off = ref["offsets"]
         counts = ref["counts"]
-        assert np.array_equal(po, np.concatenate([[0], np.cumsum((counts + 127) // 128 * 128)]))
+        mt = im["m_tile"]
+        assert np.array_equal(po, np.concatenate([[0], np.cumsum((counts + mt - 1) // mt * mt)]))
         # padded row -> unpadded row: same expert, same rank
         e_of_pair = ref["ids"].reshape(-1)
         assert np.array_equal(p2r - po[e_of_pair] + off[e_of_pair], ref["pair_to_row"])

@@ -77,6 +77,7 @@ def test_workspace_queries(so):
     d.x_scale_mode = C.SCALE_DYNAMIC
     L = C.MoeFfnWsLayout()
     assert so.moe_ffn_workspace_layout(ctypes.byref(d), ctypes.byref(L)) == C.OK
+    # no GPU here: the tensor-core path is unavailable, AUTO falls back to the GEMV layout
     assert L.path == C.PATH_GEMV and L.m_tile == 1
     assert so.moe_ffn_workspace_size(ctypes.byref(d)) == L.total > 0
     offs = sorted([L.topk_ids, L.topk_w, L.counts, L.offsets, L.padded_offsets, L.pair_to_row, L.row_token,

@@ -125,8 +125,9 @@ def test_route_rejects_k_above_32(dev):
 
 
 # ------------------------------------------------------------ permutation ----
-@pytest.mark.parametrize("T,E,k", [(8, 8, 2), (16, 512, 10), (512, 512, 10), (4096, 256, 8), (1, 4, 4), (100, 1, 1)])
-@pytest.mark.parametrize("m_tile", [1, 128])
+@pytest.mark.parametrize("T,E,k", [(8, 8, 2), (16, 512, 10), (512, 512, 10), (4096, 256, 8), (1, 4, 4), (100, 1, 1),
+                                   (33, 1024, 32), (77, 600, 3), (3000, 40, 7)])
+@pytest.mark.parametrize("m_tile", [1, 32, 64, 128])
 def test_permute_parity(dev, T, E, k, m_tile):
     g = torch.Generator().manual_seed(T + E)
     logits = torch.randn(T, E, generator=g)

@@ -33,6 +33,9 @@ GEMM_CASES = {
     "long_prefill_small": W.scaled(W.WORKLOADS["long_prefill"], T=67, E=16, H=768, I=384, k=4),
     "dense_small": W.scaled(W.WORKLOADS["dense"], T=150, H=512, I=640),
     "one_expert_many_tiles": W.scaled(TINY, T=300, E=3, k=1, H=256, I=128),
+    "decode_shape": W.scaled(W.WORKLOADS["decode"], E=64, H=1024, I=256),
+    "decode_T1": W.scaled(W.WORKLOADS["decode"], T=1, E=64, H=1024, I=256),
+    "popular_expert_chunks": W.scaled(W.WORKLOADS["prefill_chunk"], T=450, E=16, H=512, I=128, k=2),
 }
 
 
