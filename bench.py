@@ -3,8 +3,10 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode] [--impl ours|reference]
 
 One step = one full pass of the layer (route, permute, quantise x, gate/up + SwiGLU +
-requantise, down, combine) over one batch of synthetic tokens, inputs resident in HBM.
-L2 is flushed (a 256 MiB write) before every timed step, outside the timed events.
+requantise, down, combine) over one batch of synthetic tokens, inputs resident in HBM,
+timed as a replay of the forward captured once into a CUDA graph (the kernels and buffers of
+an eager call, without the host's per-launch gaps).  L2 is flushed before every timed step (a 256 MiB write, then a 256 MiB read so the step
+starts from a clean, cold L2), outside the timed events.
 Prints one JSON line on rank 0.  With N > 1 (torchrun) every rank runs an independent
 replica on its own GPU (the layer has no cross-GPU exchange on one device's batch), the
 timed region is bracketed by barriers and the reported time is the max over ranks.
@@ -35,6 +37,23 @@ from nvfp4_mixture_experts_w4a4_b200 import ops, workloads as W  # noqa: E402
 METRIC = "NVFP4 MoE-layer tokens/s; % of HBM BW (decode) / % FP4 TC peak (prefill)"
 FP4_BYTES_PER_ELT = 0.5625  # 4-bit code + one E4M3 scale per 16 elements
 L2_FLUSH_BYTES = 256 << 20
+
+
+class L2Flush:
+    """Leaves L2 cold before a timed step: writes a 256 MiB buffer (evicting everything),
+    then reads another 256 MiB buffer so the write-backs of those dirty lines happen here,
+    outside the timed events, and the step starts from a clean, cold L2 (as after a previous
+    layer's weight reads) instead of paying for the flush's own write-backs."""
+
+    def __init__(self, dev):
+        self.w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+        self.sink = torch.empty((), dtype=torch.int32, device=dev)
+
+    def zero_(self):
+        self.w.zero_()
+        torch.amax(self.r, dim=0, out=self.sink)
+        return self
 
 
 def peaks():
@@ -176,27 +195,81 @@ def roofline(bytes_, flops, ms, pk):
             "frac": ach / pk["fp4_tflops"]}
 
 
-def time_steps(layer, act, steps: int, warmup: int, flush: torch.Tensor, dist_on: bool):
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(C.STAGES)] for _ in range(steps)]
+def capture_layer(layer, act, out, stage_events=None):
+    """The layer's forward captured once into a CUDA graph (with its stage marks as timing
+    nodes when stage_events is given); replays launch the same kernels on the same buffers."""
+    if stage_events is not None:
+        for e in stage_events:
+            e.record()  # materialise the events outside the capture
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph(keep_graph=True)
+    with torch.cuda.stream(s):
+        layer(act["x"], act["logits"], out=out)
+        s.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            layer(act["x"], act["logits"], out=out, stage_events=stage_events)
+    torch.cuda.current_stream().wait_stream(s)
+    g.instantiate()
+    torch.cuda.synchronize()
+    return g
+
+
+def kernel_nodes(g) -> int | None:
+    """Number of kernel launches in a captured graph (None when cuda-python cannot tell)."""
+    try:
+        from cuda.bindings import runtime as rt
+        graph = rt.cudaGraph_t(init_value=g.raw_cuda_graph())
+        err, nodes, n = rt.cudaGraphGetNodes(graph, numNodes=0)
+        err, nodes, n = rt.cudaGraphGetNodes(graph, numNodes=n)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        kinds = [rt.cudaGraphNodeGetType(nd)[1] for nd in nodes[:n]]
+        return sum(1 for t in kinds if t == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel)
+    except Exception:  # noqa: BLE001 - an introspection failure only loses the count
+        return None
+
+
+def time_steps(layer, act, steps: int, warmup: int, flush: L2Flush, dist_on: bool):
+    """Device time of K layer passes, each a replay of the captured forward between CUDA
+    events on the replay stream, L2 flushed before each; then K more replays of a capture that
+    carries the stage marks, for the per-stage split (its marks cost a little time each)."""
     out = torch.empty(act["x"].shape[0], layer.w.H, dtype=torch.bfloat16, device=act["x"].device)
+    g = capture_layer(layer, act, out)
+    launches = kernel_nodes(g)
     for _ in range(warmup):
         flush.zero_()
-        layer(act["x"], act["logits"], out=out)
+        g.replay()
     torch.cuda.synchronize()
     if dist_on:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    for i in range(steps):
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in ev:
         flush.zero_()
-        layer(act["x"], act["logits"], out=out, stage_events=ev[i])
+        a.record()
+        g.replay()
+        b.record()
     torch.cuda.synchronize()
     if dist_on:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    step_ms = [e[0].elapsed_time(e[C.STAGES - 1]) for e in ev]
-    stage_ms = {name: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in ev)
-                for j, name in enumerate(C.STAGE_NAMES)}
-    return step_ms, stage_ms
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+
+    marks = [torch.cuda.Event(enable_timing=True) for _ in range(C.STAGES)]
+    gs = capture_layer(layer, act, out, stage_events=marks)
+    per_stage = {name: [] for name in C.STAGE_NAMES}
+    for i in range(warmup + steps):
+        flush.zero_()
+        gs.replay()
+        torch.cuda.synchronize()
+        if i >= warmup:
+            for j, name in enumerate(C.STAGE_NAMES):
+                per_stage[name].append(marks[j].elapsed_time(marks[j + 1]))
+    stage_ms = {name: statistics.mean(v) for name, v in per_stage.items()}
+    del g, gs
+    return step_ms, stage_ms, launches
 
 
 def time_e2e(layer, act, steps: int, warmup: int, flush: torch.Tensor):
@@ -307,7 +380,7 @@ def main():
                                              device_id=dev)
     wl = W.WORKLOADS[args.workload]
     cfg = {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "top_k": wl.k,
-           "zipf_s": wl.zipf_s, "outlier_frac": wl.outlier_frac, "l2": "flushed before every step (256 MiB write)",
+           "zipf_s": wl.zipf_s, "outlier_frac": wl.outlier_frac, "l2": "flushed before every step (256 MiB write, then 256 MiB read)",
            "seed": 0, "parallelism": f"replicas x{world}"}
 
     if args.impl == "reference":
@@ -349,9 +422,9 @@ def main():
     path = {"auto": C.PATH_AUTO, "gemv": C.PATH_GEMV, "tcgen05": C.PATH_GEMM}[args.path]
     act, host, experts, layer = setup_layer(wl, dev, keep_tokens=n_cpu if (rank == 0 and world == 1) else 0,
                                             path=path)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     with ClockSampler(local) as clk:
-        step_ms, stage_ms = time_steps(layer, act, args.steps, args.warmup, flush, dist_on)
+        step_ms, stage_ms, launches = time_steps(layer, act, args.steps, args.warmup, flush, dist_on)
     total_ms = sum(step_ms)
     if dist_on:
         t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
@@ -398,7 +471,8 @@ def main():
             "config": cfg, "roofline": roof, "cpu_baseline": cpu,
             "e2e": {"value": world * wl.T / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": gpu_launches_per_step(layer) * args.steps,
+            "gpu_launches": (launches if launches is not None else gpu_launches_per_step(layer)) * args.steps,
+            "launches_per_step": launches, "timing": "CUDA-graph replay of the layer's forward, events on the replay stream",
             "clocks": clk.summary(),
             "stages_ms": stage_ms,
             "layer": {"bytes": alg["layer_bytes"], "flops": alg["flops"], "hbm_gbs": layer_bw,

@@ -140,27 +140,44 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   const int T = d->T, H = d->H, I = d->I, E = d->E, k = d->top_k;
   const int64_t rows_cap = moe_permute_rows_capacity(T, E, k, L.m_tile);
   auto mark = [&](int i) {
-    if (d->stage_events) cudaEventRecord(reinterpret_cast<cudaEvent_t>(d->stage_events[i]), s);
+    // external records, so the marks become timing nodes when the stream is being captured
+    if (d->stage_events) cudaEventRecordWithFlags(reinterpret_cast<cudaEvent_t>(d->stage_events[i]), s,
+                                                  cudaEventRecordExternal);
   };
-
-  mark(0);
-  st = moe_route(logits, T, E, k, I32(L.topk_ids), F32(L.topk_w), stream);
-  if (st != NVFP4MOE_OK) return st;
-  mark(1);
-  st = moe_permute(I32(L.topk_ids), T, E, k, L.m_tile, rows_cap, I32(L.counts), I32(L.offsets),
-                   I32(L.padded_offsets), I32(L.pair_to_row), I32(L.row_token), I32(L.row_pair),
-                   I32(L.tile_expert), I32(L.active), d->h_amax, stream);
-  if (st != NVFP4MOE_OK) return st;
-  mark(2);
 
   const bool dyn = d->x_scale_mode == NVFP4MOE_SCALE_DYNAMIC;
   float* xs = dyn ? F32(L.x_scale) : const_cast<float*>(d->x_scale);
   const size_t qws = nvfp4_quantize_workspace_size(1, T, H);
+  const bool fused = prologue_fits(T, E, k);
+
+  mark(0);
+  if (fused) {
+    // small batch: routing, permutation and x quantisation in one cluster launch
+    st = launch_prologue(x, logits, T, H, E, k, L.m_tile, dyn ? 1 : 0, xs, I32(L.topk_ids), F32(L.topk_w),
+                         I32(L.counts), I32(L.offsets), I32(L.padded_offsets), I32(L.pair_to_row), I32(L.row_token),
+                         I32(L.row_pair), I32(L.tile_expert), I32(L.active), d->h_amax,
+                         L.path == NVFP4MOE_PATH_GEMM ? 1 : 0, ws + L.x_codes, ws + L.x_sf, s);
+    if (st != NVFP4MOE_OK) return st;
+    mark(1);
+    mark(2);
+  } else {
+    st = moe_route(logits, T, E, k, I32(L.topk_ids), F32(L.topk_w), stream);
+    if (st != NVFP4MOE_OK) return st;
+    mark(1);
+    st = moe_permute(I32(L.topk_ids), T, E, k, L.m_tile, rows_cap, I32(L.counts), I32(L.offsets),
+                     I32(L.padded_offsets), I32(L.pair_to_row), I32(L.row_token), I32(L.row_pair),
+                     I32(L.tile_expert), I32(L.active), d->h_amax, stream);
+    if (st != NVFP4MOE_OK) return st;
+    mark(2);
+  }
+
   if (L.path == NVFP4MOE_PATH_GEMV) {
     // x quantised once per token, token-major
-    st = nvfp4_quantize(x, NVFP4MOE_DTYPE_BF16, 1, T, H, H, 0, nullptr, T, d->x_scale_mode, xs,
-                        ws + L.x_codes, 0, ws + L.x_sf, 0, NVFP4MOE_SF_MMA, ws + L.amax_partials, qws, stream);
-    if (st != NVFP4MOE_OK) return st;
+    if (!fused) {
+      st = nvfp4_quantize(x, NVFP4MOE_DTYPE_BF16, 1, T, H, H, 0, nullptr, T, d->x_scale_mode, xs, ws + L.x_codes, 0,
+                          ws + L.x_sf, 0, NVFP4MOE_SF_MMA, ws + L.amax_partials, qws, stream);
+      if (st != NVFP4MOE_OK) return st;
+    }
     mark(3);
     GemvGateUpArgs g;
     g.H = H; g.I = I;
@@ -191,14 +208,16 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
 
   // tensor-core path: x quantised once per token (into the slot region, which is free until
   // the down GEMM), then copied into the padded expert-order rows
-  uint8_t* xt_codes = ws + L.slots;
-  uint8_t* xt_sf = xt_codes + ((int64_t(T) * H / 2 + 255) / 256) * 256;
-  st = nvfp4_quantize(x, NVFP4MOE_DTYPE_BF16, 1, T, H, H, 0, nullptr, T, d->x_scale_mode, xs, xt_codes, 0, xt_sf, 0,
-                      NVFP4MOE_SF_MMA, ws + L.amax_partials, qws, stream);
-  if (st != NVFP4MOE_OK) return st;
-  st = launch_replicate_rows(xt_codes, xt_sf, I32(L.row_token), I32(L.padded_offsets) + E, rows_cap, T, H,
-                             ws + L.x_codes, ws + L.x_sf, s);
-  if (st != NVFP4MOE_OK) return st;
+  if (!fused) {
+    uint8_t* xt_codes = ws + L.slots;
+    uint8_t* xt_sf = xt_codes + ((int64_t(T) * H / 2 + 255) / 256) * 256;
+    st = nvfp4_quantize(x, NVFP4MOE_DTYPE_BF16, 1, T, H, H, 0, nullptr, T, d->x_scale_mode, xs, xt_codes, 0, xt_sf,
+                        0, NVFP4MOE_SF_MMA, ws + L.amax_partials, qws, stream);
+    if (st != NVFP4MOE_OK) return st;
+    st = launch_replicate_rows(xt_codes, xt_sf, I32(L.row_token), I32(L.padded_offsets) + E, rows_cap, T, H,
+                               ws + L.x_codes, ws + L.x_sf, s);
+    if (st != NVFP4MOE_OK) return st;
+  }
   mark(3);
   GemmFfnArgs a;
   a.T = T; a.H = H; a.I = I; a.E = E; a.k = k;

@@ -55,4 +55,13 @@ nvfp4moe_status launch_replicate_rows(const uint8_t* codes_tok, const uint8_t* s
 nvfp4moe_status launch_combine_bf16(const void* slots, const int32_t* pair_to_row, int T, int H, int k,
                                     void* out, cudaStream_t s);
 
+// Small-batch prologue (route + permute + quantise x) in one launch of an 8-CTA cluster;
+// see prologue.cu.
+bool prologue_fits(int T, int E, int k);
+nvfp4moe_status launch_prologue(const void* x, const float* logits, int T, int H, int E, int k, int m_tile,
+                                int dynamic, float* x_scale, int32_t* ids, float* w, int32_t* counts, int32_t* offsets,
+                                int32_t* padded_offsets, int32_t* pair_to_row, int32_t* row_token, int32_t* row_pair,
+                                int32_t* tile_expert, int32_t* active, float* zero_f32, int expert_order,
+                                uint8_t* x_codes, uint8_t* x_sf, cudaStream_t s);
+
 }  // namespace nvfp4moe

@@ -28,33 +28,42 @@ namespace {
 using namespace sm100;
 
 constexpr int WM = 128;         // weight rows per tile
-constexpr int BNMAX = 192;      // tokens per tile (max MMA N)
 constexpr int TOK_ALIGN = 64;   // token rows per permutation block (scale atoms start at 0 or 64)
 constexpr int NQ = 16;          // MMA N granularity and the small token box height
 constexpr int BK = 256;
 constexpr int KB = BK / 2;
-constexpr int STAGES = 4;
 constexpr int EPI_WARPS = 8;    // two per TMEM lane quarter
 constexpr int kThreads = 64 + 32 * EPI_WARPS;
 constexpr uint32_t kTmemCols = 512;
-constexpr int ACC_COLS = BNMAX;          // two accumulators: [0, 192), [192, 384)
-constexpr int SFA_COL = 2 * ACC_COLS;    // 16 columns
-constexpr int SFB_COL = SFA_COL + 16;    // 8 columns per k-block, 32 in all
-constexpr int SFB_PER_KB = 8;
 constexpr int MAX_E = 1024;
 constexpr uint32_t kDevTimeout = 1u << 3;
-
-constexpr int A_BYTES = WM * KB;         // 16 KB
-constexpr int B_BYTES = BNMAX * KB;      // 24 KB
-constexpr int SFA_BYTES = WM * BK / 16;  // 2 KB
-constexpr int SFB_BYTES = 2 * 2048;      // up to two 128-row atom rows
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-constexpr int TR_STRIDE = 17;                      // h transpose tile: 32 tokens x 16 (+1) floats
+constexpr int TR_STRIDE = 17;   // h transpose tile: 32 tokens x 16 (+1) floats
 constexpr int TR_FLOATS = 32 * TR_STRIDE;
-constexpr int SMEM_BYTES =
-    1024 + STAGES * STAGE_BYTES + (2 * STAGES + 5) * 8 + 16 + (5 * MAX_E + 1) * 4 + EPI_WARPS * TR_FLOATS * 4;
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-constexpr int MAX_CHUNKS = BNMAX / 32;
+constexpr int SFB_PER_KB = 8;   // TMEM columns of token scales per k-block (two atoms)
+
+// Tile configuration: BNMAX tokens per tile at most, STAGES shared-memory stages.
+//   <192, 4> general; <64, 6> when no expert can hold more than 64 tokens (T <= 64), which
+//   keeps more weight bytes in flight for the small decode tiles.
+template <int BN_, int STAGES_>
+struct Cfg {
+  static constexpr int BNMAX = BN_;
+  static constexpr int STAGES = STAGES_;
+  static constexpr int ACC_COLS = BNMAX;                 // two accumulators
+  static constexpr int SFA_COL = 2 * ACC_COLS;           // 16 columns
+  static constexpr int SFB_COL = SFA_COL + 16;           // 32 columns
+  static constexpr int A_BYTES = WM * KB;                // 16 KB
+  static constexpr int B_BYTES = BNMAX * KB;
+  static constexpr int SFA_BYTES = WM * BK / 16;         // 2 KB
+  static constexpr int SFB_BYTES = 2 * 2048;             // up to two 128-row atom rows
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int SMEM_BYTES =
+      1024 + STAGES * STAGE_BYTES + (2 * STAGES + 5) * 8 + 16 + (5 * MAX_E + 1) * 4 + EPI_WARPS * TR_FLOATS * 4;
+  static constexpr int MAX_CHUNKS = BNMAX / 32;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(SFB_COL + 32 <= int(kTmemCols), "TMEM budget");
+};
+using CfgWide = Cfg<192, 4>;
+using CfgDecode = Cfg<64, 6>;
 
 enum { EPI_GATEUP = 0, EPI_DOWN = 1 };
 
@@ -88,6 +97,7 @@ struct Item {
 };
 
 // Work item idx -> (expert, weight tile, token chunk); every input comes from shared memory.
+template <int BNMAX>
 __device__ __forceinline__ Item get_item(int idx, int na, const int* prefix, const int* s_e, const int* s_ch,
                                          const int* s_off, const int* s_cnt) {
   int lo = 0, hi = na;  // find a with prefix[a] <= idx < prefix[a+1]
@@ -111,23 +121,23 @@ __device__ __forceinline__ Item get_item(int idx, int na, const int* prefix, con
 // a few ulp here only move values that sit on a rounding boundary of the 4-bit grid).
 __device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
-template <int EPI>
+template <int EPI, class C>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                const __grid_constant__ CUtensorMap tmXs, GroupedParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = sA + STAGES * A_BYTES;
-  uint8_t* sSFA = sB + STAGES * B_BYTES;
-  uint8_t* sSFB = sSFA + STAGES * SFA_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sSFB + STAGES * SFB_BYTES);
+  uint8_t* sB = sA + C::STAGES * C::A_BYTES;
+  uint8_t* sSFA = sB + C::STAGES * C::B_BYTES;
+  uint8_t* sSFB = sSFA + C::STAGES * C::SFA_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sSFB + C::STAGES * C::SFB_BYTES);
   uint64_t* full = bars;
-  uint64_t* empty = bars + STAGES;
-  uint64_t* acc_full = bars + 2 * STAGES;   // [2]
+  uint64_t* empty = bars + C::STAGES;
+  uint64_t* acc_full = bars + 2 * C::STAGES;   // [2]
   uint64_t* acc_empty = acc_full + 2;       // [2]
   uint64_t* drain = acc_full + 4;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   int* prefix = reinterpret_cast<int*>(tmem_holder + 4);  // [MAX_E + 1]
   int* s_e = prefix + MAX_E + 1;                           // [MAX_E]
@@ -139,17 +149,17 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int na = p.active[0];
   const int wtiles = p.NW / WM;
-  // per active expert: chunks of <= BNMAX tokens, and the number of work items before it
+  // per active expert: chunks of <= C::BNMAX tokens, and the number of work items before it
   for (int a = threadIdx.x; a < na; a += kThreads) {
     const int e = p.active[1 + a];
     const int c = p.counts[e];
     s_e[a] = e;
     s_cnt[a] = c;
     s_off[a] = p.padded_offsets[e];
-    s_ch[a] = (c + BNMAX - 1) / BNMAX;
+    s_ch[a] = (c + C::BNMAX - 1) / C::BNMAX;
   }
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -204,34 +214,34 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
     if (elect_one()) {
       uint32_t it = 0;
       for (int idx = blockIdx.x; idx < total && !*abort_flag; idx += gridDim.x) {
-        const Item w = get_item(idx, na, prefix, s_e, s_ch, s_off, s_cnt);
+        const Item w = get_item<C::BNMAX>(idx, na, prefix, s_e, s_ch, s_off, s_cnt);
         const uint8_t* wsf = p.w_sf + int64_t(w.e) * p.NW * (p.K / 16);
         const int a0 = w.r0 / 128;
         const int natoms = (w.r0 + w.N - 1) / 128 - a0 + 1;
         for (int kt = 0; kt < k_tiles; ++kt, ++it) {
-          const int s = it % STAGES;
-          if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1)) {
+          const int s = it % C::STAGES;
+          if (!mbar_wait(&empty[s], ((it / C::STAGES) & 1) ^ 1)) {
             abort_now();
             break;
           }
           const int nkb = min(4, (p.K - kt * BK) / 64);
           const uint32_t sfb = nkb * 512;
-          mbar_arrive_expect_tx(&full[s], A_BYTES + w.N * KB + sfb * (1 + natoms));
-          tma_load_2d(sA + s * A_BYTES, &tmW, kt * KB, w.e * p.NW + w.mt * WM, &full[s]);
+          mbar_arrive_expect_tx(&full[s], C::A_BYTES + w.N * KB + sfb * (1 + natoms));
+          tma_load_2d(sA + s * C::A_BYTES, &tmW, kt * KB, w.e * p.NW + w.mt * WM, &full[s]);
           int b = 0;
           for (; b + TOK_ALIGN <= w.N; b += TOK_ALIGN)
-            tma_load_2d(sB + s * B_BYTES + b * KB, &tmX, kt * KB, w.r0 + b, &full[s]);
-          for (; b < w.N; b += NQ) tma_load_2d(sB + s * B_BYTES + b * KB, &tmXs, kt * KB, w.r0 + b, &full[s]);
-          bulk_load(sSFA + s * SFA_BYTES, wsf + (int64_t(w.mt) * katoms + kt * 4) * 512, sfb, &full[s]);
+            tma_load_2d(sB + s * C::B_BYTES + b * KB, &tmX, kt * KB, w.r0 + b, &full[s]);
+          for (; b < w.N; b += NQ) tma_load_2d(sB + s * C::B_BYTES + b * KB, &tmXs, kt * KB, w.r0 + b, &full[s]);
+          bulk_load(sSFA + s * C::SFA_BYTES, wsf + (int64_t(w.mt) * katoms + kt * 4) * 512, sfb, &full[s]);
           for (int ar = 0; ar < natoms; ++ar)
-            bulk_load(sSFB + s * SFB_BYTES + ar * 2048, p.x_sf + (int64_t(a0 + ar) * katoms + kt * 4) * 512, sfb,
+            bulk_load(sSFB + s * C::SFB_BYTES + ar * 2048, p.x_sf + (int64_t(a0 + ar) * katoms + kt * 4) * 512, sfb,
                       &full[s]);
         }
       }
       if (*abort_flag) {
-        for (uint32_t back = 0; back < STAGES && back < it; ++back) {
+        for (uint32_t back = 0; back < C::STAGES && back < it; ++back) {
           const uint32_t j = it - 1 - back;
-          mbar_wait(&full[j % STAGES], (j / STAGES) & 1, 1u << 16);
+          mbar_wait(&full[j % C::STAGES], (j / C::STAGES) & 1, 1u << 16);
         }
       }
     }
@@ -240,7 +250,7 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
     if (elect_one()) {
       uint32_t it = 0, li = 0;
       for (int idx = blockIdx.x; idx < total && !*abort_flag; idx += gridDim.x, ++li) {
-        const Item w = get_item(idx, na, prefix, s_e, s_ch, s_off, s_cnt);
+        const Item w = get_item<C::BNMAX>(idx, na, prefix, s_e, s_ch, s_off, s_cnt);
         const uint32_t ab = li & 1;
         if (!mbar_wait(&acc_empty[ab], ((li >> 1) & 1) ^ 1)) {
           abort_now();
@@ -250,11 +260,11 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
         const uint32_t idesc = idesc_mxf4nvf4(WM, w.N);
         const int natoms = (w.r0 + w.N - 1) / 128 - w.r0 / 128 + 1;
         const uint32_t g0 = (w.r0 % 128) / 32;  // 0 or 2
-        const uint32_t d_acc = tmem + ab * ACC_COLS;
+        const uint32_t d_acc = tmem + ab * C::ACC_COLS;
         bool ok = true;
         for (int kt = 0; kt < k_tiles; ++kt, ++it) {
-          const int s = it % STAGES;
-          if (!mbar_wait(&full[s], (it / STAGES) & 1)) {
+          const int s = it % C::STAGES;
+          if (!mbar_wait(&full[s], (it / C::STAGES) & 1)) {
             abort_now();
             ok = false;
             break;
@@ -262,30 +272,30 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
           tc_fence_after();
           const int nkb = min(4, (p.K - kt * BK) / 64);
           // descriptor start addresses advance in 16-byte units: 512-byte atoms (32), 32 bytes of K (2)
-          const uint64_t sfa_d = desc_sf_atom(sSFA + s * SFA_BYTES);
-          const uint64_t sfb_d = desc_sf_atom(sSFB + s * SFB_BYTES);
-          const uint64_t a_d = desc_kmajor_sw128(sA + s * A_BYTES);
-          const uint64_t b_d = desc_kmajor_sw128(sB + s * B_BYTES);
+          const uint64_t sfa_d = desc_sf_atom(sSFA + s * C::SFA_BYTES);
+          const uint64_t sfb_d = desc_sf_atom(sSFB + s * C::SFB_BYTES);
+          const uint64_t a_d = desc_kmajor_sw128(sA + s * C::A_BYTES);
+          const uint64_t b_d = desc_kmajor_sw128(sB + s * C::B_BYTES);
           if (nkb == 4) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              tc_cp_sf(tmem + SFA_COL + 4 * j, sfa_d + 32 * j);
-              tc_cp_sf(tmem + SFB_COL + SFB_PER_KB * j, sfb_d + 32 * j);
-              if (natoms > 1) tc_cp_sf(tmem + SFB_COL + SFB_PER_KB * j + 4, sfb_d + 128 + 32 * j);
+              tc_cp_sf(tmem + C::SFA_COL + 4 * j, sfa_d + 32 * j);
+              tc_cp_sf(tmem + C::SFB_COL + SFB_PER_KB * j, sfb_d + 32 * j);
+              if (natoms > 1) tc_cp_sf(tmem + C::SFB_COL + SFB_PER_KB * j + 4, sfb_d + 128 + 32 * j);
             }
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              tc_mma_mxf4nvf4(d_acc, a_d + 2 * j, b_d + 2 * j, idesc, tmem + SFA_COL + 4 * j,
-                              tmem + SFB_COL + SFB_PER_KB * j + g0, (kt | j) != 0 ? 1u : 0u);
+              tc_mma_mxf4nvf4(d_acc, a_d + 2 * j, b_d + 2 * j, idesc, tmem + C::SFA_COL + 4 * j,
+                              tmem + C::SFB_COL + SFB_PER_KB * j + g0, (kt | j) != 0 ? 1u : 0u);
           } else {
             for (int j = 0; j < nkb; ++j) {
-              tc_cp_sf(tmem + SFA_COL + 4 * j, sfa_d + 32 * j);
+              tc_cp_sf(tmem + C::SFA_COL + 4 * j, sfa_d + 32 * j);
               for (int ar = 0; ar < natoms; ++ar)
-                tc_cp_sf(tmem + SFB_COL + SFB_PER_KB * j + 4 * ar, sfb_d + 128 * ar + 32 * j);
+                tc_cp_sf(tmem + C::SFB_COL + SFB_PER_KB * j + 4 * ar, sfb_d + 128 * ar + 32 * j);
             }
             for (int j = 0; j < nkb; ++j)
-              tc_mma_mxf4nvf4(d_acc, a_d + 2 * j, b_d + 2 * j, idesc, tmem + SFA_COL + 4 * j,
-                              tmem + SFB_COL + SFB_PER_KB * j + g0, (kt | j) != 0 ? 1u : 0u);
+              tc_mma_mxf4nvf4(d_acc, a_d + 2 * j, b_d + 2 * j, idesc, tmem + C::SFA_COL + 4 * j,
+                              tmem + C::SFB_COL + SFB_PER_KB * j + g0, (kt | j) != 0 ? 1u : 0u);
           }
           tc_commit(&empty[s]);
         }
@@ -303,13 +313,13 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
     float* tr = s_tr + (warp - 2) * TR_FLOATS;
     uint32_t li = 0;
     for (int idx = blockIdx.x; idx < total && !*abort_flag; idx += gridDim.x, ++li) {
-      const Item w = get_item(idx, na, prefix, s_e, s_ch, s_off, s_cnt);
+      const Item w = get_item<C::BNMAX>(idx, na, prefix, s_e, s_ch, s_off, s_cnt);
       const uint32_t ab = li & 1;
       const int wrow = w.mt * WM + q * 32 + lane;  // this lane's weight row inside the expert
       // per-item data, fetched before the accumulator is ready so its latency is hidden
       float sg = 0.f, su = 0.f, sh = 0.f, sc = 0.f;
-      int32_t pr[MAX_CHUNKS / 2];
-      float wt[MAX_CHUNKS / 2];
+      int32_t pr[C::MAX_CHUNKS / 2];
+      float wt[C::MAX_CHUNKS / 2];
       if constexpr (EPI == EPI_GATEUP) {
         const float sx = p.x_scale[0];
         sg = sx * p.w13_scale[2 * w.e];
@@ -318,12 +328,12 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
       } else {
         sc = p.h_scale[w.e] * p.w2_scale[w.e];
 #pragma unroll
-        for (int c2 = 0; c2 < MAX_CHUNKS / 2; ++c2) {
+        for (int c2 = 0; c2 < C::MAX_CHUNKS / 2; ++c2) {
           const int tok = (2 * c2 + half) * 32 + lane;
           pr[c2] = tok < w.n_rows ? p.row_pair[w.r0 + tok] : -1;
         }
 #pragma unroll
-        for (int c2 = 0; c2 < MAX_CHUNKS / 2; ++c2) wt[c2] = pr[c2] >= 0 ? p.topk_w[pr[c2]] * sc : 0.0f;
+        for (int c2 = 0; c2 < C::MAX_CHUNKS / 2; ++c2) wt[c2] = pr[c2] >= 0 ? p.topk_w[pr[c2]] * sc : 0.0f;
       }
       if (!mbar_wait(&acc_full[ab], (li >> 1) & 1)) {
         abort_now();
@@ -337,7 +347,7 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
 #pragma unroll 1
         for (int cc = half; cc * 32 < w.N; cc += 2) {
           uint32_t r[32];
-          tmem_ld_32x32b_x32(trow + ab * ACC_COLS + cc * 32, r);
+          tmem_ld_32x32b_x32(trow + ab * C::ACC_COLS + cc * 32, r);
           tmem_ld_wait();
           // lane l < 16 finishes tokens 0..15 of gate/up row pair l, lane l + 16 tokens 16..31
 #pragma unroll
@@ -374,11 +384,11 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
         }
       } else {
 #pragma unroll
-        for (int c2 = 0; c2 < MAX_CHUNKS / 2; ++c2) {
+        for (int c2 = 0; c2 < C::MAX_CHUNKS / 2; ++c2) {
           const int cc = 2 * c2 + half;
           if (cc * 32 >= w.N) break;
           uint32_t r[32];
-          tmem_ld_32x32b_x32(trow + ab * ACC_COLS + cc * 32, r);
+          tmem_ld_32x32b_x32(trow + ab * C::ACC_COLS + cc * 32, r);
           tmem_ld_wait();
           const int nj = min(32, w.n_rows - cc * 32);
 #pragma unroll
@@ -401,22 +411,34 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
-template <int EPI>
-nvfp4moe_status launch(const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& xs, const GroupedParams& p,
-                       int64_t max_items, cudaStream_t s) {
-  auto kern = grouped_kernel<EPI>;
+template <int EPI, class C>
+nvfp4moe_status launch_cfg(const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& xs, const GroupedParams& p,
+                           int64_t max_items, cudaStream_t s) {
+  auto kern = grouped_kernel<EPI, C>;
   static int configured[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !configured[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return fail(NVFP4MOE_CUDA_ERROR, "grouped GEMM smem attribute: %s", cudaGetErrorString(e));
     configured[dev] = 1;
   }
   int64_t grid = num_sms();
   if (max_items < grid) grid = max_items > 0 ? max_items : 1;
-  kern<<<static_cast<int>(grid), kThreads, SMEM_BYTES, s>>>(w, x, xs, p);
+  kern<<<static_cast<int>(grid), kThreads, C::SMEM_BYTES, s>>>(w, x, xs, p);
   return check_launch("grouped tcgen05 GEMM");
+}
+
+template <int EPI>
+nvfp4moe_status launch(bool decode, const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& xs,
+                       const GroupedParams& p, int64_t max_rows_per_expert, int64_t P, int64_t E, cudaStream_t s) {
+  // upper bound of work items: every expert its chunks, weight tiles per chunk
+  const int64_t bn = decode ? CfgDecode::BNMAX : CfgWide::BNMAX;
+  const int64_t chunks = (P < E ? P : E) + P / bn + 1;
+  const int64_t items = chunks * (p.NW / WM);
+  (void)max_rows_per_expert;
+  if (decode) return launch_cfg<EPI, CfgDecode>(w, x, xs, p, items, s);
+  return launch_cfg<EPI, CfgWide>(w, x, xs, p, items, s);
 }
 
 }  // namespace
@@ -427,9 +449,9 @@ nvfp4moe_status launch_grouped_ffn(const GemmFfnArgs& a, cudaStream_t s) {
   uint32_t* status = device_status_ptr();
   if (!status) return fail(NVFP4MOE_CUDA_ERROR, "device status word unavailable");
   if (a.E > MAX_E) return fail(NVFP4MOE_UNSUPPORTED_SHAPE, "grouped GEMM: E > %d", MAX_E);
-  // upper bound of work items: every pair its own chunk
   const int64_t P = int64_t(a.T) * a.k;
-  const int64_t max_chunks = (P < a.E ? P : a.E) + P / BNMAX + 1;
+  // no expert receives more than T tokens (a token names an expert at most once)
+  const bool decode = a.T <= CfgDecode::BNMAX;
   CUtensorMap tw, tx, txs;
   GroupedParams p{};
   p.counts = a.counts;
@@ -455,9 +477,10 @@ nvfp4moe_status launch_grouped_ffn(const GemmFfnArgs& a, cudaStream_t s) {
   p.h_codes = a.h_codes;
   p.h_sf = a.h_sf;
   p.I = a.I;
-  st = launch<EPI_GATEUP>(tw, tx, txs, p, max_chunks * (p.NW / WM), s);
+  st = launch<EPI_GATEUP>(decode, tw, tx, txs, p, a.T, P, a.E, s);
   if (st != NVFP4MOE_OK) return st;
-  if (a.stage_events) cudaEventRecord(reinterpret_cast<cudaEvent_t>(a.stage_events[4]), s);
+  if (a.stage_events)
+    cudaEventRecordWithFlags(reinterpret_cast<cudaEvent_t>(a.stage_events[4]), s, cudaEventRecordExternal);
   // down: weights W2 [E*H][I], tokens h [rows_cap][I]
   st = make_code_map(&tw, a.w2_codes, int64_t(a.E) * a.H, a.I, WM);
   if (st != NVFP4MOE_OK) return st;
@@ -473,7 +496,7 @@ nvfp4moe_status launch_grouped_ffn(const GemmFfnArgs& a, cudaStream_t s) {
   p.topk_w = a.topk_w;
   p.slots = static_cast<__nv_bfloat16*>(a.slots_bf16);
   p.H = a.H;
-  return launch<EPI_DOWN>(tw, tx, txs, p, max_chunks * (p.NW / WM), s);
+  return launch<EPI_DOWN>(decode, tw, tx, txs, p, a.T, P, a.E, s);
 }
 
 }  // namespace nvfp4moe

@@ -1,0 +1,68 @@
+// Warp top-k over one token's router logits, shared by moe_route and the small-batch
+// prologue so both select and weight experts identically.
+//
+// Lane l holds logits l, l+32, ... (PER_LANE slots, E <= 32*PER_LANE) as 64-bit keys: the
+// high word is the logit mapped to an unsigned integer with the same order (after -0 is
+// turned into +0, so the two zeros tie), the low word is 0xFFFF - index, so among equal
+// logits the lower index has the larger key.  Each lane keeps its best remaining key; a
+// round is a warp max over those (5 shuffles) and only the winning lane rescans its slots.
+// Integer compares make the selection exact; the softmax over the k selected logits
+// (relative to the largest) is fp32.
+#pragma once
+
+#include "common.cuh"
+
+namespace nvfp4moe {
+
+__device__ __forceinline__ uint64_t topk_key(float v, int idx) {
+  uint32_t u = __float_as_uint(v + 0.0f);  // -0 + +0 = +0 under round-to-nearest
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return (uint64_t(u) << 32) | uint32_t(0xFFFF - idx);
+}
+
+__device__ __forceinline__ int topk_key_index(uint64_t key) { return 0xFFFF - int(uint32_t(key) & 0xFFFFu); }
+
+// Selects the top k (k <= 32) of l[0..E) for the calling warp.  Lane j < k returns the j-th
+// expert in *id and its softmax weight in *w.
+template <int PER_LANE>
+__device__ __forceinline__ void warp_topk(const float* __restrict__ l, int E, int k, int* id, float* w) {
+  const int lane = threadIdx.x & 31;
+  uint64_t key[PER_LANE];
+#pragma unroll
+  for (int i = 0; i < PER_LANE; ++i) {
+    const int e = lane + 32 * i;
+    key[i] = e < E ? topk_key(l[e], e) : 0ull;  // 0 marks an absent or taken slot
+  }
+  uint64_t mine = 0;
+#pragma unroll
+  for (int i = 0; i < PER_LANE; ++i) mine = key[i] > mine ? key[i] : mine;
+  uint64_t sel = 0;  // lane j keeps the j-th selected key
+  for (int j = 0; j < k; ++j) {
+    uint64_t best = mine;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const uint64_t other = __shfl_xor_sync(0xffffffffu, best, o);
+      best = other > best ? other : best;
+    }
+    if (lane == j) sel = best;
+    if (best == mine) {  // this lane owned the winner (keys are unique): drop it, rescan
+      mine = 0;
+#pragma unroll
+      for (int i = 0; i < PER_LANE; ++i) {
+        if (key[i] == best) key[i] = 0;
+        mine = key[i] > mine ? key[i] : mine;
+      }
+    }
+  }
+  const int bi = topk_key_index(sel);
+  const float sel_v = lane < k ? l[bi] : 0.0f;
+  const float l0 = __shfl_sync(0xffffffffu, sel_v, 0);
+  const float ex = lane < k ? expf(sel_v - l0) : 0.0f;
+  float sum = ex;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  *id = bi;
+  *w = ex / sum;
+}
+
+}  // namespace nvfp4moe
