@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <string>
+#include <utility>
 
 #include "../../include/nvfp4moe.h"
 
@@ -37,6 +38,42 @@ inline int num_sms() {
 }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------- programmatic dependent launch ----
+// A kernel launched with launch_dependent() may start while the previous kernel on the stream
+// is still running: it must call griddep_wait() before touching that kernel's output, and
+// griddep_wait() returns once the previous grid has completed and its writes are visible.
+// griddep_launch_dependents() lets the next such launch start early (its blocks still only
+// get SMs that are free).  Both are no-ops for kernels launched the ordinary way.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Records a timing mark on stream s.  Under stream capture the record must be an external
+// event node to stay a timing point of the graph; outside capture that flag is not allowed.
+inline cudaError_t record_mark(void* event, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(s, &cs);
+  if (e != cudaSuccess) return e;
+  cudaEvent_t ev = static_cast<cudaEvent_t>(event);
+  return cs == cudaStreamCaptureStatusActive ? cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal)
+                                              : cudaEventRecord(ev, s);
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                             Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // ---------------------------------------------------------- element codec ----
 // Two fp32 -> two E2M1 codes, round to nearest even, saturating (hardware cvt).

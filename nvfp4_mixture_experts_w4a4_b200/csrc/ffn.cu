@@ -139,10 +139,12 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int T = d->T, H = d->H, I = d->I, E = d->E, k = d->top_k;
   const int64_t rows_cap = moe_permute_rows_capacity(T, E, k, L.m_tile);
+  nvfp4moe_status mark_st = NVFP4MOE_OK;
   auto mark = [&](int i) {
-    // external records, so the marks become timing nodes when the stream is being captured
-    if (d->stage_events) cudaEventRecordWithFlags(reinterpret_cast<cudaEvent_t>(d->stage_events[i]), s,
-                                                  cudaEventRecordExternal);
+    if (d->stage_events && mark_st == NVFP4MOE_OK) {
+      const cudaError_t e = record_mark(d->stage_events[i], s);
+      if (e != cudaSuccess) mark_st = fail(NVFP4MOE_CUDA_ERROR, "%s: stage mark %d: %s", fn, i, cudaGetErrorString(e));
+    }
   };
 
   const bool dyn = d->x_scale_mode == NVFP4MOE_SCALE_DYNAMIC;
@@ -203,7 +205,7 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
     st = launch_combine(F32(L.slots), dn.slot_stride, dn.ksplit, I32(L.pair_to_row), T, H, k, out, s);
     if (st != NVFP4MOE_OK) return st;
     mark(6);
-    return NVFP4MOE_OK;
+    return mark_st;
   }
 
   // tensor-core path: x quantised once per token (into the slot region, which is free until
@@ -237,7 +239,7 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   st = launch_combine_bf16(ws + L.slots, I32(L.pair_to_row), T, H, k, out, s);
   if (st != NVFP4MOE_OK) return st;
   mark(6);
-  return NVFP4MOE_OK;
+  return mark_st;
 }
 
 }  // extern "C"

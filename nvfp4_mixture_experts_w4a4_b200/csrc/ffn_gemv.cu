@@ -209,6 +209,7 @@ __global__ void combine_kernel(const float* __restrict__ slots, int64_t slot_str
 // Same as combine_kernel over bf16 slot rows: 8 outputs per thread, eight slots in flight.
 __global__ void combine_bf16_kernel(const __nv_bfloat16* __restrict__ slots, const int32_t* __restrict__ pair_to_row,
                                     int T, int H, int k, __nv_bfloat16* __restrict__ out) {
+  griddep_wait();  // the slot rows come from the down GEMM launched just before
   const int64_t per_row = H / 8;
   const int64_t total = int64_t(T) * per_row;
   for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total;
@@ -359,8 +360,10 @@ nvfp4moe_status launch_combine_bf16(const void* slots, const int32_t* pair_to_ro
   if (total == 0) return NVFP4MOE_OK;
   int64_t blocks = (total + 255) / 256;
   if (blocks > int64_t(num_sms()) * 16) blocks = int64_t(num_sms()) * 16;
-  combine_bf16_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(slots), pair_to_row,
-                                                              T, H, k, static_cast<__nv_bfloat16*>(out));
+  const cudaError_t e = launch_dependent(combine_bf16_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s,
+                                         static_cast<const __nv_bfloat16*>(slots), pair_to_row, T, H, k,
+                                         static_cast<__nv_bfloat16*>(out));
+  if (e != cudaSuccess) return fail(NVFP4MOE_CUDA_ERROR, "combine: %s", cudaGetErrorString(e));
   return check_launch("combine");
 }
 

@@ -40,6 +40,8 @@ constexpr uint32_t kDevTimeout = 1u << 3;
 constexpr int TR_STRIDE = 17;   // h transpose tile: 32 tokens x 16 (+1) floats
 constexpr int TR_FLOATS = 32 * TR_STRIDE;
 constexpr int SFB_PER_KB = 8;   // TMEM columns of token scales per k-block (two atoms)
+constexpr int SCHED_CAP = 1264; // work items of one CTA kept as a list (over the per-expert arrays)
+constexpr int SCHED_PER_THREAD = (SCHED_CAP + 64 + 32 * 8 - 1) / (64 + 32 * 8);
 
 // Tile configuration: BNMAX tokens per tile at most, STAGES shared-memory stages.
 //   <192, 4> general; <64, 6> when no expert can hold more than 64 tokens (T <= 64), which
@@ -70,9 +72,9 @@ enum { EPI_GATEUP = 0, EPI_DOWN = 1 };
 struct GroupedParams {
   int K;             // reduction size
   int NW;            // weight rows per expert
+  int E;
   const int32_t* counts;
   const int32_t* padded_offsets;
-  const int32_t* active;
   const int32_t* row_pair;
   const uint8_t* x_sf;   // token scales, MMA layout over the padded permuted rows
   const uint8_t* w_sf;   // per expert NW*K/16 bytes
@@ -97,16 +99,17 @@ struct Item {
 };
 
 // Work item idx -> (expert, weight tile, token chunk); every input comes from shared memory.
+// prefix[e] = items of the experts before e (experts without tokens add none).
 template <int BNMAX>
-__device__ __forceinline__ Item get_item(int idx, int na, const int* prefix, const int* s_e, const int* s_ch,
-                                         const int* s_off, const int* s_cnt) {
-  int lo = 0, hi = na;  // find a with prefix[a] <= idx < prefix[a+1]
+__device__ __forceinline__ Item get_item(int idx, int E, const int* prefix, const int* s_ch, const int* s_off,
+                                         const int* s_cnt) {
+  int lo = 0, hi = E;  // the last e with prefix[e] <= idx, which has prefix[e+1] > idx
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if (prefix[mid] <= idx) lo = mid; else hi = mid;
   }
   Item it;
-  it.e = s_e[lo];
+  it.e = lo;
   const int ch = s_ch[lo];
   const int rem = idx - prefix[lo];
   it.mt = rem / ch;
@@ -140,24 +143,15 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   int* prefix = reinterpret_cast<int*>(tmem_holder + 4);  // [MAX_E + 1]
-  int* s_e = prefix + MAX_E + 1;                           // [MAX_E]
-  int* s_ch = s_e + MAX_E;                                 // [MAX_E]
+  int* s_wsum = prefix + MAX_E + 1;                        // [8] scan partials (room for MAX_E)
+  int* s_ch = s_wsum + MAX_E;                              // [MAX_E]
   int* s_off = s_ch + MAX_E;                               // [MAX_E] first padded row
   int* s_cnt = s_off + MAX_E;                              // [MAX_E] rows
   float* s_tr = reinterpret_cast<float*>(s_cnt + MAX_E);   // [EPI_WARPS][TR_FLOATS]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int na = p.active[0];
+  const int E = p.E;
   const int wtiles = p.NW / WM;
-  // per active expert: chunks of <= C::BNMAX tokens, and the number of work items before it
-  for (int a = threadIdx.x; a < na; a += kThreads) {
-    const int e = p.active[1 + a];
-    const int c = p.counts[e];
-    s_e[a] = e;
-    s_cnt[a] = c;
-    s_off[a] = p.padded_offsets[e];
-    s_ch[a] = (c + C::BNMAX - 1) / C::BNMAX;
-  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -180,28 +174,93 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
     prefetch_tensormap(&tmX);
     prefetch_tensormap(&tmXs);
   }
-  __syncthreads();
-  if (warp == 2) {  // exclusive scan of items per active expert
-    int carry = 0;
-    for (int base = 0; base < na; base += 32) {
-      const int a = base + lane;
-      const int v = a < na ? s_ch[a] * wtiles : 0;
-      int sum = v;
+  // The expert counts and offsets come from the permutation.  Gate/up waits for the kernel
+  // before it (the permutation, or the copy of x into expert order) and only then lets the
+  // down launch start, so the down kernel may read the counts before its own wait.
+  if (EPI == EPI_GATEUP) griddep_wait();
+  griddep_launch_dependents();
+  // counts and first padded rows of all experts, every load in flight at once; thread t < 256
+  // owns experts 4t .. 4t+3, whose item counts (chunks x weight tiles) one block scan sums
+  int tot = 0, nit[4];
+  if (threadIdx.x < MAX_E / 4) {
+    int c[4], o[4];
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, sum, o);
-        if (lane >= o) sum += y;
-      }
-      if (a < na) prefix[a] = carry + sum - v;
-      carry += __shfl_sync(0xffffffffu, sum, 31);
+    for (int i = 0; i < 4; ++i) {
+      const int e = 4 * int(threadIdx.x) + i;
+      c[i] = e < E ? __ldcg(p.counts + e) : 0;
+      o[i] = e < E ? __ldcg(p.padded_offsets + e) : 0;
     }
-    if (lane == 0) prefix[na] = carry;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = 4 * int(threadIdx.x) + i;
+      const int ch = (c[i] + C::BNMAX - 1) / C::BNMAX;
+      nit[i] = ch * wtiles;
+      tot += nit[i];
+      if (e < E) {
+        s_cnt[e] = c[i];
+        s_off[e] = o[i];
+        s_ch[e] = ch;
+      }
+    }
+  }
+  int incl = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31 && warp < MAX_E / 128) s_wsum[warp] = incl;
+  __syncthreads();
+  if (threadIdx.x < MAX_E / 4) {
+    int run = incl - tot;
+    for (int w = 0; w < warp; ++w) run += s_wsum[w];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = 4 * int(threadIdx.x) + i;
+      if (e <= E) prefix[e] = run;
+      run += nit[i];
+    }
+    if (threadIdx.x == MAX_E / 4 - 1 && E == MAX_E) prefix[E] = run;
+  }
+  __syncthreads();
+  // This CTA's items are blockIdx.x + j * gridDim.x.  Each thread resolves a few of them now,
+  // in parallel, and the list replaces the per-expert arrays, so that every role then reads
+  // one 16-byte entry per item instead of searching the expert prefix sums.
+  const int total = prefix[E];
+  const int n_my = total > int(blockIdx.x) ? (total - int(blockIdx.x) + int(gridDim.x) - 1) / int(gridDim.x) : 0;
+  const bool sched = n_my <= SCHED_CAP;
+  int4* s_items = reinterpret_cast<int4*>((reinterpret_cast<uintptr_t>(prefix) + 15) & ~uintptr_t(15));
+  if (sched) {
+    int4 mine[SCHED_PER_THREAD];
+#pragma unroll
+    for (int q = 0; q < SCHED_PER_THREAD; ++q) {
+      const int j = threadIdx.x + q * kThreads;
+      if (j < n_my) {
+        const Item w = get_item<C::BNMAX>(int(blockIdx.x) + j * int(gridDim.x), E, prefix, s_ch, s_off, s_cnt);
+        mine[q] = make_int4(w.e, w.mt, w.r0, w.n_rows);
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < SCHED_PER_THREAD; ++q) {
+      const int j = threadIdx.x + q * kThreads;
+      if (j < n_my) s_items[j] = mine[q];
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const int total = prefix[na];
+  auto item_at = [&](int j) -> Item {
+    if (sched) {
+      const int4 v = s_items[j];
+      Item w;
+      w.e = v.x; w.mt = v.y; w.r0 = v.z; w.n_rows = v.w;
+      w.N = (v.w + NQ - 1) / NQ * NQ;
+      return w;
+    }
+    return get_item<C::BNMAX>(int(blockIdx.x) + j * int(gridDim.x), E, prefix, s_ch, s_off, s_cnt);
+  };
   const int k_tiles = (p.K + BK - 1) / BK;
   const int64_t katoms = p.K / 64;
   auto abort_now = [&]() {
@@ -212,35 +271,56 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
   if (warp == 0) {
     // ------------------------------------------------------------ producer ----
     if (elect_one()) {
+      // Down: the weight half of the first ring pass (A tiles and their scales) does not
+      // depend on the gate/up kernel, which may still be finishing, so it goes out before the
+      // dependency wait; the token half follows after it.
+      uint32_t pre = 0;
+      if constexpr (EPI == EPI_DOWN) {
+        for (int j = 0; j < n_my && pre < uint32_t(C::STAGES); ++j) {
+          const Item w = item_at(j);
+          const uint8_t* wsf = p.w_sf + int64_t(w.e) * p.NW * (p.K / 16);
+          const int natoms = (w.r0 + w.N - 1) / 128 - w.r0 / 128 + 1;
+          for (int kt = 0; kt < k_tiles && pre < uint32_t(C::STAGES); ++kt, ++pre) {
+            const uint32_t sfb = min(4, (p.K - kt * BK) / 64) * 512;
+            mbar_arrive_expect_tx(&full[pre], C::A_BYTES + w.N * KB + sfb * (1 + natoms));
+            tma_load_2d(sA + pre * C::A_BYTES, &tmW, kt * KB, w.e * p.NW + w.mt * WM, &full[pre]);
+            bulk_load(sSFA + pre * C::SFA_BYTES, wsf + (int64_t(w.mt) * katoms + kt * 4) * 512, sfb, &full[pre]);
+          }
+        }
+        griddep_wait();
+      }
       uint32_t it = 0;
-      for (int idx = blockIdx.x; idx < total && !*abort_flag; idx += gridDim.x) {
-        const Item w = get_item<C::BNMAX>(idx, na, prefix, s_e, s_ch, s_off, s_cnt);
+      for (int j = 0; j < n_my && !*abort_flag; ++j) {
+        const Item w = item_at(j);
         const uint8_t* wsf = p.w_sf + int64_t(w.e) * p.NW * (p.K / 16);
         const int a0 = w.r0 / 128;
         const int natoms = (w.r0 + w.N - 1) / 128 - a0 + 1;
         for (int kt = 0; kt < k_tiles; ++kt, ++it) {
           const int s = it % C::STAGES;
-          if (!mbar_wait(&empty[s], ((it / C::STAGES) & 1) ^ 1)) {
-            abort_now();
-            break;
-          }
           const int nkb = min(4, (p.K - kt * BK) / 64);
           const uint32_t sfb = nkb * 512;
-          mbar_arrive_expect_tx(&full[s], C::A_BYTES + w.N * KB + sfb * (1 + natoms));
-          tma_load_2d(sA + s * C::A_BYTES, &tmW, kt * KB, w.e * p.NW + w.mt * WM, &full[s]);
+          if (it >= pre) {
+            if (!mbar_wait(&empty[s], ((it / C::STAGES) & 1) ^ 1)) {
+              abort_now();
+              break;
+            }
+            mbar_arrive_expect_tx(&full[s], C::A_BYTES + w.N * KB + sfb * (1 + natoms));
+            tma_load_2d(sA + s * C::A_BYTES, &tmW, kt * KB, w.e * p.NW + w.mt * WM, &full[s]);
+            bulk_load(sSFA + s * C::SFA_BYTES, wsf + (int64_t(w.mt) * katoms + kt * 4) * 512, sfb, &full[s]);
+          }
           int b = 0;
           for (; b + TOK_ALIGN <= w.N; b += TOK_ALIGN)
             tma_load_2d(sB + s * C::B_BYTES + b * KB, &tmX, kt * KB, w.r0 + b, &full[s]);
           for (; b < w.N; b += NQ) tma_load_2d(sB + s * C::B_BYTES + b * KB, &tmXs, kt * KB, w.r0 + b, &full[s]);
-          bulk_load(sSFA + s * C::SFA_BYTES, wsf + (int64_t(w.mt) * katoms + kt * 4) * 512, sfb, &full[s]);
           for (int ar = 0; ar < natoms; ++ar)
             bulk_load(sSFB + s * C::SFB_BYTES + ar * 2048, p.x_sf + (int64_t(a0 + ar) * katoms + kt * 4) * 512, sfb,
                       &full[s]);
         }
       }
       if (*abort_flag) {
-        for (uint32_t back = 0; back < C::STAGES && back < it; ++back) {
-          const uint32_t j = it - 1 - back;
+        const uint32_t issued = it > pre ? it : pre;
+        for (uint32_t back = 0; back < C::STAGES && back < issued; ++back) {
+          const uint32_t j = issued - 1 - back;
           mbar_wait(&full[j % C::STAGES], (j / C::STAGES) & 1, 1u << 16);
         }
       }
@@ -249,8 +329,8 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
     // ----------------------------------------------------------------- MMA ----
     if (elect_one()) {
       uint32_t it = 0, li = 0;
-      for (int idx = blockIdx.x; idx < total && !*abort_flag; idx += gridDim.x, ++li) {
-        const Item w = get_item<C::BNMAX>(idx, na, prefix, s_e, s_ch, s_off, s_cnt);
+      for (int j = 0; j < n_my && !*abort_flag; ++j, ++li) {
+        const Item w = item_at(j);
         const uint32_t ab = li & 1;
         if (!mbar_wait(&acc_empty[ab], ((li >> 1) & 1) ^ 1)) {
           abort_now();
@@ -312,8 +392,8 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
     const uint32_t trow = tmem + (uint32_t(q * 32) << 16);
     float* tr = s_tr + (warp - 2) * TR_FLOATS;
     uint32_t li = 0;
-    for (int idx = blockIdx.x; idx < total && !*abort_flag; idx += gridDim.x, ++li) {
-      const Item w = get_item<C::BNMAX>(idx, na, prefix, s_e, s_ch, s_off, s_cnt);
+    for (int j = 0; j < n_my && !*abort_flag; ++j, ++li) {
+      const Item w = item_at(j);
       const uint32_t ab = li & 1;
       const int wrow = w.mt * WM + q * 32 + lane;  // this lane's weight row inside the expert
       // per-item data, fetched before the accumulator is ready so its latency is hidden
@@ -425,7 +505,9 @@ nvfp4moe_status launch_cfg(const CUtensorMap& w, const CUtensorMap& x, const CUt
   }
   int64_t grid = num_sms();
   if (max_items < grid) grid = max_items > 0 ? max_items : 1;
-  kern<<<static_cast<int>(grid), kThreads, C::SMEM_BYTES, s>>>(w, x, xs, p);
+  const cudaError_t e = launch_dependent(kern, dim3(static_cast<unsigned>(grid)), dim3(kThreads), C::SMEM_BYTES, s,
+                                         w, x, xs, p);
+  if (e != cudaSuccess) return fail(NVFP4MOE_CUDA_ERROR, "grouped tcgen05 GEMM: %s", cudaGetErrorString(e));
   return check_launch("grouped tcgen05 GEMM");
 }
 
@@ -454,9 +536,9 @@ nvfp4moe_status launch_grouped_ffn(const GemmFfnArgs& a, cudaStream_t s) {
   const bool decode = a.T <= CfgDecode::BNMAX;
   CUtensorMap tw, tx, txs;
   GroupedParams p{};
+  p.E = a.E;
   p.counts = a.counts;
   p.padded_offsets = a.padded_offsets;
-  p.active = a.active;
   p.row_pair = a.row_pair;
   p.status = status;
   // gate/up: weights W13 [E*2I][H], tokens x [rows_cap][H]
@@ -479,8 +561,10 @@ nvfp4moe_status launch_grouped_ffn(const GemmFfnArgs& a, cudaStream_t s) {
   p.I = a.I;
   st = launch<EPI_GATEUP>(decode, tw, tx, txs, p, a.T, P, a.E, s);
   if (st != NVFP4MOE_OK) return st;
-  if (a.stage_events)
-    cudaEventRecordWithFlags(reinterpret_cast<cudaEvent_t>(a.stage_events[4]), s, cudaEventRecordExternal);
+  if (a.stage_events) {
+    const cudaError_t e = record_mark(a.stage_events[4], s);
+    if (e != cudaSuccess) return fail(NVFP4MOE_CUDA_ERROR, "stage mark 4: %s", cudaGetErrorString(e));
+  }
   // down: weights W2 [E*H][I], tokens h [rows_cap][I]
   st = make_code_map(&tw, a.w2_codes, int64_t(a.E) * a.H, a.I, WM);
   if (st != NVFP4MOE_OK) return st;

@@ -84,6 +84,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1) 
   const int gi = c * kThreads + tid;
   constexpr int kAll = kCluster * kThreads;
 
+  griddep_launch_dependents();  // the grouped GEMM may take the other SMs and set itself up
   // every CTA must have started before any writes into its shared memory
   cluster_arrive_relaxed();
   for (int e = tid; e < E; e += kThreads) s_mask[e] = 0ull;

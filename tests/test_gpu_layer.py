@@ -106,3 +106,38 @@ def test_weights_quantised_on_gpu_match_oracle():
     got = [ex.w13_codes, ex.w13_sf, ex.w13_scale, ex.w2_codes, ex.w2_sf, ex.w2_scale]
     for r, g in zip(ref, got):
         assert np.array_equal(g.cpu().numpy(), r)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name", ["tiny", "prefill_chunk_small"])
+def test_stage_marks_eager_and_in_a_cuda_graph(name):
+    """Stage marks work on an eager call and inside a captured CUDA graph (where they are
+    external event nodes), and neither the marks nor graph replay change the output."""
+    wl = GEMM_CASES.get(name) or CASES[name]
+    ref, out, layer, _ = G.run_layer_pair(wl, C.PATH_AUTO)
+    dev = out.device
+    act, *_ = G.layer_inputs(wl, 0)
+    x, logits = act["x"].to(dev), act["logits"].to(dev)
+    marks = [torch.cuda.Event(enable_timing=True) for _ in range(C.STAGES)]
+    eager = layer(x, logits, stage_events=marks)
+    torch.cuda.synchronize()
+    assert torch.equal(eager, out)
+    times = [marks[i].elapsed_time(marks[i + 1]) for i in range(C.STAGES - 1)]
+    assert all(t >= 0.0 for t in times) and sum(times) > 0.0
+
+    graph_out = torch.empty_like(out)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        layer(x, logits, out=graph_out)
+        side.synchronize()
+        with torch.cuda.graph(g, stream=side):
+            layer(x, logits, out=graph_out, stage_events=marks)
+    torch.cuda.current_stream().wait_stream(side)
+    graph_out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(graph_out, out)
+    times = [marks[i].elapsed_time(marks[i + 1]) for i in range(C.STAGES - 1)]
+    assert all(t >= 0.0 for t in times) and sum(times) > 0.0
