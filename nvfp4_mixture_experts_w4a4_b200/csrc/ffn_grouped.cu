@@ -39,6 +39,8 @@ constexpr int MAX_E = 1024;
 constexpr uint32_t kDevTimeout = 1u << 3;
 constexpr int TR_STRIDE = 17;   // h transpose tile: 32 tokens x 16 (+1) floats
 constexpr int TR_FLOATS = 32 * TR_STRIDE;
+constexpr int DOWN_TR_STRIDE = 33;  // down transpose tile: 16 tokens x 32 (+1) floats
+static_assert(16 * DOWN_TR_STRIDE <= TR_FLOATS, "down tile fits the transpose buffer");
 constexpr int SFB_PER_KB = 8;   // TMEM columns of token scales per k-block (two atoms)
 constexpr int SCHED_CAP = 1264; // work items of one CTA kept as a list (over the per-expert arrays)
 constexpr int SCHED_PER_THREAD = (SCHED_CAP + 64 + 32 * 8 - 1) / (64 + 32 * 8);
@@ -463,6 +465,11 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
           if (lane == 0 && amax_all > 0.0f) atomicMax(reinterpret_cast<int*>(p.h_amax + w.e), __float_as_int(amax_all));
         }
       } else {
+        // Each 32-token chunk goes through the warp's transpose tile in two halves of 16 tokens:
+        // lanes (= weight rows) park their 16 accumulators, then lane l takes token l & 15 and
+        // rows 16 * (l >> 4) .. +16, scales them by that token's routing weight and writes one
+        // 32-byte sector of its slot row.
+        const int tl = lane & 15, rh = lane >> 4;
 #pragma unroll
         for (int c2 = 0; c2 < C::MAX_CHUNKS / 2; ++c2) {
           const int cc = 2 * c2 + half;
@@ -471,12 +478,38 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
           tmem_ld_32x32b_x32(trow + ab * C::ACC_COLS + cc * 32, r);
           tmem_ld_wait();
           const int nj = min(32, w.n_rows - cc * 32);
+          if (nj <= 8) {
+            // a few tokens (decode): each token's 32 rows are one 64-byte store of the warp
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            if (j >= nj) break;
-            const int32_t pair = __shfl_sync(0xffffffffu, pr[c2], j);
-            const float wj = __shfl_sync(0xffffffffu, wt[c2], j);
-            if (pair >= 0) p.slots[int64_t(pair) * p.H + wrow] = __float2bfloat16_rn(__uint_as_float(r[j]) * wj);
+            for (int j = 0; j < 8; ++j) {
+              if (j >= nj) break;
+              const int32_t pair = __shfl_sync(0xffffffffu, pr[c2], j);
+              const float wj = __shfl_sync(0xffffffffu, wt[c2], j);
+              if (pair >= 0) p.slots[int64_t(pair) * p.H + wrow] = __float2bfloat16_rn(__uint_as_float(r[j]) * wj);
+            }
+            continue;
+          }
+#pragma unroll
+          for (int sub = 0; sub < 2; ++sub) {
+            if (sub * 16 >= nj) break;
+#pragma unroll
+            for (int t = 0; t < 16; ++t) tr[t * DOWN_TR_STRIDE + lane] = __uint_as_float(r[sub * 16 + t]);
+            __syncwarp();
+            const int32_t pair = __shfl_sync(0xffffffffu, pr[c2], sub * 16 + tl);
+            const float wj = __shfl_sync(0xffffffffu, wt[c2], sub * 16 + tl);
+            uint32_t packed[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float* src = tr + tl * DOWN_TR_STRIDE + rh * 16 + 2 * i;
+              const __nv_bfloat162 b2 = __floats2bfloat162_rn(src[0] * wj, src[1] * wj);
+              packed[i] = *reinterpret_cast<const uint32_t*>(&b2);
+            }
+            __syncwarp();
+            if (pair >= 0) {
+              uint4* dst = reinterpret_cast<uint4*>(p.slots + int64_t(pair) * p.H + w.mt * WM + q * 32 + rh * 16);
+              dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+              dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+            }
           }
         }
       }
