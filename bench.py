@@ -231,6 +231,41 @@ def kernel_nodes(g) -> int | None:
         return None
 
 
+def measured_traffic(workload: str):
+    """DRAM bytes per launch of the gate/up kernel from the committed ncu capture of this
+    workload, or None when there is none or the kernel source changed since it was taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
+            rec = json.load(f).get(workload)
+        src = os.path.join(ROOT, "nvfp4_mixture_experts_w4a4_b200", "csrc", "ffn_grouped.cu")
+        with open(src, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("source_sha256") != digest:
+        return None
+    return rec["dram_read_bytes"] + rec["dram_write_bytes"]
+
+
+def max_over_ranks(x: float) -> float:
+    """The max of a per-rank time over all ranks (identity without a process group).  Uses a
+    CPU tensor under gloo and a device tensor under nccl."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return x
+    dev = "cpu" if torch.distributed.get_backend() == "gloo" else torch.device("cuda", torch.cuda.current_device())
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(total_ms_max: float, steps: int, world: int, tokens_per_rank: int):
+    """(ms per step, whole-job tokens/s): every rank processes its own batch of tokens_per_rank
+    tokens per step, and the job's step time is the slowest rank's."""
+    ms_per_step = total_ms_max / steps
+    return ms_per_step, world * tokens_per_rank / (ms_per_step * 1e-3)
+
+
 def time_steps(layer, act, steps: int, warmup: int, flush: L2Flush, dist_on: bool):
     """Device time of K layer passes, each a replay of the captured forward between CUDA
     events on the replay stream, L2 flushed before each; then K more replays of a capture that
@@ -425,19 +460,10 @@ def main():
     flush = L2Flush(dev)
     with ClockSampler(local) as clk:
         step_ms, stage_ms, launches = time_steps(layer, act, args.steps, args.warmup, flush, dist_on)
-    total_ms = sum(step_ms)
-    if dist_on:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
-    ms_per_step = total_ms / args.steps
-    value = world * wl.T / (ms_per_step * 1e-3)
+    ms_per_step, value = job_throughput(max_over_ranks(sum(step_ms)), args.steps, world, wl.T)
 
     e2e_ms, h2d, d2h = time_e2e(layer, act, args.steps, args.warmup, flush)
-    if dist_on:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms)
 
     im = layer.intermediates(wl.T)
     n_active = int(im["active"][0].item())
@@ -448,7 +474,7 @@ def main():
     roof = roofline(alg["gate_up_bytes"], alg["gate_up_flops"], dom_ms, pk)
     roof.update({"kernel": ("gate_up tcgen05 grouped GEMM + SwiGLU + requant" if gemm_path
                             else "gate_up GEMV + SwiGLU + requant"),
-                 "traffic": None, "peak_source": pk["source"] + (" (fp4 = bf16 burst x 4)" if roof["bound"] == "tensor"
+                 "traffic": measured_traffic(wl.name) if gemm_path else None, "peak_source": pk["source"] + (" (fp4 = bf16 burst x 4)" if roof["bound"] == "tensor"
                                                                 else ""),
                  "algorithmic_bytes_per_launch": alg["gate_up_bytes"],
                  "algorithmic_flops_per_launch": alg["gate_up_flops"], "touched_experts": n_active,
