@@ -78,10 +78,13 @@ void make_layout(const moe_ffn_desc* d, moe_ffn_ws_layout* L) {
   L->h_sf = take(sf_mma_bytes(L->h_rows, I));
   // per-slot rows of the down projection: fp32 split-K partials on the GEMV path, bf16 on
   // the tensor-core path (halves the slot round trip of large prefills)
-  if (path == NVFP4MOE_PATH_GEMM)  // also holds x quantised per token until the down GEMM
-    L->slots = take(std::max<int64_t>(P * H * 2, ((T * H / 2 + 255) / 256) * 256 + sf_mma_bytes(T, H)));
+  // (the region also holds the batch prologue's slice histograms until the down GEMM)
+  const int64_t prologue_scratch = batch_prologue_scratch_bytes(d->T, d->E);
+  if (path == NVFP4MOE_PATH_GEMM)
+    L->slots = take(std::max<int64_t>(P * H * 2, prologue_scratch));
   else
-    L->slots = take(int64_t(gemv_down_ksplit(max_active_experts(d), H, I)) * P * H * 4);
+    L->slots = take(std::max<int64_t>(int64_t(gemv_down_ksplit(max_active_experts(d), H, I)) * P * H * 4,
+                                      prologue_scratch));
   L->total = o;
 }
 
@@ -149,7 +152,6 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
 
   const bool dyn = d->x_scale_mode == NVFP4MOE_SCALE_DYNAMIC;
   float* xs = dyn ? F32(L.x_scale) : const_cast<float*>(d->x_scale);
-  const size_t qws = nvfp4_quantize_workspace_size(1, T, H);
   const bool fused = prologue_fits(T, E, k);
 
   mark(0);
@@ -163,23 +165,17 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
     mark(1);
     mark(2);
   } else {
-    st = moe_route(logits, T, E, k, I32(L.topk_ids), F32(L.topk_w), stream);
+    // larger batch: slices of 32 tokens; x is quantised straight into its rows
+    st = launch_batch_prologue(x, logits, T, H, E, k, L.m_tile, dyn ? 1 : 0, xs, I32(L.topk_ids), F32(L.topk_w),
+                               I32(L.counts), I32(L.offsets), I32(L.padded_offsets), I32(L.pair_to_row),
+                               I32(L.row_token), I32(L.row_pair), I32(L.tile_expert), I32(L.active), d->h_amax,
+                               L.path == NVFP4MOE_PATH_GEMM ? 1 : 0, ws + L.x_codes, ws + L.x_sf, ws + L.slots,
+                               d->stage_events, s);
     if (st != NVFP4MOE_OK) return st;
-    mark(1);
-    st = moe_permute(I32(L.topk_ids), T, E, k, L.m_tile, rows_cap, I32(L.counts), I32(L.offsets),
-                     I32(L.padded_offsets), I32(L.pair_to_row), I32(L.row_token), I32(L.row_pair),
-                     I32(L.tile_expert), I32(L.active), d->h_amax, stream);
-    if (st != NVFP4MOE_OK) return st;
-    mark(2);
   }
 
   if (L.path == NVFP4MOE_PATH_GEMV) {
     // x quantised once per token, token-major
-    if (!fused) {
-      st = nvfp4_quantize(x, NVFP4MOE_DTYPE_BF16, 1, T, H, H, 0, nullptr, T, d->x_scale_mode, xs, ws + L.x_codes, 0,
-                          ws + L.x_sf, 0, NVFP4MOE_SF_MMA, ws + L.amax_partials, qws, stream);
-      if (st != NVFP4MOE_OK) return st;
-    }
     mark(3);
     GemvGateUpArgs g;
     g.H = H; g.I = I;
@@ -208,18 +204,6 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
     return mark_st;
   }
 
-  // tensor-core path: x quantised once per token (into the slot region, which is free until
-  // the down GEMM), then copied into the padded expert-order rows
-  if (!fused) {
-    uint8_t* xt_codes = ws + L.slots;
-    uint8_t* xt_sf = xt_codes + ((int64_t(T) * H / 2 + 255) / 256) * 256;
-    st = nvfp4_quantize(x, NVFP4MOE_DTYPE_BF16, 1, T, H, H, 0, nullptr, T, d->x_scale_mode, xs, xt_codes, 0, xt_sf,
-                        0, NVFP4MOE_SF_MMA, ws + L.amax_partials, qws, stream);
-    if (st != NVFP4MOE_OK) return st;
-    st = launch_replicate_rows(xt_codes, xt_sf, I32(L.row_token), I32(L.padded_offsets) + E, rows_cap, T, H,
-                               ws + L.x_codes, ws + L.x_sf, s);
-    if (st != NVFP4MOE_OK) return st;
-  }
   mark(3);
   GemmFfnArgs a;
   a.T = T; a.H = H; a.I = I; a.E = E; a.k = k;

@@ -23,6 +23,7 @@ CASES = {
     "long_prefill_small": W.scaled(W.WORKLOADS["long_prefill"], T=67, E=16, H=768, I=320, k=4),
     "dense_small": W.scaled(W.WORKLOADS["dense"], T=9, H=512, I=576),
     "top1_E2": W.scaled(TINY, T=13, E=2, k=1),
+    "slices_E1024_k32": W.scaled(TINY, T=70, E=1024, k=32, H=256, I=128),
 }
 
 
@@ -36,6 +37,7 @@ GEMM_CASES = {
     "decode_shape": W.scaled(W.WORKLOADS["decode"], E=64, H=1024, I=256),
     "decode_T1": W.scaled(W.WORKLOADS["decode"], T=1, E=64, H=1024, I=256),
     "popular_expert_chunks": W.scaled(W.WORKLOADS["prefill_chunk"], T=450, E=16, H=512, I=128, k=2),
+    "slices_E1024_k32": W.scaled(TINY, T=97, E=1024, k=32, H=256, I=128),
 }
 
 
