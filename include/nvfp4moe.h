@@ -91,7 +91,7 @@ enum {
 /* Message for the last failing call on this host thread ("" if none). */
 const char* nvfp4moe_last_error(void);
 
-/* Library version, e.g. 0x000100 = 0.1.0. */
+/* Library version, e.g. 0x000200 = 0.2.0. */
 int32_t nvfp4moe_version(void);
 
 /* Waits for `stream`, then returns the sticky device status word of the current device
@@ -250,6 +250,8 @@ typedef struct {
       amax_partials, total;
   int64_t x_rows;   /* rows of x_codes / x_sf (T on the GEMV path, rows_cap otherwise) */
   int64_t h_rows;   /* rows of h_codes / h_sf */
+  int64_t items;    /* small batches on the GEMM path: the grouped GEMMs' work lists, written by
+                       the routing step (int4 entries; see csrc/ffn_grouped.cu); else unused */
   int32_t m_tile;   /* 1 on the GEMV path, 64 on the GEMM path */
   int32_t path;     /* resolved path */
 } moe_ffn_ws_layout;

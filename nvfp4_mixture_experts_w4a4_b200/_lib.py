@@ -51,7 +51,7 @@ class MoeFfnWsLayout(ctypes.Structure):
     _fields_ = [(n, _i64) for n in (
         "topk_ids", "topk_w", "counts", "offsets", "padded_offsets", "pair_to_row", "row_token",
         "row_pair", "tile_expert", "active", "x_scale", "x_codes", "x_sf", "h_codes", "h_sf",
-        "slots", "amax_partials", "total", "x_rows", "h_rows")] + [("m_tile", _i32), ("path", _i32)]
+        "slots", "amax_partials", "total", "x_rows", "h_rows", "items")] + [("m_tile", _i32), ("path", _i32)]
 
 
 # name -> (restype, argtypes)

@@ -94,6 +94,8 @@ struct GroupedParams {
   __nv_bfloat16* slots;
   int H;
   uint32_t* status;
+  const int4* list;  // nullable work list written by the routing step (entry 0: item count)
+  int64_t list_cap;  // items the list can hold
 };
 
 struct Item {
@@ -181,72 +183,93 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
   // down launch start, so the down kernel may read the counts before its own wait.
   if (EPI == EPI_GATEUP) griddep_wait();
   griddep_launch_dependents();
-  // counts and first padded rows of all experts, every load in flight at once; thread t < 256
-  // owns experts 4t .. 4t+3, whose item counts (chunks x weight tiles) one block scan sums
-  int tot = 0, nit[4];
-  if (threadIdx.x < MAX_E / 4) {
-    int c[4], o[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int e = 4 * int(threadIdx.x) + i;
-      c[i] = e < E ? __ldcg(p.counts + e) : 0;
-      o[i] = e < E ? __ldcg(p.padded_offsets + e) : 0;
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int e = 4 * int(threadIdx.x) + i;
-      const int ch = (c[i] + C::BNMAX - 1) / C::BNMAX;
-      nit[i] = ch * wtiles;
-      tot += nit[i];
-      if (e < E) {
-        s_cnt[e] = c[i];
-        s_off[e] = o[i];
-        s_ch[e] = ch;
-      }
-    }
-  }
-  int incl = tot;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31 && warp < MAX_E / 128) s_wsum[warp] = incl;
-  __syncthreads();
-  if (threadIdx.x < MAX_E / 4) {
-    int run = incl - tot;
-    for (int w = 0; w < warp; ++w) run += s_wsum[w];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int e = 4 * int(threadIdx.x) + i;
-      if (e <= E) prefix[e] = run;
-      run += nit[i];
-    }
-    if (threadIdx.x == MAX_E / 4 - 1 && E == MAX_E) prefix[E] = run;
-  }
-  __syncthreads();
-  // This CTA's items are blockIdx.x + j * gridDim.x.  Each thread resolves a few of them now,
-  // in parallel, and the list replaces the per-expert arrays, so that every role then reads
-  // one 16-byte entry per item instead of searching the expert prefix sums.
-  const int total = prefix[E];
-  const int n_my = total > int(blockIdx.x) ? (total - int(blockIdx.x) + int(gridDim.x) - 1) / int(gridDim.x) : 0;
-  const bool sched = n_my <= SCHED_CAP;
   int4* s_items = reinterpret_cast<int4*>((reinterpret_cast<uintptr_t>(prefix) + 15) & ~uintptr_t(15));
-  if (sched) {
+  int total = 0, n_my = 0;
+  bool sched = true;
+  if (p.list) {
+    // The routing step wrote this GEMM's work list: its length and this CTA's entries arrive in
+    // one round trip (the host only passes a list whose per-CTA share fits SCHED_CAP).
     int4 mine[SCHED_PER_THREAD];
 #pragma unroll
     for (int q = 0; q < SCHED_PER_THREAD; ++q) {
       const int j = threadIdx.x + q * kThreads;
-      if (j < n_my) {
-        const Item w = get_item<C::BNMAX>(int(blockIdx.x) + j * int(gridDim.x), E, prefix, s_ch, s_off, s_cnt);
-        mine[q] = make_int4(w.e, w.mt, w.r0, w.n_rows);
-      }
+      const int64_t idx = int64_t(blockIdx.x) + int64_t(j) * gridDim.x;
+      mine[q] = (j < SCHED_CAP && idx < p.list_cap) ? __ldcg(p.list + 1 + idx) : make_int4(0, 0, 0, 0);
     }
-    __syncthreads();
+    total = __ldcg(p.list).x;
+    n_my = total > int(blockIdx.x) ? (total - int(blockIdx.x) + int(gridDim.x) - 1) / int(gridDim.x) : 0;
 #pragma unroll
     for (int q = 0; q < SCHED_PER_THREAD; ++q) {
       const int j = threadIdx.x + q * kThreads;
       if (j < n_my) s_items[j] = mine[q];
+    }
+  } else {
+    // counts and first padded rows of all experts, every load in flight at once; thread t < 256
+    // owns experts 4t .. 4t+3, whose item counts (chunks x weight tiles) one block scan sums
+    int tot = 0, nit[4];
+    if (threadIdx.x < MAX_E / 4) {
+      int c[4], o[4];
+  #pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int e = 4 * int(threadIdx.x) + i;
+        c[i] = e < E ? __ldcg(p.counts + e) : 0;
+        o[i] = e < E ? __ldcg(p.padded_offsets + e) : 0;
+      }
+  #pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int e = 4 * int(threadIdx.x) + i;
+        const int ch = (c[i] + C::BNMAX - 1) / C::BNMAX;
+        nit[i] = ch * wtiles;
+        tot += nit[i];
+        if (e < E) {
+          s_cnt[e] = c[i];
+          s_off[e] = o[i];
+          s_ch[e] = ch;
+        }
+      }
+    }
+    int incl = tot;
+  #pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31 && warp < MAX_E / 128) s_wsum[warp] = incl;
+    __syncthreads();
+    if (threadIdx.x < MAX_E / 4) {
+      int run = incl - tot;
+      for (int w = 0; w < warp; ++w) run += s_wsum[w];
+  #pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int e = 4 * int(threadIdx.x) + i;
+        if (e <= E) prefix[e] = run;
+        run += nit[i];
+      }
+      if (threadIdx.x == MAX_E / 4 - 1 && E == MAX_E) prefix[E] = run;
+    }
+    __syncthreads();
+    // This CTA's items are blockIdx.x + j * gridDim.x.  Each thread resolves a few of them now,
+    // in parallel, and the list replaces the per-expert arrays, so that every role then reads
+    // one 16-byte entry per item instead of searching the expert prefix sums.
+    total = prefix[E];
+    n_my = total > int(blockIdx.x) ? (total - int(blockIdx.x) + int(gridDim.x) - 1) / int(gridDim.x) : 0;
+    sched = n_my <= SCHED_CAP;
+    if (sched) {
+      int4 mine[SCHED_PER_THREAD];
+  #pragma unroll
+      for (int q = 0; q < SCHED_PER_THREAD; ++q) {
+        const int j = threadIdx.x + q * kThreads;
+        if (j < n_my) {
+          const Item w = get_item<C::BNMAX>(int(blockIdx.x) + j * int(gridDim.x), E, prefix, s_ch, s_off, s_cnt);
+          mine[q] = make_int4(w.e, w.mt, w.r0, w.n_rows);
+        }
+      }
+      __syncthreads();
+  #pragma unroll
+      for (int q = 0; q < SCHED_PER_THREAD; ++q) {
+        const int j = threadIdx.x + q * kThreads;
+        if (j < n_my) s_items[j] = mine[q];
+      }
     }
   }
   tc_fence_before();
@@ -546,12 +569,17 @@ nvfp4moe_status launch_cfg(const CUtensorMap& w, const CUtensorMap& x, const CUt
 
 template <int EPI>
 nvfp4moe_status launch(bool decode, const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& xs,
-                       const GroupedParams& p, int64_t max_rows_per_expert, int64_t P, int64_t E, cudaStream_t s) {
+                       GroupedParams p, const int4* list, int64_t list_cap, int64_t P, int64_t E, cudaStream_t s) {
   // upper bound of work items: every expert its chunks, weight tiles per chunk
   const int64_t bn = decode ? CfgDecode::BNMAX : CfgWide::BNMAX;
   const int64_t chunks = (P < E ? P : E) + P / bn + 1;
   const int64_t items = chunks * (p.NW / WM);
-  (void)max_rows_per_expert;
+  // a work list (one chunk per expert) matches the decode tiling; use it when every CTA's
+  // share of it fits the shared-memory list
+  const int64_t grid = items < num_sms() ? (items > 0 ? items : 1) : num_sms();
+  const bool use_list = decode && list != nullptr && (list_cap + grid - 1) / grid <= SCHED_CAP;
+  p.list = use_list ? list : nullptr;
+  p.list_cap = use_list ? list_cap : 0;
   if (decode) return launch_cfg<EPI, CfgDecode>(w, x, xs, p, items, s);
   return launch_cfg<EPI, CfgWide>(w, x, xs, p, items, s);
 }
@@ -592,7 +620,7 @@ nvfp4moe_status launch_grouped_ffn(const GemmFfnArgs& a, cudaStream_t s) {
   p.h_codes = a.h_codes;
   p.h_sf = a.h_sf;
   p.I = a.I;
-  st = launch<EPI_GATEUP>(decode, tw, tx, txs, p, a.T, P, a.E, s);
+  st = launch<EPI_GATEUP>(decode, tw, tx, txs, p, a.list_gateup, a.list_gateup_cap, P, a.E, s);
   if (st != NVFP4MOE_OK) return st;
   if (a.stage_events) {
     const cudaError_t e = record_mark(a.stage_events[4], s);
@@ -613,7 +641,7 @@ nvfp4moe_status launch_grouped_ffn(const GemmFfnArgs& a, cudaStream_t s) {
   p.topk_w = a.topk_w;
   p.slots = static_cast<__nv_bfloat16*>(a.slots_bf16);
   p.H = a.H;
-  return launch<EPI_DOWN>(decode, tw, tx, txs, p, a.T, P, a.E, s);
+  return launch<EPI_DOWN>(decode, tw, tx, txs, p, a.list_down, a.list_down_cap, P, a.E, s);
 }
 
 }  // namespace nvfp4moe

@@ -65,6 +65,9 @@ struct PrologueArgs {
   int expert_order;         // 1: x rows go to the padded expert-order rows; 0: token-major
   uint8_t* x_codes;
   uint8_t* x_sf;            // MMA layout
+  int4* list_gateup;        // nullable: work lists of the grouped GEMMs (one chunk per expert)
+  int4* list_down;
+  int wt_gateup, wt_down;   // weight tiles per expert of each
 };
 
 template <int PER_LANE>
@@ -74,6 +77,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1) 
   __shared__ unsigned long long s_mask[MAX_E];
   __shared__ int32_t s_cnt[MAX_E];
   __shared__ int32_t s_off[MAX_E + 1], s_poff[MAX_E + 1], s_aoff[MAX_E + 1];
+  __shared__ int32_t s_act[MAX_E];  // active slot -> expert
   __shared__ float s_part[kCluster];
   __shared__ unsigned long long s_wsum[kWarps];
   __shared__ float s_red[kWarps];
@@ -90,17 +94,31 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1) 
   for (int e = tid; e < E; e += kThreads) s_mask[e] = 0ull;
 
   // ---- 1. route this CTA's tokens; partial amax of x -------------------------------------
+  // The first x chunks are requested before the top-k so that both loads are in flight at once.
+  const int64_t chunks = a.dynamic ? int64_t(T) * H / 8 : 0;  // 16-byte chunks of x
+  const int64_t per = (chunks + kCluster - 1) / kCluster;
+  const int64_t lo = c * per, hi = min(chunks, lo + per);
+  const uint4* base = reinterpret_cast<const uint4*>(a.x);
+  uint4 first[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int64_t i = lo + tid + int64_t(j) * kThreads;
+    first[j] = i < hi ? __ldg(base + i) : make_uint4(0u, 0u, 0u, 0u);
+  }
   const int t = c + kCluster * warp;
   int my_id = 0;
   float my_w = 0.0f;
   if (t < T) warp_topk<PER_LANE>(a.logits + int64_t(t) * E, E, k, &my_id, &my_w);
   float m = 0.0f;
   if (a.dynamic) {
-    const int64_t chunks = int64_t(T) * H / 8;  // 16-byte chunks of x
-    const int64_t per = (chunks + kCluster - 1) / kCluster;
-    const int64_t lo = c * per, hi = min(chunks, lo + per);
-    const uint4* base = reinterpret_cast<const uint4*>(a.x);
-    for (int64_t i0 = lo + tid; i0 < hi; i0 += 4 * kThreads) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const uint32_t q[4] = {first[j].x, first[j].y, first[j].z, first[j].w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h)
+        m = fmaxf(m, fmaxf(fabsf(__uint_as_float(q[h] << 16)), fabsf(__uint_as_float(q[h] & 0xFFFF0000u))));
+    }
+    for (int64_t i0 = lo + tid + 2 * kThreads; i0 < hi; i0 += 4 * kThreads) {
       uint4 u[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -187,6 +205,9 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1) 
     const int tk = p / k;
     s_row[p] = s_poff[e] + __popcll(s_mask[e] & ((1ull << tk) - 1ull));
   }
+  if (a.list_gateup)
+    for (int e = tid; e < E; e += kThreads)
+      if (s_cnt[e] > 0) s_act[s_aoff[e]] = e;
   __syncthreads();
 
   // ---- 3. global writes, split over the cluster ------------------------------------------
@@ -218,20 +239,30 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1) 
     a.active[0] = s_aoff[E];
     if (a.dynamic) *a.x_scale = s_t;
   }
-  // padding rows and the tile -> expert map: row r belongs to the last expert whose
-  // padded offset is <= r
-  const int rows = s_poff[E];
-  for (int r = gi; r < rows; r += kAll) {
-    int lo = 0, hi = E - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (s_poff[mid] <= r) lo = mid; else hi = mid - 1;
+  if (a.list_gateup) {
+    // the grouped GEMMs' work lists: item (active expert, weight tile), chunk = all its tokens
+    const int na = s_aoff[E];
+    const int ng = na * a.wt_gateup, nd = na * a.wt_down;
+    if (gi == 0) {
+      a.list_gateup[0] = make_int4(ng, 0, 0, 0);
+      a.list_down[0] = make_int4(nd, 0, 0, 0);
     }
-    if (r - s_poff[lo] >= s_cnt[lo]) {
+    for (int i = gi; i < ng + nd; i += kAll) {
+      const bool g = i < ng;
+      const int idx = g ? i : i - ng;
+      const int wt = g ? a.wt_gateup : a.wt_down;
+      const int e = s_act[idx / wt];
+      (g ? a.list_gateup : a.list_down)[1 + idx] = make_int4(e, idx % wt, s_poff[e], s_cnt[e]);
+    }
+  }
+  // padding rows and the tile -> expert map: one warp of the cluster per expert at a time
+  for (int e = c * kWarps + warp; e < E; e += kCluster * kWarps) {
+    const int p0 = s_poff[e], p1 = s_poff[e + 1];
+    for (int r = p0 + s_cnt[e] + lane; r < p1; r += 32) {
       a.row_token[r] = -1;
       a.row_pair[r] = -1;
     }
-    if ((r & ((1 << a.m_tile_log2) - 1)) == 0) a.tile_expert[r >> a.m_tile_log2] = lo;
+    for (int tl = (p0 >> a.m_tile_log2) + lane; tl < (p1 >> a.m_tile_log2); tl += 32) a.tile_expert[tl] = e;
   }
 
   // quantise each 16-element block of x once; write it to its row(s)
@@ -271,7 +302,8 @@ nvfp4moe_status launch_prologue(const void* x, const float* logits, int T, int H
                                 int dynamic, float* x_scale, int32_t* ids, float* w, int32_t* counts, int32_t* offsets,
                                 int32_t* padded_offsets, int32_t* pair_to_row, int32_t* row_token, int32_t* row_pair,
                                 int32_t* tile_expert, int32_t* active, float* zero_f32, int expert_order,
-                                uint8_t* x_codes, uint8_t* x_sf, cudaStream_t s) {
+                                uint8_t* x_codes, uint8_t* x_sf, int4* list_gateup, int wt_gateup, int4* list_down,
+                                int wt_down, cudaStream_t s) {
   NVFP4_REQUIRE(prologue_fits(T, E, k), NVFP4MOE_UNSUPPORTED_SHAPE, "prologue: T=%d E=%d k=%d out of range", T, E, k);
   int lg = 0;
   while ((1 << lg) < m_tile) ++lg;
@@ -287,6 +319,8 @@ nvfp4moe_status launch_prologue(const void* x, const float* logits, int T, int H
   a.zero_f32 = zero_f32;
   a.expert_order = expert_order;
   a.x_codes = x_codes; a.x_sf = x_sf;
+  a.list_gateup = list_gateup; a.list_down = list_down;
+  a.wt_gateup = wt_gateup; a.wt_down = wt_down;
   const int per = (E + 31) / 32;
   if (per <= 1)
     prologue_kernel<1><<<kCluster, kThreads, 0, s>>>(a);

@@ -22,6 +22,12 @@ __device__ __forceinline__ uint64_t topk_key(float v, int idx) {
 
 __device__ __forceinline__ int topk_key_index(uint64_t key) { return 0xFFFF - int(uint32_t(key) & 0xFFFFu); }
 
+// The logit a key was built from (the order-preserving map inverted; -0 comes back as +0).
+__device__ __forceinline__ float topk_key_value(uint64_t key) {
+  const uint32_t u = uint32_t(key >> 32);
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
+}
+
 // Selects the top k (k <= 32) of l[0..E) for the calling warp.  Lane j < k returns the j-th
 // expert in *id and its softmax weight in *w.
 template <int PER_LANE>
@@ -55,7 +61,7 @@ __device__ __forceinline__ void warp_topk(const float* __restrict__ l, int E, in
     }
   }
   const int bi = topk_key_index(sel);
-  const float sel_v = lane < k ? l[bi] : 0.0f;
+  const float sel_v = lane < k ? topk_key_value(sel) : 0.0f;
   const float l0 = __shfl_sync(0xffffffffu, sel_v, 0);
   const float ex = lane < k ? expf(sel_v - l0) : 0.0f;
   float sum = ex;
