@@ -179,8 +179,10 @@ def algorithmic(wl: W.Workload, n_active: int, gemm_path: bool):
     gate_up_bytes = w13 + x_q + h_q
     layer_bytes = w13 + w2 + wl.T * wl.H * 2 * 2 + x_q + 2 * h_q + wl.T * wl.E * 4
     flops = 2.0 * P * 3 * wl.H * wl.I
+    # both GEMMs in one launch (small batches): weights, x and h codes, bf16 slot rows
+    gemms_bytes = w13 + w2 + x_q + 2 * h_q + P * wl.H * 2
     return {"gate_up_bytes": gate_up_bytes, "layer_bytes": layer_bytes, "flops": flops,
-            "gate_up_flops": 2.0 * P * 2 * wl.H * wl.I}
+            "gate_up_flops": 2.0 * P * 2 * wl.H * wl.I, "gemms_bytes": gemms_bytes}
 
 
 def roofline(bytes_, flops, ms, pk):
@@ -470,14 +472,21 @@ def main():
     gemm_path = im["path"] == C.PATH_GEMM
     alg = algorithmic(wl, n_active, gemm_path)
     pk = peaks()
+    # the dominant kernel: for batches of at most 64 tokens on the tensor-core path with H <= 2I
+    # both GEMMs run in one fused launch (its stage is "gate_up"); otherwise the gate/up GEMM
+    fused = gemm_path and wl.T <= 64 and wl.H <= 2 * wl.I
     dom_ms = stage_ms["gate_up"]
-    roof = roofline(alg["gate_up_bytes"], alg["gate_up_flops"], dom_ms, pk)
-    roof.update({"kernel": ("gate_up tcgen05 grouped GEMM + SwiGLU + requant" if gemm_path
-                            else "gate_up GEMV + SwiGLU + requant"),
-                 "traffic": measured_traffic(wl.name) if gemm_path else None, "peak_source": pk["source"] + (" (fp4 = bf16 burst x 4)" if roof["bound"] == "tensor"
-                                                                else ""),
-                 "algorithmic_bytes_per_launch": alg["gate_up_bytes"],
-                 "algorithmic_flops_per_launch": alg["gate_up_flops"], "touched_experts": n_active,
+    dom_bytes = alg["gemms_bytes"] if fused else alg["gate_up_bytes"]
+    dom_flops = alg["flops"] if fused else alg["gate_up_flops"]
+    roof = roofline(dom_bytes, dom_flops, dom_ms, pk)
+    kernel = ("fused gate/up + down tcgen05 grouped GEMM (SwiGLU + requant, weighted slots)" if fused
+              else "gate_up tcgen05 grouped GEMM + SwiGLU + requant" if gemm_path
+              else "gate_up GEMV + SwiGLU + requant")
+    roof.update({"kernel": kernel,
+                 "traffic": measured_traffic(wl.name) if gemm_path else None,
+                 "peak_source": pk["source"] + (" (fp4 = bf16 burst x 4)" if roof["bound"] == "tensor" else ""),
+                 "algorithmic_bytes_per_launch": dom_bytes,
+                 "algorithmic_flops_per_launch": dom_flops, "touched_experts": n_active,
                  "launch_ms": dom_ms})
     layer_roof = roofline(alg["layer_bytes"], alg["flops"], ms_per_step, pk)
     layer_bw = alg["layer_bytes"] / (ms_per_step * 1e-3) / 1e9

@@ -85,10 +85,10 @@ void make_layout(const moe_ffn_desc* d, moe_ffn_ws_layout* L) {
   else
     L->slots = take(std::max<int64_t>(int64_t(gemv_down_ksplit(max_active_experts(d), H, I)) * P * H * 4,
                                       prologue_scratch));
-  // work lists of the two grouped GEMMs, written by the small-batch prologue
+  // the fused GEMM's work list and per-expert counters, written by the small-batch prologue
   const int64_t A = P < E ? P : E;
   L->items = take(path == NVFP4MOE_PATH_GEMM && prologue_fits(d->T, d->E, d->top_k)
-                      ? (worklist_entries(A, 2 * I / 128) + worklist_entries(A, H / 128)) * 16
+                      ? grouped_fused_list_entries(A, 2 * I / 128, H / 128) * 16 + E * 4
                       : 0);
   L->total = o;
 }
@@ -161,8 +161,9 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   // small batches on the tensor-core path: the prologue also writes the GEMMs' work lists
   const bool lists = fused && L.path == NVFP4MOE_PATH_GEMM;
   const int64_t n_act = max_active_experts(d);
-  int4* list_g = reinterpret_cast<int4*>(ws + L.items);
-  int4* list_d = list_g + worklist_entries(n_act, 2 * I / 128);
+  const int64_t list_entries = grouped_fused_list_entries(n_act, 2 * I / 128, H / 128);
+  int4* list = reinterpret_cast<int4*>(ws + L.items);
+  int* done = reinterpret_cast<int*>(list + list_entries);
 
   mark(0);
   if (fused) {
@@ -170,8 +171,8 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
     st = launch_prologue(x, logits, T, H, E, k, L.m_tile, dyn ? 1 : 0, xs, I32(L.topk_ids), F32(L.topk_w),
                          I32(L.counts), I32(L.offsets), I32(L.padded_offsets), I32(L.pair_to_row), I32(L.row_token),
                          I32(L.row_pair), I32(L.tile_expert), I32(L.active), d->h_amax,
-                         L.path == NVFP4MOE_PATH_GEMM ? 1 : 0, ws + L.x_codes, ws + L.x_sf, lists ? list_g : nullptr,
-                         2 * I / 128, lists ? list_d : nullptr, H / 128, s);
+                         L.path == NVFP4MOE_PATH_GEMM ? 1 : 0, ws + L.x_codes, ws + L.x_sf, lists ? list : nullptr,
+                         lists ? done : nullptr, 2 * I / 128, H / 128, s);
     if (st != NVFP4MOE_OK) return st;
     mark(1);
     mark(2);
@@ -228,10 +229,9 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   a.h_codes = ws + L.h_codes; a.h_sf = ws + L.h_sf;
   a.topk_w = F32(L.topk_w); a.slots_bf16 = ws + L.slots;
   a.stage_events = d->stage_events;
-  a.list_gateup = lists ? list_g : nullptr;
-  a.list_down = lists ? list_d : nullptr;
-  a.list_gateup_cap = n_act * (2 * I / 128);
-  a.list_down_cap = n_act * (H / 128);
+  a.list = lists ? list : nullptr;
+  a.list_cap = list_entries - 1;
+  a.done = lists ? done : nullptr;
   st = launch_grouped_ffn(a, s);
   if (st != NVFP4MOE_OK) return st;
   mark(5);

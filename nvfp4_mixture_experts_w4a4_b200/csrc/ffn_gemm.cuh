@@ -5,10 +5,11 @@
 
 namespace nvfp4moe {
 
-// Work list of one grouped GEMM, written by the small-batch prologue (T <= 64, so every active
-// expert is one token chunk): entry 0 = {items, 0, 0, 0}; entry 1 + idx = {expert, weight tile,
-// first padded row, rows} of item idx, items ordered (active expert ascending, weight tile).
-inline int64_t worklist_entries(int64_t active_max, int64_t weight_tiles) { return 1 + active_max * weight_tiles; }
+// Work list of the fused decode GEMM, written by the small-batch prologue (T <= 64, so every
+// active expert is one token chunk): entry 0 = {gate/up items, down items, 0, 0}; then one entry
+// {expert, weight tile, first padded row, rows} per item: the gate/up items, then the down
+// items, each ordered (active expert ascending, weight tile).
+int64_t grouped_fused_list_entries(int64_t active_max, int64_t wt_gateup, int64_t wt_down);
 
 struct GemmFfnArgs {
   int T, H, I, E, k;
@@ -34,9 +35,9 @@ struct GemmFfnArgs {
   const float* topk_w;            // [T*k] by pair
   void* slots_bf16;               // [T*k][H] bf16, by pair
   void* const* stage_events;      // nullable; [4] is recorded between gate/up and down
-  const int4* list_gateup;        // nullable work lists (see worklist_entries) and their
-  const int4* list_down;          //   capacities in items
-  int64_t list_gateup_cap, list_down_cap;
+  const int4* list;               // nullable: the fused work list and the items it can hold
+  int64_t list_cap;
+  int* done;                      // with list: [E] gate/up completion counters, zeroed by its writer
 };
 
 bool gemm_path_available();

@@ -62,8 +62,8 @@ nvfp4moe_status launch_prologue(const void* x, const float* logits, int T, int H
                                 int dynamic, float* x_scale, int32_t* ids, float* w, int32_t* counts, int32_t* offsets,
                                 int32_t* padded_offsets, int32_t* pair_to_row, int32_t* row_token, int32_t* row_pair,
                                 int32_t* tile_expert, int32_t* active, float* zero_f32, int expert_order,
-                                uint8_t* x_codes, uint8_t* x_sf, int4* list_gateup, int wt_gateup, int4* list_down,
-                                int wt_down, cudaStream_t s);
+                                uint8_t* x_codes, uint8_t* x_sf, int4* list, int* done, int wt_gateup, int wt_down,
+                                cudaStream_t s);
 
 // Larger-batch prologue (route + permute + quantise x) over 32-token slices in three launches;
 // scratch: batch_prologue_scratch_bytes(T, E) bytes, free until the down GEMM; see

@@ -33,7 +33,8 @@ constexpr int NQ = 16;          // MMA N granularity and the small token box hei
 constexpr int BK = 256;
 constexpr int KB = BK / 2;
 constexpr int EPI_WARPS = 8;    // two per TMEM lane quarter
-constexpr int kThreads = 64 + 32 * EPI_WARPS;
+constexpr int TOKEN_WARP = 2 + EPI_WARPS;  // the producer of token tiles, after the epilogue warps
+constexpr int kThreads = 32 * (TOKEN_WARP + 1);
 constexpr uint32_t kTmemCols = 512;
 constexpr int MAX_E = 1024;
 constexpr uint32_t kDevTimeout = 1u << 3;
@@ -43,17 +44,20 @@ constexpr int DOWN_TR_STRIDE = 33;  // down transpose tile: 16 tokens x 32 (+1) 
 static_assert(16 * DOWN_TR_STRIDE <= TR_FLOATS, "down tile fits the transpose buffer");
 constexpr int SFB_PER_KB = 8;   // TMEM columns of token scales per k-block (two atoms)
 constexpr int SCHED_CAP = 1264; // work items of one CTA kept as a list (over the per-expert arrays)
-constexpr int SCHED_PER_THREAD = (SCHED_CAP + 64 + 32 * 8 - 1) / (64 + 32 * 8);
+constexpr int SCHED_PER_THREAD = (SCHED_CAP + kThreads - 1) / kThreads;
 
-// Tile configuration: BNMAX tokens per tile at most, STAGES shared-memory stages.
-//   <192, 4> general; <64, 6> when no expert can hold more than 64 tokens (T <= 64), which
-//   keeps more weight bytes in flight for the small decode tiles.
-template <int BN_, int STAGES_>
+// Tile configuration: BNMAX tokens per tile at most, STAGES shared-memory stages, NACC TMEM
+// accumulators.
+//   <192, 4, 2> general; <64, 6, 4> when no expert can hold more than 64 tokens (T <= 64): more
+//   weight bytes in flight for the small decode tiles, and the MMA may run three items ahead
+//   of a slow epilogue.
+template <int BN_, int STAGES_, int NACC_>
 struct Cfg {
   static constexpr int BNMAX = BN_;
   static constexpr int STAGES = STAGES_;
-  static constexpr int ACC_COLS = BNMAX;                 // two accumulators
-  static constexpr int SFA_COL = 2 * ACC_COLS;           // 16 columns
+  static constexpr int NACC = NACC_;                     // TMEM accumulators (items in flight)
+  static constexpr int ACC_COLS = BNMAX;
+  static constexpr int SFA_COL = NACC * ACC_COLS;        // 16 columns
   static constexpr int SFB_COL = SFA_COL + 16;           // 32 columns
   static constexpr int A_BYTES = WM * KB;                // 16 KB
   static constexpr int B_BYTES = BNMAX * KB;
@@ -61,25 +65,29 @@ struct Cfg {
   static constexpr int SFB_BYTES = 2 * 2048;             // up to two 128-row atom rows
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int SMEM_BYTES =
-      1024 + STAGES * STAGE_BYTES + (2 * STAGES + 5) * 8 + 16 + (5 * MAX_E + 1) * 4 + EPI_WARPS * TR_FLOATS * 4;
+      1024 + STAGES * STAGE_BYTES + (2 * STAGES + 2 * NACC + 1) * 8 + 16 + (5 * MAX_E + 1) * 4 +
+      EPI_WARPS * TR_FLOATS * 4;
   static constexpr int MAX_CHUNKS = BNMAX / 32;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(SFB_COL + 32 <= int(kTmemCols), "TMEM budget");
 };
-using CfgWide = Cfg<192, 4>;
-using CfgDecode = Cfg<64, 6>;
+using CfgWide = Cfg<192, 4, 2>;
+using CfgDecode = Cfg<64, 6, 4>;
 
-enum { EPI_GATEUP = 0, EPI_DOWN = 1 };
+// Modes: one GEMM per launch (gate/up or down), or both in one persistent launch (decode):
+// the CTAs work through gate/up items and then down items of one list, and a down item waits
+// only until every gate/up tile of its expert has written h (per-expert counters).
+enum { EPI_GATEUP = 0, EPI_DOWN = 1, EPI_FUSED = 2 };
 
 struct GroupedParams {
-  int K;             // reduction size
-  int NW;            // weight rows per expert
+  int K[2];          // reduction size, per phase (0 gate/up, 1 down)
+  int NW[2];         // weight rows per expert, per phase
+  const uint8_t* x_sf[2];  // token scales per phase (x, h), MMA layout over the padded rows
+  const uint8_t* w_sf[2];  // weight scales per phase, per expert NW*K/16 bytes
   int E;
   const int32_t* counts;
   const int32_t* padded_offsets;
   const int32_t* row_pair;
-  const uint8_t* x_sf;   // token scales, MMA layout over the padded permuted rows
-  const uint8_t* w_sf;   // per expert NW*K/16 bytes
   // gate/up
   const float* x_scale;
   const float* w13_scale;
@@ -94,12 +102,15 @@ struct GroupedParams {
   __nv_bfloat16* slots;
   int H;
   uint32_t* status;
-  const int4* list;  // nullable work list written by the routing step (entry 0: item count)
+  const int4* list;  // fused mode: work list written by the routing step (entry 0: {gate/up
+                     // items, down items}; then the gate/up items, then the down items)
   int64_t list_cap;  // items the list can hold
+  int* done;         // fused mode: per expert, epilogue warps that finished a gate/up tile
+  int done_target;   // EPI_WARPS x gate/up weight tiles
 };
 
 struct Item {
-  int e, mt, r0, n_rows, N;
+  int e, mt, r0, n_rows, N, ph;
 };
 
 // Work item idx -> (expert, weight tile, token chunk); every input comes from shared memory.
@@ -121,6 +132,7 @@ __device__ __forceinline__ Item get_item(int idx, int E, const int* prefix, cons
   it.r0 = s_off[lo] + c * BNMAX;
   it.n_rows = min(BNMAX, s_cnt[lo] - c * BNMAX);
   it.N = (it.n_rows + NQ - 1) / NQ * NQ;
+  it.ph = 0;
   return it;
 }
 
@@ -128,10 +140,35 @@ __device__ __forceinline__ Item get_item(int idx, int E, const int* prefix, cons
 // a few ulp here only move values that sit on a rounding boundary of the 4-bit grid).
 __device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
+// acquire load of a counter written by other CTAs (release side: fence + atomic add)
+__device__ __forceinline__ int ld_acquire(const int* ptr) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+  return v;
+}
+__device__ __forceinline__ int ld_relaxed(const int* ptr) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
 template <int EPI, class C>
 __global__ void __launch_bounds__(kThreads, 1)
-grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-               const __grid_constant__ CUtensorMap tmXs, GroupedParams p) {
+grouped_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__ CUtensorMap tmX0,
+               const __grid_constant__ CUtensorMap tmXs0, const __grid_constant__ CUtensorMap tmW1,
+               const __grid_constant__ CUtensorMap tmX1, const __grid_constant__ CUtensorMap tmXs1,
+               GroupedParams p) {
+  // the phase of a single-GEMM launch; fused launches take it from each item
+  constexpr int PH = EPI == EPI_DOWN ? 1 : 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -141,10 +178,10 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
   uint64_t* bars = reinterpret_cast<uint64_t*>(sSFB + C::STAGES * C::SFB_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + C::STAGES;
-  uint64_t* acc_full = bars + 2 * C::STAGES;   // [2]
-  uint64_t* acc_empty = acc_full + 2;       // [2]
-  uint64_t* drain = acc_full + 4;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 5);
+  uint64_t* acc_full = bars + 2 * C::STAGES;   // [NACC]
+  uint64_t* acc_empty = acc_full + C::NACC;    // [NACC]
+  uint64_t* drain = acc_empty + C::NACC;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   int* prefix = reinterpret_cast<int*>(tmem_holder + 4);  // [MAX_E + 1]
   int* s_wsum = prefix + MAX_E + 1;                        // [8] scan partials (room for MAX_E)
@@ -155,13 +192,13 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = p.E;
-  const int wtiles = p.NW / WM;
+  const int wtiles = p.NW[PH] / WM;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < C::NACC; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], EPI_WARPS * 32);
     }
@@ -174,34 +211,56 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tensormap(&tmW);
-    prefetch_tensormap(&tmX);
-    prefetch_tensormap(&tmXs);
+    if (EPI != EPI_DOWN) {
+      prefetch_tensormap(&tmW0);
+      prefetch_tensormap(&tmX0);
+      prefetch_tensormap(&tmXs0);
+    }
+    if (EPI != EPI_GATEUP) {
+      prefetch_tensormap(&tmW1);
+      prefetch_tensormap(&tmX1);
+      prefetch_tensormap(&tmXs1);
+    }
   }
   // The expert counts and offsets come from the permutation.  Gate/up waits for the kernel
   // before it (the permutation, or the copy of x into expert order) and only then lets the
   // down launch start, so the down kernel may read the counts before its own wait.
-  if (EPI == EPI_GATEUP) griddep_wait();
+  if (EPI != EPI_DOWN) griddep_wait();
   griddep_launch_dependents();
   int4* s_items = reinterpret_cast<int4*>((reinterpret_cast<uintptr_t>(prefix) + 15) & ~uintptr_t(15));
   int total = 0, n_my = 0;
   bool sched = true;
-  if (p.list) {
-    // The routing step wrote this GEMM's work list: its length and this CTA's entries arrive in
-    // one round trip (the host only passes a list whose per-CTA share fits SCHED_CAP).
+  if (p.list != nullptr) {
+    // The routing step wrote the work list (entry 0: {gate/up items, down items}, then the
+    // gate/up items, then the down items).  Gate/up and fused launches read their length and
+    // this CTA's entries in one round trip; a down launch first learns where its entries start.
+    // The host only passes the list when a CTA's share fits SCHED_CAP.  In a fused launch the
+    // entries past the gate/up items are down items; the phase goes into bit 30 of the tile.
+    int4 head = make_int4(0, 0, 0, 0);
+    int64_t base = 1;
+    if (EPI == EPI_DOWN) {
+      head = __ldcg(p.list);
+      base = 1 + head.x;
+    }
     int4 mine[SCHED_PER_THREAD];
 #pragma unroll
     for (int q = 0; q < SCHED_PER_THREAD; ++q) {
       const int j = threadIdx.x + q * kThreads;
       const int64_t idx = int64_t(blockIdx.x) + int64_t(j) * gridDim.x;
-      mine[q] = (j < SCHED_CAP && idx < p.list_cap) ? __ldcg(p.list + 1 + idx) : make_int4(0, 0, 0, 0);
+      mine[q] = (j < SCHED_CAP && idx < p.list_cap) ? __ldcg(p.list + base + idx) : make_int4(0, 0, 0, 0);
     }
-    total = __ldcg(p.list).x;
+    if (EPI != EPI_DOWN) head = __ldcg(p.list);
+    total = EPI == EPI_GATEUP ? head.x : EPI == EPI_DOWN ? head.y : head.x + head.y;
     n_my = total > int(blockIdx.x) ? (total - int(blockIdx.x) + int(gridDim.x) - 1) / int(gridDim.x) : 0;
 #pragma unroll
     for (int q = 0; q < SCHED_PER_THREAD; ++q) {
       const int j = threadIdx.x + q * kThreads;
-      if (j < n_my) s_items[j] = mine[q];
+      const int idx = int(blockIdx.x) + j * int(gridDim.x);
+      if (j < n_my) {
+        int4 v = mine[q];
+        if (EPI == EPI_FUSED) v.y |= int(idx >= head.x) << 30;
+        s_items[j] = v;
+      }
     }
   } else {
     // counts and first padded rows of all experts, every load in flight at once; thread t < 256
@@ -280,73 +339,122 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
     if (sched) {
       const int4 v = s_items[j];
       Item w;
-      w.e = v.x; w.mt = v.y; w.r0 = v.z; w.n_rows = v.w;
+      w.e = v.x; w.mt = v.y & 0xFFFF; w.r0 = v.z; w.n_rows = v.w;
       w.N = (v.w + NQ - 1) / NQ * NQ;
+      w.ph = EPI == EPI_FUSED ? (v.y >> 30) & 1 : PH;
       return w;
     }
-    return get_item<C::BNMAX>(int(blockIdx.x) + j * int(gridDim.x), E, prefix, s_ch, s_off, s_cnt);
+    Item w = get_item<C::BNMAX>(int(blockIdx.x) + j * int(gridDim.x), E, prefix, s_ch, s_off, s_cnt);
+    w.ph = PH;
+    return w;
   };
-  const int k_tiles = (p.K + BK - 1) / BK;
-  const int64_t katoms = p.K / 64;
+  auto k_tiles_of = [&](int ph) { return (p.K[ph] + BK - 1) / BK; };
   auto abort_now = [&]() {
     *abort_flag = 1;
     atomicOr(p.status, kDevTimeout);
   };
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer ----
+    // ----------------------------------------------------- producer: weights ----
+    // Weight tiles and their scales need nothing from earlier kernels (the item list was
+    // written before the preceding launch let this one start), so this warp never waits on
+    // them; it arms each stage with the bytes of both halves.
     if (elect_one()) {
-      // Down: the weight half of the first ring pass (A tiles and their scales) does not
-      // depend on the gate/up kernel, which may still be finishing, so it goes out before the
-      // dependency wait; the token half follows after it.
-      uint32_t pre = 0;
-      if constexpr (EPI == EPI_DOWN) {
-        for (int j = 0; j < n_my && pre < uint32_t(C::STAGES); ++j) {
-          const Item w = item_at(j);
-          const uint8_t* wsf = p.w_sf + int64_t(w.e) * p.NW * (p.K / 16);
-          const int natoms = (w.r0 + w.N - 1) / 128 - w.r0 / 128 + 1;
-          for (int kt = 0; kt < k_tiles && pre < uint32_t(C::STAGES); ++kt, ++pre) {
-            const uint32_t sfb = min(4, (p.K - kt * BK) / 64) * 512;
-            mbar_arrive_expect_tx(&full[pre], C::A_BYTES + w.N * KB + sfb * (1 + natoms));
-            tma_load_2d(sA + pre * C::A_BYTES, &tmW, kt * KB, w.e * p.NW + w.mt * WM, &full[pre]);
-            bulk_load(sSFA + pre * C::SFA_BYTES, wsf + (int64_t(w.mt) * katoms + kt * 4) * 512, sfb, &full[pre]);
-          }
-        }
-        griddep_wait();
-      }
       uint32_t it = 0;
       for (int j = 0; j < n_my && !*abort_flag; ++j) {
         const Item w = item_at(j);
-        const uint8_t* wsf = p.w_sf + int64_t(w.e) * p.NW * (p.K / 16);
+        const int ph = w.ph;
+        const int K = p.K[ph], NW = p.NW[ph], kt_n = k_tiles_of(ph);
+        const int64_t katoms = K / 64;
+        const CUtensorMap* mW = ph ? &tmW1 : &tmW0;
+        const uint8_t* wsf = p.w_sf[ph] + int64_t(w.e) * NW * (K / 16);
+        const int natoms = (w.r0 + w.N - 1) / 128 - w.r0 / 128 + 1;
+        for (int kt = 0; kt < kt_n; ++kt, ++it) {
+          const int s = it % C::STAGES;
+          const uint32_t sfb = min(4, (K - kt * BK) / 64) * 512;
+          if (!mbar_wait(&empty[s], ((it / C::STAGES) & 1) ^ 1)) {
+            abort_now();
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], C::A_BYTES + w.N * KB + sfb * (1 + natoms));
+          tma_load_2d(sA + s * C::A_BYTES, mW, kt * KB, w.e * NW + w.mt * WM, &full[s]);
+          bulk_load(sSFA + s * C::SFA_BYTES, wsf + (int64_t(w.mt) * katoms + kt * 4) * 512, sfb, &full[s]);
+        }
+      }
+      if (*abort_flag) {  // let the copies in flight land before the CTA exits
+        for (uint32_t back = 0; back < C::STAGES && back < it; ++back) {
+          const uint32_t jj = it - 1 - back;
+          mbar_wait(&full[jj % C::STAGES], (jj / C::STAGES) & 1, 1u << 16);
+        }
+      }
+    }
+  } else if (warp == TOKEN_WARP) {
+    // ------------------------------------------------------ producer: tokens ----
+    // Token tiles and their scales are the previous kernel's output (down: h), or, fused, the
+    // h rows that gate/up epilogues of this launch write: a down item's first stage waits until
+    // every gate/up epilogue warp of its expert has counted itself done.  The counters of this
+    // CTA's next down items are read in one round trip (relaxed loads, then one acquire fence)
+    // and kept as a bit mask.  The copies complete bytes on the stage barrier that the weight
+    // producer arms (a stage may receive them first).
+    if (elect_one()) {
+      if (EPI == EPI_DOWN) griddep_wait();
+      uint64_t ready = 0;
+      int ready_base = -1;
+      auto ensure_ready = [&](int j, int e) -> bool {
+        if (ready_base >= 0 && j >= ready_base && j < ready_base + 64 && ((ready >> (j - ready_base)) & 1)) return true;
+        ready_base = j;
+        ready = 0;
+        int v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = j + i < n_my ? ld_relaxed(p.done + item_at(j + i).e) : 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          if (j + i < n_my && v[i] >= p.done_target) ready |= 1ull << i;
+        fence_acq_rel_gpu();
+        if (!(ready & 1ull)) {
+          const uint64_t t0 = global_ns();
+          while (ld_acquire(p.done + e) < p.done_target)
+            if (global_ns() - t0 > 200000000ull) return false;  // 0.2 s: a gate/up tile never finished
+          ready |= 1ull;
+        }
+        fence_proxy_async_global();
+        return true;
+      };
+      uint32_t it = 0;
+      for (int j = 0; j < n_my && !*abort_flag; ++j) {
+        const Item w = item_at(j);
+        const int ph = w.ph;
+        const int K = p.K[ph], kt_n = k_tiles_of(ph);
+        const int64_t katoms = K / 64;
+        const CUtensorMap* mX = ph ? &tmX1 : &tmX0;
+        const CUtensorMap* mXs = ph ? &tmXs1 : &tmXs0;
+        const uint8_t* xsf = p.x_sf[ph];
         const int a0 = w.r0 / 128;
         const int natoms = (w.r0 + w.N - 1) / 128 - a0 + 1;
-        for (int kt = 0; kt < k_tiles; ++kt, ++it) {
+        if (EPI == EPI_FUSED && ph == 1 && !ensure_ready(j, w.e)) {
+          abort_now();
+          break;
+        }
+        for (int kt = 0; kt < kt_n; ++kt, ++it) {
           const int s = it % C::STAGES;
-          const int nkb = min(4, (p.K - kt * BK) / 64);
-          const uint32_t sfb = nkb * 512;
-          if (it >= pre) {
-            if (!mbar_wait(&empty[s], ((it / C::STAGES) & 1) ^ 1)) {
-              abort_now();
-              break;
-            }
-            mbar_arrive_expect_tx(&full[s], C::A_BYTES + w.N * KB + sfb * (1 + natoms));
-            tma_load_2d(sA + s * C::A_BYTES, &tmW, kt * KB, w.e * p.NW + w.mt * WM, &full[s]);
-            bulk_load(sSFA + s * C::SFA_BYTES, wsf + (int64_t(w.mt) * katoms + kt * 4) * 512, sfb, &full[s]);
+          const uint32_t sfb = min(4, (K - kt * BK) / 64) * 512;
+          if (!mbar_wait(&empty[s], ((it / C::STAGES) & 1) ^ 1)) {
+            abort_now();
+            break;
           }
           int b = 0;
           for (; b + TOK_ALIGN <= w.N; b += TOK_ALIGN)
-            tma_load_2d(sB + s * C::B_BYTES + b * KB, &tmX, kt * KB, w.r0 + b, &full[s]);
-          for (; b < w.N; b += NQ) tma_load_2d(sB + s * C::B_BYTES + b * KB, &tmXs, kt * KB, w.r0 + b, &full[s]);
+            tma_load_2d(sB + s * C::B_BYTES + b * KB, mX, kt * KB, w.r0 + b, &full[s]);
+          for (; b < w.N; b += NQ) tma_load_2d(sB + s * C::B_BYTES + b * KB, mXs, kt * KB, w.r0 + b, &full[s]);
           for (int ar = 0; ar < natoms; ++ar)
-            bulk_load(sSFB + s * C::SFB_BYTES + ar * 2048, p.x_sf + (int64_t(a0 + ar) * katoms + kt * 4) * 512, sfb,
+            bulk_load(sSFB + s * C::SFB_BYTES + ar * 2048, xsf + (int64_t(a0 + ar) * katoms + kt * 4) * 512, sfb,
                       &full[s]);
         }
       }
       if (*abort_flag) {
-        const uint32_t issued = it > pre ? it : pre;
-        for (uint32_t back = 0; back < C::STAGES && back < issued; ++back) {
-          const uint32_t j = issued - 1 - back;
-          mbar_wait(&full[j % C::STAGES], (j / C::STAGES) & 1, 1u << 16);
+        for (uint32_t back = 0; back < C::STAGES && back < it; ++back) {
+          const uint32_t jj = it - 1 - back;
+          mbar_wait(&full[jj % C::STAGES], (jj / C::STAGES) & 1, 1u << 16);
         }
       }
     }
@@ -356,8 +464,8 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
       uint32_t it = 0, li = 0;
       for (int j = 0; j < n_my && !*abort_flag; ++j, ++li) {
         const Item w = item_at(j);
-        const uint32_t ab = li & 1;
-        if (!mbar_wait(&acc_empty[ab], ((li >> 1) & 1) ^ 1)) {
+        const uint32_t ab = li % C::NACC;
+        if (!mbar_wait(&acc_empty[ab], ((li / C::NACC) & 1) ^ 1)) {
           abort_now();
           break;
         }
@@ -367,7 +475,8 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
         const uint32_t g0 = (w.r0 % 128) / 32;  // 0 or 2
         const uint32_t d_acc = tmem + ab * C::ACC_COLS;
         bool ok = true;
-        for (int kt = 0; kt < k_tiles; ++kt, ++it) {
+        const int kt_n = k_tiles_of(w.ph), K = p.K[w.ph];
+        for (int kt = 0; kt < kt_n; ++kt, ++it) {
           const int s = it % C::STAGES;
           if (!mbar_wait(&full[s], (it / C::STAGES) & 1)) {
             abort_now();
@@ -375,7 +484,7 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
             break;
           }
           tc_fence_after();
-          const int nkb = min(4, (p.K - kt * BK) / 64);
+          const int nkb = min(4, (K - kt * BK) / 64);
           // descriptor start addresses advance in 16-byte units: 512-byte atoms (32), 32 bytes of K (2)
           const uint64_t sfa_d = desc_sf_atom(sSFA + s * C::SFA_BYTES);
           const uint64_t sfb_d = desc_sf_atom(sSFB + s * C::SFB_BYTES);
@@ -417,15 +526,28 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
     const uint32_t trow = tmem + (uint32_t(q * 32) << 16);
     float* tr = s_tr + (warp - 2) * TR_FLOATS;
     uint32_t li = 0;
+    // Fused: this warp's h stores of a gate/up tile are counted for the expert's down items one
+    // item later (or at the end), so the fence that orders them before the count finds them
+    // drained instead of stalling the epilogue.
+    int pending = -1;
+    auto release_pending = [&]() {
+      if (EPI == EPI_FUSED && pending >= 0) {
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(p.done + pending, 1);
+        pending = -1;
+      }
+    };
     for (int j = 0; j < n_my && !*abort_flag; ++j, ++li) {
       const Item w = item_at(j);
-      const uint32_t ab = li & 1;
+      const uint32_t ab = li % C::NACC;
       const int wrow = w.mt * WM + q * 32 + lane;  // this lane's weight row inside the expert
       // per-item data, fetched before the accumulator is ready so its latency is hidden
       float sg = 0.f, su = 0.f, sh = 0.f, sc = 0.f;
       int32_t pr[C::MAX_CHUNKS / 2];
       float wt[C::MAX_CHUNKS / 2];
-      if constexpr (EPI == EPI_GATEUP) {
+      const bool gateup = EPI == EPI_FUSED ? w.ph == 0 : EPI == EPI_GATEUP;
+      if (gateup) {
         const float sx = p.x_scale[0];
         sg = sx * p.w13_scale[2 * w.e];
         su = sx * p.w13_scale[2 * w.e + 1];
@@ -440,12 +562,13 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
 #pragma unroll
         for (int c2 = 0; c2 < C::MAX_CHUNKS / 2; ++c2) wt[c2] = pr[c2] >= 0 ? p.topk_w[pr[c2]] * sc : 0.0f;
       }
-      if (!mbar_wait(&acc_full[ab], (li >> 1) & 1)) {
+      release_pending();
+      if (!mbar_wait(&acc_full[ab], (li / C::NACC) & 1)) {
         abort_now();
         break;
       }
       tc_fence_after();
-      if constexpr (EPI == EPI_GATEUP) {
+      if (gateup) {
         // lanes 0..15 hold gate rows i, lanes 16..31 the up rows i of one 16-wide block of h
         const int64_t iblk = wrow >> 5;
         float amax_all = 0.0f;
@@ -487,6 +610,7 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
           for (int o = 16; o > 0; o >>= 1) amax_all = fmaxf(amax_all, __shfl_xor_sync(0xffffffffu, amax_all, o));
           if (lane == 0 && amax_all > 0.0f) atomicMax(reinterpret_cast<int*>(p.h_amax + w.e), __float_as_int(amax_all));
         }
+        if (EPI == EPI_FUSED) pending = w.e;  // counted once its stores have drained
       } else {
         // Each 32-token chunk goes through the warp's transpose tile in two halves of 16 tokens:
         // lanes (= weight rows) park their 16 accumulators, then lane l takes token l & 15 and
@@ -539,6 +663,7 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
       tc_fence_before();
       mbar_arrive(&acc_empty[ab]);
     }
+    release_pending();
   }
 
   tc_fence_before();
@@ -547,9 +672,12 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
+struct Maps {
+  CUtensorMap w, x, xs;
+};
+
 template <int EPI, class C>
-nvfp4moe_status launch_cfg(const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& xs, const GroupedParams& p,
-                           int64_t max_items, cudaStream_t s) {
+nvfp4moe_status launch_cfg(const Maps& m0, const Maps& m1, const GroupedParams& p, int64_t max_items, cudaStream_t s) {
   auto kern = grouped_kernel<EPI, C>;
   static int configured[64] = {0};
   int dev = 0;
@@ -562,31 +690,23 @@ nvfp4moe_status launch_cfg(const CUtensorMap& w, const CUtensorMap& x, const CUt
   int64_t grid = num_sms();
   if (max_items < grid) grid = max_items > 0 ? max_items : 1;
   const cudaError_t e = launch_dependent(kern, dim3(static_cast<unsigned>(grid)), dim3(kThreads), C::SMEM_BYTES, s,
-                                         w, x, xs, p);
+                                         m0.w, m0.x, m0.xs, m1.w, m1.x, m1.xs, p);
   if (e != cudaSuccess) return fail(NVFP4MOE_CUDA_ERROR, "grouped tcgen05 GEMM: %s", cudaGetErrorString(e));
   return check_launch("grouped tcgen05 GEMM");
 }
 
-template <int EPI>
-nvfp4moe_status launch(bool decode, const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& xs,
-                       GroupedParams p, const int4* list, int64_t list_cap, int64_t P, int64_t E, cudaStream_t s) {
-  // upper bound of work items: every expert its chunks, weight tiles per chunk
-  const int64_t bn = decode ? CfgDecode::BNMAX : CfgWide::BNMAX;
-  const int64_t chunks = (P < E ? P : E) + P / bn + 1;
-  const int64_t items = chunks * (p.NW / WM);
-  // a work list (one chunk per expert) matches the decode tiling; use it when every CTA's
-  // share of it fits the shared-memory list
-  const int64_t grid = items < num_sms() ? (items > 0 ? items : 1) : num_sms();
-  const bool use_list = decode && list != nullptr && (list_cap + grid - 1) / grid <= SCHED_CAP;
-  p.list = use_list ? list : nullptr;
-  p.list_cap = use_list ? list_cap : 0;
-  if (decode) return launch_cfg<EPI, CfgDecode>(w, x, xs, p, items, s);
-  return launch_cfg<EPI, CfgWide>(w, x, xs, p, items, s);
+// upper bound of one GEMM's work items: every expert its token chunks, weight tiles per chunk
+int64_t max_items(int64_t P, int64_t E, int64_t bn, int64_t weight_tiles) {
+  return ((P < E ? P : E) + P / bn + 1) * weight_tiles;
 }
 
 }  // namespace
 
 int grouped_token_align() { return TOK_ALIGN; }
+
+int64_t grouped_fused_list_entries(int64_t active_max, int64_t wt_gateup, int64_t wt_down) {
+  return 1 + active_max * (wt_gateup + wt_down);
+}
 
 nvfp4moe_status launch_grouped_ffn(const GemmFfnArgs& a, cudaStream_t s) {
   uint32_t* status = device_status_ptr();
@@ -595,24 +715,30 @@ nvfp4moe_status launch_grouped_ffn(const GemmFfnArgs& a, cudaStream_t s) {
   const int64_t P = int64_t(a.T) * a.k;
   // no expert receives more than T tokens (a token names an expert at most once)
   const bool decode = a.T <= CfgDecode::BNMAX;
-  CUtensorMap tw, tx, txs;
+  const int wt_g = 2 * a.I / WM, wt_d = a.H / WM;
+  Maps g, d;
+  // gate/up: weights W13 [E*2I][H], tokens x [rows_cap][H]; down: W2 [E*H][I], tokens h [rows_cap][I]
+  nvfp4moe_status st = make_code_map(&g.w, a.w13_codes, int64_t(a.E) * 2 * a.I, a.H, WM);
+  if (st == NVFP4MOE_OK) st = make_code_map(&g.x, a.x_codes, a.rows_cap, a.H, TOK_ALIGN);
+  if (st == NVFP4MOE_OK) st = make_code_map(&g.xs, a.x_codes, a.rows_cap, a.H, NQ);
+  if (st == NVFP4MOE_OK) st = make_code_map(&d.w, a.w2_codes, int64_t(a.E) * a.H, a.I, WM);
+  if (st == NVFP4MOE_OK) st = make_code_map(&d.x, a.h_codes, a.rows_cap, a.I, TOK_ALIGN);
+  if (st == NVFP4MOE_OK) st = make_code_map(&d.xs, a.h_codes, a.rows_cap, a.I, NQ);
+  if (st != NVFP4MOE_OK) return st;
   GroupedParams p{};
   p.E = a.E;
   p.counts = a.counts;
   p.padded_offsets = a.padded_offsets;
   p.row_pair = a.row_pair;
   p.status = status;
-  // gate/up: weights W13 [E*2I][H], tokens x [rows_cap][H]
-  nvfp4moe_status st = make_code_map(&tw, a.w13_codes, int64_t(a.E) * 2 * a.I, a.H, WM);
-  if (st != NVFP4MOE_OK) return st;
-  st = make_code_map(&tx, a.x_codes, a.rows_cap, a.H, TOK_ALIGN);
-  if (st != NVFP4MOE_OK) return st;
-  st = make_code_map(&txs, a.x_codes, a.rows_cap, a.H, NQ);
-  if (st != NVFP4MOE_OK) return st;
-  p.K = a.H;
-  p.NW = 2 * a.I;
-  p.x_sf = a.x_sf;
-  p.w_sf = a.w13_sf;
+  p.K[0] = a.H;
+  p.NW[0] = 2 * a.I;
+  p.x_sf[0] = a.x_sf;
+  p.w_sf[0] = a.w13_sf;
+  p.K[1] = a.I;
+  p.NW[1] = a.H;
+  p.x_sf[1] = a.h_sf;
+  p.w_sf[1] = a.w2_sf;
   p.x_scale = a.x_scale;
   p.w13_scale = a.w13_scale;
   p.h_scale = a.h_scale;
@@ -620,28 +746,52 @@ nvfp4moe_status launch_grouped_ffn(const GemmFfnArgs& a, cudaStream_t s) {
   p.h_codes = a.h_codes;
   p.h_sf = a.h_sf;
   p.I = a.I;
-  st = launch<EPI_GATEUP>(decode, tw, tx, txs, p, a.list_gateup, a.list_gateup_cap, P, a.E, s);
-  if (st != NVFP4MOE_OK) return st;
-  if (a.stage_events) {
-    const cudaError_t e = record_mark(a.stage_events[4], s);
-    if (e != cudaSuccess) return fail(NVFP4MOE_CUDA_ERROR, "stage mark 4: %s", cudaGetErrorString(e));
-  }
-  // down: weights W2 [E*H][I], tokens h [rows_cap][I]
-  st = make_code_map(&tw, a.w2_codes, int64_t(a.E) * a.H, a.I, WM);
-  if (st != NVFP4MOE_OK) return st;
-  st = make_code_map(&tx, a.h_codes, a.rows_cap, a.I, TOK_ALIGN);
-  if (st != NVFP4MOE_OK) return st;
-  st = make_code_map(&txs, a.h_codes, a.rows_cap, a.I, NQ);
-  if (st != NVFP4MOE_OK) return st;
-  p.K = a.I;
-  p.NW = a.H;
-  p.x_sf = a.h_sf;
-  p.w_sf = a.w2_sf;
   p.w2_scale = a.w2_scale;
   p.topk_w = a.topk_w;
   p.slots = static_cast<__nv_bfloat16*>(a.slots_bf16);
   p.H = a.H;
-  return launch<EPI_DOWN>(decode, tw, tx, txs, p, a.list_down, a.list_down_cap, P, a.E, s);
+  auto mark4 = [&]() -> nvfp4moe_status {
+    if (!a.stage_events) return NVFP4MOE_OK;
+    const cudaError_t e = record_mark(a.stage_events[4], s);
+    return e == cudaSuccess ? NVFP4MOE_OK : fail(NVFP4MOE_CUDA_ERROR, "stage mark 4: %s", cudaGetErrorString(e));
+  };
+
+  // Decode batches with a work list from the routing step: both GEMMs in one launch, when
+  // every CTA's share of the list fits the shared-memory list.
+  const int64_t items_g = max_items(P, a.E, CfgDecode::BNMAX, wt_g), items_d = max_items(P, a.E, CfgDecode::BNMAX, wt_d);
+  const int64_t fused_items = items_g + items_d;
+  const int64_t fused_grid = fused_items < num_sms() ? fused_items : num_sms();
+  // One launch pays off when the down GEMM has no more weight tiles than gate/up (H <= 2I):
+  // then a second launch's ramp-up is not amortised.  Otherwise the down launch starts on the
+  // SMs that gate/up frees and streams its first weight tiles meanwhile.
+  const bool fits = [&](int64_t cap, int64_t grid) { return (cap + grid - 1) / grid <= SCHED_CAP; }(
+      a.list_cap, fused_grid);
+  if (decode && a.list != nullptr && a.done != nullptr && wt_d <= wt_g && fits) {
+    p.list = a.list;
+    p.list_cap = a.list_cap;
+    p.done = a.done;
+    p.done_target = EPI_WARPS * wt_g;
+    st = launch_cfg<EPI_FUSED, CfgDecode>(g, d, p, fused_items, s);
+    if (st != NVFP4MOE_OK) return st;
+    return mark4();  // one launch: the gate/up stage holds both GEMMs
+  }
+  if (decode) {
+    const int64_t cap_g = a.list_cap / (wt_g + wt_d) * wt_g, cap_d = a.list_cap - cap_g;
+    const int64_t grid_g = items_g < num_sms() ? items_g : num_sms(), grid_d = items_d < num_sms() ? items_d : num_sms();
+    const bool use = a.list != nullptr && (cap_g + grid_g - 1) / grid_g <= SCHED_CAP &&
+                     (cap_d + grid_d - 1) / grid_d <= SCHED_CAP;
+    p.list = use ? a.list : nullptr;
+    p.list_cap = cap_g;
+    st = launch_cfg<EPI_GATEUP, CfgDecode>(g, g, p, items_g, s);
+    if (st == NVFP4MOE_OK) st = mark4();
+    p.list_cap = cap_d;
+    if (st == NVFP4MOE_OK) st = launch_cfg<EPI_DOWN, CfgDecode>(d, d, p, items_d, s);
+    return st;
+  }
+  st = launch_cfg<EPI_GATEUP, CfgWide>(g, g, p, max_items(P, a.E, CfgWide::BNMAX, wt_g), s);
+  if (st == NVFP4MOE_OK) st = mark4();
+  if (st == NVFP4MOE_OK) st = launch_cfg<EPI_DOWN, CfgWide>(d, d, p, max_items(P, a.E, CfgWide::BNMAX, wt_d), s);
+  return st;
 }
 
 }  // namespace nvfp4moe

@@ -65,9 +65,9 @@ struct PrologueArgs {
   int expert_order;         // 1: x rows go to the padded expert-order rows; 0: token-major
   uint8_t* x_codes;
   uint8_t* x_sf;            // MMA layout
-  int4* list_gateup;        // nullable: work lists of the grouped GEMMs (one chunk per expert)
-  int4* list_down;
-  int wt_gateup, wt_down;   // weight tiles per expert of each
+  int4* list;               // nullable: the fused grouped GEMM's work list (one chunk per expert)
+  int* done;                //   and its per-expert counters, zeroed here
+  int wt_gateup, wt_down;   // weight tiles per expert of each GEMM
 };
 
 template <int PER_LANE>
@@ -205,7 +205,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1) 
     const int tk = p / k;
     s_row[p] = s_poff[e] + __popcll(s_mask[e] & ((1ull << tk) - 1ull));
   }
-  if (a.list_gateup)
+  if (a.list)
     for (int e = tid; e < E; e += kThreads)
       if (s_cnt[e] > 0) s_act[s_aoff[e]] = e;
   __syncthreads();
@@ -239,21 +239,20 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1) 
     a.active[0] = s_aoff[E];
     if (a.dynamic) *a.x_scale = s_t;
   }
-  if (a.list_gateup) {
-    // the grouped GEMMs' work lists: item (active expert, weight tile), chunk = all its tokens
+  if (a.list) {
+    // the fused GEMM's work list: gate/up items then down items, each (active expert, weight
+    // tile) with all the expert's tokens as one chunk; and its counters, zeroed
     const int na = s_aoff[E];
     const int ng = na * a.wt_gateup, nd = na * a.wt_down;
-    if (gi == 0) {
-      a.list_gateup[0] = make_int4(ng, 0, 0, 0);
-      a.list_down[0] = make_int4(nd, 0, 0, 0);
-    }
+    if (gi == 0) a.list[0] = make_int4(ng, nd, 0, 0);
     for (int i = gi; i < ng + nd; i += kAll) {
       const bool g = i < ng;
       const int idx = g ? i : i - ng;
       const int wt = g ? a.wt_gateup : a.wt_down;
       const int e = s_act[idx / wt];
-      (g ? a.list_gateup : a.list_down)[1 + idx] = make_int4(e, idx % wt, s_poff[e], s_cnt[e]);
+      a.list[1 + i] = make_int4(e, idx % wt, s_poff[e], s_cnt[e]);
     }
+    for (int e = gi; e < E; e += kAll) a.done[e] = 0;
   }
   // padding rows and the tile -> expert map: one warp of the cluster per expert at a time
   for (int e = c * kWarps + warp; e < E; e += kCluster * kWarps) {
@@ -302,8 +301,8 @@ nvfp4moe_status launch_prologue(const void* x, const float* logits, int T, int H
                                 int dynamic, float* x_scale, int32_t* ids, float* w, int32_t* counts, int32_t* offsets,
                                 int32_t* padded_offsets, int32_t* pair_to_row, int32_t* row_token, int32_t* row_pair,
                                 int32_t* tile_expert, int32_t* active, float* zero_f32, int expert_order,
-                                uint8_t* x_codes, uint8_t* x_sf, int4* list_gateup, int wt_gateup, int4* list_down,
-                                int wt_down, cudaStream_t s) {
+                                uint8_t* x_codes, uint8_t* x_sf, int4* list, int* done, int wt_gateup, int wt_down,
+                                cudaStream_t s) {
   NVFP4_REQUIRE(prologue_fits(T, E, k), NVFP4MOE_UNSUPPORTED_SHAPE, "prologue: T=%d E=%d k=%d out of range", T, E, k);
   int lg = 0;
   while ((1 << lg) < m_tile) ++lg;
@@ -319,7 +318,7 @@ nvfp4moe_status launch_prologue(const void* x, const float* logits, int T, int H
   a.zero_f32 = zero_f32;
   a.expert_order = expert_order;
   a.x_codes = x_codes; a.x_sf = x_sf;
-  a.list_gateup = list_gateup; a.list_down = list_down;
+  a.list = list; a.done = done;
   a.wt_gateup = wt_gateup; a.wt_down = wt_down;
   const int per = (E + 31) / 32;
   if (per <= 1)
