@@ -179,8 +179,8 @@ def algorithmic(wl: W.Workload, n_active: int, gemm_path: bool):
     gate_up_bytes = w13 + x_q + h_q
     layer_bytes = w13 + w2 + wl.T * wl.H * 2 * 2 + x_q + 2 * h_q + wl.T * wl.E * 4
     flops = 2.0 * P * 3 * wl.H * wl.I
-    # both GEMMs in one launch (small batches): weights, x and h codes, bf16 slot rows
-    gemms_bytes = w13 + w2 + x_q + 2 * h_q + P * wl.H * 2
+    # both GEMMs in one launch (small batches): weights, x and h codes, fp32 slot rows
+    gemms_bytes = w13 + w2 + x_q + 2 * h_q + P * wl.H * 4
     return {"gate_up_bytes": gate_up_bytes, "layer_bytes": layer_bytes, "flops": flops,
             "gate_up_flops": 2.0 * P * 2 * wl.H * wl.I, "gemms_bytes": gemms_bytes}
 

@@ -81,7 +81,7 @@ void make_layout(const moe_ffn_desc* d, moe_ffn_ws_layout* L) {
   // (the region also holds the batch prologue's slice histograms until the down GEMM)
   const int64_t prologue_scratch = batch_prologue_scratch_bytes(d->T, d->E);
   if (path == NVFP4MOE_PATH_GEMM)
-    L->slots = take(std::max<int64_t>(P * H * 2, prologue_scratch));
+    L->slots = take(std::max<int64_t>(P * H * 4, prologue_scratch));
   else
     L->slots = take(std::max<int64_t>(int64_t(gemv_down_ksplit(max_active_experts(d), H, I)) * P * H * 4,
                                       prologue_scratch));
@@ -227,7 +227,7 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   a.w2_codes = d->w2_codes; a.w2_sf = d->w2_sf; a.w2_scale = d->w2_scale;
   a.h_scale = d->h_scale; a.h_amax = d->h_amax;
   a.h_codes = ws + L.h_codes; a.h_sf = ws + L.h_sf;
-  a.topk_w = F32(L.topk_w); a.slots_bf16 = ws + L.slots;
+  a.topk_w = F32(L.topk_w); a.slots_f32 = ws + L.slots;
   a.stage_events = d->stage_events;
   a.list = lists ? list : nullptr;
   a.list_cap = list_entries - 1;
@@ -235,7 +235,7 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   st = launch_grouped_ffn(a, s);
   if (st != NVFP4MOE_OK) return st;
   mark(5);
-  st = launch_combine_bf16(ws + L.slots, I32(L.pair_to_row), T, H, k, out, s);
+  st = launch_combine(F32(L.slots), int64_t(T) * k * H, 1, I32(L.pair_to_row), T, H, k, out, s);
   if (st != NVFP4MOE_OK) return st;
   mark(6);
   return mark_st;

@@ -33,7 +33,7 @@ struct GemmFfnArgs {
   uint8_t* h_codes;               // [rows_cap][I/2]
   uint8_t* h_sf;                  // MMA layout over rows_cap rows
   const float* topk_w;            // [T*k] by pair
-  void* slots_bf16;               // [T*k][H] bf16, by pair
+  void* slots_f32;                // [T*k][H] fp32, by pair
   void* const* stage_events;      // nullable; [4] is recorded between gate/up and down
   const int4* list;               // nullable: the fused work list and the items it can hold
   int64_t list_cap;

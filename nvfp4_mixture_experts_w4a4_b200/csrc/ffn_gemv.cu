@@ -167,6 +167,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) gemv_down_kernel(GemvDownAr
 __global__ void combine_kernel(const float* __restrict__ slots, int64_t slot_stride, int ksplit,
                                const int32_t* __restrict__ pair_to_row, int T, int H, int k,
                                __nv_bfloat16* __restrict__ out) {
+  griddep_wait();  // the slot rows come from the down GEMM launched just before
   const int64_t per_row = H / 8;
   const int64_t total = int64_t(T) * per_row;
   for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total;
@@ -206,45 +207,6 @@ __global__ void combine_kernel(const float* __restrict__ slots, int64_t slot_str
   }
 }
 
-// Same as combine_kernel over bf16 slot rows: 8 outputs per thread, eight slots in flight.
-__global__ void combine_bf16_kernel(const __nv_bfloat16* __restrict__ slots, const int32_t* __restrict__ pair_to_row,
-                                    int T, int H, int k, __nv_bfloat16* __restrict__ out) {
-  griddep_wait();  // the slot rows come from the down GEMM launched just before
-  const int64_t per_row = H / 8;
-  const int64_t total = int64_t(T) * per_row;
-  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total;
-       i += int64_t(gridDim.x) * blockDim.x) {
-    const int64_t t = i / per_row, n = (i - t * per_row) * 8;
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int j0 = 0; j0 < k; j0 += 8) {
-      uint4 v[8];
-      bool ok[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) ok[u] = j0 + u < k && pair_to_row[t * k + j0 + u] >= 0;
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (ok[u]) v[u] = *reinterpret_cast<const uint4*>(slots + (t * k + j0 + u) * H + n);
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (ok[u]) {
-          const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            acc[2 * q] += __uint_as_float(w[q] << 16);
-            acc[2 * q + 1] += __uint_as_float(w[q] & 0xFFFF0000u);
-          }
-        }
-    }
-    uint4 o;
-    uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
-      ow[q] = *reinterpret_cast<const uint32_t*>(&b);
-    }
-    *reinterpret_cast<uint4*>(out + t * H + n) = o;
-  }
-}
 
 // Copies quantised token rows into the padded expert-order rows: codes (32 bytes) and the
 // 4-byte scale word of one 64-element group per thread; padding rows are left untouched.
@@ -337,8 +299,9 @@ nvfp4moe_status launch_combine(const float* slots, int64_t slot_stride, int kspl
   if (total == 0) return NVFP4MOE_OK;
   int64_t blocks = (total + 255) / 256;
   if (blocks > int64_t(num_sms()) * 8) blocks = int64_t(num_sms()) * 8;
-  combine_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(slots, slot_stride, ksplit, pair_to_row, T,
-                                                         H, k, static_cast<__nv_bfloat16*>(out));
+  const cudaError_t e = launch_dependent(combine_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, slots,
+                                         slot_stride, ksplit, pair_to_row, T, H, k, static_cast<__nv_bfloat16*>(out));
+  if (e != cudaSuccess) return fail(NVFP4MOE_CUDA_ERROR, "combine: %s", cudaGetErrorString(e));
   return check_launch("combine");
 }
 
@@ -354,17 +317,5 @@ nvfp4moe_status launch_replicate_rows(const uint8_t* codes_tok, const uint8_t* s
   return check_launch("replicate rows");
 }
 
-nvfp4moe_status launch_combine_bf16(const void* slots, const int32_t* pair_to_row, int T, int H, int k, void* out,
-                                    cudaStream_t s) {
-  const int64_t total = int64_t(T) * (H / 8);
-  if (total == 0) return NVFP4MOE_OK;
-  int64_t blocks = (total + 255) / 256;
-  if (blocks > int64_t(num_sms()) * 16) blocks = int64_t(num_sms()) * 16;
-  const cudaError_t e = launch_dependent(combine_bf16_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s,
-                                         static_cast<const __nv_bfloat16*>(slots), pair_to_row, T, H, k,
-                                         static_cast<__nv_bfloat16*>(out));
-  if (e != cudaSuccess) return fail(NVFP4MOE_CUDA_ERROR, "combine: %s", cudaGetErrorString(e));
-  return check_launch("combine");
-}
 
 }  // namespace nvfp4moe

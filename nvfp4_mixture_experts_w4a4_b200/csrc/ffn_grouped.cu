@@ -99,7 +99,7 @@ struct GroupedParams {
   // down
   const float* w2_scale;
   const float* topk_w;
-  __nv_bfloat16* slots;
+  float* slots;      // [T*k][H] fp32 rows, by pair
   int H;
   uint32_t* status;
   const int4* list;  // fused mode: work list written by the routing step (entry 0: {gate/up
@@ -614,8 +614,8 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__
       } else {
         // Each 32-token chunk goes through the warp's transpose tile in two halves of 16 tokens:
         // lanes (= weight rows) park their 16 accumulators, then lane l takes token l & 15 and
-        // rows 16 * (l >> 4) .. +16, scales them by that token's routing weight and writes one
-        // 32-byte sector of its slot row.
+        // rows 16 * (l >> 4) .. +16, scales them by that token's routing weight and writes those
+        // 64 contiguous bytes of its fp32 slot row.
         const int tl = lane & 15, rh = lane >> 4;
 #pragma unroll
         for (int c2 = 0; c2 < C::MAX_CHUNKS / 2; ++c2) {
@@ -632,7 +632,7 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__
               if (j >= nj) break;
               const int32_t pair = __shfl_sync(0xffffffffu, pr[c2], j);
               const float wj = __shfl_sync(0xffffffffu, wt[c2], j);
-              if (pair >= 0) p.slots[int64_t(pair) * p.H + wrow] = __float2bfloat16_rn(__uint_as_float(r[j]) * wj);
+              if (pair >= 0) p.slots[int64_t(pair) * p.H + wrow] = __uint_as_float(r[j]) * wj;
             }
             continue;
           }
@@ -644,18 +644,14 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__
             __syncwarp();
             const int32_t pair = __shfl_sync(0xffffffffu, pr[c2], sub * 16 + tl);
             const float wj = __shfl_sync(0xffffffffu, wt[c2], sub * 16 + tl);
-            uint32_t packed[8];
+            float v[16];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float* src = tr + tl * DOWN_TR_STRIDE + rh * 16 + 2 * i;
-              const __nv_bfloat162 b2 = __floats2bfloat162_rn(src[0] * wj, src[1] * wj);
-              packed[i] = *reinterpret_cast<const uint32_t*>(&b2);
-            }
+            for (int i = 0; i < 16; ++i) v[i] = tr[tl * DOWN_TR_STRIDE + rh * 16 + i] * wj;
             __syncwarp();
             if (pair >= 0) {
-              uint4* dst = reinterpret_cast<uint4*>(p.slots + int64_t(pair) * p.H + w.mt * WM + q * 32 + rh * 16);
-              dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-              dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+              float4* dst = reinterpret_cast<float4*>(p.slots + int64_t(pair) * p.H + w.mt * WM + q * 32 + rh * 16);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
             }
           }
         }
@@ -748,7 +744,7 @@ nvfp4moe_status launch_grouped_ffn(const GemmFfnArgs& a, cudaStream_t s) {
   p.I = a.I;
   p.w2_scale = a.w2_scale;
   p.topk_w = a.topk_w;
-  p.slots = static_cast<__nv_bfloat16*>(a.slots_bf16);
+  p.slots = static_cast<float*>(a.slots_f32);
   p.H = a.H;
   auto mark4 = [&]() -> nvfp4moe_status {
     if (!a.stage_events) return NVFP4MOE_OK;

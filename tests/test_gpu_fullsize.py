@@ -1,0 +1,117 @@
+"""Parity at the full sizes the benchmark times (gpu), on sampled tokens.
+
+The library runs each workload's whole batch on the device with the benchmark's settings
+(dynamic x scale, path chosen automatically, seeded draws of workloads.py).  The oracle
+computes, from the same fp32 weights and bf16 inputs and without anything from the device:
+  * the routing of every token and the permutation (bit-exact against the device's);
+  * the layer input's tensor scale over the whole batch (bit-exact);
+  * the NVFP4 codes of every expert the sampled tokens use (bit-exact against the device's
+    quantised weights);
+  * the sampled tokens' x codes, h codes and outputs, with per-expert h scales that it
+    calibrates on the sample and that the device then uses too.
+The oracle runs the sample with only the experts the sample uses: a token's top-k over a set
+of experts that contains its own top-k is the same top-k in the same order, so restricting the
+logits to those columns changes neither the selection nor the weights."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from nvfp4_mixture_experts_w4a4_b200 import _lib as C
+from nvfp4_mixture_experts_w4a4_b200 import ops, workloads as W
+from tests import gpu_util as G
+from tests.helpers import layouts as LY
+from tests.helpers import refquant as R
+
+pytestmark = pytest.mark.gpu
+
+SAMPLE = 3  # tokens per workload checked against the oracle
+
+
+@pytest.mark.parametrize("name", ["decode", "prefill_chunk", "long_prefill", "dense", "dense_t1"])
+def test_fullsize_sampled_tokens(name):
+    wl = W.WORKLOADS[name]
+    dev = G.need_gpu()
+    T, H, I, E, k = wl.T, wl.H, wl.I, wl.E, wl.k
+    act = W.make_activations(wl, 0, dev)
+    wts = W.make_weights(wl, 0, dev)
+    experts = ops.NVFP4Experts.from_float(wts["w_gate"], wts["w_up"], wts["w_down"])
+    torch.cuda.synchronize()
+
+    x_bits = G.bf16_bits(act["x"])
+    logits = act["logits"].cpu().numpy()
+    sample = np.unique(np.linspace(0, T - 1, min(SAMPLE, T)).round().astype(np.int64))
+
+    # oracle: routing of the whole batch, permutation, the layer input's tensor scale
+    ids_all, w_all = O.route(logits, k)
+    perm = O.permute(ids_all, E)
+    _, _, s_x = O.quantize(G.bits_to_f32(x_bits))
+    touched = np.unique(ids_all[sample])
+
+    # oracle quantisation of the touched experts, checked against the device's codes
+    tt = torch.as_tensor(touched, device=dev)
+    wg = G.quantize_experts_parallel(wts["w_gate"][tt].cpu().numpy())
+    wu = G.quantize_experts_parallel(wts["w_up"][tt].cpu().numpy())
+    wd = G.quantize_experts_parallel(wts["w_down"][tt].cpu().numpy())
+    del wts
+    ref_w = LY.experts_to_device_layout(wg, wu, wd)
+    got_w = [experts.w13_codes, experts.w13_sf, experts.w13_scale, experts.w2_codes, experts.w2_sf,
+             experts.w2_scale]
+    for r, g in zip(ref_w, got_w):
+        assert np.array_equal(g[tt].cpu().numpy(), r)
+
+    # oracle on the sample, restricted to the touched experts; it calibrates s_h on the sample
+    ref = O.moe_ffn(x_bits[sample], logits[sample][:, touched], k, wg, wu, wd, x_scale=s_x)
+    assert np.array_equal(touched[ref["ids"]], ids_all[sample])
+    s_h = np.ones(E, np.float32)
+    s_h[touched] = ref["h_scale"]
+
+    # the device: the whole batch, dynamic x scale, automatic path (as the benchmark runs it)
+    layer = ops.MoeFFN(experts, k, torch.from_numpy(s_h).to(dev))
+    out = layer(act["x"], act["logits"])
+    torch.cuda.synchronize()
+    im = layer.intermediates(T)
+
+    # routing and permutation of the whole batch: bit-exact
+    assert np.array_equal(im["topk_ids"].cpu().numpy(), ids_all)
+    np.testing.assert_allclose(im["topk_w"].cpu().numpy(), w_all, rtol=2e-6, atol=1e-7)
+    assert np.array_equal(im["counts"].cpu().numpy(), perm["counts"])
+    assert np.array_equal(im["offsets"].cpu().numpy(), perm["offsets"])
+    p2r = im["pair_to_row"].cpu().numpy()
+    po = im["padded_offsets"].cpu().numpy()
+    e_of_pair = ids_all.reshape(-1)
+    assert np.array_equal(p2r - po[e_of_pair] + perm["offsets"][e_of_pair], perm["pair_to_row"])
+    # x scale: bit-exact
+    assert im["x_scale"].item() == np.float32(s_x)
+
+    # sampled pairs: x codes bit-exact, h codes within the requantisation tolerance
+    gpu_pairs = (sample[:, None] * k + np.arange(k)[None, :]).reshape(-1)
+    ref_pairs = np.arange(len(sample) * k)
+    gpu_rows = p2r[gpu_pairs]
+    ref_rows = ref["pair_to_row"][ref_pairs]
+    x_rows = gpu_rows if im["path"] == C.PATH_GEMM else np.repeat(sample, k)
+    xc = im["x_codes"].cpu().numpy()[x_rows]
+    xsf = LY.from_mma(im["x_sf"].cpu().numpy(), im["x_rows"], H)[x_rows]
+    tok = np.repeat(np.arange(len(sample)), k)
+    assert np.array_equal(xc, ref["x_codes"][tok])
+    assert np.array_equal(xsf, ref["x_sf"][tok])
+    hc_pairs = im["h_codes"].cpu().numpy()[gpu_rows]
+    hsf_pairs = LY.from_mma(im["h_sf"].cpu().numpy(), im["h_rows"], I)[gpu_rows]
+    # reorder into the oracle's row order
+    order = np.argsort(ref_rows)
+    hc = np.empty_like(hc_pairs)
+    hsf = np.empty_like(hsf_pairs)
+    hc[ref_rows[order]] = hc_pairs[order]
+    hsf[ref_rows[order]] = hsf_pairs[order]
+    n_diff = G.check_h_codes(hc, hsf, ref["h_codes"], ref["h_sf"])
+
+    # sampled outputs within the stated tolerance (widened by the first-order effect of any
+    # allowed h code difference)
+    extra = None
+    if n_diff:
+        wl_s = W.scaled(wl, T=len(sample), E=len(touched))
+        extra = G.h_diff_effect(hc, hsf, ref, wl_s, lambda e: R.dequantize(wd[0][e], wd[1][e], wd[2][e]))
+    print(f"[full size] {name}: tokens {sample.tolist()}, {len(touched)} experts, {n_diff} h codes differ")
+    G.check_out(G.bf16_bits(out)[sample], ref["out_f64"], extra=extra)
