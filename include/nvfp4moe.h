@@ -91,7 +91,7 @@ enum {
 /* Message for the last failing call on this host thread ("" if none). */
 const char* nvfp4moe_last_error(void);
 
-/* Library version, e.g. 0x000200 = 0.2.0. */
+/* Library version, e.g. 0x000300 = 0.3.0. */
 int32_t nvfp4moe_version(void);
 
 /* Waits for `stream`, then returns the sticky device status word of the current device
@@ -220,6 +220,15 @@ nvfp4moe_status nvfp4_gemm(const uint8_t* A, const uint8_t* A_sf, const float* a
  * moe_ffn_forward - the whole routed feed-forward layer.
  * ---------------------------------------------------------------------------- */
 enum { NVFP4MOE_PATH_AUTO = 0, NVFP4MOE_PATH_GEMV = 1, NVFP4MOE_PATH_GEMM = 2 };
+/* How the k weighted expert rows of a token are combined:
+ *   ORDERED     each row is kept in fp32 and a token's rows are summed in slot order, one
+ *               rounding to bf16 (deterministic);
+ *   ACCUMULATE  the down GEMM adds each row into an fp32 [T][H] accumulator (reduction order
+ *               not fixed, so the last bits of an fp32 sum may differ between calls), then one
+ *               rounding to bf16; no per-slot rows, far less memory traffic for large batches
+ *               (tensor-core path only);
+ *   AUTO        ORDERED for T <= 64, ACCUMULATE above on the tensor-core path. */
+enum { NVFP4MOE_COMBINE_AUTO = 0, NVFP4MOE_COMBINE_ORDERED = 1, NVFP4MOE_COMBINE_ACCUMULATE = 2 };
 
 typedef struct {
   int32_t T, H, I, E, top_k;
@@ -239,6 +248,7 @@ typedef struct {
    * [1] after routing, [2] after the permutation, [3] after quantising x, [4] after the
    * gate/up GEMM, [5] after the down GEMM, [6] after the combine. */
   void* const* stage_events;
+  int32_t combine;            /* NVFP4MOE_COMBINE_* */
 } moe_ffn_desc;
 
 enum { NVFP4MOE_STAGES = 7 };
@@ -254,6 +264,8 @@ typedef struct {
                        the routing step (int4 entries; see csrc/ffn_grouped.cu); else unused */
   int32_t m_tile;   /* 1 on the GEMV path, 64 on the GEMM path */
   int32_t path;     /* resolved path */
+  int32_t combine;  /* resolved combine mode; ACCUMULATE: the accumulator is at `slots` */
+  int32_t reserved;
 } moe_ffn_ws_layout;
 
 nvfp4moe_status moe_ffn_workspace_layout(const moe_ffn_desc* d, moe_ffn_ws_layout* layout);

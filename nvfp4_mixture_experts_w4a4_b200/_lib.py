@@ -15,6 +15,7 @@ SF_ROWMAJOR, SF_MMA = 0, 1
 SCALE_GIVEN, SCALE_DYNAMIC = 0, 1
 DTYPE_BF16, DTYPE_F32 = 0, 1
 PATH_AUTO, PATH_GEMV, PATH_GEMM = 0, 1, 2
+COMBINE_AUTO, COMBINE_ORDERED, COMBINE_ACCUMULATE = 0, 1, 2
 STAGES = 7
 STAGE_NAMES = ("route", "permute", "quantize_x", "gate_up", "down", "combine")
 DEV_BAD_EXPERT_ID, DEV_DUPLICATE_ID, DEV_ROW_OVERFLOW = 1, 2, 4
@@ -43,7 +44,7 @@ class MoeFfnDesc(ctypes.Structure):
         ("x_scale", _vp),
         ("w13_codes", _vp), ("w13_sf", _vp), ("w13_scale", _vp),
         ("w2_codes", _vp), ("w2_sf", _vp), ("w2_scale", _vp),
-        ("h_scale", _vp), ("h_amax", _vp), ("stage_events", _vp),
+        ("h_scale", _vp), ("h_amax", _vp), ("stage_events", _vp), ("combine", _i32),
     ]
 
 
@@ -51,7 +52,8 @@ class MoeFfnWsLayout(ctypes.Structure):
     _fields_ = [(n, _i64) for n in (
         "topk_ids", "topk_w", "counts", "offsets", "padded_offsets", "pair_to_row", "row_token",
         "row_pair", "tile_expert", "active", "x_scale", "x_codes", "x_sf", "h_codes", "h_sf",
-        "slots", "amax_partials", "total", "x_rows", "h_rows", "items")] + [("m_tile", _i32), ("path", _i32)]
+        "slots", "amax_partials", "total", "x_rows", "h_rows", "items")] + [
+        ("m_tile", _i32), ("path", _i32), ("combine", _i32), ("reserved", _i32)]
 
 
 # name -> (restype, argtypes)

@@ -43,6 +43,7 @@ struct BatchArgs {
   uint8_t* x_sf;            // MMA layout
   int32_t* hist;            // [slices][E] histogram, then each slice's first rank per expert
   float* partials;          // [slices] amax of each slice's x rows
+  float* zero_rows;         // nullable [T][H] fp32: each slice's rows are zeroed
   int slices;
   int slice;                // tokens per slice
 };
@@ -310,6 +311,12 @@ __global__ void __launch_bounds__(kThreads) place_quant_kernel(BatchArgs a) {
    }
   }
 
+  // the accumulating combine's output rows of this slice start at zero
+  if (a.zero_rows) {
+    float4* z = reinterpret_cast<float4*>(a.zero_rows + int64_t(t0) * H);
+    for (int64_t i = threadIdx.x; i < int64_t(nt) * H / 4; i += kThreads) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+
   // padding rows and the tile -> expert map for this CTA's share of the padded rows: row r
   // belongs to the last expert whose padded offset is <= r
   const int64_t rows = s_poff[E];
@@ -350,7 +357,7 @@ nvfp4moe_status launch_batch_prologue(const void* x, const float* logits, int T,
                                       int32_t* offsets, int32_t* padded_offsets, int32_t* pair_to_row,
                                       int32_t* row_token, int32_t* row_pair, int32_t* tile_expert, int32_t* active,
                                       float* zero_f32, int expert_order, uint8_t* x_codes, uint8_t* x_sf,
-                                      void* scratch, void* const* stage_events, cudaStream_t s) {
+                                      void* scratch, float* zero_rows, void* const* stage_events, cudaStream_t s) {
   NVFP4_REQUIRE(batch_prologue_fits(T, E, k), NVFP4MOE_UNSUPPORTED_SHAPE, "batch prologue: T=%d E=%d k=%d out of range",
                 T, E, k);
   int lg = 0;
@@ -367,6 +374,7 @@ nvfp4moe_status launch_batch_prologue(const void* x, const float* logits, int T,
   a.zero_f32 = zero_f32;
   a.expert_order = expert_order;
   a.x_codes = x_codes; a.x_sf = x_sf;
+  a.zero_rows = zero_rows;
   a.slice = slice_tokens(T);
   a.slices = (T + a.slice - 1) / a.slice;
   a.hist = static_cast<int32_t*>(scratch);

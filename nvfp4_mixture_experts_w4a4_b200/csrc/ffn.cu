@@ -29,6 +29,8 @@ nvfp4moe_status check_desc(const moe_ffn_desc* d, const char* fn) {
                 "%s: bad path %d", fn, d->path);
   NVFP4_REQUIRE(d->x_scale_mode == NVFP4MOE_SCALE_GIVEN || d->x_scale_mode == NVFP4MOE_SCALE_DYNAMIC,
                 NVFP4MOE_INVALID_ARG, "%s: bad x_scale_mode", fn);
+  NVFP4_REQUIRE(d->combine >= NVFP4MOE_COMBINE_AUTO && d->combine <= NVFP4MOE_COMBINE_ACCUMULATE,
+                NVFP4MOE_INVALID_ARG, "%s: bad combine mode %d", fn, d->combine);
   return NVFP4MOE_OK;
 }
 
@@ -38,6 +40,18 @@ int resolve_path(const moe_ffn_desc* d) {
   // (decode included); the GEMV serves the shapes it does not (I % 128 != 0)
   if (d->I % 128 != 0) return NVFP4MOE_PATH_GEMV;
   return gemm_path_available() ? NVFP4MOE_PATH_GEMM : NVFP4MOE_PATH_GEMV;
+}
+
+// AUTO: the ordered combine while it is cheap (T <= 64), accumulation above (tensor cores)
+int resolve_combine(const moe_ffn_desc* d, int path) {
+  if (d->combine != NVFP4MOE_COMBINE_AUTO) return d->combine;
+  return path == NVFP4MOE_PATH_GEMM && d->T > 64 ? NVFP4MOE_COMBINE_ACCUMULATE : NVFP4MOE_COMBINE_ORDERED;
+}
+
+// in the slot region: the fp32 accumulator [T][H] first when accumulating, then the batch
+// prologue's scratch
+int64_t prologue_scratch_offset(const moe_ffn_desc* d, int combine) {
+  return combine == NVFP4MOE_COMBINE_ACCUMULATE ? align_up(int64_t(d->T) * d->H * 4) : 0;
 }
 
 int64_t max_active_experts(const moe_ffn_desc* d) {
@@ -79,8 +93,13 @@ void make_layout(const moe_ffn_desc* d, moe_ffn_ws_layout* L) {
   // per-slot rows of the down projection: fp32 split-K partials on the GEMV path, bf16 on
   // the tensor-core path (halves the slot round trip of large prefills)
   // (the region also holds the batch prologue's slice histograms until the down GEMM)
+  const int combine = resolve_combine(d, path);
   const int64_t prologue_scratch = batch_prologue_scratch_bytes(d->T, d->E);
-  if (path == NVFP4MOE_PATH_GEMM)
+  L->combine = combine;
+  L->reserved = 0;
+  if (combine == NVFP4MOE_COMBINE_ACCUMULATE)
+    L->slots = take(prologue_scratch_offset(d, combine) + prologue_scratch);
+  else if (path == NVFP4MOE_PATH_GEMM)
     L->slots = take(std::max<int64_t>(P * H * 4, prologue_scratch));
   else
     L->slots = take(std::max<int64_t>(int64_t(gemv_down_ksplit(max_active_experts(d), H, I)) * P * H * 4,
@@ -140,6 +159,8 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
     NVFP4_REQUIRE(d->E <= 1024, NVFP4MOE_UNSUPPORTED_SHAPE, "%s: E > 1024", fn);
     NVFP4_REQUIRE(gemm_path_available(), NVFP4MOE_CUDA_ERROR, "%s: the tensor-core path is unavailable", fn);
   }
+  NVFP4_REQUIRE(L.combine != NVFP4MOE_COMBINE_ACCUMULATE || L.path == NVFP4MOE_PATH_GEMM, NVFP4MOE_UNSUPPORTED_SHAPE,
+                "%s: the accumulating combine needs the tensor-core path", fn);
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   auto I32 = [&](int64_t off) { return reinterpret_cast<int32_t*>(ws + off); };
@@ -164,6 +185,9 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   const int64_t list_entries = grouped_fused_list_entries(n_act, 2 * I / 128, H / 128);
   int4* list = reinterpret_cast<int4*>(ws + L.items);
   int* done = reinterpret_cast<int*>(list + list_entries);
+  const bool accumulate = L.combine == NVFP4MOE_COMBINE_ACCUMULATE;
+  float* accum = F32(L.slots);  // fp32 [T][H] when accumulating
+  uint8_t* prologue_scratch = ws + L.slots + prologue_scratch_offset(d, L.combine);
 
   mark(0);
   if (fused) {
@@ -181,8 +205,8 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
     st = launch_batch_prologue(x, logits, T, H, E, k, L.m_tile, dyn ? 1 : 0, xs, I32(L.topk_ids), F32(L.topk_w),
                                I32(L.counts), I32(L.offsets), I32(L.padded_offsets), I32(L.pair_to_row),
                                I32(L.row_token), I32(L.row_pair), I32(L.tile_expert), I32(L.active), d->h_amax,
-                               L.path == NVFP4MOE_PATH_GEMM ? 1 : 0, ws + L.x_codes, ws + L.x_sf, ws + L.slots,
-                               d->stage_events, s);
+                               L.path == NVFP4MOE_PATH_GEMM ? 1 : 0, ws + L.x_codes, ws + L.x_sf, prologue_scratch,
+                               accumulate ? accum : nullptr, d->stage_events, s);
     if (st != NVFP4MOE_OK) return st;
   }
 
@@ -216,6 +240,10 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
     return mark_st;
   }
 
+  if (accumulate && fused) {  // the batch prologue zeroes the accumulator itself
+    const cudaError_t e = cudaMemsetAsync(accum, 0, size_t(T) * H * 4, s);
+    NVFP4_REQUIRE(e == cudaSuccess, NVFP4MOE_CUDA_ERROR, "%s: zeroing the accumulator: %s", fn, cudaGetErrorString(e));
+  }
   mark(3);
   GemmFfnArgs a;
   a.T = T; a.H = H; a.I = I; a.E = E; a.k = k;
@@ -232,10 +260,12 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   a.list = lists ? list : nullptr;
   a.list_cap = list_entries - 1;
   a.done = lists ? done : nullptr;
+  a.accum = accumulate ? accum : nullptr;
   st = launch_grouped_ffn(a, s);
   if (st != NVFP4MOE_OK) return st;
   mark(5);
-  st = launch_combine(F32(L.slots), int64_t(T) * k * H, 1, I32(L.pair_to_row), T, H, k, out, s);
+  st = accumulate ? launch_accum_to_bf16(accum, int64_t(T) * H, out, s)
+                  : launch_combine(F32(L.slots), int64_t(T) * k * H, 1, I32(L.pair_to_row), T, H, k, out, s);
   if (st != NVFP4MOE_OK) return st;
   mark(6);
   return mark_st;

@@ -38,6 +38,7 @@ struct GemmFfnArgs {
   const int4* list;               // nullable: the fused work list and the items it can hold
   int64_t list_cap;
   int* done;                      // with list: [E] gate/up completion counters, zeroed by its writer
+  float* accum;                   // nullable [T][H] fp32: the down GEMM adds its rows here (zeroed)
 };
 
 bool gemm_path_available();

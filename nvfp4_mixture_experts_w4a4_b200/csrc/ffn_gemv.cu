@@ -305,6 +305,29 @@ nvfp4moe_status launch_combine(const float* slots, int64_t slot_stride, int kspl
   return check_launch("combine");
 }
 
+__global__ void accum_to_bf16_kernel(const float* __restrict__ acc, int64_t n, __nv_bfloat16* __restrict__ out) {
+  griddep_wait();  // the accumulator is complete when the down GEMM is
+  for (int64_t i = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) * 8; i < n; i += int64_t(gridDim.x) * blockDim.x * 8) {
+    const float4 a = *reinterpret_cast<const float4*>(acc + i);
+    const float4 b = *reinterpret_cast<const float4*>(acc + i + 4);
+    const __nv_bfloat162 q0 = __floats2bfloat162_rn(a.x, a.y), q1 = __floats2bfloat162_rn(a.z, a.w);
+    const __nv_bfloat162 q2 = __floats2bfloat162_rn(b.x, b.y), q3 = __floats2bfloat162_rn(b.z, b.w);
+    *reinterpret_cast<uint4*>(out + i) =
+        make_uint4(*reinterpret_cast<const uint32_t*>(&q0), *reinterpret_cast<const uint32_t*>(&q1),
+                   *reinterpret_cast<const uint32_t*>(&q2), *reinterpret_cast<const uint32_t*>(&q3));
+  }
+}
+
+nvfp4moe_status launch_accum_to_bf16(const float* acc, int64_t n, void* out, cudaStream_t s) {
+  if (n == 0) return NVFP4MOE_OK;
+  int64_t blocks = (n / 8 + 255) / 256;
+  if (blocks > int64_t(num_sms()) * 8) blocks = int64_t(num_sms()) * 8;
+  const cudaError_t e = launch_dependent(accum_to_bf16_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, acc, n,
+                                         static_cast<__nv_bfloat16*>(out));
+  if (e != cudaSuccess) return fail(NVFP4MOE_CUDA_ERROR, "accumulator to bf16: %s", cudaGetErrorString(e));
+  return check_launch("accumulator to bf16");
+}
+
 nvfp4moe_status launch_replicate_rows(const uint8_t* codes_tok, const uint8_t* sf_tok, const int32_t* row_token,
                                       const int32_t* rows_used, int64_t rows_cap, int64_t T, int64_t K,
                                       uint8_t* codes_out, uint8_t* sf_out, cudaStream_t s) {

@@ -72,6 +72,8 @@ nvfp4moe_status launch_batch_prologue(const void* x, const float* logits, int T,
                                       int32_t* offsets, int32_t* padded_offsets, int32_t* pair_to_row,
                                       int32_t* row_token, int32_t* row_pair, int32_t* tile_expert, int32_t* active,
                                       float* zero_f32, int expert_order, uint8_t* x_codes, uint8_t* x_sf,
-                                      void* scratch, void* const* stage_events, cudaStream_t s);
+                                      void* scratch, float* zero_rows, void* const* stage_events, cudaStream_t s);
+// out[i] = bf16(acc[i]) for the accumulating combine (a programmatic dependent of the down GEMM)
+nvfp4moe_status launch_accum_to_bf16(const float* acc, int64_t n, void* out, cudaStream_t s);
 
 }  // namespace nvfp4moe

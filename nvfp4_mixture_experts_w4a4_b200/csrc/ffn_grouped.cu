@@ -99,7 +99,9 @@ struct GroupedParams {
   // down
   const float* w2_scale;
   const float* topk_w;
-  float* slots;      // [T*k][H] fp32 rows, by pair
+  float* slots;      // [T*k][H] fp32 rows, by pair (ordered combine)
+  float* accum;      // nullable [T][H] fp32: when set, weighted rows are added here instead
+  int k;             // top_k (pair -> token)
   int H;
   uint32_t* status;
   const int4* list;  // fused mode: work list written by the routing step (entry 0: {gate/up
@@ -150,6 +152,13 @@ __device__ __forceinline__ int ld_relaxed(const int* ptr) {
   int v;
   asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
   return v;
+}
+__device__ __forceinline__ void red_add_f32(float* p, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+__device__ __forceinline__ void red_add_v4_f32(float* p, float4 v) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
 }
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async_global() {
@@ -612,11 +621,13 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__
         }
         if (EPI == EPI_FUSED) pending = w.e;  // counted once its stores have drained
       } else {
-        // Each 32-token chunk goes through the warp's transpose tile in two halves of 16 tokens:
-        // lanes (= weight rows) park their 16 accumulators, then lane l takes token l & 15 and
-        // rows 16 * (l >> 4) .. +16, scales them by that token's routing weight and writes those
-        // 64 contiguous bytes of its fp32 slot row.
-        const int tl = lane & 15, rh = lane >> 4;
+        // A chunk's 32 token columns go through the warp's transpose tile in two halves of 16
+        // tokens: lanes (= weight rows) park their accumulators, then each store instruction of
+        // the warp covers 4 tokens x the quarter's 32 rows, 128 contiguous bytes per token
+        // (lane l: token l >> 3 of the step, rows 4 * (l & 7) .. +4), scaled by the token's
+        // routing weight.  The rows go to the token's fp32 slot row, or, accumulating, are
+        // added into its output row.
+        const int tq = lane >> 3, cq = lane & 7;
 #pragma unroll
         for (int c2 = 0; c2 < C::MAX_CHUNKS / 2; ++c2) {
           const int cc = 2 * c2 + half;
@@ -626,13 +637,17 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__
           tmem_ld_wait();
           const int nj = min(32, w.n_rows - cc * 32);
           if (nj <= 8) {
-            // a few tokens (decode): each token's 32 rows are one 64-byte store of the warp
+            // a few tokens (decode): each token's 32 rows are one 128-byte access of the warp
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
               if (j >= nj) break;
               const int32_t pair = __shfl_sync(0xffffffffu, pr[c2], j);
               const float wj = __shfl_sync(0xffffffffu, wt[c2], j);
-              if (pair >= 0) p.slots[int64_t(pair) * p.H + wrow] = __uint_as_float(r[j]) * wj;
+              if (pair >= 0) {
+                const float v = __uint_as_float(r[j]) * wj;
+                if (p.accum) red_add_f32(p.accum + int64_t(pair / p.k) * p.H + wrow, v);
+                else p.slots[int64_t(pair) * p.H + wrow] = v;
+              }
             }
             continue;
           }
@@ -642,17 +657,20 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__
 #pragma unroll
             for (int t = 0; t < 16; ++t) tr[t * DOWN_TR_STRIDE + lane] = __uint_as_float(r[sub * 16 + t]);
             __syncwarp();
-            const int32_t pair = __shfl_sync(0xffffffffu, pr[c2], sub * 16 + tl);
-            const float wj = __shfl_sync(0xffffffffu, wt[c2], sub * 16 + tl);
-            float v[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = tr[tl * DOWN_TR_STRIDE + rh * 16 + i] * wj;
-            __syncwarp();
-            if (pair >= 0) {
-              float4* dst = reinterpret_cast<float4*>(p.slots + int64_t(pair) * p.H + w.mt * WM + q * 32 + rh * 16);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            for (int st = 0; st < 4; ++st) {
+              const int tok = 4 * st + tq;
+              const int32_t pair = __shfl_sync(0xffffffffu, pr[c2], sub * 16 + tok);
+              const float wj = __shfl_sync(0xffffffffu, wt[c2], sub * 16 + tok);
+              const float* src = tr + tok * DOWN_TR_STRIDE + 4 * cq;
+              const float4 v = make_float4(src[0] * wj, src[1] * wj, src[2] * wj, src[3] * wj);
+              if (pair >= 0) {
+                const int64_t col = int64_t(w.mt) * WM + q * 32 + 4 * cq;
+                if (p.accum) red_add_v4_f32(p.accum + int64_t(pair / p.k) * p.H + col, v);
+                else *reinterpret_cast<float4*>(p.slots + int64_t(pair) * p.H + col) = v;
+              }
             }
+            __syncwarp();
           }
         }
       }
@@ -745,6 +763,8 @@ nvfp4moe_status launch_grouped_ffn(const GemmFfnArgs& a, cudaStream_t s) {
   p.w2_scale = a.w2_scale;
   p.topk_w = a.topk_w;
   p.slots = static_cast<float*>(a.slots_f32);
+  p.accum = a.accum;
+  p.k = a.k;
   p.H = a.H;
   auto mark4 = [&]() -> nvfp4moe_status {
     if (!a.stage_events) return NVFP4MOE_OK;

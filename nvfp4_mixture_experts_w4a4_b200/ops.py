@@ -189,12 +189,13 @@ class MoeFFN:
     """The routed NVFP4 W4A4 feed-forward layer (moe_ffn_forward) with a cached workspace."""
 
     def __init__(self, experts: NVFP4Experts, top_k: int, h_scale: torch.Tensor, x_scale: torch.Tensor | None = None,
-                 path: int = C.PATH_AUTO):
+                 path: int = C.PATH_AUTO, combine: int = C.COMBINE_AUTO):
         self.w = experts
         self.top_k = top_k
         self.h_scale = h_scale.to(torch.float32).contiguous()
         self.x_scale = None if x_scale is None else x_scale.to(torch.float32).contiguous().view(1)
         self.path = path
+        self.combine = combine
         self._ws = {}
 
     def desc(self, T: int, h_amax: torch.Tensor | None = None, events=None) -> C.MoeFfnDesc:
@@ -202,6 +203,7 @@ class MoeFFN:
         d = C.MoeFfnDesc()
         d.T, d.H, d.I, d.E, d.top_k = T, w.H, w.I, w.E, self.top_k
         d.path = self.path
+        d.combine = self.combine
         d.x_scale_mode = C.SCALE_DYNAMIC if self.x_scale is None else C.SCALE_GIVEN
         d.x_scale = None if self.x_scale is None else self.x_scale.data_ptr()
         d.w13_codes, d.w13_sf, d.w13_scale = w.w13_codes.data_ptr(), w.w13_sf.data_ptr(), w.w13_scale.data_ptr()
@@ -261,7 +263,7 @@ class MoeFFN:
             return ws[off:off + nbytes].view(dtype)
 
         return dict(
-            path=L.path, m_tile=L.m_tile,
+            path=L.path, m_tile=L.m_tile, combine=L.combine,
             topk_ids=view(L.topk_ids, P, torch.int32).view(T, k),
             topk_w=view(L.topk_w, P, torch.float32).view(T, k),
             counts=view(L.counts, w.E, torch.int32), offsets=view(L.offsets, w.E + 1, torch.int32),

@@ -118,7 +118,8 @@ def experts_from_oracle(wg, wu, wd, dev) -> ops.NVFP4Experts:
     return ops.NVFP4Experts(*t)
 
 
-def run_layer_pair(wl: W.Workload, path: int, seed: int = 0, dev=None, given_x_scale: bool = False):
+def run_layer_pair(wl: W.Workload, path: int, seed: int = 0, dev=None, given_x_scale: bool = False,
+                   combine: int = C.COMBINE_AUTO):
     """Runs oracle and library on the same inputs; returns (oracle result, gpu out, layer)."""
     dev = dev or need_gpu()
     act, wts, wg, wu, wd = layer_inputs(wl, seed)
@@ -130,7 +131,7 @@ def run_layer_pair(wl: W.Workload, path: int, seed: int = 0, dev=None, given_x_s
     ref = O.moe_ffn(x_bits, logits, wl.k, wg, wu, wd, x_scale=xs)
     experts = experts_from_oracle(wg, wu, wd, dev)
     layer = ops.MoeFFN(experts, wl.k, torch.from_numpy(ref["h_scale"]).to(dev),
-                       x_scale=None if xs is None else torch.tensor([xs], device=dev), path=path)
+                       x_scale=None if xs is None else torch.tensor([xs], device=dev), path=path, combine=combine)
     h_amax = torch.empty(wl.E, dtype=torch.float32, device=dev)
     out = layer(act["x"].to(dev), act["logits"].to(dev), h_amax=h_amax)
     torch.cuda.synchronize()

@@ -143,3 +143,20 @@ def test_stage_marks_eager_and_in_a_cuda_graph(name):
     assert torch.equal(graph_out, out)
     times = [marks[i].elapsed_time(marks[i + 1]) for i in range(C.STAGES - 1)]
     assert all(t >= 0.0 for t in times) and sum(times) > 0.0
+
+
+@pytest.mark.parametrize("combine", [C.COMBINE_ORDERED, C.COMBINE_ACCUMULATE])
+@pytest.mark.parametrize("name", ["tiny", "long_prefill_small", "dense_small", "popular_expert_chunks"])
+def test_layer_gemm_combine_modes(name, combine):
+    """Both ways of combining a token's k weighted rows (ordered fp32 slots; fp32 accumulation
+    into the output rows) meet the stated tolerance, with either prologue."""
+    wl = GEMM_CASES[name]
+    ref, out, layer, h_amax = G.run_layer_pair(wl, C.PATH_GEMM, combine=combine)
+    assert layer.intermediates(wl.T)["combine"] == combine
+    G.check_layer(wl, ref, out, layer, h_amax)
+
+
+def test_accumulate_needs_the_tensor_core_path():
+    wl = CASES["long_prefill_small"]
+    with pytest.raises(C.Nvfp4MoeError):
+        G.run_layer_pair(wl, C.PATH_GEMV, combine=C.COMBINE_ACCUMULATE)
