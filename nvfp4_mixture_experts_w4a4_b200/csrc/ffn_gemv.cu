@@ -167,30 +167,28 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) gemv_down_kernel(GemvDownAr
 __global__ void combine_kernel(const float* __restrict__ slots, int64_t slot_stride, int ksplit,
                                const int32_t* __restrict__ pair_to_row, int T, int H, int k,
                                __nv_bfloat16* __restrict__ out) {
-  griddep_wait();  // the slot rows come from the down GEMM launched just before
+  (void)pair_to_row;  // every pair has a row: slots are addressed by pair directly
+  griddep_wait();     // the slot rows come from the down GEMM launched just before
   const int64_t per_row = H / 8;
   const int64_t total = int64_t(T) * per_row;
   for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total;
        i += int64_t(gridDim.x) * blockDim.x) {
     const int64_t t = i / per_row, n = (i - t * per_row) * 8;
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int j0 = 0; j0 < k; j0 += 4) {
-      // up to four slots' rows in flight at once; summed in slot order
-      bool ok[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) ok[u] = j0 + u < k && pair_to_row[t * k + j0 + u] >= 0;
+    for (int j0 = 0; j0 < k; j0 += 8) {
       for (int s = 0; s < ksplit; ++s) {
-        float4 a[4], b[4];
+        // up to eight slots' rows in flight at once; summed in slot order
+        float4 a[8], b[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          if (ok[u]) {
+        for (int u = 0; u < 8; ++u)
+          if (j0 + u < k) {
             const float4* src = reinterpret_cast<const float4*>(slots + s * slot_stride + (t * k + j0 + u) * H + n);
             a[u] = src[0];
             b[u] = src[1];
           }
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          if (ok[u]) {
+        for (int u = 0; u < 8; ++u)
+          if (j0 + u < k) {
             acc[0] += a[u].x; acc[1] += a[u].y; acc[2] += a[u].z; acc[3] += a[u].w;
             acc[4] += b[u].x; acc[5] += b[u].y; acc[6] += b[u].z; acc[7] += b[u].w;
           }
