@@ -5,7 +5,7 @@
 // high word is the logit mapped to an unsigned integer with the same order (after -0 is
 // turned into +0, so the two zeros tie), the low word is 0xFFFF - index, so among equal
 // logits the lower index has the larger key.  Each lane keeps its best remaining key; a
-// round is a warp max over those (5 shuffles) and only the winning lane rescans its slots.
+// round is a warp max over those and only the winning lane recomputes its best.
 // Integer compares make the selection exact; the softmax over the k selected logits
 // (relative to the largest) is fp32.
 #pragma once
@@ -28,8 +28,24 @@ __device__ __forceinline__ float topk_key_value(uint64_t key) {
   return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
 }
 
+// Largest of a lane's keys: a pairwise tree (depth log2 PER_LANE) instead of a linear chain.
+template <int PER_LANE>
+__device__ __forceinline__ uint64_t topk_lane_max(const uint64_t (&key)[PER_LANE]) {
+  uint64_t t[PER_LANE];
+#pragma unroll
+  for (int i = 0; i < PER_LANE; ++i) t[i] = key[i];
+#pragma unroll
+  for (int w = PER_LANE / 2; w >= 1; w /= 2)
+#pragma unroll
+    for (int i = 0; i < w; ++i) t[i] = t[i + w] > t[i] ? t[i + w] : t[i];
+  return t[0];
+}
+
 // Selects the top k (k <= 32) of l[0..E) for the calling warp.  Lane j < k returns the j-th
-// expert in *id and its softmax weight in *w.
+// expert in *id and its softmax weight in *w.  A round takes the warp maximum of the lanes'
+// best keys with two hardware reductions (the logit word, then the index word among the lanes
+// that hold that logit, which picks the lower expert index), and only the winning lane drops
+// the key and recomputes its best.
 template <int PER_LANE>
 __device__ __forceinline__ void warp_topk(const float* __restrict__ l, int E, int k, int* id, float* w) {
   const int lane = threadIdx.x & 31;
@@ -39,25 +55,18 @@ __device__ __forceinline__ void warp_topk(const float* __restrict__ l, int E, in
     const int e = lane + 32 * i;
     key[i] = e < E ? topk_key(l[e], e) : 0ull;  // 0 marks an absent or taken slot
   }
-  uint64_t mine = 0;
-#pragma unroll
-  for (int i = 0; i < PER_LANE; ++i) mine = key[i] > mine ? key[i] : mine;
+  uint64_t mine = topk_lane_max<PER_LANE>(key);
   uint64_t sel = 0;  // lane j keeps the j-th selected key
   for (int j = 0; j < k; ++j) {
-    uint64_t best = mine;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const uint64_t other = __shfl_xor_sync(0xffffffffu, best, o);
-      best = other > best ? other : best;
-    }
+    const uint32_t hi = uint32_t(mine >> 32), lo = uint32_t(mine);
+    const uint32_t mhi = __reduce_max_sync(0xffffffffu, hi);
+    const uint32_t mlo = __reduce_max_sync(0xffffffffu, hi == mhi ? lo : 0u);
+    const uint64_t best = (uint64_t(mhi) << 32) | mlo;
     if (lane == j) sel = best;
-    if (best == mine) {  // this lane owned the winner (keys are unique): drop it, rescan
-      mine = 0;
+    if (best == mine) {  // this lane owned the winner (keys are unique): drop it
 #pragma unroll
-      for (int i = 0; i < PER_LANE; ++i) {
-        if (key[i] == best) key[i] = 0;
-        mine = key[i] > mine ? key[i] : mine;
-      }
+      for (int i = 0; i < PER_LANE; ++i) key[i] = key[i] == best ? 0ull : key[i];
+      mine = topk_lane_max<PER_LANE>(key);
     }
   }
   const int bi = topk_key_index(sel);
