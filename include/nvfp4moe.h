@@ -227,7 +227,8 @@ enum { NVFP4MOE_PATH_AUTO = 0, NVFP4MOE_PATH_GEMV = 1, NVFP4MOE_PATH_GEMM = 2 };
  *               not fixed, so the last bits of an fp32 sum may differ between calls), then one
  *               rounding to bf16; no per-slot rows, far less memory traffic for large batches
  *               (tensor-core path only);
- *   AUTO        ORDERED for T <= 64, ACCUMULATE above on the tensor-core path. */
+ *   AUTO        ORDERED; ACCUMULATE when top_k == 1 on the tensor-core path (one term per
+ *               output: exact and deterministic). */
 enum { NVFP4MOE_COMBINE_AUTO = 0, NVFP4MOE_COMBINE_ORDERED = 1, NVFP4MOE_COMBINE_ACCUMULATE = 2 };
 
 typedef struct {

@@ -42,10 +42,12 @@ int resolve_path(const moe_ffn_desc* d) {
   return gemm_path_available() ? NVFP4MOE_PATH_GEMM : NVFP4MOE_PATH_GEMV;
 }
 
-// AUTO: the ordered combine while it is cheap (T <= 64), accumulation above (tensor cores)
+// AUTO: the ordered combine (faster than accumulation at the routed benchmark sizes once the
+// down GEMM stores its rows with tile stores); with top_k = 1 accumulation adds one term per
+// output, so it is exact and deterministic too, and saves the slot round trip
 int resolve_combine(const moe_ffn_desc* d, int path) {
   if (d->combine != NVFP4MOE_COMBINE_AUTO) return d->combine;
-  return path == NVFP4MOE_PATH_GEMM && d->T > 64 ? NVFP4MOE_COMBINE_ACCUMULATE : NVFP4MOE_COMBINE_ORDERED;
+  return path == NVFP4MOE_PATH_GEMM && d->top_k == 1 ? NVFP4MOE_COMBINE_ACCUMULATE : NVFP4MOE_COMBINE_ORDERED;
 }
 
 // in the slot region: the fp32 accumulator [T][H] first when accumulating, then the batch
@@ -99,8 +101,8 @@ void make_layout(const moe_ffn_desc* d, moe_ffn_ws_layout* L) {
   L->reserved = 0;
   if (combine == NVFP4MOE_COMBINE_ACCUMULATE)
     L->slots = take(prologue_scratch_offset(d, combine) + prologue_scratch);
-  else if (path == NVFP4MOE_PATH_GEMM)
-    L->slots = take(std::max<int64_t>(P * H * 4, prologue_scratch));
+  else if (path == NVFP4MOE_PATH_GEMM)  // rows by pair; above 64 tokens by padded expert row
+    L->slots = take(std::max<int64_t>((prologue_fits(d->T, d->E, d->top_k) ? P : rows_cap) * H * 4, prologue_scratch));
   else
     L->slots = take(std::max<int64_t>(int64_t(gemv_down_ksplit(max_active_experts(d), H, I)) * P * H * 4,
                                       prologue_scratch));
@@ -261,11 +263,16 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   a.list_cap = list_entries - 1;
   a.done = lists ? done : nullptr;
   a.accum = accumulate ? accum : nullptr;
+  a.slots_by_row = (!accumulate && !fused) ? 1 : 0;
   st = launch_grouped_ffn(a, s);
   if (st != NVFP4MOE_OK) return st;
   mark(5);
-  st = accumulate ? launch_accum_to_bf16(accum, int64_t(T) * H, out, s)
-                  : launch_combine(F32(L.slots), int64_t(T) * k * H, 1, I32(L.pair_to_row), T, H, k, out, s);
+  if (accumulate)
+    st = launch_accum_to_bf16(accum, int64_t(T) * H, out, s);
+  else if (a.slots_by_row)
+    st = launch_combine_rows(F32(L.slots), I32(L.pair_to_row), F32(L.topk_w), T, H, k, out, s);
+  else
+    st = launch_combine(F32(L.slots), int64_t(T) * k * H, 1, I32(L.pair_to_row), T, H, k, out, s);
   if (st != NVFP4MOE_OK) return st;
   mark(6);
   return mark_st;

@@ -39,6 +39,8 @@ struct GemmFfnArgs {
   int64_t list_cap;
   int* done;                      // with list: [E] gate/up completion counters, zeroed by its writer
   float* accum;                   // nullable [T][H] fp32: the down GEMM adds its rows here (zeroed)
+  int slots_by_row;               // batches above 64 tokens, ordered combine: slots_f32 is
+                                  // [rows_cap][H], rows in padded expert order, unweighted
 };
 
 bool gemm_path_available();

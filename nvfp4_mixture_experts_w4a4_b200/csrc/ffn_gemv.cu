@@ -303,6 +303,62 @@ nvfp4moe_status launch_combine(const float* slots, int64_t slot_stride, int kspl
   return check_launch("combine");
 }
 
+__global__ void combine_rows_kernel(const float* __restrict__ slots, const int32_t* __restrict__ pair_to_row,
+                                    const float* __restrict__ topk_w, int T, int H, int k,
+                                    __nv_bfloat16* __restrict__ out) {
+  griddep_wait();  // the slot rows come from the down GEMM launched just before
+  const int64_t per_row = H / 8;
+  const int64_t total = int64_t(T) * per_row;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t t = i / per_row, n = (i - t * per_row) * 8;
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int j0 = 0; j0 < k; j0 += 8) {
+      int32_t row[8];
+      float wj[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        row[u] = j0 + u < k ? __ldg(pair_to_row + t * k + j0 + u) : 0;
+        wj[u] = j0 + u < k ? __ldg(topk_w + t * k + j0 + u) : 0.0f;
+      }
+      float4 a[8], b[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (j0 + u < k) {
+          const float4* src = reinterpret_cast<const float4*>(slots + int64_t(row[u]) * H + n);
+          a[u] = src[0];
+          b[u] = src[1];
+        }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (j0 + u < k) {  // in slot order
+          acc[0] += wj[u] * a[u].x; acc[1] += wj[u] * a[u].y; acc[2] += wj[u] * a[u].z; acc[3] += wj[u] * a[u].w;
+          acc[4] += wj[u] * b[u].x; acc[5] += wj[u] * b[u].y; acc[6] += wj[u] * b[u].z; acc[7] += wj[u] * b[u].w;
+        }
+    }
+    uint4 o;
+    uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
+      ow[q] = *reinterpret_cast<const uint32_t*>(&b2);
+    }
+    *reinterpret_cast<uint4*>(out + t * H + n) = o;
+  }
+}
+
+nvfp4moe_status launch_combine_rows(const float* slots, const int32_t* pair_to_row, const float* topk_w, int T, int H,
+                                    int k, void* out, cudaStream_t s) {
+  const int64_t total = int64_t(T) * (H / 8);
+  if (total == 0) return NVFP4MOE_OK;
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > int64_t(num_sms()) * 8) blocks = int64_t(num_sms()) * 8;
+  const cudaError_t e = launch_dependent(combine_rows_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, slots,
+                                         pair_to_row, topk_w, T, H, k, static_cast<__nv_bfloat16*>(out));
+  if (e != cudaSuccess) return fail(NVFP4MOE_CUDA_ERROR, "combine (rows): %s", cudaGetErrorString(e));
+  return check_launch("combine (rows)");
+}
+
 __global__ void accum_to_bf16_kernel(const float* __restrict__ acc, int64_t n, __nv_bfloat16* __restrict__ out) {
   griddep_wait();  // the accumulator is complete when the down GEMM is
   for (int64_t i = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) * 8; i < n; i += int64_t(gridDim.x) * blockDim.x * 8) {

@@ -73,6 +73,10 @@ nvfp4moe_status launch_batch_prologue(const void* x, const float* logits, int T,
                                       int32_t* row_token, int32_t* row_pair, int32_t* tile_expert, int32_t* active,
                                       float* zero_f32, int expert_order, uint8_t* x_codes, uint8_t* x_sf,
                                       void* scratch, float* zero_rows, void* const* stage_events, cudaStream_t s);
+// out[t] = bf16(sum_j topk_w[t*k+j] * slots[pair_to_row[t*k+j]]) in slot order, over fp32 slot
+// rows in padded expert order (a programmatic dependent of the down GEMM)
+nvfp4moe_status launch_combine_rows(const float* slots, const int32_t* pair_to_row, const float* topk_w, int T, int H,
+                                    int k, void* out, cudaStream_t s);
 // out[i] = bf16(acc[i]) for the accumulating combine (a programmatic dependent of the down GEMM)
 nvfp4moe_status launch_accum_to_bf16(const float* acc, int64_t n, void* out, cudaStream_t s);
 

@@ -48,14 +48,20 @@ constexpr int SCHED_PER_THREAD = (SCHED_CAP + kThreads - 1) / kThreads;
 
 // Tile configuration: BNMAX tokens per tile at most, STAGES shared-memory stages, NACC TMEM
 // accumulators.
-//   <192, 4, 2> general; <64, 6, 4> when no expert can hold more than 64 tokens (T <= 64): more
-//   weight bytes in flight for the small decode tiles, and the MMA may run three items ahead
-//   of a slow epilogue.
-template <int BN_, int STAGES_, int NACC_>
+//   <192, 4, 2> gate/up and <192, 3, 2, tile stores> down above 64 tokens (the down epilogue
+//   stores its output through per-warp staging tiles with TMA, slot rows in expert order);
+//   <64, 6, 4> when no expert can hold more than 64 tokens (T <= 64): more weight bytes in
+//   flight for the small decode tiles, and the MMA may run three items ahead of a slow
+//   epilogue.
+template <int BN_, int STAGES_, int NACC_, bool OUT_TMA_>
 struct Cfg {
   static constexpr int BNMAX = BN_;
   static constexpr int STAGES = STAGES_;
   static constexpr int NACC = NACC_;                     // TMEM accumulators (items in flight)
+  // down output by tile stores: two 16-token x 32-row fp32 staging tiles per epilogue warp
+  static constexpr bool OUT_TMA = OUT_TMA_;
+  static constexpr int OUT_TILE_BYTES = 16 * 32 * 4;
+  static constexpr int OUT_BYTES = OUT_TMA ? EPI_WARPS * 2 * OUT_TILE_BYTES : 0;
   static constexpr int ACC_COLS = BNMAX;
   static constexpr int SFA_COL = NACC * ACC_COLS;        // 16 columns
   static constexpr int SFB_COL = SFA_COL + 16;           // 32 columns
@@ -66,13 +72,14 @@ struct Cfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int SMEM_BYTES =
       1024 + STAGES * STAGE_BYTES + (2 * STAGES + 2 * NACC + 1) * 8 + 16 + (5 * MAX_E + 1) * 4 +
-      EPI_WARPS * TR_FLOATS * 4;
+      EPI_WARPS * TR_FLOATS * 4 + (OUT_TMA ? 128 + OUT_BYTES : 0);
   static constexpr int MAX_CHUNKS = BNMAX / 32;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(SFB_COL + 32 <= int(kTmemCols), "TMEM budget");
 };
-using CfgWide = Cfg<192, 4, 2>;
-using CfgDecode = Cfg<64, 6, 4>;
+using CfgWide = Cfg<192, 4, 2, false>;      // gate/up, batches above 64 tokens
+using CfgWideDown = Cfg<192, 3, 2, true>;   // down, batches above 64 tokens (room for the tiles)
+using CfgDecode = Cfg<64, 6, 4, false>;
 
 // Modes: one GEMM per launch (gate/up or down), or both in one persistent launch (decode):
 // the CTAs work through gate/up items and then down items of one list, and a down item waits
@@ -100,6 +107,8 @@ struct GroupedParams {
   const float* w2_scale;
   const float* topk_w;
   float* slots;      // [T*k][H] fp32 rows, by pair (ordered combine)
+  int slots_by_row;  // tile-store configurations: slot rows in padded expert order, unweighted,
+                     // written through tmO (the combine applies the routing weights)
   float* accum;      // nullable [T][H] fp32: when set, weighted rows are added here instead
   int k;             // top_k (pair -> token)
   int H;
@@ -175,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 grouped_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__ CUtensorMap tmX0,
                const __grid_constant__ CUtensorMap tmXs0, const __grid_constant__ CUtensorMap tmW1,
                const __grid_constant__ CUtensorMap tmX1, const __grid_constant__ CUtensorMap tmXs1,
-               GroupedParams p) {
+               const __grid_constant__ CUtensorMap tmO, GroupedParams p) {
   // the phase of a single-GEMM launch; fused launches take it from each item
   constexpr int PH = EPI == EPI_DOWN ? 1 : 0;
   extern __shared__ uint8_t smem_raw[];
@@ -198,6 +207,9 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__
   int* s_off = s_ch + MAX_E;                               // [MAX_E] first padded row
   int* s_cnt = s_off + MAX_E;                              // [MAX_E] rows
   float* s_tr = reinterpret_cast<float*>(s_cnt + MAX_E);   // [EPI_WARPS][TR_FLOATS]
+  // [EPI_WARPS][2] output staging tiles (tile-store configurations), 128-byte aligned
+  float* s_out = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(s_tr + EPI_WARPS * TR_FLOATS) + 127) &
+                                          ~uintptr_t(127));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = p.E;
@@ -539,6 +551,10 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__
     // item later (or at the end), so the fence that orders them before the count finds them
     // drained instead of stalling the epilogue.
     int pending = -1;
+    // down output through staging tiles and tile stores (slot rows in expert order, unweighted)
+    const bool tile_out = C::OUT_TMA && p.slots_by_row && p.accum == nullptr;
+    float* out_tiles = s_out + (warp - 2) * 2 * (C::OUT_TILE_BYTES / 4);
+    uint32_t out_seq = 0;  // tile stores this warp has issued
     auto release_pending = [&]() {
       if (EPI == EPI_FUSED && pending >= 0) {
         __threadfence();
@@ -563,13 +579,15 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__
         sh = p.h_scale[w.e];
       } else {
         sc = p.h_scale[w.e] * p.w2_scale[w.e];
+        if (!tile_out) {
 #pragma unroll
-        for (int c2 = 0; c2 < C::MAX_CHUNKS / 2; ++c2) {
-          const int tok = (2 * c2 + half) * 32 + lane;
-          pr[c2] = tok < w.n_rows ? p.row_pair[w.r0 + tok] : -1;
+          for (int c2 = 0; c2 < C::MAX_CHUNKS / 2; ++c2) {
+            const int tok = (2 * c2 + half) * 32 + lane;
+            pr[c2] = tok < w.n_rows ? p.row_pair[w.r0 + tok] : -1;
+          }
+#pragma unroll
+          for (int c2 = 0; c2 < C::MAX_CHUNKS / 2; ++c2) wt[c2] = pr[c2] >= 0 ? p.topk_w[pr[c2]] * sc : 0.0f;
         }
-#pragma unroll
-        for (int c2 = 0; c2 < C::MAX_CHUNKS / 2; ++c2) wt[c2] = pr[c2] >= 0 ? p.topk_w[pr[c2]] * sc : 0.0f;
       }
       release_pending();
       if (!mbar_wait(&acc_full[ab], (li / C::NACC) & 1)) {
@@ -621,6 +639,41 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__
         }
         if (EPI == EPI_FUSED) pending = w.e;  // counted once its stores have drained
       } else {
+        if (tile_out) {
+          // Each 16-token half of a chunk: this quarter's 32 rows x 16 tokens, scaled by
+          // s_h * s_w2, are parked row-major in one of the warp's two staging tiles and stored
+          // by one lane with a tile store into the tokens' slot rows (expert order), which the
+          // combine weights and sums.  A tile is rewritten only once the store issued from it
+          // two steps earlier has read it.
+#pragma unroll 1
+          for (int c2 = 0; c2 < C::MAX_CHUNKS / 2; ++c2) {
+            const int cc = 2 * c2 + half;
+            if (cc * 32 >= w.N) break;
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(trow + ab * C::ACC_COLS + cc * 32, r);
+            tmem_ld_wait();
+            const int nj = min(32, w.n_rows - cc * 32);
+#pragma unroll
+            for (int sub = 0; sub < 2; ++sub) {
+              if (sub * 16 >= nj) break;
+              float* tile = out_tiles + (out_seq & 1u) * (C::OUT_TILE_BYTES / 4);
+              if (lane == 0 && out_seq >= 2) bulk_wait_group_read<1>();
+              __syncwarp();
+#pragma unroll
+              for (int t = 0; t < 16; ++t) tile[t * 32 + lane] = __uint_as_float(r[sub * 16 + t]) * sc;
+              fence_proxy_async_shared();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&tmO, w.mt * WM + q * 32, w.r0 + cc * 32 + sub * 16, tile);
+                bulk_commit_group();
+              }
+              ++out_seq;
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(&acc_empty[ab]);
+          continue;
+        }
         // A chunk's 32 token columns go through the warp's transpose tile in two halves of 16
         // tokens: lanes (= weight rows) park their accumulators, then each store instruction of
         // the warp covers 4 tokens x the quarter's 32 rows, 128 contiguous bytes per token
@@ -678,6 +731,7 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__
       mbar_arrive(&acc_empty[ab]);
     }
     release_pending();
+    if (tile_out && lane == 0) bulk_wait_group<0>();  // the tile stores are complete before exit
   }
 
   tc_fence_before();
@@ -691,7 +745,8 @@ struct Maps {
 };
 
 template <int EPI, class C>
-nvfp4moe_status launch_cfg(const Maps& m0, const Maps& m1, const GroupedParams& p, int64_t max_items, cudaStream_t s) {
+nvfp4moe_status launch_cfg(const Maps& m0, const Maps& m1, const CUtensorMap& out, const GroupedParams& p,
+                           int64_t max_items, cudaStream_t s) {
   auto kern = grouped_kernel<EPI, C>;
   static int configured[64] = {0};
   int dev = 0;
@@ -704,7 +759,7 @@ nvfp4moe_status launch_cfg(const Maps& m0, const Maps& m1, const GroupedParams& 
   int64_t grid = num_sms();
   if (max_items < grid) grid = max_items > 0 ? max_items : 1;
   const cudaError_t e = launch_dependent(kern, dim3(static_cast<unsigned>(grid)), dim3(kThreads), C::SMEM_BYTES, s,
-                                         m0.w, m0.x, m0.xs, m1.w, m1.x, m1.xs, p);
+                                         m0.w, m0.x, m0.xs, m1.w, m1.x, m1.xs, out, p);
   if (e != cudaSuccess) return fail(NVFP4MOE_CUDA_ERROR, "grouped tcgen05 GEMM: %s", cudaGetErrorString(e));
   return check_launch("grouped tcgen05 GEMM");
 }
@@ -764,6 +819,13 @@ nvfp4moe_status launch_grouped_ffn(const GemmFfnArgs& a, cudaStream_t s) {
   p.topk_w = a.topk_w;
   p.slots = static_cast<float*>(a.slots_f32);
   p.accum = a.accum;
+  // wide tiling, ordered combine: the down epilogue stores tiles into slot rows in expert order
+  CUtensorMap out_map = d.w;  // unused unless tile stores are on
+  p.slots_by_row = (!decode && a.slots_by_row && a.accum == nullptr) ? 1 : 0;
+  if (p.slots_by_row) {
+    st = make_f32_rows_map(&out_map, a.slots_f32, a.rows_cap, a.H, 32, 16);
+    if (st != NVFP4MOE_OK) return st;
+  }
   p.k = a.k;
   p.H = a.H;
   auto mark4 = [&]() -> nvfp4moe_status {
@@ -787,7 +849,7 @@ nvfp4moe_status launch_grouped_ffn(const GemmFfnArgs& a, cudaStream_t s) {
     p.list_cap = a.list_cap;
     p.done = a.done;
     p.done_target = EPI_WARPS * wt_g;
-    st = launch_cfg<EPI_FUSED, CfgDecode>(g, d, p, fused_items, s);
+    st = launch_cfg<EPI_FUSED, CfgDecode>(g, d, out_map, p, fused_items, s);
     if (st != NVFP4MOE_OK) return st;
     return mark4();  // one launch: the gate/up stage holds both GEMMs
   }
@@ -798,15 +860,16 @@ nvfp4moe_status launch_grouped_ffn(const GemmFfnArgs& a, cudaStream_t s) {
                      (cap_d + grid_d - 1) / grid_d <= SCHED_CAP;
     p.list = use ? a.list : nullptr;
     p.list_cap = cap_g;
-    st = launch_cfg<EPI_GATEUP, CfgDecode>(g, g, p, items_g, s);
+    st = launch_cfg<EPI_GATEUP, CfgDecode>(g, g, out_map, p, items_g, s);
     if (st == NVFP4MOE_OK) st = mark4();
     p.list_cap = cap_d;
-    if (st == NVFP4MOE_OK) st = launch_cfg<EPI_DOWN, CfgDecode>(d, d, p, items_d, s);
+    if (st == NVFP4MOE_OK) st = launch_cfg<EPI_DOWN, CfgDecode>(d, d, out_map, p, items_d, s);
     return st;
   }
-  st = launch_cfg<EPI_GATEUP, CfgWide>(g, g, p, max_items(P, a.E, CfgWide::BNMAX, wt_g), s);
+  st = launch_cfg<EPI_GATEUP, CfgWide>(g, g, out_map, p, max_items(P, a.E, CfgWide::BNMAX, wt_g), s);
   if (st == NVFP4MOE_OK) st = mark4();
-  if (st == NVFP4MOE_OK) st = launch_cfg<EPI_DOWN, CfgWide>(d, d, p, max_items(P, a.E, CfgWide::BNMAX, wt_d), s);
+  if (st == NVFP4MOE_OK)
+    st = launch_cfg<EPI_DOWN, CfgWideDown>(d, d, out_map, p, max_items(P, a.E, CfgWideDown::BNMAX, wt_d), s);
   return st;
 }
 
