@@ -91,7 +91,7 @@ enum {
 /* Message for the last failing call on this host thread ("" if none). */
 const char* nvfp4moe_last_error(void);
 
-/* Library version, e.g. 0x000300 = 0.3.0. */
+/* Library version, e.g. 0x000400 = 0.4.0. */
 int32_t nvfp4moe_version(void);
 
 /* Waits for `stream`, then returns the sticky device status word of the current device
@@ -250,6 +250,10 @@ typedef struct {
    * gate/up GEMM, [5] after the down GEMM, [6] after the combine. */
   void* const* stage_events;
   int32_t combine;            /* NVFP4MOE_COMBINE_* */
+  /* NVFP4MOE_SCALE_GIVEN: h is requantised with h_scale[e] (a calibrated constant);
+   * NVFP4MOE_SCALE_DYNAMIC: with amax(h of expert e in this call) / 2688, h_scale unused
+   * (tensor-core path only; h_amax, when given, receives those maxima as well). */
+  int32_t h_scale_mode;
 } moe_ffn_desc;
 
 enum { NVFP4MOE_STAGES = 7 };
@@ -267,6 +271,8 @@ typedef struct {
   int32_t path;     /* resolved path */
   int32_t combine;  /* resolved combine mode; ACCUMULATE: the accumulator is at `slots` */
   int32_t reserved;
+  int64_t h_f32;    /* dynamic h scale: fp32 h [h_rows][I] before requantisation */
+  int64_t h_stats;  /* dynamic h scale: amax[E] then the scales used, s_h[E] (fp32) */
 } moe_ffn_ws_layout;
 
 nvfp4moe_status moe_ffn_workspace_layout(const moe_ffn_desc* d, moe_ffn_ws_layout* layout);

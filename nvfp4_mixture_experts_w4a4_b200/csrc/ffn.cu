@@ -31,6 +31,8 @@ nvfp4moe_status check_desc(const moe_ffn_desc* d, const char* fn) {
                 NVFP4MOE_INVALID_ARG, "%s: bad x_scale_mode", fn);
   NVFP4_REQUIRE(d->combine >= NVFP4MOE_COMBINE_AUTO && d->combine <= NVFP4MOE_COMBINE_ACCUMULATE,
                 NVFP4MOE_INVALID_ARG, "%s: bad combine mode %d", fn, d->combine);
+  NVFP4_REQUIRE(d->h_scale_mode == NVFP4MOE_SCALE_GIVEN || d->h_scale_mode == NVFP4MOE_SCALE_DYNAMIC,
+                NVFP4MOE_INVALID_ARG, "%s: bad h_scale_mode", fn);
   return NVFP4MOE_OK;
 }
 
@@ -92,9 +94,10 @@ void make_layout(const moe_ffn_desc* d, moe_ffn_ws_layout* L) {
   L->h_rows = path == NVFP4MOE_PATH_GEMM ? rows_cap : P;
   L->h_codes = take(L->h_rows * I / 2);
   L->h_sf = take(sf_mma_bytes(L->h_rows, I));
-  // per-slot rows of the down projection: fp32 split-K partials on the GEMV path, bf16 on
-  // the tensor-core path (halves the slot round trip of large prefills)
-  // (the region also holds the batch prologue's slice histograms until the down GEMM)
+  // fp32 rows of the down projection: split-K partials by pair on the GEMV path; on the
+  // tensor-core path rows by pair (up to 64 tokens) or by padded expert row (above), or the
+  // [T][H] accumulator of the accumulating combine (the region also holds the batch
+  // prologue's slice histograms until the down GEMM)
   const int combine = resolve_combine(d, path);
   const int64_t prologue_scratch = batch_prologue_scratch_bytes(d->T, d->E);
   L->combine = combine;
@@ -111,6 +114,10 @@ void make_layout(const moe_ffn_desc* d, moe_ffn_ws_layout* L) {
   L->items = take(path == NVFP4MOE_PATH_GEMM && prologue_fits(d->T, d->E, d->top_k)
                       ? grouped_fused_list_entries(A, 2 * I / 128, H / 128) * 16 + E * 4
                       : 0);
+  // dynamic h scale: fp32 h before requantisation, per-expert amax and scale
+  const bool dyn_h = d->h_scale_mode == NVFP4MOE_SCALE_DYNAMIC;
+  L->h_f32 = take(dyn_h ? L->h_rows * I * 4 : 0);
+  L->h_stats = take(dyn_h ? 2 * E * 4 : 0);
   L->total = o;
 }
 
@@ -143,8 +150,7 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   if (st != NVFP4MOE_OK) return st;
   if (d->T == 0) return NVFP4MOE_OK;
   NVFP4_REQUIRE(x && logits && out && workspace, NVFP4MOE_INVALID_ARG, "%s: NULL pointer", fn);
-  NVFP4_REQUIRE(d->w13_codes && d->w13_sf && d->w13_scale && d->w2_codes && d->w2_sf && d->w2_scale &&
-                    d->h_scale,
+  NVFP4_REQUIRE(d->w13_codes && d->w13_sf && d->w13_scale && d->w2_codes && d->w2_sf && d->w2_scale,
                 NVFP4MOE_INVALID_ARG, "%s: NULL weight pointer in desc", fn);
   NVFP4_REQUIRE(d->x_scale_mode == NVFP4MOE_SCALE_DYNAMIC || d->x_scale != nullptr, NVFP4MOE_INVALID_ARG,
                 "%s: GIVEN x scale needs desc->x_scale", fn);
@@ -163,6 +169,10 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   }
   NVFP4_REQUIRE(L.combine != NVFP4MOE_COMBINE_ACCUMULATE || L.path == NVFP4MOE_PATH_GEMM, NVFP4MOE_UNSUPPORTED_SHAPE,
                 "%s: the accumulating combine needs the tensor-core path", fn);
+  const bool dyn_h = d->h_scale_mode == NVFP4MOE_SCALE_DYNAMIC;
+  NVFP4_REQUIRE(!dyn_h || L.path == NVFP4MOE_PATH_GEMM, NVFP4MOE_UNSUPPORTED_SHAPE,
+                "%s: the dynamic h scale needs the tensor-core path", fn);
+  NVFP4_REQUIRE(dyn_h || d->h_scale != nullptr, NVFP4MOE_INVALID_ARG, "%s: GIVEN h scale needs desc->h_scale", fn);
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   auto I32 = [&](int64_t off) { return reinterpret_cast<int32_t*>(ws + off); };
@@ -190,13 +200,16 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   const bool accumulate = L.combine == NVFP4MOE_COMBINE_ACCUMULATE;
   float* accum = F32(L.slots);  // fp32 [T][H] when accumulating
   uint8_t* prologue_scratch = ws + L.slots + prologue_scratch_offset(d, L.combine);
+  // dynamic h scale: per-expert amax of h over this call, then the scales derived from it
+  float* h_amax_int = dyn_h ? F32(L.h_stats) : d->h_amax;
+  float* h_scale_dyn = dyn_h ? F32(L.h_stats) + E : nullptr;
 
   mark(0);
   if (fused) {
     // small batch: routing, permutation and x quantisation in one cluster launch
     st = launch_prologue(x, logits, T, H, E, k, L.m_tile, dyn ? 1 : 0, xs, I32(L.topk_ids), F32(L.topk_w),
                          I32(L.counts), I32(L.offsets), I32(L.padded_offsets), I32(L.pair_to_row), I32(L.row_token),
-                         I32(L.row_pair), I32(L.tile_expert), I32(L.active), d->h_amax,
+                         I32(L.row_pair), I32(L.tile_expert), I32(L.active), h_amax_int,
                          L.path == NVFP4MOE_PATH_GEMM ? 1 : 0, ws + L.x_codes, ws + L.x_sf, lists ? list : nullptr,
                          lists ? done : nullptr, 2 * I / 128, H / 128, s);
     if (st != NVFP4MOE_OK) return st;
@@ -206,7 +219,7 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
     // larger batch: slices of 32 tokens; x is quantised straight into its rows
     st = launch_batch_prologue(x, logits, T, H, E, k, L.m_tile, dyn ? 1 : 0, xs, I32(L.topk_ids), F32(L.topk_w),
                                I32(L.counts), I32(L.offsets), I32(L.padded_offsets), I32(L.pair_to_row),
-                               I32(L.row_token), I32(L.row_pair), I32(L.tile_expert), I32(L.active), d->h_amax,
+                               I32(L.row_token), I32(L.row_pair), I32(L.tile_expert), I32(L.active), h_amax_int,
                                L.path == NVFP4MOE_PATH_GEMM ? 1 : 0, ws + L.x_codes, ws + L.x_sf, prologue_scratch,
                                accumulate ? accum : nullptr, d->stage_events, s);
     if (st != NVFP4MOE_OK) return st;
@@ -255,8 +268,12 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   a.row_token = I32(L.row_token); a.row_pair = I32(L.row_pair);
   a.w13_codes = d->w13_codes; a.w13_sf = d->w13_sf; a.w13_scale = d->w13_scale;
   a.w2_codes = d->w2_codes; a.w2_sf = d->w2_sf; a.w2_scale = d->w2_scale;
-  a.h_scale = d->h_scale; a.h_amax = d->h_amax;
+  a.h_scale = dyn_h ? h_scale_dyn : d->h_scale; a.h_amax = h_amax_int;
   a.h_codes = ws + L.h_codes; a.h_sf = ws + L.h_sf;
+  a.h_f32 = dyn_h ? F32(L.h_f32) : nullptr;
+  a.h_amax_user = dyn_h ? d->h_amax : nullptr;
+  a.tile_expert = I32(L.tile_expert);
+  a.m_tile_log2 = __builtin_ctz(unsigned(L.m_tile));
   a.topk_w = F32(L.topk_w); a.slots_f32 = ws + L.slots;
   a.stage_events = d->stage_events;
   a.list = lists ? list : nullptr;

@@ -41,7 +41,22 @@ struct GemmFfnArgs {
   float* accum;                   // nullable [T][H] fp32: the down GEMM adds its rows here (zeroed)
   int slots_by_row;               // batches above 64 tokens, ordered combine: slots_f32 is
                                   // [rows_cap][H], rows in padded expert order, unweighted
+  // dynamic h scale (h_f32 non-null): gate/up writes h in fp32 and its per-expert amax into
+  // h_amax (zeroed); then h is requantised with h_scale[e] = h_amax[e] / 2688, which this
+  // step writes, and h_amax_user (nullable) receives the maxima
+  float* h_f32;
+  float* h_amax_user;
+  const int32_t* tile_expert;
+  int m_tile_log2;
 };
+
+// Requantises fp32 h rows (the rows of padded expert order that hold a pair) with the
+// per-expert scale amax / 2688; writes the scales to h_scale and, when h_amax_user is
+// non-null, copies the maxima there.  A programmatic dependent of the gate/up GEMM.
+nvfp4moe_status launch_requant_h(const float* h_f32, int64_t rows_cap, int I, int E, const int32_t* padded_offsets,
+                                 const int32_t* row_pair, const int32_t* tile_expert, int m_tile_log2,
+                                 const float* h_amax, float* h_amax_user, float* h_scale, uint8_t* h_codes,
+                                 uint8_t* h_sf, cudaStream_t s);
 
 bool gemm_path_available();
 int grouped_token_align();

@@ -102,6 +102,7 @@ struct GroupedParams {
   float* h_amax;
   uint8_t* h_codes;
   uint8_t* h_sf;
+  float* h_f32;      // nullable: dynamic h scale, h goes out in fp32 [rows][I] (and its amax)
   int I;
   // down
   const float* w2_scale;
@@ -624,11 +625,19 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__
             float amax = 0.0f;
 #pragma unroll
             for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(hb[i]));
-            float inv;
-            const uint32_t sf = block_scale(amax, sh, &inv);
             const int64_t row = int64_t(w.r0) + tok;
-            *reinterpret_cast<uint2*>(p.h_codes + row * (p.I / 2) + iblk * 8) = encode_block16(hb, inv);
-            p.h_sf[sf_mma_offset(row, iblk, p.I)] = static_cast<uint8_t>(sf);
+            if (p.h_f32) {
+              // dynamic h scale: the block goes out in fp32; it is requantised once the
+              // expert's amax over the whole call is known
+              float4* dst = reinterpret_cast<float4*>(p.h_f32 + row * p.I + iblk * 16);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) dst[i] = make_float4(hb[4 * i], hb[4 * i + 1], hb[4 * i + 2], hb[4 * i + 3]);
+            } else {
+              float inv;
+              const uint32_t sf = block_scale(amax, sh, &inv);
+              *reinterpret_cast<uint2*>(p.h_codes + row * (p.I / 2) + iblk * 8) = encode_block16(hb, inv);
+              p.h_sf[sf_mma_offset(row, iblk, p.I)] = static_cast<uint8_t>(sf);
+            }
             amax_all = fmaxf(amax_all, amax);
           }
         }
@@ -814,6 +823,7 @@ nvfp4moe_status launch_grouped_ffn(const GemmFfnArgs& a, cudaStream_t s) {
   p.h_amax = a.h_amax;
   p.h_codes = a.h_codes;
   p.h_sf = a.h_sf;
+  p.h_f32 = a.h_f32;
   p.I = a.I;
   p.w2_scale = a.w2_scale;
   p.topk_w = a.topk_w;
@@ -844,7 +854,13 @@ nvfp4moe_status launch_grouped_ffn(const GemmFfnArgs& a, cudaStream_t s) {
   // SMs that gate/up frees and streams its first weight tiles meanwhile.
   const bool fits = [&](int64_t cap, int64_t grid) { return (cap + grid - 1) / grid <= SCHED_CAP; }(
       a.list_cap, fused_grid);
-  if (decode && a.list != nullptr && a.done != nullptr && wt_d <= wt_g && fits) {
+  auto requant = [&]() -> nvfp4moe_status {
+    return a.h_f32 ? launch_requant_h(a.h_f32, a.rows_cap, a.I, a.E, a.padded_offsets, a.row_pair, a.tile_expert,
+                                      a.m_tile_log2, a.h_amax, a.h_amax_user, const_cast<float*>(a.h_scale), a.h_codes,
+                                      a.h_sf, s)
+                   : NVFP4MOE_OK;
+  };
+  if (decode && a.list != nullptr && a.done != nullptr && wt_d <= wt_g && fits && a.h_f32 == nullptr) {
     p.list = a.list;
     p.list_cap = a.list_cap;
     p.done = a.done;
@@ -862,12 +878,14 @@ nvfp4moe_status launch_grouped_ffn(const GemmFfnArgs& a, cudaStream_t s) {
     p.list_cap = cap_g;
     st = launch_cfg<EPI_GATEUP, CfgDecode>(g, g, out_map, p, items_g, s);
     if (st == NVFP4MOE_OK) st = mark4();
+    if (st == NVFP4MOE_OK) st = requant();
     p.list_cap = cap_d;
     if (st == NVFP4MOE_OK) st = launch_cfg<EPI_DOWN, CfgDecode>(d, d, out_map, p, items_d, s);
     return st;
   }
   st = launch_cfg<EPI_GATEUP, CfgWide>(g, g, out_map, p, max_items(P, a.E, CfgWide::BNMAX, wt_g), s);
   if (st == NVFP4MOE_OK) st = mark4();
+  if (st == NVFP4MOE_OK) st = requant();
   if (st == NVFP4MOE_OK)
     st = launch_cfg<EPI_DOWN, CfgWideDown>(d, d, out_map, p, max_items(P, a.E, CfgWideDown::BNMAX, wt_d), s);
   return st;

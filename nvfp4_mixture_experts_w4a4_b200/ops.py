@@ -188,11 +188,13 @@ class NVFP4Experts:
 class MoeFFN:
     """The routed NVFP4 W4A4 feed-forward layer (moe_ffn_forward) with a cached workspace."""
 
-    def __init__(self, experts: NVFP4Experts, top_k: int, h_scale: torch.Tensor, x_scale: torch.Tensor | None = None,
-                 path: int = C.PATH_AUTO, combine: int = C.COMBINE_AUTO):
+    def __init__(self, experts: NVFP4Experts, top_k: int, h_scale: torch.Tensor | None,
+                 x_scale: torch.Tensor | None = None, path: int = C.PATH_AUTO, combine: int = C.COMBINE_AUTO):
+        """h_scale: per-expert requantisation scales of h, or None for the dynamic scale
+        (amax of each expert's h in the call / 2688; tensor-core path)."""
         self.w = experts
         self.top_k = top_k
-        self.h_scale = h_scale.to(torch.float32).contiguous()
+        self.h_scale = None if h_scale is None else h_scale.to(torch.float32).contiguous()
         self.x_scale = None if x_scale is None else x_scale.to(torch.float32).contiguous().view(1)
         self.path = path
         self.combine = combine
@@ -208,7 +210,8 @@ class MoeFFN:
         d.x_scale = None if self.x_scale is None else self.x_scale.data_ptr()
         d.w13_codes, d.w13_sf, d.w13_scale = w.w13_codes.data_ptr(), w.w13_sf.data_ptr(), w.w13_scale.data_ptr()
         d.w2_codes, d.w2_sf, d.w2_scale = w.w2_codes.data_ptr(), w.w2_sf.data_ptr(), w.w2_scale.data_ptr()
-        d.h_scale = self.h_scale.data_ptr()
+        d.h_scale = None if self.h_scale is None else self.h_scale.data_ptr()
+        d.h_scale_mode = C.SCALE_DYNAMIC if self.h_scale is None else C.SCALE_GIVEN
         d.h_amax = None if h_amax is None else h_amax.data_ptr()
         d.stage_events = None if events is None else ctypes.cast(events, ctypes.c_void_p).value
         return d
@@ -262,8 +265,12 @@ class MoeFFN:
             nbytes = n * torch.tensor([], dtype=dtype).element_size()
             return ws[off:off + nbytes].view(dtype)
 
+        dyn_h = self.h_scale is None
         return dict(
             path=L.path, m_tile=L.m_tile, combine=L.combine,
+            # the scales h was requantised with: given, or derived in the call (amax / 2688)
+            h_scale=view(L.h_stats + 4 * w.E, w.E, torch.float32) if dyn_h else self.h_scale,
+            h_amax=view(L.h_stats, w.E, torch.float32) if dyn_h else None,
             topk_ids=view(L.topk_ids, P, torch.int32).view(T, k),
             topk_w=view(L.topk_w, P, torch.float32).view(T, k),
             counts=view(L.counts, w.E, torch.int32), offsets=view(L.offsets, w.E + 1, torch.int32),

@@ -119,8 +119,10 @@ def experts_from_oracle(wg, wu, wd, dev) -> ops.NVFP4Experts:
 
 
 def run_layer_pair(wl: W.Workload, path: int, seed: int = 0, dev=None, given_x_scale: bool = False,
-                   combine: int = C.COMBINE_AUTO):
-    """Runs oracle and library on the same inputs; returns (oracle result, gpu out, layer)."""
+                   combine: int = C.COMBINE_AUTO, dynamic_h: bool = False):
+    """Runs oracle and library on the same inputs; returns (oracle result, gpu out, layer).
+    The oracle calibrates s_h (amax of each expert's h / 2688); the library is given those
+    scales, or with dynamic_h derives its own in the call."""
     dev = dev or need_gpu()
     act, wts, wg, wu, wd = layer_inputs(wl, seed)
     x_bits = bf16_bits(act["x"])
@@ -130,7 +132,7 @@ def run_layer_pair(wl: W.Workload, path: int, seed: int = 0, dev=None, given_x_s
         xs = float(np.float32(np.abs(bits_to_f32(x_bits)).max()) / np.float32(2688) * np.float32(1.5))
     ref = O.moe_ffn(x_bits, logits, wl.k, wg, wu, wd, x_scale=xs)
     experts = experts_from_oracle(wg, wu, wd, dev)
-    layer = ops.MoeFFN(experts, wl.k, torch.from_numpy(ref["h_scale"]).to(dev),
+    layer = ops.MoeFFN(experts, wl.k, None if dynamic_h else torch.from_numpy(ref["h_scale"]).to(dev),
                        x_scale=None if xs is None else torch.tensor([xs], device=dev), path=path, combine=combine)
     h_amax = torch.empty(wl.E, dtype=torch.float32, device=dev)
     out = layer(act["x"].to(dev), act["logits"].to(dev), h_amax=h_amax)

@@ -48,7 +48,7 @@ def test_binding_declares_every_symbol():
 
 def test_argument_errors_are_statuses(so):
     from nvfp4_mixture_experts_w4a4_b200 import _lib as C
-    assert so.nvfp4moe_version() == 0x000300
+    assert so.nvfp4moe_version() == 0x000400
     # bad E, bad k: rejected before any device work
     assert so.moe_route(None, 4, 2000, 2, None, None, None) == C.UNSUPPORTED_SHAPE
     assert b"E=2000" in so.nvfp4moe_last_error()

@@ -160,3 +160,24 @@ def test_accumulate_needs_the_tensor_core_path():
     wl = CASES["long_prefill_small"]
     with pytest.raises(C.Nvfp4MoeError):
         G.run_layer_pair(wl, C.PATH_GEMV, combine=C.COMBINE_ACCUMULATE)
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode_shape", "decode_T1", "prefill_chunk_small", "long_prefill_small",
+                                  "dense_small", "popular_expert_chunks", "slices_E1024_k32"])
+def test_layer_dynamic_h_scale(name):
+    """Dynamic per-expert h scale: the library derives s_h[e] = amax_e(h) / 2688 inside the
+    call (h leaves the gate/up GEMM in fp32, then is requantised) and meets the same
+    tolerances against the oracle's calibrating run; experts without tokens keep scale 1."""
+    wl = GEMM_CASES[name]
+    ref, out, layer, h_amax = G.run_layer_pair(wl, C.PATH_GEMM, dynamic_h=True)
+    im = layer.intermediates(wl.T)
+    used = ref["counts"] > 0
+    s_dev = im["h_scale"].cpu().numpy()
+    np.testing.assert_allclose(s_dev[used], ref["h_scale"][used], rtol=1e-4)
+    assert (s_dev[~used] == 1.0).all()
+    # the scale is the maximum divided by 2688, rounded once
+    a_dev = im["h_amax"].cpu().numpy()
+    assert np.array_equal(s_dev[used], a_dev[used] / np.float32(2688))
+    assert np.array_equal(h_amax.cpu().numpy()[used], a_dev[used])
+    G.check_layer(wl, ref, out, layer, h_amax)
+    assert ops.device_status() == 0
