@@ -251,8 +251,10 @@ typedef struct {
   void* const* stage_events;
   int32_t combine;            /* NVFP4MOE_COMBINE_* */
   /* NVFP4MOE_SCALE_GIVEN: h is requantised with h_scale[e] (a calibrated constant);
-   * NVFP4MOE_SCALE_DYNAMIC: with amax(h of expert e in this call) / 2688, h_scale unused
-   * (tensor-core path only; h_amax, when given, receives those maxima as well). */
+   * NVFP4MOE_SCALE_DYNAMIC: with amax(h of expert e in this call) / 2688 (1 for an expert
+   * without tokens), h_scale unused; the scales used are left in the workspace at
+   * layout.h_stats + 4*E (tensor-core path only, else NVFP4MOE_UNSUPPORTED_SHAPE; h_amax,
+   * when given, receives the maxima as well).  NVFP4 pretraining paper, two-level scaling. */
   int32_t h_scale_mode;
 } moe_ffn_desc;
 
