@@ -254,7 +254,7 @@ typedef struct {
    * NVFP4MOE_SCALE_DYNAMIC: with amax(h of expert e in this call) / 2688 (1 for an expert
    * without tokens), h_scale unused; the scales used are left in the workspace at
    * layout.h_stats + 4*E (tensor-core path only, else NVFP4MOE_UNSUPPORTED_SHAPE; h_amax,
-   * when given, receives the maxima as well).  NVFP4 pretraining paper, two-level scaling. */
+   * when given, receives the maxima as well). */
   int32_t h_scale_mode;
 } moe_ffn_desc;
 

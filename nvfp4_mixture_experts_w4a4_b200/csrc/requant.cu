@@ -2,9 +2,10 @@
 // the amax of each expert's h over the call; here every row of padded expert order that holds
 // a (token, expert) pair is quantised once that amax is known, with s_h[e] = amax_e / 2688 and
 // the same block quantiser (E4M3 block scales, E2M1 codes, MMA scale layout) as the gate/up
-// epilogue uses for a given scale (NVFP4 pretraining paper, section on the two-level scaling:
-// the tensor scale maps the tensor's amax onto the largest E2M1 value times the largest E4M3
-// block scale, 6 x 448 = 2688).
+// epilogue uses for a given scale.  The tensor scale maps the amax onto the largest E2M1
+// value times the largest E4M3 block scale, 6 x 448 = 2688, as for the layer input (the
+// two-level NVFP4 scaling of the Qwen3.8-Flash-Next-NVFP4-SSD-Stream model card, "What this
+// model is", read as a dynamic per-tensor scale).
 #include "ffn_gemm.cuh"
 
 namespace nvfp4moe {
