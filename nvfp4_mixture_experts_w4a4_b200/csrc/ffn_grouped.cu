@@ -554,6 +554,9 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__
     int pending = -1;
     // down output through staging tiles and tile stores (slot rows in expert order, unweighted)
     const bool tile_out = C::OUT_TMA && p.slots_by_row && p.accum == nullptr;
+    // accumulating with the staging tiles: each token's 32 weighted rows are added into its
+    // output row by one bulk reduction (L2 performs the fp32 adds)
+    const bool tile_red = C::OUT_TMA && p.accum != nullptr;
     float* out_tiles = s_out + (warp - 2) * 2 * (C::OUT_TILE_BYTES / 4);
     uint32_t out_seq = 0;  // tile stores this warp has issued
     auto release_pending = [&]() {
@@ -683,6 +686,40 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__
           mbar_arrive(&acc_empty[ab]);
           continue;
         }
+        if (tile_red) {
+          // As above, but each row is scaled by its token's routing weight and lanes 0..15
+          // each add one token's 32 values (128 bytes) into the token's accumulator row.
+#pragma unroll 1
+          for (int c2 = 0; c2 < C::MAX_CHUNKS / 2; ++c2) {
+            const int cc = 2 * c2 + half;
+            if (cc * 32 >= w.N) break;
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(trow + ab * C::ACC_COLS + cc * 32, r);
+            tmem_ld_wait();
+            const int nj = min(32, w.n_rows - cc * 32);
+#pragma unroll
+            for (int sub = 0; sub < 2; ++sub) {
+              if (sub * 16 >= nj) break;
+              float* tile = out_tiles + (out_seq & 1u) * (C::OUT_TILE_BYTES / 4);
+              if (out_seq >= 2) bulk_wait_group_read<1>();
+              __syncwarp();
+#pragma unroll
+              for (int t = 0; t < 16; ++t)
+                tile[t * 32 + lane] = __uint_as_float(r[sub * 16 + t]) * __shfl_sync(0xffffffffu, wt[c2], sub * 16 + t);
+              fence_proxy_async_shared();
+              __syncwarp();
+              const int32_t pair = __shfl_sync(0xffffffffu, pr[c2], sub * 16 + (lane & 15));
+              if (lane < 16 && pair >= 0)
+                bulk_reduce_add_f32(p.accum + int64_t(pair / p.k) * p.H + int64_t(w.mt) * WM + q * 32, tile + lane * 32,
+                                    128u);
+              bulk_commit_group();
+              ++out_seq;
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(&acc_empty[ab]);
+          continue;
+        }
         // A chunk's 32 token columns go through the warp's transpose tile in two halves of 16
         // tokens: lanes (= weight rows) park their accumulators, then each store instruction of
         // the warp covers 4 tokens x the quarter's 32 rows, 128 contiguous bytes per token
@@ -740,7 +777,7 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__
       mbar_arrive(&acc_empty[ab]);
     }
     release_pending();
-    if (tile_out && lane == 0) bulk_wait_group<0>();  // the tile stores are complete before exit
+    if ((tile_out && lane == 0) || tile_red) bulk_wait_group<0>();  // the bulk writes are complete before exit
   }
 
   tc_fence_before();

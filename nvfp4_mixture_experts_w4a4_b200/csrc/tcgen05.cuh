@@ -72,6 +72,13 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int32_t x, 
                ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(src))
                : "memory");
 }
+// dst[i] += src[i] (fp32) over `bytes` bytes, performed at L2; both 16-byte aligned,
+// bytes % 16 == 0.  Completion is tracked like a tile store (bulk groups of this thread).
+__device__ __forceinline__ void bulk_reduce_add_f32(float* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;"
+               ::"l"(reinterpret_cast<uint64_t>(dst)), "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Waits until at most N of this thread's bulk groups still read shared memory.
 template <int N>
