@@ -51,6 +51,20 @@ class MoeArgs(ctypes.Structure):
     ]
 
 
+class MoeW4A16Args(ctypes.Structure):
+    _fields_ = [
+        ("T", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32),
+        ("E", ctypes.c_int32), ("k", ctypes.c_int32), ("nthreads", ctypes.c_int32),
+        ("x_bf16", _u16p), ("logits", _f32p),
+        ("wg_codes", _u8p), ("wg_sf", _u8p), ("wg_scale", _f32p),
+        ("wu_codes", _u8p), ("wu_sf", _u8p), ("wu_scale", _f32p),
+        ("wd_codes", _u8p), ("wd_sf", _u8p), ("wd_scale", _f32p),
+        ("out_bf16", _u16p), ("out_f64", _f64p),
+        ("ids", _i32p), ("w", _f32p), ("counts", _i32p), ("offsets", _i32p),
+        ("row_token", _i32p), ("pair_to_row", _i32p), ("h_bf16", _u16p), ("y_f64", _f64p),
+    ]
+
+
 def _declare(L):
     L.orc_e2m1_value.restype = ctypes.c_double
     L.orc_e2m1_value.argtypes = [ctypes.c_int]
@@ -82,6 +96,8 @@ def _declare(L):
                               _i32p, _i32p, _i32p]
     L.orc_moe_ffn.restype = ctypes.c_int
     L.orc_moe_ffn.argtypes = [ctypes.POINTER(MoeArgs)]
+    L.orc_moe_ffn_w4a16.restype = ctypes.c_int
+    L.orc_moe_ffn_w4a16.argtypes = [ctypes.POINTER(MoeW4A16Args)]
 
 
 def _p(a: np.ndarray | None, ctype):
@@ -284,4 +300,52 @@ def moe_ffn(x_bf16: np.ndarray, logits: np.ndarray, k: int, wg, wu, wd, *, x_sca
         raise ValueError(f"orc_moe_ffn failed ({rc})")
     r["x_scale"] = float(xs[0])
     r["h_scale"] = hs
+    return r
+
+
+def moe_ffn_w4a16(x_bf16: np.ndarray, logits: np.ndarray, k: int, wg, wu, wd, *,
+                  nthreads: int | None = None, want_y: bool = False) -> dict:
+    """The weight-only (W4A16) layer on the CPU (reading R10 of nvfp4_oracle.cpp): bf16 x
+    into the gate/up products, h rounded to bf16, NVFP4 weights dequantised, fp64 sums.
+    Arguments as for moe_ffn.  Returns out_bf16, out_f64, the routing and permutation, and
+    h_bf16 (uint16 [T*k, I], permuted rows)."""
+    x_bf16 = np.ascontiguousarray(x_bf16, np.uint16)
+    logits = np.ascontiguousarray(logits, np.float32)
+    T, H = x_bf16.shape
+    E = logits.shape[1]
+    I = wg[0].shape[1]
+    P = T * k
+    wg = [np.ascontiguousarray(v) for v in wg]
+    wu = [np.ascontiguousarray(v) for v in wu]
+    wd = [np.ascontiguousarray(v) for v in wd]
+    r = dict(
+        out_bf16=np.zeros((T, H), np.uint16), out_f64=np.zeros((T, H), np.float64),
+        ids=np.zeros((T, k), np.int32), w=np.zeros((T, k), np.float32),
+        counts=np.zeros(E, np.int32), offsets=np.zeros(E + 1, np.int32),
+        row_token=np.zeros(P, np.int32), pair_to_row=np.zeros(P, np.int32),
+        h_bf16=np.zeros((P, I), np.uint16),
+        y_f64=np.zeros((P, H), np.float64) if want_y else None,
+    )
+    a = MoeW4A16Args()
+    a.T, a.H, a.I, a.E, a.k = T, H, I, E, k
+    a.nthreads = nthreads or default_threads()
+    a.x_bf16 = _p(x_bf16, ctypes.c_uint16)
+    a.logits = _p(logits, ctypes.c_float)
+    a.wg_codes, a.wg_sf, a.wg_scale = (_p(wg[0], ctypes.c_uint8), _p(wg[1], ctypes.c_uint8),
+                                       _p(wg[2], ctypes.c_float))
+    a.wu_codes, a.wu_sf, a.wu_scale = (_p(wu[0], ctypes.c_uint8), _p(wu[1], ctypes.c_uint8),
+                                       _p(wu[2], ctypes.c_float))
+    a.wd_codes, a.wd_sf, a.wd_scale = (_p(wd[0], ctypes.c_uint8), _p(wd[1], ctypes.c_uint8),
+                                       _p(wd[2], ctypes.c_float))
+    for name, ct in (("out_bf16", ctypes.c_uint16), ("out_f64", ctypes.c_double),
+                     ("ids", ctypes.c_int32), ("w", ctypes.c_float), ("counts", ctypes.c_int32),
+                     ("offsets", ctypes.c_int32), ("row_token", ctypes.c_int32),
+                     ("pair_to_row", ctypes.c_int32), ("h_bf16", ctypes.c_uint16),
+                     ("y_f64", ctypes.c_double)):
+        setattr(a, name, _p(r[name], ct))
+    keep = (x_bf16, logits, wg, wu, wd, r)
+    rc = lib().orc_moe_ffn_w4a16(ctypes.byref(a))
+    del keep
+    if rc != 0:
+        raise ValueError(f"orc_moe_ffn_w4a16 failed ({rc})")
     return r

@@ -39,6 +39,10 @@
 //   R8 SwiGLU: h = silu(g) * u with silu(g) = g / (1 + exp(-g)).
 //   R9 combine: out[t] = sum over slots j = 0..k-1 (in order) of w[t][j] * y[t][j],
 //      rounded once to bf16 (fp64 -> fp32 -> bf16, each round to nearest even).
+//   R10 weight-only variant (W4A16; the NInfer card's "Limits" names NVFP4 weights without
+//      an activation-quantisation site): x enters the gate/up products as bf16, the
+//      intermediate h = silu(g) * u is rounded to bf16 (fp64 -> fp32 -> bf16) as the down
+//      projection's activation, weights are dequantised NVFP4; products and sums in fp64.
 //
 // Build: g++ -O2 -std=c++17 -ffp-contract=off -fPIC -shared -pthread (see build.py).
 // -ffp-contract=off keeps every fp32 step a separately rounded operation.
@@ -488,6 +492,127 @@ int orc_moe_ffn(const orc_moe_args* a) {
   put(a->h_codes, hc);
   put(a->h_sf, hs);
   put(a->h_amax, amax);
+  put(a->y_f64, y);
+  return 0;
+}
+
+
+// The weight-only (W4A16) layer, reading R10: routing, permutation and combine as in
+// orc_moe_ffn; the expert products use dequantised weights and bf16 activations.
+struct orc_moe_w4a16_args {
+  int32_t T, H, I, E, k;
+  int32_t nthreads;
+  const uint16_t* x_bf16;    // [T][H]
+  const float* logits;       // [T][E]
+  const uint8_t* wg_codes;   // [E][I][H/2]
+  const uint8_t* wg_sf;      // [E][I][H/16]
+  const float* wg_scale;     // [E]
+  const uint8_t* wu_codes;
+  const uint8_t* wu_sf;
+  const float* wu_scale;
+  const uint8_t* wd_codes;   // [E][H][I/2]
+  const uint8_t* wd_sf;      // [E][H][I/16]
+  const float* wd_scale;     // [E]
+  uint16_t* out_bf16;        // [T][H]
+  // optional outputs (nullable)
+  double* out_f64;           // [T][H], before the bf16 rounding
+  int32_t* ids;              // [T][k]
+  float* w;                  // [T][k]
+  int32_t* counts;           // [E]
+  int32_t* offsets;          // [E+1]
+  int32_t* row_token;        // [T*k]
+  int32_t* pair_to_row;      // [T*k]
+  uint16_t* h_bf16;          // [T*k][I], permuted rows
+  double* y_f64;             // [T*k][H], down projection per permuted row, before w
+};
+
+namespace {
+// Row r of an NVFP4 matrix with K columns as doubles: e2m1(code) * e4m3(sf) * s.
+void dequant_row(const uint8_t* codes, const uint8_t* sf, double s, int64_t r, int64_t K, double* out) {
+  for (int64_t c = 0; c < K; ++c) {
+    const int byte = codes[(r * K + c) / 2];
+    const int code = (c & 1) ? (byte >> 4) : (byte & 15);
+    out[c] = e2m1_value(code) * e4m3_value(sf[(r * K + c) / 16]) * s;
+  }
+}
+}  // namespace
+
+int orc_moe_ffn_w4a16(const orc_moe_w4a16_args* a) {
+  const int T = a->T, H = a->H, I = a->I, E = a->E, k = a->k;
+  if (H % 16 || I % 16 || k < 1 || k > E || T < 0) return -1;
+  const int64_t P = int64_t(T) * k;
+  const int nth = std::max(1, int(a->nthreads));
+
+  // 1. routing and permutation (R5, R6)
+  std::vector<int32_t> ids(static_cast<size_t>(P)), counts(static_cast<size_t>(E)), offsets(static_cast<size_t>(E) + 1),
+      row_token(static_cast<size_t>(P)), row_slot(static_cast<size_t>(P)), pair_to_row(static_cast<size_t>(P));
+  std::vector<float> w(static_cast<size_t>(P));
+  orc_route(a->logits, T, E, k, ids.data(), w.data());
+  if (orc_permute(ids.data(), T, E, k, counts.data(), offsets.data(), row_token.data(), row_slot.data(),
+                  pair_to_row.data()) != 0)
+    return -2;
+
+  // 2. gate/up with bf16 x and dequantised weights, SwiGLU (R8), h rounded to bf16 (R10)
+  std::vector<uint16_t> h(static_cast<size_t>(P * I));
+  parallel_for(E, nth, [&](int64_t e) {
+    if (counts[e] == 0) return;
+    std::vector<double> wg(static_cast<size_t>(int64_t(I) * H)), wu(static_cast<size_t>(int64_t(I) * H)),
+        x(static_cast<size_t>(H));
+    for (int64_t i = 0; i < I; ++i) {
+      dequant_row(a->wg_codes, a->wg_sf, a->wg_scale[e], e * I + i, H, &wg[size_t(i * H)]);
+      dequant_row(a->wu_codes, a->wu_sf, a->wu_scale[e], e * I + i, H, &wu[size_t(i * H)]);
+    }
+    for (int64_t r = offsets[e]; r < offsets[e + 1]; ++r) {
+      const int t = row_token[r];
+      for (int64_t c = 0; c < H; ++c) x[size_t(c)] = bf16_to_float(a->x_bf16[int64_t(t) * H + c]);
+      for (int64_t i = 0; i < I; ++i) {
+        double g = 0.0, u = 0.0;
+        for (int64_t c = 0; c < H; ++c) {
+          g += x[size_t(c)] * wg[size_t(i * H + c)];
+          u += x[size_t(c)] * wu[size_t(i * H + c)];
+        }
+        const double hv = g / (1.0 + std::exp(-g)) * u;
+        h[size_t(r * I + i)] = float_to_bf16(static_cast<float>(hv));
+      }
+    }
+  });
+
+  // 3. down projection per permuted row
+  std::vector<double> y(static_cast<size_t>(P * H));
+  parallel_for(E, nth, [&](int64_t e) {
+    if (counts[e] == 0) return;
+    std::vector<double> wd(static_cast<size_t>(int64_t(H) * I));
+    for (int64_t n = 0; n < H; ++n) dequant_row(a->wd_codes, a->wd_sf, a->wd_scale[e], e * H + n, I, &wd[size_t(n * I)]);
+    for (int64_t r = offsets[e]; r < offsets[e + 1]; ++r)
+      for (int64_t n = 0; n < H; ++n) {
+        double acc = 0.0;
+        for (int64_t i = 0; i < I; ++i) acc += double(bf16_to_float(h[size_t(r * I + i)])) * wd[size_t(n * I + i)];
+        y[size_t(r * H + n)] = acc;
+      }
+  });
+
+  // 4. weighted combine (R9)
+  for (int t = 0; t < T; ++t)
+    for (int64_t n = 0; n < H; ++n) {
+      double acc = 0.0;
+      for (int j = 0; j < k; ++j) {
+        const int64_t r = pair_to_row[size_t(int64_t(t) * k + j)];
+        acc += double(w[size_t(int64_t(t) * k + j)]) * y[size_t(r * H + n)];
+      }
+      if (a->out_f64) a->out_f64[int64_t(t) * H + n] = acc;
+      a->out_bf16[int64_t(t) * H + n] = float_to_bf16(static_cast<float>(acc));
+    }
+
+  auto put = [](auto* dst, const auto& src) {
+    if (dst) std::copy(src.begin(), src.end(), dst);
+  };
+  put(a->ids, ids);
+  put(a->w, w);
+  put(a->counts, counts);
+  put(a->offsets, offsets);
+  put(a->row_token, row_token);
+  put(a->pair_to_row, pair_to_row);
+  put(a->h_bf16, h);
   put(a->y_f64, y);
   return 0;
 }

@@ -363,3 +363,68 @@ def test_layer_expert_with_no_tokens_and_all_tokens_one_expert():
     assert list(r["row_token"]) == list(range(6))
     assert (r["w"] == 1.0).all()
     assert r["h_scale"][0] == 1.0 and r["h_scale"][2] > 0
+
+
+# ------------------------------------------------------- weight-only layer ----
+def _bf16_round(a):
+    """fp64 -> fp32 -> bf16 (round to nearest even at each step, by torch), as float64."""
+    t = torch.from_numpy(np.asarray(a, np.float64).astype(np.float32)).to(torch.bfloat16)
+    return t.to(torch.float64).numpy()
+
+
+def test_w4a16_layer_vs_direct_per_token_formulation():
+    """Weight-only variant against a per-token formulation: no permutation, weights
+    dequantised by the independent ml_dtypes formulation, fp64 matmuls, h rounded to bf16
+    by torch."""
+    wl, x, logits, wg, wu, wd = _tiny_layer_inputs(T=7, E=6, k=3)
+    r = O.moe_ffn_w4a16(x, logits, wl.k, wg, wu, wd, nthreads=2)
+    xf = ((x.astype(np.uint32) << 16).view(np.float32)).astype(np.float64)
+    ids = _ref_topk(logits, wl.k)
+    assert np.array_equal(r["ids"], ids)
+    ref = np.zeros((wl.T, wl.H))
+    for t in range(wl.T):
+        sel = logits[t, ids[t]].astype(np.float64)
+        wts = np.exp(sel - sel[0])
+        wts = (wts / wts.sum()).astype(np.float32).astype(np.float64)
+        for j in range(wl.k):
+            e = ids[t, j]
+            g = R.dequantize(wg[0][e], wg[1][e], wg[2][e]) @ xf[t]
+            u = R.dequantize(wu[0][e], wu[1][e], wu[2][e]) @ xf[t]
+            h = _bf16_round(g / (1 + np.exp(-g)) * u)
+            ref[t] += wts[j] * (R.dequantize(wd[0][e], wd[1][e], wd[2][e]) @ h)
+            row = r["pair_to_row"][t * wl.k + j]
+            hb = (r["h_bf16"][row].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+            # h is bf16(fp32(silu(g) u)); the fp64 sums may differ in the last bits, so a
+            # rounding boundary may fall either way: at most one bf16 step apart
+            assert np.all(np.abs(hb - h) <= np.abs(h) * 2.0 ** -7 + 1e-30)
+    assert np.abs(r["out_f64"] - ref).max() <= 1e-6 * np.abs(ref).max()
+
+
+def test_w4a16_identity_experts_closed_form():
+    """Experts whose NVFP4 weights encode identities (gate = up = I, down = c_e I): the layer
+    reduces to out[t][n] = sum_j w_tj c_{e_tj} bf16(silu(x_tn) x_tn), written out here
+    with math.exp."""
+    import math
+    T, H, E, k = 5, 16, 4, 2
+    I = H
+    rng = np.random.default_rng(3)
+    x = torch.from_numpy(rng.standard_normal((T, H)).astype(np.float32)).to(torch.bfloat16)
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    xf = x.to(torch.float64).numpy()
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    codes = np.zeros((E, I, H // 2), np.uint8)
+    for i in range(I):  # E2M1 code 2 is 1.0; element i sits in byte i // 2, nibble i % 2
+        codes[:, i, i // 2] = 2 << (4 * (i % 2))
+    sf = np.full((E, I, H // 16), 0x38, np.uint8)  # E4M3 0x38 is 1.0
+    ones = np.ones(E, np.float32)
+    c = np.array([0.5, 1.0, 2.0, 0.25], np.float32)
+    r = O.moe_ffn_w4a16(xb, logits, k, (codes, sf, ones), (codes, sf, ones), (codes, sf, c))
+    ids = _ref_topk(logits, k)
+    for t in range(T):
+        sel = [float(logits[t, e]) for e in ids[t]]
+        ex = [math.exp(v - sel[0]) for v in sel]
+        wts = [float(np.float32(v / sum(ex))) for v in ex]
+        for n in range(H):
+            h = float(_bf16_round(xf[t, n] / (1 + math.exp(-xf[t, n])) * xf[t, n]))
+            want = sum(wts[j] * float(c[ids[t, j]]) * h for j in range(k))
+            assert abs(r["out_f64"][t, n] - want) <= 1e-6 * max(abs(want), 1e-30), (t, n)
