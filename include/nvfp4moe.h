@@ -230,6 +230,14 @@ enum { NVFP4MOE_PATH_AUTO = 0, NVFP4MOE_PATH_GEMV = 1, NVFP4MOE_PATH_GEMM = 2 };
  *   AUTO        ORDERED; ACCUMULATE when top_k == 1 on the tensor-core path (one term per
  *               output: exact and deterministic). */
 enum { NVFP4MOE_COMBINE_AUTO = 0, NVFP4MOE_COMBINE_ORDERED = 1, NVFP4MOE_COMBINE_ACCUMULATE = 2 };
+/* Activation format of the expert products:
+ *   NVFP4  W4A4: x and the intermediate h are quantised to NVFP4 (the layer the model cards
+ *          describe as "NVFP4 W4A4", Qwen3.8-Flash-Next-NVFP4-SSD-Stream card);
+ *   BF16   W4A16, weight-only: x enters the products in bf16 and h is rounded to bf16 (no
+ *          activation-quantisation site, as the Qwen3.8-27B-nvfp4full-dflash2-NInfer card's
+ *          "Limits" names it); x_scale, h_scale, h_scale_mode and h_amax are unused.  Runs the
+ *          split-K GEMV path (PATH_AUTO resolves to it; PATH_GEMM is UNSUPPORTED_SHAPE). */
+enum { NVFP4MOE_ACT_NVFP4 = 0, NVFP4MOE_ACT_BF16 = 1 };
 
 typedef struct {
   int32_t T, H, I, E, top_k;
@@ -256,6 +264,7 @@ typedef struct {
    * layout.h_stats + 4*E (tensor-core path only, else NVFP4MOE_UNSUPPORTED_SHAPE; h_amax,
    * when given, receives the maxima as well). */
   int32_t h_scale_mode;
+  int32_t act_mode;           /* NVFP4MOE_ACT_* */
 } moe_ffn_desc;
 
 enum { NVFP4MOE_STAGES = 7 };
@@ -275,6 +284,8 @@ typedef struct {
   int32_t reserved;
   int64_t h_f32;    /* dynamic h scale: fp32 h [h_rows][I] before requantisation */
   int64_t h_stats;  /* dynamic h scale: amax[E] then the scales used, s_h[E] (fp32) */
+  int64_t h_bf16;   /* weight-only layer: h in bf16 [T*k][I], permuted rows (x_codes, x_sf,
+                       h_codes, h_sf are empty then) */
 } moe_ffn_ws_layout;
 
 nvfp4moe_status moe_ffn_workspace_layout(const moe_ffn_desc* d, moe_ffn_ws_layout* layout);

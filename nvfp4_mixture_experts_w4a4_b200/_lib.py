@@ -16,6 +16,7 @@ SCALE_GIVEN, SCALE_DYNAMIC = 0, 1
 DTYPE_BF16, DTYPE_F32 = 0, 1
 PATH_AUTO, PATH_GEMV, PATH_GEMM = 0, 1, 2
 COMBINE_AUTO, COMBINE_ORDERED, COMBINE_ACCUMULATE = 0, 1, 2
+ACT_NVFP4, ACT_BF16 = 0, 1
 STAGES = 7
 STAGE_NAMES = ("route", "permute", "quantize_x", "gate_up", "down", "combine")
 DEV_BAD_EXPERT_ID, DEV_DUPLICATE_ID, DEV_ROW_OVERFLOW = 1, 2, 4
@@ -45,6 +46,7 @@ class MoeFfnDesc(ctypes.Structure):
         ("w13_codes", _vp), ("w13_sf", _vp), ("w13_scale", _vp),
         ("w2_codes", _vp), ("w2_sf", _vp), ("w2_scale", _vp),
         ("h_scale", _vp), ("h_amax", _vp), ("stage_events", _vp), ("combine", _i32), ("h_scale_mode", _i32),
+        ("act_mode", _i32),
     ]
 
 
@@ -53,7 +55,8 @@ class MoeFfnWsLayout(ctypes.Structure):
         "topk_ids", "topk_w", "counts", "offsets", "padded_offsets", "pair_to_row", "row_token",
         "row_pair", "tile_expert", "active", "x_scale", "x_codes", "x_sf", "h_codes", "h_sf",
         "slots", "amax_partials", "total", "x_rows", "h_rows", "items")] + [
-        ("m_tile", _i32), ("path", _i32), ("combine", _i32), ("reserved", _i32), ("h_f32", _i64), ("h_stats", _i64)]
+        ("m_tile", _i32), ("path", _i32), ("combine", _i32), ("reserved", _i32), ("h_f32", _i64), ("h_stats", _i64),
+        ("h_bf16", _i64)]
 
 
 # name -> (restype, argtypes)

@@ -39,7 +39,7 @@ struct BatchArgs {
   int32_t *counts, *offsets, *padded_offsets, *pair_to_row, *row_token, *row_pair, *tile_expert, *active;
   float* zero_f32;          // nullable [E]
   int expert_order;         // 1: x rows go to the padded expert-order rows; 0: token-major
-  uint8_t* x_codes;
+  uint8_t* x_codes;         // nullable: x is not quantised (weight-only layer)
   uint8_t* x_sf;            // MMA layout
   int32_t* hist;            // [slices][E] histogram, then each slice's first rank per expert
   float* partials;          // [slices] amax of each slice's x rows
@@ -223,7 +223,8 @@ __global__ void __launch_bounds__(kThreads) place_quant_kernel(BatchArgs a) {
     ftotal += s_w32[w];
     mx = fmaxf(mx, s_red[w]);
   }
-  const float s_t = a.dynamic ? __fdiv_rn(mx, 2688.0f) : *a.x_scale;
+  // (no x codes: the weight-only layer keeps x in bf16 and has no x scale)
+  const float s_t = a.dynamic ? __fdiv_rn(mx, 2688.0f) : (a.x_codes ? *a.x_scale : 0.0f);
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     const int e = 2 * int(threadIdx.x) + i;
@@ -270,7 +271,7 @@ __global__ void __launch_bounds__(kThreads) place_quant_kernel(BatchArgs a) {
   // quantise each 16-element block of the slice's x rows once; write it to its row(s)
   const int nb = H / 16;
   const int64_t rb = H / 2;
-  const int n_items = nt * nb;
+  const int n_items = a.x_codes ? nt * nb : 0;
   for (int item0 = threadIdx.x; item0 < n_items; item0 += 2 * kThreads) {
    uint4 uu[2][2];
 #pragma unroll

@@ -33,10 +33,15 @@ nvfp4moe_status check_desc(const moe_ffn_desc* d, const char* fn) {
                 NVFP4MOE_INVALID_ARG, "%s: bad combine mode %d", fn, d->combine);
   NVFP4_REQUIRE(d->h_scale_mode == NVFP4MOE_SCALE_GIVEN || d->h_scale_mode == NVFP4MOE_SCALE_DYNAMIC,
                 NVFP4MOE_INVALID_ARG, "%s: bad h_scale_mode", fn);
+  NVFP4_REQUIRE(d->act_mode == NVFP4MOE_ACT_NVFP4 || d->act_mode == NVFP4MOE_ACT_BF16, NVFP4MOE_INVALID_ARG,
+                "%s: bad act_mode %d", fn, d->act_mode);
+  NVFP4_REQUIRE(d->act_mode != NVFP4MOE_ACT_BF16 || d->path != NVFP4MOE_PATH_GEMM, NVFP4MOE_UNSUPPORTED_SHAPE,
+                "%s: the weight-only layer runs the GEMV path", fn);
   return NVFP4MOE_OK;
 }
 
 int resolve_path(const moe_ffn_desc* d) {
+  if (d->act_mode == NVFP4MOE_ACT_BF16) return NVFP4MOE_PATH_GEMV;
   if (d->path != NVFP4MOE_PATH_AUTO) return d->path;
   // the weight-stationary tensor-core kernel is faster than the GEMV at every measured size
   // (decode included); the GEMV serves the shapes it does not (I % 128 != 0)
@@ -88,12 +93,14 @@ void make_layout(const moe_ffn_desc* d, moe_ffn_ws_layout* L) {
   L->active = take((E + 1) * 4);
   L->x_scale = take(4);
   L->amax_partials = take(static_cast<int64_t>(nvfp4_quantize_workspace_size(1, T > 0 ? T : 1, H)));
-  L->x_rows = path == NVFP4MOE_PATH_GEMM ? rows_cap : T;
+  const bool a16 = d->act_mode == NVFP4MOE_ACT_BF16;  // weight-only: no activation codes
+  L->x_rows = a16 ? 0 : (path == NVFP4MOE_PATH_GEMM ? rows_cap : T);
   L->x_codes = take(L->x_rows * H / 2);
   L->x_sf = take(sf_mma_bytes(L->x_rows, H));
-  L->h_rows = path == NVFP4MOE_PATH_GEMM ? rows_cap : P;
+  L->h_rows = a16 ? 0 : (path == NVFP4MOE_PATH_GEMM ? rows_cap : P);
   L->h_codes = take(L->h_rows * I / 2);
   L->h_sf = take(sf_mma_bytes(L->h_rows, I));
+  L->h_bf16 = take(a16 ? P * I * 2 : 0);
   // fp32 rows of the down projection: split-K partials by pair on the GEMV path; on the
   // tensor-core path rows by pair (up to 64 tokens) or by padded expert row (above), or the
   // [T][H] accumulator of the accumulating combine (the region also holds the batch
@@ -115,7 +122,7 @@ void make_layout(const moe_ffn_desc* d, moe_ffn_ws_layout* L) {
                       ? grouped_fused_list_entries(A, 2 * I / 128, H / 128) * 16 + E * 4
                       : 0);
   // dynamic h scale: fp32 h before requantisation, per-expert amax and scale
-  const bool dyn_h = d->h_scale_mode == NVFP4MOE_SCALE_DYNAMIC;
+  const bool dyn_h = !a16 && d->h_scale_mode == NVFP4MOE_SCALE_DYNAMIC;
   L->h_f32 = take(dyn_h ? L->h_rows * I * 4 : 0);
   L->h_stats = take(dyn_h ? 2 * E * 4 : 0);
   L->total = o;
@@ -152,7 +159,8 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   NVFP4_REQUIRE(x && logits && out && workspace, NVFP4MOE_INVALID_ARG, "%s: NULL pointer", fn);
   NVFP4_REQUIRE(d->w13_codes && d->w13_sf && d->w13_scale && d->w2_codes && d->w2_sf && d->w2_scale,
                 NVFP4MOE_INVALID_ARG, "%s: NULL weight pointer in desc", fn);
-  NVFP4_REQUIRE(d->x_scale_mode == NVFP4MOE_SCALE_DYNAMIC || d->x_scale != nullptr, NVFP4MOE_INVALID_ARG,
+  const bool a16 = d->act_mode == NVFP4MOE_ACT_BF16;  // weight-only: no activation scales
+  NVFP4_REQUIRE(a16 || d->x_scale_mode == NVFP4MOE_SCALE_DYNAMIC || d->x_scale != nullptr, NVFP4MOE_INVALID_ARG,
                 "%s: GIVEN x scale needs desc->x_scale", fn);
   NVFP4_REQUIRE(aligned16(x) && aligned16(out) && aligned16(workspace) && aligned16(d->w13_codes) &&
                     aligned16(d->w13_sf) && aligned16(d->w2_codes) && aligned16(d->w2_sf),
@@ -169,10 +177,11 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   }
   NVFP4_REQUIRE(L.combine != NVFP4MOE_COMBINE_ACCUMULATE || L.path == NVFP4MOE_PATH_GEMM, NVFP4MOE_UNSUPPORTED_SHAPE,
                 "%s: the accumulating combine needs the tensor-core path", fn);
-  const bool dyn_h = d->h_scale_mode == NVFP4MOE_SCALE_DYNAMIC;
+  const bool dyn_h = !a16 && d->h_scale_mode == NVFP4MOE_SCALE_DYNAMIC;
   NVFP4_REQUIRE(!dyn_h || L.path == NVFP4MOE_PATH_GEMM, NVFP4MOE_UNSUPPORTED_SHAPE,
                 "%s: the dynamic h scale needs the tensor-core path", fn);
-  NVFP4_REQUIRE(dyn_h || d->h_scale != nullptr, NVFP4MOE_INVALID_ARG, "%s: GIVEN h scale needs desc->h_scale", fn);
+  NVFP4_REQUIRE(a16 || dyn_h || d->h_scale != nullptr, NVFP4MOE_INVALID_ARG, "%s: GIVEN h scale needs desc->h_scale",
+                fn);
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   auto I32 = [&](int64_t off) { return reinterpret_cast<int32_t*>(ws + off); };
@@ -188,8 +197,9 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
     }
   };
 
-  const bool dyn = d->x_scale_mode == NVFP4MOE_SCALE_DYNAMIC;
-  float* xs = dyn ? F32(L.x_scale) : const_cast<float*>(d->x_scale);
+  const bool dyn = !a16 && d->x_scale_mode == NVFP4MOE_SCALE_DYNAMIC;
+  float* xs = a16 ? nullptr : (dyn ? F32(L.x_scale) : const_cast<float*>(d->x_scale));
+  uint8_t* x_codes = a16 ? nullptr : ws + L.x_codes;  // the prologues quantise x only for W4A4
   const bool fused = prologue_fits(T, E, k);
   // small batches on the tensor-core path: the prologue also writes the GEMMs' work lists
   const bool lists = fused && L.path == NVFP4MOE_PATH_GEMM;
@@ -201,7 +211,7 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   float* accum = F32(L.slots);  // fp32 [T][H] when accumulating
   uint8_t* prologue_scratch = ws + L.slots + prologue_scratch_offset(d, L.combine);
   // dynamic h scale: per-expert amax of h over this call, then the scales derived from it
-  float* h_amax_int = dyn_h ? F32(L.h_stats) : d->h_amax;
+  float* h_amax_int = dyn_h ? F32(L.h_stats) : (a16 ? nullptr : d->h_amax);
   float* h_scale_dyn = dyn_h ? F32(L.h_stats) + E : nullptr;
 
   mark(0);
@@ -210,7 +220,7 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
     st = launch_prologue(x, logits, T, H, E, k, L.m_tile, dyn ? 1 : 0, xs, I32(L.topk_ids), F32(L.topk_w),
                          I32(L.counts), I32(L.offsets), I32(L.padded_offsets), I32(L.pair_to_row), I32(L.row_token),
                          I32(L.row_pair), I32(L.tile_expert), I32(L.active), h_amax_int,
-                         L.path == NVFP4MOE_PATH_GEMM ? 1 : 0, ws + L.x_codes, ws + L.x_sf, lists ? list : nullptr,
+                         L.path == NVFP4MOE_PATH_GEMM ? 1 : 0, x_codes, ws + L.x_sf, lists ? list : nullptr,
                          lists ? done : nullptr, 2 * I / 128, H / 128, s);
     if (st != NVFP4MOE_OK) return st;
     mark(1);
@@ -220,7 +230,7 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
     st = launch_batch_prologue(x, logits, T, H, E, k, L.m_tile, dyn ? 1 : 0, xs, I32(L.topk_ids), F32(L.topk_w),
                                I32(L.counts), I32(L.offsets), I32(L.padded_offsets), I32(L.pair_to_row),
                                I32(L.row_token), I32(L.row_pair), I32(L.tile_expert), I32(L.active), h_amax_int,
-                               L.path == NVFP4MOE_PATH_GEMM ? 1 : 0, ws + L.x_codes, ws + L.x_sf, prologue_scratch,
+                               L.path == NVFP4MOE_PATH_GEMM ? 1 : 0, x_codes, ws + L.x_sf, prologue_scratch,
                                accumulate ? accum : nullptr, d->stage_events, s);
     if (st != NVFP4MOE_OK) return st;
   }
@@ -228,17 +238,21 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   if (L.path == NVFP4MOE_PATH_GEMV) {
     // x quantised once per token, token-major
     mark(3);
-    GemvGateUpArgs g;
+    GemvGateUpArgs g{};
     g.H = H; g.I = I;
     g.x_codes = ws + L.x_codes; g.x_sf = ws + L.x_sf; g.x_scale = xs;
     g.offsets = I32(L.offsets); g.row_token = I32(L.row_token); g.active = I32(L.active);
     g.w13_codes = d->w13_codes; g.w13_sf = d->w13_sf; g.w13_scale = d->w13_scale;
     g.h_scale = d->h_scale; g.h_amax = d->h_amax;
     g.h_codes = ws + L.h_codes; g.h_sf = ws + L.h_sf;
+    if (a16) {  // weight-only: bf16 x in, bf16 h out
+      g.x_bf16 = static_cast<const uint16_t*>(x);
+      g.h_bf16 = reinterpret_cast<uint16_t*>(ws + L.h_bf16);
+    }
     st = launch_gemv_gateup(g, max_active_experts(d), s);
     if (st != NVFP4MOE_OK) return st;
     mark(4);
-    GemvDownArgs dn;
+    GemvDownArgs dn{};
     dn.H = H; dn.I = I;
     dn.ksplit = gemv_down_ksplit(max_active_experts(d), H, I);
     dn.h_codes = ws + L.h_codes; dn.h_sf = ws + L.h_sf;
@@ -246,6 +260,7 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
     dn.w2_codes = d->w2_codes; dn.w2_sf = d->w2_sf; dn.w2_scale = d->w2_scale;
     dn.h_scale = d->h_scale; dn.topk_w = F32(L.topk_w);
     dn.slots = F32(L.slots); dn.slot_stride = int64_t(T) * k * H;
+    if (a16) dn.h_bf16 = reinterpret_cast<const uint16_t*>(ws + L.h_bf16);
     st = launch_gemv_down(dn, max_active_experts(d), s);
     if (st != NVFP4MOE_OK) return st;
     mark(5);

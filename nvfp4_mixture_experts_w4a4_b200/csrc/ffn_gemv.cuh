@@ -20,6 +20,10 @@ struct GemvGateUpArgs {
   float* h_amax;            // nullable [E]
   uint8_t* h_codes;         // [P][I/2]
   uint8_t* h_sf;            // MMA layout over P rows
+  // weight-only (W4A16) layer when x_bf16 is set: x is read in bf16 [T][H], h is written in
+  // bf16 [P][I] (x_codes, x_sf, x_scale, h_scale, h_codes, h_sf unused)
+  const uint16_t* x_bf16;
+  uint16_t* h_bf16;
 };
 
 struct GemvDownArgs {
@@ -37,6 +41,7 @@ struct GemvDownArgs {
   const float* topk_w;      // [P] by pair; nullable (weight 1)
   float* slots;             // [ksplit][P][H]
   int64_t slot_stride;      // P*H
+  const uint16_t* h_bf16;   // weight-only layer when set: h in bf16 [P][I] (h codes unused)
 };
 
 int gemv_lanes_per_row(int64_t K);

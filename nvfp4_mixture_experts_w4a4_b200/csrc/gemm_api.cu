@@ -93,7 +93,7 @@ nvfp4moe_status nvfp4_gemm(const uint8_t* A, const uint8_t* A_sf, const float* a
   gemv_gemm_init<<<1, 256, 0, s>>>(offsets, row_pair, active, static_cast<int>(M));
   nvfp4moe_status st = check_launch(fn);
   if (st != NVFP4MOE_OK) return st;
-  GemvDownArgs a;
+  GemvDownArgs a{};
   a.H = static_cast<int>(N);
   a.I = static_cast<int>(K);
   a.ksplit = L.ksplit;

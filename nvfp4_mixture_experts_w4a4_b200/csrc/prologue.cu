@@ -63,7 +63,7 @@ struct PrologueArgs {
   int32_t *counts, *offsets, *padded_offsets, *pair_to_row, *row_token, *row_pair, *tile_expert, *active;
   float* zero_f32;          // nullable [E]
   int expert_order;         // 1: x rows go to the padded expert-order rows; 0: token-major
-  uint8_t* x_codes;
+  uint8_t* x_codes;         // nullable: x is not quantised (weight-only layer)
   uint8_t* x_sf;            // MMA layout
   int4* list;               // nullable: the fused grouped GEMM's work list (one chunk per expert)
   int* done;                //   and its per-expert counters, zeroed here
@@ -231,7 +231,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1) 
     for (int i = 0; i < kCluster; ++i) mx = fmaxf(mx, s_part[i]);
     s_t = __fdiv_rn(mx, 2688.0f);
   } else {
-    s_t = *a.x_scale;
+    s_t = a.x_codes ? *a.x_scale : 0.0f;  // no x codes: the weight-only layer keeps x in bf16
   }
   if (gi == 0) {
     a.offsets[E] = s_off[E];
@@ -267,7 +267,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1) 
   // quantise each 16-element block of x once; write it to its row(s)
   const int nb = H / 16;
   const int64_t rb = H / 2;
-  for (int item = gi; item < T * nb; item += kAll) {
+  for (int item = gi; a.x_codes && item < T * nb; item += kAll) {
     const int tk = item / nb, b = item - tk * nb;
     const uint4* src = reinterpret_cast<const uint4*>(a.x + int64_t(tk) * H + b * 16);
     const uint4 u0 = __ldg(src), u1 = __ldg(src + 1);

@@ -189,15 +189,18 @@ class MoeFFN:
     """The routed NVFP4 W4A4 feed-forward layer (moe_ffn_forward) with a cached workspace."""
 
     def __init__(self, experts: NVFP4Experts, top_k: int, h_scale: torch.Tensor | None,
-                 x_scale: torch.Tensor | None = None, path: int = C.PATH_AUTO, combine: int = C.COMBINE_AUTO):
+                 x_scale: torch.Tensor | None = None, path: int = C.PATH_AUTO, combine: int = C.COMBINE_AUTO,
+                 act: int = C.ACT_NVFP4):
         """h_scale: per-expert requantisation scales of h, or None for the dynamic scale
-        (amax of each expert's h in the call / 2688; tensor-core path)."""
+        (amax of each expert's h in the call / 2688; tensor-core path).  act: ACT_NVFP4 (W4A4)
+        or ACT_BF16 (weight-only W4A16: bf16 activations, the GEMV path; no scales used)."""
         self.w = experts
         self.top_k = top_k
         self.h_scale = None if h_scale is None else h_scale.to(torch.float32).contiguous()
         self.x_scale = None if x_scale is None else x_scale.to(torch.float32).contiguous().view(1)
         self.path = path
         self.combine = combine
+        self.act = act
         self._ws = {}
 
     def desc(self, T: int, h_amax: torch.Tensor | None = None, events=None) -> C.MoeFfnDesc:
@@ -213,6 +216,7 @@ class MoeFFN:
         d.h_scale = None if self.h_scale is None else self.h_scale.data_ptr()
         d.h_scale_mode = C.SCALE_DYNAMIC if self.h_scale is None else C.SCALE_GIVEN
         d.h_amax = None if h_amax is None else h_amax.data_ptr()
+        d.act_mode = self.act
         d.stage_events = None if events is None else ctypes.cast(events, ctypes.c_void_p).value
         return d
 
@@ -285,6 +289,7 @@ class MoeFFN:
             h_codes=view(L.h_codes, L.h_rows * w.I // 2, torch.uint8).view(L.h_rows, w.I // 2),
             h_sf=view(L.h_sf, sf_mma_bytes(L.h_rows, w.I), torch.uint8),
             x_rows=L.x_rows, h_rows=L.h_rows,
+            h_bf16=view(L.h_bf16, P * w.I, torch.int16).view(P, w.I) if self.act == C.ACT_BF16 else None,
         )
 
 

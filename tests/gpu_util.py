@@ -213,3 +213,43 @@ def h_diff_effect(hc, hsf, ref, wl, wd_dequant):
         dh = np.abs(gv[r] - rv[r]) * s_h[e]
         extra[t] += ref["w"][t, j] * (np.abs(wd_dequant(e)) @ dh)
     return extra
+
+
+def run_layer_pair_w4a16(wl: W.Workload, seed: int = 0, dev=None):
+    """The weight-only (W4A16) layer on the device and in the oracle, on the same inputs."""
+    dev = dev or need_gpu()
+    act, wts, wg, wu, wd = layer_inputs(wl, seed)
+    ref = O.moe_ffn_w4a16(bf16_bits(act["x"]), act["logits"].numpy(), wl.k, wg, wu, wd)
+    layer = ops.MoeFFN(experts_from_oracle(wg, wu, wd, dev), wl.k, None, act=C.ACT_BF16)
+    out = layer(act["x"].to(dev), act["logits"].to(dev))
+    torch.cuda.synchronize()
+    return ref, out, layer
+
+
+def check_layer_w4a16(wl: W.Workload, ref: dict, out: torch.Tensor, layer: ops.MoeFFN):
+    """Routing and permutation bit-exact; h (bf16) equal except for at most H_CODE_FRAC of its
+    elements, each one bf16 step away (a rounding boundary that the fp32 sums of the device
+    and the fp64 sums of the oracle put on different sides); outputs within the tolerance."""
+    T, k = wl.T, wl.k
+    im = layer.intermediates(T)
+    assert im["path"] == C.PATH_GEMV
+    assert np.array_equal(im["topk_ids"].cpu().numpy(), ref["ids"])
+    np.testing.assert_allclose(im["topk_w"].cpu().numpy(), ref["w"], rtol=2e-6, atol=1e-7)
+    assert np.array_equal(im["counts"].cpu().numpy(), ref["counts"])
+    assert np.array_equal(im["offsets"].cpu().numpy(), ref["offsets"])
+    assert np.array_equal(im["pair_to_row"].cpu().numpy(), ref["pair_to_row"])
+    hg = im["h_bf16"].cpu().numpy().view(np.uint16).astype(np.int64)
+    hr = ref["h_bf16"].astype(np.int64)
+    diff = hg != hr
+    assert diff.sum() <= H_CODE_FRAC * diff.size, f"{diff.sum()} of {diff.size} h values differ"
+    # a differing value is one bf16 step away (bit patterns of one sign are ordered like their
+    # values), or it sits where g or u cancel: within 2^-16 of its row's largest |h| (the fp32
+    # sums of the device carry an absolute error of that order there, the oracle's fp64 none)
+    vg = bits_to_f32(hg.astype(np.uint16)).astype(np.float64)
+    vr = bits_to_f32(hr.astype(np.uint16)).astype(np.float64)
+    one_step = ((hg >> 15) == (hr >> 15)) & (np.abs(hg - hr) == 1)
+    near_zero = np.abs(vg - vr) <= 2.0 ** -16 * np.abs(vr).max(axis=1, keepdims=True)
+    bad = diff & ~one_step & ~near_zero
+    assert not bad.any(), f"h differs beyond one bf16 step: gpu {vg[bad][:4]} oracle {vr[bad][:4]}"
+    print(f"[parity w4a16] {wl.name} T={T}: {int(diff.sum())} of {diff.size} h values differ")
+    return check_out(bf16_bits(out), ref["out_f64"])

@@ -48,7 +48,7 @@ def test_binding_declares_every_symbol():
 
 def test_argument_errors_are_statuses(so):
     from nvfp4_mixture_experts_w4a4_b200 import _lib as C
-    assert so.nvfp4moe_version() == 0x000400
+    assert so.nvfp4moe_version() == 0x000500
     # bad E, bad k: rejected before any device work
     assert so.moe_route(None, 4, 2000, 2, None, None, None) == C.UNSUPPORTED_SHAPE
     assert b"E=2000" in so.nvfp4moe_last_error()
@@ -88,3 +88,20 @@ def test_workspace_queries(so):
     assert so.moe_ffn_workspace_layout(ctypes.byref(d), ctypes.byref(L)) == C.UNSUPPORTED_SHAPE
     assert so.moe_permute_rows_capacity(16, 512, 10, 128) == 160 + 160 * 127
     assert so.moe_permute_rows_capacity(4096, 256, 8, 128) == 32768 + 256 * 127
+
+
+def test_weight_only_workspace_and_mode_checks(so):
+    """The weight-only (W4A16) mode: no activation codes in the workspace, a bf16 h region,
+    the GEMV path whatever AUTO would pick, and the tensor-core path or a bad mode refused."""
+    from nvfp4_mixture_experts_w4a4_b200 import _lib as C
+    d = C.MoeFfnDesc()
+    d.T, d.H, d.I, d.E, d.top_k = 16, 2048, 512, 512, 10
+    d.act_mode = C.ACT_BF16
+    L = C.MoeFfnWsLayout()
+    assert so.moe_ffn_workspace_layout(ctypes.byref(d), ctypes.byref(L)) == C.OK
+    assert L.path == C.PATH_GEMV and L.x_rows == 0 and L.h_rows == 0
+    assert L.h_bf16 % 256 == 0 and L.h_bf16 + 16 * 10 * 512 * 2 <= L.total
+    d.path = C.PATH_GEMM
+    assert so.moe_ffn_workspace_layout(ctypes.byref(d), ctypes.byref(L)) == C.UNSUPPORTED_SHAPE
+    d.path, d.act_mode = C.PATH_AUTO, 7
+    assert so.moe_ffn_workspace_layout(ctypes.byref(d), ctypes.byref(L)) == C.INVALID_ARG

@@ -181,3 +181,22 @@ def test_layer_dynamic_h_scale(name):
     assert np.array_equal(h_amax.cpu().numpy()[used], a_dev[used])
     G.check_layer(wl, ref, out, layer, h_amax)
     assert ops.device_status() == 0
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_layer_weight_only_w4a16(name):
+    """The weight-only variant (bf16 activations, NVFP4 weights, split-K GEMV) against the
+    oracle's W4A16 layer."""
+    wl = CASES[name]
+    ref, out, layer = G.run_layer_pair_w4a16(wl)
+    G.check_layer_w4a16(wl, ref, out, layer)
+    assert ops.device_status() == 0
+
+
+def test_weight_only_rejects_the_tensor_core_path():
+    wl = CASES["tiny"]
+    act, wts, wg, wu, wd = G.layer_inputs(wl)
+    dev = G.need_gpu()
+    layer = ops.MoeFFN(G.experts_from_oracle(wg, wu, wd, dev), wl.k, None, path=C.PATH_GEMM, act=C.ACT_BF16)
+    with pytest.raises(C.Nvfp4MoeError):
+        layer(act["x"].to(dev), act["logits"].to(dev))
