@@ -166,16 +166,17 @@ def setup_layer(wl: W.Workload, dev, seed: int = 0, keep_tokens: int = 0, path: 
     return act, host, experts, layer
 
 
-def algorithmic(wl: W.Workload, n_active: int, gemm_path: bool):
+def algorithmic(wl: W.Workload, n_active: int, gemm_path: bool, a16: bool = False):
     """Algorithmic (compulsory) bytes and FLOPs of one layer pass and of its gate/up stage:
     each touched expert's weights once, the quantised activations once (per permuted row on
-    the tensor-core path, which gathers x into expert order), h written and read once."""
+    the tensor-core path, which gathers x into expert order), h written and read once.
+    Weight-only (a16): x and h in bf16."""
     e = FP4_BYTES_PER_ELT
     P = wl.T * wl.k
     w13 = n_active * 2 * wl.I * wl.H * e
     w2 = n_active * wl.H * wl.I * e
-    x_q = (P if gemm_path else wl.T) * wl.H * e
-    h_q = P * wl.I * e
+    x_q = (P if gemm_path else wl.T) * wl.H * (2 if a16 else e)
+    h_q = P * wl.I * (2 if a16 else e)
     gate_up_bytes = w13 + x_q + h_q
     layer_bytes = w13 + w2 + wl.T * wl.H * 2 * 2 + x_q + 2 * h_q + wl.T * wl.E * 4
     flops = 2.0 * P * 3 * wl.H * wl.I
@@ -368,17 +369,20 @@ def oracle_inputs(wl: W.Workload, act, host, tokens: np.ndarray):
     return x[tokens], logits[tokens], arrays, float(s_x)
 
 
-def oracle_rate(wl: W.Workload, act, host, layer, budget_s: float, max_tokens: int):
+def oracle_rate(wl: W.Workload, act, host, layer, budget_s: float, max_tokens: int, a16: bool = False):
     """Tokens/s of the oracle on a bounded token sample of the workload (host cores)."""
     import oracle as O
     n = min(wl.T, max_tokens)
     tokens = np.arange(n)
     x, logits, arr, s_x = oracle_inputs(wl, act, host, tokens)
-    s_h = layer.h_scale.cpu().numpy()
+    s_h = None if a16 else layer.h_scale.cpu().numpy()
     nth = O.default_threads()
     done, t0 = 0, time.perf_counter()
     while True:
-        O.moe_ffn(x, logits, wl.k, arr["g"], arr["u"], arr["d"], x_scale=s_x, h_scale=s_h, nthreads=nth)
+        if a16:
+            O.moe_ffn_w4a16(x, logits, wl.k, arr["g"], arr["u"], arr["d"], nthreads=nth)
+        else:
+            O.moe_ffn(x, logits, wl.k, arr["g"], arr["u"], arr["d"], x_scale=s_x, h_scale=s_h, nthreads=nth)
         done += n
         el = time.perf_counter() - t0
         if el >= budget_s or done >= 64 * n:
@@ -402,6 +406,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--path", default="auto", choices=["auto", "gemv", "tcgen05"],
                     help="layer path: auto (GEMV for T <= 16), the GEMV path or the tcgen05 grouped GEMM")
+    ap.add_argument("--act", default="nvfp4", choices=["nvfp4", "bf16"],
+                    help="activations: nvfp4 (W4A4) or bf16 (the weight-only W4A16 variant, GEMV path)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -419,6 +425,9 @@ def main():
     cfg = {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "top_k": wl.k,
            "zipf_s": wl.zipf_s, "outlier_frac": wl.outlier_frac, "l2": "flushed before every step (256 MiB write, then 256 MiB read)",
            "seed": 0, "parallelism": f"replicas x{world}"}
+    a16 = args.act == "bf16"
+    if a16:
+        cfg["act"] = "w4a16 (bf16 activations, NVFP4 weights)"
 
     if args.impl == "reference":
         if rank != 0:
@@ -434,13 +443,18 @@ def main():
         nth = O.default_threads()
         # a step is a bounded sample of the workload's tokens, sized to keep the run short
         sample = n
+
+        def one_step():
+            if a16:
+                O.moe_ffn_w4a16(x[:sample], logits[:sample], wl.k, arr["g"], arr["u"], arr["d"], nthreads=nth)
+            else:
+                O.moe_ffn(x[:sample], logits[:sample], wl.k, arr["g"], arr["u"], arr["d"], x_scale=s_x,
+                          h_scale=s_h, nthreads=nth)
         for _ in range(args.warmup):
-            O.moe_ffn(x[:sample], logits[:sample], wl.k, arr["g"], arr["u"], arr["d"], x_scale=s_x,
-                      h_scale=s_h, nthreads=nth)
+            one_step()
         t0 = time.perf_counter()
         for _ in range(args.steps):
-            O.moe_ffn(x[:sample], logits[:sample], wl.k, arr["g"], arr["u"], arr["d"], x_scale=s_x,
-                      h_scale=s_h, nthreads=nth)
+            one_step()
         el = time.perf_counter() - t0
         value = sample * args.steps / el
         line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -459,6 +473,8 @@ def main():
     path = {"auto": C.PATH_AUTO, "gemv": C.PATH_GEMV, "tcgen05": C.PATH_GEMM}[args.path]
     act, host, experts, layer = setup_layer(wl, dev, keep_tokens=n_cpu if (rank == 0 and world == 1) else 0,
                                             path=path)
+    if a16:  # the same experts, weight-only
+        layer = ops.MoeFFN(experts, wl.k, None, act=C.ACT_BF16)
     flush = L2Flush(dev)
     with ClockSampler(local) as clk:
         step_ms, stage_ms, launches = time_steps(layer, act, args.steps, args.warmup, flush, dist_on)
@@ -470,7 +486,7 @@ def main():
     im = layer.intermediates(wl.T)
     n_active = int(im["active"][0].item())
     gemm_path = im["path"] == C.PATH_GEMM
-    alg = algorithmic(wl, n_active, gemm_path)
+    alg = algorithmic(wl, n_active, gemm_path, a16)
     pk = peaks()
     # the dominant kernel: for batches of at most 64 tokens on the tensor-core path with H <= 2I
     # both GEMMs run in one fused launch (its stage is "gate_up"); otherwise the gate/up GEMM
@@ -481,6 +497,7 @@ def main():
     roof = roofline(dom_bytes, dom_flops, dom_ms, pk)
     kernel = ("fused gate/up + down tcgen05 grouped GEMM (SwiGLU + requant, weighted slots)" if fused
               else "gate_up tcgen05 grouped GEMM + SwiGLU + requant" if gemm_path
+              else "gate_up GEMV (bf16 x, NVFP4 weights) + SwiGLU" if a16
               else "gate_up GEMV + SwiGLU + requant")
     roof.update({"kernel": kernel,
                  "traffic": measured_traffic(wl.name) if gemm_path else None,
@@ -495,14 +512,16 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, sample = oracle_rate(wl, act, host, layer, args.cpu_budget, max_tokens=n_cpu)
+        v, cores, sample = oracle_rate(wl, act, host, layer, args.cpu_budget, max_tokens=n_cpu, a16=a16)
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3, fp32 accumulate)", "data": "synthetic",
+            "vs_baseline": None,
+            "dtype": "bf16 x nvfp4 (w4a16, fp32 accumulate)" if a16 else "nvfp4 (e2m1 x e4m3, fp32 accumulate)",
+            "data": "synthetic",
             "config": cfg, "roofline": roof, "cpu_baseline": cpu,
             "e2e": {"value": world * wl.T / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},

@@ -15,6 +15,9 @@ namespace nvfp4moe {
 namespace {
 
 constexpr int kWarpsPerCta = 4;
+// resident CTAs per SM the kernels are compiled for (registers per thread <= 128): the weight
+// stream's bytes in flight grow with the warps an SM holds
+constexpr int kMinCtas = 4;
 
 // ------------------------------------------------------------- gate / up ----
 template <int L, int NT, bool A16>
@@ -80,7 +83,7 @@ __device__ __forceinline__ void gateup_group(const GemvGateUpArgs& a, int e, int
 }
 
 template <int L, bool A16>
-__global__ void __launch_bounds__(kWarpsPerCta * 32) gemv_gateup_kernel(GemvGateUpArgs a) {
+__global__ void __launch_bounds__(kWarpsPerCta * 32, kMinCtas) gemv_gateup_kernel(GemvGateUpArgs a) {
   __shared__ float tots_all[kWarpsPerCta][32][4];
   const int warp = threadIdx.x >> 5;
   float(*tots)[4] = tots_all[warp];
@@ -95,8 +98,6 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) gemv_gateup_kernel(GemvGate
     const float sg = a.w13_scale[2 * e] * s_x, su = a.w13_scale[2 * e + 1] * s_x;
     const float sh = A16 ? 1.0f : a.h_scale[e];
     int64_t g = 0;
-    if (!A16)  // (four bf16 rows of x per chunk would not fit the registers)
-      for (; g + 4 <= n_e; g += 4) gateup_group<L, 4, A16>(a, e, row0, r0 + g, sg, su, sh, tots);
     for (; g + 2 <= n_e; g += 2) gateup_group<L, 2, A16>(a, e, row0, r0 + g, sg, su, sh, tots);
     if (g < n_e) gateup_group<L, 1, A16>(a, e, row0, r0 + g, sg, su, sh, tots);
   }
@@ -143,7 +144,7 @@ __device__ __forceinline__ void down_group(const GemvDownArgs& a, int e, int64_t
 }
 
 template <int L, bool A16>
-__global__ void __launch_bounds__(kWarpsPerCta * 32) gemv_down_kernel(GemvDownArgs a) {
+__global__ void __launch_bounds__(kWarpsPerCta * 32, kMinCtas) gemv_down_kernel(GemvDownArgs a) {
   const int warp = threadIdx.x >> 5;
   const int64_t H = a.H, I = a.I;
   const int64_t row_groups = (H + 31) / 32;
@@ -163,8 +164,6 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) gemv_down_kernel(GemvDownAr
     const int64_t r0 = a.offsets[e], n_e = a.offsets[e + 1] - r0;
     const float sc = (A16 ? 1.0f : a.h_scale[e]) * a.w2_scale[e];
     int64_t g = 0;
-    if (!A16)
-      for (; g + 4 <= n_e; g += 4) down_group<L, 4, A16>(a, e, row0, r0 + g, c0, c1, sc, slots);
     for (; g + 2 <= n_e; g += 2) down_group<L, 2, A16>(a, e, row0, r0 + g, c0, c1, sc, slots);
     if (g < n_e) down_group<L, 1, A16>(a, e, row0, r0 + g, c0, c1, sc, slots);
   }

@@ -115,3 +115,46 @@ def test_fullsize_sampled_tokens(name):
         extra = G.h_diff_effect(hc, hsf, ref, wl_s, lambda e: R.dequantize(wd[0][e], wd[1][e], wd[2][e]))
     print(f"[full size] {name}: tokens {sample.tolist()}, {len(touched)} experts, {n_diff} h codes differ")
     G.check_out(G.bf16_bits(out)[sample], ref["out_f64"], extra=extra)
+
+
+@pytest.mark.parametrize("name", ["decode", "dense_t1"])
+def test_fullsize_weight_only_sampled_tokens(name):
+    """The weight-only (W4A16) variant at full size, as the benchmark runs it with --act bf16:
+    routing and permutation of the whole batch bit-exact, sampled tokens' h (bf16) and
+    outputs against the oracle's W4A16 layer over the experts they use."""
+    wl = W.WORKLOADS[name]
+    dev = G.need_gpu()
+    T, E, k = wl.T, wl.E, wl.k
+    act = W.make_activations(wl, 0, dev)
+    wts = W.make_weights(wl, 0, dev)
+    experts = ops.NVFP4Experts.from_float(wts["w_gate"], wts["w_up"], wts["w_down"])
+    x_bits = G.bf16_bits(act["x"])
+    logits = act["logits"].cpu().numpy()
+    sample = np.unique(np.linspace(0, T - 1, min(SAMPLE, T)).round().astype(np.int64))
+    ids_all, _ = O.route(logits, k)
+    perm = O.permute(ids_all, E)
+    touched = np.unique(ids_all[sample])
+    tt = torch.as_tensor(touched, device=dev)
+    wg = G.quantize_experts_parallel(wts["w_gate"][tt].cpu().numpy())
+    wu = G.quantize_experts_parallel(wts["w_up"][tt].cpu().numpy())
+    wd = G.quantize_experts_parallel(wts["w_down"][tt].cpu().numpy())
+    del wts
+    ref = O.moe_ffn_w4a16(x_bits[sample], logits[sample][:, touched], k, wg, wu, wd)
+    assert np.array_equal(touched[ref["ids"]], ids_all[sample])
+
+    layer = ops.MoeFFN(experts, k, None, act=C.ACT_BF16)
+    out = layer(act["x"], act["logits"])
+    torch.cuda.synchronize()
+    im = layer.intermediates(T)
+    assert np.array_equal(im["topk_ids"].cpu().numpy(), ids_all)
+    assert np.array_equal(im["counts"].cpu().numpy(), perm["counts"])
+    assert np.array_equal(im["pair_to_row"].cpu().numpy(), perm["pair_to_row"])
+    # sampled pairs' h rows, in the oracle's row order
+    gpu_rows = perm["pair_to_row"][(sample[:, None] * k + np.arange(k)[None, :]).reshape(-1)]
+    ref_rows = ref["pair_to_row"][np.arange(len(sample) * k)]
+    hg = np.empty_like(ref["h_bf16"])
+    hg[ref_rows] = im["h_bf16"].cpu().numpy().view(np.uint16)[gpu_rows]
+    diff = hg != ref["h_bf16"]
+    assert diff.sum() <= G.H_CODE_FRAC * diff.size + 1
+    print(f"[full size w4a16] {name}: tokens {sample.tolist()}, {len(touched)} experts, {int(diff.sum())} h differ")
+    G.check_out(G.bf16_bits(out)[sample], ref["out_f64"])
