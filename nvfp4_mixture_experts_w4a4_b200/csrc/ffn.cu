@@ -235,6 +235,31 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
     if (st != NVFP4MOE_OK) return st;
   }
 
+  if (a16) {
+    // weight-only: the expert products stream their weights through shared memory
+    mark(3);
+    StreamA16Args sa{};
+    sa.H = H; sa.I = I; sa.E = E;
+    sa.offsets = I32(L.offsets); sa.row_token = I32(L.row_token); sa.row_pair = I32(L.row_pair);
+    sa.active = I32(L.active);
+    sa.act = static_cast<const uint16_t*>(x);
+    sa.w_codes = d->w13_codes; sa.w_sf = d->w13_sf; sa.w_scale = d->w13_scale;
+    sa.h_out = reinterpret_cast<uint16_t*>(ws + L.h_bf16);
+    st = launch_stream_gemv_a16(0, sa, max_active_experts(d), s);
+    if (st != NVFP4MOE_OK) return st;
+    mark(4);
+    sa.act = reinterpret_cast<const uint16_t*>(ws + L.h_bf16);
+    sa.w_codes = d->w2_codes; sa.w_sf = d->w2_sf; sa.w_scale = d->w2_scale;
+    sa.topk_w = F32(L.topk_w);
+    sa.slots = F32(L.slots);
+    st = launch_stream_gemv_a16(1, sa, max_active_experts(d), s);
+    if (st != NVFP4MOE_OK) return st;
+    mark(5);
+    st = launch_combine(F32(L.slots), int64_t(T) * k * H, 1, I32(L.pair_to_row), T, H, k, out, s);
+    if (st != NVFP4MOE_OK) return st;
+    mark(6);
+    return mark_st;
+  }
   if (L.path == NVFP4MOE_PATH_GEMV) {
     // x quantised once per token, token-major
     mark(3);
@@ -245,10 +270,6 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
     g.w13_codes = d->w13_codes; g.w13_sf = d->w13_sf; g.w13_scale = d->w13_scale;
     g.h_scale = d->h_scale; g.h_amax = d->h_amax;
     g.h_codes = ws + L.h_codes; g.h_sf = ws + L.h_sf;
-    if (a16) {  // weight-only: bf16 x in, bf16 h out
-      g.x_bf16 = static_cast<const uint16_t*>(x);
-      g.h_bf16 = reinterpret_cast<uint16_t*>(ws + L.h_bf16);
-    }
     st = launch_gemv_gateup(g, max_active_experts(d), s);
     if (st != NVFP4MOE_OK) return st;
     mark(4);
@@ -260,7 +281,6 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
     dn.w2_codes = d->w2_codes; dn.w2_sf = d->w2_sf; dn.w2_scale = d->w2_scale;
     dn.h_scale = d->h_scale; dn.topk_w = F32(L.topk_w);
     dn.slots = F32(L.slots); dn.slot_stride = int64_t(T) * k * H;
-    if (a16) dn.h_bf16 = reinterpret_cast<const uint16_t*>(ws + L.h_bf16);
     st = launch_gemv_down(dn, max_active_experts(d), s);
     if (st != NVFP4MOE_OK) return st;
     mark(5);

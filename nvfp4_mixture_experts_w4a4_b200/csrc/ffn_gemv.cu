@@ -20,7 +20,7 @@ constexpr int kWarpsPerCta = 4;
 constexpr int kMinCtas = 4;
 
 // ------------------------------------------------------------- gate / up ----
-template <int L, int NT, bool A16>
+template <int L, int NT>
 __device__ __forceinline__ void gateup_group(const GemvGateUpArgs& a, int e, int64_t item_row0,
                                              int64_t r_first, float sg, float su, float sh,
                                              float (*tots)[4]) {
@@ -36,10 +36,7 @@ __device__ __forceinline__ void gateup_group(const GemvGateUpArgs& a, int e, int
 #pragma unroll
   for (int G = 0; G < GROUPS; ++G) {
     float tot[8][NT];
-    if (A16)
-      warp_dot8_w4a16<L, NT>(wc, wsf, item_row0 + G * 8 * RP, 2 * I, a.x_bf16, arow, H, 0, H / 32, tot);
-    else
-      warp_dot8<L, NT>(wc, wsf, item_row0 + G * 8 * RP, 2 * I, a.x_codes, a.x_sf, arow, H, 0, H / 32, tot);
+    warp_dot8<L, NT>(wc, wsf, item_row0 + G * 8 * RP, 2 * I, a.x_codes, a.x_sf, arow, H, 0, H / 32, tot);
     if (lane % L == 0) {
 #pragma unroll
       for (int q = 0; q < 8; ++q)
@@ -56,13 +53,6 @@ __device__ __forceinline__ void gateup_group(const GemvGateUpArgs& a, int e, int
       const float g = tots[lane][t] * sg;
       const float u = tots[16 + lane][t] * su;
       h = g / (1.0f + expf(-g)) * u;
-    }
-    if (A16) {  // weight-only: h is the down projection's bf16 activation
-      if (lane < 16) {
-        const __nv_bfloat16 hb = __float2bfloat16_rn(h);
-        a.h_bf16[(r_first + t) * I + iblk * 16 + lane] = *reinterpret_cast<const uint16_t*>(&hb);
-      }
-      continue;
     }
     float amax = fabsf(h);
 #pragma unroll
@@ -82,29 +72,29 @@ __device__ __forceinline__ void gateup_group(const GemvGateUpArgs& a, int e, int
   __syncwarp();
 }
 
-template <int L, bool A16>
+template <int L>
 __global__ void __launch_bounds__(kWarpsPerCta * 32, kMinCtas) gemv_gateup_kernel(GemvGateUpArgs a) {
   __shared__ float tots_all[kWarpsPerCta][32][4];
   const int warp = threadIdx.x >> 5;
   float(*tots)[4] = tots_all[warp];
   const int64_t per_expert = (2 * int64_t(a.I)) / 32;
   const int64_t n_items = int64_t(a.active[0]) * per_expert;
-  const float s_x = A16 ? 1.0f : *a.x_scale;
+  const float s_x = *a.x_scale;
   for (int64_t item = int64_t(blockIdx.x) * kWarpsPerCta + warp; item < n_items;
        item += int64_t(gridDim.x) * kWarpsPerCta) {
     const int e = a.active[1 + item / per_expert];
     const int64_t row0 = (item % per_expert) * 32;
     const int64_t r0 = a.offsets[e], n_e = a.offsets[e + 1] - r0;
     const float sg = a.w13_scale[2 * e] * s_x, su = a.w13_scale[2 * e + 1] * s_x;
-    const float sh = A16 ? 1.0f : a.h_scale[e];
+    const float sh = a.h_scale[e];
     int64_t g = 0;
-    for (; g + 2 <= n_e; g += 2) gateup_group<L, 2, A16>(a, e, row0, r0 + g, sg, su, sh, tots);
-    if (g < n_e) gateup_group<L, 1, A16>(a, e, row0, r0 + g, sg, su, sh, tots);
+    for (; g + 2 <= n_e; g += 2) gateup_group<L, 2>(a, e, row0, r0 + g, sg, su, sh, tots);
+    if (g < n_e) gateup_group<L, 1>(a, e, row0, r0 + g, sg, su, sh, tots);
   }
 }
 
 // ------------------------------------------------------------------ down ----
-template <int L, int NT, bool A16>
+template <int L, int NT>
 __device__ __forceinline__ void down_group(const GemvDownArgs& a, int e, int64_t item_row0,
                                            int64_t r_first, int64_t c0, int64_t c1, float sc,
                                            float* slots) {
@@ -126,10 +116,7 @@ __device__ __forceinline__ void down_group(const GemvDownArgs& a, int e, int64_t
 #pragma unroll
   for (int G = 0; G < GROUPS; ++G) {
     float tot[8][NT];
-    if (A16)
-      warp_dot8_w4a16<L, NT>(wc, wsf, item_row0 + G * 8 * RP, H, a.h_bf16, arow, I, c0, c1, tot);
-    else
-      warp_dot8<L, NT>(wc, wsf, item_row0 + G * 8 * RP, H, a.h_codes, a.h_sf, arow, I, c0, c1, tot);
+    warp_dot8<L, NT>(wc, wsf, item_row0 + G * 8 * RP, H, a.h_codes, a.h_sf, arow, I, c0, c1, tot);
     if (lane % L == 0) {
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
@@ -143,7 +130,7 @@ __device__ __forceinline__ void down_group(const GemvDownArgs& a, int e, int64_t
   }
 }
 
-template <int L, bool A16>
+template <int L>
 __global__ void __launch_bounds__(kWarpsPerCta * 32, kMinCtas) gemv_down_kernel(GemvDownArgs a) {
   const int warp = threadIdx.x >> 5;
   const int64_t H = a.H, I = a.I;
@@ -162,10 +149,10 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kMinCtas) gemv_down_kernel(
     const int64_t c1 = c0 + cps < nchunks ? c0 + cps : nchunks;
     float* slots = a.slots + split * a.slot_stride;
     const int64_t r0 = a.offsets[e], n_e = a.offsets[e + 1] - r0;
-    const float sc = (A16 ? 1.0f : a.h_scale[e]) * a.w2_scale[e];
+    const float sc = a.h_scale[e] * a.w2_scale[e];
     int64_t g = 0;
-    for (; g + 2 <= n_e; g += 2) down_group<L, 2, A16>(a, e, row0, r0 + g, c0, c1, sc, slots);
-    if (g < n_e) down_group<L, 1, A16>(a, e, row0, r0 + g, c0, c1, sc, slots);
+    for (; g + 2 <= n_e; g += 2) down_group<L, 2>(a, e, row0, r0 + g, c0, c1, sc, slots);
+    if (g < n_e) down_group<L, 1>(a, e, row0, r0 + g, c0, c1, sc, slots);
   }
 }
 
@@ -262,34 +249,15 @@ int gemv_lanes_per_row(int64_t K) {
   return chunks >= 32 ? 32 : (chunks >= 16 ? 16 : 8);
 }
 
-namespace {
-template <bool A16>
-void gateup_launch(const GemvGateUpArgs& a, int L, int64_t items, cudaStream_t s) {
-  if (L == 32)
-    gemv_gateup_kernel<32, A16><<<grid_for(gemv_gateup_kernel<32, A16>, items), kWarpsPerCta * 32, 0, s>>>(a);
-  else if (L == 16)
-    gemv_gateup_kernel<16, A16><<<grid_for(gemv_gateup_kernel<16, A16>, items), kWarpsPerCta * 32, 0, s>>>(a);
-  else
-    gemv_gateup_kernel<8, A16><<<grid_for(gemv_gateup_kernel<8, A16>, items), kWarpsPerCta * 32, 0, s>>>(a);
-}
-template <bool A16>
-void down_launch(const GemvDownArgs& a, int L, int64_t items, cudaStream_t s) {
-  if (L == 32)
-    gemv_down_kernel<32, A16><<<grid_for(gemv_down_kernel<32, A16>, items), kWarpsPerCta * 32, 0, s>>>(a);
-  else if (L == 16)
-    gemv_down_kernel<16, A16><<<grid_for(gemv_down_kernel<16, A16>, items), kWarpsPerCta * 32, 0, s>>>(a);
-  else
-    gemv_down_kernel<8, A16><<<grid_for(gemv_down_kernel<8, A16>, items), kWarpsPerCta * 32, 0, s>>>(a);
-}
-}  // namespace
-
 nvfp4moe_status launch_gemv_gateup(const GemvGateUpArgs& a, int64_t max_active, cudaStream_t s) {
   const int L = gemv_lanes_per_row(a.H);
   const int64_t items = max_active * (2 * int64_t(a.I) / 32);
-  if (a.x_bf16)
-    gateup_launch<true>(a, L, items, s);
+  if (L == 32)
+    gemv_gateup_kernel<32><<<grid_for(gemv_gateup_kernel<32>, items), kWarpsPerCta * 32, 0, s>>>(a);
+  else if (L == 16)
+    gemv_gateup_kernel<16><<<grid_for(gemv_gateup_kernel<16>, items), kWarpsPerCta * 32, 0, s>>>(a);
   else
-    gateup_launch<false>(a, L, items, s);
+    gemv_gateup_kernel<8><<<grid_for(gemv_gateup_kernel<8>, items), kWarpsPerCta * 32, 0, s>>>(a);
   return check_launch("gemv gate/up");
 }
 
@@ -308,10 +276,12 @@ int gemv_down_ksplit(int64_t max_active, int64_t H, int64_t I) {
 nvfp4moe_status launch_gemv_down(const GemvDownArgs& a, int64_t max_active, cudaStream_t s) {
   const int L = gemv_lanes_per_row(a.I);
   const int64_t items = max_active * ((int64_t(a.H) + 31) / 32) * a.ksplit;
-  if (a.h_bf16)
-    down_launch<true>(a, L, items, s);
+  if (L == 32)
+    gemv_down_kernel<32><<<grid_for(gemv_down_kernel<32>, items), kWarpsPerCta * 32, 0, s>>>(a);
+  else if (L == 16)
+    gemv_down_kernel<16><<<grid_for(gemv_down_kernel<16>, items), kWarpsPerCta * 32, 0, s>>>(a);
   else
-    down_launch<false>(a, L, items, s);
+    gemv_down_kernel<8><<<grid_for(gemv_down_kernel<8>, items), kWarpsPerCta * 32, 0, s>>>(a);
   return check_launch("gemv down");
 }
 

@@ -20,10 +20,6 @@ struct GemvGateUpArgs {
   float* h_amax;            // nullable [E]
   uint8_t* h_codes;         // [P][I/2]
   uint8_t* h_sf;            // MMA layout over P rows
-  // weight-only (W4A16) layer when x_bf16 is set: x is read in bf16 [T][H], h is written in
-  // bf16 [P][I] (x_codes, x_sf, x_scale, h_scale, h_codes, h_sf unused)
-  const uint16_t* x_bf16;
-  uint16_t* h_bf16;
 };
 
 struct GemvDownArgs {
@@ -41,8 +37,27 @@ struct GemvDownArgs {
   const float* topk_w;      // [P] by pair; nullable (weight 1)
   float* slots;             // [ksplit][P][H]
   int64_t slot_stride;      // P*H
-  const uint16_t* h_bf16;   // weight-only layer when set: h in bf16 [P][I] (h codes unused)
 };
+
+// Weight-only (W4A16) expert products for the layer's GEMV path, with the weights streamed by
+// the copy engine through shared memory (stream_gemv.cu).  epi 0: gate/up (act = x [T][H] bf16
+// by token, writes h_out bf16 [P][I]); epi 1: down (act = h [P][I] bf16 by permuted row,
+// writes weighted fp32 slot rows [P][H] by pair).  Needs 2I % 128 == 0 and H % 128 == 0.
+struct StreamA16Args {
+  int H, I, E;
+  const uint16_t* act;
+  const int32_t* offsets;    // [E+1] unpadded permutation
+  const int32_t* row_token;  // [P]
+  const int32_t* row_pair;   // [P]
+  const int32_t* active;     // [E+1]
+  const uint8_t* w_codes;    // W13 [E][2I][H/2] or W2 [E][H][I/2]
+  const uint8_t* w_sf;       // MMA layout per expert
+  const float* w_scale;      // W13: [E][2]; W2: [E]
+  const float* topk_w;       // [P] by pair (down)
+  uint16_t* h_out;           // gate/up output
+  float* slots;              // down output
+};
+nvfp4moe_status launch_stream_gemv_a16(int epi, const StreamA16Args& a, int64_t max_active, cudaStream_t s);
 
 int gemv_lanes_per_row(int64_t K);
 int gemv_down_ksplit(int64_t max_active, int64_t H, int64_t I);

@@ -115,83 +115,8 @@ __device__ __forceinline__ void warp_dot8(const uint8_t* __restrict__ wc, const 
       for (int o = L / 2; o > 0; o >>= 1) tot[q][t] += __shfl_xor_sync(0xffffffffu, tot[q][t], o);
 }
 
-// The weight-only (W4A16) form: the activations are bf16 rows (act + arow[t] * K), taken as
-// 32 values (four 16-byte loads) per weight chunk.  Codes are widened to f16 (exact) and then
-// to fp32; products and the two block sums are fp32, each block sum is multiplied by its
-// E4M3 weight scale.  Same lane split, row set and result as warp_dot8.
+// bf16 halves of a 32-bit word (element 2i in the low half) as fp32.
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-template <int L, int NT>
-__device__ __forceinline__ void warp_dot8_w4a16(const uint8_t* __restrict__ wc, const uint8_t* __restrict__ wsf,
-                                                int64_t row0, int64_t nrows, const uint16_t* __restrict__ act,
-                                                const int64_t arow[NT], int64_t K, int64_t c_begin, int64_t c_end,
-                                                float tot[8][NT]) {
-  constexpr int RP = 32 / L;
-  const int lane = threadIdx.x & 31;
-  const int s = lane / L, cl = lane % L;
-  const int64_t rb = K / 2;
-#pragma unroll
-  for (int q = 0; q < 8; ++q)
-#pragma unroll
-    for (int t = 0; t < NT; ++t) tot[q][t] = 0.0f;
-  for (int64_t c = c_begin + cl; c < c_end; c += L) {
-    uint4 wv[8];
-    uint32_t ws[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int64_t r = row0 + q * RP + s;
-      if (r < nrows) {
-        wv[q] = ldg_stream16(wc + r * rb + c * 16);
-        ws[q] = ldg_u16(wsf + sf_mma_offset(r, 2 * c, K));
-      } else {
-        wv[q] = make_uint4(0, 0, 0, 0);
-        ws[q] = 0;
-      }
-    }
-    uint32_t xw[NT][16];
-#pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      const uint4* src = reinterpret_cast<const uint4*>(act + arow[t] * K + c * 32);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 v = __ldg(src + i);
-        xw[t][4 * i] = v.x;
-        xw[t][4 * i + 1] = v.y;
-        xw[t][4 * i + 2] = v.z;
-        xw[t][4 * i + 3] = v.w;
-      }
-    }
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      uint32_t wf[16];
-      decode_chunk(wv[q], wf);
-      const float2 wsc = decode_sf2(ws[q]);
-#pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        float b0 = 0.0f, b1 = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float2 w2 = __half22float2(*reinterpret_cast<const __half2*>(&wf[i]));
-          b0 = __fmaf_rn(w2.x, bf16_lo(xw[t][i]), b0);
-          b0 = __fmaf_rn(w2.y, bf16_hi(xw[t][i]), b0);
-        }
-#pragma unroll
-        for (int i = 8; i < 16; ++i) {
-          const float2 w2 = __half22float2(*reinterpret_cast<const __half2*>(&wf[i]));
-          b1 = __fmaf_rn(w2.x, bf16_lo(xw[t][i]), b1);
-          b1 = __fmaf_rn(w2.y, bf16_hi(xw[t][i]), b1);
-        }
-        tot[q][t] = __fmaf_rn(b1, wsc.y, __fmaf_rn(b0, wsc.x, tot[q][t]));
-      }
-    }
-  }
-#pragma unroll
-  for (int q = 0; q < 8; ++q)
-#pragma unroll
-    for (int t = 0; t < NT; ++t)
-#pragma unroll
-      for (int o = L / 2; o > 0; o >>= 1) tot[q][t] += __shfl_xor_sync(0xffffffffu, tot[q][t], o);
-}
 
 }  // namespace nvfp4moe
