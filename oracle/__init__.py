@@ -96,6 +96,14 @@ def _declare(L):
                               _i32p, _i32p, _i32p]
     L.orc_moe_ffn.restype = ctypes.c_int
     L.orc_moe_ffn.argtypes = [ctypes.POINTER(MoeArgs)]
+    L.orc_e8m0_value.restype = ctypes.c_double
+    L.orc_e8m0_value.argtypes = [ctypes.c_int]
+    L.orc_mx_quantize.restype = ctypes.c_int
+    L.orc_mx_quantize.argtypes = [_f32p, ctypes.c_int64, ctypes.c_int64, _u8p, _u8p]
+    L.orc_mx_dequantize.restype = None
+    L.orc_mx_dequantize.argtypes = [_u8p, _u8p, ctypes.c_int64, ctypes.c_int64, _f64p]
+    L.orc_mx_to_nvfp4.restype = ctypes.c_int
+    L.orc_mx_to_nvfp4.argtypes = [_u8p, _u8p, ctypes.c_int64, ctypes.c_int64, _u8p, _f32p]
     L.orc_moe_ffn_w4a16.restype = ctypes.c_int
     L.orc_moe_ffn_w4a16.argtypes = [ctypes.POINTER(MoeW4A16Args)]
 
@@ -349,3 +357,54 @@ def moe_ffn_w4a16(x_bf16: np.ndarray, logits: np.ndarray, k: int, wg, wu, wd, *,
     if rc != 0:
         raise ValueError(f"orc_moe_ffn_w4a16 failed ({rc})")
     return r
+
+
+# ------------------------------------------------------------------ MXFP4 (R11) ----
+def e8m0_value(code: int) -> float:
+    return lib().orc_e8m0_value(int(code))
+
+
+def mx_quantize(x: np.ndarray):
+    """MXFP4 quantisation of fp32 [rows, K] (K % 32 == 0): codes [rows, K/2] u8 and E8M0
+    scales [rows, K/32] u8."""
+    x = np.ascontiguousarray(x, np.float32)
+    rows, K = x.shape
+    codes = np.zeros((rows, K // 2), np.uint8)
+    e8m0 = np.zeros((rows, K // 32), np.uint8)
+    if lib().orc_mx_quantize(_p(x, ctypes.c_float), rows, K, _p(codes, ctypes.c_uint8), _p(e8m0, ctypes.c_uint8)):
+        raise ValueError("orc_mx_quantize: K must be a multiple of 32")
+    return codes, e8m0
+
+
+def mx_dequantize(codes: np.ndarray, e8m0: np.ndarray) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, np.uint8)
+    e8m0 = np.ascontiguousarray(e8m0, np.uint8)
+    rows, K = codes.shape[0], codes.shape[1] * 2
+    out = np.zeros((rows, K), np.float64)
+    lib().orc_mx_dequantize(_p(codes, ctypes.c_uint8), _p(e8m0, ctypes.c_uint8), rows, K, _p(out, ctypes.c_double))
+    return out
+
+
+def mx_to_nvfp4(codes: np.ndarray, e8m0: np.ndarray):
+    """The exact NVFP4 form of an MXFP4 matrix: (codes unchanged, row-major E4M3 scales
+    [rows, K/16], tensor scale).  Raises ValueError when no exact form exists."""
+    codes = np.ascontiguousarray(codes, np.uint8)
+    e8m0 = np.ascontiguousarray(e8m0, np.uint8)
+    rows, K = codes.shape[0], codes.shape[1] * 2
+    sf = np.zeros((rows, K // 16), np.uint8)
+    ts = np.zeros(1, np.float32)
+    rc = lib().orc_mx_to_nvfp4(_p(codes, ctypes.c_uint8), _p(e8m0, ctypes.c_uint8), rows, K, _p(sf, ctypes.c_uint8),
+                               _p(ts, ctypes.c_float))
+    if rc:
+        raise ValueError(f"orc_mx_to_nvfp4 failed ({rc})")
+    return codes, sf, float(ts[0])
+
+
+def mx_experts_to_nvfp4(codes: np.ndarray, e8m0: np.ndarray):
+    """mx_to_nvfp4 per expert of stacked [E, N, ...] arrays: (codes, sf [E, N, K/16], scale [E])."""
+    E = codes.shape[0]
+    sf = np.zeros(codes.shape[:2] + (codes.shape[2] // 8,), np.uint8)
+    sc = np.zeros(E, np.float32)
+    for e in range(E):
+        _, sf[e], sc[e] = mx_to_nvfp4(codes[e], e8m0[e])
+    return codes, sf, sc

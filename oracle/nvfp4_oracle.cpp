@@ -39,6 +39,15 @@
 //   R8 SwiGLU: h = silu(g) * u with silu(g) = g / (1 + exp(-g)).
 //   R9 combine: out[t] = sum over slots j = 0..k-1 (in order) of w[t][j] * y[t][j],
 //      rounded once to bf16 (fp64 -> fp32 -> bf16, each round to nearest even).
+//   R11 MXFP4 (the DwarfStar launcher's default format, read as the OCP microscaling
+//      definition): E2M1 elements, one E8M0 scale 2^(E-127) per 32 consecutive elements
+//      along K, no tensor scale; quantisation takes X = floor(log2(amax)) - 2 (2 = the
+//      largest E2M1 exponent), clamped to [-127, 127], and codes e2m1(x / 2^X) (R1, so values
+//      above 6 * 2^X saturate); an all-zero block gets E = 0.  Element packing as R4.
+//      MXFP4 weights enter the NVFP4 layer exactly: a power of two 2^j is an E4M3 value for
+//      j in [-9, 8], so each 16-element half of a block takes the E4M3 scale 2^(E-127-shift)
+//      and the matrix the tensor scale 2^shift, shift = (largest E of a nonzero block) - 135;
+//      a matrix whose nonzero blocks span more than 18 binades has no exact form (refused).
 //   R10 weight-only variant (W4A16; the NInfer card's "Limits" names NVFP4 weights without
 //      an activation-quantisation site): x enters the gate/up products as bf16, the
 //      intermediate h = silu(g) * u is rounded to bf16 (fp64 -> fp32 -> bf16) as the down
@@ -228,6 +237,10 @@ void parallel_for(int64_t n, int nthreads, F fn) {
   }
   for (auto& th : pool) th.join();
 }
+
+// ---------------------------------------------------------------- E8M0 ----
+// Unsigned power-of-two scale: 2^(code - 127); 0xFF is NaN.
+double e8m0_value(int code) { return code == 255 ? NAN : std::ldexp(1.0, code - 127); }
 
 }  // namespace
 
@@ -614,6 +627,77 @@ int orc_moe_ffn_w4a16(const orc_moe_w4a16_args* a) {
   put(a->pair_to_row, pair_to_row);
   put(a->h_bf16, h);
   put(a->y_f64, y);
+  return 0;
+}
+
+
+// ---------------------------------------------------------------- MXFP4 (R11) ----
+double orc_e8m0_value(int code) { return e8m0_value(code & 255); }
+
+// Quantises rows x K fp32 values to MXFP4: codes [rows][K/2], e8m0 [rows][K/32].
+int orc_mx_quantize(const float* x, int64_t rows, int64_t K, uint8_t* codes, uint8_t* e8m0) {
+  if (K % 32 != 0 || rows < 0) return -1;
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t b = 0; b < K / 32; ++b) {
+      const float* v = x + r * K + b * 32;
+      float amax = 0.0f;
+      for (int i = 0; i < 32; ++i) amax = std::max(amax, std::fabs(v[i]));
+      int X = -127;
+      if (amax > 0.0f) {
+        int e = 0;
+        std::frexp(static_cast<double>(amax), &e);  // amax = m 2^e, m in [0.5, 1): floor(log2) = e - 1
+        X = std::min(127, std::max(-127, e - 1 - 2));
+      }
+      e8m0[r * (K / 32) + b] = static_cast<uint8_t>(X + 127);
+      for (int i = 0; i < 32; ++i) {
+        const float q = static_cast<float>(std::ldexp(static_cast<double>(v[i]), -X));  // exact
+        const int c = e2m1_encode(q);
+        const int64_t k = b * 32 + i;
+        uint8_t& byte = codes[r * (K / 2) + k / 2];
+        byte = (k & 1) ? static_cast<uint8_t>((byte & 0x0F) | (c << 4)) : static_cast<uint8_t>((byte & 0xF0) | c);
+      }
+    }
+  return 0;
+}
+
+// v = e2m1(code) * 2^(E - 127), in fp64.
+void orc_mx_dequantize(const uint8_t* codes, const uint8_t* e8m0, int64_t rows, int64_t K, double* out) {
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t k = 0; k < K; ++k) {
+      const uint8_t byte = codes[r * (K / 2) + k / 2];
+      const int c = (k & 1) ? (byte >> 4) : (byte & 0xF);
+      out[r * K + k] = e2m1_value(c) * e8m0_value(e8m0[r * (K / 32) + k / 32]);
+    }
+}
+
+// The NVFP4 form of an MXFP4 matrix (R11): the codes are unchanged; writes the row-major
+// E4M3 block scales sf [rows][K/16] and the tensor scale.  Returns -3 when the nonzero
+// blocks span more than 18 binades.
+int orc_mx_to_nvfp4(const uint8_t* codes, const uint8_t* e8m0, int64_t rows, int64_t K, uint8_t* sf,
+                    float* tensor_scale) {
+  if (K % 32 != 0 || rows < 0) return -1;
+  auto nonzero = [&](int64_t r, int64_t b) {
+    for (int i = 0; i < 16; ++i)
+      if (codes[r * (K / 2) + b * 16 + i] & 0x77) return true;  // a nonzero magnitude nibble
+    return false;
+  };
+  int emax = -1;
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t b = 0; b < K / 32; ++b)
+      if (nonzero(r, b)) emax = std::max(emax, int(e8m0[r * (K / 32) + b]));
+  const int shift = emax < 0 ? 0 : emax - 127 - 8;
+  *tensor_scale = static_cast<float>(std::ldexp(1.0, shift));
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t b = 0; b < K / 32; ++b) {
+      uint8_t code = 0;
+      if (nonzero(r, b)) {
+        const int j = int(e8m0[r * (K / 32) + b]) - 127 - shift;
+        if (j < -9) return -3;
+        code = static_cast<uint8_t>(e4m3_encode(static_cast<float>(std::ldexp(1.0, j))));
+      }
+      sf[r * (K / 16) + 2 * b] = code;
+      sf[r * (K / 16) + 2 * b + 1] = code;
+    }
   return 0;
 }
 

@@ -428,3 +428,71 @@ def test_w4a16_identity_experts_closed_form():
             h = float(_bf16_round(xf[t, n] / (1 + math.exp(-xf[t, n])) * xf[t, n]))
             want = sum(wts[j] * float(c[ids[t, j]]) * h for j in range(k))
             assert abs(r["out_f64"][t, n] - want) <= 1e-6 * max(abs(want), 1e-30), (t, n)
+
+
+# -------------------------------------------------------------------- MXFP4 ----
+def test_e8m0_table_vs_ml_dtypes():
+    F80 = ml_dtypes.float8_e8m0fnu
+    for c in range(256):
+        ref = float(np.array([c], np.uint8).view(F80)[0])
+        got = O.e8m0_value(c)
+        assert (np.isnan(ref) and np.isnan(got)) or ref == got, c
+
+
+def _mx_golden():
+    with open(os.path.join(HERE, "golden", "mx_blocks.json")) as f:
+        return json.load(f)["blocks"]
+
+
+@pytest.mark.parametrize("blk", _mx_golden(), ids=lambda b: b["name"])
+def test_mx_hand_worked_blocks(blk):
+    x = np.array(blk["x"], np.float32)[None, :]
+    codes, e8m0 = O.mx_quantize(x)
+    assert int(e8m0[0, 0]) == blk["e8m0"]
+    unpacked = [(int(codes[0, i // 2]) >> (4 * (i % 2))) & 0xF for i in range(32)]
+    assert unpacked == blk["codes"]
+
+
+def test_mx_quantiser_vs_numpy_formulation():
+    """MX quantisation written with numpy (frexp for the exponent) and ml_dtypes' E2M1 cast,
+    bit for bit on random blocks of several magnitudes."""
+    rng = np.random.default_rng(11)
+    x = (rng.standard_normal((24, 128)) * np.exp2(rng.integers(-20, 20, (24, 1)))).astype(np.float32)
+    x[3, :32] = 0.0
+    codes, e8m0 = O.mx_quantize(x)
+    blocks = x.reshape(24, 4, 32).astype(np.float64)
+    amax = np.abs(blocks).max(axis=2)
+    _, e = np.frexp(amax)
+    X = np.where(amax > 0, np.clip(e - 3, -127, 127), -127)
+    assert np.array_equal(e8m0, (X + 127).astype(np.uint8))
+    q = np.clip(blocks / np.exp2(X)[..., None], -6.0, 6.0).astype(np.float32)
+    ref = q.astype(F4).view(np.uint8).reshape(24, 128) & 0xF
+    got = np.stack([(codes >> 0) & 0xF, codes >> 4], axis=2).reshape(24, 128)
+    assert np.array_equal(got, ref)
+
+
+def test_mx_roundtrip_of_representable_blocks():
+    """A block built from E2M1 values times one power of two comes back exactly."""
+    rng = np.random.default_rng(12)
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float64)
+    vals = grid[rng.integers(0, 8, (16, 64))] * np.where(rng.random((16, 64)) < 0.5, -1, 1)
+    vals[:, ::32] = 6.0  # pin each block's largest magnitude to 6 so X is the power chosen below
+    p = np.exp2(rng.integers(-30, 30, (16, 2)).repeat(32, axis=1))
+    x = (vals * p).astype(np.float32)
+    codes, e8m0 = O.mx_quantize(x)
+    assert np.array_equal(O.mx_dequantize(codes, e8m0), x.astype(np.float64))
+
+
+def test_mx_to_nvfp4_is_exact_and_refuses_wide_spans():
+    rng = np.random.default_rng(13)
+    x = (rng.standard_normal((32, 256)) * np.exp2(rng.integers(-8, 9, (32, 1)))).astype(np.float32)
+    codes, e8m0 = O.mx_quantize(x)
+    c2, sf, ts = O.mx_to_nvfp4(codes, e8m0)
+    assert np.array_equal(c2, codes)
+    assert np.array_equal(O.dequantize(codes, sf, ts), O.mx_dequantize(codes, e8m0))
+    # 2^-20 next to 2^0 spans more than the 18 binades of E4M3 powers of two
+    y = np.ones((2, 64), np.float32)
+    y[1, :32] = 2.0 ** -20
+    c, e = O.mx_quantize(y)
+    with pytest.raises(ValueError):
+        O.mx_to_nvfp4(c, e)
