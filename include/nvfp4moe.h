@@ -169,6 +169,30 @@ nvfp4moe_status nvfp4_quantize_dynamic_noalloc(const void* x, int32_t x_dtype, i
                                                int32_t sf_layout, nvfp4moe_stream_t stream);
 
 /* ------------------------------------------------------------------------------
+ * nvfp4_from_mxfp4 - the exact NVFP4 form of MXFP4 weight matrices, so that MXFP4 weights
+ * run on every path of the layer.  MXFP4 (the DwarfStar CUDA multi-GPU doc's launcher default,
+ * read as the OCP microscaling definition): E2M1 codes packed as NVFP4's (element 2i in the
+ * low nibble of byte i) and one E8M0 scale 2^(E-127) per 32 elements along K.  A power of two
+ * 2^j is an E4M3 value for j in [-9, 8]: both 16-element halves of a block get the E4M3 scale
+ * 2^(E-127-shift) and the matrix the fp32 tensor scale 2^shift, shift = (largest E of a
+ * block with a nonzero code) - 135; a zero block gets scale 0.
+ *
+ * codes [batch][rows][K/2], e8m0 [batch][rows][K/32] (device).  Out row r of each matrix
+ * takes input row row_gather[r] (nullable: r; -1: the row is left untouched, for building
+ * the interleaved W13 from gate and up in two calls), out_rows rows.  Writes
+ * sf_out [batch][sf_mma_bytes(out_rows, K)] (MMA layout), tensor_scale [batch], and, when
+ * codes_out is non-null, the codes [batch][out_rows][K/2].  K % 64 == 0; codes 16-byte
+ * aligned.  Workspace: nvfp4_from_mxfp4_workspace_size(batch) bytes.  Synchronous (a setup
+ * step): returns NVFP4MOE_UNSUPPORTED_SHAPE, naming the matrices, when the scales of a
+ * matrix's nonzero blocks span more than 18 binades (no exact NVFP4 form).
+ * ---------------------------------------------------------------------------- */
+size_t nvfp4_from_mxfp4_workspace_size(int64_t batch);
+nvfp4moe_status nvfp4_from_mxfp4(const uint8_t* codes, const uint8_t* e8m0, int64_t batch, int64_t rows,
+                                 int64_t K, const int32_t* row_gather, int64_t out_rows,
+                                 uint8_t* codes_out, uint8_t* sf_out, float* tensor_scale,
+                                 void* workspace, size_t workspace_bytes, nvfp4moe_stream_t stream);
+
+/* ------------------------------------------------------------------------------
  * moe_route - router top-k (DwarfStar CUDA multi-GPU doc: routers run replicated next to
  * the routed experts).
  * logits: fp32 [T][E] (finite).  ids: int32 [T][k], experts in descending logit order,

@@ -70,6 +70,8 @@ SIGNATURES = {
                               _i64, _vp, _i64, _i32, _vp, _sz, _vp]),
     "nvfp4_quantize_dynamic_noalloc": (_i32, [_vp, _i32, _i64, _i64, _i64, _i64, _i64, _vp, _i64, _vp, _vp,
                                               _i64, _vp, _i64, _i32, _vp]),
+    "nvfp4_from_mxfp4_workspace_size": (_sz, [_i64]),
+    "nvfp4_from_mxfp4": (_i32, [_vp, _vp, _i64, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_route": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moe_permute_rows_capacity": (_i64, [_i32, _i32, _i32, _i32]),
     "moe_permute": (_i32, [_vp, _i32, _i32, _i32, _i32, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp,

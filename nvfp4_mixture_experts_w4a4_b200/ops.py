@@ -153,6 +153,35 @@ def nvfp4_gemm(A: torch.Tensor, A_sf: torch.Tensor, a_scale: torch.Tensor, B: to
     return D
 
 
+def nvfp4_from_mxfp4(codes: torch.Tensor, e8m0: torch.Tensor, row_gather: torch.Tensor | None = None,
+                     out_rows: int | None = None, codes_out: torch.Tensor | None = None,
+                     sf_out: torch.Tensor | None = None):
+    """The exact NVFP4 form of MXFP4 matrices codes [B, rows, K/2] / [rows, K/2] with E8M0 scales
+    [.., rows, K/32]: returns (codes, MMA-layout sf [B, sf_mma_bytes(out_rows, K)], tensor scale [B]).
+    Synchronous; raises when a matrix has no exact form."""
+    _need_cuda(codes, e8m0)
+    squeeze = codes.dim() == 2
+    if squeeze:
+        codes, e8m0 = codes[None], e8m0[None]
+    codes, e8m0 = codes.contiguous(), e8m0.contiguous()
+    B, rows, K = codes.shape[0], codes.shape[1], codes.shape[2] * 2
+    out_rows = rows if out_rows is None else out_rows
+    dev = codes.device
+    if sf_out is None:
+        sf_out = torch.empty(B, sf_mma_bytes(out_rows, K), dtype=torch.uint8, device=dev)
+    scale = torch.empty(B, dtype=torch.float32, device=dev)
+    wsb = lib().nvfp4_from_mxfp4_workspace_size(B)
+    ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+    gather = None if row_gather is None else row_gather.to(torch.int32).contiguous()
+    st = lib().nvfp4_from_mxfp4(_p(codes), _p(e8m0), B, rows, K, _p(gather), out_rows, _p(codes_out), _p(sf_out),
+                                _p(scale), _p(ws), wsb, _s())
+    check(st, "nvfp4_from_mxfp4")
+    out_codes = codes if codes_out is None else codes_out
+    if squeeze:
+        return out_codes[0], sf_out[0], scale
+    return out_codes, sf_out, scale
+
+
 class NVFP4Experts:
     """Per-expert NVFP4 weights in the library's layout (W13 interleaved, MMA scales)."""
 
@@ -170,6 +199,22 @@ class NVFP4Experts:
         gate = torch.where(j < 16, 16 * c + j, torch.full_like(r, -1))
         up = torch.where(j >= 16, 16 * c + j - 16, torch.full_like(r, -1))
         return gate, up
+
+    @classmethod
+    def from_mxfp4(cls, gate: tuple, up: tuple, down: tuple) -> "NVFP4Experts":
+        """MXFP4 expert weights, each (codes [E, N, K/2], E8M0 scales [E, N, K/32]) for gate/up
+        [E, I, H] and down [E, H, I], in their exact NVFP4 form (nvfp4_from_mxfp4)."""
+        E, I, h2 = gate[0].shape
+        H = h2 * 2
+        dev = gate[0].device
+        g_map, u_map = cls.interleave_maps(I, dev)
+        w13_codes = torch.empty(E, 2 * I, H // 2, dtype=torch.uint8, device=dev)
+        w13_sf = torch.empty(E, sf_mma_bytes(2 * I, H), dtype=torch.uint8, device=dev)
+        _, _, sg = nvfp4_from_mxfp4(gate[0], gate[1], g_map, 2 * I, w13_codes, w13_sf)
+        _, _, su = nvfp4_from_mxfp4(up[0], up[1], u_map, 2 * I, w13_codes, w13_sf)
+        w2_codes, w2_sf, sd = nvfp4_from_mxfp4(down[0], down[1])
+        return cls(w13_codes, w13_sf, torch.stack([sg, su], 1).contiguous(), w2_codes.contiguous(), w2_sf,
+                   sd.contiguous())
 
     @classmethod
     def from_float(cls, w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor) -> "NVFP4Experts":

@@ -253,3 +253,44 @@ def check_layer_w4a16(wl: W.Workload, ref: dict, out: torch.Tensor, layer: ops.M
     assert not bad.any(), f"h differs beyond one bf16 step: gpu {vg[bad][:4]} oracle {vr[bad][:4]}"
     print(f"[parity w4a16] {wl.name} T={T}: {int(diff.sum())} of {diff.size} h values differ")
     return check_out(bf16_bits(out), ref["out_f64"])
+
+
+def mx_experts(wts):
+    """MXFP4 weights of a workload (oracle MX quantiser on the fp32 draws): dict of (codes, e8m0)
+    per matrix, [E, N, K/2] and [E, N, K/32]."""
+    out = {}
+    for name in ("w_gate", "w_up", "w_down"):
+        w = wts[name].numpy()
+        mx = [O.mx_quantize(w[e]) for e in range(w.shape[0])]
+        out[name] = (np.stack([m[0] for m in mx]), np.stack([m[1] for m in mx]))
+    return out
+
+
+def run_layer_pair_mxfp4(wl: W.Workload, path: int, act_mode: int = C.ACT_NVFP4, seed: int = 0, dev=None):
+    """MXFP4 weights: the device converts them (NVFP4Experts.from_mxfp4), the oracle converts its
+    own copy (reading R11); both layers then run on those weights."""
+    dev = dev or need_gpu()
+    act = W.make_activations(wl, seed, "cpu")
+    wts = W.make_weights(wl, seed, "cpu")
+    mx = mx_experts(wts)
+    wg, wu, wd = (O.mx_experts_to_nvfp4(*mx[n]) for n in ("w_gate", "w_up", "w_down"))
+    to = lambda t: torch.from_numpy(np.ascontiguousarray(t)).to(dev)  # noqa: E731
+    experts = ops.NVFP4Experts.from_mxfp4(*((to(mx[n][0]), to(mx[n][1])) for n in ("w_gate", "w_up", "w_down")))
+    torch.cuda.synchronize()
+    ref_w = LY.experts_to_device_layout(wg, wu, wd)
+    got_w = [experts.w13_codes, experts.w13_sf, experts.w13_scale, experts.w2_codes, experts.w2_sf, experts.w2_scale]
+    for r, g in zip(ref_w, got_w):
+        assert np.array_equal(g.cpu().numpy(), r)
+    x_bits = bf16_bits(act["x"])
+    logits = act["logits"].numpy()
+    if act_mode == C.ACT_BF16:
+        ref = O.moe_ffn_w4a16(x_bits, logits, wl.k, wg, wu, wd)
+        layer = ops.MoeFFN(experts, wl.k, None, act=C.ACT_BF16)
+    else:
+        ref = O.moe_ffn(x_bits, logits, wl.k, wg, wu, wd)
+        layer = ops.MoeFFN(experts, wl.k, torch.from_numpy(ref["h_scale"]).to(dev), path=path)
+    h_amax = torch.empty(wl.E, dtype=torch.float32, device=dev)
+    out = layer(act["x"].to(dev), act["logits"].to(dev), h_amax=None if act_mode == C.ACT_BF16 else h_amax)
+    torch.cuda.synchronize()
+    layer.oracle_wd = wd
+    return ref, out, layer, h_amax

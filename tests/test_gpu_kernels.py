@@ -198,3 +198,36 @@ def test_gemm_parity(dev, M, N, K):
     Db = ops.nvfp4_gemm(t(ac), t(LY.to_mma(asf, K)), torch.tensor([sa], device=dev), t(bc),
                         t(LY.to_mma(bsf, K)), torch.tensor([sb], device=dev), out_dtype=torch.bfloat16)
     G.check_out(G.bf16_bits(Db), ref)
+
+
+def _mx_matrices(B, rows, K, seed):
+    """MXFP4 matrices from the oracle's MX quantiser: rows of different magnitudes, a zero row
+    and a zero block."""
+    rng = np.random.default_rng(seed)
+    x = (rng.standard_normal((B, rows, K)) * np.exp2(rng.integers(-5, 6, (B, rows, 1)))).astype(np.float32)
+    x[0, 1] = 0.0
+    x[-1, 2, 32:64] = 0.0
+    mx = [O.mx_quantize(x[b]) for b in range(B)]
+    return np.stack([m[0] for m in mx]), np.stack([m[1] for m in mx])
+
+
+@pytest.mark.parametrize("B,rows,K", [(1, 3, 64), (3, 130, 256), (2, 256, 2048)])
+def test_from_mxfp4_matches_oracle(dev, B, rows, K):
+    """The exact NVFP4 form of MXFP4 matrices: codes unchanged, E4M3 block scales and the tensor
+    scale bit-exact against the oracle's conversion (reading R11)."""
+    codes, e8m0 = _mx_matrices(B, rows, K, seed=rows)
+    c_d, sf_d, sc_d = ops.nvfp4_from_mxfp4(torch.from_numpy(codes).to(dev), torch.from_numpy(e8m0).to(dev))
+    torch.cuda.synchronize()
+    for b in range(B):
+        _, sf_ref, sc_ref = O.mx_to_nvfp4(codes[b], e8m0[b])
+        assert np.array_equal(LY.from_mma(sf_d[b].cpu().numpy(), rows, K), sf_ref)
+        assert sc_d[b].item() == np.float32(sc_ref)
+    assert np.array_equal(c_d.cpu().numpy(), codes)
+
+
+def test_from_mxfp4_refuses_spans_without_an_exact_form(dev):
+    y = np.ones((4, 64), np.float32)
+    y[2, :32] = 2.0 ** -20  # 20 binades below the largest block
+    c, e = O.mx_quantize(y)
+    with pytest.raises(C.Nvfp4MoeError, match="18 binades"):
+        ops.nvfp4_from_mxfp4(torch.from_numpy(c).to(dev), torch.from_numpy(e).to(dev))

@@ -200,3 +200,18 @@ def test_weight_only_rejects_the_tensor_core_path():
     layer = ops.MoeFFN(G.experts_from_oracle(wg, wu, wd, dev), wl.k, None, path=C.PATH_GEMM, act=C.ACT_BF16)
     with pytest.raises(C.Nvfp4MoeError):
         layer(act["x"].to(dev), act["logits"].to(dev))
+
+
+@pytest.mark.parametrize("name,path,act", [("tiny", C.PATH_GEMM, C.ACT_NVFP4), ("decode_shape", C.PATH_GEMM, C.ACT_NVFP4),
+                                           ("long_prefill_small", C.PATH_GEMM, C.ACT_NVFP4),
+                                           ("tiny", C.PATH_GEMV, C.ACT_NVFP4), ("decode_shape", C.PATH_AUTO, C.ACT_BF16)])
+def test_layer_mxfp4_weights(name, path, act):
+    """MXFP4 weights on the NVFP4 layer: the device's exact NVFP4 form equals the oracle's
+    (codes, scales, tensor scales, bit for bit), and the layer meets the usual tolerances."""
+    wl = GEMM_CASES[name]
+    ref, out, layer, h_amax = G.run_layer_pair_mxfp4(wl, path, act)
+    if act == C.ACT_BF16:
+        G.check_layer_w4a16(wl, ref, out, layer)
+    else:
+        G.check_layer(wl, ref, out, layer, h_amax)
+    assert ops.device_status() == 0
