@@ -48,6 +48,7 @@ class MoeArgs(ctypes.Structure):
         ("row_token", _i32p), ("row_slot", _i32p), ("pair_to_row", _i32p),
         ("x_codes", _u8p), ("x_sf", _u8p), ("h_f32", _f32p), ("h_codes", _u8p),
         ("h_sf", _u8p), ("h_amax", _f32p), ("y_f64", _f64p),
+        ("shared_I", ctypes.c_int32), ("shared_g", _u16p), ("shared_u", _u16p), ("shared_d", _u16p),
     ]
 
 
@@ -62,6 +63,7 @@ class MoeW4A16Args(ctypes.Structure):
         ("out_bf16", _u16p), ("out_f64", _f64p),
         ("ids", _i32p), ("w", _f32p), ("counts", _i32p), ("offsets", _i32p),
         ("row_token", _i32p), ("pair_to_row", _i32p), ("h_bf16", _u16p), ("y_f64", _f64p),
+        ("shared_I", ctypes.c_int32), ("shared_g", _u16p), ("shared_u", _u16p), ("shared_d", _u16p),
     ]
 
 
@@ -242,8 +244,19 @@ def quantize_experts(w: np.ndarray):
     return codes, sf, sc
 
 
+def _set_shared(a, shared, keep: list):
+    """shared: None or (g [I_s, H], u [I_s, H], d [H, I_s]) bf16 bit patterns (reading R12)."""
+    if shared is None:
+        a.shared_I = 0
+        return
+    g, u, d = (np.ascontiguousarray(v, np.uint16) for v in shared)
+    keep += [g, u, d]
+    a.shared_I = g.shape[0]
+    a.shared_g, a.shared_u, a.shared_d = (_p(v, ctypes.c_uint16) for v in (g, u, d))
+
+
 def moe_ffn(x_bf16: np.ndarray, logits: np.ndarray, k: int, wg, wu, wd, *, x_scale=None,
-            h_scale=None, nthreads: int | None = None, want_y: bool = False) -> dict:
+            h_scale=None, nthreads: int | None = None, want_y: bool = False, shared=None) -> dict:
     """Runs the whole layer on the CPU.
 
     x_bf16: uint16 [T, H] bf16 bit patterns; logits fp32 [T, E];
@@ -301,7 +314,8 @@ def moe_ffn(x_bf16: np.ndarray, logits: np.ndarray, k: int, wg, wu, wd, *, x_sca
                      ("y_f64", ctypes.c_double)):
         setattr(a, name, _p(r[name], ct))
     # keep every buffer alive for the duration of the call
-    keep = (x_bf16, logits, wg, wu, wd, xs, hs, r)
+    keep = [x_bf16, logits, wg, wu, wd, xs, hs, r]
+    _set_shared(a, shared, keep)
     rc = lib().orc_moe_ffn(ctypes.byref(a))
     del keep
     if rc != 0:
@@ -312,7 +326,7 @@ def moe_ffn(x_bf16: np.ndarray, logits: np.ndarray, k: int, wg, wu, wd, *, x_sca
 
 
 def moe_ffn_w4a16(x_bf16: np.ndarray, logits: np.ndarray, k: int, wg, wu, wd, *,
-                  nthreads: int | None = None, want_y: bool = False) -> dict:
+                  nthreads: int | None = None, want_y: bool = False, shared=None) -> dict:
     """The weight-only (W4A16) layer on the CPU (reading R10 of nvfp4_oracle.cpp): bf16 x
     into the gate/up products, h rounded to bf16, NVFP4 weights dequantised, fp64 sums.
     Arguments as for moe_ffn.  Returns out_bf16, out_f64, the routing and permutation, and
@@ -351,7 +365,8 @@ def moe_ffn_w4a16(x_bf16: np.ndarray, logits: np.ndarray, k: int, wg, wu, wd, *,
                      ("pair_to_row", ctypes.c_int32), ("h_bf16", ctypes.c_uint16),
                      ("y_f64", ctypes.c_double)):
         setattr(a, name, _p(r[name], ct))
-    keep = (x_bf16, logits, wg, wu, wd, r)
+    keep = [x_bf16, logits, wg, wu, wd, r]
+    _set_shared(a, shared, keep)
     rc = lib().orc_moe_ffn_w4a16(ctypes.byref(a))
     del keep
     if rc != 0:

@@ -48,6 +48,11 @@
 //      j in [-9, 8], so each 16-element half of a block takes the E4M3 scale 2^(E-127-shift)
 //      and the matrix the tensor scale 2^shift, shift = (largest E of a nonzero block) - 135;
 //      a matrix whose nonzero blocks span more than 18 binades has no exact form (refused).
+//   R12 shared expert (the SSD-Stream card's "shared experts ... remain BF16"; replicated
+//      beside the routed experts in DwarfStar's expert-parallel pairs): a dense SwiGLU MLP
+//      with bf16 weights, ys = Wd_s . bf16(silu(Wg_s x) * (Wu_s x)) for every token, x in bf16,
+//      products and sums in fp64, its h rounded to bf16 (fp64 -> fp32 -> bf16); the layer's
+//      output is bf16(routed + ys), one rounding of the fp64 sum.
 //   R10 weight-only variant (W4A16; the NInfer card's "Limits" names NVFP4 weights without
 //      an activation-quantisation site): x enters the gate/up products as bf16, the
 //      intermediate h = silu(g) * u is rounded to bf16 (fp64 -> fp32 -> bf16) as the down
@@ -238,6 +243,31 @@ void parallel_for(int64_t n, int nthreads, F fn) {
   for (auto& th : pool) th.join();
 }
 
+// ------------------------------------------------------- shared expert (R12) ----
+// ys[t][n] for all T tokens: bf16 weights g, u [I][H] and d [H][I].
+std::vector<double> shared_expert(const uint16_t* x_bf16, int64_t T, int64_t H, int64_t I, const uint16_t* g,
+                                  const uint16_t* u, const uint16_t* d, int nth) {
+  std::vector<double> ys(static_cast<size_t>(T * H), 0.0);
+  parallel_for(T, nth, [&](int64_t t) {
+    std::vector<double> h(static_cast<size_t>(I));
+    for (int64_t i = 0; i < I; ++i) {
+      double gv = 0.0, uv = 0.0;
+      for (int64_t c = 0; c < H; ++c) {
+        const double xv = bf16_to_float(x_bf16[t * H + c]);
+        gv += xv * double(bf16_to_float(g[i * H + c]));
+        uv += xv * double(bf16_to_float(u[i * H + c]));
+      }
+      h[size_t(i)] = double(bf16_to_float(float_to_bf16(static_cast<float>(gv / (1.0 + std::exp(-gv)) * uv))));
+    }
+    for (int64_t n = 0; n < H; ++n) {
+      double acc = 0.0;
+      for (int64_t i = 0; i < I; ++i) acc += h[size_t(i)] * double(bf16_to_float(d[n * I + i]));
+      ys[size_t(t * H + n)] = acc;
+    }
+  });
+  return ys;
+}
+
 // ---------------------------------------------------------------- E8M0 ----
 // Unsigned power-of-two scale: 2^(code - 127); 0xFF is NaN.
 double e8m0_value(int code) { return code == 255 ? NAN : std::ldexp(1.0, code - 127); }
@@ -384,6 +414,11 @@ struct orc_moe_args {
   uint8_t* h_sf;             // [T*k][I/16]
   float* h_amax;             // [E]
   double* y_f64;             // [T*k][H], down-projection per permuted row, before w
+  // optional shared expert (R12): shared_I = 0 for none; bf16 gate/up [I_s][H], down [H][I_s]
+  int32_t shared_I;
+  const uint16_t* shared_g;
+  const uint16_t* shared_u;
+  const uint16_t* shared_d;
 };
 
 int orc_moe_ffn(const orc_moe_args* a) {
@@ -476,7 +511,9 @@ int orc_moe_ffn(const orc_moe_args* a) {
     }
   });
 
-  // 6. weighted combine (R9)
+  // 6. weighted combine (R9), plus the shared expert (R12)
+  std::vector<double> ys;
+  if (a->shared_I > 0) ys = shared_expert(a->x_bf16, T, H, a->shared_I, a->shared_g, a->shared_u, a->shared_d, nth);
   for (int t = 0; t < T; ++t)
     for (int64_t n = 0; n < H; ++n) {
       double acc = 0.0;
@@ -484,6 +521,7 @@ int orc_moe_ffn(const orc_moe_args* a) {
         const int64_t r = pair_to_row[size_t(int64_t(t) * k + j)];
         acc += double(w[size_t(int64_t(t) * k + j)]) * y[size_t(r * H + n)];
       }
+      if (!ys.empty()) acc += ys[size_t(int64_t(t) * H + n)];
       if (a->out_f64) a->out_f64[int64_t(t) * H + n] = acc;
       a->out_bf16[int64_t(t) * H + n] = float_to_bf16(static_cast<float>(acc));
     }
@@ -537,6 +575,10 @@ struct orc_moe_w4a16_args {
   int32_t* pair_to_row;      // [T*k]
   uint16_t* h_bf16;          // [T*k][I], permuted rows
   double* y_f64;             // [T*k][H], down projection per permuted row, before w
+  int32_t shared_I;          // optional shared expert (R12), as in orc_moe_args
+  const uint16_t* shared_g;
+  const uint16_t* shared_u;
+  const uint16_t* shared_d;
 };
 
 namespace {
@@ -604,7 +646,9 @@ int orc_moe_ffn_w4a16(const orc_moe_w4a16_args* a) {
       }
   });
 
-  // 4. weighted combine (R9)
+  // 4. weighted combine (R9), plus the shared expert (R12)
+  std::vector<double> ys;
+  if (a->shared_I > 0) ys = shared_expert(a->x_bf16, T, H, a->shared_I, a->shared_g, a->shared_u, a->shared_d, nth);
   for (int t = 0; t < T; ++t)
     for (int64_t n = 0; n < H; ++n) {
       double acc = 0.0;
@@ -612,6 +656,7 @@ int orc_moe_ffn_w4a16(const orc_moe_w4a16_args* a) {
         const int64_t r = pair_to_row[size_t(int64_t(t) * k + j)];
         acc += double(w[size_t(int64_t(t) * k + j)]) * y[size_t(r * H + n)];
       }
+      if (!ys.empty()) acc += ys[size_t(int64_t(t) * H + n)];
       if (a->out_f64) a->out_f64[int64_t(t) * H + n] = acc;
       a->out_bf16[int64_t(t) * H + n] = float_to_bf16(static_cast<float>(acc));
     }

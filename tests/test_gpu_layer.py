@@ -215,3 +215,19 @@ def test_layer_mxfp4_weights(name, path, act):
     else:
         G.check_layer(wl, ref, out, layer, h_amax)
     assert ops.device_status() == 0
+
+
+@pytest.mark.parametrize("path,act", [(C.PATH_GEMM, C.ACT_NVFP4), (C.PATH_GEMV, C.ACT_NVFP4), (C.PATH_AUTO, C.ACT_BF16)])
+def test_layer_empty_batch(path, act):
+    """T = 0: the call succeeds, launches nothing and leaves an empty output."""
+    wl = CASES["tiny"]
+    dev = G.need_gpu()
+    act_d, wts, wg, wu, wd = G.layer_inputs(wl)
+    experts = G.experts_from_oracle(wg, wu, wd, dev)
+    layer = ops.MoeFFN(experts, wl.k, None if act == C.ACT_BF16 else torch.ones(wl.E, device=dev), path=path, act=act)
+    x = torch.empty(0, wl.H, dtype=torch.bfloat16, device=dev)
+    logits = torch.empty(0, wl.E, dtype=torch.float32, device=dev)
+    out = layer(x, logits)
+    torch.cuda.synchronize()
+    assert out.shape == (0, wl.H)
+    assert ops.device_status() == 0

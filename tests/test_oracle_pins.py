@@ -496,3 +496,54 @@ def test_mx_to_nvfp4_is_exact_and_refuses_wide_spans():
     c, e = O.mx_quantize(y)
     with pytest.raises(ValueError):
         O.mx_to_nvfp4(c, e)
+
+
+# ------------------------------------------------------------- shared expert ----
+def _bf16_bits(a):
+    return torch.from_numpy(np.asarray(a, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_shared_expert_identity_closed_form():
+    """Shared expert with identity gate/up and down = c * I (bf16, exact): the layer output moves
+    by exactly c * bf16(silu(x) x) per element (math.exp), with the routed part unchanged."""
+    import math
+    wl, x, logits, wg, wu, wd = _tiny_layer_inputs(T=4, H=256, I=128, E=4, k=2)
+    H = wl.H
+    eye = np.eye(H, dtype=np.float32)
+    c = 0.75
+    shared = (_bf16_bits(eye), _bf16_bits(eye), _bf16_bits(c * eye))
+    r0 = O.moe_ffn(x, logits, wl.k, wg, wu, wd, nthreads=2)
+    r1 = O.moe_ffn(x, logits, wl.k, wg, wu, wd, h_scale=r0["h_scale"], x_scale=r0["x_scale"], shared=shared,
+                   nthreads=2)
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    for t in range(wl.T):
+        for n in range(H):
+            v = xf[t, n]
+            want = c * float(_bf16_round(v / (1 + math.exp(-v)) * v))
+            assert abs((r1["out_f64"][t, n] - r0["out_f64"][t, n]) - want) <= 1e-9 * max(1.0, abs(want))
+    # the weight-only layer adds the same term
+    a0 = O.moe_ffn_w4a16(x, logits, wl.k, wg, wu, wd, nthreads=2)
+    a1 = O.moe_ffn_w4a16(x, logits, wl.k, wg, wu, wd, shared=shared, nthreads=2)
+    assert np.allclose(a1["out_f64"] - a0["out_f64"], r1["out_f64"] - r0["out_f64"], rtol=0, atol=1e-9)
+
+
+def test_shared_expert_vs_numpy_formulation():
+    """Random bf16 shared weights: the added term equals Wd . bf16(silu(Wg x) (Wu x)) written with
+    numpy matmuls and torch's bf16 rounding."""
+    rng = np.random.default_rng(21)
+    wl, x, logits, wg, wu, wd = _tiny_layer_inputs(T=5, H=256, I=128, E=4, k=2)
+    Is = 64
+    g = rng.standard_normal((Is, wl.H)) / 16
+    u = rng.standard_normal((Is, wl.H)) / 16
+    d = rng.standard_normal((wl.H, Is)) / 8
+    shared = (_bf16_bits(g), _bf16_bits(u), _bf16_bits(d))
+    back = lambda b: (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)  # noqa: E731
+    r0 = O.moe_ffn(x, logits, wl.k, wg, wu, wd, nthreads=2)
+    r1 = O.moe_ffn(x, logits, wl.k, wg, wu, wd, h_scale=r0["h_scale"], x_scale=r0["x_scale"], shared=shared,
+                   nthreads=2)
+    xf = back(x)
+    gv = xf @ back(shared[0]).T
+    uv = xf @ back(shared[1]).T
+    h = _bf16_round(gv / (1 + np.exp(-gv)) * uv)
+    ys = h @ back(shared[2]).T
+    assert np.abs((r1["out_f64"] - r0["out_f64"]) - ys).max() <= 1e-9 * np.abs(ys).max()
