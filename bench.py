@@ -166,11 +166,12 @@ def setup_layer(wl: W.Workload, dev, seed: int = 0, keep_tokens: int = 0, path: 
     return act, host, experts, layer
 
 
-def algorithmic(wl: W.Workload, n_active: int, gemm_path: bool, a16: bool = False):
+def algorithmic(wl: W.Workload, n_active: int, gemm_path: bool, a16: bool = False, shared_I: int = 0):
     """Algorithmic (compulsory) bytes and FLOPs of one layer pass and of its gate/up stage:
     each touched expert's weights once, the quantised activations once (per permuted row on
     the tensor-core path, which gathers x into expert order), h written and read once.
-    Weight-only (a16): x and h in bf16."""
+    Weight-only (a16): x and h in bf16.  A shared expert adds its bf16 weights and its FLOPs to
+    the layer (not to the gate/up stage)."""
     e = FP4_BYTES_PER_ELT
     P = wl.T * wl.k
     w13 = n_active * 2 * wl.I * wl.H * e
@@ -178,8 +179,8 @@ def algorithmic(wl: W.Workload, n_active: int, gemm_path: bool, a16: bool = Fals
     x_q = (P if gemm_path else wl.T) * wl.H * (2 if a16 else e)
     h_q = P * wl.I * (2 if a16 else e)
     gate_up_bytes = w13 + x_q + h_q
-    layer_bytes = w13 + w2 + wl.T * wl.H * 2 * 2 + x_q + 2 * h_q + wl.T * wl.E * 4
-    flops = 2.0 * P * 3 * wl.H * wl.I
+    layer_bytes = w13 + w2 + wl.T * wl.H * 2 * 2 + x_q + 2 * h_q + wl.T * wl.E * 4 + 3 * wl.H * shared_I * 2
+    flops = 2.0 * P * 3 * wl.H * wl.I + 2.0 * wl.T * 3 * wl.H * shared_I
     # both GEMMs in one launch (small batches): weights, x and h codes, fp32 slot rows
     gemms_bytes = w13 + w2 + x_q + 2 * h_q + P * wl.H * 4
     return {"gate_up_bytes": gate_up_bytes, "layer_bytes": layer_bytes, "flops": flops,
@@ -369,7 +370,8 @@ def oracle_inputs(wl: W.Workload, act, host, tokens: np.ndarray):
     return x[tokens], logits[tokens], arrays, float(s_x)
 
 
-def oracle_rate(wl: W.Workload, act, host, layer, budget_s: float, max_tokens: int, a16: bool = False):
+def oracle_rate(wl: W.Workload, act, host, layer, budget_s: float, max_tokens: int, a16: bool = False,
+                shared=None):
     """Tokens/s of the oracle on a bounded token sample of the workload (host cores)."""
     import oracle as O
     n = min(wl.T, max_tokens)
@@ -380,9 +382,10 @@ def oracle_rate(wl: W.Workload, act, host, layer, budget_s: float, max_tokens: i
     done, t0 = 0, time.perf_counter()
     while True:
         if a16:
-            O.moe_ffn_w4a16(x, logits, wl.k, arr["g"], arr["u"], arr["d"], nthreads=nth)
+            O.moe_ffn_w4a16(x, logits, wl.k, arr["g"], arr["u"], arr["d"], nthreads=nth, shared=shared)
         else:
-            O.moe_ffn(x, logits, wl.k, arr["g"], arr["u"], arr["d"], x_scale=s_x, h_scale=s_h, nthreads=nth)
+            O.moe_ffn(x, logits, wl.k, arr["g"], arr["u"], arr["d"], x_scale=s_x, h_scale=s_h, nthreads=nth,
+                      shared=shared)
         done += n
         el = time.perf_counter() - t0
         if el >= budget_s or done >= 64 * n:
@@ -408,6 +411,8 @@ def main():
                     help="layer path: auto (GEMV for T <= 16), the GEMV path or the tcgen05 grouped GEMM")
     ap.add_argument("--act", default="nvfp4", choices=["nvfp4", "bf16"],
                     help="activations: nvfp4 (W4A4) or bf16 (the weight-only W4A16 variant, GEMV path)")
+    ap.add_argument("--shared-I", type=int, default=0,
+                    help="add a BF16 shared expert of this intermediate size (0: none)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -428,6 +433,8 @@ def main():
     a16 = args.act == "bf16"
     if a16:
         cfg["act"] = "w4a16 (bf16 activations, NVFP4 weights)"
+    if args.shared_I:
+        cfg["shared_expert"] = f"bf16 SwiGLU, I_s={args.shared_I}"
 
     if args.impl == "reference":
         if rank != 0:
@@ -473,8 +480,19 @@ def main():
     path = {"auto": C.PATH_AUTO, "gemv": C.PATH_GEMV, "tcgen05": C.PATH_GEMM}[args.path]
     act, host, experts, layer = setup_layer(wl, dev, keep_tokens=n_cpu if (rank == 0 and world == 1) else 0,
                                             path=path)
+    shared, shared_bits = None, None
+    if args.shared_I:  # a BF16 shared expert, N(0, 1/sqrt(fan_in)) rounded to bf16
+        gen = torch.Generator(device=dev).manual_seed(7)
+        Is = args.shared_I
+        sg = (torch.randn(Is, wl.H, generator=gen, device=dev) / wl.H ** 0.5).to(torch.bfloat16)
+        su = (torch.randn(Is, wl.H, generator=gen, device=dev) / wl.H ** 0.5).to(torch.bfloat16)
+        sd = (torch.randn(wl.H, Is, generator=gen, device=dev) / Is ** 0.5).to(torch.bfloat16)
+        shared = (ops.shared_expert_w13(sg, su), sd)
+        shared_bits = tuple(t.cpu().view(torch.int16).numpy().view(np.uint16) for t in (sg, su, sd))
     if a16:  # the same experts, weight-only
-        layer = ops.MoeFFN(experts, wl.k, None, act=C.ACT_BF16)
+        layer = ops.MoeFFN(experts, wl.k, None, act=C.ACT_BF16, shared=shared)
+    elif shared is not None:
+        layer = ops.MoeFFN(experts, wl.k, layer.h_scale, path=path, shared=shared)
     flush = L2Flush(dev)
     with ClockSampler(local) as clk:
         step_ms, stage_ms, launches = time_steps(layer, act, args.steps, args.warmup, flush, dist_on)
@@ -486,7 +504,7 @@ def main():
     im = layer.intermediates(wl.T)
     n_active = int(im["active"][0].item())
     gemm_path = im["path"] == C.PATH_GEMM
-    alg = algorithmic(wl, n_active, gemm_path, a16)
+    alg = algorithmic(wl, n_active, gemm_path, a16, args.shared_I)
     pk = peaks()
     # the dominant kernel: for batches of at most 64 tokens on the tensor-core path with H <= 2I
     # both GEMMs run in one fused launch (its stage is "gate_up"); otherwise the gate/up GEMM
@@ -512,7 +530,8 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, sample = oracle_rate(wl, act, host, layer, args.cpu_budget, max_tokens=n_cpu, a16=a16)
+        v, cores, sample = oracle_rate(wl, act, host, layer, args.cpu_budget, max_tokens=n_cpu, a16=a16,
+                                       shared=shared_bits)
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
 
     if rank == 0:

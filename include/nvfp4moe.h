@@ -289,6 +289,15 @@ typedef struct {
    * when given, receives the maxima as well). */
   int32_t h_scale_mode;
   int32_t act_mode;           /* NVFP4MOE_ACT_* */
+  /* Optional shared expert, a dense BF16 SwiGLU MLP beside the routed experts (the SSD-Stream
+   * card: "shared experts ... remain BF16"): shared_I = its intermediate size (0: none;
+   * else a positive multiple of 64), shared_w13 bf16 [2*shared_I][H] with gate and up rows
+   * interleaved like w13_codes (rows 32c+j: gate row 16c+j for j < 16, up row 16c+j-16
+   * otherwise), shared_w2 bf16 [H][shared_I].  out = bf16(routed + w2 . bf16(silu(g) * u)),
+   * one rounding of the fp32 sum; the shared expert's products are fp32. */
+  int32_t shared_I;
+  const uint16_t* shared_w13;
+  const uint16_t* shared_w2;
 } moe_ffn_desc;
 
 enum { NVFP4MOE_STAGES = 7 };
@@ -310,6 +319,8 @@ typedef struct {
   int64_t h_stats;  /* dynamic h scale: amax[E] then the scales used, s_h[E] (fp32) */
   int64_t h_bf16;   /* weight-only layer: h in bf16 [T*k][I], permuted rows (x_codes, x_sf,
                        h_codes, h_sf are empty then) */
+  int64_t shared_h; /* shared expert: its h in bf16 [T][shared_I] */
+  int64_t shared_y; /* shared expert: its output rows in fp32 [T][H] */
 } moe_ffn_ws_layout;
 
 nvfp4moe_status moe_ffn_workspace_layout(const moe_ffn_desc* d, moe_ffn_ws_layout* layout);

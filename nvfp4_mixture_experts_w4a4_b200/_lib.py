@@ -46,7 +46,7 @@ class MoeFfnDesc(ctypes.Structure):
         ("w13_codes", _vp), ("w13_sf", _vp), ("w13_scale", _vp),
         ("w2_codes", _vp), ("w2_sf", _vp), ("w2_scale", _vp),
         ("h_scale", _vp), ("h_amax", _vp), ("stage_events", _vp), ("combine", _i32), ("h_scale_mode", _i32),
-        ("act_mode", _i32),
+        ("act_mode", _i32), ("shared_I", _i32), ("shared_w13", _vp), ("shared_w2", _vp),
     ]
 
 
@@ -56,7 +56,7 @@ class MoeFfnWsLayout(ctypes.Structure):
         "row_pair", "tile_expert", "active", "x_scale", "x_codes", "x_sf", "h_codes", "h_sf",
         "slots", "amax_partials", "total", "x_rows", "h_rows", "items")] + [
         ("m_tile", _i32), ("path", _i32), ("combine", _i32), ("reserved", _i32), ("h_f32", _i64), ("h_stats", _i64),
-        ("h_bf16", _i64)]
+        ("h_bf16", _i64), ("shared_h", _i64), ("shared_y", _i64)]
 
 
 # name -> (restype, argtypes)

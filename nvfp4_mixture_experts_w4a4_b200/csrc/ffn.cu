@@ -37,6 +37,8 @@ nvfp4moe_status check_desc(const moe_ffn_desc* d, const char* fn) {
                 "%s: bad act_mode %d", fn, d->act_mode);
   NVFP4_REQUIRE(d->act_mode != NVFP4MOE_ACT_BF16 || d->path != NVFP4MOE_PATH_GEMM, NVFP4MOE_UNSUPPORTED_SHAPE,
                 "%s: the weight-only layer runs the GEMV path", fn);
+  NVFP4_REQUIRE(d->shared_I >= 0 && d->shared_I % 64 == 0, NVFP4MOE_UNSUPPORTED_SHAPE,
+                "%s: shared_I=%d must be a multiple of 64", fn, d->shared_I);
   return NVFP4MOE_OK;
 }
 
@@ -101,6 +103,8 @@ void make_layout(const moe_ffn_desc* d, moe_ffn_ws_layout* L) {
   L->h_codes = take(L->h_rows * I / 2);
   L->h_sf = take(sf_mma_bytes(L->h_rows, I));
   L->h_bf16 = take(a16 ? P * I * 2 : 0);
+  L->shared_h = take(T * int64_t(d->shared_I) * 2);
+  L->shared_y = take(d->shared_I > 0 ? T * H * 4 : 0);
   // fp32 rows of the down projection: split-K partials by pair on the GEMV path; on the
   // tensor-core path rows by pair (up to 64 tokens) or by padded expert row (above), or the
   // [T][H] accumulator of the accumulating combine (the region also holds the batch
@@ -159,6 +163,8 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   NVFP4_REQUIRE(x && logits && out && workspace, NVFP4MOE_INVALID_ARG, "%s: NULL pointer", fn);
   NVFP4_REQUIRE(d->w13_codes && d->w13_sf && d->w13_scale && d->w2_codes && d->w2_sf && d->w2_scale,
                 NVFP4MOE_INVALID_ARG, "%s: NULL weight pointer in desc", fn);
+  NVFP4_REQUIRE(d->shared_I == 0 || (d->shared_w13 && d->shared_w2 && aligned16(d->shared_w13) && aligned16(d->shared_w2)),
+                NVFP4MOE_INVALID_ARG, "%s: the shared expert needs 16-byte aligned shared_w13 and shared_w2", fn);
   const bool a16 = d->act_mode == NVFP4MOE_ACT_BF16;  // weight-only: no activation scales
   NVFP4_REQUIRE(a16 || d->x_scale_mode == NVFP4MOE_SCALE_DYNAMIC || d->x_scale != nullptr, NVFP4MOE_INVALID_ARG,
                 "%s: GIVEN x scale needs desc->x_scale", fn);
@@ -214,6 +220,25 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   float* h_amax_int = dyn_h ? F32(L.h_stats) : (a16 ? nullptr : d->h_amax);
   float* h_scale_dyn = dyn_h ? F32(L.h_stats) + E : nullptr;
 
+  // the shared expert (bf16 weights, streamed like the weight-only products), run before the
+  // combine, which adds its fp32 rows; nullptr when there is none
+  float* shared_y = d->shared_I > 0 ? F32(L.shared_y) : nullptr;
+  auto run_shared = [&]() -> nvfp4moe_status {
+    if (!shared_y) return NVFP4MOE_OK;
+    StreamA16Args sa{};
+    sa.H = H; sa.I = d->shared_I; sa.E = 1;
+    sa.wbf16 = 1; sa.shared_T = T;
+    sa.act = static_cast<const uint16_t*>(x);
+    sa.w_codes = reinterpret_cast<const uint8_t*>(d->shared_w13);
+    sa.h_out = reinterpret_cast<uint16_t*>(ws + L.shared_h);
+    nvfp4moe_status r = launch_stream_gemv_a16(0, sa, 1, s);
+    if (r != NVFP4MOE_OK) return r;
+    sa.act = reinterpret_cast<const uint16_t*>(ws + L.shared_h);
+    sa.w_codes = reinterpret_cast<const uint8_t*>(d->shared_w2);
+    sa.slots = shared_y;
+    return launch_stream_gemv_a16(1, sa, 1, s);
+  };
+
   mark(0);
   if (fused) {
     // small batch: routing, permutation and x quantisation in one cluster launch
@@ -255,7 +280,9 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
     st = launch_stream_gemv_a16(1, sa, max_active_experts(d), s);
     if (st != NVFP4MOE_OK) return st;
     mark(5);
-    st = launch_combine(F32(L.slots), int64_t(T) * k * H, 1, I32(L.pair_to_row), T, H, k, out, s);
+    st = run_shared();
+    if (st != NVFP4MOE_OK) return st;
+    st = launch_combine(F32(L.slots), int64_t(T) * k * H, 1, I32(L.pair_to_row), T, H, k, out, s, shared_y);
     if (st != NVFP4MOE_OK) return st;
     mark(6);
     return mark_st;
@@ -284,7 +311,9 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
     st = launch_gemv_down(dn, max_active_experts(d), s);
     if (st != NVFP4MOE_OK) return st;
     mark(5);
-    st = launch_combine(F32(L.slots), dn.slot_stride, dn.ksplit, I32(L.pair_to_row), T, H, k, out, s);
+    st = run_shared();
+    if (st != NVFP4MOE_OK) return st;
+    st = launch_combine(F32(L.slots), dn.slot_stride, dn.ksplit, I32(L.pair_to_row), T, H, k, out, s, shared_y);
     if (st != NVFP4MOE_OK) return st;
     mark(6);
     return mark_st;
@@ -318,13 +347,15 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   a.slots_by_row = (!accumulate && !fused) ? 1 : 0;
   st = launch_grouped_ffn(a, s);
   if (st != NVFP4MOE_OK) return st;
+  st = run_shared();
+  if (st != NVFP4MOE_OK) return st;
   mark(5);
   if (accumulate)
-    st = launch_accum_to_bf16(accum, int64_t(T) * H, out, s);
+    st = launch_accum_to_bf16(accum, int64_t(T) * H, out, s, shared_y);
   else if (a.slots_by_row)
-    st = launch_combine_rows(F32(L.slots), I32(L.pair_to_row), F32(L.topk_w), T, H, k, out, s);
+    st = launch_combine_rows(F32(L.slots), I32(L.pair_to_row), F32(L.topk_w), T, H, k, out, s, shared_y);
   else
-    st = launch_combine(F32(L.slots), int64_t(T) * k * H, 1, I32(L.pair_to_row), T, H, k, out, s);
+    st = launch_combine(F32(L.slots), int64_t(T) * k * H, 1, I32(L.pair_to_row), T, H, k, out, s, shared_y);
   if (st != NVFP4MOE_OK) return st;
   mark(6);
   return mark_st;

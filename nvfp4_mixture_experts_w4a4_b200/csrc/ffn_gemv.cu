@@ -157,11 +157,20 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kMinCtas) gemv_down_kernel(
 }
 
 // --------------------------------------------------------------- combine ----
-// out[t][n] = bf16( sum_j sum_s slots[s][t*k + j][n] ), j and s ascending; pairs whose
-// row is -1 (skipped ids) contribute nothing.
+// out[t][n] = bf16( sum_j sum_s slots[s][t*k + j][n] (+ shared[t][n]) ), j and s ascending;
+// pairs whose row is -1 (skipped ids) contribute nothing.  shared (nullable): the shared
+// expert's fp32 output rows, added last.
+__device__ __forceinline__ void add_shared(float (&acc)[8], const float* shared, int64_t off) {
+  if (!shared) return;
+  const float4 a = *reinterpret_cast<const float4*>(shared + off);
+  const float4 b = *reinterpret_cast<const float4*>(shared + off + 4);
+  acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+  acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+}
+
 __global__ void combine_kernel(const float* __restrict__ slots, int64_t slot_stride, int ksplit,
                                const int32_t* __restrict__ pair_to_row, int T, int H, int k,
-                               __nv_bfloat16* __restrict__ out) {
+                               const float* __restrict__ shared, __nv_bfloat16* __restrict__ out) {
   (void)pair_to_row;  // every pair has a row: slots are addressed by pair directly
   griddep_wait();     // the slot rows come from the down GEMM launched just before
   const int64_t per_row = H / 8;
@@ -189,6 +198,7 @@ __global__ void combine_kernel(const float* __restrict__ slots, int64_t slot_str
           }
       }
     }
+    add_shared(acc, shared, t * H + n);
     uint4 o;
     uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
@@ -287,20 +297,21 @@ nvfp4moe_status launch_gemv_down(const GemvDownArgs& a, int64_t max_active, cuda
 
 nvfp4moe_status launch_combine(const float* slots, int64_t slot_stride, int ksplit,
                                const int32_t* pair_to_row, int T, int H, int k, void* out,
-                               cudaStream_t s) {
+                               cudaStream_t s, const float* shared) {
   const int64_t total = int64_t(T) * (H / 8);
   if (total == 0) return NVFP4MOE_OK;
   int64_t blocks = (total + 255) / 256;
   if (blocks > int64_t(num_sms()) * 8) blocks = int64_t(num_sms()) * 8;
   const cudaError_t e = launch_dependent(combine_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, slots,
-                                         slot_stride, ksplit, pair_to_row, T, H, k, static_cast<__nv_bfloat16*>(out));
+                                         slot_stride, ksplit, pair_to_row, T, H, k, shared,
+                                         static_cast<__nv_bfloat16*>(out));
   if (e != cudaSuccess) return fail(NVFP4MOE_CUDA_ERROR, "combine: %s", cudaGetErrorString(e));
   return check_launch("combine");
 }
 
 __global__ void combine_rows_kernel(const float* __restrict__ slots, const int32_t* __restrict__ pair_to_row,
                                     const float* __restrict__ topk_w, int T, int H, int k,
-                                    __nv_bfloat16* __restrict__ out) {
+                                    const float* __restrict__ shared, __nv_bfloat16* __restrict__ out) {
   griddep_wait();  // the slot rows come from the down GEMM launched just before
   const int64_t per_row = H / 8;
   const int64_t total = int64_t(T) * per_row;
@@ -331,6 +342,7 @@ __global__ void combine_rows_kernel(const float* __restrict__ slots, const int32
           acc[4] += wj[u] * b[u].x; acc[5] += wj[u] * b[u].y; acc[6] += wj[u] * b[u].z; acc[7] += wj[u] * b[u].w;
         }
     }
+    add_shared(acc, shared, t * H + n);
     uint4 o;
     uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
@@ -343,22 +355,28 @@ __global__ void combine_rows_kernel(const float* __restrict__ slots, const int32
 }
 
 nvfp4moe_status launch_combine_rows(const float* slots, const int32_t* pair_to_row, const float* topk_w, int T, int H,
-                                    int k, void* out, cudaStream_t s) {
+                                    int k, void* out, cudaStream_t s, const float* shared) {
   const int64_t total = int64_t(T) * (H / 8);
   if (total == 0) return NVFP4MOE_OK;
   int64_t blocks = (total + 255) / 256;
   if (blocks > int64_t(num_sms()) * 8) blocks = int64_t(num_sms()) * 8;
   const cudaError_t e = launch_dependent(combine_rows_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, slots,
-                                         pair_to_row, topk_w, T, H, k, static_cast<__nv_bfloat16*>(out));
+                                         pair_to_row, topk_w, T, H, k, shared, static_cast<__nv_bfloat16*>(out));
   if (e != cudaSuccess) return fail(NVFP4MOE_CUDA_ERROR, "combine (rows): %s", cudaGetErrorString(e));
   return check_launch("combine (rows)");
 }
 
-__global__ void accum_to_bf16_kernel(const float* __restrict__ acc, int64_t n, __nv_bfloat16* __restrict__ out) {
+__global__ void accum_to_bf16_kernel(const float* __restrict__ acc, int64_t n, const float* __restrict__ shared,
+                                     __nv_bfloat16* __restrict__ out) {
   griddep_wait();  // the accumulator is complete when the down GEMM is
   for (int64_t i = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) * 8; i < n; i += int64_t(gridDim.x) * blockDim.x * 8) {
-    const float4 a = *reinterpret_cast<const float4*>(acc + i);
-    const float4 b = *reinterpret_cast<const float4*>(acc + i + 4);
+    float4 a = *reinterpret_cast<const float4*>(acc + i);
+    float4 b = *reinterpret_cast<const float4*>(acc + i + 4);
+    if (shared) {  // the shared expert's rows, added last
+      const float4 sa = *reinterpret_cast<const float4*>(shared + i), sb = *reinterpret_cast<const float4*>(shared + i + 4);
+      a = make_float4(a.x + sa.x, a.y + sa.y, a.z + sa.z, a.w + sa.w);
+      b = make_float4(b.x + sb.x, b.y + sb.y, b.z + sb.z, b.w + sb.w);
+    }
     const __nv_bfloat162 q0 = __floats2bfloat162_rn(a.x, a.y), q1 = __floats2bfloat162_rn(a.z, a.w);
     const __nv_bfloat162 q2 = __floats2bfloat162_rn(b.x, b.y), q3 = __floats2bfloat162_rn(b.z, b.w);
     *reinterpret_cast<uint4*>(out + i) =
@@ -367,12 +385,12 @@ __global__ void accum_to_bf16_kernel(const float* __restrict__ acc, int64_t n, _
   }
 }
 
-nvfp4moe_status launch_accum_to_bf16(const float* acc, int64_t n, void* out, cudaStream_t s) {
+nvfp4moe_status launch_accum_to_bf16(const float* acc, int64_t n, void* out, cudaStream_t s, const float* shared) {
   if (n == 0) return NVFP4MOE_OK;
   int64_t blocks = (n / 8 + 255) / 256;
   if (blocks > int64_t(num_sms()) * 8) blocks = int64_t(num_sms()) * 8;
   const cudaError_t e = launch_dependent(accum_to_bf16_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, acc, n,
-                                         static_cast<__nv_bfloat16*>(out));
+                                         shared, static_cast<__nv_bfloat16*>(out));
   if (e != cudaSuccess) return fail(NVFP4MOE_CUDA_ERROR, "accumulator to bf16: %s", cudaGetErrorString(e));
   return check_launch("accumulator to bf16");
 }

@@ -56,6 +56,10 @@ struct StreamA16Args {
   const float* topk_w;       // [P] by pair (down)
   uint16_t* h_out;           // gate/up output
   float* slots;              // down output
+  // the shared expert (bf16 weights, no scales; E = 1): shared_T > 0 tokens taken in order
+  // (act rows 0..T-1, h_out [T][I], slots = its fp32 output rows [T][H], unweighted)
+  int wbf16;
+  int shared_T;
 };
 nvfp4moe_status launch_stream_gemv_a16(int epi, const StreamA16Args& a, int64_t max_active, cudaStream_t s);
 
@@ -63,9 +67,11 @@ int gemv_lanes_per_row(int64_t K);
 int gemv_down_ksplit(int64_t max_active, int64_t H, int64_t I);
 nvfp4moe_status launch_gemv_gateup(const GemvGateUpArgs& a, int64_t max_active, cudaStream_t s);
 nvfp4moe_status launch_gemv_down(const GemvDownArgs& a, int64_t max_active, cudaStream_t s);
+// shared (nullable, here and in the two combines below): the shared expert's fp32 rows [T][H],
+// added to each output before its bf16 rounding
 nvfp4moe_status launch_combine(const float* slots, int64_t slot_stride, int ksplit,
                                const int32_t* pair_to_row, int T, int H, int k, void* out,
-                               cudaStream_t s);
+                               cudaStream_t s, const float* shared = nullptr);
 // codes_out[r] = codes_tok[row_token[r]] (and the scales, MMA layout) for the rows below
 // *rows_used (device) whose token is in [0, T)
 nvfp4moe_status launch_replicate_rows(const uint8_t* codes_tok, const uint8_t* sf_tok, const int32_t* row_token,
@@ -96,8 +102,9 @@ nvfp4moe_status launch_batch_prologue(const void* x, const float* logits, int T,
 // out[t] = bf16(sum_j topk_w[t*k+j] * slots[pair_to_row[t*k+j]]) in slot order, over fp32 slot
 // rows in padded expert order (a programmatic dependent of the down GEMM)
 nvfp4moe_status launch_combine_rows(const float* slots, const int32_t* pair_to_row, const float* topk_w, int T, int H,
-                                    int k, void* out, cudaStream_t s);
+                                    int k, void* out, cudaStream_t s, const float* shared = nullptr);
 // out[i] = bf16(acc[i]) for the accumulating combine (a programmatic dependent of the down GEMM)
-nvfp4moe_status launch_accum_to_bf16(const float* acc, int64_t n, void* out, cudaStream_t s);
+nvfp4moe_status launch_accum_to_bf16(const float* acc, int64_t n, void* out, cudaStream_t s,
+                                     const float* shared = nullptr);
 
 }  // namespace nvfp4moe

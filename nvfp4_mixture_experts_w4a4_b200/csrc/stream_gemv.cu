@@ -35,6 +35,7 @@ constexpr int kThreadsS = (kConsumers + 1) * 32;    // + the producer warp
 constexpr int kRows = 128;                          // weight rows per item
 constexpr int kNT = 2;                              // tokens per group
 constexpr uint32_t kStatusTimeout = 1u << 3;
+constexpr int kSharedTok = kNT;                     // shared expert: tokens per work item (one group)
 
 struct StreamParams {
   int K;            // reduction size (H for gate/up, I for down)
@@ -52,8 +53,9 @@ struct StreamParams {
   const float* w_scale;      // gate/up: [E][2]; down: [E]
   const float* topk_w;       // [P] by pair
   uint16_t* h_out;           // gate/up: bf16 [P][I]
-  float* slots;              // down: fp32 [P][H]
+  float* slots;              // down: fp32 [P][H] (shared expert: [T][H] by token, unweighted)
   uint32_t* status;
+  int shared_T;              // > 0: the shared expert (one expert, tokens 0..T-1 in order, bf16 weights)
 };
 
 __device__ __forceinline__ void bar_consumers() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumers * 32) : "memory"); }
@@ -73,7 +75,7 @@ struct GroupCtx {
 // The products of one token group with this warp's 16 rows over all K stages (NT tokens,
 // a compile-time count so that no work or register is spent on absent tokens); the row
 // results land in sres[row][t].  `it` counts stages consumed, `ok` turns false on a timeout.
-template <int NT>
+template <int NT, bool WB>
 __device__ __forceinline__ void group_products(const GroupCtx& c, uint32_t& it, bool& ok) {
   const int rsel = c.lane >> 4, cl = c.lane & 15;
   const bool chunk_on = cl * 16 < c.KSB;
@@ -90,7 +92,32 @@ __device__ __forceinline__ void group_products(const GroupCtx& c, uint32_t& it, 
       atomicOr(c.status, kStatusTimeout);
       ok = false;
     }
-    if (ok && chunk_on) {
+    if (WB && ok && chunk_on) {
+      // bf16 weights: a 16-byte chunk is 8 weights, against this lane's 8 activations per token
+      uint4 xv[NT];
+      const int e0 = ks * (c.KSB / 2) + cl * 8;
+#pragma unroll
+      for (int t = 0; t < NT; ++t) xv[t] = *reinterpret_cast<const uint4*>(c.xs + t * c.K + e0);
+      const uint8_t* a = c.sA + s * c.a_bytes;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int row = 16 * c.warp + 2 * q + rsel;
+        const uint4 wv = *reinterpret_cast<const uint4*>(a + row * c.KSB + cl * 16);
+        const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          const uint32_t xw[4] = {xv[t].x, xv[t].y, xv[t].z, xv[t].w};
+          float b = acc[q][t];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            b = __fmaf_rn(bf16_lo(ww[i]), bf16_lo(xw[i]), b);
+            b = __fmaf_rn(bf16_hi(ww[i]), bf16_hi(xw[i]), b);
+          }
+          acc[q][t] = b;
+        }
+      }
+    }
+    if (!WB && ok && chunk_on) {
       // this lane's 32 activation values of each token (shared by its 8 rows)
       uint32_t xw[NT][16];
       const int e0 = ks * 2 * c.KSB + cl * 32;
@@ -156,12 +183,13 @@ __device__ __forceinline__ void group_products(const GroupCtx& c, uint32_t& it, 
     }
 }
 
-template <int EPI>
+// WB: bf16 weights (the shared expert), no block scales; otherwise NVFP4 codes + E4M3 scales.
+template <int EPI, bool WB>
 __global__ void __launch_bounds__(kThreadsS, 1) stream_gemv_kernel(const __grid_constant__ CUtensorMap tmW, StreamParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = p.stages, KSB = p.KSB, K = p.K;
-  const int a_bytes = kRows * KSB, sf_bytes = 16 * KSB;  // KSB / 32 scale atoms of 512 bytes
+  const int a_bytes = kRows * KSB, sf_bytes = WB ? 0 : 16 * KSB;  // KSB / 32 scale atoms of 512 bytes
   uint8_t* sA = smem;
   uint8_t* sSF = sA + S * a_bytes;
   uint16_t* xs = reinterpret_cast<uint16_t*>(sSF + S * sf_bytes);  // [kNT][K] bf16
@@ -183,8 +211,11 @@ __global__ void __launch_bounds__(kThreadsS, 1) stream_gemv_kernel(const __grid_
   __syncthreads();
   griddep_wait();  // the routing step's counts and, for down, the gate/up output
 
-  const int n_items = p.active[0] * p.n_mt;
-  const int kst = (K / 2) / KSB;  // stages per pass over K
+  // the shared expert's items are (weight tile, one token group): every SM takes part, and no item
+  // streams its weight tile twice
+  const bool shared = p.shared_T > 0;
+  const int n_items = (shared ? (p.shared_T + kSharedTok - 1) / kSharedTok : p.active[0]) * p.n_mt;
+  const int kst = (WB ? 2 * K : K / 2) / KSB;  // stages per pass over K
   auto abort_now = [&]() {
     *abort_flag = 1;
     atomicOr(p.status, kStatusTimeout);
@@ -195,10 +226,11 @@ __global__ void __launch_bounds__(kThreadsS, 1) stream_gemv_kernel(const __grid_
     if (elect_one()) {
       uint32_t it = 0;
       for (int item = blockIdx.x; item < n_items && !*abort_flag; item += gridDim.x) {
-        const int e = p.active[1 + item / p.n_mt], mt = item % p.n_mt;
-        const int n_e = p.offsets[e + 1] - p.offsets[e];
+        const int e = shared ? 0 : p.active[1 + item / p.n_mt], mt = item % p.n_mt;
+        const int t0 = (item / p.n_mt) * kSharedTok;
+        const int n_e = shared ? min(kSharedTok, p.shared_T - t0) : p.offsets[e + 1] - p.offsets[e];
         const int64_t row0 = int64_t(e) * p.NW + int64_t(mt) * kRows;
-        const uint8_t* sf = p.w_sf + row0 * (K / 16);
+        const uint8_t* sf = WB ? nullptr : p.w_sf + row0 * (K / 16);
         for (int g = 0; g < n_e && !*abort_flag; g += kNT)
           for (int ks = 0; ks < kst; ++ks, ++it) {
             const int s = it % S;
@@ -208,7 +240,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) stream_gemv_kernel(const __grid_
             }
             mbar_arrive_expect_tx(&full[s], a_bytes + sf_bytes);
             tma_load_2d(sA + s * a_bytes, &tmW, ks * KSB, static_cast<int32_t>(row0), &full[s]);
-            bulk_load(sSF + s * sf_bytes, sf + int64_t(ks) * sf_bytes, sf_bytes, &full[s]);
+            if (!WB) bulk_load(sSF + s * sf_bytes, sf + int64_t(ks) * sf_bytes, sf_bytes, &full[s]);
           }
       }
       if (*abort_flag)  // let the copies in flight land before the CTA exits
@@ -226,8 +258,9 @@ __global__ void __launch_bounds__(kThreadsS, 1) stream_gemv_kernel(const __grid_
   uint32_t it = 0;
   bool ok = true;  // false once a wait timed out (here or in another warp): no more waits
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-    const int e = p.active[1 + item / p.n_mt], mt = item % p.n_mt;
-    const int r0 = p.offsets[e], n_e = p.offsets[e + 1] - r0;
+    const int e = shared ? 0 : p.active[1 + item / p.n_mt], mt = item % p.n_mt;
+    const int r0 = shared ? (item / p.n_mt) * kSharedTok : p.offsets[e];
+    const int n_e = shared ? min(kSharedTok, p.shared_T - r0) : p.offsets[e + 1] - r0;
     for (int g = 0; g < n_e; g += kNT) {
       const int nt = min(kNT, n_e - g);
       // stage the group's activation rows (zeros past nt)
@@ -236,23 +269,23 @@ __global__ void __launch_bounds__(kThreadsS, 1) stream_gemv_kernel(const __grid_
         const int t = v / vec_per_row, c = v - t * vec_per_row;
         uint4 val = make_uint4(0u, 0u, 0u, 0u);
         if (t < nt) {
-          const int64_t src_row = EPI == 0 ? int64_t(p.row_token[r0 + g + t]) : int64_t(r0 + g + t);
+          const int64_t src_row = EPI == 0 && !shared ? int64_t(p.row_token[r0 + g + t]) : int64_t(r0 + g + t);
           val = __ldg(reinterpret_cast<const uint4*>(p.act + src_row * K) + c);
         }
         reinterpret_cast<uint4*>(xs + t * K)[c] = val;
       }
       bar_consumers();
       if (nt == 1)
-        group_products<1>(g_args, it, ok);
+        group_products<1, WB>(g_args, it, ok);
       else
-        group_products<2>(g_args, it, ok);
+        group_products<2, WB>(g_args, it, ok);
       bar_consumers();
       const int l = lane & 15, tt = lane >> 4;
       if (!ok) continue;  // (the next group's barriers are still passed by every warp)
       if (EPI == 0) {
         // warps 0..3: one 16-wide block of h each (gate rows 32w.., up rows 32w+16..)
         if (warp < 4) {
-          const float sg = p.w_scale[2 * e], su = p.w_scale[2 * e + 1];
+          const float sg = WB ? 1.0f : p.w_scale[2 * e], su = WB ? 1.0f : p.w_scale[2 * e + 1];
           const int col = (mt * 4 + warp) * 16 + l;
           for (int t = tt; t < nt; t += 2) {
             const float gv = sres[(32 * warp + l) * kNT + t] * sg;
@@ -264,9 +297,13 @@ __global__ void __launch_bounds__(kThreadsS, 1) stream_gemv_kernel(const __grid_
         }
       } else {
         // each warp writes its 16 output features of every token to the token's slot row
-        const float sw = p.w_scale[e];
+        const float sw = WB ? 1.0f : p.w_scale[e];
         const int n = mt * kRows + 16 * warp + l;
         for (int t = tt; t < nt; t += 2) {
+          if (shared) {  // the shared expert's row of token g + t, unweighted
+            p.slots[int64_t(r0 + g + t) * p.H + n] = sres[(16 * warp + l) * kNT + t];
+            continue;
+          }
           const int32_t pair = p.row_pair[r0 + g + t];
           p.slots[int64_t(pair) * p.H + n] = sres[(16 * warp + l) * kNT + t] * sw * p.topk_w[pair];
         }
@@ -280,13 +317,14 @@ __global__ void __launch_bounds__(kThreadsS, 1) stream_gemv_kernel(const __grid_
 nvfp4moe_status launch_stream_gemv_a16(int epi, const StreamA16Args& a, int64_t max_active, cudaStream_t s) {
   uint32_t* status = device_status_ptr();
   if (!status) return fail(NVFP4MOE_CUDA_ERROR, "device status word unavailable");
+  const bool wb = a.wbf16 != 0;
   StreamParams p{};
   p.K = epi == 0 ? a.H : a.I;
   p.NW = epi == 0 ? 2 * a.I : a.H;
-  const int half = p.K / 2;
-  p.KSB = half % 256 == 0 ? 256 : half % 128 == 0 ? 128 : half % 64 == 0 ? 64 : 32;
-  if (half % p.KSB != 0 || p.NW % kRows != 0)
-    return fail(NVFP4MOE_UNSUPPORTED_SHAPE, "weight-only stream GEMV: K=%d, rows=%d", p.K, p.NW);
+  const int row_bytes = wb ? 2 * p.K : p.K / 2;  // weight bytes per row
+  p.KSB = row_bytes % 256 == 0 ? 256 : row_bytes % 128 == 0 ? 128 : row_bytes % 64 == 0 ? 64 : 32;
+  if (row_bytes % p.KSB != 0 || p.NW % kRows != 0)
+    return fail(NVFP4MOE_UNSUPPORTED_SHAPE, "stream GEMV: K=%d, rows=%d", p.K, p.NW);
   p.n_mt = p.NW / kRows;
   p.H = a.H;
   p.I = a.I;
@@ -301,22 +339,23 @@ nvfp4moe_status launch_stream_gemv_a16(int epi, const StreamA16Args& a, int64_t 
   p.h_out = a.h_out;
   p.slots = a.slots;
   p.status = status;
-  const int stage_bytes = kRows * p.KSB + 16 * p.KSB;
+  p.shared_T = a.shared_T;
+  const int stage_bytes = kRows * p.KSB + (wb ? 0 : 16 * p.KSB);
   const int fixed = 1024 + kNT * p.K * 2 + kRows * kNT * 4 + 64;
   const int budget = 227 * 1024;
   int stages = (budget - fixed - 16 * 8) / stage_bytes;
   if (stages > 6) stages = 6;
-  if (stages < 2) return fail(NVFP4MOE_UNSUPPORTED_SHAPE, "weight-only stream GEMV: K=%d leaves no room", p.K);
+  if (stages < 2) return fail(NVFP4MOE_UNSUPPORTED_SHAPE, "stream GEMV: K=%d leaves no room", p.K);
   p.stages = stages;
   const size_t smem = size_t(fixed) + size_t(stages) * (stage_bytes + 16);
 
-  // weight codes as [E*NW][K/2] bytes, box KSB bytes x 128 rows, no swizzle
+  // weights as [E*NW][row_bytes] bytes, box KSB bytes x 128 rows, no swizzle
   auto fn = tensor_map_encoder();
   if (!fn) return fail(NVFP4MOE_CUDA_ERROR, "cuTensorMapEncodeTiled is unavailable");
   CUtensorMap map;
   const int64_t rows = int64_t(a.E) * p.NW;
-  const cuuint64_t dims[2] = {cuuint64_t(half), cuuint64_t(rows)};
-  const cuuint64_t strides[1] = {cuuint64_t(half)};
+  const cuuint64_t dims[2] = {cuuint64_t(row_bytes), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(row_bytes)};
   const cuuint32_t box[2] = {cuuint32_t(p.KSB), cuuint32_t(kRows)};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = fn(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.w_codes), dims, strides, box,
@@ -324,20 +363,18 @@ nvfp4moe_status launch_stream_gemv_a16(int epi, const StreamA16Args& a, int64_t 
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(NVFP4MOE_CUDA_ERROR, "cuTensorMapEncodeTiled (stream GEMV) failed (%d)", int(r));
 
-  const int64_t items = max_active * p.n_mt;
+  const int64_t items =
+      (a.shared_T > 0 ? (int64_t(a.shared_T) + kSharedTok - 1) / kSharedTok : max_active) * p.n_mt;
   const int grid = static_cast<int>(items < num_sms() ? (items > 0 ? items : 1) : num_sms());
-  cudaError_t e;
-  if (epi == 0) {
-    e = cudaFuncSetAttribute(stream_gemv_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e == cudaSuccess)
-      e = launch_dependent(stream_gemv_kernel<0>, dim3(grid), dim3(kThreadsS), smem, s, map, p);
-  } else {
-    e = cudaFuncSetAttribute(stream_gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e == cudaSuccess)
-      e = launch_dependent(stream_gemv_kernel<1>, dim3(grid), dim3(kThreadsS), smem, s, map, p);
-  }
-  if (e != cudaSuccess) return fail(NVFP4MOE_CUDA_ERROR, "weight-only stream GEMV: %s", cudaGetErrorString(e));
-  return check_launch("weight-only stream GEMV");
+  auto go = [&](auto kern) -> cudaError_t {
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (err == cudaSuccess) err = launch_dependent(kern, dim3(grid), dim3(kThreadsS), smem, s, map, p);
+    return err;
+  };
+  const cudaError_t e = epi == 0 ? (wb ? go(stream_gemv_kernel<0, true>) : go(stream_gemv_kernel<0, false>))
+                                 : (wb ? go(stream_gemv_kernel<1, true>) : go(stream_gemv_kernel<1, false>));
+  if (e != cudaSuccess) return fail(NVFP4MOE_CUDA_ERROR, "stream GEMV: %s", cudaGetErrorString(e));
+  return check_launch("stream GEMV");
 }
 
 }  // namespace nvfp4moe

@@ -182,6 +182,18 @@ def nvfp4_from_mxfp4(codes: torch.Tensor, e8m0: torch.Tensor, row_gather: torch.
     return out_codes, sf_out, scale
 
 
+def shared_expert_w13(gate: torch.Tensor, up: torch.Tensor) -> torch.Tensor:
+    """bf16 gate and up [I_s, H] of a shared expert -> the interleaved [2 I_s, H] the layer takes
+    (rows 32c+j: gate row 16c+j for j < 16, up row 16c+j-16 otherwise); a setup-time layout step."""
+    I = gate.shape[0]
+    g_map, u_map = NVFP4Experts.interleave_maps(I, gate.device)
+    out = torch.empty(2 * I, gate.shape[1], dtype=gate.dtype, device=gate.device)
+    gm, um = g_map >= 0, u_map >= 0
+    out[gm] = gate[g_map[gm].long()]
+    out[um] = up[u_map[um].long()]
+    return out
+
+
 class NVFP4Experts:
     """Per-expert NVFP4 weights in the library's layout (W13 interleaved, MMA scales)."""
 
@@ -235,10 +247,12 @@ class MoeFFN:
 
     def __init__(self, experts: NVFP4Experts, top_k: int, h_scale: torch.Tensor | None,
                  x_scale: torch.Tensor | None = None, path: int = C.PATH_AUTO, combine: int = C.COMBINE_AUTO,
-                 act: int = C.ACT_NVFP4):
+                 act: int = C.ACT_NVFP4, shared: tuple | None = None):
         """h_scale: per-expert requantisation scales of h, or None for the dynamic scale
         (amax of each expert's h in the call / 2688; tensor-core path).  act: ACT_NVFP4 (W4A4)
-        or ACT_BF16 (weight-only W4A16: bf16 activations, the GEMV path; no scales used)."""
+        or ACT_BF16 (weight-only W4A16: bf16 activations, the GEMV path; no scales used).
+        shared: None or a BF16 shared expert (w13 bf16 [2I_s, H] interleaved, see
+        shared_expert_w13; w2 bf16 [H, I_s]), added to every token's output."""
         self.w = experts
         self.top_k = top_k
         self.h_scale = None if h_scale is None else h_scale.to(torch.float32).contiguous()
@@ -246,6 +260,7 @@ class MoeFFN:
         self.path = path
         self.combine = combine
         self.act = act
+        self.shared = None if shared is None else tuple(t.contiguous() for t in shared)
         self._ws = {}
 
     def desc(self, T: int, h_amax: torch.Tensor | None = None, events=None) -> C.MoeFfnDesc:
@@ -262,6 +277,9 @@ class MoeFFN:
         d.h_scale_mode = C.SCALE_DYNAMIC if self.h_scale is None else C.SCALE_GIVEN
         d.h_amax = None if h_amax is None else h_amax.data_ptr()
         d.act_mode = self.act
+        if self.shared is not None:
+            d.shared_I = self.shared[1].shape[1]
+            d.shared_w13, d.shared_w2 = self.shared[0].data_ptr(), self.shared[1].data_ptr()
         d.stage_events = None if events is None else ctypes.cast(events, ctypes.c_void_p).value
         return d
 

@@ -294,3 +294,37 @@ def run_layer_pair_mxfp4(wl: W.Workload, path: int, act_mode: int = C.ACT_NVFP4,
     torch.cuda.synchronize()
     layer.oracle_wd = wd
     return ref, out, layer, h_amax
+
+
+def shared_weights(wl: W.Workload, I_s: int, seed: int = 5):
+    """A BF16 shared expert for a workload: gate/up [I_s, H] and down [H, I_s], N(0, 1/sqrt(fan_in))
+    rounded to bf16; returned as bf16 bit patterns (oracle) and device tensors (library)."""
+    g = torch.Generator().manual_seed(seed)
+    gate = (torch.randn(I_s, wl.H, generator=g) / wl.H ** 0.5).to(torch.bfloat16)
+    up = (torch.randn(I_s, wl.H, generator=g) / wl.H ** 0.5).to(torch.bfloat16)
+    down = (torch.randn(wl.H, I_s, generator=g) / I_s ** 0.5).to(torch.bfloat16)
+    bits = tuple(t.view(torch.int16).numpy().view(np.uint16) for t in (gate, up, down))
+    return gate, up, down, bits
+
+
+def run_layer_pair_shared(wl: W.Workload, path: int, I_s: int, act_mode: int = C.ACT_NVFP4,
+                          combine: int = C.COMBINE_AUTO, seed: int = 0, dev=None):
+    dev = dev or need_gpu()
+    act, wts, wg, wu, wd = layer_inputs(wl, seed)
+    gate, up, down, bits = shared_weights(wl, I_s)
+    x_bits = bf16_bits(act["x"])
+    logits = act["logits"].numpy()
+    experts = experts_from_oracle(wg, wu, wd, dev)
+    shared = (ops.shared_expert_w13(gate.to(dev), up.to(dev)), down.to(dev))
+    if act_mode == C.ACT_BF16:
+        ref = O.moe_ffn_w4a16(x_bits, logits, wl.k, wg, wu, wd, shared=bits)
+        layer = ops.MoeFFN(experts, wl.k, None, act=C.ACT_BF16, shared=shared)
+    else:
+        ref = O.moe_ffn(x_bits, logits, wl.k, wg, wu, wd, shared=bits)
+        layer = ops.MoeFFN(experts, wl.k, torch.from_numpy(ref["h_scale"]).to(dev), path=path, combine=combine,
+                           shared=shared)
+    h_amax = torch.empty(wl.E, dtype=torch.float32, device=dev)
+    out = layer(act["x"].to(dev), act["logits"].to(dev), h_amax=None if act_mode == C.ACT_BF16 else h_amax)
+    torch.cuda.synchronize()
+    layer.oracle_wd = wd
+    return ref, out, layer, h_amax

@@ -231,3 +231,25 @@ def test_layer_empty_batch(path, act):
     torch.cuda.synchronize()
     assert out.shape == (0, wl.H)
     assert ops.device_status() == 0
+
+
+@pytest.mark.parametrize("name,path,act,combine", [
+    ("tiny", C.PATH_GEMM, C.ACT_NVFP4, C.COMBINE_AUTO),
+    ("decode_shape", C.PATH_GEMM, C.ACT_NVFP4, C.COMBINE_AUTO),
+    ("long_prefill_small", C.PATH_GEMM, C.ACT_NVFP4, C.COMBINE_ORDERED),
+    ("long_prefill_small", C.PATH_GEMM, C.ACT_NVFP4, C.COMBINE_ACCUMULATE),
+    ("dense_small", C.PATH_GEMM, C.ACT_NVFP4, C.COMBINE_AUTO),
+    ("tiny", C.PATH_GEMV, C.ACT_NVFP4, C.COMBINE_AUTO),
+    ("decode_shape", C.PATH_AUTO, C.ACT_BF16, C.COMBINE_AUTO),
+])
+def test_layer_with_shared_expert(name, path, act, combine):
+    """A BF16 shared expert beside the routed experts, added before the output's one rounding,
+    on every path and combine mode, against the oracle (reading R12)."""
+    wl = GEMM_CASES[name]
+    ref, out, layer, h_amax = G.run_layer_pair_shared(wl, path, I_s=128 if wl.H <= 512 else 256, act_mode=act,
+                                                      combine=combine)
+    if act == C.ACT_BF16:
+        G.check_layer_w4a16(wl, ref, out, layer)
+    else:
+        G.check_layer(wl, ref, out, layer, h_amax)
+    assert ops.device_status() == 0
