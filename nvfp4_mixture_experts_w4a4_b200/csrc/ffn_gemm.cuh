@@ -60,7 +60,8 @@ nvfp4moe_status launch_requant_h(const float* h_f32, int64_t rows_cap, int I, in
 
 bool gemm_path_available();
 int grouped_token_align();
-// gate/up (SwiGLU + requant) then down (weighted bf16 slots), weight-stationary grouped GEMM
+// gate/up (SwiGLU + requant) then down (fp32 slot rows or accumulator), weight-stationary
+// grouped GEMM
 nvfp4moe_status launch_grouped_ffn(const GemmFfnArgs& a, cudaStream_t s);
 // D[M][N] = A . B^T * a_scale[0] * b_scale[0]; N % 128 == 0, K % 128 == 0.
 nvfp4moe_status launch_gemm_plain(const uint8_t* A, const uint8_t* A_sf, const float* a_scale, const uint8_t* B,

@@ -211,31 +211,6 @@ __global__ void combine_kernel(const float* __restrict__ slots, int64_t slot_str
 }
 
 
-// Copies quantised token rows into the padded expert-order rows: codes (32 bytes) and the
-// 4-byte scale word of one 64-element group per thread; padding rows are left untouched.
-// Only rows below *rows_used (the permutation's padded total) carry a row -> token entry;
-// the token index is checked against T as well.
-__global__ void replicate_rows_kernel(const uint8_t* __restrict__ codes_tok, const uint8_t* __restrict__ sf_tok,
-                                      const int32_t* __restrict__ row_token, const int32_t* __restrict__ rows_used,
-                                      int64_t rows_cap, int64_t T, int64_t K, uint8_t* __restrict__ codes_out,
-                                      uint8_t* __restrict__ sf_out) {
-  const int64_t groups = K / 64;
-  const int64_t rows = min(rows_cap, int64_t(*rows_used));
-  const int64_t total = rows * groups;
-  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total;
-       i += int64_t(gridDim.x) * blockDim.x) {
-    const int64_t r = i / groups, g = i - r * groups;
-    const int32_t t = row_token[r];
-    if (t < 0 || t >= T) continue;
-    const uint4* src = reinterpret_cast<const uint4*>(codes_tok + int64_t(t) * (K / 2) + g * 32);
-    uint4* dst = reinterpret_cast<uint4*>(codes_out + r * (K / 2) + g * 32);
-    dst[0] = src[0];
-    dst[1] = src[1];
-    *reinterpret_cast<uint32_t*>(sf_out + sf_mma_offset(r, 4 * g, K)) =
-        *reinterpret_cast<const uint32_t*>(sf_tok + sf_mma_offset(t, 4 * g, K));
-  }
-}
-
 template <typename K>
 int grid_for(K kernel, int64_t warp_items) {
   static int occ_cache[64] = {0};
@@ -394,18 +369,5 @@ nvfp4moe_status launch_accum_to_bf16(const float* acc, int64_t n, void* out, cud
   if (e != cudaSuccess) return fail(NVFP4MOE_CUDA_ERROR, "accumulator to bf16: %s", cudaGetErrorString(e));
   return check_launch("accumulator to bf16");
 }
-
-nvfp4moe_status launch_replicate_rows(const uint8_t* codes_tok, const uint8_t* sf_tok, const int32_t* row_token,
-                                      const int32_t* rows_used, int64_t rows_cap, int64_t T, int64_t K,
-                                      uint8_t* codes_out, uint8_t* sf_out, cudaStream_t s) {
-  const int64_t total = rows_cap * (K / 64);
-  if (total == 0) return NVFP4MOE_OK;
-  int64_t blocks = (total + 255) / 256;
-  if (blocks > int64_t(num_sms()) * 16) blocks = int64_t(num_sms()) * 16;
-  replicate_rows_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(codes_tok, sf_tok, row_token, rows_used, rows_cap, T,
-                                                                 K, codes_out, sf_out);
-  return check_launch("replicate rows");
-}
-
 
 }  // namespace nvfp4moe

@@ -72,11 +72,6 @@ nvfp4moe_status launch_gemv_down(const GemvDownArgs& a, int64_t max_active, cuda
 nvfp4moe_status launch_combine(const float* slots, int64_t slot_stride, int ksplit,
                                const int32_t* pair_to_row, int T, int H, int k, void* out,
                                cudaStream_t s, const float* shared = nullptr);
-// codes_out[r] = codes_tok[row_token[r]] (and the scales, MMA layout) for the rows below
-// *rows_used (device) whose token is in [0, T)
-nvfp4moe_status launch_replicate_rows(const uint8_t* codes_tok, const uint8_t* sf_tok, const int32_t* row_token,
-                                      const int32_t* rows_used, int64_t rows_cap, int64_t T, int64_t K,
-                                      uint8_t* codes_out, uint8_t* sf_out, cudaStream_t s);
 
 // Small-batch prologue (route + permute + quantise x) in one launch of an 8-CTA cluster;
 // see prologue.cu.

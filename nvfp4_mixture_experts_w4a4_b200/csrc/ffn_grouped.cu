@@ -1,23 +1,33 @@
-// Weight-stationary grouped GEMM of the routed layer on tcgen05 block-scaled MMA.
+// Weight-stationary grouped GEMM of the routed layer on tcgen05 block-scaled MMA
+// (kind::mxf4nvf4, E4M3 scales per 16 elements, fp32 accumulators in TMEM).
 //
 // The expert weights are the MMA's M operand (128 weight rows per tile) and an expert's
-// tokens are its N operand: N = the expert's token count rounded up to 64 (tokens are
-// grouped in 64-row blocks by the permutation), at most 192 per tile.  So a weight tile is
-// streamed once per 192 tokens of its expert whatever the skew, and no MMA work or load is
-// spent on 128-row padding of experts that received a handful of tokens.  This one kernel
-// serves decode (N = 64 for 1..64 tokens) and prefill.
+// tokens are its N operand: N = the expert's token count in the tile's chunk rounded up to 16,
+// at most BNMAX (64 for batches of at most 64 tokens, 192 above).  A weight tile is streamed
+// once per chunk of its expert's tokens whatever the routing skew, and no MMA work or load
+// is spent on 128-row padding of experts that received a handful of tokens.  One kernel
+// serves decode and prefill, gate/up (EPI_GATEUP), down (EPI_DOWN) or both in one launch
+// (EPI_FUSED).
 //
 // Persistent CTA per SM; work items ordered (expert, weight tile, token chunk) with the
 // chunk fastest, so CTAs of one wave that share a weight tile run together (L2 hits).
-//   warp 0      TMA producer: weights (128 rows x 128 B, 128-byte swizzle), tokens (64-row
-//               boxes), and bulk copies of the 512-byte scale atoms, 4-stage ring;
+//   warp 0      weight producer: TMA loads of 128 rows x 128 B (128-byte swizzle) and bulk
+//               copies of their 512-byte scale atoms into a ring of STAGES stages; it arms
+//               each stage with the bytes of both operands;
+//   warp 10     token producer: TMA loads of the tokens' rows (64- and 16-row boxes) and
+//               their scale atoms into the same stages (for a fused down item, once its
+//               expert's gate/up tiles are counted done);
 //   warp 1      TMEM owner and MMA issuer: tcgen05.cp of the scales, four K=64 MMAs per
-//               stage into one of two fp32 accumulators (double buffered, 192 columns);
-//   warps 2..5  epilogue, one 32-row slice of weight rows each: SwiGLU + requantise (gate/up,
-//               gate row i and up row i are lanes i and 16+i of the same warp by the W13
-//               interleave) or the weighted bf16 slot rows (down).
+//               stage into one of NACC fp32 accumulators;
+//   warps 2..9  epilogue, two warps per 32-row TMEM lane quarter (alternate token chunks):
+//               SwiGLU + requantise to NVFP4 (gate/up; gate row i and up row i are lanes i
+//               and 16+i of the same warp by the W13 interleave), or the down rows scaled by
+//               s_h * s_w2 into fp32 slot rows (by pair, weighted; or, above 64 tokens, by
+//               padded row through staging tiles and TMA tile stores) or added into the
+//               fp32 accumulator (bulk reductions).
 // Scale atoms of the tokens start at a 64-row boundary inside a 128-row atom, so the MMA
-// reads them at a TMEM column offset of 0 or 2.  Waits are bounded (status bit on timeout).
+// reads them at a TMEM column offset of 0 or 2.  Every wait is bounded (status bit on
+// timeout; copies in flight land before the CTA exits).
 #include "ffn_gemm.cuh"
 #include "tcgen05.cuh"
 #include "tma.cuh"
