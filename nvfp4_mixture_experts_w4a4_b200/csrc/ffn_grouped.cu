@@ -262,32 +262,40 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__
   int4* s_items = reinterpret_cast<int4*>((reinterpret_cast<uintptr_t>(prefix) + 15) & ~uintptr_t(15));
   int total = 0, n_my = 0;
   bool sched = true;
+  // Items are dealt round-robin over the fewest CTAs that keep the largest share (ceil(total /
+  // grid) items): then every working CTA has the same count but for the last round, no CTA
+  // carries one item more than most others, and the CTAs left over exit at once (their SMs
+  // go to the next launch).
+  int geff = int(gridDim.x);
+  auto balance = [&](int tot) {
+    if (tot > 0) {
+      const int per = (tot + int(gridDim.x) - 1) / int(gridDim.x);
+      geff = (tot + per - 1) / per;
+    }
+  };
   if (p.list != nullptr) {
     // The routing step wrote the work list (entry 0: {gate/up items, down items}, then the
     // gate/up items, then the down items).  Gate/up and fused launches read their length and
     // this CTA's entries in one round trip; a down launch first learns where its entries start.
     // The host only passes the list when a CTA's share fits SCHED_CAP.  In a fused launch the
     // entries past the gate/up items are down items; the phase goes into bit 30 of the tile.
-    int4 head = make_int4(0, 0, 0, 0);
-    int64_t base = 1;
-    if (EPI == EPI_DOWN) {
-      head = __ldcg(p.list);
-      base = 1 + head.x;
-    }
+    const int4 head = __ldcg(p.list);
+    const int64_t base = EPI == EPI_DOWN ? 1 + head.x : 1;
+    total = EPI == EPI_GATEUP ? head.x : EPI == EPI_DOWN ? head.y : head.x + head.y;
+    balance(total);
     int4 mine[SCHED_PER_THREAD];
 #pragma unroll
     for (int q = 0; q < SCHED_PER_THREAD; ++q) {
       const int j = threadIdx.x + q * kThreads;
-      const int64_t idx = int64_t(blockIdx.x) + int64_t(j) * gridDim.x;
-      mine[q] = (j < SCHED_CAP && idx < p.list_cap) ? __ldcg(p.list + base + idx) : make_int4(0, 0, 0, 0);
+      const int64_t idx = int64_t(blockIdx.x) + int64_t(j) * geff;
+      mine[q] = (j < SCHED_CAP && idx < p.list_cap && idx < total) ? __ldcg(p.list + base + idx)
+                                                                    : make_int4(0, 0, 0, 0);
     }
-    if (EPI != EPI_DOWN) head = __ldcg(p.list);
-    total = EPI == EPI_GATEUP ? head.x : EPI == EPI_DOWN ? head.y : head.x + head.y;
-    n_my = total > int(blockIdx.x) ? (total - int(blockIdx.x) + int(gridDim.x) - 1) / int(gridDim.x) : 0;
+    n_my = int(blockIdx.x) < geff && total > int(blockIdx.x) ? (total - int(blockIdx.x) + geff - 1) / geff : 0;
 #pragma unroll
     for (int q = 0; q < SCHED_PER_THREAD; ++q) {
       const int j = threadIdx.x + q * kThreads;
-      const int idx = int(blockIdx.x) + j * int(gridDim.x);
+      const int idx = int(blockIdx.x) + j * geff;
       if (j < n_my) {
         int4 v = mine[q];
         if (EPI == EPI_FUSED) v.y |= int(idx >= head.x) << 30;
@@ -339,11 +347,12 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__
       if (threadIdx.x == MAX_E / 4 - 1 && E == MAX_E) prefix[E] = run;
     }
     __syncthreads();
-    // This CTA's items are blockIdx.x + j * gridDim.x.  Each thread resolves a few of them now,
-    // in parallel, and the list replaces the per-expert arrays, so that every role then reads
-    // one 16-byte entry per item instead of searching the expert prefix sums.
+    // This CTA's items are blockIdx.x + j * geff.  Each thread resolves a few of them now, in
+    // parallel, and the list replaces the per-expert arrays, so that every role then reads one
+    // 16-byte entry per item instead of searching the expert prefix sums.
     total = prefix[E];
-    n_my = total > int(blockIdx.x) ? (total - int(blockIdx.x) + int(gridDim.x) - 1) / int(gridDim.x) : 0;
+    balance(total);
+    n_my = int(blockIdx.x) < geff && total > int(blockIdx.x) ? (total - int(blockIdx.x) + geff - 1) / geff : 0;
     sched = n_my <= SCHED_CAP;
     if (sched) {
       int4 mine[SCHED_PER_THREAD];
@@ -351,7 +360,7 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__
       for (int q = 0; q < SCHED_PER_THREAD; ++q) {
         const int j = threadIdx.x + q * kThreads;
         if (j < n_my) {
-          const Item w = get_item<C::BNMAX>(int(blockIdx.x) + j * int(gridDim.x), E, prefix, s_ch, s_off, s_cnt);
+          const Item w = get_item<C::BNMAX>(int(blockIdx.x) + j * geff, E, prefix, s_ch, s_off, s_cnt);
           mine[q] = make_int4(w.e, w.mt, w.r0, w.n_rows);
         }
       }
@@ -376,7 +385,7 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__
       w.ph = EPI == EPI_FUSED ? (v.y >> 30) & 1 : PH;
       return w;
     }
-    Item w = get_item<C::BNMAX>(int(blockIdx.x) + j * int(gridDim.x), E, prefix, s_ch, s_off, s_cnt);
+    Item w = get_item<C::BNMAX>(int(blockIdx.x) + j * geff, E, prefix, s_ch, s_off, s_cnt);
     w.ph = PH;
     return w;
   };
