@@ -249,6 +249,7 @@ nvfp4moe_status launch_gemv_gateup(const GemvGateUpArgs& a, int64_t max_active, 
 int gemv_down_ksplit(int64_t max_active, int64_t H, int64_t I) {
   const int L = gemv_lanes_per_row(I);
   const int64_t items = max_active * ((H + 31) / 32);
+  if (items <= 0) return 1;  // an empty batch
   const int64_t want = int64_t(num_sms()) * 16;
   int64_t ks = (want + items - 1) / items;
   const int64_t max_ks = (I / 32) / L;

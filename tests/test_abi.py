@@ -105,3 +105,17 @@ def test_weight_only_workspace_and_mode_checks(so):
     assert so.moe_ffn_workspace_layout(ctypes.byref(d), ctypes.byref(L)) == C.UNSUPPORTED_SHAPE
     d.path, d.act_mode = C.PATH_AUTO, 7
     assert so.moe_ffn_workspace_layout(ctypes.byref(d), ctypes.byref(L)) == C.INVALID_ARG
+
+
+@pytest.mark.parametrize("path", [0, 1, 2])
+@pytest.mark.parametrize("act", [0, 1])
+@pytest.mark.parametrize("shared_I", [0, 128])
+def test_workspace_layout_of_an_empty_batch(so, path, act, shared_I):
+    """T = 0 lays out a workspace (no division by the empty batch) on every path and mode."""
+    from nvfp4_mixture_experts_w4a4_b200 import _lib as C
+    d = C.MoeFfnDesc()
+    d.T, d.H, d.I, d.E, d.top_k = 0, 256, 128, 8, 2
+    d.path, d.act_mode, d.shared_I = path, act, shared_I
+    L = C.MoeFfnWsLayout()
+    st = so.moe_ffn_workspace_layout(ctypes.byref(d), ctypes.byref(L))
+    assert st == (C.UNSUPPORTED_SHAPE if (act == 1 and path == 2) else C.OK)
