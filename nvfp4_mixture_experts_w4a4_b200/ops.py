@@ -356,5 +356,36 @@ class MoeFFN:
         )
 
 
+class GraphedMoeFFN:
+    """The layer for a fixed batch size T, captured once into a CUDA graph over static buffers:
+    a call copies x and logits into the static inputs (device or pinned host tensors), replays
+    the graph (the same kernels as an eager call, without the per-call host work of building
+    the call and launching each kernel) and returns the static output (overwritten by the next
+    call)."""
+
+    def __init__(self, layer: MoeFFN, T: int):
+        dev = layer.w.w13_codes.device
+        self.layer, self.T = layer, T
+        self.x = torch.zeros(T, layer.w.H, dtype=torch.bfloat16, device=dev)
+        self.logits = torch.zeros(T, layer.w.E, dtype=torch.float32, device=dev)
+        self.out = torch.empty(T, layer.w.H, dtype=torch.bfloat16, device=dev)
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            layer(self.x, self.logits, out=self.out)  # workspace and kernel attributes set up
+        torch.cuda.current_stream(dev).wait_stream(side)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            layer(self.x, self.logits, out=self.out)
+
+    def __call__(self, x: torch.Tensor, logits: torch.Tensor) -> torch.Tensor:
+        if x.shape != self.x.shape or logits.shape != self.logits.shape:
+            raise ValueError(f"captured for x {tuple(self.x.shape)}, logits {tuple(self.logits.shape)}")
+        self.x.copy_(x, non_blocking=True)
+        self.logits.copy_(logits, non_blocking=True)
+        self.graph.replay()
+        return self.out
+
+
 def moe_ffn_forward(layer: MoeFFN, x: torch.Tensor, logits: torch.Tensor, **kw) -> torch.Tensor:
     return layer.forward(x, logits, **kw)

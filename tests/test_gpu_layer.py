@@ -253,3 +253,23 @@ def test_layer_with_shared_expert(name, path, act, combine):
     else:
         G.check_layer(wl, ref, out, layer, h_amax)
     assert ops.device_status() == 0
+
+
+@pytest.mark.parametrize("name", ["tiny", "long_prefill_small"])
+def test_graphed_layer_matches_eager(name):
+    """The graph-replayed layer (ops.GraphedMoeFFN) gives the eager call's output bit for bit,
+    from device and from pinned host inputs, call after call."""
+    wl = GEMM_CASES[name]
+    dev = G.need_gpu()
+    act, wts, wg, wu, wd = G.layer_inputs(wl)
+    experts = G.experts_from_oracle(wg, wu, wd, dev)
+    layer = ops.MoeFFN(experts, wl.k, torch.ones(wl.E, device=dev) * 0.01)
+    x, logits = act["x"].to(dev), act["logits"].to(dev)
+    eager = layer(x, logits).clone()
+    graphed = ops.GraphedMoeFFN(layer, wl.T)
+    for src in ((x, logits), (act["x"].pin_memory(), act["logits"].pin_memory())):
+        out = graphed(*src)
+        torch.cuda.synchronize()
+        assert torch.equal(out, eager)
+    with pytest.raises(ValueError):
+        graphed(x[:1], logits[:1])
