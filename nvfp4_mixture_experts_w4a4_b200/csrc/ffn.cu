@@ -42,6 +42,10 @@ nvfp4moe_status check_desc(const moe_ffn_desc* d, const char* fn) {
   return NVFP4MOE_OK;
 }
 
+// The shared expert runs the streamed CUDA-core kernel up to this many tokens (decode) and the
+// tcgen05 bf16 GEMMs above.
+constexpr int kSharedStreamMaxT = 32;
+
 int resolve_path(const moe_ffn_desc* d) {
   if (d->act_mode == NVFP4MOE_ACT_BF16) return NVFP4MOE_PATH_GEMV;
   if (d->path != NVFP4MOE_PATH_AUTO) return d->path;
@@ -225,6 +229,13 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   float* shared_y = d->shared_I > 0 ? F32(L.shared_y) : nullptr;
   auto run_shared = [&]() -> nvfp4moe_status {
     if (!shared_y) return NVFP4MOE_OK;
+    uint16_t* hs = reinterpret_cast<uint16_t*>(ws + L.shared_h);
+    if (T > kSharedStreamMaxT) {  // larger batches: tensor-core GEMMs
+      nvfp4moe_status r = launch_dense_bf16(0, d->shared_w13, static_cast<const uint16_t*>(x), H, 2 * d->shared_I, T,
+                                            hs, nullptr, s);
+      if (r != NVFP4MOE_OK) return r;
+      return launch_dense_bf16(1, d->shared_w2, hs, d->shared_I, H, T, nullptr, shared_y, s);
+    }
     StreamA16Args sa{};
     sa.H = H; sa.I = d->shared_I; sa.E = 1;
     sa.wbf16 = 1; sa.shared_T = T;

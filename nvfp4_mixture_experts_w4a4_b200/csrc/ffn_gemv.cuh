@@ -63,6 +63,12 @@ struct StreamA16Args {
 };
 nvfp4moe_status launch_stream_gemv_a16(int epi, const StreamA16Args& a, int64_t max_active, cudaStream_t s);
 
+// The shared expert's GEMMs on the tensor cores (tcgen05 kind::f16, dense_bf16.cu), for larger
+// batches: epi 0 writes h bf16 [T][NW/2] from the interleaved W13 bf16 [NW][K] and act bf16
+// [T][K]; epi 1 writes fp32 rows [T][NW] from W2 bf16 [NW][K] and h.  K % 64 == 0, NW % 128 == 0.
+nvfp4moe_status launch_dense_bf16(int epi, const uint16_t* weights, const uint16_t* act, int K, int NW, int T,
+                                  uint16_t* h_out, float* y_out, cudaStream_t s);
+
 int gemv_lanes_per_row(int64_t K);
 int gemv_down_ksplit(int64_t max_active, int64_t H, int64_t I);
 nvfp4moe_status launch_gemv_gateup(const GemvGateUpArgs& a, int64_t max_active, cudaStream_t s);
