@@ -30,8 +30,11 @@ pytestmark = pytest.mark.gpu
 SAMPLE = 3  # tokens per workload checked against the oracle
 
 
-@pytest.mark.parametrize("name", ["decode", "prefill_chunk", "long_prefill", "dense", "dense_t1"])
-def test_fullsize_sampled_tokens(name):
+@pytest.mark.parametrize("name,shared_I", [("decode", 0), ("prefill_chunk", 0), ("long_prefill", 0), ("dense", 0),
+                                           ("dense_t1", 0), ("decode", 512), ("prefill_chunk", 512)])
+def test_fullsize_sampled_tokens(name, shared_I):
+    """shared_I > 0: with a BF16 shared expert of that size (the streamed kernel at 16 tokens,
+    the tcgen05 bf16 GEMMs at 512)."""
     wl = W.WORKLOADS[name]
     dev = G.need_gpu()
     T, H, I, E, k = wl.T, wl.H, wl.I, wl.E, wl.k
@@ -63,13 +66,17 @@ def test_fullsize_sampled_tokens(name):
         assert np.array_equal(g[tt].cpu().numpy(), r)
 
     # oracle on the sample, restricted to the touched experts; it calibrates s_h on the sample
-    ref = O.moe_ffn(x_bits[sample], logits[sample][:, touched], k, wg, wu, wd, x_scale=s_x)
+    shared, shared_bits = None, None
+    if shared_I:
+        gate, up, down, shared_bits = G.shared_weights(wl, shared_I)
+        shared = (ops.shared_expert_w13(gate.to(dev), up.to(dev)), down.to(dev))
+    ref = O.moe_ffn(x_bits[sample], logits[sample][:, touched], k, wg, wu, wd, x_scale=s_x, shared=shared_bits)
     assert np.array_equal(touched[ref["ids"]], ids_all[sample])
     s_h = np.ones(E, np.float32)
     s_h[touched] = ref["h_scale"]
 
     # the device: the whole batch, dynamic x scale, automatic path (as the benchmark runs it)
-    layer = ops.MoeFFN(experts, k, torch.from_numpy(s_h).to(dev))
+    layer = ops.MoeFFN(experts, k, torch.from_numpy(s_h).to(dev), shared=shared)
     out = layer(act["x"], act["logits"])
     torch.cuda.synchronize()
     im = layer.intermediates(T)
