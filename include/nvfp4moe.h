@@ -179,7 +179,8 @@ nvfp4moe_status nvfp4_quantize_dynamic_noalloc(const void* x, int32_t x_dtype, i
  *
  * codes [batch][rows][K/2], e8m0 [batch][rows][K/32] (device).  Out row r of each matrix
  * takes input row row_gather[r] (nullable: r; -1: the row is left untouched, for building
- * the interleaved W13 from gate and up in two calls), out_rows rows.  Writes
+ * the interleaved W13 from gate and up in two calls; an entry >= rows is NVFP4MOE_INVALID_ARG),
+ * out_rows rows.  Writes
  * sf_out [batch][sf_mma_bytes(out_rows, K)] (MMA layout), tensor_scale [batch], and, when
  * codes_out is non-null, the codes [batch][out_rows][K/2].  K % 64 == 0; codes 16-byte
  * aligned.  Workspace: nvfp4_from_mxfp4_workspace_size(batch) bytes.  Synchronous (a setup

@@ -52,6 +52,10 @@ __global__ void mx_convert_kernel(const uint8_t* __restrict__ codes, const uint8
     if (rb == 0) tensor_scale[b] = pow2f(shift);
     const int64_t src = gather ? gather[r] : r;
     if (src < 0) continue;  // an out row another call fills
+    if (src >= rows) {      // a gather entry past the input: flagged, the row left untouched
+      atomicOr(&ws[2 * b + 1], 2);
+      continue;
+    }
     const uint8_t* c = codes + (b * rows + src) * (K / 2) + k * 16;
     uint32_t code = 0u;
     if (block_nonzero(c)) {
@@ -114,7 +118,10 @@ nvfp4moe_status nvfp4_from_mxfp4(const uint8_t* codes, const uint8_t* e8m0, int6
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     NVFP4_REQUIRE(e == cudaSuccess, NVFP4MOE_CUDA_ERROR, "%s: %s", fn, cudaGetErrorString(e));
     for (int64_t b = 0; b < batch && bad.size() < 64; ++b)
-      if (host[size_t(2 * b + 1)]) bad += (bad.empty() ? "" : ",") + std::to_string(b);
+      if (host[size_t(2 * b + 1)] & 1) bad += (bad.empty() ? "" : ",") + std::to_string(b);
+    for (int64_t b = 0; b < batch; ++b)
+      NVFP4_REQUIRE(!(host[size_t(2 * b + 1)] & 2), NVFP4MOE_INVALID_ARG, "%s: row_gather names a row >= rows (%lld)",
+                    fn, (long long)rows);
   }
   NVFP4_REQUIRE(bad.empty(), NVFP4MOE_UNSUPPORTED_SHAPE,
                 "%s: matrices [%s] have nonzero blocks whose scales span more than 18 binades (no exact NVFP4 form)",

@@ -231,3 +231,11 @@ def test_from_mxfp4_refuses_spans_without_an_exact_form(dev):
     c, e = O.mx_quantize(y)
     with pytest.raises(C.Nvfp4MoeError, match="18 binades"):
         ops.nvfp4_from_mxfp4(torch.from_numpy(c).to(dev), torch.from_numpy(e).to(dev))
+
+
+def test_from_mxfp4_rejects_a_gather_past_the_input(dev):
+    codes, e8m0 = _mx_matrices(1, 4, 64, seed=3)
+    gather = torch.tensor([0, 1, 7, -1], dtype=torch.int32, device=dev)  # row 7 does not exist
+    with pytest.raises(C.Nvfp4MoeError, match="row_gather"):
+        ops.nvfp4_from_mxfp4(torch.from_numpy(codes).to(dev), torch.from_numpy(e8m0).to(dev), gather, 4,
+                             torch.zeros(1, 4, 32, dtype=torch.uint8, device=dev))
