@@ -58,7 +58,7 @@ template <int EPI>
 __global__ void __launch_bounds__(DTHREADS, 1)
 dense_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, DenseParams p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_shared_1024(smem_raw);
   uint8_t* sA = smem;
   uint8_t* sB = sA + DSTAGES * D_A_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sB + DSTAGES * D_B_BYTES);

@@ -59,7 +59,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p) {
   using S = Smem<BN>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_shared_1024(smem_raw);
   uint8_t* sA = smem;
   uint8_t* sB = sA + STAGES * S::A;
   uint8_t* sSFA = sB + STAGES * S::B;

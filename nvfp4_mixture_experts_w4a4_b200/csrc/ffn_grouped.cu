@@ -199,7 +199,7 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__
   // the phase of a single-GEMM launch; fused launches take it from each item
   constexpr int PH = EPI == EPI_DOWN ? 1 : 0;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_shared_1024(smem_raw);
   uint8_t* sA = smem;
   uint8_t* sB = sA + C::STAGES * C::A_BYTES;
   uint8_t* sSFA = sB + C::STAGES * C::B_BYTES;

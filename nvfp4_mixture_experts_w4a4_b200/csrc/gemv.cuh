@@ -119,4 +119,21 @@ __device__ __forceinline__ void warp_dot8(const uint8_t* __restrict__ wc, const 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// c + w.lo * x.lo, then + w.hi * x.hi: two fused multiply-adds whose f16 (or bf16) operands are
+// multiplied exactly and added in fp32 with one rounding each (the mixed-precision fma of sm_100)
+__device__ __forceinline__ float fma2_f16_f32(uint32_t w, uint32_t x, float c) {
+  asm("{\n .reg .f16 wl, wh, xl, xh;\n mov.b32 {wl, wh}, %1;\n mov.b32 {xl, xh}, %2;\n"
+      " fma.rn.f32.f16 %0, wl, xl, %0;\n fma.rn.f32.f16 %0, wh, xh, %0;\n}"
+      : "+f"(c)
+      : "r"(w), "r"(x));
+  return c;
+}
+__device__ __forceinline__ float fma2_bf16_f32(uint32_t w, uint32_t x, float c) {
+  asm("{\n .reg .b16 wl, wh, xl, xh;\n mov.b32 {wl, wh}, %1;\n mov.b32 {xl, xh}, %2;\n"
+      " fma.rn.f32.bf16 %0, wl, xl, %0;\n fma.rn.f32.bf16 %0, wh, xh, %0;\n}"
+      : "+f"(c)
+      : "r"(w), "r"(x));
+  return c;
+}
+
 }  // namespace nvfp4moe

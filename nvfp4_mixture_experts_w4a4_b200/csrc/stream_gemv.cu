@@ -11,8 +11,12 @@
 //     shared memory once per group of two;
 //   * consumer warp w owns rows 16w..16w+15 of the tile; lane (rsel, cl) takes 16-byte chunk cl
 //     (32 codes, two 16-element blocks) of rows 16w + 2p + rsel, p = 0..7; codes are widened
-//     to f16 (exact) and then fp32, products and the two block sums are fp32, each block sum
-//     is multiplied by its E4M3 scale; the 16 lanes of a row are summed with a butterfly;
+//     to f16 (exact); each token's activations are staged in f16 times a power of two that puts
+//     their largest magnitude in [2^14, 2^15) (exact for every element within a factor 2^28 of it);
+//     products are mixed f16 x f16 + fp32 fused multiply-adds (exact product, one fp32
+//     rounding), the two block sums are fp32, each is multiplied by its E4M3 scale and the
+//     power of two is taken back out of the row result; the 16 lanes of a row are summed with
+//     a butterfly;
 //   * gate/up: rows come as 16 gate rows then 16 up rows per 16-wide block of h; the epilogue
 //     applies the tensor scales, h = silu(g) * u, rounded to bf16;
 //   * down: the 128 rows are output features; each token's row is scaled by its routing
@@ -60,6 +64,33 @@ struct StreamParams {
 
 __device__ __forceinline__ void bar_consumers() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumers * 32) : "memory"); }
 
+// largest finite magnitude among eight bf16 values (0 if none)
+__device__ __forceinline__ float finite_amax8(const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float a = fabsf(bf16_lo(w[i])), b = fabsf(bf16_hi(w[i]));
+    if (a < __int_as_float(0x7F800000)) m = fmaxf(m, a);  // not inf, not NaN
+    if (b < __int_as_float(0x7F800000)) m = fmaxf(m, b);
+  }
+  return m;
+}
+
+// p with amax * 2^p in [2^14, 2^15) (0 for amax 0), kept within [-126, 126] so that 2^p and
+// 2^-p are normal fp32 values
+__device__ __forceinline__ int act_shift(float amax) {
+  if (!(amax > 0.0f)) return 0;
+  const int e = int((__float_as_uint(amax) >> 23) & 0xFFu);
+  return min(max(141 - max(e, 1), -126), 126);
+}
+
+// two bf16 values times the power of two sc, rounded to f16 (exact unless below the f16 normal range)
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w, float sc) {
+  const __half2 h = __floats2half2_rn(bf16_lo(w) * sc, bf16_hi(w) * sc);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 struct GroupCtx {
   const uint8_t* sA;
   const uint8_t* sSF;
@@ -74,9 +105,10 @@ struct GroupCtx {
 
 // The products of one token group with this warp's 16 rows over all K stages (NT tokens,
 // a compile-time count so that no work or register is spent on absent tokens); the row
-// results land in sres[row][t].  `it` counts stages consumed, `ok` turns false on a timeout.
+// results, times xd[t] (the inverse of token t's staging scale), land in sres[row][t].
+// `it` counts stages consumed, `ok` turns false on a timeout.
 template <int NT, bool WB>
-__device__ __forceinline__ void group_products(const GroupCtx& c, uint32_t& it, bool& ok) {
+__device__ __forceinline__ void group_products(const GroupCtx& c, const float (&xd)[kNT], uint32_t& it, bool& ok) {
   const int rsel = c.lane >> 4, cl = c.lane & 15;
   const bool chunk_on = cl * 16 < c.KSB;
   float acc[8][NT];
@@ -109,16 +141,13 @@ __device__ __forceinline__ void group_products(const GroupCtx& c, uint32_t& it, 
           const uint32_t xw[4] = {xv[t].x, xv[t].y, xv[t].z, xv[t].w};
           float b = acc[q][t];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            b = __fmaf_rn(bf16_lo(ww[i]), bf16_lo(xw[i]), b);
-            b = __fmaf_rn(bf16_hi(ww[i]), bf16_hi(xw[i]), b);
-          }
+          for (int i = 0; i < 4; ++i) b = fma2_bf16_f32(ww[i], xw[i], b);
           acc[q][t] = b;
         }
       }
     }
     if (!WB && ok && chunk_on) {
-      // this lane's 32 activation values of each token (shared by its 8 rows)
+      // this lane's 32 activation values of each token as f16 pairs (shared by its 8 rows)
       uint32_t xw[NT][16];
       const int e0 = ks * 2 * c.KSB + cl * 32;
 #pragma unroll
@@ -144,26 +173,13 @@ __device__ __forceinline__ void group_products(const GroupCtx& c, uint32_t& it, 
         uint32_t wf[16];
         decode_chunk(wv, wf);
         const float2 wsc = decode_sf2(sfw);
-        float w32[32];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float2 w2 = __half22float2(*reinterpret_cast<const __half2*>(&wf[i]));
-          w32[2 * i] = w2.x;
-          w32[2 * i + 1] = w2.y;
-        }
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
           float b0 = 0.0f, b1 = 0.0f;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            b0 = __fmaf_rn(w32[2 * i], bf16_lo(xw[t][i]), b0);
-            b0 = __fmaf_rn(w32[2 * i + 1], bf16_hi(xw[t][i]), b0);
-          }
+          for (int i = 0; i < 8; ++i) b0 = fma2_f16_f32(wf[i], xw[t][i], b0);
 #pragma unroll
-          for (int i = 8; i < 16; ++i) {
-            b1 = __fmaf_rn(w32[2 * i], bf16_lo(xw[t][i]), b1);
-            b1 = __fmaf_rn(w32[2 * i + 1], bf16_hi(xw[t][i]), b1);
-          }
+          for (int i = 8; i < 16; ++i) b1 = fma2_f16_f32(wf[i], xw[t][i], b1);
           acc[q][t] = __fmaf_rn(b1, wsc.y, __fmaf_rn(b0, wsc.x, acc[q][t]));
         }
       }
@@ -179,7 +195,7 @@ __device__ __forceinline__ void group_products(const GroupCtx& c, uint32_t& it, 
       float v = acc[q][t];
 #pragma unroll
       for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (cl == 0) c.sres[(16 * c.warp + 2 * q + rsel) * kNT + t] = v;
+      if (cl == 0) c.sres[(16 * c.warp + 2 * q + rsel) * kNT + t] = v * xd[t];
     }
 }
 
@@ -187,14 +203,15 @@ __device__ __forceinline__ void group_products(const GroupCtx& c, uint32_t& it, 
 template <int EPI, bool WB>
 __global__ void __launch_bounds__(kThreadsS, 1) stream_gemv_kernel(const __grid_constant__ CUtensorMap tmW, StreamParams p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_shared_1024(smem_raw);
   const int S = p.stages, KSB = p.KSB, K = p.K;
   const int a_bytes = kRows * KSB, sf_bytes = WB ? 0 : 16 * KSB;  // KSB / 32 scale atoms of 512 bytes
   uint8_t* sA = smem;
   uint8_t* sSF = sA + S * a_bytes;
   uint16_t* xs = reinterpret_cast<uint16_t*>(sSF + S * sf_bytes);  // [kNT][K] bf16
   float* sres = reinterpret_cast<float*>(xs + kNT * K);             // [kRows][kNT]
-  uint64_t* full = reinterpret_cast<uint64_t*>(sres + kRows * kNT);
+  float* sred = sres + kRows * kNT;                                 // [kConsumers][kNT] amax partials
+  uint64_t* full = reinterpret_cast<uint64_t*>(sred + kConsumers * kNT);
   uint64_t* empty = full + S;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + S);
 
@@ -265,6 +282,9 @@ __global__ void __launch_bounds__(kThreadsS, 1) stream_gemv_kernel(const __grid_
       const int nt = min(kNT, n_e - g);
       // stage the group's activation rows (zeros past nt)
       const int vec_per_row = K / 8;  // 16-byte vectors of one bf16 row
+      float lmax[kNT];
+#pragma unroll
+      for (int t = 0; t < kNT; ++t) lmax[t] = 0.0f;
       for (int v = threadIdx.x; v < kNT * vec_per_row; v += kConsumers * 32) {
         const int t = v / vec_per_row, c = v - t * vec_per_row;
         uint4 val = make_uint4(0u, 0u, 0u, 0u);
@@ -273,12 +293,53 @@ __global__ void __launch_bounds__(kThreadsS, 1) stream_gemv_kernel(const __grid_
           val = __ldg(reinterpret_cast<const uint4*>(p.act + src_row * K) + c);
         }
         reinterpret_cast<uint4*>(xs + t * K)[c] = val;
+        if (!WB) {
+          const float am = finite_amax8(val);
+#pragma unroll
+          for (int u = 0; u < kNT; ++u)  // (unrolled: no local-memory array)
+            if (t == u) lmax[u] = fmaxf(lmax[u], am);
+        }
+      }
+      // NVFP4 weights: each token's row becomes f16 times 2^p_t, p_t putting its largest finite
+      // magnitude in [2^14, 2^15); the row results are scaled back by 2^-p_t
+      float xd[kNT];
+#pragma unroll
+      for (int t = 0; t < kNT; ++t) xd[t] = 1.0f;
+      if (!WB) {
+#pragma unroll
+        for (int t = 0; t < kNT; ++t) {
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) lmax[t] = fmaxf(lmax[t], __shfl_xor_sync(0xffffffffu, lmax[t], o));
+          if (lane == 0) sred[warp * kNT + t] = lmax[t];
+        }
+        bar_consumers();
+        float xsc[kNT];
+#pragma unroll
+        for (int t = 0; t < kNT; ++t) {
+          float m = sred[t];
+#pragma unroll
+          for (int w = 1; w < kConsumers; ++w) m = fmaxf(m, sred[w * kNT + t]);
+          const int sh = act_shift(m);
+          xsc[t] = __uint_as_float(uint32_t(127 + sh) << 23);
+          xd[t] = __uint_as_float(uint32_t(127 - sh) << 23);
+        }
+        for (int v = threadIdx.x; v < kNT * vec_per_row; v += kConsumers * 32) {
+          const int t = v / vec_per_row, c = v - t * vec_per_row;
+          uint4* ptr = reinterpret_cast<uint4*>(xs + t * K) + c;
+          float sc = xsc[0];
+#pragma unroll
+          for (int u = 1; u < kNT; ++u)
+            if (t == u) sc = xsc[u];
+          const uint4 raw = *ptr;
+          *ptr = make_uint4(bf16x2_to_f16x2(raw.x, sc), bf16x2_to_f16x2(raw.y, sc), bf16x2_to_f16x2(raw.z, sc),
+                            bf16x2_to_f16x2(raw.w, sc));
+        }
       }
       bar_consumers();
       if (nt == 1)
-        group_products<1, WB>(g_args, it, ok);
+        group_products<1, WB>(g_args, xd, it, ok);
       else
-        group_products<2, WB>(g_args, it, ok);
+        group_products<2, WB>(g_args, xd, it, ok);
       bar_consumers();
       const int l = lane & 15, tt = lane >> 4;
       if (!ok) continue;  // (the next group's barriers are still passed by every warp)
@@ -341,7 +402,7 @@ nvfp4moe_status launch_stream_gemv_a16(int epi, const StreamA16Args& a, int64_t 
   p.status = status;
   p.shared_T = a.shared_T;
   const int stage_bytes = kRows * p.KSB + (wb ? 0 : 16 * p.KSB);
-  const int fixed = 1024 + kNT * p.K * 2 + kRows * kNT * 4 + 64;
+  const int fixed = 1024 + kNT * p.K * 2 + kRows * kNT * 4 + kConsumers * kNT * 4 + 64;
   const int budget = 227 * 1024;
   int stages = (budget - fixed - 16 * 8) / stage_bytes;
   if (stages > 6) stages = 6;

@@ -18,6 +18,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The first 1024-byte aligned byte of dynamic shared memory (the 128-byte swizzle atoms' and
+// the tensor-core descriptors' alignment).  Derived from the shared array by pointer arithmetic,
+// not through an integer, so that the compiler still knows the pointer (and everything derived
+// from it) addresses shared memory and emits shared loads and stores rather than generic ones.
+__device__ __forceinline__ uint8_t* align_shared_1024(uint8_t* base) {
+  return base + ((1024u - (smem_u32(base) & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
 }
