@@ -313,25 +313,24 @@ def time_steps(layer, act, steps: int, warmup: int, flush: L2Flush, dist_on: boo
 
 def time_e2e(layer, act, steps: int, warmup: int, flush: torch.Tensor):
     """The same pass through the public API with host buffers: the graphed layer
-    (ops.GraphedMoeFFN) takes x and logits from pinned host memory (host -> device copies),
-    runs, and its output is copied back to pinned host memory, all inside the events."""
-    x_h = act["x"].cpu().pin_memory()
-    l_h = act["logits"].cpu().pin_memory()
-    o_h = torch.empty(x_h.shape[0], layer.w.H, dtype=torch.bfloat16).pin_memory()
-    graphed = ops.GraphedMoeFFN(layer, x_h.shape[0])
+    (ops.GraphedMoeFFN with host_io) copies x and logits from its pinned host inputs to the
+    device, runs, and copies the output back to its pinned host output, all in one replay
+    inside the events."""
+    graphed = ops.GraphedMoeFFN(layer, act["x"].shape[0], host_io=True)
+    graphed.x_host.copy_(act["x"].cpu())
+    graphed.logits_host.copy_(act["logits"].cpu())
     ms = []
     for i in range(warmup + steps):
         flush.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        out = graphed(x_h, l_h)
-        o_h.copy_(out, non_blocking=True)
+        graphed()
         b.record()
         b.synchronize()
         if i >= warmup:
             ms.append(a.elapsed_time(b))
-    h2d = x_h.numel() * x_h.element_size() + l_h.numel() * l_h.element_size()
-    d2h = o_h.numel() * o_h.element_size()
+    h2d = sum(t.numel() * t.element_size() for t in (graphed.x_host, graphed.logits_host))
+    d2h = graphed.out_host.numel() * graphed.out_host.element_size()
     return statistics.mean(ms), h2d, d2h
 
 

@@ -361,14 +361,25 @@ class GraphedMoeFFN:
     a call copies x and logits into the static inputs (device or pinned host tensors), replays
     the graph (the same kernels as an eager call, without the per-call host work of building
     the call and launching each kernel) and returns the static output (overwritten by the next
-    call)."""
+    call).
 
-    def __init__(self, layer: MoeFFN, T: int):
+    host_io=True also captures the transfers: the graph copies x and logits from pinned host
+    buffers (`x_host`, `logits_host`) to the device, runs the layer and copies the output back
+    to a pinned host buffer (`out_host`), so one replay is the whole host-to-host step.  Fill
+    the host inputs in place (or pass host tensors, which are first copied into them on the
+    CPU); the returned `out_host` is valid once the current stream has reached the replay's
+    end (e.g. after torch.cuda.current_stream().synchronize())."""
+
+    def __init__(self, layer: MoeFFN, T: int, host_io: bool = False):
         dev = layer.w.w13_codes.device
-        self.layer, self.T = layer, T
+        self.layer, self.T, self.host_io = layer, T, host_io
         self.x = torch.zeros(T, layer.w.H, dtype=torch.bfloat16, device=dev)
         self.logits = torch.zeros(T, layer.w.E, dtype=torch.float32, device=dev)
         self.out = torch.empty(T, layer.w.H, dtype=torch.bfloat16, device=dev)
+        if host_io:
+            self.x_host = torch.zeros(T, layer.w.H, dtype=torch.bfloat16).pin_memory()
+            self.logits_host = torch.zeros(T, layer.w.E, dtype=torch.float32).pin_memory()
+            self.out_host = torch.empty(T, layer.w.H, dtype=torch.bfloat16).pin_memory()
         side = torch.cuda.Stream(device=dev)
         side.wait_stream(torch.cuda.current_stream(dev))
         with torch.cuda.stream(side):
@@ -376,9 +387,24 @@ class GraphedMoeFFN:
         torch.cuda.current_stream(dev).wait_stream(side)
         self.graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.graph):
+            if host_io:
+                self.x.copy_(self.x_host, non_blocking=True)
+                self.logits.copy_(self.logits_host, non_blocking=True)
             layer(self.x, self.logits, out=self.out)
+            if host_io:
+                self.out_host.copy_(self.out, non_blocking=True)
 
-    def __call__(self, x: torch.Tensor, logits: torch.Tensor) -> torch.Tensor:
+    def __call__(self, x: torch.Tensor = None, logits: torch.Tensor = None) -> torch.Tensor:
+        if self.host_io:
+            for src, dst in ((x, self.x_host), (logits, self.logits_host)):
+                if src is not None and src.data_ptr() != dst.data_ptr():
+                    if src.shape != dst.shape or src.dtype != dst.dtype or src.is_cuda:
+                        raise ValueError(f"host_io takes host {dst.dtype} {tuple(dst.shape)} inputs")
+                    dst.copy_(src)
+            self.graph.replay()
+            return self.out_host
+        if x is None or logits is None:
+            raise ValueError("x and logits are required")
         if x.shape != self.x.shape or logits.shape != self.logits.shape:
             raise ValueError(f"captured for x {tuple(self.x.shape)}, logits {tuple(self.logits.shape)}")
         self.x.copy_(x, non_blocking=True)

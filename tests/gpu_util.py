@@ -215,10 +215,18 @@ def h_diff_effect(hc, hsf, ref, wl, wd_dequant):
     return extra
 
 
-def run_layer_pair_w4a16(wl: W.Workload, seed: int = 0, dev=None):
-    """The weight-only (W4A16) layer on the device and in the oracle, on the same inputs."""
+def run_layer_pair_w4a16(wl: W.Workload, seed: int = 0, dev=None, x_scale_log2=None):
+    """The weight-only (W4A16) layer on the device and in the oracle, on the same inputs.
+    x_scale_log2 (an int array shaped like x, or one value per token) multiplies x by those
+    powers of two first (exact in bf16 while the results stay normal)."""
     dev = dev or need_gpu()
     act, wts, wg, wu, wd = layer_inputs(wl, seed)
+    if x_scale_log2 is not None:
+        e = np.asarray(x_scale_log2, np.float64)
+        e = e.reshape(-1, 1) if e.ndim == 1 else e
+        scaled = act["x"].double() * torch.from_numpy(np.exp2(e))
+        act["x"] = scaled.to(torch.bfloat16)
+        assert torch.equal(act["x"].double(), scaled), "the scaled x must be exact in bf16"
     ref = O.moe_ffn_w4a16(bf16_bits(act["x"]), act["logits"].numpy(), wl.k, wg, wu, wd)
     layer = ops.MoeFFN(experts_from_oracle(wg, wu, wd, dev), wl.k, None, act=C.ACT_BF16)
     out = layer(act["x"].to(dev), act["logits"].to(dev))

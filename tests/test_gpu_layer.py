@@ -193,6 +193,21 @@ def test_layer_weight_only_w4a16(name):
     assert ops.device_status() == 0
 
 
+def test_weight_only_activations_outside_the_f16_range():
+    """The weight-only products stage each token's bf16 activations in f16 times a power of two
+    chosen from the token's largest magnitude.  Tokens scaled by 2^40, 2^24, 2^-24 and 2^-40
+    (beyond f16's range either way), and tokens whose elements span 2^60 (half of them scaled by
+    2^-60, far below f16's subnormals once the large half sets the power), must meet the same
+    bounds as unscaled ones."""
+    wl = CASES["decode_small_E"]
+    per_token = np.array([40, 24, 0, -24, -40, 0, 12, -12] * ((wl.T + 7) // 8))[:wl.T]
+    e = np.repeat(per_token[:, None], wl.H, axis=1)
+    e[5::8, wl.H // 2:] = -60
+    ref, out, layer = G.run_layer_pair_w4a16(wl, x_scale_log2=e)
+    G.check_layer_w4a16(wl, ref, out, layer)
+    assert ops.device_status() == 0
+
+
 def test_weight_only_rejects_the_tensor_core_path():
     wl = CASES["tiny"]
     act, wts, wg, wu, wd = G.layer_inputs(wl)
@@ -273,3 +288,29 @@ def test_graphed_layer_matches_eager(name):
         assert torch.equal(out, eager)
     with pytest.raises(ValueError):
         graphed(x[:1], logits[:1])
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode_shape"])
+def test_graphed_host_io_matches_eager(name):
+    """With host_io the graph carries the transfers as well: x and logits from pinned host
+    buffers, the output back to one.  Three different batches in turn (two passed to the call,
+    one written into the host inputs in place) each give the eager call's output bit for bit."""
+    wl = GEMM_CASES[name]
+    dev = G.need_gpu()
+    _, wts, wg, wu, wd = G.layer_inputs(wl)
+    layer = ops.MoeFFN(G.experts_from_oracle(wg, wu, wd, dev), wl.k, torch.ones(wl.E, device=dev) * 0.01)
+    graphed = ops.GraphedMoeFFN(layer, wl.T, host_io=True)
+    for seed in (3, 4, 5):
+        act = W.make_activations(wl, seed, "cpu")
+        eager = layer(act["x"].to(dev), act["logits"].to(dev)).cpu()
+        if seed == 5:
+            graphed.x_host.copy_(act["x"])
+            graphed.logits_host.copy_(act["logits"])
+            out = graphed()
+        else:
+            out = graphed(act["x"], act["logits"])
+        torch.cuda.current_stream().synchronize()
+        assert not out.is_cuda
+        assert torch.equal(out, eager)
+    with pytest.raises(ValueError):
+        graphed(act["x"].to(dev), act["logits"].to(dev))
