@@ -85,7 +85,8 @@ enum {
   NVFP4MOE_DEV_BAD_EXPERT_ID = 1u << 0,  /* a routing id outside [0, E) was skipped */
   NVFP4MOE_DEV_DUPLICATE_ID = 1u << 1,   /* a token listed the same expert twice */
   NVFP4MOE_DEV_ROW_OVERFLOW = 1u << 2,   /* permuted rows exceeded the stated capacity */
-  NVFP4MOE_DEV_TIMEOUT = 1u << 3         /* a bounded wait inside a kernel gave up */
+  NVFP4MOE_DEV_TIMEOUT = 1u << 3,        /* a bounded wait inside a kernel gave up */
+  NVFP4MOE_DEV_BAD_GATHER = 1u << 4      /* a row_gather entry past the input rows was skipped */
 };
 
 /* Message for the last failing call on this host thread ("" if none). */
@@ -192,6 +193,29 @@ nvfp4moe_status nvfp4_from_mxfp4(const uint8_t* codes, const uint8_t* e8m0, int6
                                  int64_t K, const int32_t* row_gather, int64_t out_rows,
                                  uint8_t* codes_out, uint8_t* sf_out, float* tensor_scale,
                                  void* workspace, size_t workspace_bytes, nvfp4moe_stream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * nvfp4_prep_weights - weights that arrive already quantised to NVFP4 (E2M1 codes, E4M3 block
+ * scales, fp32 tensor scales: the form the Qwen3.8-Flash-Next-NVFP4-SSD-Stream model card's
+ * checkpoint keeps its routed experts in, two codes per byte) into the layout the layer reads.
+ * Bytes only, nothing is recomputed:
+ *  - out row r of each matrix takes input row row_gather[r] (nullable: row r); a negative
+ *    entry leaves out row r untouched, so the interleaved W13 is built from gate and up in
+ *    two calls (see the gate/up layout above); an entry >= rows also leaves it untouched and
+ *    sets NVFP4MOE_DEV_BAD_GATHER in the device status word;
+ *  - the row's block scales are written in sf_out_layout (the layer needs NVFP4MOE_SF_MMA);
+ *  - the row's codes are copied to codes_out, unless codes_out is NULL: the call then only
+ *    converts the scales between the two layouts (either direction).
+ * Tensor scales are used as they are (moe_ffn_desc.w13_scale keeps gate's and up's apart).
+ * codes [batch][rows][K/2] (16-byte aligned when codes_out is given), sf [batch][...] in
+ * sf_layout (ROWMAJOR: rows*K/16 bytes per matrix; MMA: ceil(rows/128)*128*K/16), 4-byte
+ * aligned; codes_out [batch][out_rows][K/2]; sf_out like sf for out_rows rows.
+ * K % 64 == 0.  Asynchronous on `stream`; allocates nothing.
+ * ---------------------------------------------------------------------------- */
+nvfp4moe_status nvfp4_prep_weights(const uint8_t* codes, const uint8_t* sf, int32_t sf_layout, int64_t batch,
+                                   int64_t rows, int64_t K, const int32_t* row_gather, int64_t out_rows,
+                                   uint8_t* codes_out, uint8_t* sf_out, int32_t sf_out_layout,
+                                   nvfp4moe_stream_t stream);
 
 /* ------------------------------------------------------------------------------
  * moe_route - router top-k (DwarfStar CUDA multi-GPU doc: routers run replicated next to

@@ -19,7 +19,7 @@ COMBINE_AUTO, COMBINE_ORDERED, COMBINE_ACCUMULATE = 0, 1, 2
 ACT_NVFP4, ACT_BF16 = 0, 1
 STAGES = 7
 STAGE_NAMES = ("route", "permute", "quantize_x", "gate_up", "down", "combine")
-DEV_BAD_EXPERT_ID, DEV_DUPLICATE_ID, DEV_ROW_OVERFLOW = 1, 2, 4
+DEV_BAD_EXPERT_ID, DEV_DUPLICATE_ID, DEV_ROW_OVERFLOW, DEV_TIMEOUT, DEV_BAD_GATHER = 1, 2, 4, 8, 16
 
 STATUS_NAMES = {OK: "OK", INVALID_ARG: "INVALID_ARG", UNSUPPORTED_SHAPE: "UNSUPPORTED_SHAPE",
                 WORKSPACE_TOO_SMALL: "WORKSPACE_TOO_SMALL", CUDA_ERROR: "CUDA_ERROR",
@@ -72,6 +72,7 @@ SIGNATURES = {
                                               _i64, _vp, _i64, _i32, _vp]),
     "nvfp4_from_mxfp4_workspace_size": (_sz, [_i64]),
     "nvfp4_from_mxfp4": (_i32, [_vp, _vp, _i64, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "nvfp4_prep_weights": (_i32, [_vp, _vp, _i32, _i64, _i64, _i64, _vp, _i64, _vp, _vp, _i32, _vp]),
     "moe_route": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moe_permute_rows_capacity": (_i64, [_i32, _i32, _i32, _i32]),
     "moe_permute": (_i32, [_vp, _i32, _i32, _i32, _i32, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp,

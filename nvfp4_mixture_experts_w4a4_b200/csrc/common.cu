@@ -65,7 +65,7 @@ extern "C" {
 
 const char* nvfp4moe_last_error(void) { return g_last_error.c_str(); }
 
-int32_t nvfp4moe_version(void) { return 0x000500; }
+int32_t nvfp4moe_version(void) { return 0x000600; }
 
 nvfp4moe_status nvfp4moe_device_status(nvfp4moe_stream_t stream, int32_t clear, uint32_t* status) {
   NVFP4_REQUIRE(status != nullptr, NVFP4MOE_INVALID_ARG, "nvfp4moe_device_status: status is NULL");

@@ -182,6 +182,53 @@ def nvfp4_from_mxfp4(codes: torch.Tensor, e8m0: torch.Tensor, row_gather: torch.
     return out_codes, sf_out, scale
 
 
+def nvfp4_prep_weights(codes: torch.Tensor | None, sf: torch.Tensor, K: int, *, rows: int | None = None,
+                       sf_layout: int = C.SF_ROWMAJOR, row_gather: torch.Tensor | None = None,
+                       out_rows: int | None = None, codes_out: torch.Tensor | None = None,
+                       sf_out: torch.Tensor | None = None, sf_out_layout: int = C.SF_MMA):
+    """Already-quantised NVFP4 matrices into the layer's layout (bytes only): out row r takes
+    input row row_gather[r] (None: r; negative: left untouched), its codes copied to codes_out
+    and its block scales written in sf_out_layout.  codes [B, rows, K/2] or [rows, K/2], or None
+    to convert the scales alone (then give `rows`); sf [B, n] or [n] in sf_layout.  Returns
+    (codes_out or None, sf_out).  A gather entry >= rows is skipped and reported in the device
+    status word (DEV_BAD_GATHER)."""
+    _need_cuda(sf, codes, row_gather)
+    single = codes.dim() == 2 if codes is not None else sf.dim() == 1
+    if codes is not None:
+        codes = (codes[None] if single else codes).contiguous()
+        rows = codes.shape[1]
+    elif rows is None:
+        raise ValueError("rows is required when only the scales are converted")
+    sf = (sf.reshape(1, -1) if single else sf.reshape(sf.shape[0], -1)).contiguous()
+    B = sf.shape[0]
+    out_rows = rows if out_rows is None else out_rows
+    dev = sf.device
+    # outputs the call allocates are [B, ...] and lose the batch axis again for a single matrix;
+    # the caller's own come back as they were given
+    ret_codes, ret_sf = codes_out, sf_out
+    if codes is not None and codes_out is None:
+        codes_out = torch.empty(B, out_rows, K // 2, dtype=torch.uint8, device=dev)
+        ret_codes = codes_out[0] if single else codes_out
+    if sf_out is None:
+        n = sf_mma_bytes(out_rows, K) if sf_out_layout == C.SF_MMA else out_rows * (K // 16)
+        sf_out = torch.empty(B, n, dtype=torch.uint8, device=dev)
+        ret_sf = sf_out[0] if single else sf_out
+    def per_matrix(layout, n_rows):
+        return sf_mma_bytes(n_rows, K) if layout == C.SF_MMA else n_rows * (K // 16)
+
+    if sf.shape[1] != per_matrix(sf_layout, rows):
+        raise ValueError(f"sf holds {sf.shape[1]} bytes per matrix, {per_matrix(sf_layout, rows)} expected")
+    if sf_out.numel() != B * per_matrix(sf_out_layout, out_rows) or not sf_out.is_contiguous():
+        raise ValueError("sf_out must be contiguous, one matrix of scales per batch item")
+    if codes_out is not None and (codes_out.numel() != B * out_rows * (K // 2) or not codes_out.is_contiguous()):
+        raise ValueError("codes_out must be contiguous [B, out_rows, K/2]")
+    gather = None if row_gather is None else row_gather.to(torch.int32).contiguous()
+    st = lib().nvfp4_prep_weights(_p(codes), _p(sf), sf_layout, B, rows, K, _p(gather), out_rows,
+                                  _p(codes_out), _p(sf_out), sf_out_layout, _s())
+    check(st, "nvfp4_prep_weights")
+    return ret_codes, ret_sf
+
+
 def shared_expert_w13(gate: torch.Tensor, up: torch.Tensor) -> torch.Tensor:
     """bf16 gate and up [I_s, H] of a shared expert -> the interleaved [2 I_s, H] the layer takes
     (rows 32c+j: gate row 16c+j for j < 16, up row 16c+j-16 otherwise); a setup-time layout step."""
@@ -227,6 +274,26 @@ class NVFP4Experts:
         w2_codes, w2_sf, sd = nvfp4_from_mxfp4(down[0], down[1])
         return cls(w13_codes, w13_sf, torch.stack([sg, su], 1).contiguous(), w2_codes.contiguous(), w2_sf,
                    sd.contiguous())
+
+    @classmethod
+    def from_nvfp4(cls, gate: tuple, up: tuple, down: tuple, sf_layout: int = C.SF_ROWMAJOR) -> "NVFP4Experts":
+        """Expert weights already quantised to NVFP4, each (codes [E, N, K/2], block scales in
+        sf_layout [E, ...], tensor scales [E]) for gate/up [E, I, H] and down [E, H, I]:
+        gate and up interleaved into W13 and every block scale moved to the MMA layout
+        (nvfp4_prep_weights); the tensor scales are kept as they are."""
+        E, I, h2 = gate[0].shape
+        H = h2 * 2
+        dev = gate[0].device
+        g_map, u_map = cls.interleave_maps(I, dev)
+        w13_codes = torch.empty(E, 2 * I, H // 2, dtype=torch.uint8, device=dev)
+        w13_sf = torch.empty(E, sf_mma_bytes(2 * I, H), dtype=torch.uint8, device=dev)
+        nvfp4_prep_weights(gate[0], gate[1], H, sf_layout=sf_layout, row_gather=g_map, out_rows=2 * I,
+                           codes_out=w13_codes, sf_out=w13_sf)
+        nvfp4_prep_weights(up[0], up[1], H, sf_layout=sf_layout, row_gather=u_map, out_rows=2 * I,
+                           codes_out=w13_codes, sf_out=w13_sf)
+        w2_codes, w2_sf = nvfp4_prep_weights(down[0], down[1], I, sf_layout=sf_layout)
+        w13_scale = torch.stack([gate[2].float(), up[2].float()], 1).contiguous()
+        return cls(w13_codes, w13_sf, w13_scale, w2_codes, w2_sf, down[2].float().contiguous())
 
     @classmethod
     def from_float(cls, w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor) -> "NVFP4Experts":

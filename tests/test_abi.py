@@ -48,7 +48,7 @@ def test_binding_declares_every_symbol():
 
 def test_argument_errors_are_statuses(so):
     from nvfp4_mixture_experts_w4a4_b200 import _lib as C
-    assert so.nvfp4moe_version() == 0x000500
+    assert so.nvfp4moe_version() == 0x000600
     # bad E, bad k: rejected before any device work
     assert so.moe_route(None, 4, 2000, 2, None, None, None) == C.UNSUPPORTED_SHAPE
     assert b"E=2000" in so.nvfp4moe_last_error()
@@ -68,6 +68,12 @@ def test_argument_errors_are_statuses(so):
         C.UNSUPPORTED_SHAPE
     assert so.nvfp4_gemm(None, None, None, None, None, None, 4, 100, 256, None, 0, None, 0, None) == \
         C.UNSUPPORTED_SHAPE
+    # weight preparation: K % 64, unknown layouts, out_rows without a gather, codes_out without codes
+    assert so.nvfp4_prep_weights(None, None, 0, 1, 4, 96, None, 4, None, None, 1, None) == C.UNSUPPORTED_SHAPE
+    assert so.nvfp4_prep_weights(None, None, 2, 1, 4, 64, None, 4, None, None, 1, None) == C.INVALID_ARG
+    assert so.nvfp4_prep_weights(None, None, 0, 1, 4, 64, None, 8, None, None, 1, None) == C.INVALID_ARG
+    assert so.nvfp4_prep_weights(None, 64, 0, 1, 4, 64, None, 4, 128, 128, 1, None) == C.INVALID_ARG
+    assert so.nvfp4_prep_weights(None, None, 0, 0, 4, 64, None, 4, None, None, 1, None) == C.OK
 
 
 def test_workspace_queries(so):

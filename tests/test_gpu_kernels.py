@@ -7,7 +7,7 @@ import torch
 
 import oracle as O
 from nvfp4_mixture_experts_w4a4_b200 import _lib as C
-from nvfp4_mixture_experts_w4a4_b200 import ops
+from nvfp4_mixture_experts_w4a4_b200 import ops, workloads as W
 from tests import gpu_util as G
 from tests.helpers import layouts as LY
 
@@ -231,6 +231,56 @@ def test_from_mxfp4_refuses_spans_without_an_exact_form(dev):
     c, e = O.mx_quantize(y)
     with pytest.raises(C.Nvfp4MoeError, match="18 binades"):
         ops.nvfp4_from_mxfp4(torch.from_numpy(c).to(dev), torch.from_numpy(e).to(dev))
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode_small"])
+def test_from_nvfp4_gives_the_library_layout(dev, name):
+    """Already-quantised NVFP4 experts (the oracle's codes, row-major E4M3 scales and tensor
+    scales) prepared on the device (W13 interleave, MMA scales) equal, byte for byte, the
+    layout the header defines, built on the host from the same arrays."""
+    wl = {"tiny": W.WORKLOADS["tiny"], "decode_small": W.scaled(W.WORKLOADS["decode"], E=12, H=512, I=192)}[name]
+    _, _, wg, wu, wd = G.layer_inputs(wl)
+    up = [tuple(torch.from_numpy(np.ascontiguousarray(a)).to(dev) for a in w) for w in (wg, wu, wd)]
+    got = ops.NVFP4Experts.from_nvfp4(*up)
+    want = LY.experts_to_device_layout(wg, wu, wd)
+    torch.cuda.synchronize()
+    names = ("w13_codes", "w13_sf", "w13_scale", "w2_codes", "w2_sf", "w2_scale")
+    for n, ref in zip(names, want):
+        assert np.array_equal(getattr(got, n).cpu().numpy().reshape(ref.shape), ref), n
+    assert ops.device_status() == 0
+
+
+@pytest.mark.parametrize("B,rows,K", [(1, 5, 64), (3, 200, 192), (2, 256, 1024)])
+def test_prep_weights_scale_layouts_round_trip(dev, B, rows, K):
+    """Scales alone: row-major -> MMA equals the header's layout (padding rows untouched), and
+    MMA -> row-major gives the input back."""
+    rng = np.random.default_rng(rows)
+    sf = rng.integers(0, 256, size=(B, rows * (K // 16)), dtype=np.uint8)
+    mma = torch.zeros(B, LY.sf_mma_bytes(rows, K), dtype=torch.uint8, device=dev)
+    _, mma = ops.nvfp4_prep_weights(None, torch.from_numpy(sf).to(dev), K, rows=rows, sf_out=mma)
+    _, back = ops.nvfp4_prep_weights(None, mma, K, rows=rows, sf_layout=C.SF_MMA, sf_out_layout=C.SF_ROWMAJOR)
+    torch.cuda.synchronize()
+    for b in range(B):
+        assert np.array_equal(mma[b].cpu().numpy(), LY.to_mma(sf[b].reshape(rows, K // 16), K))
+    assert np.array_equal(back.cpu().numpy(), sf)
+
+
+def test_prep_weights_reports_a_gather_past_the_input(dev):
+    """A gather entry past the input rows is skipped and sets DEV_BAD_GATHER; the other rows
+    are still written, a negative entry leaves its row as it was."""
+    assert ops.device_status() == 0
+    rows, K = 4, 64
+    codes = torch.arange(rows * K // 2, dtype=torch.int32, device=dev).to(torch.uint8).reshape(rows, K // 2)
+    sf = torch.arange(1, rows * K // 16 + 1, dtype=torch.uint8, device=dev)
+    gather = torch.tensor([3, 9, -1, 0], dtype=torch.int32, device=dev)
+    out = torch.full((4, K // 2), 0xAB, dtype=torch.uint8, device=dev)
+    ops.nvfp4_prep_weights(codes, sf, K, row_gather=gather, out_rows=4, codes_out=out,
+                           sf_out=torch.zeros(LY.sf_mma_bytes(4, K), dtype=torch.uint8, device=dev))
+    assert ops.device_status(clear=True) == C.DEV_BAD_GATHER
+    assert ops.device_status() == 0
+    o = out.cpu()
+    assert torch.equal(o[0], codes[3].cpu()) and torch.equal(o[3], codes[0].cpu())
+    assert (o[1] == 0xAB).all() and (o[2] == 0xAB).all()
 
 
 def test_from_mxfp4_rejects_a_gather_past_the_input(dev):
