@@ -22,7 +22,7 @@
 //   definition: a value is e2m1(code) * e4m3(block scale) * fp32 tensor scale, with one
 //   E4M3 block scale per 16 consecutive elements along K and the tensor scale of a
 //   dynamically quantised tensor equal to amax / (6 * 448).
-// * Readings taken where nothing fixes a step (each is listed in the design doc):
+// * Readings taken where nothing fixes a step (the kernels take the same ones):
 //   R1 E2M1 encode: round to nearest, ties to the even code, saturate at 6, keep the
 //      sign (a negative value that rounds to zero encodes as 0x8).
 //   R2 E4M3 encode: round to nearest even, saturate to +-448 (no NaN produced).
