@@ -374,14 +374,14 @@ def oracle_rate(wl: W.Workload, act, host, layer, budget_s: float, max_tokens: i
     n = min(wl.T, max_tokens)
     tokens = np.arange(n)
     x, logits, arr, s_x = oracle_inputs(wl, act, host, tokens)
-    s_h = None if a16 else layer.h_scale.cpu().numpy()
     nth = O.default_threads()
     done, t0 = 0, time.perf_counter()
     while True:
         if a16:
             O.moe_ffn_w4a16(x, logits, wl.k, arr["g"], arr["u"], arr["d"], nthreads=nth, shared=shared)
         else:
-            O.moe_ffn(x, logits, wl.k, arr["g"], arr["u"], arr["d"], x_scale=s_x, h_scale=s_h, nthreads=nth,
+            # h_scale None: the oracle calibrates its own per-expert h scales (no device value enters it)
+            O.moe_ffn(x, logits, wl.k, arr["g"], arr["u"], arr["d"], x_scale=s_x, h_scale=None, nthreads=nth,
                       shared=shared)
         done += n
         el = time.perf_counter() - t0
@@ -443,7 +443,6 @@ def main():
         import oracle as O
         tokens = np.arange(n)
         x, logits, arr, s_x = oracle_inputs(wl, act, host, tokens)
-        s_h = layer.h_scale.cpu().numpy()
         nth = O.default_threads()
         # a step is a bounded sample of the workload's tokens, sized to keep the run short
         sample = n
@@ -453,7 +452,7 @@ def main():
                 O.moe_ffn_w4a16(x[:sample], logits[:sample], wl.k, arr["g"], arr["u"], arr["d"], nthreads=nth)
             else:
                 O.moe_ffn(x[:sample], logits[:sample], wl.k, arr["g"], arr["u"], arr["d"], x_scale=s_x,
-                          h_scale=s_h, nthreads=nth)
+                          h_scale=None, nthreads=nth)
         for _ in range(args.warmup):
             one_step()
         t0 = time.perf_counter()
