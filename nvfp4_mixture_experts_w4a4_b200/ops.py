@@ -328,7 +328,8 @@ class MoeFFN:
         self.combine = combine
         self.act = act
         self.shared = None if shared is None else tuple(t.contiguous() for t in shared)
-        self._ws = {}
+        self._ws = {}    # size class (bytes) -> buffer
+        self._need = {}  # T -> workspace bytes
 
     def desc(self, T: int, h_amax: torch.Tensor | None = None, events=None) -> C.MoeFfnDesc:
         w = self.w
@@ -357,17 +358,37 @@ class MoeFFN:
         return L
 
     def workspace(self, T: int) -> torch.Tensor:
-        if T not in self._ws:
-            L = self.layout(T)
-            self._ws[T] = torch.empty(max(L.total, 16), dtype=torch.uint8, device=self.w.w13_codes.device)
-        return self._ws[T]
+        """The device workspace of a T-token call.  Workspaces are pooled by power-of-two size
+        class (at least 1 MiB): batch sizes whose needs fall in one class share a buffer, so
+        serving many batch sizes costs at most twice the largest need in total rather than one
+        buffer per size.  A buffer is never freed, so a CUDA graph that captured a call keeps a
+        valid workspace; calls on one layer must be ordered (one stream), as each call uses the
+        whole workspace."""
+        if T not in self._need:
+            self._need[T] = max(int(self.layout(T).total), 16)
+        need = self._need[T]
+        size_class = max(1 << 20, 1 << (need - 1).bit_length())
+        if size_class not in self._ws:
+            self._ws[size_class] = torch.empty(size_class, dtype=torch.uint8, device=self.w.w13_codes.device)
+        return self._ws[size_class]
 
     def forward(self, x: torch.Tensor, logits: torch.Tensor, out: torch.Tensor | None = None,
                 h_amax: torch.Tensor | None = None, stage_events=None) -> torch.Tensor:
         """stage_events: optional list of 7 torch.cuda.Event (enable_timing) recorded at the
         layer's stage boundaries (see NVFP4MOE_STAGES)."""
         _need_cuda(x, logits, out, h_amax)
+        w = self.w
+        if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[1] != w.H:
+            raise ValueError(f"x must be bf16 [T, {w.H}], got {x.dtype} {tuple(x.shape)}")
         T = x.shape[0]
+        if tuple(logits.shape) != (T, w.E):
+            raise ValueError(f"logits must be [{T}, {w.E}], got {tuple(logits.shape)}")
+        if out is not None and (out.dtype != torch.bfloat16 or tuple(out.shape) != (T, w.H)
+                                or not out.is_contiguous()):
+            raise ValueError(f"out must be a contiguous bf16 [{T}, {w.H}] tensor")
+        if h_amax is not None and (h_amax.dtype != torch.float32 or h_amax.numel() != w.E
+                                   or not h_amax.is_contiguous()):
+            raise ValueError(f"h_amax must be a contiguous fp32 tensor of {w.E} values")
         x = x.contiguous()
         logits = logits.to(torch.float32).contiguous()
         if out is None:
