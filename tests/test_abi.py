@@ -125,3 +125,45 @@ def test_workspace_layout_of_an_empty_batch(so, path, act, shared_I):
     L = C.MoeFfnWsLayout()
     st = so.moe_ffn_workspace_layout(ctypes.byref(d), ctypes.byref(L))
     assert st == (C.UNSUPPORTED_SHAPE if (act == 1 and path == 2) else C.OK)
+
+
+C_CLIENT = r"""
+/* A plain C99 client of the boundary: the header must compile as C, and argument errors
+   come back as status codes (no device is touched). */
+#include <stdio.h>
+#include <string.h>
+#include "nvfp4moe.h"
+
+int main(void) {
+  moe_ffn_desc d;
+  memset(&d, 0, sizeof d);
+  d.T = 4; d.H = 100; d.I = 128; d.E = 8; d.top_k = 2;      /* H not a multiple of 64 */
+  if (nvfp4moe_version() != 0x000600) return 1;
+  if (moe_ffn_workspace_size(&d) != 0) return 2;             /* an invalid desc needs nothing */
+  if (moe_route(NULL, 4, 8, 9, NULL, NULL, NULL) != NVFP4MOE_UNSUPPORTED_SHAPE) return 3;
+  if (strstr(nvfp4moe_last_error(), "k=9") == NULL) return 4;
+  if (nvfp4_prep_weights(NULL, NULL, NVFP4MOE_SF_ROWMAJOR, 0, 4, 64, NULL, 4, NULL, NULL, NVFP4MOE_SF_MMA,
+                         NULL) != NVFP4MOE_OK) return 5;       /* an empty batch is a no-op */
+  printf("ok\n");
+  return 0;
+}
+"""
+
+
+def test_header_compiles_as_c99_and_links(so):
+    """The boundary as a C program sees it: include/nvfp4moe.h compiles with a C compiler in
+    strict C99, and a program linked against libnvfp4moe.so gets status codes and messages."""
+    import subprocess
+    from nvfp4_mixture_experts_w4a4_b200 import _lib
+    work = os.path.join(ROOT, "_build", "c_client")
+    os.makedirs(work, exist_ok=True)
+    src, exe = os.path.join(work, "client.c"), os.path.join(work, "client")
+    with open(src, "w") as f:
+        f.write(C_CLIENT)
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    cc = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                         src, "-o", exe, "-L", libdir, "-l:libnvfp4moe.so", "-Wl,-rpath," + libdir],
+                        capture_output=True, text=True)
+    assert cc.returncode == 0, cc.stderr
+    run = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0 and run.stdout.strip() == "ok", (run.returncode, run.stdout, run.stderr)
