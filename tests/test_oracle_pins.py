@@ -365,6 +365,30 @@ def test_layer_expert_with_no_tokens_and_all_tokens_one_expert():
     assert r["h_scale"][0] == 1.0 and r["h_scale"][2] > 0
 
 
+@pytest.mark.parametrize("seed", [1, 2])
+def test_layer_invariant_under_expert_relabeling(seed):
+    """Experts have no order of their own: relabeling them (permuting the logit columns and the
+    weight stacks together) must leave routing, combine weights and the output bit-for-bit
+    unchanged, while the permuted rows follow the new labels.  A mix-up of expert indices
+    anywhere (weights, per-expert scales, counts, offsets) breaks it."""
+    wl, x, logits, wg, wu, wd = _tiny_layer_inputs()
+    p = np.random.default_rng(seed).permutation(wl.E)  # new expert i is old expert p[i]
+    relabel = lambda w: tuple(np.ascontiguousarray(a[p]) for a in w)  # noqa: E731
+    r0 = O.moe_ffn(x, logits, wl.k, wg, wu, wd, nthreads=2)
+    r1 = O.moe_ffn(x, np.ascontiguousarray(logits[:, p]), wl.k, relabel(wg), relabel(wu), relabel(wd), nthreads=2)
+    assert np.array_equal(p[r1["ids"]], r0["ids"])
+    assert np.array_equal(r1["w"], r0["w"])
+    assert np.array_equal(r1["counts"], r0["counts"][p])
+    assert np.array_equal(r1["h_scale"], r0["h_scale"][p])
+    assert np.array_equal(r1["out_bf16"], r0["out_bf16"])
+    assert np.array_equal(r1["out_f64"], r0["out_f64"])
+    # the same pair lands in a row of its expert's new segment, with the same h codes
+    for t in range(wl.T):
+        for j in range(wl.k):
+            a, b_ = r0["pair_to_row"][t * wl.k + j], r1["pair_to_row"][t * wl.k + j]
+            assert np.array_equal(r0["h_codes"][a], r1["h_codes"][b_])
+
+
 # ------------------------------------------------------- weight-only layer ----
 def _bf16_round(a):
     """fp64 -> fp32 -> bf16 (round to nearest even at each step, by torch), as float64."""
