@@ -389,6 +389,23 @@ def test_layer_invariant_under_expert_relabeling(seed):
             assert np.array_equal(r0["h_codes"][a], r1["h_codes"][b_])
 
 
+@pytest.mark.parametrize("w4a16", [False, True])
+def test_layer_equivariant_under_token_reordering(w4a16):
+    """Tokens are independent apart from the shared scales (the x tensor scale and the per-
+    expert h scales, maxima that ignore order): reordering the tokens reorders the output rows
+    and changes nothing else.  A mix-up of token and row indices breaks it."""
+    wl, x, logits, wg, wu, wd = _tiny_layer_inputs()
+    q = np.random.default_rng(5).permutation(wl.T)
+    run = O.moe_ffn_w4a16 if w4a16 else O.moe_ffn
+    r0 = run(x, logits, wl.k, wg, wu, wd, nthreads=2)
+    r1 = run(np.ascontiguousarray(x[q]), np.ascontiguousarray(logits[q]), wl.k, wg, wu, wd, nthreads=2)
+    assert np.array_equal(r1["ids"], r0["ids"][q])
+    assert np.array_equal(r1["out_bf16"], r0["out_bf16"][q])
+    assert np.array_equal(r1["out_f64"], r0["out_f64"][q])
+    if not w4a16:
+        assert np.array_equal(r1["h_scale"], r0["h_scale"]) and r1["x_scale"] == r0["x_scale"]
+
+
 # ------------------------------------------------------- weight-only layer ----
 def _bf16_round(a):
     """fp64 -> fp32 -> bf16 (round to nearest even at each step, by torch), as float64."""
