@@ -187,16 +187,24 @@ def algorithmic(wl: W.Workload, n_active: int, gemm_path: bool, a16: bool = Fals
             "gate_up_flops": 2.0 * P * 2 * wl.H * wl.I, "gemms_bytes": gemms_bytes}
 
 
+# nominal B200 figures, for the fractions quoted beside the measured ones: HBM3e at 8 TB/s and
+# the published dense FP4 tensor peak (9 PFLOP/s; the doubled figure assumes 2:4 sparsity)
+NOMINAL_HBM_GBS = 8000.0
+NOMINAL_FP4_TFLOPS = 9000.0
+
+
 def roofline(bytes_, flops, ms, pk):
-    """Binding roofline of a kernel that moves `bytes_` and does `flops` in `ms`."""
+    """Binding roofline of a kernel that moves `bytes_` and does `flops` in `ms`: the fraction
+    of the measured peak, and beside it the fraction of the nominal one."""
     t_hbm = bytes_ / (pk["hbm_gbs"] * 1e9)
     t_tc = flops / (pk["fp4_tflops"] * 1e12)
     if t_hbm >= t_tc:
         ach = bytes_ / (ms * 1e-3) / 1e9
-        return {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": ach / pk["hbm_gbs"]}
+        return {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": ach / pk["hbm_gbs"],
+                "nominal": {"peak": NOMINAL_HBM_GBS, "frac": ach / NOMINAL_HBM_GBS}}
     ach = flops / (ms * 1e-3) / 1e12
     return {"bound": "tensor", "achieved": ach, "peak": pk["fp4_tflops"], "unit": "TFLOP/s",
-            "frac": ach / pk["fp4_tflops"]}
+            "frac": ach / pk["fp4_tflops"], "nominal": {"peak": NOMINAL_FP4_TFLOPS, "frac": ach / NOMINAL_FP4_TFLOPS}}
 
 
 def capture_layer(layer, act, out, stage_events=None):

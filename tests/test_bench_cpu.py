@@ -48,12 +48,14 @@ def test_roofline_picks_the_binding_resource():
     assert r["bound"] == "hbm" and r["unit"] == "GB/s"
     assert r["achieved"] == pytest.approx(165_381_120 / 37e-6 / 1e9)
     assert r["frac"] == pytest.approx(r["achieved"] / 6532.9)
+    assert r["nominal"] == {"peak": 8000.0, "frac": pytest.approx(r["achieved"] / 8000.0)}
     # the dense 512-token gate/up: 2*512*2*5120*17408 FLOPs over about 200 MB is compute-bound
     wl = W.WORKLOADS["dense"]
     alg = bench.algorithmic(wl, 1, True)
     r = bench.roofline(alg["gate_up_bytes"], alg["gate_up_flops"], 0.0615, PEAKS)
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert r["frac"] == pytest.approx(alg["gate_up_flops"] / 61.5e-6 / 1e12 / PEAKS["fp4_tflops"])
+    assert r["nominal"]["peak"] == 9000.0 and r["nominal"]["frac"] == pytest.approx(r["achieved"] / 9000.0)
 
 
 @pytest.mark.parametrize("a16", [False, True])
