@@ -3,7 +3,6 @@ seeded inputs and applying the stated tolerances."""
 from __future__ import annotations
 
 import concurrent.futures as cf
-import os
 
 import numpy as np
 import torch
