@@ -56,7 +56,11 @@ class L2Flush:
         return self
 
 
-def peaks():
+def peaks(dev=None):
+    """Roofline denominators: HBM copy and bf16 GEMM from MEASURED_PEAKS.json (or the pool's
+    fallback figures), and the dense FP4 tensor peak measured on this device by the library's
+    tcgen05 kind::mxf4nvf4 MMA loop (operands resident in shared memory) when a device is
+    given, else the bf16 burst figure times the nominal FP4/BF16 ratio (9 / 2.25)."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
@@ -65,8 +69,12 @@ def peaks():
               "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
     else:
         pk = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
-    # dense FP4 tensor peak: the measured bf16 burst figure times the nominal FP4/BF16 ratio (9 / 2.25)
     pk["fp4_tflops"] = pk["bf16_tflops"] * 4.0
+    pk["fp4_source"] = "bf16 burst x 4"
+    if dev is not None:
+        pk["fp4_tflops"] = ops.mma_peak_tflops()
+        pk["fp4_source"] = ("measured: tcgen05 mxf4nvf4 MMA loop, M128 N256 K64, one CTA per SM, operands "
+                            "resident in shared memory")
     return pk
 
 
@@ -140,30 +148,22 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm), "source": "nvml" if self.ok else "unavailable"}
 
 
-def setup_layer(wl: W.Workload, dev, seed: int = 0, keep_tokens: int = 0, path: int = C.PATH_AUTO):
+def setup_layer(wl: W.Workload, dev, seed: int = 0, path: int = C.PATH_AUTO):
     """Draws the workload on the device, quantises the weights with the library, and
-    calibrates the per-expert requantisation scales with one forward (h_amax / 2688).
-
-    The fp32 weights are freed afterwards; host copies are kept only for the experts that
-    the first `keep_tokens` tokens select (what the CPU baseline needs)."""
+    calibrates the per-expert requantisation scales with one forward (h_amax / 2688)."""
     act = W.make_activations(wl, seed, dev)
     wts = W.make_weights(wl, seed, dev)
     experts = ops.NVFP4Experts.from_float(wts["w_gate"], wts["w_up"], wts["w_down"])
+    del wts
     ones = torch.ones(wl.E, dtype=torch.float32, device=dev)
     layer = ops.MoeFFN(experts, wl.k, ones, path=path)
     h_amax = torch.empty(wl.E, dtype=torch.float32, device=dev)
     layer(act["x"], act["logits"], h_amax=h_amax)
     torch.cuda.synchronize()
-    host = {}
-    if keep_tokens:
-        ids = layer.intermediates(wl.T)["topk_ids"][:keep_tokens].cpu().numpy()
-        for e in np.unique(ids):
-            host[int(e)] = {n: wts[n][int(e)].cpu().numpy() for n in ("w_gate", "w_up", "w_down")}
-    del wts
     torch.cuda.empty_cache()
     s_h = torch.where(h_amax > 0, h_amax / 2688.0, ones)
     layer = ops.MoeFFN(experts, wl.k, s_h, path=path)
-    return act, host, experts, layer
+    return act, experts, layer
 
 
 def algorithmic(wl: W.Workload, n_active: int, gemm_path: bool, a16: bool = False, shared_I: int = 0):
@@ -243,19 +243,19 @@ def kernel_nodes(g) -> int | None:
         return None
 
 
-def measured_traffic(workload: str):
-    """DRAM bytes per launch of the gate/up kernel from the committed ncu capture of this
-    workload, or None when there is none or the kernel source changed since it was taken."""
+def measured_traffic(workload: str, source: str = "ffn_grouped.cu"):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu capture of this
+    workload, or None when there is none or the kernel's source file changed since it was taken."""
     import hashlib
     try:
         with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
             rec = json.load(f).get(workload)
-        src = os.path.join(ROOT, "nvfp4_mixture_experts_w4a4_b200", "csrc", "ffn_grouped.cu")
+        src = os.path.join(ROOT, "nvfp4_mixture_experts_w4a4_b200", "csrc", source)
         with open(src, "rb") as f:
             digest = hashlib.sha256(f.read()).hexdigest()
     except (OSError, ValueError):
         return None
-    if not rec or rec.get("source_sha256") != digest:
+    if not rec or rec.get("source_sha256") != digest or rec.get("source", "ffn_grouped.cu") != source:
         return None
     return rec["dram_read_bytes"] + rec["dram_write_bytes"]
 
@@ -343,54 +343,77 @@ def time_e2e(layer, act, steps: int, warmup: int, flush: torch.Tensor):
 
 
 # ----------------------------------------------------------- oracle (CPU) ----
-def oracle_inputs(wl: W.Workload, act, host, tokens: np.ndarray):
-    """Host copies of the inputs for the oracle: x and logits of the sampled tokens and the
-    oracle's own quantisation of the fp32 weights of every expert those tokens select."""
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_inputs(wl: W.Workload, n: int, seed: int = 0):
+    """Inputs of the oracle's timed leg, drawn on the host alone: the workload's activations
+    (same recipe as the device's, from the CPU generator), the first n tokens, and the oracle's
+    own quantisation of the fp32 weights of every expert those tokens select, each expert
+    drawn by workloads.make_expert_weights.  Nothing here touches the GPU or the library."""
     import oracle as O
-    x = act["x"].cpu().view(torch.int16).numpy().view(np.uint16)
-    logits = act["logits"].cpu().numpy()
+    act = W.make_activations(wl, seed, "cpu")
+    x = act["x"].view(torch.int16).numpy().view(np.uint16)
+    logits = act["logits"].numpy()
+    tokens = np.arange(n)
     ids, _ = O.route(logits[tokens], wl.k)
-    need = np.unique(ids)
-    missing = [int(e) for e in need if int(e) not in host]
-    if missing:
-        raise RuntimeError(f"host weights missing for experts {missing[:8]}")
+    need = [int(e) for e in np.unique(ids)]
     shp = {"g": (wl.E, wl.I, wl.H), "d": (wl.E, wl.H, wl.I)}
+    drawn = {}
+
+    def draw(e):
+        drawn[e] = {n_: t.numpy() for n_, t in W.make_expert_weights(wl, e, seed, "cpu").items()}
+
+    with cf.ThreadPoolExecutor(min(8, O.default_threads())) as ex:
+        list(ex.map(draw, need))
     arrays = {}
     for key, name in (("g", "w_gate"), ("u", "w_up"), ("d", "w_down")):
         s = shp["d" if key == "d" else "g"]
-        codes = np.zeros((s[0], s[1], s[2] // 2), np.uint8)
+        codes = np.zeros((s[0], s[1], s[2] // 2), np.uint8)  # untouched experts stay unallocated pages
         sf = np.zeros((s[0], s[1], s[2] // 16), np.uint8)
         sc = np.ones(s[0], np.float32)
-        src = {int(e): host[int(e)][name] for e in need}
 
         def one(e):
-            c, f, t = O.quantize(src[e])
+            c, f, t = O.quantize(drawn[e][name])
             codes[e], sf[e], sc[e] = c, f, t
 
         # ctypes releases the GIL while the oracle runs, so threads quantise in parallel
         with cf.ThreadPoolExecutor(O.default_threads()) as ex:
-            list(ex.map(one, src))
+            list(ex.map(one, need))
         arrays[key] = (codes, sf, sc)
     s_x = np.float32(np.abs((x.astype(np.uint32) << 16).view(np.float32)).max()) / np.float32(2688)
     return x[tokens], logits[tokens], arrays, float(s_x)
 
 
-def oracle_rate(wl: W.Workload, act, host, layer, budget_s: float, max_tokens: int, a16: bool = False,
-                shared=None):
+def oracle_call(wl: W.Workload, inp, nthreads: int, a16: bool = False, shared=None):
+    """One oracle pass over the sampled tokens (h scales calibrated by the oracle itself)."""
+    import oracle as O
+    x, logits, arr, s_x = inp
+    if a16:
+        O.moe_ffn_w4a16(x, logits, wl.k, arr["g"], arr["u"], arr["d"], nthreads=nthreads, shared=shared)
+    else:
+        O.moe_ffn(x, logits, wl.k, arr["g"], arr["u"], arr["d"], x_scale=s_x, h_scale=None, nthreads=nthreads,
+                  shared=shared)
+
+
+def oracle_rate(wl: W.Workload, budget_s: float, max_tokens: int, a16: bool = False, shared=None,
+                nthreads: int | None = None, inp=None):
     """Tokens/s of the oracle on a bounded token sample of the workload (host cores)."""
     import oracle as O
     n = min(wl.T, max_tokens)
-    tokens = np.arange(n)
-    x, logits, arr, s_x = oracle_inputs(wl, act, host, tokens)
-    nth = O.default_threads()
+    inp = inp if inp is not None else oracle_inputs(wl, n)
+    nth = nthreads or O.default_threads()
     done, t0 = 0, time.perf_counter()
     while True:
-        if a16:
-            O.moe_ffn_w4a16(x, logits, wl.k, arr["g"], arr["u"], arr["d"], nthreads=nth, shared=shared)
-        else:
-            # h_scale None: the oracle calibrates its own per-expert h scales (no device value enters it)
-            O.moe_ffn(x, logits, wl.k, arr["g"], arr["u"], arr["d"], x_scale=s_x, h_scale=None, nthreads=nth,
-                      shared=shared)
+        oracle_call(wl, inp, nth, a16, shared)
         done += n
         el = time.perf_counter() - t0
         if el >= budget_s or done >= 64 * n:
@@ -403,87 +426,27 @@ def gpu_launches_per_step(layer) -> int:
     return 6 + (1 if layer.x_scale is None else 0)
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="decode", choices=sorted(W.WORKLOADS))
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--path", default="auto", choices=["auto", "gemv", "tcgen05"],
-                    help="layer path: auto (GEMV for T <= 16), the GEMV path or the tcgen05 grouped GEMM")
-    ap.add_argument("--act", default="nvfp4", choices=["nvfp4", "bf16"],
-                    help="activations: nvfp4 (W4A4) or bf16 (the weight-only W4A16 variant, GEMV path)")
-    ap.add_argument("--shared-I", type=int, default=0,
-                    help="add a BF16 shared expert of this intermediate size (0: none)")
-    args = ap.parse_args()
-    args.warmup = max(args.warmup, 3)
+# the default run: the headline workload first, then the other configurations
+HEADLINE = "decode"
+ALL_WORKLOADS = ("decode", "tiny", "prefill_chunk", "long_prefill", "dense", "dense_t1")
+# workloads whose oracle is also timed on one host thread (small enough to finish in seconds)
+SINGLE_THREAD = ("tiny", "decode", "dense_t1")
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    dist_on = world > 1
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if dist_on:
-        import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                             device_id=dev)
-    wl = W.WORKLOADS[args.workload]
-    cfg = {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "top_k": wl.k,
-           "zipf_s": wl.zipf_s, "outlier_frac": wl.outlier_frac, "l2": "flushed before every step (256 MiB write, then 256 MiB read)",
-           "seed": 0, "parallelism": f"replicas x{world}"}
+
+def workload_config(wl: W.Workload, world: int) -> dict:
+    return {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "top_k": wl.k,
+            "zipf_s": wl.zipf_s, "outlier_frac": wl.outlier_frac,
+            "l2": "flushed before every step (256 MiB write, then 256 MiB read)",
+            "seed": 0, "parallelism": f"replicas x{world}"}
+
+
+def measure(wl: W.Workload, args, dev, local: int, rank: int, world: int, dist_on: bool, cpu_budget: float,
+            pk: dict) -> dict:
+    """Times one workload on this rank's GPU (every rank takes the same collective steps) and,
+    on rank 0 of a one-GPU run, the oracle on a bounded sample of it."""
     a16 = args.act == "bf16"
-    if a16:
-        cfg["act"] = "w4a16 (bf16 activations, NVFP4 weights)"
-    if args.shared_I:
-        cfg["shared_expert"] = f"bf16 SwiGLU, I_s={args.shared_I}"
-
-    if args.impl == "reference":
-        if rank != 0:
-            if dist_on:
-                torch.distributed.destroy_process_group()
-            return
-        n = min(wl.T, ORACLE_SAMPLE.get(wl.name, 4))
-        act, host, _, layer = setup_layer(wl, dev, keep_tokens=n)
-        import oracle as O
-        tokens = np.arange(n)
-        x, logits, arr, s_x = oracle_inputs(wl, act, host, tokens)
-        nth = O.default_threads()
-        # a step is a bounded sample of the workload's tokens, sized to keep the run short
-        sample = n
-
-        def one_step():
-            if a16:
-                O.moe_ffn_w4a16(x[:sample], logits[:sample], wl.k, arr["g"], arr["u"], arr["d"], nthreads=nth)
-            else:
-                O.moe_ffn(x[:sample], logits[:sample], wl.k, arr["g"], arr["u"], arr["d"], x_scale=s_x,
-                          h_scale=None, nthreads=nth)
-        for _ in range(args.warmup):
-            one_step()
-        t0 = time.perf_counter()
-        for _ in range(args.steps):
-            one_step()
-        el = time.perf_counter() - t0
-        value = sample * args.steps / el
-        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                "data": "synthetic", "config": cfg,
-                "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nth, "kind": "oracle",
-                                 "sample": f"{sample} of {wl.T} tokens per step"},
-                "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-        print(json.dumps(line), flush=True)
-        if dist_on:
-            torch.distributed.destroy_process_group()
-        return
-
-    n_cpu = min(wl.T, ORACLE_SAMPLE.get(wl.name, 4))
     path = {"auto": C.PATH_AUTO, "gemv": C.PATH_GEMV, "tcgen05": C.PATH_GEMM}[args.path]
-    act, host, experts, layer = setup_layer(wl, dev, keep_tokens=n_cpu if (rank == 0 and world == 1) else 0,
-                                            path=path)
+    act, experts, layer = setup_layer(wl, dev, path=path)
     shared, shared_bits = None, None
     if args.shared_I:  # a BF16 shared expert, N(0, 1/sqrt(fan_in)) rounded to bf16
         gen = torch.Generator(device=dev).manual_seed(7)
@@ -508,57 +471,174 @@ def main():
     im = layer.intermediates(wl.T)
     n_active = int(im["active"][0].item())
     gemm_path = im["path"] == C.PATH_GEMM
+    single = bool(layer.layout(wl.T).single_launch)
     alg = algorithmic(wl, n_active, gemm_path, a16, args.shared_I)
-    pk = peaks()
-    # the dominant kernel: for batches of at most 64 tokens on the tensor-core path with H <= 2I
-    # both GEMMs run in one fused launch (its stage is "gate_up"); otherwise the gate/up GEMM
-    fused = gemm_path and wl.T <= 64 and wl.H <= 2 * wl.I
+    # the dominant kernel (its stage is "gate_up"): the whole layer in one launch for batches of
+    # at most 16 tokens on the tensor-core path; else, up to 64 tokens with H <= 2I, both GEMMs
+    # in one fused launch; otherwise the gate/up GEMM
+    fused = not single and gemm_path and wl.T <= 64 and wl.H <= 2 * wl.I
     dom_ms = stage_ms["gate_up"]
-    dom_bytes = alg["gemms_bytes"] if fused else alg["gate_up_bytes"]
-    dom_flops = alg["flops"] if fused else alg["gate_up_flops"]
+    dom_bytes = alg["layer_bytes"] if single else alg["gemms_bytes"] if fused else alg["gate_up_bytes"]
+    dom_flops = alg["flops"] if (single or fused) else alg["gate_up_flops"]
     roof = roofline(dom_bytes, dom_flops, dom_ms, pk)
-    kernel = ("fused gate/up + down tcgen05 grouped GEMM (SwiGLU + requant, weighted slots)" if fused
+    kernel = ("single-launch layer: routing, x quantisation, tcgen05 gate/up + SwiGLU + requant, down, "
+              "ordered combine" if single
+              else "fused gate/up + down tcgen05 grouped GEMM (SwiGLU + requant, weighted slots)" if fused
               else "gate_up tcgen05 grouped GEMM + SwiGLU + requant" if gemm_path
               else "gate_up GEMV (bf16 x, NVFP4 weights) + SwiGLU" if a16
               else "gate_up GEMV + SwiGLU + requant")
     roof.update({"kernel": kernel,
-                 "traffic": measured_traffic(wl.name) if gemm_path else None,
-                 "peak_source": pk["source"] + (" (fp4 = bf16 burst x 4)" if roof["bound"] == "tensor" else ""),
+                 "traffic": (measured_traffic(wl.name, "layer_fused.cu") if single
+                             else measured_traffic(wl.name) if gemm_path else None),
+                 "peak_source": pk["source"] + (f" ({pk['fp4_source']})" if roof["bound"] == "tensor" else ""),
                  "algorithmic_bytes_per_launch": dom_bytes,
                  "algorithmic_flops_per_launch": dom_flops, "touched_experts": n_active,
                  "launch_ms": dom_ms})
     layer_roof = roofline(alg["layer_bytes"], alg["flops"], ms_per_step, pk)
     layer_bw = alg["layer_bytes"] / (ms_per_step * 1e-3) / 1e9
+    del layer, experts, act
+    torch.cuda.empty_cache()
     if dist_on:
         torch.distributed.barrier()
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, sample = oracle_rate(wl, act, host, layer, args.cpu_budget, max_tokens=n_cpu, a16=a16,
-                                       shared=shared_bits)
-        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
+    if rank == 0 and world == 1 and cpu_budget > 0:
+        n_cpu = min(wl.T, ORACLE_SAMPLE.get(wl.name, 4))
+        inp = oracle_inputs(wl, n_cpu)
+        v, cores, sample = oracle_rate(wl, cpu_budget, max_tokens=n_cpu, a16=a16, shared=shared_bits, inp=inp)
+        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "cpu_model": cpu_model(), "kind": "oracle",
+               "sample": sample}
+        if wl.name in SINGLE_THREAD:
+            v1, _, s1 = oracle_rate(wl, min(cpu_budget, 4.0), max_tokens=n_cpu, a16=a16, shared=shared_bits,
+                                    nthreads=1, inp=inp)
+            cpu["single_thread"] = {"value": v1, "unit": "tokens/s", "cores": 1, "sample": s1}
+
+    return {
+        "value": value, "ms_per_step": ms_per_step, "config": workload_config(wl, world),
+        "roofline": roof, "cpu_baseline": cpu,
+        "e2e": {"value": world * wl.T / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": (launches if launches is not None else 7) * args.steps,
+        "launches_per_step": launches, "clocks": clk.summary(), "stages_ms": stage_ms,
+        "layer": {"bytes": alg["layer_bytes"], "flops": alg["flops"], "hbm_gbs": layer_bw,
+                  "hbm_frac": layer_bw / pk["hbm_gbs"], "hbm_frac_of_8tbs": layer_bw / NOMINAL_HBM_GBS,
+                  "tflops": alg["flops"] / (ms_per_step * 1e-3) / 1e12,
+                  "fp4_frac": alg["flops"] / (ms_per_step * 1e-3) / 1e12 / pk["fp4_tflops"],
+                  "binding": layer_roof},
+        "path": {C.PATH_GEMV: "gemv", C.PATH_GEMM: "tcgen05"}.get(im["path"], "?"),
+    }
+
+
+def compact(rec: dict) -> dict:
+    """A workload's entry in the headline line's `workloads` object."""
+    out = {k: rec[k] for k in ("value", "ms_per_step", "roofline", "e2e", "clocks", "stages_ms", "path",
+                               "launches_per_step")}
+    out["unit"] = "tokens/s"
+    out["config"] = rec["config"]
+    out["layer_binding"] = rec["layer"]["binding"]
+    out["layer_bytes"] = rec["layer"]["bytes"]
+    out["layer_flops"] = rec["layer"]["flops"]
+    out["cpu_baseline"] = rec["cpu_baseline"]
+    return out
+
+
+def reference_arm(args, wl: W.Workload, rank: int, world: int, dist_on: bool):
+    """The oracle on the host cores, on a bounded token sample of the workload per step.
+    Inputs are drawn on the host (oracle_inputs): this arm never touches the GPU library."""
+    if rank != 0:
+        if dist_on:
+            torch.distributed.destroy_process_group()
+        return
+    import oracle as O
+    n = min(wl.T, ORACLE_SAMPLE.get(wl.name, 4))
+    inp = oracle_inputs(wl, n)
+    nth = O.default_threads()
+    a16 = args.act == "bf16"
+    for _ in range(args.warmup):
+        oracle_call(wl, inp, nth, a16)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_call(wl, inp, nth, a16)
+    el = time.perf_counter() - t0
+    value = n * args.steps / el
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(wl, world),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nth, "cpu_model": cpu_model(),
+                             "kind": "oracle", "sample": f"{n} of {wl.T} tokens per step"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    if dist_on:
+        torch.distributed.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="all", choices=["all"] + sorted(W.WORKLOADS),
+                    help="all: the headline decode workload, then every other configuration (default)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of oracle time for the headline's cpu_baseline (a third of it per other workload)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", default="auto", choices=["auto", "gemv", "tcgen05"],
+                    help="layer path: auto, the GEMV path or the tcgen05 grouped GEMM")
+    ap.add_argument("--act", default="nvfp4", choices=["nvfp4", "bf16"],
+                    help="activations: nvfp4 (W4A4) or bf16 (the weight-only W4A16 variant, GEMV path)")
+    ap.add_argument("--shared-I", type=int, default=0,
+                    help="add a BF16 shared expert of this intermediate size (0: none)")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist_on = world > 1
+    names = ALL_WORKLOADS if args.workload == "all" else (args.workload,)
+
+    if args.impl == "reference":
+        if dist_on:
+            import datetime
+            torch.distributed.init_process_group("gloo", timeout=datetime.timedelta(seconds=300))
+        reference_arm(args, W.WORKLOADS[names[0]], rank, world, dist_on)
+        return
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if dist_on:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    pk = peaks(dev)
+    recs = {}
+    for i, name in enumerate(names):
+        budget = 0.0 if args.no_cpu_baseline else (args.cpu_budget if i == 0 else args.cpu_budget / 3)
+        recs[name] = measure(W.WORKLOADS[name], args, dev, local, rank, world, dist_on, budget, pk)
 
     if rank == 0:
+        head = recs[names[0]]
+        a16 = args.act == "bf16"
+        cfg = dict(head["config"])
+        if a16:
+            cfg["act"] = "w4a16 (bf16 activations, NVFP4 weights)"
+        if args.shared_I:
+            cfg["shared_expert"] = f"bf16 SwiGLU, I_s={args.shared_I}"
         line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None,
+            "metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16 x nvfp4 (w4a16, fp32 accumulate)" if a16 else "nvfp4 (e2m1 x e4m3, fp32 accumulate)",
-            "data": "synthetic",
-            "config": cfg, "roofline": roof, "cpu_baseline": cpu,
-            "e2e": {"value": world * wl.T / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
-            "gpu_launches": (launches if launches is not None else gpu_launches_per_step(layer)) * args.steps,
-            "launches_per_step": launches, "timing": "CUDA-graph replay of the layer's forward, events on the replay stream",
-            "clocks": clk.summary(),
-            "stages_ms": stage_ms,
-            "layer": {"bytes": alg["layer_bytes"], "flops": alg["flops"], "hbm_gbs": layer_bw,
-                      "hbm_frac": layer_bw / pk["hbm_gbs"], "hbm_frac_of_8tbs": layer_bw / 8000.0,
-                      "tflops": alg["flops"] / (ms_per_step * 1e-3) / 1e12,
-                      "fp4_frac": alg["flops"] / (ms_per_step * 1e-3) / 1e12 / pk["fp4_tflops"],
-                      "binding": layer_roof},
-            "path": {C.PATH_GEMV: "gemv", C.PATH_GEMM: "tcgen05"}.get(im["path"], "?"),
+            "data": "synthetic", "config": cfg, "roofline": head["roofline"], "cpu_baseline": head["cpu_baseline"],
+            "e2e": head["e2e"],
+            "gpu_launches": head["gpu_launches"], "launches_per_step": head["launches_per_step"],
+            "timing": "CUDA-graph replay of the layer's forward, events on the replay stream",
+            "clocks": head["clocks"], "stages_ms": head["stages_ms"], "layer": head["layer"], "path": head["path"],
+            "peaks": {k: pk[k] for k in ("hbm_gbs", "bf16_tflops", "fp4_tflops", "source", "fp4_source")},
         }
+        if len(names) > 1:
+            line["workloads"] = {n: compact(r) for n, r in recs.items()}
         print(json.dumps(line), flush=True)
     if dist_on:
         torch.distributed.destroy_process_group()

@@ -159,7 +159,11 @@ nvfp4moe_status nvfp4_quantize(const void* x, int32_t x_dtype, int64_t batch, in
  *  - Every call on a device shares the array and it keeps the last call's contents; each
  *    call overwrites every partial it reads, so nothing has to be cleared.  Calls whose
  *    kernels overlap on the GPU (unordered streams) race on the array: order them.
- *  - The call itself allocates nothing.
+ *  - The call itself allocates nothing.  The array is part of the library's device module:
+ *    the driver places it in device memory when it loads that module on a device, which
+ *    under CUDA's default lazy module loading can be the first call into the library on
+ *    that device.  A host that must see no device allocation after its set-up makes one
+ *    warm-up call of this entry point at set-up (or runs with CUDA_MODULE_LOADING=EAGER).
  * ---------------------------------------------------------------------------- */
 nvfp4moe_status nvfp4_quantize_dynamic_noalloc(const void* x, int32_t x_dtype, int64_t batch,
                                                int64_t rows, int64_t K, int64_t ldx,
@@ -339,7 +343,10 @@ typedef struct {
   int32_t m_tile;   /* 1 on the GEMV path, 64 on the GEMM path */
   int32_t path;     /* resolved path */
   int32_t combine;  /* resolved combine mode; ACCUMULATE: the accumulator is at `slots` */
-  int32_t reserved;
+  int32_t single_launch; /* 1: the whole layer runs as one persistent launch (batches of at most
+                            16 tokens on the GEMM path, ordered combine, given h scales, no
+                            shared expert); `items` then holds its counters, `slots` its fp32
+                            rows by (pair, K chunk of at most 2048) */
   int64_t h_f32;    /* dynamic h scale: fp32 h [h_rows][I] before requantisation */
   int64_t h_stats;  /* dynamic h scale: amax[E] then the scales used, s_h[E] (fp32) */
   int64_t h_bf16;   /* weight-only layer: h in bf16 [T*k][I], permuted rows (x_codes, x_sf,
@@ -356,6 +363,27 @@ size_t moe_ffn_workspace_size(const moe_ffn_desc* d);
 nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* desc, const void* x, const float* logits,
                                 void* out, void* workspace, size_t workspace_bytes,
                                 nvfp4moe_stream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * Measurement and self-test entry points.  The pages have no counterpart of these: they
+ * measure the device and exercise the library's failure reporting, and compute nothing of
+ * the layer.
+ *
+ * nvfp4moe_mma_peak_probe - the block-scaled FP4 tensor-core ceiling of this device.  One
+ * CTA per SM issues iters x 4 tcgen05.mma kind::mxf4nvf4 (M=128, N=256, K=64, E4M3 scales
+ * per 16 elements) on operands resident in shared memory; time the launch on `stream` and
+ * divide nvfp4moe_mma_peak_probe_flops(iters) by it.  1 <= iters <= 2^24.  Writes nothing
+ * but the device status word (NVFP4MOE_DEV_TIMEOUT if a bounded wait gave up).
+ *
+ * nvfp4moe_wait_selftest - one thread waits, at most `polls` polls (1 <= polls <= 2^20),
+ * on an mbarrier phase that never completes, with the bounded wait every tcgen05 kernel of
+ * the library uses.  When the polls run out it sets NVFP4MOE_DEV_TIMEOUT in the device
+ * status word and stores 0 in *result (device int32; 1 if the wait had completed), then
+ * returns.  Nothing faults: the context and later calls stay usable.
+ * ---------------------------------------------------------------------------- */
+nvfp4moe_status nvfp4moe_mma_peak_probe(int64_t iters, nvfp4moe_stream_t stream);
+int64_t nvfp4moe_mma_peak_probe_flops(int64_t iters);
+nvfp4moe_status nvfp4moe_wait_selftest(uint32_t polls, int32_t* result, nvfp4moe_stream_t stream);
 
 #if defined(__GNUC__)
 #pragma GCC visibility pop

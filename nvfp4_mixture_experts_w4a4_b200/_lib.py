@@ -55,7 +55,7 @@ class MoeFfnWsLayout(ctypes.Structure):
         "topk_ids", "topk_w", "counts", "offsets", "padded_offsets", "pair_to_row", "row_token",
         "row_pair", "tile_expert", "active", "x_scale", "x_codes", "x_sf", "h_codes", "h_sf",
         "slots", "amax_partials", "total", "x_rows", "h_rows", "items")] + [
-        ("m_tile", _i32), ("path", _i32), ("combine", _i32), ("reserved", _i32), ("h_f32", _i64), ("h_stats", _i64),
+        ("m_tile", _i32), ("path", _i32), ("combine", _i32), ("single_launch", _i32), ("h_f32", _i64), ("h_stats", _i64),
         ("h_bf16", _i64), ("shared_h", _i64), ("shared_y", _i64)]
 
 
@@ -82,6 +82,9 @@ SIGNATURES = {
     "moe_ffn_workspace_layout": (_i32, [ctypes.POINTER(MoeFfnDesc), ctypes.POINTER(MoeFfnWsLayout)]),
     "moe_ffn_workspace_size": (_sz, [ctypes.POINTER(MoeFfnDesc)]),
     "moe_ffn_forward": (_i32, [ctypes.POINTER(MoeFfnDesc), _vp, _vp, _vp, _vp, _sz, _vp]),
+    "nvfp4moe_mma_peak_probe": (_i32, [_i64, _vp]),
+    "nvfp4moe_mma_peak_probe_flops": (_i64, [_i64]),
+    "nvfp4moe_wait_selftest": (_i32, [ctypes.c_uint32, _vp, _vp]),
 }
 
 _lib = None

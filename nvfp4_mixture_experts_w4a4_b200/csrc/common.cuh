@@ -4,8 +4,10 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <atomic>
 #include <cstdint>
 #include <cstdio>
+#include <mutex>
 #include <string>
 #include <utility>
 
@@ -25,16 +27,33 @@ uint32_t* device_status_ptr();  // sticky fault word of the current device (null
   } while (0)
 
 inline int num_sms() {
-  static int sms[64] = {0};
+  static std::atomic<int> sms[64];  // zero-initialised (static storage); 0 = not read yet
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return 148;
-  if (sms[dev] == 0) {
-    int v = 0;
+  int v = sms[dev].load(std::memory_order_relaxed);
+  if (v == 0) {
     cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    sms[dev] = v > 0 ? v : 148;
+    if (v <= 0) v = 148;
+    sms[dev].store(v, std::memory_order_relaxed);  // every thread computes the same value
   }
-  return sms[dev];
+  return v;
+}
+
+// Raises kernel Kern's dynamic shared-memory limit to `bytes` on the current device, once per
+// device and thread-safe.  A failed attempt is returned and retried by the next call.
+template <auto Kern>
+cudaError_t set_smem_limit_once(int bytes) {
+  static std::mutex mu;
+  static int done[64] = {0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+  e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = 1;
+  return e;
 }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

@@ -55,11 +55,21 @@ int resolve_path(const moe_ffn_desc* d) {
   return gemm_path_available() ? NVFP4MOE_PATH_GEMM : NVFP4MOE_PATH_GEMV;
 }
 
+// The whole layer as one persistent launch: batches of at most 16 tokens on the tensor-core
+// path with the ordered combine (AUTO included), given h scales and no shared expert.
+bool single_launch(const moe_ffn_desc* d, int path) {
+  return path == NVFP4MOE_PATH_GEMM && d->act_mode == NVFP4MOE_ACT_NVFP4 && d->h_scale_mode == NVFP4MOE_SCALE_GIVEN &&
+         d->shared_I == 0 && d->combine != NVFP4MOE_COMBINE_ACCUMULATE &&
+         layer_fused_fits(d->T, d->H, d->I, d->E, d->top_k);
+}
+
 // AUTO: the ordered combine (faster than accumulation at the routed benchmark sizes once the
-// down GEMM stores its rows with tile stores); with top_k = 1 accumulation adds one term per
-// output, so it is exact and deterministic too, and saves the slot round trip
+// down GEMM stores its rows with tile stores; the single launch combines in slot order too);
+// with top_k = 1 on the multi-launch path accumulation adds one term per output, so it is
+// exact and deterministic too, and saves the slot round trip
 int resolve_combine(const moe_ffn_desc* d, int path) {
   if (d->combine != NVFP4MOE_COMBINE_AUTO) return d->combine;
+  if (single_launch(d, path)) return NVFP4MOE_COMBINE_ORDERED;
   return path == NVFP4MOE_PATH_GEMM && d->top_k == 1 ? NVFP4MOE_COMBINE_ACCUMULATE : NVFP4MOE_COMBINE_ORDERED;
 }
 
@@ -116,8 +126,10 @@ void make_layout(const moe_ffn_desc* d, moe_ffn_ws_layout* L) {
   const int combine = resolve_combine(d, path);
   const int64_t prologue_scratch = batch_prologue_scratch_bytes(d->T, d->E);
   L->combine = combine;
-  L->reserved = 0;
-  if (combine == NVFP4MOE_COMBINE_ACCUMULATE)
+  L->single_launch = single_launch(d, path) ? 1 : 0;
+  if (L->single_launch)  // weighted rows by (pair, K chunk)
+    L->slots = take(P * layer_fused_chunks(d->I) * H * 4);
+  else if (combine == NVFP4MOE_COMBINE_ACCUMULATE)
     L->slots = take(prologue_scratch_offset(d, combine) + prologue_scratch);
   else if (path == NVFP4MOE_PATH_GEMM)  // rows by pair; above 64 tokens by padded expert row
     L->slots = take(std::max<int64_t>((prologue_fits(d->T, d->E, d->top_k) ? P : rows_cap) * H * 4, prologue_scratch));
@@ -126,9 +138,12 @@ void make_layout(const moe_ffn_desc* d, moe_ffn_ws_layout* L) {
                                       prologue_scratch));
   // the fused GEMM's work list and per-expert counters, written by the small-batch prologue
   const int64_t A = P < E ? P : E;
-  L->items = take(path == NVFP4MOE_PATH_GEMM && prologue_fits(d->T, d->E, d->top_k)
-                      ? grouped_fused_list_entries(A, 2 * I / 128, H / 128) * 16 + E * 4
-                      : 0);
+  if (L->single_launch)  // per (active expert, K chunk) counters, then per (token, 32 columns) tickets
+    L->items = take((A * layer_fused_chunks(d->I) + T * (H / 32)) * 4);
+  else
+    L->items = take(path == NVFP4MOE_PATH_GEMM && prologue_fits(d->T, d->E, d->top_k)
+                        ? grouped_fused_list_entries(A, 2 * I / 128, H / 128) * 16 + E * 4
+                        : 0);
   // dynamic h scale: fp32 h before requantisation, per-expert amax and scale
   const bool dyn_h = !a16 && d->h_scale_mode == NVFP4MOE_SCALE_DYNAMIC;
   L->h_f32 = take(dyn_h ? L->h_rows * I * 4 : 0);
@@ -251,6 +266,36 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
   };
 
   mark(0);
+  if (L.single_launch) {
+    // one reset launch, then the whole layer as one persistent launch
+    LayerFusedArgs f{};
+    f.x = x; f.logits = logits;
+    f.T = T; f.H = H; f.I = I; f.E = E; f.k = k;
+    f.dynamic = dyn ? 1 : 0; f.x_scale = xs;
+    f.w13_codes = d->w13_codes; f.w13_sf = d->w13_sf; f.w2_codes = d->w2_codes; f.w2_sf = d->w2_sf;
+    f.w13_scale = d->w13_scale; f.w2_scale = d->w2_scale; f.h_scale = d->h_scale; f.h_amax = d->h_amax;
+    f.ids = I32(L.topk_ids); f.w = F32(L.topk_w);
+    f.counts = I32(L.counts); f.offsets = I32(L.offsets); f.padded_offsets = I32(L.padded_offsets);
+    f.pair_to_row = I32(L.pair_to_row); f.row_token = I32(L.row_token); f.row_pair = I32(L.row_pair);
+    f.tile_expert = I32(L.tile_expert); f.active = I32(L.active);
+    f.x_codes = ws + L.x_codes; f.x_sf = ws + L.x_sf; f.h_codes = ws + L.h_codes; f.h_sf = ws + L.h_sf;
+    f.rows_cap = rows_cap;
+    f.slots = F32(L.slots);
+    f.done = I32(L.items);
+    f.tickets = I32(L.items) + max_active_experts(d) * layer_fused_chunks(I);
+    f.out = out;
+    st = launch_layer_fused_reset(f, s);
+    if (st != NVFP4MOE_OK) return st;
+    mark(1);
+    mark(2);
+    mark(3);
+    st = launch_layer_fused(f, s);
+    if (st != NVFP4MOE_OK) return st;
+    mark(4);
+    mark(5);
+    mark(6);
+    return mark_st;
+  }
   if (fused) {
     // small batch: routing, permutation and x quantisation in one cluster launch
     st = launch_prologue(x, logits, T, H, E, k, L.m_tile, dyn ? 1 : 0, xs, I32(L.topk_ids), F32(L.topk_w),

@@ -250,13 +250,9 @@ template <int BN>
 nvfp4moe_status launch(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p, int64_t max_tiles,
                        cudaStream_t s) {
   auto kern = gemm_kernel<BN>;
-  static int configured[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem<BN>::BYTES);
+  {
+    const cudaError_t e = set_smem_limit_once<gemm_kernel<BN>>(Smem<BN>::BYTES);
     if (e != cudaSuccess) return fail(NVFP4MOE_CUDA_ERROR, "tcgen05 GEMM smem attribute: %s", cudaGetErrorString(e));
-    configured[dev] = 1;
   }
   int64_t grid = num_sms();
   if (max_tiles < grid) grid = max_tiles > 0 ? max_tiles : 1;

@@ -68,4 +68,34 @@ nvfp4moe_status launch_gemm_plain(const uint8_t* A, const uint8_t* A_sf, const f
                                   const uint8_t* B_sf, const float* b_scale, int64_t M, int64_t N, int64_t K, void* D,
                                   int d_f32, cudaStream_t s);
 
+// The whole layer as one persistent launch (plus a small reset launch before it) for batches
+// of at most 16 tokens: routing, permutation, x quantisation, both GEMMs and the ordered
+// combine.  It writes the same intermediates as the multi-launch path (padded expert order,
+// m_tile = 64) and the output.
+struct LayerFusedArgs {
+  const void* x;
+  const float* logits;
+  int T, H, I, E, k;
+  int dynamic;
+  float* x_scale;
+  const uint8_t *w13_codes, *w13_sf, *w2_codes, *w2_sf;
+  const float *w13_scale, *w2_scale, *h_scale;
+  float* h_amax;  // nullable
+  int32_t* ids;
+  float* w;
+  int32_t *counts, *offsets, *padded_offsets, *pair_to_row, *row_token, *row_pair, *tile_expert, *active;
+  uint8_t *x_codes, *x_sf, *h_codes, *h_sf;
+  int64_t rows_cap;
+  float* slots;   // [T*k*layer_fused_chunks(I)][H] fp32
+  int* done;      // [min(T*k, E) * layer_fused_chunks(I)]
+  int* tickets;   // [T][H/32]
+  void* out;
+};
+bool layer_fused_fits(int T, int H, int I, int E, int k);
+int layer_fused_chunks(int I);
+// the reset launch (counters, tickets, h maxima to zero), then the layer launch, its
+// programmatic dependent; nothing else may run on the stream between the two
+nvfp4moe_status launch_layer_fused_reset(const LayerFusedArgs& f, cudaStream_t s);
+nvfp4moe_status launch_layer_fused(const LayerFusedArgs& f, cudaStream_t s);
+
 }  // namespace nvfp4moe

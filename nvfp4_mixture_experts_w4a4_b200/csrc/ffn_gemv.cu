@@ -213,14 +213,14 @@ __global__ void combine_kernel(const float* __restrict__ slots, int64_t slot_str
 
 template <typename K>
 int grid_for(K kernel, int64_t warp_items) {
-  static int occ_cache[64] = {0};
+  static std::atomic<int> occ_cache[64];  // zero-initialised; 0 = not queried yet
   int dev = 0;
   cudaGetDevice(&dev);
-  int occ = (dev >= 0 && dev < 64) ? occ_cache[dev] : 0;
+  int occ = (dev >= 0 && dev < 64) ? occ_cache[dev].load(std::memory_order_relaxed) : 0;
   if (occ == 0) {
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kWarpsPerCta * 32, 0);
     if (occ < 1) occ = 1;
-    if (dev >= 0 && dev < 64) occ_cache[dev] = occ;
+    if (dev >= 0 && dev < 64) occ_cache[dev].store(occ, std::memory_order_relaxed);  // same value on every thread
   }
   const int64_t full = int64_t(num_sms()) * occ;
   const int64_t need = (warp_items + kWarpsPerCta - 1) / kWarpsPerCta;

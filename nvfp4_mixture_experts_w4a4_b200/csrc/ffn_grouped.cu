@@ -813,13 +813,9 @@ template <int EPI, class C>
 nvfp4moe_status launch_cfg(const Maps& m0, const Maps& m1, const CUtensorMap& out, const GroupedParams& p,
                            int64_t max_items, cudaStream_t s) {
   auto kern = grouped_kernel<EPI, C>;
-  static int configured[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  {
+    const cudaError_t e = set_smem_limit_once<grouped_kernel<EPI, C>>(C::SMEM_BYTES);
     if (e != cudaSuccess) return fail(NVFP4MOE_CUDA_ERROR, "grouped GEMM smem attribute: %s", cudaGetErrorString(e));
-    configured[dev] = 1;
   }
   int64_t grid = num_sms();
   if (max_items < grid) grid = max_items > 0 ? max_items : 1;

@@ -205,14 +205,10 @@ nvfp4moe_status moe_permute(const int32_t* ids, int32_t T, int32_t E, int32_t k,
   NVFP4_REQUIRE(status != nullptr, NVFP4MOE_CUDA_ERROR, "%s: device status word unavailable", fn);
   const int W = E <= 512 ? 32 : 16;  // warps with a private histogram (smem: W*E ints)
   const size_t smem = sizeof(int32_t) * (size_t(W) * E + 6 * size_t(E) + 3);
-  static int configured[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
-    cudaFuncSetAttribute(permute_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, 100 * 1024);
-    cudaFuncSetAttribute(permute_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, 100 * 1024);
-    configured[dev] = 1;
-  }
+  cudaError_t attr = set_smem_limit_once<permute_kernel<32>>(100 * 1024);
+  if (attr == cudaSuccess) attr = set_smem_limit_once<permute_kernel<16>>(100 * 1024);
+  NVFP4_REQUIRE(attr == cudaSuccess, NVFP4MOE_CUDA_ERROR, "%s: shared-memory attribute: %s", fn,
+                cudaGetErrorString(attr));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (W == 32)
     permute_kernel<32><<<1, kThreads, smem, s>>>(ids, T, E, k, m_tile, rows_cap, counts, offsets, padded_offsets,

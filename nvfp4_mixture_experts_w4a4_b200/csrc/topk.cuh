@@ -5,7 +5,7 @@
 // high word is the logit mapped to an unsigned integer with the same order (after -0 is
 // turned into +0, so the two zeros tie), the low word is 0xFFFF - index, so among equal
 // logits the lower index has the larger key.  Each lane keeps its best remaining key; a
-// round is a warp max over those and only the winning lane recomputes its best.
+// round is a warp max over those and only the winning lane advances its own best.
 // Integer compares make the selection exact; the softmax over the k selected logits
 // (relative to the largest) is fp32.
 #pragma once
@@ -28,24 +28,14 @@ __device__ __forceinline__ float topk_key_value(uint64_t key) {
   return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
 }
 
-// Largest of a lane's keys: a pairwise tree (depth log2 PER_LANE) instead of a linear chain.
-template <int PER_LANE>
-__device__ __forceinline__ uint64_t topk_lane_max(const uint64_t (&key)[PER_LANE]) {
-  uint64_t t[PER_LANE];
-#pragma unroll
-  for (int i = 0; i < PER_LANE; ++i) t[i] = key[i];
-#pragma unroll
-  for (int w = PER_LANE / 2; w >= 1; w /= 2)
-#pragma unroll
-    for (int i = 0; i < w; ++i) t[i] = t[i + w] > t[i] ? t[i + w] : t[i];
-  return t[0];
-}
-
 // Selects the top k (k <= 32) of l[0..E) for the calling warp.  Lane j < k returns the j-th
-// expert in *id and its softmax weight in *w.  A round takes the warp maximum of the lanes'
-// best keys with two hardware reductions (the logit word, then the index word among the lanes
-// that hold that logit, which picks the lower expert index), and only the winning lane drops
-// the key and recomputes its best.
+// expert in *id and its softmax weight in *w.  Each lane first finds its two largest keys.
+// A round takes the warp maximum of the lanes' current best keys with two hardware reductions
+// (the logit word, then the index word among the lanes that hold that logit, which picks the
+// lower expert index); the lane that held the winner moves on to its second key, and only on
+// a further win rescans its keys for the largest one below the key just taken (keys are
+// unique, so "below" excludes exactly the keys already taken).  A lane rarely holds more than
+// two of the k winners, so the rescans are rare and most rounds cost two reductions.
 template <int PER_LANE>
 __device__ __forceinline__ void warp_topk(const float* __restrict__ l, int E, int k, int* id, float* w) {
   const int lane = threadIdx.x & 31;
@@ -53,20 +43,34 @@ __device__ __forceinline__ void warp_topk(const float* __restrict__ l, int E, in
 #pragma unroll
   for (int i = 0; i < PER_LANE; ++i) {
     const int e = lane + 32 * i;
-    key[i] = e < E ? topk_key(l[e], e) : 0ull;  // 0 marks an absent or taken slot
+    key[i] = e < E ? topk_key(l[e], e) : 0ull;  // 0 marks an absent slot (real keys are > 0)
   }
-  uint64_t mine = topk_lane_max<PER_LANE>(key);
-  uint64_t sel = 0;  // lane j keeps the j-th selected key
+  uint64_t m1 = 0, m2 = 0;  // this lane's largest and second largest key
+#pragma unroll
+  for (int i = 0; i < PER_LANE; ++i) {
+    const uint64_t v = key[i];
+    const bool top = v > m1;
+    m2 = top ? m1 : (v > m2 ? v : m2);
+    m1 = top ? v : m1;
+  }
+  bool second = true;  // m2 is still this lane's next key
+  uint64_t sel = 0;    // lane j keeps the j-th selected key
   for (int j = 0; j < k; ++j) {
-    const uint32_t hi = uint32_t(mine >> 32), lo = uint32_t(mine);
+    const uint32_t hi = uint32_t(m1 >> 32), lo = uint32_t(m1);
     const uint32_t mhi = __reduce_max_sync(0xffffffffu, hi);
     const uint32_t mlo = __reduce_max_sync(0xffffffffu, hi == mhi ? lo : 0u);
     const uint64_t best = (uint64_t(mhi) << 32) | mlo;
     if (lane == j) sel = best;
-    if (best == mine) {  // this lane owned the winner (keys are unique): drop it
+    if (best == m1) {  // this lane held the winner
+      if (second) {
+        m1 = m2;
+        second = false;
+      } else {
+        uint64_t nm = 0;
 #pragma unroll
-      for (int i = 0; i < PER_LANE; ++i) key[i] = key[i] == best ? 0ull : key[i];
-      mine = topk_lane_max<PER_LANE>(key);
+        for (int i = 0; i < PER_LANE; ++i) nm = (key[i] < best && key[i] > nm) ? key[i] : nm;
+        m1 = nm;
+      }
     }
   }
   const int bi = topk_key_index(sel);

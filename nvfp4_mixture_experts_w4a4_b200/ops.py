@@ -8,6 +8,7 @@ from __future__ import annotations
 
 import ctypes
 
+import numpy as np
 import torch
 
 from . import _lib as C
@@ -56,6 +57,31 @@ def device_status(clear: bool = True) -> int:
     v = ctypes.c_uint32(0)
     check(lib().nvfp4moe_device_status(_s(), int(clear), ctypes.byref(v)), "nvfp4moe_device_status")
     return int(v.value)
+
+
+def mma_peak_tflops(iters: int = 20000, repeats: int = 3) -> float:
+    """Measured block-scaled FP4 tensor-core ceiling of the current device in TFLOP/s: the
+    best of `repeats` timed launches of nvfp4moe_mma_peak_probe (after one warm-up launch),
+    CUDA events on the current stream."""
+    s = torch.cuda.current_stream()
+    check(lib().nvfp4moe_mma_peak_probe(max(1, iters // 10), _s()), "nvfp4moe_mma_peak_probe")
+    best = float("inf")
+    for _ in range(repeats):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        check(lib().nvfp4moe_mma_peak_probe(iters, _s()), "nvfp4moe_mma_peak_probe")
+        b.record(s)
+        b.synchronize()
+        best = min(best, a.elapsed_time(b))
+    return lib().nvfp4moe_mma_peak_probe_flops(iters) / (best * 1e-3) / 1e12
+
+
+def wait_selftest(polls: int) -> int:
+    """Runs the bounded-wait self-test kernel (a wait on a barrier nothing arrives on, limited
+    to `polls` polls) and returns its result word: 0 when the wait gave up."""
+    r = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    check(lib().nvfp4moe_wait_selftest(polls, _p(r), _s()), "nvfp4moe_wait_selftest")
+    return int(r.item())
 
 
 def nvfp4_quantize(x: torch.Tensor, tensor_scale: torch.Tensor | None = None, *, sf_layout: int = C.SF_MMA,
@@ -232,12 +258,13 @@ def nvfp4_prep_weights(codes: torch.Tensor | None, sf: torch.Tensor, K: int, *, 
 def shared_expert_w13(gate: torch.Tensor, up: torch.Tensor) -> torch.Tensor:
     """bf16 gate and up [I_s, H] of a shared expert -> the interleaved [2 I_s, H] the layer takes
     (rows 32c+j: gate row 16c+j for j < 16, up row 16c+j-16 otherwise); a setup-time layout step."""
-    I = gate.shape[0]
-    g_map, u_map = NVFP4Experts.interleave_maps(I, gate.device)
-    out = torch.empty(2 * I, gate.shape[1], dtype=gate.dtype, device=gate.device)
-    gm, um = g_map >= 0, u_map >= 0
-    out[gm] = gate[g_map[gm].long()]
-    out[um] = up[u_map[um].long()]
+    I, H = gate.shape
+    if I % 16 or up.shape != gate.shape:
+        raise ValueError("gate and up must both be [I_s, H] with I_s a multiple of 16")
+    out = torch.empty(2 * I, H, dtype=gate.dtype, device=gate.device)
+    groups = out.view(I // 16, 2, 16, H)  # row 32c+j = groups[c, j // 16, j % 16]
+    groups[:, 0].copy_(gate.reshape(I // 16, 16, H))
+    groups[:, 1].copy_(up.reshape(I // 16, 16, H))
     return out
 
 
@@ -252,12 +279,14 @@ class NVFP4Experts:
 
     @staticmethod
     def interleave_maps(I: int, device) -> tuple[torch.Tensor, torch.Tensor]:
-        """Row gathers that place gate rows at W13 rows 32c+j (j<16) and up rows at 32c+16+j."""
-        r = torch.arange(2 * I, device=device, dtype=torch.int32)
+        """Row gathers that place gate rows at W13 rows 32c+j (j<16) and up rows at 32c+16+j
+        (-1: the row is the other matrix's).  Built on the host and copied to the device once;
+        the library's gathers (nvfp4_quantize, nvfp4_prep_weights, nvfp4_from_mxfp4) apply them."""
+        r = np.arange(2 * I, dtype=np.int32)
         c, j = r // 32, r % 32
-        gate = torch.where(j < 16, 16 * c + j, torch.full_like(r, -1))
-        up = torch.where(j >= 16, 16 * c + j - 16, torch.full_like(r, -1))
-        return gate, up
+        gate = np.where(j < 16, 16 * c + j, -1).astype(np.int32)
+        up = np.where(j >= 16, 16 * c + j - 16, -1).astype(np.int32)
+        return torch.from_numpy(gate).to(device), torch.from_numpy(up).to(device)
 
     @classmethod
     def from_mxfp4(cls, gate: tuple, up: tuple, down: tuple) -> "NVFP4Experts":

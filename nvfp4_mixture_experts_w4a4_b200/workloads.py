@@ -103,3 +103,17 @@ def make_weights(w: Workload, seed: int = 0, device="cpu") -> dict:
     w_up = torch.randn(w.E, w.I, w.H, generator=g, device=device, dtype=torch.float32) * sg
     w_down = torch.randn(w.E, w.H, w.I, generator=g, device=device, dtype=torch.float32) * sd
     return {"w_gate": w_gate, "w_up": w_up, "w_down": w_down}
+
+
+def make_expert_weights(w: Workload, e: int, seed: int = 0, device="cpu") -> dict:
+    """fp32 weights of expert e alone, same distributions as make_weights, drawn from a
+    generator of their own (seeded by seed and e).  For CPU-side consumers that need a few
+    experts of a large layer without drawing all of them: the values differ from
+    make_weights' draw of the same expert."""
+    g = _gen(1_000_003 * (seed + 1) + e, device)
+    sg = 1.0 / math.sqrt(w.H)
+    sd = 1.0 / math.sqrt(w.I)
+    w_gate = torch.randn(w.I, w.H, generator=g, device=device, dtype=torch.float32) * sg
+    w_up = torch.randn(w.I, w.H, generator=g, device=device, dtype=torch.float32) * sg
+    w_down = torch.randn(w.H, w.I, generator=g, device=device, dtype=torch.float32) * sd
+    return {"w_gate": w_gate, "w_up": w_up, "w_down": w_down}

@@ -233,6 +233,26 @@ def run_layer_pair_w4a16(wl: W.Workload, seed: int = 0, dev=None, x_scale_log2=N
     return ref, out, layer
 
 
+def check_h_bf16(gpu_bits: np.ndarray, ref_bits: np.ndarray, frac: float = H_CODE_FRAC) -> int:
+    """Weight-only h (bf16 bit patterns, rows of one token-expert pair): equal except for at
+    most `frac` of the elements, each one bf16 step away (a rounding boundary that the fp32
+    sums of the device and the fp64 sums of the oracle put on different sides), or where g or
+    u cancel: within 2^-16 of its row's largest |h| (the fp32 sums of the device carry an
+    absolute error of that order there, the oracle's fp64 none).  Returns the differing count."""
+    hg = gpu_bits.astype(np.int64)
+    hr = ref_bits.astype(np.int64)
+    diff = hg != hr
+    assert diff.sum() <= frac * diff.size, f"{diff.sum()} of {diff.size} h values differ"
+    vg = bits_to_f32(hg.astype(np.uint16)).astype(np.float64)
+    vr = bits_to_f32(hr.astype(np.uint16)).astype(np.float64)
+    # bit patterns of one sign are ordered like their values
+    one_step = ((hg >> 15) == (hr >> 15)) & (np.abs(hg - hr) == 1)
+    near_zero = np.abs(vg - vr) <= 2.0 ** -16 * np.abs(vr).max(axis=1, keepdims=True)
+    bad = diff & ~one_step & ~near_zero
+    assert not bad.any(), f"h differs beyond one bf16 step: gpu {vg[bad][:4]} oracle {vr[bad][:4]}"
+    return int(diff.sum())
+
+
 def check_layer_w4a16(wl: W.Workload, ref: dict, out: torch.Tensor, layer: ops.MoeFFN):
     """Routing and permutation bit-exact; h (bf16) equal except for at most H_CODE_FRAC of its
     elements, each one bf16 step away (a rounding boundary that the fp32 sums of the device
@@ -245,20 +265,8 @@ def check_layer_w4a16(wl: W.Workload, ref: dict, out: torch.Tensor, layer: ops.M
     assert np.array_equal(im["counts"].cpu().numpy(), ref["counts"])
     assert np.array_equal(im["offsets"].cpu().numpy(), ref["offsets"])
     assert np.array_equal(im["pair_to_row"].cpu().numpy(), ref["pair_to_row"])
-    hg = im["h_bf16"].cpu().numpy().view(np.uint16).astype(np.int64)
-    hr = ref["h_bf16"].astype(np.int64)
-    diff = hg != hr
-    assert diff.sum() <= H_CODE_FRAC * diff.size, f"{diff.sum()} of {diff.size} h values differ"
-    # a differing value is one bf16 step away (bit patterns of one sign are ordered like their
-    # values), or it sits where g or u cancel: within 2^-16 of its row's largest |h| (the fp32
-    # sums of the device carry an absolute error of that order there, the oracle's fp64 none)
-    vg = bits_to_f32(hg.astype(np.uint16)).astype(np.float64)
-    vr = bits_to_f32(hr.astype(np.uint16)).astype(np.float64)
-    one_step = ((hg >> 15) == (hr >> 15)) & (np.abs(hg - hr) == 1)
-    near_zero = np.abs(vg - vr) <= 2.0 ** -16 * np.abs(vr).max(axis=1, keepdims=True)
-    bad = diff & ~one_step & ~near_zero
-    assert not bad.any(), f"h differs beyond one bf16 step: gpu {vg[bad][:4]} oracle {vr[bad][:4]}"
-    print(f"[parity w4a16] {wl.name} T={T}: {int(diff.sum())} of {diff.size} h values differ")
+    n = check_h_bf16(im["h_bf16"].cpu().numpy().view(np.uint16), ref["h_bf16"])
+    print(f"[parity w4a16] {wl.name} T={T}: {n} of {ref['h_bf16'].size} h values differ")
     return check_out(bf16_bits(out), ref["out_f64"])
 
 

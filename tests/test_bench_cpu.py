@@ -60,13 +60,47 @@ def test_roofline_picks_the_binding_resource():
 
 @pytest.mark.parametrize("a16", [False, True])
 def test_oracle_leg_runs_on_the_cpu(a16):
-    """The cpu_baseline leg times the oracle alone: seeded inputs, the oracle's own weight
-    quantisation and (W4A4) its own per-expert h calibration."""
+    """The cpu_baseline leg times the oracle alone: seeded inputs drawn on the host, the
+    oracle's own weight quantisation and (W4A4) its own per-expert h calibration."""
     wl = W.WORKLOADS["tiny"]
-    act = W.make_activations(wl, 0, "cpu")
-    wts = W.make_weights(wl, 0, "cpu")
-    host = {e: {n: wts[n][e].numpy() for n in ("w_gate", "w_up", "w_down")} for e in range(wl.E)}
-    rate, threads, sample = bench.oracle_rate(wl, act, host, None, budget_s=0.5, max_tokens=4, a16=a16)
+    rate, threads, sample = bench.oracle_rate(wl, budget_s=0.5, max_tokens=4, a16=a16)
     assert rate > 0 and threads >= 1
     assert sample.startswith("4 of 8 tokens per pass")
     assert np.isfinite(rate)
+    r1, t1, _ = bench.oracle_rate(wl, budget_s=0.2, max_tokens=4, a16=a16, nthreads=1)
+    assert t1 == 1 and r1 > 0
+
+
+def test_reference_arm_never_loads_the_gpu_library():
+    """bench.py --impl reference: the oracle on host-drawn inputs; libnvfp4moe.so is never
+    mapped into the process (checked in a fresh interpreter)."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = (
+        "import argparse, bench\n"
+        "from nvfp4_mixture_experts_w4a4_b200 import workloads as W\n"
+        "bench.reference_arm(argparse.Namespace(steps=1, warmup=1, act='nvfp4'), W.WORKLOADS['tiny'], 0, 1, False)\n"
+        "maps = open('/proc/self/maps').read()\n"
+        "print('MAPPED' if 'libnvfp4moe' in maps else 'NOT_MAPPED')\n")
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    out = r.stdout.strip().splitlines()
+    assert out[-1] == "NOT_MAPPED"
+    line = json.loads(out[-2])
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["cpu_baseline"]["cores"] >= 1 and "cpu_model" in line["cpu_baseline"]
+
+
+def test_oracle_inputs_draw_only_the_sampled_tokens_experts():
+    import oracle as O
+    wl = W.WORKLOADS["decode"]
+    x, logits, arr, s_x = bench.oracle_inputs(wl, 2)
+    ids, _ = O.route(logits, wl.k)
+    used = set(np.unique(ids).tolist())
+    sc = arr["g"][2]
+    assert {int(e) for e in np.nonzero(sc != 1.0)[0]} <= used
+    assert all(sc[e] != 1.0 for e in used)  # every used expert was quantised (tensor scale set)
+    assert x.shape == (2, wl.H) and s_x > 0

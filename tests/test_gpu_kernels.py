@@ -289,3 +289,26 @@ def test_from_mxfp4_rejects_a_gather_past_the_input(dev):
     with pytest.raises(C.Nvfp4MoeError, match="row_gather"):
         ops.nvfp4_from_mxfp4(torch.from_numpy(codes).to(dev), torch.from_numpy(e8m0).to(dev), gather, 4,
                              torch.zeros(1, 4, 32, dtype=torch.uint8, device=dev))
+
+
+def test_bounded_wait_gives_up_and_reports_timeout(dev):
+    """The bounded-wait path of the tcgen05 kernels, made to run out: a wait limited to a few
+    polls on a barrier nothing arrives on gives up, sets the timeout bit of the device status
+    word and returns; the context stays usable and the next call reports no fault."""
+    ops.device_status(clear=True)
+    assert ops.wait_selftest(4) == 0
+    assert ops.device_status(clear=True) & C.DEV_TIMEOUT
+    x = torch.randn(8, 64, device=dev)
+    codes, sf, scale = ops.nvfp4_quantize(x)
+    torch.cuda.synchronize()
+    assert codes.shape == (8, 32) and float(scale.item()) > 0
+    assert ops.device_status(clear=True) == 0
+
+
+def test_mma_peak_probe_measures_a_plausible_ceiling(dev):
+    """The FP4 MMA ceiling loop runs to completion (no bounded wait gives up) and gives a rate
+    between a tenth of and twice the published dense FP4 figure (9 PFLOP/s)."""
+    ops.device_status(clear=True)
+    tf = ops.mma_peak_tflops(iters=4000, repeats=1)
+    assert ops.device_status(clear=True) == 0
+    assert 900.0 < tf < 18000.0, tf

@@ -314,3 +314,48 @@ def test_graphed_host_io_matches_eager(name):
         assert torch.equal(out, eager)
     with pytest.raises(ValueError):
         graphed(act["x"].to(dev), act["logits"].to(dev))
+
+
+# Batches of at most 16 tokens on the tensor-core path run the whole layer as one persistent
+# launch (routing, permutation, x quantisation, both GEMMs, the ordered combine).
+SINGLE_CASES = {
+    "decode_E512_k10": W.scaled(W.WORKLOADS["decode"], E=512, H=1024, I=256),
+    "k32_E1024": W.scaled(TINY, T=16, E=1024, k=32, H=256, I=256),
+    "tiny_I128": TINY,
+    "crowded_E4_T16": W.scaled(TINY, T=16, E=4, k=2, H=512, I=384),
+    "ragged_T7": W.scaled(TINY, T=7, E=24, k=3, H=768, I=640),
+    # K chunks of the down items: 2048 + 2048 + 512
+    "dense_T1_three_chunks": W.scaled(W.WORKLOADS["dense"], T=1, H=512, I=4608),
+    # a wide hidden size: fewer weight stages beside the resident x tile
+    "dense_T3_H5120": W.scaled(W.WORKLOADS["dense"], T=3, H=5120, I=384),
+}
+
+
+@pytest.mark.parametrize("name", list(SINGLE_CASES))
+def test_layer_single_launch(name):
+    """The single-launch layer against the oracle with the usual tolerances, then called again
+    on the same workspace: its counters and tickets start from zero in every call, so the second
+    output is the first bit for bit."""
+    wl = SINGLE_CASES[name]
+    ref, out, layer, h_amax = G.run_layer_pair(wl, C.PATH_GEMM)
+    assert layer.layout(wl.T).single_launch == 1
+    G.check_layer(wl, ref, out, layer, h_amax)
+    act = W.make_activations(wl, 0, "cpu")
+    again = layer(act["x"].cuda(), act["logits"].cuda())
+    torch.cuda.synchronize()
+    assert torch.equal(out, again)
+    assert ops.device_status() == 0
+
+
+def test_single_launch_is_not_taken_where_it_does_not_apply():
+    """17 tokens, the accumulating combine, a dynamic h scale or a shared expert keep the
+    multi-launch path."""
+    dev = G.need_gpu()
+    wl = W.scaled(TINY, T=17)
+    _, wts, wg, wu, wd = G.layer_inputs(wl)
+    ex = G.experts_from_oracle(wg, wu, wd, dev)
+    ones = torch.ones(wl.E, device=dev)
+    assert ops.MoeFFN(ex, wl.k, ones).layout(17).single_launch == 0
+    assert ops.MoeFFN(ex, wl.k, ones).layout(16).single_launch == 1
+    assert ops.MoeFFN(ex, wl.k, ones, combine=C.COMBINE_ACCUMULATE).layout(16).single_launch == 0
+    assert ops.MoeFFN(ex, wl.k, None).layout(16).single_launch == 0
