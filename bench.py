@@ -148,7 +148,7 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm), "source": "nvml" if self.ok else "unavailable"}
 
 
-def setup_layer(wl: W.Workload, dev, seed: int = 0, path: int = C.PATH_AUTO):
+def setup_layer(wl: W.Workload, dev, seed: int = 0, path: int = C.PATH_AUTO, launch: int = C.LAUNCH_AUTO):
     """Draws the workload on the device, quantises the weights with the library, and
     calibrates the per-expert requantisation scales with one forward (h_amax / 2688)."""
     act = W.make_activations(wl, seed, dev)
@@ -156,13 +156,13 @@ def setup_layer(wl: W.Workload, dev, seed: int = 0, path: int = C.PATH_AUTO):
     experts = ops.NVFP4Experts.from_float(wts["w_gate"], wts["w_up"], wts["w_down"])
     del wts
     ones = torch.ones(wl.E, dtype=torch.float32, device=dev)
-    layer = ops.MoeFFN(experts, wl.k, ones, path=path)
+    layer = ops.MoeFFN(experts, wl.k, ones, path=path, launch=launch)
     h_amax = torch.empty(wl.E, dtype=torch.float32, device=dev)
     layer(act["x"], act["logits"], h_amax=h_amax)
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
     s_h = torch.where(h_amax > 0, h_amax / 2688.0, ones)
-    layer = ops.MoeFFN(experts, wl.k, s_h, path=path)
+    layer = ops.MoeFFN(experts, wl.k, s_h, path=path, launch=launch)
     return act, experts, layer
 
 
@@ -446,7 +446,11 @@ def measure(wl: W.Workload, args, dev, local: int, rank: int, world: int, dist_o
     on rank 0 of a one-GPU run, the oracle on a bounded sample of it."""
     a16 = args.act == "bf16"
     path = {"auto": C.PATH_AUTO, "gemv": C.PATH_GEMV, "tcgen05": C.PATH_GEMM}[args.path]
-    act, experts, layer = setup_layer(wl, dev, path=path)
+    launch = {"auto": C.LAUNCH_AUTO, "single": C.LAUNCH_SINGLE, "multi": C.LAUNCH_MULTI}[args.launch]
+    if launch == C.LAUNCH_SINGLE and not (wl.T <= 16 and path != C.PATH_GEMV and args.act == "nvfp4"
+                                          and not args.shared_I):
+        launch = C.LAUNCH_AUTO  # the single launch does not apply to this workload
+    act, experts, layer = setup_layer(wl, dev, path=path, launch=launch)
     shared, shared_bits = None, None
     if args.shared_I:  # a BF16 shared expert, N(0, 1/sqrt(fan_in)) rounded to bf16
         gen = torch.Generator(device=dev).manual_seed(7)
@@ -459,7 +463,7 @@ def measure(wl: W.Workload, args, dev, local: int, rank: int, world: int, dist_o
     if a16:  # the same experts, weight-only
         layer = ops.MoeFFN(experts, wl.k, None, act=C.ACT_BF16, shared=shared)
     elif shared is not None:
-        layer = ops.MoeFFN(experts, wl.k, layer.h_scale, path=path, shared=shared)
+        layer = ops.MoeFFN(experts, wl.k, layer.h_scale, path=path, shared=shared, launch=launch)
     flush = L2Flush(dev)
     with ClockSampler(local) as clk:
         step_ms, stage_ms, launches = time_steps(layer, act, args.steps, args.warmup, flush, dist_on)
@@ -525,7 +529,8 @@ def measure(wl: W.Workload, args, dev, local: int, rank: int, world: int, dist_o
                   "tflops": alg["flops"] / (ms_per_step * 1e-3) / 1e12,
                   "fp4_frac": alg["flops"] / (ms_per_step * 1e-3) / 1e12 / pk["fp4_tflops"],
                   "binding": layer_roof},
-        "path": {C.PATH_GEMV: "gemv", C.PATH_GEMM: "tcgen05"}.get(im["path"], "?"),
+        "path": {C.PATH_GEMV: "gemv", C.PATH_GEMM: "tcgen05"}.get(im["path"], "?")
+                + (" (single launch)" if single else ""),
     }
 
 
@@ -590,6 +595,8 @@ def main():
                     help="activations: nvfp4 (W4A4) or bf16 (the weight-only W4A16 variant, GEMV path)")
     ap.add_argument("--shared-I", type=int, default=0,
                     help="add a BF16 shared expert of this intermediate size (0: none)")
+    ap.add_argument("--launch", default="auto", choices=["auto", "single", "multi"],
+                    help="batches of at most 16 tokens: one persistent launch, the multi-launch path, or automatic")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 

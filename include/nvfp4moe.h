@@ -327,7 +327,20 @@ typedef struct {
   int32_t shared_I;
   const uint16_t* shared_w13;
   const uint16_t* shared_w2;
+  /* NVFP4MOE_LAUNCH_*: how a batch that the single-launch layer supports (tensor-core path,
+   * at most 16 tokens, ordered combine, given h scales, no shared expert) is run:
+   *   SINGLE  one persistent launch for the whole layer (after a small launch that resets its
+   *           counters): every CTA routes the batch, x stays quantised in shared memory, the
+   *           down tiles of an expert wait on counters of its gate/up tiles, and the combine is
+   *           done by the last writer of each token's rows;
+   *   MULTI   the routing/permutation/quantisation prologue, then the grouped GEMMs, then the
+   *           combine (the path every larger batch takes);
+   *   AUTO    the faster of the two for the shape (see moe_ffn_workspace_layout's single_launch).
+   * Both give the same routing, permutation and codes, and outputs within the stated tolerance. */
+  int32_t launch_mode;
 } moe_ffn_desc;
+
+enum { NVFP4MOE_LAUNCH_AUTO = 0, NVFP4MOE_LAUNCH_SINGLE = 1, NVFP4MOE_LAUNCH_MULTI = 2 };
 
 enum { NVFP4MOE_STAGES = 7 };
 

@@ -17,6 +17,7 @@ DTYPE_BF16, DTYPE_F32 = 0, 1
 PATH_AUTO, PATH_GEMV, PATH_GEMM = 0, 1, 2
 COMBINE_AUTO, COMBINE_ORDERED, COMBINE_ACCUMULATE = 0, 1, 2
 ACT_NVFP4, ACT_BF16 = 0, 1
+LAUNCH_AUTO, LAUNCH_SINGLE, LAUNCH_MULTI = 0, 1, 2
 STAGES = 7
 STAGE_NAMES = ("route", "permute", "quantize_x", "gate_up", "down", "combine")
 DEV_BAD_EXPERT_ID, DEV_DUPLICATE_ID, DEV_ROW_OVERFLOW, DEV_TIMEOUT, DEV_BAD_GATHER = 1, 2, 4, 8, 16
@@ -46,7 +47,7 @@ class MoeFfnDesc(ctypes.Structure):
         ("w13_codes", _vp), ("w13_sf", _vp), ("w13_scale", _vp),
         ("w2_codes", _vp), ("w2_sf", _vp), ("w2_scale", _vp),
         ("h_scale", _vp), ("h_amax", _vp), ("stage_events", _vp), ("combine", _i32), ("h_scale_mode", _i32),
-        ("act_mode", _i32), ("shared_I", _i32), ("shared_w13", _vp), ("shared_w2", _vp),
+        ("act_mode", _i32), ("shared_I", _i32), ("shared_w13", _vp), ("shared_w2", _vp), ("launch_mode", _i32),
     ]
 
 

@@ -39,6 +39,8 @@ nvfp4moe_status check_desc(const moe_ffn_desc* d, const char* fn) {
                 "%s: the weight-only layer runs the GEMV path", fn);
   NVFP4_REQUIRE(d->shared_I >= 0 && d->shared_I % 64 == 0, NVFP4MOE_UNSUPPORTED_SHAPE,
                 "%s: shared_I=%d must be a multiple of 64", fn, d->shared_I);
+  NVFP4_REQUIRE(d->launch_mode >= NVFP4MOE_LAUNCH_AUTO && d->launch_mode <= NVFP4MOE_LAUNCH_MULTI,
+                NVFP4MOE_INVALID_ARG, "%s: bad launch_mode %d", fn, d->launch_mode);
   return NVFP4MOE_OK;
 }
 
@@ -55,12 +57,21 @@ int resolve_path(const moe_ffn_desc* d) {
   return gemm_path_available() ? NVFP4MOE_PATH_GEMM : NVFP4MOE_PATH_GEMV;
 }
 
-// The whole layer as one persistent launch: batches of at most 16 tokens on the tensor-core
-// path with the ordered combine (AUTO included), given h scales and no shared expert.
-bool single_launch(const moe_ffn_desc* d, int path) {
+// Batches the single-launch layer supports: at most 16 tokens on the tensor-core path with the
+// ordered combine (AUTO included), given h scales and no shared expert.
+bool single_launch_fits(const moe_ffn_desc* d, int path) {
   return path == NVFP4MOE_PATH_GEMM && d->act_mode == NVFP4MOE_ACT_NVFP4 && d->h_scale_mode == NVFP4MOE_SCALE_GIVEN &&
          d->shared_I == 0 && d->combine != NVFP4MOE_COMBINE_ACCUMULATE &&
          layer_fused_fits(d->T, d->H, d->I, d->E, d->top_k);
+}
+
+// Whether this call runs as one launch.  AUTO takes it where it measured faster than the
+// multi-launch path: the dense layer (one expert), whose down tiles then split along K.  For
+// routed batches the multi-launch path is faster: there the single launch's gate/up -> down
+// counters and per-tile tickets cost more than the launches they save.
+bool single_launch(const moe_ffn_desc* d, int path) {
+  if (d->launch_mode == NVFP4MOE_LAUNCH_MULTI || !single_launch_fits(d, path)) return false;
+  return d->launch_mode == NVFP4MOE_LAUNCH_SINGLE || d->E == 1;
 }
 
 // AUTO: the ordered combine (faster than accumulation at the routed benchmark sizes once the
@@ -200,6 +211,9 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
     NVFP4_REQUIRE(d->E <= 1024, NVFP4MOE_UNSUPPORTED_SHAPE, "%s: E > 1024", fn);
     NVFP4_REQUIRE(gemm_path_available(), NVFP4MOE_CUDA_ERROR, "%s: the tensor-core path is unavailable", fn);
   }
+  NVFP4_REQUIRE(d->launch_mode != NVFP4MOE_LAUNCH_SINGLE || L.single_launch, NVFP4MOE_UNSUPPORTED_SHAPE,
+                "%s: the single launch takes at most 16 tokens on the tensor-core path with the ordered combine, "
+                "given h scales and no shared expert", fn);
   NVFP4_REQUIRE(L.combine != NVFP4MOE_COMBINE_ACCUMULATE || L.path == NVFP4MOE_PATH_GEMM, NVFP4MOE_UNSUPPORTED_SHAPE,
                 "%s: the accumulating combine needs the tensor-core path", fn);
   const bool dyn_h = !a16 && d->h_scale_mode == NVFP4MOE_SCALE_DYNAMIC;

@@ -32,7 +32,7 @@
 // A small launch before this one zeroes the counters and tickets; this kernel is its
 // programmatic dependent and waits for it only before touching them (well after its start).
 //
-// Warp roles after the routing phase:
+// Warp roles after the routing phase (all 16 warps route, one token each, and quantise x):
 //   warp 0      weight producer: TMA loads of 128 x 128-byte tiles (128-byte swizzle) and the
 //               bulk copies of their scale atoms into a ring of stages;
 //   warp 1      TMEM owner and MMA issuer: tcgen05.cp of the scales, four K=64 block-scaled
@@ -40,7 +40,8 @@
 //   warps 2..9  epilogue: four warps (one per 32-lane TMEM quarter) per item, the two sets of
 //               four taking alternate items;
 //   warp 10     h producer: for down tiles, acquires the expert's chunk counter and loads
-//               the h rows and their scale atoms into the stage the weight producer armed.
+//               the h rows and their scale atoms into the stage the weight producer armed;
+//   warps 11-15 routing, x quantisation and the inspection copies only.
 // Every wait is bounded (status bit on timeout; copies in flight land before the CTA exits).
 #include "ffn_gemm.cuh"
 #include "tcgen05.cuh"
@@ -52,7 +53,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int LF_WARPS = 11;
+constexpr int LF_WARPS = 16;
 constexpr int LF_THREADS = 32 * LF_WARPS;
 constexpr int LF_MAXT = 16;             // tokens = the MMA's N (one 16-row token tile)
 constexpr int LF_MAXE = 1024;
@@ -61,7 +62,7 @@ constexpr int WM = 128;                 // weight rows per tile (the MMA's M)
 constexpr int BK = 256;                 // K per stage
 constexpr int KB = BK / 2;              // bytes per row per stage
 constexpr int TOK_ALIGN = 64;           // padded rows per active expert (h and the x copies)
-constexpr int EPI_FIRST = 2, EPI_WARPS = 8, HPROD_WARP = 10;
+constexpr int EPI_FIRST = 2, EPI_WARPS = 8, HPROD_WARP = 10;  // warps 11..15: set-up only
 constexpr int NACC = 8;                 // TMEM accumulators (items in flight past the MMA)
 constexpr int KC_MAX = 2048;            // K chunk of a down item
 constexpr int A_BYTES = WM * KB;        // 16 KB
@@ -329,10 +330,19 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
     tmem_relinquish();
     tc_fence_before();
   }
-  if (warp == 0 && lane == 0) {
-    prefetch_tensormap(&tmW13);
-    prefetch_tensormap(&tmW2);
-    prefetch_tensormap(&tmH);
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tensormap(&tmW13);
+      prefetch_tensormap(&tmW2);
+      prefetch_tensormap(&tmH);
+    }
+    // the per-expert scales are read once the active experts are known: bring them into L2 now
+    for (int off = lane * 128; off < E * 8; off += 32 * 128)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char*>(a.w13_scale) + off));
+    for (int off = lane * 128; off < E * 4; off += 32 * 128) {
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char*>(a.w2_scale) + off));
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char*>(a.h_scale) + off));
+    }
   }
   for (int e = tid; e < E; e += LF_THREADS) s_mask[e] = 0u;
 
@@ -783,7 +793,7 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
             bulk_load(sSFB + s * SFB_BYTES, hsf + int64_t(kt) * 4 * 512, uint32_t(steps_of(w, kt)) * 512, &full[s]);
           }
         }
-      } else {
+      } else if (warp >= EPI_FIRST && warp < EPI_FIRST + EPI_WARPS) {
         // ---------------------------------------------------------- epilogue ----
         const int q = warp & 3;                    // TMEM lane quarter of this warp
         const int half = (warp - EPI_FIRST) >> 2;  // items j with j % 2 == half
@@ -857,7 +867,8 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
             }
             pending = w.a * nkc + (w.mt * 64) / KC;
           } else {
-            // lane = output row mt*128 + 32q + lane; column c = the expert's c-th token
+            // lane = output row mt*128 + 32q + lane; column c = the expert's c-th token; the
+            // weighted row of each (pair, K chunk) goes to its slot, summed by the combine
             const int col = w.mt * WM + q * 32 + lane;
             const int base = s_aoff[w.a];
             int my_pair = -1;
@@ -875,10 +886,7 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
             // for the last one, makes the other warps' rows visible to the reads below.
             __syncwarp();
             bool last = false;
-            if (lane < cnt) {
-              const int t = my_pair / k;
-              last = atom_acq_rel_add1(a.tickets + t * cols32 + (col >> 5)) == k * nkc - 1;
-            }
+            if (lane < cnt) last = atom_acq_rel_add1(a.tickets + (my_pair / k) * cols32 + (col >> 5)) == k * nkc - 1;
             uint32_t lastm = __ballot_sync(0xffffffffu, last);
             while (lastm) {
               const int c = __ffs(lastm) - 1;

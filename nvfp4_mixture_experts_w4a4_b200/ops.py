@@ -343,12 +343,14 @@ class MoeFFN:
 
     def __init__(self, experts: NVFP4Experts, top_k: int, h_scale: torch.Tensor | None,
                  x_scale: torch.Tensor | None = None, path: int = C.PATH_AUTO, combine: int = C.COMBINE_AUTO,
-                 act: int = C.ACT_NVFP4, shared: tuple | None = None):
+                 act: int = C.ACT_NVFP4, shared: tuple | None = None, launch: int = C.LAUNCH_AUTO):
         """h_scale: per-expert requantisation scales of h, or None for the dynamic scale
         (amax of each expert's h in the call / 2688; tensor-core path).  act: ACT_NVFP4 (W4A4)
         or ACT_BF16 (weight-only W4A16: bf16 activations, the GEMV path; no scales used).
         shared: None or a BF16 shared expert (w13 bf16 [2I_s, H] interleaved, see
-        shared_expert_w13; w2 bf16 [H, I_s]), added to every token's output."""
+        shared_expert_w13; w2 bf16 [H, I_s]), added to every token's output.  launch: LAUNCH_AUTO,
+        LAUNCH_SINGLE (the whole layer as one persistent launch, where the batch allows it) or
+        LAUNCH_MULTI (prologue, grouped GEMMs, combine)."""
         self.w = experts
         self.top_k = top_k
         self.h_scale = None if h_scale is None else h_scale.to(torch.float32).contiguous()
@@ -357,6 +359,7 @@ class MoeFFN:
         self.combine = combine
         self.act = act
         self.shared = None if shared is None else tuple(t.contiguous() for t in shared)
+        self.launch = launch
         self._ws = {}    # size class (bytes) -> buffer
         self._need = {}  # T -> workspace bytes
 
@@ -374,6 +377,7 @@ class MoeFFN:
         d.h_scale_mode = C.SCALE_DYNAMIC if self.h_scale is None else C.SCALE_GIVEN
         d.h_amax = None if h_amax is None else h_amax.data_ptr()
         d.act_mode = self.act
+        d.launch_mode = self.launch
         if self.shared is not None:
             d.shared_I = self.shared[1].shape[1]
             d.shared_w13, d.shared_w2 = self.shared[0].data_ptr(), self.shared[1].data_ptr()

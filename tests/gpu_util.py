@@ -118,7 +118,7 @@ def experts_from_oracle(wg, wu, wd, dev) -> ops.NVFP4Experts:
 
 
 def run_layer_pair(wl: W.Workload, path: int, seed: int = 0, dev=None, given_x_scale: bool = False,
-                   combine: int = C.COMBINE_AUTO, dynamic_h: bool = False):
+                   combine: int = C.COMBINE_AUTO, dynamic_h: bool = False, launch: int = C.LAUNCH_AUTO):
     """Runs oracle and library on the same inputs; returns (oracle result, gpu out, layer).
     The oracle calibrates s_h (amax of each expert's h / 2688); the library is given those
     scales, or with dynamic_h derives its own in the call."""
@@ -132,7 +132,8 @@ def run_layer_pair(wl: W.Workload, path: int, seed: int = 0, dev=None, given_x_s
     ref = O.moe_ffn(x_bits, logits, wl.k, wg, wu, wd, x_scale=xs)
     experts = experts_from_oracle(wg, wu, wd, dev)
     layer = ops.MoeFFN(experts, wl.k, None if dynamic_h else torch.from_numpy(ref["h_scale"]).to(dev),
-                       x_scale=None if xs is None else torch.tensor([xs], device=dev), path=path, combine=combine)
+                       x_scale=None if xs is None else torch.tensor([xs], device=dev), path=path, combine=combine,
+                       launch=launch)
     h_amax = torch.empty(wl.E, dtype=torch.float32, device=dev)
     out = layer(act["x"].to(dev), act["logits"].to(dev), h_amax=h_amax)
     torch.cuda.synchronize()

@@ -202,7 +202,7 @@ def test_fullsize_calls_with_changing_routing(name):
     wts = W.make_weights(wl, 0, dev)
     experts = ops.NVFP4Experts.from_float(wts["w_gate"], wts["w_up"], wts["w_down"])
     del wts
-    layer = ops.MoeFFN(experts, wl.k, torch.full((wl.E,), 0.01, device=dev))
+    layer = ops.MoeFFN(experts, wl.k, torch.full((wl.E,), 0.01, device=dev), launch=C.LAUNCH_SINGLE)
     assert layer.layout(wl.T).single_launch == 1
     ops.device_status(clear=True)
     first = layer(act["x"], act["logits"]).clone()

@@ -337,7 +337,7 @@ def test_layer_single_launch(name):
     on the same workspace: its counters and tickets start from zero in every call, so the second
     output is the first bit for bit."""
     wl = SINGLE_CASES[name]
-    ref, out, layer, h_amax = G.run_layer_pair(wl, C.PATH_GEMM)
+    ref, out, layer, h_amax = G.run_layer_pair(wl, C.PATH_GEMM, launch=C.LAUNCH_SINGLE)
     assert layer.layout(wl.T).single_launch == 1
     G.check_layer(wl, ref, out, layer, h_amax)
     act = W.make_activations(wl, 0, "cpu")
@@ -347,15 +347,24 @@ def test_layer_single_launch(name):
     assert ops.device_status() == 0
 
 
-def test_single_launch_is_not_taken_where_it_does_not_apply():
-    """17 tokens, the accumulating combine, a dynamic h scale or a shared expert keep the
-    multi-launch path."""
+def test_single_launch_selection():
+    """LAUNCH_SINGLE takes the single launch where the batch allows it and is refused where it
+    does not (17 tokens); the accumulating combine, a dynamic h scale or LAUNCH_MULTI keep the
+    multi-launch path; LAUNCH_AUTO takes the single launch for the dense layer (one expert)."""
     dev = G.need_gpu()
     wl = W.scaled(TINY, T=17)
     _, wts, wg, wu, wd = G.layer_inputs(wl)
     ex = G.experts_from_oracle(wg, wu, wd, dev)
     ones = torch.ones(wl.E, device=dev)
-    assert ops.MoeFFN(ex, wl.k, ones).layout(17).single_launch == 0
-    assert ops.MoeFFN(ex, wl.k, ones).layout(16).single_launch == 1
-    assert ops.MoeFFN(ex, wl.k, ones, combine=C.COMBINE_ACCUMULATE).layout(16).single_launch == 0
-    assert ops.MoeFFN(ex, wl.k, None).layout(16).single_launch == 0
+    single = lambda **kw: ops.MoeFFN(ex, wl.k, kw.pop("h", ones), launch=C.LAUNCH_SINGLE, **kw)  # noqa: E731
+    assert single().layout(16).single_launch == 1
+    assert single().layout(17).single_launch == 0
+    with pytest.raises(C.Nvfp4MoeError):
+        single()(torch.zeros(17, wl.H, dtype=torch.bfloat16, device=dev), torch.zeros(17, wl.E, device=dev))
+    assert single(combine=C.COMBINE_ACCUMULATE).layout(16).single_launch == 0
+    assert single(h=None).layout(16).single_launch == 0
+    assert ops.MoeFFN(ex, wl.k, ones, launch=C.LAUNCH_MULTI).layout(16).single_launch == 0
+    dense = W.scaled(W.WORKLOADS["dense"], T=4, H=256, I=256)
+    _, _, dg, du, dd = G.layer_inputs(dense)
+    dex = G.experts_from_oracle(dg, du, dd, dev)
+    assert ops.MoeFFN(dex, 1, torch.ones(1, device=dev)).layout(4).single_launch == 1
