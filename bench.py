@@ -446,9 +446,11 @@ def measure(wl: W.Workload, args, dev, local: int, rank: int, world: int, dist_o
     on rank 0 of a one-GPU run, the oracle on a bounded sample of it."""
     a16 = args.act == "bf16"
     path = {"auto": C.PATH_AUTO, "gemv": C.PATH_GEMV, "tcgen05": C.PATH_GEMM}[args.path]
-    launch = {"auto": C.LAUNCH_AUTO, "single": C.LAUNCH_SINGLE, "multi": C.LAUNCH_MULTI}[args.launch]
-    if launch == C.LAUNCH_SINGLE and not (wl.T <= 16 and path != C.PATH_GEMV and args.act == "nvfp4"
-                                          and not args.shared_I):
+    launch = {"auto": C.LAUNCH_AUTO, "single": C.LAUNCH_SINGLE, "multi": C.LAUNCH_MULTI,
+              "single_tile": C.LAUNCH_SINGLE_TILE, "single_local": C.LAUNCH_SINGLE_LOCAL}[args.launch]
+    single = launch in (C.LAUNCH_SINGLE, C.LAUNCH_SINGLE_TILE, C.LAUNCH_SINGLE_LOCAL)
+    if single and not (wl.T <= 16 and path != C.PATH_GEMV and args.act == "nvfp4" and not args.shared_I
+                       and (launch != C.LAUNCH_SINGLE_LOCAL or wl.I % 256 == 0)):
         launch = C.LAUNCH_AUTO  # the single launch does not apply to this workload
     act, experts, layer = setup_layer(wl, dev, path=path, launch=launch)
     shared, shared_bits = None, None
@@ -595,8 +597,9 @@ def main():
                     help="activations: nvfp4 (W4A4) or bf16 (the weight-only W4A16 variant, GEMV path)")
     ap.add_argument("--shared-I", type=int, default=0,
                     help="add a BF16 shared expert of this intermediate size (0: none)")
-    ap.add_argument("--launch", default="auto", choices=["auto", "single", "multi"],
-                    help="batches of at most 16 tokens: one persistent launch, the multi-launch path, or automatic")
+    ap.add_argument("--launch", default="auto", choices=["auto", "single", "multi", "single_tile", "single_local"],
+                    help="batches of at most 16 tokens: one persistent launch (its schedule chosen per call, or "
+                         "forced tile-level / expert-local), the multi-launch path, or automatic")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 

@@ -329,18 +329,35 @@ typedef struct {
   const uint16_t* shared_w2;
   /* NVFP4MOE_LAUNCH_*: how a batch that the single-launch layer supports (tensor-core path,
    * at most 16 tokens, ordered combine, given h scales, no shared expert) is run:
-   *   SINGLE  one persistent launch for the whole layer (after a small launch that resets its
-   *           counters): every CTA routes the batch, x stays quantised in shared memory, the
-   *           down tiles of an expert wait on counters of its gate/up tiles, and the combine is
-   *           done by the last writer of each token's rows;
+   *   SINGLE  one persistent, cooperative launch for the whole layer (after a small launch
+   *           that resets its counters): every CTA routes the batch and keeps x quantised in
+   *           shared memory, then runs one of two schedules, chosen per call from the routing
+   *           (every CTA takes the same decision):
+   *             expert-local: units of (active expert, 256 columns of h); a CTA runs a unit's
+   *               gate/up tiles, keeps its h chunk in shared memory and runs the unit's down
+   *               tiles from it.  Taken when I % 256 == 0 and the units fill the grid's rounds
+   *               to at least 80 %;
+   *             tile-level: gate/up and down tiles spread over all CTAs, h through global
+   *               memory, the down tiles of an expert waiting on counters of its gate/up tiles;
+   *           then, after a grid-wide barrier, every CTA sums a slice of the outputs over the
+   *           k x K-chunk slot rows in slot order;
+   *   SINGLE_TILE, SINGLE_LOCAL  SINGLE with that schedule (SINGLE_LOCAL needs I % 256 == 0);
    *   MULTI   the routing/permutation/quantisation prologue, then the grouped GEMMs, then the
    *           combine (the path every larger batch takes);
-   *   AUTO    the faster of the two for the shape (see moe_ffn_workspace_layout's single_launch).
-   * Both give the same routing, permutation and codes, and outputs within the stated tolerance. */
+   *   AUTO    the faster of SINGLE and MULTI for the shape (see moe_ffn_workspace_layout's
+   *           single_launch).
+   * All give the same routing, permutation and codes, and outputs within the stated tolerance
+   * (the schedules differ only in the order of the fp32 sums over K). */
   int32_t launch_mode;
 } moe_ffn_desc;
 
-enum { NVFP4MOE_LAUNCH_AUTO = 0, NVFP4MOE_LAUNCH_SINGLE = 1, NVFP4MOE_LAUNCH_MULTI = 2 };
+enum {
+  NVFP4MOE_LAUNCH_AUTO = 0,
+  NVFP4MOE_LAUNCH_SINGLE = 1,
+  NVFP4MOE_LAUNCH_MULTI = 2,
+  NVFP4MOE_LAUNCH_SINGLE_TILE = 3,
+  NVFP4MOE_LAUNCH_SINGLE_LOCAL = 4
+};
 
 enum { NVFP4MOE_STAGES = 7 };
 
@@ -359,7 +376,8 @@ typedef struct {
   int32_t single_launch; /* 1: the whole layer runs as one persistent launch (batches of at most
                             16 tokens on the GEMM path, ordered combine, given h scales, no
                             shared expert); `items` then holds its counters, `slots` its fp32
-                            rows by (pair, K chunk of at most 2048) */
+                            rows by (pair, K chunk): chunks of 256 under the expert-local
+                            schedule, of at most 2048 under the tile-level one */
   int64_t h_f32;    /* dynamic h scale: fp32 h [h_rows][I] before requantisation */
   int64_t h_stats;  /* dynamic h scale: amax[E] then the scales used, s_h[E] (fp32) */
   int64_t h_bf16;   /* weight-only layer: h in bf16 [T*k][I], permuted rows (x_codes, x_sf,

@@ -17,7 +17,7 @@ DTYPE_BF16, DTYPE_F32 = 0, 1
 PATH_AUTO, PATH_GEMV, PATH_GEMM = 0, 1, 2
 COMBINE_AUTO, COMBINE_ORDERED, COMBINE_ACCUMULATE = 0, 1, 2
 ACT_NVFP4, ACT_BF16 = 0, 1
-LAUNCH_AUTO, LAUNCH_SINGLE, LAUNCH_MULTI = 0, 1, 2
+LAUNCH_AUTO, LAUNCH_SINGLE, LAUNCH_MULTI, LAUNCH_SINGLE_TILE, LAUNCH_SINGLE_LOCAL = 0, 1, 2, 3, 4
 STAGES = 7
 STAGE_NAMES = ("route", "permute", "quantize_x", "gate_up", "down", "combine")
 DEV_BAD_EXPERT_ID, DEV_DUPLICATE_ID, DEV_ROW_OVERFLOW, DEV_TIMEOUT, DEV_BAD_GATHER = 1, 2, 4, 8, 16

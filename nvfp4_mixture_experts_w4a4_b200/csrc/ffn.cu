@@ -39,7 +39,7 @@ nvfp4moe_status check_desc(const moe_ffn_desc* d, const char* fn) {
                 "%s: the weight-only layer runs the GEMV path", fn);
   NVFP4_REQUIRE(d->shared_I >= 0 && d->shared_I % 64 == 0, NVFP4MOE_UNSUPPORTED_SHAPE,
                 "%s: shared_I=%d must be a multiple of 64", fn, d->shared_I);
-  NVFP4_REQUIRE(d->launch_mode >= NVFP4MOE_LAUNCH_AUTO && d->launch_mode <= NVFP4MOE_LAUNCH_MULTI,
+  NVFP4_REQUIRE(d->launch_mode >= NVFP4MOE_LAUNCH_AUTO && d->launch_mode <= NVFP4MOE_LAUNCH_SINGLE_LOCAL,
                 NVFP4MOE_INVALID_ARG, "%s: bad launch_mode %d", fn, d->launch_mode);
   return NVFP4MOE_OK;
 }
@@ -62,16 +62,24 @@ int resolve_path(const moe_ffn_desc* d) {
 bool single_launch_fits(const moe_ffn_desc* d, int path) {
   return path == NVFP4MOE_PATH_GEMM && d->act_mode == NVFP4MOE_ACT_NVFP4 && d->h_scale_mode == NVFP4MOE_SCALE_GIVEN &&
          d->shared_I == 0 && d->combine != NVFP4MOE_COMBINE_ACCUMULATE &&
-         layer_fused_fits(d->T, d->H, d->I, d->E, d->top_k);
+         layer_fused_fits(d->T, d->H, d->I, d->E, d->top_k) &&
+         (d->launch_mode != NVFP4MOE_LAUNCH_SINGLE_LOCAL || layer_fused_local_fits(d->I));
+}
+
+bool single_launch_requested(const moe_ffn_desc* d) {
+  return d->launch_mode == NVFP4MOE_LAUNCH_SINGLE || d->launch_mode == NVFP4MOE_LAUNCH_SINGLE_TILE ||
+         d->launch_mode == NVFP4MOE_LAUNCH_SINGLE_LOCAL;
 }
 
 // Whether this call runs as one launch.  AUTO takes it where it measured faster than the
-// multi-launch path: the dense layer (one expert), whose down tiles then split along K.  For
-// routed batches the multi-launch path is faster: there the single launch's gate/up -> down
-// counters and per-tile tickets cost more than the launches they save.
+// multi-launch path: the dense layer (one expert), and routed batches whose expected active
+// experts (uniform routing) fill the grid with expert-local units.  Where routing turns out
+// too skewed for those, the launch falls back to its tile-level schedule, which is correct
+// but measured slower than the multi-launch path on routed batches.
 bool single_launch(const moe_ffn_desc* d, int path) {
   if (d->launch_mode == NVFP4MOE_LAUNCH_MULTI || !single_launch_fits(d, path)) return false;
-  return d->launch_mode == NVFP4MOE_LAUNCH_SINGLE || d->E == 1;
+  return single_launch_requested(d) || d->E == 1 ||
+         layer_fused_local_likely(d->T, d->H, d->I, d->E, d->top_k);
 }
 
 // AUTO: the ordered combine (faster than accumulation at the routed benchmark sizes once the
@@ -149,8 +157,8 @@ void make_layout(const moe_ffn_desc* d, moe_ffn_ws_layout* L) {
                                       prologue_scratch));
   // the fused GEMM's work list and per-expert counters, written by the small-batch prologue
   const int64_t A = P < E ? P : E;
-  if (L->single_launch)  // per (active expert, K chunk) counters, then per (token, 32 columns) tickets
-    L->items = take((A * layer_fused_chunks(d->I) + T * (H / 32)) * 4);
+  if (L->single_launch)  // per (active expert, K chunk) counters, then the combine barrier
+    L->items = take((A * layer_fused_chunks(d->I) + 1) * 4);
   else
     L->items = take(path == NVFP4MOE_PATH_GEMM && prologue_fits(d->T, d->E, d->top_k)
                         ? grouped_fused_list_entries(A, 2 * I / 128, H / 128) * 16 + E * 4
@@ -211,9 +219,9 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
     NVFP4_REQUIRE(d->E <= 1024, NVFP4MOE_UNSUPPORTED_SHAPE, "%s: E > 1024", fn);
     NVFP4_REQUIRE(gemm_path_available(), NVFP4MOE_CUDA_ERROR, "%s: the tensor-core path is unavailable", fn);
   }
-  NVFP4_REQUIRE(d->launch_mode != NVFP4MOE_LAUNCH_SINGLE || L.single_launch, NVFP4MOE_UNSUPPORTED_SHAPE,
+  NVFP4_REQUIRE(!single_launch_requested(d) || L.single_launch, NVFP4MOE_UNSUPPORTED_SHAPE,
                 "%s: the single launch takes at most 16 tokens on the tensor-core path with the ordered combine, "
-                "given h scales and no shared expert", fn);
+                "given h scales and no shared expert (and I %% 256 == 0 for the expert-local schedule)", fn);
   NVFP4_REQUIRE(L.combine != NVFP4MOE_COMBINE_ACCUMULATE || L.path == NVFP4MOE_PATH_GEMM, NVFP4MOE_UNSUPPORTED_SHAPE,
                 "%s: the accumulating combine needs the tensor-core path", fn);
   const bool dyn_h = !a16 && d->h_scale_mode == NVFP4MOE_SCALE_DYNAMIC;
@@ -296,8 +304,11 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
     f.rows_cap = rows_cap;
     f.slots = F32(L.slots);
     f.done = I32(L.items);
-    f.tickets = I32(L.items) + max_active_experts(d) * layer_fused_chunks(I);
+    f.gbar = I32(L.items) + max_active_experts(d) * layer_fused_chunks(I);
     f.out = out;
+    f.schedule = d->launch_mode == NVFP4MOE_LAUNCH_SINGLE_TILE    ? 1
+                 : d->launch_mode == NVFP4MOE_LAUNCH_SINGLE_LOCAL ? 2
+                                                                  : 0;
     st = launch_layer_fused_reset(f, s);
     if (st != NVFP4MOE_OK) return st;
     mark(1);

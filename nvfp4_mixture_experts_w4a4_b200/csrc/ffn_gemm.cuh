@@ -88,13 +88,17 @@ struct LayerFusedArgs {
   int64_t rows_cap;
   float* slots;   // [T*k*layer_fused_chunks(I)][H] fp32
   int* done;      // [min(T*k, E) * layer_fused_chunks(I)]
-  int* tickets;   // [T][H/32]
+  int* gbar;      // [1] the combine barrier
+  int schedule;   // 0: chosen per call from the routing; 1: tile-level; 2: expert-local
   void* out;
 };
 bool layer_fused_fits(int T, int H, int I, int E, int k);
 int layer_fused_chunks(int I);
-// the reset launch (counters, tickets, h maxima to zero), then the layer launch, its
-// programmatic dependent; nothing else may run on the stream between the two
+bool layer_fused_local_fits(int I);  // the expert-local schedule applies (I % 256 == 0)
+// the expert-local schedule would be taken for uniformly random routing of this shape
+bool layer_fused_local_likely(int T, int H, int I, int E, int k);
+// the reset launch (counters, barrier, h maxima to zero), then the layer launch (cooperative),
+// its programmatic dependent; nothing else may run on the stream between the two
 nvfp4moe_status launch_layer_fused_reset(const LayerFusedArgs& f, cudaStream_t s);
 nvfp4moe_status launch_layer_fused(const LayerFusedArgs& f, cudaStream_t s);
 

@@ -18,18 +18,29 @@
 //    token tile.  Each output column depends only on its own token, so the columns of the
 //    tokens an expert did not receive are simply not used; the extra MMA work is free at
 //    this size, and no token tile is loaded per item.
-//  * Items: gate/up tiles (expert, 128 rows of W13 = 64 columns of h) and down tiles
-//    (expert, K chunk of at most 2048, 128 rows of W2).  A down tile's h rows are the
-//    requantised outputs of the gate/up tiles of its expert and K chunk, written to global
-//    memory (L2) by whichever CTAs ran them; per-(expert, chunk) counters order the two
-//    (release: fence + atomic add; acquire: a load, then the proxy fence before TMA reads h).
-//    The weight tiles themselves never wait: the producer streams W2 while h is finishing.
+//  * Two schedules of the weight tiles, chosen per call from the routing (every CTA takes the
+//    same decision):
+//    - expert-local: units of (active expert, 256 columns of h), round-robin over the CTAs.
+//      A CTA runs a unit's four gate/up tiles (W13 rows of those columns), requantises the h
+//      chunk into shared memory (K-major, 128-byte swizzle: the down MMA's B operand, 16 token
+//      rows) and runs the unit's down tiles (all H rows of W2, K = the chunk) from it.  No h
+//      crosses CTAs, so nothing waits on another CTA until the combine; the next unit's
+//      gate/up tiles are issued before this unit's down tiles, so the MMA has work while the
+//      epilogue requantises, and two h buffers alternate.  Taken when I % 256 == 0 and the
+//      units fill the grid's rounds to at least 80 %.
+//    - tile-level: gate/up tiles (expert, 128 rows of W13 = 64 columns of h) and down tiles
+//      (expert, K chunk of at most 2048, 128 rows of W2) spread over all CTAs.  A down tile's
+//      h rows are the requantised outputs of the gate/up tiles of its expert and K chunk,
+//      written to global memory (L2) by whichever CTAs ran them; per-(expert, chunk)
+//      counters order the two (release: fence + atomic add; acquire: a load, then the proxy
+//      fence before TMA reads h).  The weight tiles themselves never wait: the producer
+//      streams W2 while h is finishing.
 //  * Combine: the down epilogue writes each routed pair's weighted fp32 rows (one row per K
-//    chunk) and takes a ticket per (token, 32 output columns); the warp that takes the last
-//    ticket sums that token's k x chunks rows in slot order and rounds once to bf16.  No
-//    combine launch and no waiting: the last writer does the sum.
+//    chunk) to its slots.  After a grid-wide barrier (one release per CTA; the launch is
+//    cooperative, so all CTAs are resident) every CTA sums a slice of the [T][H] outputs over
+//    the token's k x chunks rows in slot order and rounds once to bf16.
 //
-// A small launch before this one zeroes the counters and tickets; this kernel is its
+// A small launch before this one zeroes the counters and the barrier; this kernel is its
 // programmatic dependent and waits for it only before touching them (well after its start).
 //
 // Warp roles after the routing phase (all 16 warps route, one token each, and quantise x):
@@ -39,10 +50,13 @@
 //               MMAs (kind::mxf4nvf4, M = 128, N = 16) per stage into one of 8 accumulators;
 //   warps 2..9  epilogue: four warps (one per 32-lane TMEM quarter) per item, the two sets of
 //               four taking alternate items;
-//   warp 10     h producer: for down tiles, acquires the expert's chunk counter and loads
-//               the h rows and their scale atoms into the stage the weight producer armed;
+//   warp 10     h producer (tile-level schedule): for down tiles, acquires the expert's chunk
+//               counter and loads the h rows and their scale atoms into the stage the weight
+//               producer armed;
 //   warps 11-15 routing, x quantisation and the inspection copies only.
 // Every wait is bounded (status bit on timeout; copies in flight land before the CTA exits).
+#include <cmath>
+
 #include "ffn_gemm.cuh"
 #include "tcgen05.cuh"
 #include "tma.cuh"
@@ -65,6 +79,8 @@ constexpr int TOK_ALIGN = 64;           // padded rows per active expert (h and 
 constexpr int EPI_FIRST = 2, EPI_WARPS = 8, HPROD_WARP = 10;  // warps 11..15: set-up only
 constexpr int NACC = 8;                 // TMEM accumulators (items in flight past the MMA)
 constexpr int KC_MAX = 2048;            // K chunk of a down item
+constexpr int KCL = BK;                 // narrowest h chunk of an expert-local unit (one down k-tile)
+constexpr int KCL_MAX = 4 * KCL;        // widest
 constexpr int A_BYTES = WM * KB;        // 16 KB
 constexpr int B_BYTES = LF_MAXT * KB;   // 2 KB: a 16-row h tile
 constexpr int SFA_BYTES = 4 * 512;      // 4 scale atoms (one per 64 elements of K)
@@ -78,10 +94,38 @@ constexpr uint32_t ACC_COL = 0;
 constexpr uint32_t SFA_COL = NACC * LF_MAXT;  // 128
 constexpr uint32_t SFB_COL = SFA_COL + 16;
 constexpr uint32_t XSF_COL = SFB_COL + 16;    // x scales: H/32 columns (two 64-element steps per 4)
+                                              // then the two local h chunks' scales, 8 columns each
 constexpr uint32_t kDevTimeout = NVFP4MOE_DEV_TIMEOUT;
 constexpr int SMEM_LIMIT = 232448;
 
 __host__ __device__ inline int lf_kc(int I) { return I < KC_MAX ? I : KC_MAX; }
+
+// TMEM columns: accumulators, weight and h scales, x scales, then the local h chunks' scales
+// (two buffers, kcl / 32 columns each) for chunks of at most kcl columns.
+__host__ __device__ inline uint32_t lf_tmem_need(int H, int kcl = KCL) { return XSF_COL + uint32_t(H / 32 + kcl / 16); }
+
+// The expert-local schedule: unit = (active expert, kcl columns of h).  One CTA runs a unit's
+// kcl / 64 gate/up tiles, keeps the requantised h chunk in shared memory and runs the unit's
+// down tiles (all H rows of W2, K = the chunk) from it, so no h crosses CTAs and nothing waits
+// for another CTA until the combine.  Every unit is the same amount of weight bytes, so units
+// go round-robin.  The chunk width kcl is the widest of 1024, 512, 256 that divides I, fits the
+// h buffers (two in the stage ring's B region, whose `stages` 2 KB slots hold kcl / 128) and
+// TMEM, and whose units fill the grid's rounds to at least 80 %.  Wider is better where it
+// balances: a W2 row whose chunks go to different CTAs is read piecewise at different times,
+// and the down stream then runs at about half the rate.  Forced (schedule 2): the widest
+// balanced width, else 256; schedule 1 forces the tile-level schedule.  Returns kcl, or 0 when
+// the schedule is not taken.
+__host__ __device__ inline int lf_local_width(int A, int I, int G, int schedule, int H, int stages) {
+  if (schedule == 1 || A < 1) return 0;
+  int fallback = 0;
+  for (int kcl = KCL_MAX; kcl >= KCL; kcl >>= 1) {
+    if (I % kcl != 0 || I / kcl > 63 || kcl / 128 > stages || lf_tmem_need(H, kcl) > 512u) continue;
+    const int64_t U = int64_t(A) * (I / kcl), rounds = (U + G - 1) / G;
+    if (rounds * G * 4 <= U * 5) return kcl;
+    if (kcl == KCL) fallback = kcl;
+  }
+  return schedule == 2 ? fallback : 0;
+}
 
 // Shapes that size the shared-memory layout: E experts, P = T*k pairs, at most AM active experts,
 // at most IC work items per CTA, `stages` weight stages.
@@ -118,7 +162,7 @@ __host__ __device__ inline Layout lf_layout(const LfShape& f) {
   L.wsum = L.red + 32 * 4;
   L.item = L.wsum + 32 * 4;                  // this CTA's work list [IC]
   L.bars = (L.item + f.IC * 4 + HQ * 8 + 7) / 8 * 8;  // the work list, then the handoff ring [HQ][2]
-  L.total = L.bars + (2 * MAX_STAGES + 2 * NACC + 1 + 2 * HQ) * 8 + 16;
+  L.total = L.bars + (2 * MAX_STAGES + 2 * NACC + 1 + 2 * HQ + 3) * 8 + 16;
   return L;
 }
 
@@ -132,6 +176,12 @@ __host__ inline LfShape lf_shape(int T, int H, int I, int E, int k, int grid) {
   const int nkc = (I + lf_kc(I) - 1) / lf_kc(I);
   const int64_t items = int64_t(f.AM) * (2 * I / WM + int64_t(nkc) * (H / WM));
   f.IC = int((items + grid - 1) / grid);
+  for (int kcl = KCL; kcl <= KCL_MAX; kcl <<= 1) {  // the expert-local schedule, at most AM active experts
+    if (I % kcl != 0) continue;
+    const int64_t rounds = (int64_t(f.AM) * (I / kcl) + grid - 1) / grid;
+    const int64_t ic = rounds * (kcl / 64 + H / WM);
+    if (ic > f.IC) f.IC = int(ic);
+  }
   f.stages = 0;
   for (int st = MAX_STAGES; st >= MIN_STAGES; --st) {
     f.stages = st;
@@ -141,10 +191,10 @@ __host__ inline LfShape lf_shape(int T, int H, int I, int E, int k, int grid) {
   return f;
 }
 
-// Work item packing: phase (bit 0), K chunk (bits 1..6), weight tile (bits 7..19), active
-// expert slot (bits 20..31).
-__device__ __forceinline__ uint32_t lf_pack(int ph, int kc, int mt, int a) {
-  return uint32_t(ph) | (uint32_t(kc) << 1) | (uint32_t(mt) << 7) | (uint32_t(a) << 20);
+// Work item packing: phase (bit 0), h buffer of an expert-local unit (bit 1), K chunk (bits
+// 2..7), weight tile (bits 8..20), active expert slot (bits 21..31).
+__device__ __forceinline__ uint32_t lf_pack(int ph, int buf, int kc, int mt, int a) {
+  return uint32_t(ph) | (uint32_t(buf) << 1) | (uint32_t(kc) << 2) | (uint32_t(mt) << 8) | (uint32_t(a) << 21);
 }
 
 struct LayerArgs {
@@ -168,24 +218,27 @@ struct LayerArgs {
   uint8_t* x_sf;            // MMA layout over the padded rows
   uint8_t* h_codes;         // [rows][I/2], padded expert order
   uint8_t* h_sf;
-  float* slots;             // [T*k*nkc][H]: weighted fp32 rows by (pair, K chunk)
+  float* slots;             // [T*k*nkc][H]: weighted fp32 rows by (pair, K chunk); nkc of the schedule
+                            // taken, at most layer_fused_chunks(I)
   int* done;                // [min(P, E) * nkc] gate/up tiles finished per (active expert, chunk)
-  int* tickets;             // [T][H/32]
+  int* gbar;                // [1] CTAs arrived at the combine barrier
+  int schedule;             // 0: chosen from the routing; 1: tile-level; 2: expert-local
   __nv_bfloat16* out;       // [T][H]
   LfShape shape;
   uint32_t* status;
 };
 
 struct LItem {
-  int ph, a, mt, kc;
+  int ph, buf, a, mt, kc;
 };
 
 __device__ __forceinline__ LItem lf_unpack(uint32_t v) {
   LItem it;
   it.ph = int(v & 1u);
-  it.kc = int((v >> 1) & 63u);
-  it.mt = int((v >> 7) & 8191u);
-  it.a = int(v >> 20);
+  it.buf = int((v >> 1) & 1u);
+  it.kc = int((v >> 2) & 63u);
+  it.mt = int((v >> 8) & 8191u);
+  it.a = int(v >> 21);
   return it;
 }
 
@@ -193,12 +246,14 @@ __device__ __forceinline__ LItem lf_item(int idx, int ng, int wt_g, int wt_d, in
   LItem it;
   if (idx < ng) {
     it.ph = 0;
+    it.buf = 0;
     it.a = idx / wt_g;
     it.mt = idx - it.a * wt_g;
     it.kc = 0;
   } else {
     const int d = idx - ng, per = nkc * wt_d;
     it.ph = 1;
+    it.buf = 0;
     it.a = d / per;
     const int r = d - it.a * per;
     it.kc = r / wt_d;
@@ -223,12 +278,6 @@ __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_re
 __device__ __forceinline__ void red_release_add1(int* p) {
   asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(p) : "memory");
 }
-// +1 with acquire-release semantics at GPU scope; returns the previous count.
-__device__ __forceinline__ int atom_acq_rel_add1(int* p) {
-  int old;
-  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
-  return old;
-}
 __device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
@@ -251,11 +300,12 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
 // silu(g) * u with the fast exponential and division (h is requantised to E2M1 right after)
 __device__ __forceinline__ float lf_silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
-// Counters and tickets of one call back to zero, and the h maxima when they are requested.
-__global__ void layer_reset_kernel(int* done, int n_done, int* tickets, int n_tickets, float* h_amax, int E) {
+// Counters and the combine barrier of one call back to zero, and the h maxima when they are
+// requested.
+__global__ void layer_reset_kernel(int* done, int n_done, int* gbar, float* h_amax, int E) {
   griddep_launch_dependents();
   for (int i = threadIdx.x; i < n_done; i += blockDim.x) done[i] = 0;
-  for (int i = threadIdx.x; i < n_tickets; i += blockDim.x) tickets[i] = 0;
+  if (threadIdx.x == 0) *gbar = 0;
   if (h_amax)
     for (int i = threadIdx.x; i < E; i += blockDim.x) h_amax[i] = 0.0f;
 }
@@ -296,8 +346,10 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
   uint64_t* drain = acc_empty + NACC;
   uint64_t* hq_full = drain + 1;    // [HQ] a down stage was armed: its h loads may be issued
   uint64_t* hq_empty = hq_full + HQ;  // [HQ] the h producer took the entry
+  uint64_t* h_ready = hq_empty + HQ;  // [2] local schedule: a unit's h chunk is in shared memory
   uint32_t* s_hq = s_item + a.shape.IC;  // [HQ][2] entries: stage use (ring index); item | k-tile << 16
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(hq_empty + HQ);
+  uint64_t* x_full = h_ready + 2;     // x staged in the (still idle) weight stage ring
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(x_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -305,27 +357,45 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
   const int KC = lf_kc(I), nkc = (I + KC - 1) / KC;
   const int wt_g = 2 * I / WM, wt_d = H / WM;
 
+  // The router logits of this warp's token (T <= 16 warps) are requested first, so that their
+  // latency passes during the set-up.
+  float lg[PER_LANE];
+#pragma unroll
+  for (int i = 0; i < PER_LANE; ++i) {
+    const int e = lane + 32 * i;
+    lg[i] = warp < T && e < E ? __ldg(a.logits + int64_t(warp) * E + e) : 0.0f;
+  }
+
   // ---------------------------------------------------------------- set-up ----
-  if (tid == 0) {
-    for (int s = 0; s < S; ++s) {
+  if (warp == 0) {  // barrier initialisation, spread over the lanes
+    for (int s = lane; s < S; s += 32) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < NACC; ++b) {
-      mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4 * 32);  // the four epilogue warps of an item
+    if (lane < NACC) {
+      mbar_init(&acc_full[lane], 1);
+      mbar_init(&acc_empty[lane], 4 * 32);  // the four epilogue warps of an item
     }
-    mbar_init(drain, 1);
-    for (int q = 0; q < HQ; ++q) {
+    for (int q = lane; q < HQ; q += 32) {
       mbar_init(&hq_full[q], 1);
       mbar_init(&hq_empty[q], 1);
     }
-    *abort_flag = 0;
+    if (lane == 0) {
+      mbar_init(drain, 1);
+      mbar_init(x_full, 1);
+      *abort_flag = 0;
+    }
     mbar_fence_init();
+    // x (bf16, T*H*2 bytes) into the stage ring, which no weight tile uses before the routing
+    // is done: one bulk copy, so that the maximum and the quantisation below read shared memory
+    if (lane == 0 && int64_t(T) * H * 2 <= int64_t(S) * A_BYTES) {
+      mbar_arrive_expect_tx(x_full, uint32_t(T * H * 2));
+      bulk_load(sA, a.x, uint32_t(T * H * 2), x_full);
+    }
   }
   if (warp == 1) {
-    // columns: 8 accumulators x 16, the weight and h scales, then the x scales
-    const uint32_t need = XSF_COL + uint32_t(H / 32);
+    // columns: 8 accumulators x 16, the weight and h scales, the x scales, the local h scales
+    const uint32_t need = lf_tmem_need(H, KCL_MAX);
     tmem_alloc(tmem_holder, need <= 256 ? 256u : 512u);
     tmem_relinquish();
     tc_fence_before();
@@ -347,42 +417,87 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
   for (int e = tid; e < E; e += LF_THREADS) s_mask[e] = 0u;
 
   // ------------------------------------------------- routing, the x maximum ----
-  // The first NXR 16-byte chunks of x per thread are requested before the top-k, so that the
-  // x loads and the logit loads are in flight together; the maximum is taken after it.
-  constexpr int NXR = 12;
-  const int64_t chunks = a.dynamic ? int64_t(T) * H / 8 : 0;  // 16-byte chunks of x
-  const uint4* xb = reinterpret_cast<const uint4*>(a.x);
-  uint4 xr[NXR];
-#pragma unroll
-  for (int j = 0; j < NXR; ++j) {
-    const int64_t i = tid + int64_t(j) * LF_THREADS;
-    xr[j] = i < chunks ? __ldg(xb + i) : make_uint4(0u, 0u, 0u, 0u);
+  // x is staged in shared memory when it fits in the stage ring (decode sizes); else it is read
+  // from global memory, and quantised by the epilogue warps once the weight stream has started.
+  const bool xstage = int64_t(T) * H * 2 <= int64_t(S) * A_BYTES;
+  if (xstage) {  // the resident token tile and its scale staging start at zero (absent tokens, pad bytes)
+    for (int i = tid; i < ktiles * B_BYTES / 16; i += LF_THREADS)
+      reinterpret_cast<uint4*>(sX)[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = tid; i < (H / 128) * 32; i += LF_THREADS)
+      reinterpret_cast<uint4*>(sXSF)[i] = make_uint4(0u, 0u, 0u, 0u);
   }
   __syncthreads();  // the masks are zero before any routing lane marks them
-  for (int t = warp; t < T; t += LF_WARPS) {
+  if (warp < T) {
+    const int t = warp;
     int id = 0;
     float wv = 0.0f;
-    warp_topk<PER_LANE>(a.logits + int64_t(t) * E, E, k, &id, &wv);
+    warp_topk_regs<PER_LANE>(lg, E, k, &id, &wv);
     if (lane < k) {
       s_ids[t * k + lane] = id;
       s_w[t * k + lane] = wv;
       atomicOr(&s_mask[id], 1u << t);
     }
   }
-  float m = 0.0f;
-  auto amax8 = [&](const uint4& u) {
-    const uint32_t q[4] = {u.x, u.y, u.z, u.w};
+  const uint4* xs = reinterpret_cast<const uint4*>(sA);  // the staged x, 16-byte chunks
+  if (xstage && !mbar_wait(x_full, 0)) atomicOr(a.status, kDevTimeout);  // the copy never landed
+  if (a.dynamic) {
+    // the tensor scale: amax over all of x (one-shot code, so the loops stay rolled)
+    float m = 0.0f;
+    const int64_t chunks = int64_t(T) * H / 8;
+    const uint4* xb = reinterpret_cast<const uint4*>(a.x);
+#pragma unroll 1
+    for (int64_t i = tid; i < chunks; i += LF_THREADS) {
+      const uint4 u = xstage ? xs[i] : __ldg(xb + i);
+      const uint32_t q[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-    for (int h = 0; h < 4; ++h)
-      m = fmaxf(m, fmaxf(fabsf(__uint_as_float(q[h] << 16)), fabsf(__uint_as_float(q[h] & 0xFFFF0000u))));
-  };
+      for (int h = 0; h < 4; ++h)
+        m = fmaxf(m, fmaxf(fabsf(__uint_as_float(q[h] << 16)), fabsf(__uint_as_float(q[h] & 0xFFFF0000u))));
+    }
 #pragma unroll
-  for (int j = 0; j < NXR; ++j) amax8(xr[j]);
-  for (int64_t i = tid + int64_t(NXR) * LF_THREADS; i < chunks; i += LF_THREADS) amax8(__ldg(xb + i));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if (lane == 0) s_red[warp] = m;
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) s_red[warp] = m;
+  }
   __syncthreads();
+
+  float s_t;
+  if (a.dynamic) {
+    float mx = 0.0f;
+    for (int i = 0; i < LF_WARPS; ++i) mx = fmaxf(mx, s_red[i]);
+    s_t = __fdiv_rn(mx, 2688.0f);
+  } else {
+    s_t = *a.x_scale;
+  }
+  if (xstage) {
+    // x into the resident token tile: unit = one 16-element block (token t, block b) of the
+    // staged rows; codes into t's row of k-tile b / 16 (128-byte swizzle), the scale byte into
+    // the staging of the x scales (512-byte block b / 8, row t at t * 16, step (b / 4) % 2 at
+    // byte 8 of it)
+    const int bpr = H / 16;
+#pragma unroll 1
+    for (int u = tid; u < T * bpr; u += LF_THREADS) {
+      const int t = u / bpr, b = u - t * bpr;
+      const uint4 u0 = xs[2 * u], u1 = xs[2 * u + 1];
+      const uint32_t q[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+      float v[16];
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        v[2 * h] = __uint_as_float(q[h] << 16);
+        v[2 * h + 1] = __uint_as_float(q[h] & 0xFFFF0000u);
+      }
+      float am = 0.0f;
+#pragma unroll
+      for (int h = 0; h < 16; ++h) am = fmaxf(am, fabsf(v[h]));
+      float inv;
+      const uint32_t sf = block_scale(am, s_t, &inv);
+      const int bi = b & 15;
+      *reinterpret_cast<uint2*>(sX + (b >> 4) * B_BYTES + t * KB + ((((bi >> 1) ^ (t & 7)) << 4) | ((bi & 1) << 3))) =
+          encode_block16(v, inv);
+      sXSF[(b >> 3) * 512 + t * 16 + ((b >> 2) & 1) * 8 + (b & 3)] = static_cast<uint8_t>(sf);
+    }
+    // generic stores read by the tensor core, and generic reads of the ring before the weight
+    // tiles land in it: both ordered by this fence and the barriers below
+    fence_proxy_async_shared();
+  }
 
   // active experts in ascending order, their token masks, compact pair offsets: thread
   // t < 256 owns experts 4t .. 4t+3; one block scan of (pairs | active << 16)
@@ -430,17 +545,52 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
   }
   __syncthreads();
 
-  // work list: gate/up items (slot, tile), then down items (slot, chunk, tile); item idx of
-  // this CTA: blockIdx.x + j * gridDim.x, decoded once here by all threads into shared memory
-  const int ng = A * wt_g, ntot = ng + A * nkc * wt_d;
+  // this CTA's work list, decoded once here by all threads into shared memory
   const int G = int(gridDim.x);
-  const int n_my = int(blockIdx.x) < ntot ? (ntot - int(blockIdx.x) + G - 1) / G : 0;
-  for (int j = tid; j < n_my; j += LF_THREADS) {
-    const LItem u = lf_item(int(blockIdx.x) + j * G, ng, wt_g, wt_d, nkc);
-    s_item[j] = lf_pack(u.ph, u.kc, u.mt, u.a);
+  const int kcl = lf_local_width(A, I, G, a.schedule, H, S);  // every CTA takes the same decision
+  const bool local = kcl > 0;
+  const int GU = kcl / 64;                                   // gate/up tiles per local unit
+  const int U = local ? A * (I / kcl) : 0;
+  const int KCx = local ? kcl : KC, nkc_x = local ? I / kcl : nkc;  // K chunk of down items, chunks
+  if (local && tid == 0) {  // used only after the barrier below
+    mbar_init(&h_ready[0], 4 * GU);  // the four epilogue warps of each gate/up tile of a unit
+    mbar_init(&h_ready[1], 4 * GU);
+  }
+  const int n_u = local && int(blockIdx.x) < U ? (U - int(blockIdx.x) + G - 1) / G : 0;
+  int n_my;
+  if (local) {
+    // units b, b + G, ... of this CTA: unit n's gate/up tiles, then, after unit n + 1's gate/up
+    // tiles (MMA work while the epilogue requantises unit n's h), unit n's down tiles
+    const int per = GU + wt_d;
+    n_my = n_u * per;
+    for (int j = tid; j < n_my; j += LF_THREADS) {
+      int n, r;
+      bool gu;
+      if (j < GU) {
+        n = 0;
+        gu = true;
+        r = j;
+      } else {
+        const int jj = j - GU, blk = jj / per, rr = jj - blk * per;
+        gu = blk < n_u - 1 && rr < GU;
+        n = gu ? blk + 1 : blk;
+        r = gu || blk == n_u - 1 ? rr : rr - GU;
+      }
+      const int ug = int(blockIdx.x) + n * G, sl = ug / nkc_x, c = ug - sl * nkc_x;
+      s_item[j] = gu ? lf_pack(0, n & 1, c, GU * c + r, sl) : lf_pack(1, n & 1, c, r, sl);
+    }
+  } else {
+    // gate/up items (slot, tile), then down items (slot, chunk, tile); item idx of this CTA:
+    // blockIdx.x + j * gridDim.x
+    const int ng = A * wt_g, ntot = ng + A * nkc * wt_d;
+    n_my = int(blockIdx.x) < ntot ? (ntot - int(blockIdx.x) + G - 1) / G : 0;
+    for (int j = tid; j < n_my; j += LF_THREADS) {
+      const LItem u = lf_item(int(blockIdx.x) + j * G, ng, wt_g, wt_d, nkc);
+      s_item[j] = lf_pack(u.ph, 0, u.kc, u.mt, u.a);
+    }
   }
   // K of a down item's chunk; its last k-tile may hold 2 of the 4 64-element steps (I % 128 == 0)
-  auto kc_len = [&](int c) { return min(KC, I - c * KC); };
+  auto kc_len = [&](int c) { return local ? kcl : min(KC, I - c * KC); };
   auto ktiles_of = [&](const LItem& w) { return w.ph == 0 ? ktiles : (kc_len(w.kc) + BK - 1) / BK; };
   auto steps_of = [&](const LItem& w, int kt) { return w.ph == 0 ? 4 : min(4, (kc_len(w.kc) - kt * BK) / 64); };
   // gate/up tiles whose h columns fall in chunk c, times the four epilogue warps of an item
@@ -450,14 +600,6 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
     atomicOr(a.status, kDevTimeout);
   };
 
-  float s_t;
-  if (a.dynamic) {
-    float mx = 0.0f;
-    for (int i = 0; i < LF_WARPS; ++i) mx = fmaxf(mx, s_red[i]);
-    s_t = __fdiv_rn(mx, 2688.0f);
-  } else {
-    s_t = *a.x_scale;
-  }
   // per active expert: the gate/up product scales (x scale times the weight scales), the
   // requantisation scale of h, and the down product's scale
   for (int sl = tid; sl < A; sl += LF_THREADS) {
@@ -492,15 +634,17 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
         } else {
           map = &tmW2;
           row = int64_t(e) * H + w.mt * WM;
-          x0 = w.kc * KC / 2;
-          sf = a.w2_sf + int64_t(e) * H * (I / 16) + (int64_t(w.mt) * (I / 64) + w.kc * (KC / 64)) * 512;
+          x0 = w.kc * KCx / 2;
+          sf = a.w2_sf + int64_t(e) * H * (I / 16) + (int64_t(w.mt) * (I / 64) + w.kc * (KCx / 64)) * 512;
         }
         for (int kt = 0; kt < kt_n; ++kt, ++it) {
           const int s = int(it % uint32_t(S));
           // a partial k-tile still lands a whole box (zero fill past the row); its scales are
-          // the atoms that exist.  Down stages also carry the h tile and its atoms.
+          // the atoms that exist.  Down stages of the tile-level schedule also carry the h tile
+          // and its atoms (the local schedule's h is resident).
+          const bool with_h = w.ph == 1 && !local;
           const uint32_t sfb = uint32_t(steps_of(w, kt)) * 512;
-          const uint32_t bytes = A_BYTES + sfb + (w.ph == 1 ? B_BYTES + sfb : 0u);
+          const uint32_t bytes = A_BYTES + sfb + (with_h ? B_BYTES + sfb : 0u);
           if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1)) {
             abort_now();
             break;
@@ -508,7 +652,7 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
           mbar_arrive_expect_tx(&full[s], bytes);
           tma_load_2d(sA + s * A_BYTES, map, x0 + kt * KB, int32_t(row), &full[s]);
           bulk_load(sSFA + s * SFA_BYTES, sf + int64_t(kt) * 4 * 512, sfb, &full[s]);
-          if (w.ph == 1) {
+          if (with_h) {
             const uint32_t q = dq % HQ;
             if (!mbar_wait(&hq_empty[q], ((dq / HQ) & 1) ^ 1)) {
               abort_now();
@@ -529,52 +673,57 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
       }
     }
   } else {
-    // warps 1..10: x into the resident token tile (warp 1 only waits for it)
+    // warps 2..15: x into the resident token tile when it was not staged (warp 1 waits for it)
     if (warp >= EPI_FIRST) {
       const int qt = tid - 64, qn = LF_THREADS - 64;
-      // one unit = one token row's 64-element K step: four 16-element blocks, 32 bytes of codes
-      // and one 32-bit word of block scales
-      const int nsteps = H / 64;
-      for (int u = qt; u < LF_MAXT * nsteps; u += qn) {
-        const int t = u / nsteps, g = u - t * nsteps;
-        uint2 code[4] = {make_uint2(0u, 0u), make_uint2(0u, 0u), make_uint2(0u, 0u), make_uint2(0u, 0u)};
-        uint32_t sfw = 0u;
-        if (t < T) {
+      if (!xstage) {  // x did not fit in the stage ring: load and quantise it here
+        // one unit = one token row's 64-element K step: four 16-element blocks, 32 bytes of codes
+        // and one 32-bit word of block scales
+        const int nsteps = H / 64;
+        for (int u = qt; u < LF_MAXT * nsteps; u += qn) {
+          const int t = u / nsteps, g = u - t * nsteps;
+          uint2 code[4] = {make_uint2(0u, 0u), make_uint2(0u, 0u), make_uint2(0u, 0u), make_uint2(0u, 0u)};
+          uint32_t sfw = 0u;
+          if (t < T) {
 #pragma unroll
-          for (int bb = 0; bb < 4; ++bb) {
-            const uint4* src = reinterpret_cast<const uint4*>(a.x + int64_t(t) * H + (g * 4 + bb) * 16);
-            const uint4 u0 = __ldg(src), u1 = __ldg(src + 1);
-            const uint32_t q[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-            float v[16];
+            for (int bb = 0; bb < 4; ++bb) {
+              const uint4* src = reinterpret_cast<const uint4*>(a.x + int64_t(t) * H + (g * 4 + bb) * 16);
+              const uint4 u0 = __ldg(src), u1 = __ldg(src + 1);
+              const uint32_t q[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+              float v[16];
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-              v[2 * jj] = __uint_as_float(q[jj] << 16);
-              v[2 * jj + 1] = __uint_as_float(q[jj] & 0xFFFF0000u);
+              for (int jj = 0; jj < 8; ++jj) {
+                v[2 * jj] = __uint_as_float(q[jj] << 16);
+                v[2 * jj + 1] = __uint_as_float(q[jj] & 0xFFFF0000u);
+              }
+              float amax = 0.0f;
+#pragma unroll
+              for (int jj = 0; jj < 16; ++jj) amax = fmaxf(amax, fabsf(v[jj]));
+              float inv;
+              sfw |= block_scale(amax, s_t, &inv) << (8 * bb);
+              code[bb] = encode_block16(v, inv);
             }
-            float amax = 0.0f;
-#pragma unroll
-            for (int jj = 0; jj < 16; ++jj) amax = fmaxf(amax, fabsf(v[jj]));
-            float inv;
-            sfw |= block_scale(amax, s_t, &inv) << (8 * bb);
-            code[bb] = encode_block16(v, inv);
           }
+          // k-tile g / 4, bytes 32 (g % 4) .. +32 of the 128-byte row = two 16-byte chunks,
+          // swizzled by row % 8
+          const int kt = g >> 2, c16 = 2 * (g & 3);
+          uint8_t* rowp = sX + kt * B_BYTES + t * KB;
+          *reinterpret_cast<uint4*>(rowp + ((c16 ^ (t & 7)) << 4)) =
+              make_uint4(code[0].x, code[0].y, code[1].x, code[1].y);
+          *reinterpret_cast<uint4*>(rowp + (((c16 + 1) ^ (t & 7)) << 4)) =
+              make_uint4(code[2].x, code[2].y, code[3].x, code[3].y);
+          // x scales for TMEM: 512-byte block g / 2 holds row t's scales of steps g (bytes 0..3)
+          // and g + 1 (bytes 8..11) at t * 16; its copy puts them at columns +0 and +2
+          uint32_t* sfp = reinterpret_cast<uint32_t*>(sXSF + (g >> 1) * 512 + t * 16 + (g & 1) * 8);
+          sfp[0] = sfw;
+          sfp[1] = 0u;
         }
-        // k-tile g / 4, bytes 32 (g % 4) .. +32 of the 128-byte row = two 16-byte chunks,
-        // swizzled by row % 8
-        const int kt = g >> 2, c16 = 2 * (g & 3);
-        uint8_t* rowp = sX + kt * B_BYTES + t * KB;
-        *reinterpret_cast<uint4*>(rowp + ((c16 ^ (t & 7)) << 4)) =
-            make_uint4(code[0].x, code[0].y, code[1].x, code[1].y);
-        *reinterpret_cast<uint4*>(rowp + (((c16 + 1) ^ (t & 7)) << 4)) =
-            make_uint4(code[2].x, code[2].y, code[3].x, code[3].y);
-        // x scales for TMEM: 512-byte block g / 2 holds row t's scales of steps g (bytes 0..3)
-        // and g + 1 (bytes 8..11) at t * 16; its copy puts them at columns +0 and +2
-        uint32_t* sfp = reinterpret_cast<uint32_t*>(sXSF + (g >> 1) * 512 + t * 16 + (g & 1) * 8);
-        sfp[0] = sfw;
-        sfp[1] = 0u;
+        for (int i = qt; i < (H / 128) * 64; i += qn)  // rows 16..31 of each block: unused, zero
+          reinterpret_cast<uint32_t*>(sXSF + (i >> 6) * 512 + 256)[i & 63] = 0u;
       }
-      for (int i = qt; i < (H / 128) * 64; i += qn)  // rows 16..31 of each block: unused, zero
-        reinterpret_cast<uint32_t*>(sXSF + (i >> 6) * 512 + 256)[i & 63] = 0u;
+      if (local)  // the local h chunks' scale staging (two 1 KB blocks, x's packing): the bytes
+                  // the epilogue never writes stay zero
+        for (int i = qt; i < 2 * (kcl / 128) * 128; i += qn) reinterpret_cast<uint32_t*>(sSFB)[i] = 0u;
       fence_proxy_async_shared();  // generic stores above, read by the tensor core
     }
     named_sync(1, LF_THREADS - 32);
@@ -587,13 +736,28 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
       if (elect_one()) {
         for (int p = 0; p < H / 128; ++p) tc_cp_sf(tmem + XSF_COL + 4 * p, desc_sf_atom(sXSF + p * 512));
         const uint32_t idesc = idesc_mxf4nvf4(WM, LF_MAXT);
-        uint32_t it = 0;
+        const uint32_t hsf_col = XSF_COL + uint32_t(H / 32);  // local h chunk scales, 8 columns per buffer
+        uint32_t it = 0, h_par = 0u;  // bit b: the phase of h_ready[b] to wait for
         for (int j = 0; j < n_my && !*abort_flag; ++j) {
           const LItem w = item_at(j);
           const uint32_t ab = uint32_t(j) % NACC;
           if (!mbar_wait(&acc_empty[ab], ((uint32_t(j) / NACC) & 1) ^ 1)) {
             abort_now();
             break;
+          }
+          if (local && w.ph == 1 && w.mt == 0) {
+            // a unit's first down tile: its h chunk is complete in shared memory.  Its scales
+            // go to the buffer's TMEM columns; their previous reader (unit n - 2's down MMAs)
+            // was issued before, and this thread's tcgen05 operations run in order.
+            if (!mbar_wait(&h_ready[w.buf], (h_par >> w.buf) & 1u)) {
+              abort_now();
+              break;
+            }
+            h_par ^= 1u << w.buf;
+            tc_fence_after();
+            for (int p = 0; p < kcl / 128; ++p)
+              tc_cp_sf(tmem + hsf_col + uint32_t(w.buf * (kcl / 32) + 4 * p),
+                       desc_sf_atom(sSFB + (w.buf * (kcl / 128) + p) * 512));
           }
           tc_fence_after();
           const uint32_t d_acc = tmem + ACC_COL + ab * LF_MAXT;
@@ -618,6 +782,16 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
               for (int q = 0; q < 4; ++q)
                 tc_mma_mxf4nvf4(d_acc, a_d + 2 * q, b_d + 2 * q, idesc, tmem + SFA_COL + 4 * q,
                                 tmem + XSF_COL + 8 * kt + 4 * (q >> 1) + 2 * (q & 1), (kt | q) != 0 ? 1u : 0u);
+            } else if (local) {
+              // B = k-tile kt of the unit's resident h chunk (all 16 token rows)
+              const uint64_t b_d = desc_kmajor_sw128(sB + (w.buf * (kcl / BK) + kt) * B_BYTES);
+              const uint32_t hcol = hsf_col + uint32_t(w.buf * (kcl / 32) + 8 * kt);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) tc_cp_sf(tmem + SFA_COL + 4 * q, sfa_d + 32 * q);
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                tc_mma_mxf4nvf4(d_acc, a_d + 2 * q, b_d + 2 * q, idesc, tmem + SFA_COL + 4 * q,
+                                tmem + hcol + 4 * (q >> 1) + 2 * (q & 1), (kt | q) != 0 ? 1u : 0u);
             } else {
               const uint64_t sfb_d = desc_sf_atom(sSFB + s * SFB_BYTES);
               const uint64_t b_d = desc_kmajor_sw128(sB + s * B_BYTES);
@@ -639,7 +813,7 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
         mbar_wait(drain, 0, 1u << 20);
       }
     } else {
-      // counters, tickets and h maxima are zeroed by the launch before this one
+      // counters, the combine barrier and h maxima are zeroed by the launch before this one
       griddep_wait();
       // ------------------------------------ inspection copies of the routing ----
       {
@@ -700,7 +874,7 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
         }
       }
 
-      if (warp == HPROD_WARP) {
+      if (warp == HPROD_WARP && !local) {
         // ---------------------------------------------------- producer: h rows ----
         // A down item's h rows are written by the gate/up epilogues of its expert and chunk
         // (this launch); its first stage waits until their counter is complete.  The
@@ -799,7 +973,6 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
         const int half = (warp - EPI_FIRST) >> 2;  // items j with j % 2 == half
         const uint32_t trow = tmem + (uint32_t(q * 32) << 16);
         float* tr = s_tr + (warp - EPI_FIRST) * TR_FLOATS;
-        const int cols32 = H / 32;
         // a gate/up tile's h stores are counted one item later (or at the end), so that the
         // release ordering them before the count finds them drained instead of stalling
         int pending = -1;
@@ -844,63 +1017,151 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
             }
             __syncwarp();
             float amax_all = 0.0f;
-            if (lane < LF_MAXT && ((mask >> lane) & 1u)) {
-              // lane t quantises token t's 16 values of this block (one block scale)
-              float hb[16];
+            if (lane < LF_MAXT) {
+              // lane t quantises token t's 16 values of this block (one block scale) if the
+              // expert received token t; the other rows of a local h chunk are zero
+              uint2 code = make_uint2(0u, 0u);
+              uint32_t sf = 0u;
+              if ((mask >> lane) & 1u) {
+                float hb[16];
 #pragma unroll
-              for (int i = 0; i < 16; ++i) hb[i] = tr[lane * TRS + i];
-              float amax = 0.0f;
+                for (int i = 0; i < 16; ++i) hb[i] = tr[lane * TRS + i];
+                float amax = 0.0f;
 #pragma unroll
-              for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(hb[i]));
-              const int64_t row = int64_t(w.a) * TOK_ALIGN + __popc(mask & ((1u << lane) - 1u));
-              float inv;
-              const uint32_t sf = block_scale(amax, sh, &inv);
-              *reinterpret_cast<uint2*>(a.h_codes + row * (I / 2) + iblk * 8) = encode_block16(hb, inv);
-              a.h_sf[sf_mma_offset(row, iblk, I)] = static_cast<uint8_t>(sf);
-              amax_all = amax;
+                for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(hb[i]));
+                const int64_t row = int64_t(w.a) * TOK_ALIGN + __popc(mask & ((1u << lane) - 1u));
+                float inv;
+                sf = block_scale(amax, sh, &inv);
+                code = encode_block16(hb, inv);
+                *reinterpret_cast<uint2*>(a.h_codes + row * (I / 2) + iblk * 8) = code;
+                a.h_sf[sf_mma_offset(row, iblk, I)] = static_cast<uint8_t>(sf);
+                amax_all = amax;
+              }
+              if (local) {
+                // token row `lane` of the unit's h chunk (K-major, 128-byte swizzle, k-tile
+                // il / 16), and the block's scale byte in the staging the MMA warp copies to
+                // TMEM (x's packing: 512-byte block il / 8, row t at t * 16, step (il / 4) % 2
+                // at byte 8 of it)
+                const int il = iblk - (kcl / 16) * w.kc;  // block within the chunk
+                uint8_t* hrow = sB + (w.buf * (kcl / BK) + (il >> 4)) * B_BYTES + lane * KB;
+                const int i16 = il & 15;
+                *reinterpret_cast<uint2*>(hrow + ((((i16 >> 1) ^ (lane & 7)) << 4) | ((i16 & 1) << 3))) = code;
+                sSFB[(w.buf * (kcl / 128) + (il >> 3)) * 512 + lane * 16 + ((il >> 2) & 1) * 8 + (il & 3)] =
+                    uint8_t(sf);
+              }
             }
+            if (local) fence_proxy_async_shared();  // generic stores, read by the tensor core
             __syncwarp();
+            if (local && lane == 0) mbar_arrive(&h_ready[w.buf]);
             if (a.h_amax) {
 #pragma unroll
               for (int o = 16; o > 0; o >>= 1) amax_all = fmaxf(amax_all, __shfl_xor_sync(0xffffffffu, amax_all, o));
               if (lane == 0 && amax_all > 0.0f) atomicMax(reinterpret_cast<int*>(a.h_amax + e), __float_as_int(amax_all));
             }
-            pending = w.a * nkc + (w.mt * 64) / KC;
+            if (!local) pending = w.a * nkc + (w.mt * 64) / KC;
+          } else if (local) {
+            // lane = output row mt*128 + 32q + lane; accumulator column = token.  The weighted
+            // row of each (pair, chunk) goes to its slot; the combine follows the last unit.
+            const int col = w.mt * WM + q * 32 + lane;
+            const int base = s_aoff[w.a];
+            for (int c = 0; c < cnt; ++c) {
+              const int p = s_prank[base + c], t = p / k;
+              float v = 0.0f;
+#pragma unroll
+              for (int i = 0; i < LF_MAXT; ++i) v = i == t ? __uint_as_float(r[i]) : v;
+              a.slots[(int64_t(p) * nkc_x + w.kc) * H + col] = v * (s_w[p] * sc);
+            }
           } else {
             // lane = output row mt*128 + 32q + lane; column c = the expert's c-th token; the
             // weighted row of each (pair, K chunk) goes to its slot, summed by the combine
             const int col = w.mt * WM + q * 32 + lane;
             const int base = s_aoff[w.a];
-            int my_pair = -1;
 #pragma unroll
             for (int c = 0; c < LF_MAXT; ++c) {
               if (c < cnt) {
                 const int p = s_prank[base + c];
-                if (lane == c) my_pair = p;
                 a.slots[(int64_t(p) * nkc + w.kc) * H + col] = __uint_as_float(r[c]) * (s_w[p] * sc);
               }
-            }
-            // one ticket per (token, 32 columns): the warp that completes a token's k x nkc
-            // rows sums them in slot order and rounds once.  The ticket is an acquire-release
-            // add: it publishes this warp's rows (ordered before it by the __syncwarp) and,
-            // for the last one, makes the other warps' rows visible to the reads below.
-            __syncwarp();
-            bool last = false;
-            if (lane < cnt) last = atom_acq_rel_add1(a.tickets + (my_pair / k) * cols32 + (col >> 5)) == k * nkc - 1;
-            uint32_t lastm = __ballot_sync(0xffffffffu, last);
-            while (lastm) {
-              const int c = __ffs(lastm) - 1;
-              lastm &= lastm - 1;
-              const int t = __shfl_sync(0xffffffffu, my_pair, c) / k;
-              float sum = 0.0f;
-              for (int jj = 0; jj < k; ++jj)
-                for (int kc2 = 0; kc2 < nkc; ++kc2)
-                  sum += __ldcg(a.slots + ((int64_t(t) * k + jj) * nkc + kc2) * H + col);
-              a.out[int64_t(t) * H + col] = __float2bfloat16_rn(sum);
             }
           }
         }
         release_pending();
+        // ---------------------------------------------------------- combine ----
+        // Once every CTA has arrived here all slot rows are stored (one release per CTA: the
+        // named barrier orders the other epilogue warps' stores before it).  Then each CTA sums
+        // its slice of the [T][H] outputs over the token's k x chunks rows in slot order and
+        // rounds once to bf16.  The launch is cooperative (all CTAs resident), so the wait
+        // ends; it is bounded all the same.
+        named_sync(3, EPI_WARPS * 32);
+        volatile int* s_ok = reinterpret_cast<volatile int*>(s_tr);
+        float4* s_part = reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(s_tr) + 4096);  // [4][64]
+        if (tid == 32 * EPI_FIRST) {
+          int ok = 0;
+          if (!*abort_flag) {
+            fence_acq_rel_gpu();
+            atomicAdd(a.gbar, 1);
+            const uint64_t t0 = global_ns();
+            ok = 1;
+            while (ld_acquire_gpu(a.gbar) < G)
+              if (global_ns() - t0 > 200000000ull) {  // 0.2 s: a CTA never arrived
+                abort_now();
+                ok = 0;
+                break;
+              }
+          }
+          *s_ok = ok;
+        }
+        named_sync(3, EPI_WARPS * 32);
+        if (*s_ok) {
+          // thread = (float4 column c4 of 64, row quarter g): quarter g sums its rows in order
+          // (up to eight loads in flight), then the four partial sums are added in order
+          const int nr = k * nkc_x;  // a token's slot rows are consecutive (pair-major, then chunk)
+          const int64_t units = int64_t(T) * (H / 4);
+          const int64_t lo = units * blockIdx.x / G, hi = units * (blockIdx.x + 1) / G;
+          const int th = tid - 32 * EPI_FIRST, c4 = th & 63, g = th >> 6;
+          const int rq = (nr + 3) / 4, r_lo = min(nr, g * rq), r_hi = min(nr, r_lo + rq);
+          for (int64_t u0 = lo; u0 < hi; u0 += 64) {
+            const int64_t u = u0 + c4;
+            const int t = int(u / (H / 4)), col4 = int(u - int64_t(t) * (H / 4));
+            float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            if (u < hi) {
+              const float4* rows = reinterpret_cast<const float4*>(a.slots + int64_t(t) * nr * H) + col4;
+              for (int r = r_lo; r < r_hi; r += 8) {
+                float4 v[8];
+#pragma unroll
+                for (int q2 = 0; q2 < 8; ++q2)
+                  v[q2] = r + q2 < r_hi ? __ldcg(rows + int64_t(r + q2) * (H / 4)) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+                for (int q2 = 0; q2 < 8; ++q2)
+                  if (r + q2 < r_hi) {
+                    acc.x += v[q2].x;
+                    acc.y += v[q2].y;
+                    acc.z += v[q2].z;
+                    acc.w += v[q2].w;
+                  }
+              }
+            }
+            s_part[g * 64 + c4] = acc;
+            named_sync(3, EPI_WARPS * 32);
+            if (g == 0 && u < hi) {
+              float4 sum = s_part[c4];
+#pragma unroll
+              for (int q2 = 1; q2 < 4; ++q2) {
+                const float4 v = s_part[q2 * 64 + c4];
+                sum.x += v.x;
+                sum.y += v.y;
+                sum.z += v.z;
+                sum.w += v.w;
+              }
+              const __nv_bfloat162 lo2 = __floats2bfloat162_rn(sum.x, sum.y), hi2 = __floats2bfloat162_rn(sum.z, sum.w);
+              uint2 packed;
+              packed.x = *reinterpret_cast<const uint32_t*>(&lo2);
+              packed.y = *reinterpret_cast<const uint32_t*>(&hi2);
+              *reinterpret_cast<uint2*>(a.out + int64_t(t) * H + 4 * col4) = packed;
+            }
+            named_sync(3, EPI_WARPS * 32);  // s_part is rewritten next round
+          }
+        }
       }
     }
   }
@@ -909,7 +1170,7 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
   __syncthreads();
   tc_fence_after();
   if (warp == 1) {
-    const uint32_t need = XSF_COL + uint32_t(H / 32);
+    const uint32_t need = lf_tmem_need(H, KCL_MAX);
     tmem_dealloc(*tmem_holder, need <= 256 ? 256u : 512u);
   }
 }
@@ -919,14 +1180,29 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
 bool layer_fused_fits(int T, int H, int I, int E, int k) {
   if (T < 1 || T > LF_MAXT || E < 1 || E > LF_MAXE || k < 1 || k > 32 || k > E) return false;
   if (H % BK != 0 || I % 128 != 0) return false;
-  if (XSF_COL + uint32_t(H / 32) > 512u) return false;
+  if (lf_tmem_need(H) > 512u) return false;  // the narrowest local chunk's columns too
   if (int64_t(T) * k > LF_MAXP) return false;
   const int nkc = (I + lf_kc(I) - 1) / lf_kc(I);
   if (nkc > 63 || 2 * I / WM > 8191 || H / WM > 8191) return false;  // work item packing
   return lf_shape(T, H, I, E, k, num_sms()).stages >= MIN_STAGES;
 }
 
-int layer_fused_chunks(int I) { return (I + lf_kc(I) - 1) / lf_kc(I); }
+bool layer_fused_local_fits(int I) { return I % KCL == 0 && I / KCL <= 63; }  // width 256 at least
+
+// Whether the expert-local schedule would be taken for the expected number of active experts
+// of uniformly random routing, E * (1 - (1 - k/E)^T).
+bool layer_fused_local_likely(int T, int H, int I, int E, int k) {
+  if (!layer_fused_fits(T, H, I, E, k)) return false;
+  const double miss = std::pow(1.0 - double(k) / E, double(T));
+  const int A = int(std::lround(E * (1.0 - miss)));
+  return lf_local_width(A, I, num_sms(), 0, H, lf_shape(T, H, I, E, k, num_sms()).stages) > 0;
+}
+
+// slot rows per pair: K chunks of the tile-level schedule, or of the expert-local one
+int layer_fused_chunks(int I) {
+  const int tile_level = (I + lf_kc(I) - 1) / lf_kc(I);
+  return I % KCL == 0 && I / KCL > tile_level ? I / KCL : tile_level;
+}
 
 nvfp4moe_status launch_layer_fused_reset(const LayerFusedArgs& f, cudaStream_t s) {
   if (!layer_fused_fits(f.T, f.H, f.I, f.E, f.k))
@@ -934,8 +1210,7 @@ nvfp4moe_status launch_layer_fused_reset(const LayerFusedArgs& f, cudaStream_t s
                 f.k);
   const int P = f.T * f.k;
   const int n_done = (P < f.E ? P : f.E) * layer_fused_chunks(f.I);
-  const int n_tickets = f.T * (f.H / 32);
-  layer_reset_kernel<<<1, 512, 0, s>>>(f.done, n_done, f.tickets, n_tickets, f.h_amax, f.E);
+  layer_reset_kernel<<<1, 512, 0, s>>>(f.done, n_done, f.gbar, f.h_amax, f.E);
   return check_launch("fused layer reset");
 }
 
@@ -966,14 +1241,15 @@ nvfp4moe_status launch_layer_fused(const LayerFusedArgs& f, cudaStream_t s) {
   a.counts = f.counts; a.offsets = f.offsets; a.padded_offsets = f.padded_offsets; a.pair_to_row = f.pair_to_row;
   a.row_token = f.row_token; a.row_pair = f.row_pair; a.tile_expert = f.tile_expert; a.active = f.active;
   a.x_codes = f.x_codes; a.x_sf = f.x_sf; a.h_codes = f.h_codes; a.h_sf = f.h_sf;
-  a.slots = f.slots; a.done = f.done; a.tickets = f.tickets;
+  a.slots = f.slots; a.done = f.done; a.gbar = f.gbar;
+  a.schedule = f.schedule;
   a.out = static_cast<__nv_bfloat16*>(f.out);
   a.shape = lf_shape(f.T, f.H, f.I, f.E, f.k, num_sms());
   a.status = status;
   const int smem = 1024 + lf_layout(a.shape).total;
   const int per = (f.E + 31) / 32;
   auto go = [&](auto kern) -> cudaError_t {
-    return launch_dependent(kern, dim3(num_sms()), dim3(LF_THREADS), size_t(smem), s, mw13, mw2, mh, a);
+    return launch_cooperative_dependent(kern, dim3(num_sms()), dim3(LF_THREADS), size_t(smem), s, mw13, mw2, mh, a);
   };
   cudaError_t e;
   if (per <= 4) {

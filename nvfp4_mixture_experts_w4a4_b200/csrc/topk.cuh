@@ -28,22 +28,23 @@ __device__ __forceinline__ float topk_key_value(uint64_t key) {
   return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
 }
 
-// Selects the top k (k <= 32) of l[0..E) for the calling warp.  Lane j < k returns the j-th
-// expert in *id and its softmax weight in *w.  Each lane first finds its two largest keys.
-// A round takes the warp maximum of the lanes' current best keys with two hardware reductions
-// (the logit word, then the index word among the lanes that hold that logit, which picks the
-// lower expert index); the lane that held the winner moves on to its second key, and only on
-// a further win rescans its keys for the largest one below the key just taken (keys are
-// unique, so "below" excludes exactly the keys already taken).  A lane rarely holds more than
-// two of the k winners, so the rescans are rare and most rounds cost two reductions.
+// Selects the top k (k <= 32) of the E logits the calling warp holds, lane l holding logits
+// l, l+32, ... in lg[] (slots at or past E are ignored).  Lane j < k returns the j-th expert in
+// *id and its softmax weight in *w.  Each lane first finds its two largest keys.  A round takes
+// the warp maximum of the lanes' current best keys with two hardware reductions (the logit
+// word, then the index word among the lanes that hold that logit, which picks the lower expert
+// index); the lane that held the winner moves on to its second key, and only on a further win
+// rescans its keys for the largest one below the key just taken (keys are unique, so "below"
+// excludes exactly the keys already taken).  A lane rarely holds more than two of the k
+// winners, so the rescans are rare and most rounds cost two reductions.
 template <int PER_LANE>
-__device__ __forceinline__ void warp_topk(const float* __restrict__ l, int E, int k, int* id, float* w) {
+__device__ __forceinline__ void warp_topk_regs(const float (&lg)[PER_LANE], int E, int k, int* id, float* w) {
   const int lane = threadIdx.x & 31;
   uint64_t key[PER_LANE];
 #pragma unroll
   for (int i = 0; i < PER_LANE; ++i) {
     const int e = lane + 32 * i;
-    key[i] = e < E ? topk_key(l[e], e) : 0ull;  // 0 marks an absent slot (real keys are > 0)
+    key[i] = e < E ? topk_key(lg[i], e) : 0ull;  // 0 marks an absent slot (real keys are > 0)
   }
   uint64_t m1 = 0, m2 = 0;  // this lane's largest and second largest key
 #pragma unroll
@@ -82,6 +83,19 @@ __device__ __forceinline__ void warp_topk(const float* __restrict__ l, int E, in
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   *id = bi;
   *w = ex / sum;
+}
+
+// The same selection over l[0..E) in global memory.
+template <int PER_LANE>
+__device__ __forceinline__ void warp_topk(const float* __restrict__ l, int E, int k, int* id, float* w) {
+  const int lane = threadIdx.x & 31;
+  float lg[PER_LANE];
+#pragma unroll
+  for (int i = 0; i < PER_LANE; ++i) {
+    const int e = lane + 32 * i;
+    lg[i] = e < E ? l[e] : 0.0f;
+  }
+  warp_topk_regs<PER_LANE>(lg, E, k, id, w);
 }
 
 }  // namespace nvfp4moe

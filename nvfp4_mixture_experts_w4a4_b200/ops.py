@@ -349,7 +349,9 @@ class MoeFFN:
         or ACT_BF16 (weight-only W4A16: bf16 activations, the GEMV path; no scales used).
         shared: None or a BF16 shared expert (w13 bf16 [2I_s, H] interleaved, see
         shared_expert_w13; w2 bf16 [H, I_s]), added to every token's output.  launch: LAUNCH_AUTO,
-        LAUNCH_SINGLE (the whole layer as one persistent launch, where the batch allows it) or
+        LAUNCH_SINGLE (the whole layer as one persistent launch, where the batch allows it; the
+        schedule, expert-local or tile-level, is chosen per call from the routing),
+        LAUNCH_SINGLE_TILE / LAUNCH_SINGLE_LOCAL (the single launch with that schedule) or
         LAUNCH_MULTI (prologue, grouped GEMMs, combine)."""
         self.w = experts
         self.top_k = top_k

@@ -54,11 +54,14 @@ def checked_tokens(ids_all: np.ndarray, T: int, E: int) -> np.ndarray:
     return np.array(sorted(sel), np.int64)
 
 
-@pytest.mark.parametrize("name,shared_I", [("decode", 0), ("prefill_chunk", 0), ("long_prefill", 0), ("dense", 0),
-                                           ("dense_t1", 0), ("decode", 512), ("prefill_chunk", 512)])
-def test_fullsize_sampled_tokens(name, shared_I):
+@pytest.mark.parametrize("name,shared_I,launch", [
+    ("decode", 0, "auto"), ("prefill_chunk", 0, "auto"), ("long_prefill", 0, "auto"), ("dense", 0, "auto"),
+    ("dense_t1", 0, "auto"), ("decode", 512, "auto"), ("prefill_chunk", 512, "auto"),
+    ("decode", 0, "single_local"), ("decode", 0, "single_tile"), ("decode", 0, "multi")])
+def test_fullsize_sampled_tokens(name, shared_I, launch):
     """shared_I > 0: with a BF16 shared expert of that size (the streamed kernel at 16 tokens,
-    the tcgen05 bf16 GEMMs at 512)."""
+    the tcgen05 bf16 GEMMs at 512).  launch: the automatic choice (as the benchmark runs it), or
+    the decode batch forced through each single-launch schedule and the multi-launch path."""
     wl = W.WORKLOADS[name]
     dev = G.need_gpu()
     T, H, I, E, k = wl.T, wl.H, wl.I, wl.E, wl.k
@@ -98,8 +101,12 @@ def test_fullsize_sampled_tokens(name, shared_I):
     s_h = np.ones(E, np.float32)
     s_h[touched] = ref["h_scale"]
 
-    # the device: the whole batch, dynamic x scale, automatic path (as the benchmark runs it)
-    layer = ops.MoeFFN(experts, k, torch.from_numpy(s_h).to(dev), shared=shared)
+    # the device: the whole batch, dynamic x scale, automatic path
+    mode = {"auto": C.LAUNCH_AUTO, "single_local": C.LAUNCH_SINGLE_LOCAL, "single_tile": C.LAUNCH_SINGLE_TILE,
+            "multi": C.LAUNCH_MULTI}[launch]
+    layer = ops.MoeFFN(experts, k, torch.from_numpy(s_h).to(dev), shared=shared, launch=mode)
+    if launch != "auto":
+        assert layer.layout(T).single_launch == (0 if launch == "multi" else 1)
     out = layer(act["x"], act["logits"])
     torch.cuda.synchronize()
     im = layer.intermediates(T)
@@ -189,8 +196,8 @@ def test_fullsize_weight_only_sampled_tokens(name):
     G.check_out(G.bf16_bits(out)[sample], ref["out_f64"])
 
 
-@pytest.mark.parametrize("name", ["decode", "dense_t1"])
-def test_fullsize_calls_with_changing_routing(name):
+@pytest.mark.parametrize("name,launch", [("decode", "single"), ("dense_t1", "single"), ("decode", "single_local")])
+def test_fullsize_calls_with_changing_routing(name, launch):
     """Consecutive calls whose routing differs (the workload's inputs, then all-zero inputs that
     send every token to the same experts, and so on): every call completes without a device
     timeout and every call on the workload's inputs gives the same output bit for bit.  The
@@ -202,7 +209,8 @@ def test_fullsize_calls_with_changing_routing(name):
     wts = W.make_weights(wl, 0, dev)
     experts = ops.NVFP4Experts.from_float(wts["w_gate"], wts["w_up"], wts["w_down"])
     del wts
-    layer = ops.MoeFFN(experts, wl.k, torch.full((wl.E,), 0.01, device=dev), launch=C.LAUNCH_SINGLE)
+    mode = {"single": C.LAUNCH_SINGLE, "single_local": C.LAUNCH_SINGLE_LOCAL}[launch]
+    layer = ops.MoeFFN(experts, wl.k, torch.full((wl.E,), 0.01, device=dev), launch=mode)
     assert layer.layout(wl.T).single_launch == 1
     ops.device_status(clear=True)
     first = layer(act["x"], act["logits"]).clone()

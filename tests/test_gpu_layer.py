@@ -334,7 +334,7 @@ SINGLE_CASES = {
 @pytest.mark.parametrize("name", list(SINGLE_CASES))
 def test_layer_single_launch(name):
     """The single-launch layer against the oracle with the usual tolerances, then called again
-    on the same workspace: its counters and tickets start from zero in every call, so the second
+    on the same workspace: its counters and barrier start from zero in every call, so the second
     output is the first bit for bit."""
     wl = SINGLE_CASES[name]
     ref, out, layer, h_amax = G.run_layer_pair(wl, C.PATH_GEMM, launch=C.LAUNCH_SINGLE)
@@ -347,10 +347,42 @@ def test_layer_single_launch(name):
     assert ops.device_status() == 0
 
 
+# Shapes with I % 256 == 0, run under both schedules of the single launch
+SCHEDULE_CASES = {
+    "decode_E512_k10": SINGLE_CASES["decode_E512_k10"],
+    "k32_E1024": SINGLE_CASES["k32_E1024"],
+    # 18 units of one expert: 18 CTAs with one unit each, the rest idle
+    "dense_T1_18_units": SINGLE_CASES["dense_T1_three_chunks"],
+    # four h chunks per expert and about 140 active experts: several units per CTA, so both
+    # h buffers are reused and the down tiles of one unit follow the next unit's gate/up tiles
+    "decode_I1024_units_per_cta": W.scaled(W.WORKLOADS["decode"], H=512, I=1024),
+    "ragged_T5_I768": W.scaled(TINY, T=5, E=40, k=4, H=768, I=768),
+}
+
+
+@pytest.mark.parametrize("launch", ["tile", "local"])
+@pytest.mark.parametrize("name", list(SCHEDULE_CASES))
+def test_layer_single_launch_schedules(name, launch):
+    """The single launch with its schedule forced (tile-level: h through global memory; expert-
+    local: h chunks resident in shared memory) against the oracle, then called again: the
+    second output is the first bit for bit."""
+    wl = SCHEDULE_CASES[name]
+    mode = {"tile": C.LAUNCH_SINGLE_TILE, "local": C.LAUNCH_SINGLE_LOCAL}[launch]
+    ref, out, layer, h_amax = G.run_layer_pair(wl, C.PATH_GEMM, launch=mode)
+    assert layer.layout(wl.T).single_launch == 1
+    G.check_layer(wl, ref, out, layer, h_amax)
+    act = W.make_activations(wl, 0, "cpu")
+    again = layer(act["x"].cuda(), act["logits"].cuda())
+    torch.cuda.synchronize()
+    assert torch.equal(out, again)
+    assert ops.device_status() == 0
+
+
 def test_single_launch_selection():
     """LAUNCH_SINGLE takes the single launch where the batch allows it and is refused where it
     does not (17 tokens); the accumulating combine, a dynamic h scale or LAUNCH_MULTI keep the
-    multi-launch path; LAUNCH_AUTO takes the single launch for the dense layer (one expert)."""
+    multi-launch path; LAUNCH_AUTO takes the single launch for the dense layer (one expert) and
+    for routed decode batches that the expert-local schedule fits."""
     dev = G.need_gpu()
     wl = W.scaled(TINY, T=17)
     _, wts, wg, wu, wd = G.layer_inputs(wl)
@@ -364,7 +396,22 @@ def test_single_launch_selection():
     assert single(combine=C.COMBINE_ACCUMULATE).layout(16).single_launch == 0
     assert single(h=None).layout(16).single_launch == 0
     assert ops.MoeFFN(ex, wl.k, ones, launch=C.LAUNCH_MULTI).layout(16).single_launch == 0
+    # the expert-local schedule needs I % 256 == 0 (here I = 128): refused, not rerouted
+    local = ops.MoeFFN(ex, wl.k, ones, launch=C.LAUNCH_SINGLE_LOCAL)
+    assert local.layout(16).single_launch == 0
+    with pytest.raises(C.Nvfp4MoeError):
+        local(torch.zeros(16, wl.H, dtype=torch.bfloat16, device=dev), torch.zeros(16, wl.E, device=dev))
+    assert ops.MoeFFN(ex, wl.k, ones, launch=C.LAUNCH_SINGLE_TILE).layout(16).single_launch == 1
     dense = W.scaled(W.WORKLOADS["dense"], T=4, H=256, I=256)
     _, _, dg, du, dd = G.layer_inputs(dense)
     dex = G.experts_from_oracle(dg, du, dd, dev)
     assert ops.MoeFFN(dex, 1, torch.ones(1, device=dev)).layout(4).single_launch == 1
+    # routed decode whose expected active experts fill the grid with expert-local units: AUTO
+    # takes the single launch; at I = 128 (no local schedule) it keeps the multi-launch path
+    E, H, I = 512, 256, 512
+    gen = torch.Generator(device=dev).manual_seed(0)
+    rex = ops.NVFP4Experts.from_float(torch.randn(E, I, H, device=dev, generator=gen),
+                                      torch.randn(E, I, H, device=dev, generator=gen),
+                                      torch.randn(E, H, I, device=dev, generator=gen))
+    assert ops.MoeFFN(rex, 10, torch.ones(E, device=dev)).layout(16).single_launch == 1
+    assert ops.MoeFFN(ex, wl.k, ones).layout(16).single_launch == 0
