@@ -157,8 +157,8 @@ void make_layout(const moe_ffn_desc* d, moe_ffn_ws_layout* L) {
                                       prologue_scratch));
   // the fused GEMM's work list and per-expert counters, written by the small-batch prologue
   const int64_t A = P < E ? P : E;
-  if (L->single_launch)  // per (active expert, K chunk) counters, then the combine barrier
-    L->items = take((A * layer_fused_chunks(d->I) + 1) * 4);
+  if (L->single_launch)  // per (active expert, K chunk) counters, per (token, 32 columns) tickets, a barrier
+    L->items = take((A * layer_fused_chunks(d->I) + T * (H / 32) + 1) * 4);
   else
     L->items = take(path == NVFP4MOE_PATH_GEMM && prologue_fits(d->T, d->E, d->top_k)
                         ? grouped_fused_list_entries(A, 2 * I / 128, H / 128) * 16 + E * 4
@@ -304,7 +304,8 @@ nvfp4moe_status moe_ffn_forward(const moe_ffn_desc* d, const void* x, const floa
     f.rows_cap = rows_cap;
     f.slots = F32(L.slots);
     f.done = I32(L.items);
-    f.gbar = I32(L.items) + max_active_experts(d) * layer_fused_chunks(I);
+    f.tickets = I32(L.items) + max_active_experts(d) * layer_fused_chunks(I);
+    f.gbar = f.tickets + T * (H / 32);
     f.out = out;
     f.schedule = d->launch_mode == NVFP4MOE_LAUNCH_SINGLE_TILE    ? 1
                  : d->launch_mode == NVFP4MOE_LAUNCH_SINGLE_LOCAL ? 2

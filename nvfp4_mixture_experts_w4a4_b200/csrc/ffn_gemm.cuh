@@ -88,7 +88,8 @@ struct LayerFusedArgs {
   int64_t rows_cap;
   float* slots;   // [T*k*layer_fused_chunks(I)][H] fp32
   int* done;      // [min(T*k, E) * layer_fused_chunks(I)]
-  int* gbar;      // [1] the combine barrier
+  int* tickets;   // [T][H/32] tile-level combine tickets
+  int* gbar;      // [1] the expert-local combine barrier
   int schedule;   // 0: chosen per call from the routing; 1: tile-level; 2: expert-local
   void* out;
 };

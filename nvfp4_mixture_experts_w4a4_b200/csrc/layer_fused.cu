@@ -36,11 +36,13 @@
 //      fence before TMA reads h).  The weight tiles themselves never wait: the producer
 //      streams W2 while h is finishing.
 //  * Combine: the down epilogue writes each routed pair's weighted fp32 rows (one row per K
-//    chunk) to its slots.  After a grid-wide barrier (one release per CTA; the launch is
-//    cooperative, so all CTAs are resident) every CTA sums a slice of the [T][H] outputs over
-//    the token's k x chunks rows in slot order and rounds once to bf16.
+//    chunk) to its slots.  Tile-level: one ticket per (token, 32 output columns) and down
+//    tile; the warp that takes a token's last ticket sums its k x chunks rows in slot order
+//    and rounds once to bf16 (the sums are spread over the run).  Expert-local: after a
+//    grid-wide barrier (one release per CTA; the launch is cooperative, so all CTAs are
+//    resident) every CTA sums a slice of the [T][H] outputs the same way.
 //
-// A small launch before this one zeroes the counters and the barrier; this kernel is its
+// A small launch before this one zeroes the counters, tickets and barrier; this kernel is its
 // programmatic dependent and waits for it only before touching them (well after its start).
 //
 // Warp roles after the routing phase (all 16 warps route, one token each, and quantise x):
@@ -221,7 +223,8 @@ struct LayerArgs {
   float* slots;             // [T*k*nkc][H]: weighted fp32 rows by (pair, K chunk); nkc of the schedule
                             // taken, at most layer_fused_chunks(I)
   int* done;                // [min(P, E) * nkc] gate/up tiles finished per (active expert, chunk)
-  int* gbar;                // [1] CTAs arrived at the combine barrier
+  int* tickets;             // [T][H/32] tile-level combine tickets
+  int* gbar;                // [1] CTAs arrived at the combine barrier (expert-local)
   int schedule;             // 0: chosen from the routing; 1: tile-level; 2: expert-local
   __nv_bfloat16* out;       // [T][H]
   LfShape shape;
@@ -273,6 +276,12 @@ __device__ __forceinline__ int ld_relaxed_gpu(const int* ptr) {
   return v;
 }
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+// +1 with acquire-release semantics at GPU scope; returns the previous count.
+__device__ __forceinline__ int atom_acq_rel_add1(int* p) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
+  return old;
+}
 // +1 with release semantics at GPU scope: the writes that precede it, including the other
 // lanes' writes ordered before it by a __syncwarp, are visible to whoever acquires the count.
 __device__ __forceinline__ void red_release_add1(int* p) {
@@ -300,11 +309,13 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
 // silu(g) * u with the fast exponential and division (h is requantised to E2M1 right after)
 __device__ __forceinline__ float lf_silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
-// Counters and the combine barrier of one call back to zero, and the h maxima when they are
-// requested.
-__global__ void layer_reset_kernel(int* done, int n_done, int* gbar, float* h_amax, int E) {
+// Counters, tickets and the combine barrier of one call back to zero, and the h maxima when
+// they are requested.
+__global__ void layer_reset_kernel(int* done, int n_done, int* tickets, int n_tickets, int* gbar, float* h_amax,
+                                   int E) {
   griddep_launch_dependents();
   for (int i = threadIdx.x; i < n_done; i += blockDim.x) done[i] = 0;
+  for (int i = threadIdx.x; i < n_tickets; i += blockDim.x) tickets[i] = 0;
   if (threadIdx.x == 0) *gbar = 0;
   if (h_amax)
     for (int i = threadIdx.x; i < E; i += blockDim.x) h_amax[i] = 0.0f;
@@ -813,7 +824,7 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
         mbar_wait(drain, 0, 1u << 20);
       }
     } else {
-      // counters, the combine barrier and h maxima are zeroed by the launch before this one
+      // counters, tickets, the combine barrier and h maxima are zeroed by the launch before this one
       griddep_wait();
       // ------------------------------------ inspection copies of the routing ----
       {
@@ -1073,93 +1084,125 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
             }
           } else {
             // lane = output row mt*128 + 32q + lane; column c = the expert's c-th token; the
-            // weighted row of each (pair, K chunk) goes to its slot, summed by the combine
+            // weighted row of each (pair, K chunk) goes to its slot
             const int col = w.mt * WM + q * 32 + lane;
             const int base = s_aoff[w.a];
+            int my_pair = -1;
 #pragma unroll
             for (int c = 0; c < LF_MAXT; ++c) {
               if (c < cnt) {
                 const int p = s_prank[base + c];
+                if (lane == c) my_pair = p;
                 a.slots[(int64_t(p) * nkc + w.kc) * H + col] = __uint_as_float(r[c]) * (s_w[p] * sc);
               }
+            }
+            // one ticket per (token, 32 columns): the warp that completes a token's k x nkc
+            // rows sums them in slot order and rounds once.  The ticket is an acquire-release
+            // add: it publishes this warp's rows (ordered before it by the __syncwarp) and,
+            // for the last one, makes the other warps' rows visible to the reads below.  (The
+            // tile-level schedule spreads each token's rows over many CTAs and items, so the
+            // sums are spread too; the expert-local schedule combines after a barrier instead.)
+            __syncwarp();
+            bool last = false;
+            if (lane < cnt) last = atom_acq_rel_add1(a.tickets + (my_pair / k) * (H / 32) + (col >> 5)) == k * nkc - 1;
+            uint32_t lastm = __ballot_sync(0xffffffffu, last);
+            while (lastm) {
+              const int c = __ffs(lastm) - 1;
+              lastm &= lastm - 1;
+              const int t = __shfl_sync(0xffffffffu, my_pair, c) / k;
+              // the token's k x nkc rows are consecutive slot rows (pair-major, then chunk)
+              const int nr = k * nkc;
+              const float* rows = a.slots + int64_t(t) * nr * H + col;
+              float sum = 0.0f;
+              for (int r0 = 0; r0 < nr; r0 += 8) {  // up to eight loads in flight, summed in order
+                float v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) v[u] = r0 + u < nr ? __ldcg(rows + int64_t(r0 + u) * H) : 0.0f;
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                  if (r0 + u < nr) sum += v[u];
+              }
+              a.out[int64_t(t) * H + col] = __float2bfloat16_rn(sum);
             }
           }
         }
         release_pending();
-        // ---------------------------------------------------------- combine ----
+        // ------------------------------------------------ combine (expert-local) ----
         // Once every CTA has arrived here all slot rows are stored (one release per CTA: the
         // named barrier orders the other epilogue warps' stores before it).  Then each CTA sums
         // its slice of the [T][H] outputs over the token's k x chunks rows in slot order and
         // rounds once to bf16.  The launch is cooperative (all CTAs resident), so the wait
         // ends; it is bounded all the same.
-        named_sync(3, EPI_WARPS * 32);
-        volatile int* s_ok = reinterpret_cast<volatile int*>(s_tr);
-        float4* s_part = reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(s_tr) + 4096);  // [4][64]
-        if (tid == 32 * EPI_FIRST) {
-          int ok = 0;
-          if (!*abort_flag) {
-            fence_acq_rel_gpu();
-            atomicAdd(a.gbar, 1);
-            const uint64_t t0 = global_ns();
-            ok = 1;
-            while (ld_acquire_gpu(a.gbar) < G)
-              if (global_ns() - t0 > 200000000ull) {  // 0.2 s: a CTA never arrived
-                abort_now();
-                ok = 0;
-                break;
-              }
+        if (local) {
+          named_sync(3, EPI_WARPS * 32);
+          volatile int* s_ok = reinterpret_cast<volatile int*>(s_tr);
+          float4* s_part = reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(s_tr) + 4096);  // [4][64]
+          if (tid == 32 * EPI_FIRST) {
+            int ok = 0;
+            if (!*abort_flag) {
+              fence_acq_rel_gpu();
+              atomicAdd(a.gbar, 1);
+              const uint64_t t0 = global_ns();
+              ok = 1;
+              while (ld_acquire_gpu(a.gbar) < G)
+                if (global_ns() - t0 > 200000000ull) {  // 0.2 s: a CTA never arrived
+                  abort_now();
+                  ok = 0;
+                  break;
+                }
+            }
+            *s_ok = ok;
           }
-          *s_ok = ok;
-        }
-        named_sync(3, EPI_WARPS * 32);
-        if (*s_ok) {
-          // thread = (float4 column c4 of 64, row quarter g): quarter g sums its rows in order
-          // (up to eight loads in flight), then the four partial sums are added in order
-          const int nr = k * nkc_x;  // a token's slot rows are consecutive (pair-major, then chunk)
-          const int64_t units = int64_t(T) * (H / 4);
-          const int64_t lo = units * blockIdx.x / G, hi = units * (blockIdx.x + 1) / G;
-          const int th = tid - 32 * EPI_FIRST, c4 = th & 63, g = th >> 6;
-          const int rq = (nr + 3) / 4, r_lo = min(nr, g * rq), r_hi = min(nr, r_lo + rq);
-          for (int64_t u0 = lo; u0 < hi; u0 += 64) {
-            const int64_t u = u0 + c4;
-            const int t = int(u / (H / 4)), col4 = int(u - int64_t(t) * (H / 4));
-            float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-            if (u < hi) {
-              const float4* rows = reinterpret_cast<const float4*>(a.slots + int64_t(t) * nr * H) + col4;
-              for (int r = r_lo; r < r_hi; r += 8) {
-                float4 v[8];
+          named_sync(3, EPI_WARPS * 32);
+          if (*s_ok) {
+            // thread = (float4 column c4 of 64, row quarter g): quarter g sums its rows in order
+            // (up to eight loads in flight), then the four partial sums are added in order
+            const int nr = k * nkc_x;  // a token's slot rows are consecutive (pair-major, then chunk)
+            const int64_t units = int64_t(T) * (H / 4);
+            const int64_t lo = units * blockIdx.x / G, hi = units * (blockIdx.x + 1) / G;
+            const int th = tid - 32 * EPI_FIRST, c4 = th & 63, g = th >> 6;
+            const int rq = (nr + 3) / 4, r_lo = min(nr, g * rq), r_hi = min(nr, r_lo + rq);
+            for (int64_t u0 = lo; u0 < hi; u0 += 64) {
+              const int64_t u = u0 + c4;
+              const int t = int(u / (H / 4)), col4 = int(u - int64_t(t) * (H / 4));
+              float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+              if (u < hi) {
+                const float4* rows = reinterpret_cast<const float4*>(a.slots + int64_t(t) * nr * H) + col4;
+                for (int r = r_lo; r < r_hi; r += 8) {
+                  float4 v[8];
 #pragma unroll
-                for (int q2 = 0; q2 < 8; ++q2)
-                  v[q2] = r + q2 < r_hi ? __ldcg(rows + int64_t(r + q2) * (H / 4)) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                  for (int q2 = 0; q2 < 8; ++q2)
+                    v[q2] = r + q2 < r_hi ? __ldcg(rows + int64_t(r + q2) * (H / 4)) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll
-                for (int q2 = 0; q2 < 8; ++q2)
-                  if (r + q2 < r_hi) {
-                    acc.x += v[q2].x;
-                    acc.y += v[q2].y;
-                    acc.z += v[q2].z;
-                    acc.w += v[q2].w;
-                  }
+                  for (int q2 = 0; q2 < 8; ++q2)
+                    if (r + q2 < r_hi) {
+                      acc.x += v[q2].x;
+                      acc.y += v[q2].y;
+                      acc.z += v[q2].z;
+                      acc.w += v[q2].w;
+                    }
+                }
               }
-            }
-            s_part[g * 64 + c4] = acc;
-            named_sync(3, EPI_WARPS * 32);
-            if (g == 0 && u < hi) {
-              float4 sum = s_part[c4];
+              s_part[g * 64 + c4] = acc;
+              named_sync(3, EPI_WARPS * 32);
+              if (g == 0 && u < hi) {
+                float4 sum = s_part[c4];
 #pragma unroll
-              for (int q2 = 1; q2 < 4; ++q2) {
-                const float4 v = s_part[q2 * 64 + c4];
-                sum.x += v.x;
-                sum.y += v.y;
-                sum.z += v.z;
-                sum.w += v.w;
+                for (int q2 = 1; q2 < 4; ++q2) {
+                  const float4 v = s_part[q2 * 64 + c4];
+                  sum.x += v.x;
+                  sum.y += v.y;
+                  sum.z += v.z;
+                  sum.w += v.w;
+                }
+                const __nv_bfloat162 lo2 = __floats2bfloat162_rn(sum.x, sum.y), hi2 = __floats2bfloat162_rn(sum.z, sum.w);
+                uint2 packed;
+                packed.x = *reinterpret_cast<const uint32_t*>(&lo2);
+                packed.y = *reinterpret_cast<const uint32_t*>(&hi2);
+                *reinterpret_cast<uint2*>(a.out + int64_t(t) * H + 4 * col4) = packed;
               }
-              const __nv_bfloat162 lo2 = __floats2bfloat162_rn(sum.x, sum.y), hi2 = __floats2bfloat162_rn(sum.z, sum.w);
-              uint2 packed;
-              packed.x = *reinterpret_cast<const uint32_t*>(&lo2);
-              packed.y = *reinterpret_cast<const uint32_t*>(&hi2);
-              *reinterpret_cast<uint2*>(a.out + int64_t(t) * H + 4 * col4) = packed;
+              named_sync(3, EPI_WARPS * 32);  // s_part is rewritten next round
             }
-            named_sync(3, EPI_WARPS * 32);  // s_part is rewritten next round
           }
         }
       }
@@ -1210,7 +1253,7 @@ nvfp4moe_status launch_layer_fused_reset(const LayerFusedArgs& f, cudaStream_t s
                 f.k);
   const int P = f.T * f.k;
   const int n_done = (P < f.E ? P : f.E) * layer_fused_chunks(f.I);
-  layer_reset_kernel<<<1, 512, 0, s>>>(f.done, n_done, f.gbar, f.h_amax, f.E);
+  layer_reset_kernel<<<1, 512, 0, s>>>(f.done, n_done, f.tickets, f.T * (f.H / 32), f.gbar, f.h_amax, f.E);
   return check_launch("fused layer reset");
 }
 
@@ -1241,7 +1284,7 @@ nvfp4moe_status launch_layer_fused(const LayerFusedArgs& f, cudaStream_t s) {
   a.counts = f.counts; a.offsets = f.offsets; a.padded_offsets = f.padded_offsets; a.pair_to_row = f.pair_to_row;
   a.row_token = f.row_token; a.row_pair = f.row_pair; a.tile_expert = f.tile_expert; a.active = f.active;
   a.x_codes = f.x_codes; a.x_sf = f.x_sf; a.h_codes = f.h_codes; a.h_sf = f.h_sf;
-  a.slots = f.slots; a.done = f.done; a.gbar = f.gbar;
+  a.slots = f.slots; a.done = f.done; a.tickets = f.tickets; a.gbar = f.gbar;
   a.schedule = f.schedule;
   a.out = static_cast<__nv_bfloat16*>(f.out);
   a.shape = lf_shape(f.T, f.H, f.I, f.E, f.k, num_sms());
