@@ -611,14 +611,7 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
     atomicOr(a.status, kDevTimeout);
   };
 
-  // per active expert: the gate/up product scales (x scale times the weight scales), the
-  // requantisation scale of h, and the down product's scale
-  for (int sl = tid; sl < A; sl += LF_THREADS) {
-    const int e = s_act[sl];
-    const float sh = a.h_scale[e];
-    s_scl[sl] = make_float4(s_t * a.w13_scale[2 * e], s_t * a.w13_scale[2 * e + 1], sh, sh * a.w2_scale[e]);
-  }
-  __syncthreads();  // the work list and the scales are read by every role
+  __syncthreads();  // the work list is read by every role
   auto item_at = [&](int j) { return lf_unpack(s_item[j]); };
 
   if (warp == 0) {
@@ -736,6 +729,14 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
                   // the epilogue never writes stay zero
         for (int i = qt; i < 2 * (kcl / 128) * 128; i += qn) reinterpret_cast<uint32_t*>(sSFB)[i] = 0u;
       fence_proxy_async_shared();  // generic stores above, read by the tensor core
+      // per active expert: the gate/up product scales (x scale times the weight scales), the
+      // requantisation scale of h, and the down product's scale.  Only the epilogue reads them,
+      // so they are loaded here, while the weight stream starts.
+      for (int sl = qt; sl < A; sl += qn) {
+        const int e = s_act[sl];
+        const float sh = a.h_scale[e];
+        s_scl[sl] = make_float4(s_t * a.w13_scale[2 * e], s_t * a.w13_scale[2 * e + 1], sh, sh * a.w2_scale[e]);
+      }
     }
     named_sync(1, LF_THREADS - 32);
     tc_fence_after();
