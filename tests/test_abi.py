@@ -90,6 +90,16 @@ def test_workspace_queries(so):
                    L.row_pair, L.tile_expert, L.active, L.x_scale, L.x_codes, L.x_sf, L.h_codes, L.h_sf,
                    L.slots])
     assert all(o % 256 == 0 for o in offs) and len(set(offs)) == len(offs) and offs[-1] < L.total
+    # launch modes: every named one is accepted (on this host none can take the single launch,
+    # which needs the tensor-core path), anything else is an argument error
+    for mode in (C.LAUNCH_AUTO, C.LAUNCH_SINGLE, C.LAUNCH_MULTI, C.LAUNCH_SINGLE_TILE, C.LAUNCH_SINGLE_LOCAL):
+        d.launch_mode = mode
+        assert so.moe_ffn_workspace_layout(ctypes.byref(d), ctypes.byref(L)) == C.OK
+        assert L.single_launch == 0
+    for bad in (-1, 5):
+        d.launch_mode = bad
+        assert so.moe_ffn_workspace_layout(ctypes.byref(d), ctypes.byref(L)) == C.INVALID_ARG
+    d.launch_mode = C.LAUNCH_AUTO
     d.H = 100
     assert so.moe_ffn_workspace_layout(ctypes.byref(d), ctypes.byref(L)) == C.UNSUPPORTED_SHAPE
     assert so.moe_permute_rows_capacity(16, 512, 10, 128) == 160 + 160 * 127
