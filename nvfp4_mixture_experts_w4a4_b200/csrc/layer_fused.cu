@@ -2,32 +2,35 @@
 // and the dense layer at T = 1): routing, permutation, x quantisation, gate/up + SwiGLU +
 // requantisation, down and the ordered combine.
 //
-// At decode sizes the layer is a stream of expert weights (about 1.77 MB per touched expert
+// At decode sizes the layer is a stream of expert weights (about 1.69 MB per touched expert
 // at H2048/I512) with a few kilobytes of activations, so its time is the weight bytes over
 // HBM bandwidth plus whatever latency precedes and follows the stream.  This kernel keeps
 // that latency to one launch:
 //
-//  * Every CTA routes the whole batch itself (T <= 16 warps' worth of top-k over the
-//    logits, which sit in L2 after the first CTA's reads), derives the permutation and the
-//    work list locally, and starts streaming its first weight tiles at once.  No kernel
-//    before it computes anything, so nothing has to be waited for before the stream.
+//  * Every CTA routes the whole batch itself (warp t takes token t, its logits requested at
+//    kernel entry), derives the permutation and the work list locally, and starts streaming
+//    its first weight tiles at once.  No kernel before it computes anything, so nothing has
+//    to be waited for before the stream.
 //  * Every CTA quantises the whole of x (dynamic tensor scale amax / 2688 over the batch)
 //    into shared memory, in the 128-byte-swizzled K-major layout the MMA reads, with the
-//    block scales staged once into TMEM.  The gate/up MMA takes ALL T tokens (padded to the
+//    block scales staged once into TMEM.  x itself arrives by one bulk copy at entry, into
+//    the weight ring, which no tile uses before the routing is done (when x does not fit
+//    there, the epilogue warps load and quantise it once the stream has started).  The gate/up MMA takes ALL T tokens (padded to the
 //    MMA's N = 16) as its B operand for every expert: one weight tile times the resident
 //    token tile.  Each output column depends only on its own token, so the columns of the
 //    tokens an expert did not receive are simply not used; the extra MMA work is free at
 //    this size, and no token tile is loaded per item.
 //  * Two schedules of the weight tiles, chosen per call from the routing (every CTA takes the
 //    same decision):
-//    - expert-local: units of (active expert, 256 columns of h), round-robin over the CTAs.
-//      A CTA runs a unit's four gate/up tiles (W13 rows of those columns), requantises the h
-//      chunk into shared memory (K-major, 128-byte swizzle: the down MMA's B operand, 16 token
-//      rows) and runs the unit's down tiles (all H rows of W2, K = the chunk) from it.  No h
-//      crosses CTAs, so nothing waits on another CTA until the combine; the next unit's
-//      gate/up tiles are issued before this unit's down tiles, so the MMA has work while the
-//      epilogue requantises, and two h buffers alternate.  Taken when I % 256 == 0 and the
-//      units fill the grid's rounds to at least 80 %.
+//    - expert-local: units of (active expert, kcl columns of h; kcl 256, 512 or 1024),
+//      round-robin over the CTAs.  A CTA runs a unit's kcl / 64 gate/up tiles (W13 rows of
+//      those columns), requantises the h chunk into shared memory (K-major, 128-byte swizzle:
+//      the down MMA's B operand, 16 token rows) and runs the unit's down tiles (all H rows of
+//      W2, K = the chunk) from it.  No h crosses CTAs, so nothing waits on another CTA until
+//      the combine; the next unit's gate/up tiles are issued before this unit's down tiles,
+//      so the MMA has work while the epilogue requantises, and two h buffers alternate.
+//      Taken when I % 256 == 0 and the units fill the grid's rounds to at least 80 %
+//      (lf_local_width).
 //    - tile-level: gate/up tiles (expert, 128 rows of W13 = 64 columns of h) and down tiles
 //      (expert, K chunk of at most 2048, 128 rows of W2) spread over all CTAs.  A down tile's
 //      h rows are the requantised outputs of the gate/up tiles of its expert and K chunk,
@@ -45,7 +48,8 @@
 // A small launch before this one zeroes the counters, tickets and barrier; this kernel is its
 // programmatic dependent and waits for it only before touching them (well after its start).
 //
-// Warp roles after the routing phase (all 16 warps route, one token each, and quantise x):
+// Warp roles after the routing phase (all 16 warps route, one token each, and quantise x
+// when it was staged):
 //   warp 0      weight producer: TMA loads of 128 x 128-byte tiles (128-byte swizzle) and the
 //               bulk copies of their scale atoms into a ring of stages;
 //   warp 1      TMEM owner and MMA issuer: tcgen05.cp of the scales, four K=64 block-scaled
@@ -55,7 +59,8 @@
 //   warp 10     h producer (tile-level schedule): for down tiles, acquires the expert's chunk
 //               counter and loads the h rows and their scale atoms into the stage the weight
 //               producer armed;
-//   warps 11-15 routing, x quantisation and the inspection copies only.
+//   warps 10-15 the inspection copies of the routing and of x (warp 10 also the h producer);
+//   warps 2-15  x quantisation from global memory when x was not staged.
 // Every wait is bounded (status bit on timeout; copies in flight land before the CTA exits).
 #include <cmath>
 
