@@ -559,7 +559,7 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
     const int rank = __popc(s_mask[e] & ((1u << t) - 1u));
     s_prank[int(oa & 0xFFFFu) + rank] = p;
   }
-  __syncthreads();
+  // (the pair ranks are read only by the epilogue, after the barrier that follows the work list)
 
   // this CTA's work list, decoded once here by all threads into shared memory
   const int G = int(gridDim.x);
@@ -1150,12 +1150,13 @@ layer_fused_kernel(const __grid_constant__ CUtensorMap tmW13, const __grid_const
               atomicAdd(a.gbar, 1);
               const uint64_t t0 = global_ns();
               ok = 1;
-              while (ld_acquire_gpu(a.gbar) < G)
+              while (ld_relaxed_gpu(a.gbar) < G)
                 if (global_ns() - t0 > 200000000ull) {  // 0.2 s: a CTA never arrived
                   abort_now();
                   ok = 0;
                   break;
                 }
+              fence_acq_rel_gpu();  // acquire, with the load that saw every arrival
             }
             *s_ok = ok;
           }
