@@ -333,15 +333,16 @@ typedef struct {
    *           that resets its counters): every CTA routes the batch and keeps x quantised in
    *           shared memory, then runs one of two schedules, chosen per call from the routing
    *           (every CTA takes the same decision):
-   *             expert-local: units of (active expert, 256 columns of h); a CTA runs a unit's
-   *               gate/up tiles, keeps its h chunk in shared memory and runs the unit's down
-   *               tiles from it.  Taken when I % 256 == 0 and the units fill the grid's rounds
-   *               to at least 80 %;
+   *             expert-local: units of (active expert, 256, 512 or 1024 columns of h); a CTA
+   *               runs a unit's gate/up tiles, keeps its h chunk in shared memory and runs the
+   *               unit's down tiles from it.  Taken when I % 256 == 0 and the units fill the
+   *               grid's rounds to at least 80 % (the widest such chunk is used);
    *             tile-level: gate/up and down tiles spread over all CTAs, h through global
    *               memory, the down tiles of an expert waiting on counters of its gate/up tiles;
    *           then, after a grid-wide barrier, every CTA sums a slice of the outputs over the
    *           k x K-chunk slot rows in slot order;
-   *   SINGLE_TILE, SINGLE_LOCAL  SINGLE with that schedule (SINGLE_LOCAL needs I % 256 == 0);
+   *   SINGLE_TILE, SINGLE_LOCAL  SINGLE with that schedule (SINGLE_LOCAL needs I % 256 == 0 and
+   *           I <= 63 * 256, else NVFP4MOE_UNSUPPORTED_SHAPE);
    *   MULTI   the routing/permutation/quantisation prologue, then the grouped GEMMs, then the
    *           combine (the path every larger batch takes);
    *   AUTO    the faster of SINGLE and MULTI for the shape (see moe_ffn_workspace_layout's
