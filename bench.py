@@ -450,7 +450,7 @@ def measure(wl: W.Workload, args, dev, local: int, rank: int, world: int, dist_o
               "single_tile": C.LAUNCH_SINGLE_TILE, "single_local": C.LAUNCH_SINGLE_LOCAL}[args.launch]
     single = launch in (C.LAUNCH_SINGLE, C.LAUNCH_SINGLE_TILE, C.LAUNCH_SINGLE_LOCAL)
     if single and not (wl.T <= 16 and path != C.PATH_GEMV and args.act == "nvfp4" and not args.shared_I
-                       and (launch != C.LAUNCH_SINGLE_LOCAL or wl.I % 256 == 0)):
+                       and (launch != C.LAUNCH_SINGLE_LOCAL or (wl.I % 256 == 0 and wl.I // 256 <= 63))):
         launch = C.LAUNCH_AUTO  # the single launch does not apply to this workload
     act, experts, layer = setup_layer(wl, dev, path=path, launch=launch)
     shared, shared_bits = None, None
